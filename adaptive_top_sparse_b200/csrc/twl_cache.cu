@@ -1,0 +1,149 @@
+// Cache maintenance kernels: page bounds for the page selector and the INT4 copy of K.
+//
+// "Twilight: Adaptive Attention Sparsity with Hierarchical Top-p Pruning":
+//   - page bounds: per-page channel min/max of K, the metadata a Quest-style selector scores
+//     (the selector is named in the notes page, "Background", and the summary, section 5.1).
+//   - INT4 K: summary, appendix B.1 (per-head dynamic quantisation, fp16 scale and zero point,
+//     two 4-bit values per byte); notes page, "Key designs" (4-bit K cache, 1/8 extra memory).
+//
+// Both kernels give one warp to one (sequence, logical page, kv-head): the page-head tile is
+// 16 rows x 256 B, contiguous; lane l owns channels 4l .. 4l+3 (8 bytes of every row).
+#include "twl_common.cuh"
+#include "twl_kernels.h"
+
+namespace twl {
+namespace {
+
+struct Half4 {
+  uint32_t lo, hi;  // channels (4l, 4l+1) and (4l+2, 4l+3)
+};
+
+__device__ __forceinline__ Half4 load_half4(const uint16_t* p) {
+  uint2 v = *reinterpret_cast<const uint2*>(p);
+  return Half4{v.x, v.y};
+}
+
+__device__ __forceinline__ bool decode_warp(long warp, const KV& kv, int* b, int* j, int* h) {
+  long total = (long)kv.batch * kv.max_pages * kv.hkv;
+  if (warp >= total) return false;
+  *h = int(warp % kv.hkv);
+  long t = warp / kv.hkv;
+  *j = int(t % kv.max_pages);
+  *b = int(t / kv.max_pages);
+  return true;
+}
+
+__global__ void __launch_bounds__(256) k_page_bounds(KV kv, uint16_t* __restrict__ bounds,
+                                                     uint32_t* flags) {
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  int b, j, h;
+  if (!decode_warp(warp, kv, &b, &j, &h)) return;
+  Seq sq = load_seq(kv.seq_lens, b, kv.max_pages, flags, j == 0 && h == 0 && lane == 0);
+  if (j >= sq.pages) return;
+  int ph = kv.page_table[(size_t)b * kv.max_pages + j];
+  if (ph < 0 || ph >= kv.num_phys) {
+    if (lane == 0 && h == 0) raise_flag(flags, TWL_FLAG_BAD_INDEX);
+    return;
+  }
+  const int rows = page_rows(sq.n, j);
+  const uint16_t* src = kv.k + (((size_t)ph * kv.hkv + h) * kPage) * kHeadDim + lane * 4;
+  int mn[4], mx[4];
+  {
+    Half4 v = load_half4(src);
+    mn[0] = mx[0] = f16_key(v.lo);
+    mn[1] = mx[1] = f16_key(v.lo >> 16);
+    mn[2] = mx[2] = f16_key(v.hi);
+    mn[3] = mx[3] = f16_key(v.hi >> 16);
+  }
+  for (int r = 1; r < rows; ++r) {
+    Half4 v = load_half4(src + r * kHeadDim);
+    int k0 = f16_key(v.lo), k1 = f16_key(v.lo >> 16), k2 = f16_key(v.hi), k3 = f16_key(v.hi >> 16);
+    mn[0] = min(mn[0], k0); mx[0] = max(mx[0], k0);
+    mn[1] = min(mn[1], k1); mx[1] = max(mx[1], k1);
+    mn[2] = min(mn[2], k2); mx[2] = max(mx[2], k2);
+    mn[3] = min(mn[3], k3); mx[3] = max(mx[3], k3);
+  }
+  uint16_t* dst = bounds + (((size_t)ph * kv.hkv + h) * 2) * kHeadDim + lane * 4;
+  uint2 lo, hi;
+  lo.x = f16_from_key(mn[0]) | (f16_from_key(mn[1]) << 16);
+  lo.y = f16_from_key(mn[2]) | (f16_from_key(mn[3]) << 16);
+  hi.x = f16_from_key(mx[0]) | (f16_from_key(mx[1]) << 16);
+  hi.y = f16_from_key(mx[2]) | (f16_from_key(mx[3]) << 16);
+  *reinterpret_cast<uint2*>(dst) = lo;
+  *reinterpret_cast<uint2*>(dst + kHeadDim) = hi;
+}
+
+// One nibble: n = min(15, rint_even(fp32(x - z) / s)); x - z >= 0 because z is the row minimum.
+__device__ __forceinline__ uint32_t nibble(uint32_t xbits, float z, float s) {
+  float x = __half2float(__ushort_as_half((unsigned short)(xbits & 0xFFFFu)));
+  float r = rintf(__fdiv_rn(__fsub_rn(x, z), s));
+  r = fminf(fmaxf(r, 0.f), 15.f);
+  return (uint32_t)r;
+}
+
+__global__ void __launch_bounds__(256) k_quantize_k(KV kv, uint8_t* __restrict__ k_int4,
+                                                    uint16_t* __restrict__ k_sz,
+                                                    uint32_t* flags) {
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  int b, j, h;
+  if (!decode_warp(warp, kv, &b, &j, &h)) return;
+  Seq sq = load_seq(kv.seq_lens, b, kv.max_pages, flags, j == 0 && h == 0 && lane == 0);
+  if (j >= sq.pages) return;
+  int ph = kv.page_table[(size_t)b * kv.max_pages + j];
+  if (ph < 0 || ph >= kv.num_phys) {
+    if (lane == 0 && h == 0) raise_flag(flags, TWL_FLAG_BAD_INDEX);
+    return;
+  }
+  const int rows = page_rows(sq.n, j);
+  const size_t tile = ((size_t)ph * kv.hkv + h) * kPage;
+  const uint16_t* src = kv.k + tile * kHeadDim + lane * 4;
+  uint16_t* dst_q = reinterpret_cast<uint16_t*>(k_int4 + tile * (kHeadDim / 2)) + lane;
+  uint32_t* dst_sz = reinterpret_cast<uint32_t*>(k_sz + tile * 2);
+  for (int r = 0; r < kPage; ++r) {
+    if (r >= rows) {  // past the end of the sequence: zeros
+      dst_q[r * (kHeadDim / 4)] = 0;
+      if (lane == 0) dst_sz[r] = 0u;
+      continue;
+    }
+    Half4 v = load_half4(src + r * kHeadDim);
+    int k0 = f16_key(v.lo), k1 = f16_key(v.lo >> 16), k2 = f16_key(v.hi), k3 = f16_key(v.hi >> 16);
+    int kmn = min(min(k0, k1), min(k2, k3));
+    int kmx = max(max(k0, k1), max(k2, k3));
+    kmn = __reduce_min_sync(0xffffffffu, kmn);
+    kmx = __reduce_max_sync(0xffffffffu, kmx);
+    const uint32_t mn_bits = f16_from_key(kmn), mx_bits = f16_from_key(kmx);
+    const float mn = __half2float(__ushort_as_half((unsigned short)mn_bits));
+    const float mx = __half2float(__ushort_as_half((unsigned short)mx_bits));
+    const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.f));
+    const float s = __half2float(s16);
+    uint32_t packed = 0;
+    if (s != 0.f) {
+      uint32_t n0 = nibble(v.lo, mn, s), n1 = nibble(v.lo >> 16, mn, s);
+      uint32_t n2 = nibble(v.hi, mn, s), n3 = nibble(v.hi >> 16, mn, s);
+      packed = n0 | (n1 << 4) | (n2 << 8) | (n3 << 12);
+    }
+    dst_q[r * (kHeadDim / 4)] = (uint16_t)packed;
+    if (lane == 0) dst_sz[r] = uint32_t(__half_as_ushort(s16)) | (mn_bits << 16);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_page_bounds(const KV& kv, uint16_t* bounds, uint32_t* flags, cudaStream_t s) {
+  long warps = (long)kv.batch * kv.max_pages * kv.hkv;
+  long blocks = (warps * 32 + 255) / 256;
+  k_page_bounds<<<(unsigned)blocks, 256, 0, s>>>(kv, bounds, flags);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_k(const KV& kv, uint8_t* k_int4, uint16_t* k_sz, uint32_t* flags,
+                              cudaStream_t s) {
+  long warps = (long)kv.batch * kv.max_pages * kv.hkv;
+  long blocks = (warps * 32 + 255) / 256;
+  k_quantize_k<<<(unsigned)blocks, 256, 0, s>>>(kv, k_int4, k_sz, flags);
+  return cudaGetLastError();
+}
+
+}  // namespace twl

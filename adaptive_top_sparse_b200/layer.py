@@ -1,0 +1,95 @@
+"""Device-side state of one decode-attention layer and the calls a user makes on it.
+
+``DecodeLayer`` owns device tensors (PyTorch is only the allocator here): the paged fp16 K/V, the
+page table, the derived INT4 K and page bounds, a workspace, and the outputs.  Every computation
+is a call into libtwl.so.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import twl
+
+
+def budget_bound(max_pages: int, budget_pages: int, budget_div: int) -> int:
+    """Largest page budget any sequence can get (the sel_pages row stride)."""
+    if budget_pages > 0:
+        return min(budget_pages, max_pages)
+    return -(-max_pages // budget_div)
+
+
+class DecodeLayer:
+    def __init__(self, k, v, page_table, seq_lens, num_q_heads: int, num_kv_heads: int,
+                 budget_pages: int = 0, budget_div: int = 4, device="cuda"):
+        dev = torch.device(device)
+        t = lambda x, dt: torch.as_tensor(x).to(device=dev, dtype=dt).contiguous()
+        self.k = t(k, torch.float16)
+        self.v = t(v, torch.float16)
+        self.page_table = t(page_table, torch.int32)
+        self.seq_lens = t(seq_lens, torch.int32)
+        self.num_q_heads = num_q_heads
+        self.num_kv_heads = num_kv_heads
+        self.budget_pages = budget_pages
+        self.budget_div = budget_div
+        self.device = dev
+        p_phys = self.k.shape[0]
+        self.kv = twl.PagedKV(self.k, self.v, self.page_table, self.seq_lens, num_kv_heads,
+                              p_phys)
+        self.batch = self.kv.batch
+        self.max_pages = self.kv.max_pages
+        self.max_budget = budget_bound(self.max_pages, budget_pages, budget_div)
+        self.aux = twl.KAux(
+            torch.zeros((p_phys, num_kv_heads, 16, 64), dtype=torch.uint8, device=dev),
+            torch.zeros((p_phys, num_kv_heads, 16, 2), dtype=torch.float16, device=dev),
+            torch.zeros((p_phys, num_kv_heads, 2, 128), dtype=torch.float16, device=dev))
+        self.ws = twl.alloc_workspace(twl.TWL_OP_DECODE_STEP, dev, batch=self.batch,
+                                      num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+                                      max_pages=self.max_pages, max_budget=self.max_budget)
+        self.o = torch.zeros((self.batch, num_q_heads, 128), dtype=torch.float32, device=dev)
+        self.lse = torch.zeros((self.batch, num_q_heads), dtype=torch.float32, device=dev)
+
+    @classmethod
+    def from_workload(cls, wl, device="cuda"):
+        return cls(wl.k, wl.v, wl.page_table, wl.seq_lens, wl.num_q_heads, wl.num_kv_heads,
+                   wl.budget_pages, wl.budget_div, device)
+
+    # ------------------------------------------------------------------ cache maintenance
+    def build_aux(self, stream=None) -> None:
+        """INT4 K and page bounds for every referenced page."""
+        twl.twl_quantize_k(self.kv, self.aux.k_int4, self.aux.k_scale_zero, self.ws, stream)
+        twl.twl_page_bounds(self.kv, self.aux.bounds, self.ws, stream)
+
+    # ------------------------------------------------------------------ stats buffers
+    def alloc_stats(self) -> dict:
+        b, hq, hkv, mb = self.batch, self.num_q_heads, self.num_kv_heads, self.max_budget
+        dev, i32, f32 = self.device, torch.int32, torch.float32
+        cs, us = 16 * mb, 16 * self.max_pages
+        return dict(
+            sel_pages=torch.full((b, hq, mb), -1, dtype=i32, device=dev),
+            sel_count=torch.zeros((b, hq), dtype=i32, device=dev),
+            weights=torch.zeros((b, hq, cs), dtype=f32, device=dev),
+            cand_tok=torch.full((b, hq, cs), -1, dtype=i32, device=dev),
+            cand_count=torch.zeros((b, hq), dtype=i32, device=dev),
+            threshold=torch.zeros((b, hq), dtype=f32, device=dev),
+            kept_count=torch.zeros((b, hq), dtype=i32, device=dev),
+            union_tok=torch.full((b, hkv, us), -1, dtype=i32, device=dev),
+            union_count=torch.zeros((b, hkv), dtype=i32, device=dev))
+
+    # ------------------------------------------------------------------ the decode step
+    def decode(self, q, p: float = 0.85, eps: float = 1e-6, stats: dict | None = None,
+               stream=None):
+        """One select -> estimate -> prune -> union -> attend step for query q [B][Hq][128] fp16
+        (device tensor).  Returns (o, lse) device tensors owned by the layer."""
+        st = twl.make_stats(**stats) if stats is not None else None
+        twl.twl_decode_step(q, self.num_q_heads, self.kv, self.aux, self.budget_pages,
+                            self.budget_div, self.max_budget, p, eps, self.o, self.lse, st,
+                            self.ws, stream)
+        return self.o, self.lse
+
+    def status(self, clear: bool = False):
+        return twl.twl_device_status(self.ws, clear)
+
+
+SM_SCALE = 1.0 / math.sqrt(128.0)

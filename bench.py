@@ -1,0 +1,428 @@
+"""Benchmark of the select -> INT4 estimate -> top-p prune -> sparse attend decode step.
+
+Metric: decode-attention layer-steps/s on the 32K-context GQA layer (batch 1, 32 q-heads /
+8 kv-heads, head_dim 128, 16-token pages, base budget 1/4 of the pages, p = 0.85), plus the
+fraction of the HBM roofline.
+
+A bench step is one decode token through LAYERS distinct layer caches (32, the depth of a
+Llama-3.1-8B stack): LAYERS calls of twl_decode_step, captured once in a CUDA graph.  Every layer
+owns its own K/V/INT4/bounds/workspace buffers, so consecutive reads of one layer are
+LAYERS x (touched bytes per layer-step) apart, far beyond the 126 MB L2.  The layers are copies
+of one seeded synthetic layer (identical work per layer).
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun every rank runs its own LAYERS-layer stack (weak scaling, no collective on the
+data path); rank 0 prints one JSON line.  --impl reference times the CPU oracle on the host cores
+(rank 0 only) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import synth  # noqa: E402
+
+METRIC = "decode attn layer-steps/s at 32K ctx (select+prune+attend); % of HBM roofline"
+UNIT = "layer-steps/s"
+LAYERS = 32  # default; --layers overrides (profiling runs use 1)
+KERNELS_PER_LAYER_STEP = 9
+FALLBACK_HBM_GBS = 6650.0
+
+
+def workload_config():
+    return {
+        "workload": "GQA decode layer, batch 1, 32 q-heads / 8 kv-heads, head_dim 128, "
+                    "32768-token context, 16-token pages, Quest budget 1/4 of pages, INT4 K "
+                    "(group 128), p = 0.85, eps = 1e-6, seed 0",
+        "batch": 1, "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128, "ctx": 32768,
+        "page_size": 16, "budget": "ceil(P/4) pages", "p": 0.85, "eps": 1e-6,
+        "layers_per_step": LAYERS,
+        "l2": f"no flush; {LAYERS} distinct layer caches per step, so each layer's touched bytes "
+              f"are re-read only after {LAYERS - 1} other layers' (>> 126 MB L2)",
+        "inputs": "fp16 q/K/V, INT4 K + fp16 scale/zero, fp16 page bounds",
+    }
+
+
+# ---------------------------------------------------------------------------------- roofline
+
+def algorithmic_bytes(page_table, seq_lens, num_q_heads, num_kv_heads, sel_pages, sel_count,
+                      union_count):
+    """Unique bytes one layer-step must move (the method's roofline definition):
+    page metadata (bounds 512 B per page per kv-head + 4 B page-table entry per page),
+    INT4 K + scale/zero of each group's union of selected pages (1088 B per page per kv-head),
+    fp16 K+V of each group's union of kept tokens (512 B per token per kv-head),
+    q (256 B per head), o + lse (516 B per head), seq_lens (4 B per sequence)."""
+    g = num_q_heads // num_kv_heads
+    batch = len(seq_lens)
+    total = 0
+    parts = dict(bounds=0, page_table=0, int4=0, kv=0, q_o=0)
+    for b in range(batch):
+        pb = (int(seq_lens[b]) + 15) // 16
+        parts["bounds"] += pb * num_kv_heads * 512
+        parts["page_table"] += pb * 4
+        for kvh in range(num_kv_heads):
+            pages = set()
+            for h in range(kvh * g, (kvh + 1) * g):
+                pages.update(sel_pages[b, h, : int(sel_count[b, h])].tolist())
+            parts["int4"] += len(pages) * 1088
+            parts["kv"] += int(union_count[b, kvh]) * 512
+    parts["q_o"] = batch * num_q_heads * (256 + 516) + 4 * batch
+    total = sum(parts.values())
+    return total, parts
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "adaptive_top_sparse_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    """DRAM bytes per layer-step from the committed ncu summary, if it matches these sources."""
+    path = os.path.join(ROOT, "profiles", "decode_step_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("source_hash") != source_hash():
+        return None
+    return d.get("dram_bytes_per_layer_step")
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        # nvidia-smi numbers GPUs physically; select ours by UUID (CUDA_VISIBLE_DEVICES-proof)
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.dev = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:  # pragma: no cover
+            self.dev = str(device_index)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(wl, groups):
+    """Time the oracle's decode path (select -> estimate -> top-p -> union -> attention) on the
+    given (b, kv-head) groups; cache maintenance (bounds, INT4) is prepared outside the timing,
+    as it is for the GPU step."""
+    from oracle import twl_oracle as O
+    from tests.twl_checks import group_workload
+    subs = []
+    for b, kvh in groups:
+        sub = group_workload(wl, b, kvh)
+        bounds = O.page_bounds(sub.k, sub.page_table, sub.seq_lens)
+        q4, sz = O.quantize_k(sub.k, sub.page_table, sub.seq_lens)
+        subs.append((sub, bounds, q4, sz))
+    t0 = time.perf_counter()
+    for sub, bounds, q4, sz in subs:
+        O.decode_step(sub, bounds=bounds, k_int4=q4, k_sz=sz)
+    return time.perf_counter() - t0
+
+
+def cpu_threads_guard():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=1)
+    except ImportError:  # pragma: no cover
+        import contextlib
+        return contextlib.nullcontext()
+
+
+# ---------------------------------------------------------------------------------- arms
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = torch.device("cuda") if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    wl = synth.config2()
+    groups = [(0, 0), (0, 1)]
+    with cpu_threads_guard():
+        for _ in range(args.warmup):
+            oracle_sample(wl, groups[:1])
+        times = [oracle_sample(wl, groups) for _ in range(args.steps)]
+    per_layer = sum(times) / len(times) * (wl.num_kv_heads / len(groups))
+    value = 1.0 / per_layer
+    sample = (f"oracle decode path on {len(groups)} of the layer's 8 kv-head groups "
+              f"(4 q-heads each) per step, scaled x{wl.num_kv_heads // len(groups)} to one "
+              f"layer-step")
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_layer * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference", "config": workload_config(),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def run_ours(args, world, rank, local):
+    from adaptive_top_sparse_b200 import twl
+    from adaptive_top_sparse_b200.layer import DecodeLayer
+
+    dev = torch.device("cuda", local)
+    wl = synth.config2()
+    layers = []
+    for _ in range(LAYERS):
+        layer = DecodeLayer.from_workload(wl, dev)
+        layer.build_aux()
+        layers.append(layer)
+    qs = [torch.from_numpy(wl.q).to(dev) for _ in range(LAYERS)]
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+
+    # workload statistics and the roofline bytes, from one step with stats (untimed)
+    stats = layers[0].alloc_stats()
+    layers[0].decode(qs[0], wl.p, wl.eps, stats)
+    torch.cuda.synchronize(dev)
+    st = {k: v.cpu().numpy() for k, v in stats.items()}
+    alg_bytes, parts = algorithmic_bytes(wl.page_table, wl.seq_lens, wl.num_q_heads,
+                                         wl.num_kv_heads, st["sel_pages"], st["sel_count"],
+                                         st["union_count"])
+    kept = st["kept_count"].reshape(-1)
+    cand = st["cand_count"].reshape(-1)
+
+    # capture one step (LAYERS layer-steps) in a graph
+    with torch.cuda.stream(stream):
+        for layer, q in zip(layers, qs):          # eager warm-up on the capture stream
+            layer.decode(q, wl.p, wl.eps, None, stream)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for layer, q in zip(layers, qs):
+            layer.decode(q, wl.p, wl.eps, None, stream)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms, world)
+    ms_per_step = ms_max / args.steps
+    value = world * args.steps * LAYERS / (ms_max / 1e3)
+
+    for layer in layers:
+        s_, fl = layer.status()
+        if s_ != 0:
+            raise RuntimeError(f"device flags set: {fl}")
+
+    # end to end through the public API: pinned host q in, o/lse out, every layer-step
+    q_host = [torch.from_numpy(wl.q).pin_memory() for _ in range(LAYERS)]
+    o_host = [torch.empty_like(l.o, device="cpu").pin_memory() for l in layers]
+    lse_host = [torch.empty_like(l.lse, device="cpu").pin_memory() for l in layers]
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 50))
+
+    def e2e_pass():
+        for i, layer in enumerate(layers):
+            qs[i].copy_(q_host[i], non_blocking=True)
+            o, lse = layer.decode(qs[i], wl.p, wl.eps, None, stream)
+            o_host[i].copy_(o, non_blocking=True)
+            lse_host[i].copy_(lse, non_blocking=True)
+
+    e2e_value = None
+    if e2e_steps:
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, args.warmup)):
+                e2e_pass()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(e2e_steps):
+                e2e_pass()
+            e1.record(stream)
+        e1.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e_value = world * e2e_steps * LAYERS / (e2e_ms / 1e3)
+    h2d = LAYERS * wl.q.nbytes
+    d2h = LAYERS * (layers[0].o.numel() * 4 + layers[0].lse.numel() * 4)
+
+    peak, peak_kind = hbm_peak()
+    layer_step_s = ms_per_step / 1e3 / LAYERS
+    achieved = alg_bytes / layer_step_s / 1e9
+    traffic = measured_traffic()
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "twl_decode_step (whole layer-step)",
+                     "alg_bytes_per_layer_step": alg_bytes, "alg_bytes_parts": parts,
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps * LAYERS * KERNELS_PER_LAYER_STEP,
+        "clocks": clk,
+        "workload_stats": {
+            "kept_tokens_per_head_mean": float(kept.mean()),
+            "kept_tokens_per_head_min": int(kept.min()), "kept_tokens_per_head_max": int(kept.max()),
+            "kept_fraction_of_candidates_mean": float((kept / np.maximum(cand, 1)).mean()),
+            "union_tokens_per_group": st["union_count"].reshape(-1).tolist(),
+        },
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        wl_groups = [(0, 0)]
+        with cpu_threads_guard():
+            oracle_sample(wl, wl_groups)                    # warm
+            t = oracle_sample(wl, wl_groups)
+        per_layer = t * wl.num_kv_heads / len(wl_groups)
+        out["cpu_baseline"] = {
+            "value": 1.0 / per_layer, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "oracle decode path (numpy, fp64) on 1 of the layer's 8 kv-head groups, "
+                      "scaled x8 to one layer-step; bounds/INT4 prepared untimed"}
+    del graph
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=32)
+    args = ap.parse_args()
+    global LAYERS
+    LAYERS = max(1, args.layers)
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            out = run_reference(args, world, rank)
+        else:
+            out = run_ours(args, world, rank, local)
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

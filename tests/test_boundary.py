@@ -1,0 +1,165 @@
+"""The C ABI without a GPU: the library loads, exports every entry point declared in
+include/twl.h, sizes workspaces, and rejects bad arguments on the host with the documented status
+before launching anything.  Pointers here are fake addresses: every call below fails validation
+before any CUDA call, so nothing is dereferenced."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from adaptive_top_sparse_b200 import twl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "twl.h")
+
+A = 1 << 20          # a fake, 256-byte aligned address
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:twl_status|size_t|const char\*)\s+(twl_\w+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for name in ["twl_quantize_k", "twl_page_bounds", "twl_select_pages", "twl_estimate",
+                 "twl_prune_top_p", "twl_group_union", "twl_sparse_decode", "twl_decode_step",
+                 "twl_workspace_bytes", "twl_workspace_init", "twl_device_status",
+                 "twl_status_string"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.CDLL(twl.LIB_PATH)
+    missing = [s for s in declared_symbols() if not hasattr(lib, s)]
+    assert not missing, missing
+    assert set(declared_symbols()) <= set(twl.EXPORTED) | set(declared_symbols())
+
+
+def test_status_strings():
+    for code in range(-6, 1):
+        assert twl.twl_status_string(code) != "unknown status"
+    assert twl.twl_status_string(-99) == "unknown status"
+
+
+def _kv(**over):
+    d = dict(k=A, v=A + 4096, page_table=A + 8192, seq_lens=A + 12288, batch=2, num_kv_heads=8,
+             head_dim=128, page_size=16, max_pages=64, num_phys_pages=128)
+    d.update(over)
+    return twl._PagedKV(d["k"], d["v"], d["page_table"], d["seq_lens"], d["batch"],
+                        d["num_kv_heads"], d["head_dim"], d["page_size"], d["max_pages"],
+                        d["num_phys_pages"])
+
+
+def _select(kv=None, hq=32, budget_pages=0, budget_div=4, max_budget=16, ws=A, ws_bytes=1 << 30,
+            q=A, bounds=A, sel=A, cnt=A):
+    kv = kv or _kv()
+    return twl._lib.twl_select_pages(q, hq, C.byref(kv), bounds, budget_pages, budget_div,
+                                     max_budget, sel, cnt, None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(head_dim=64), twl.TWL_ERR_UNSUPPORTED),
+    (dict(page_size=32), twl.TWL_ERR_UNSUPPORTED),
+    (dict(max_pages=40000), twl.TWL_ERR_UNSUPPORTED),
+    (dict(batch=0), twl.TWL_ERR_INVALID_ARG),
+    (dict(num_kv_heads=0), twl.TWL_ERR_INVALID_ARG),
+    (dict(page_table=0), twl.TWL_ERR_INVALID_ARG),
+    (dict(seq_lens=0), twl.TWL_ERR_INVALID_ARG),
+    (dict(page_table=A + 2), twl.TWL_ERR_INVALID_ARG),
+])
+def test_select_rejects_bad_cache(over, code):
+    assert _select(kv=_kv(**over)) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(hq=12), twl.TWL_ERR_UNSUPPORTED),        # group of 12 / 8: not an integer
+    (dict(hq=24), twl.TWL_ERR_UNSUPPORTED),        # group 3
+    (dict(hq=128), twl.TWL_ERR_UNSUPPORTED),       # group 16
+    (dict(q=0), twl.TWL_ERR_INVALID_ARG),
+    (dict(q=A + 8), twl.TWL_ERR_INVALID_ARG),      # q must be 16-byte aligned
+    (dict(bounds=0), twl.TWL_ERR_INVALID_ARG),
+    (dict(sel=0), twl.TWL_ERR_INVALID_ARG),
+    (dict(max_budget=15), twl.TWL_ERR_INVALID_ARG),  # ceil(64 / 4) = 16 needed
+    (dict(max_budget=65), twl.TWL_ERR_INVALID_ARG),
+    (dict(budget_div=0), twl.TWL_ERR_INVALID_ARG),
+    (dict(budget_pages=-1), twl.TWL_ERR_INVALID_ARG),
+    (dict(budget_pages=8, max_budget=7), twl.TWL_ERR_INVALID_ARG),
+    (dict(ws=0), twl.TWL_ERR_WORKSPACE),
+    (dict(ws=A + 64), twl.TWL_ERR_WORKSPACE),
+    (dict(ws_bytes=1024), twl.TWL_ERR_WORKSPACE),
+])
+def test_select_rejects_bad_arguments(kw, code):
+    if kw.get("hq") == 12:
+        assert _select(**kw) == twl.TWL_ERR_INVALID_ARG
+        return
+    assert _select(**kw) == code
+
+
+@pytest.mark.parametrize("p,eps", [(0.0, 1e-6), (-0.5, 1e-6), (1.5, 1e-6), (float("nan"), 1e-6),
+                                   (0.9, 0.0), (0.9, -1e-6), (0.9, float("inf")),
+                                   (0.9, float("nan"))])
+def test_prune_rejects_bad_p_eps(p, eps):
+    st = twl._lib.twl_prune_top_p(A, None, 4, 1024, p, eps, A, A, None, None, 0, None)
+    assert st == twl.TWL_ERR_INVALID_ARG
+
+
+def test_prune_rejects_null_and_empty_is_ok():
+    assert twl._lib.twl_prune_top_p(0, None, 4, 16, 0.9, 1e-6, A, A, None, None, 0, None) == -1
+    assert twl._lib.twl_prune_top_p(A, None, 4, 0, 0.9, 1e-6, A, A, None, None, 0, None) == -1
+    assert twl._lib.twl_prune_top_p(A, None, -1, 16, 0.9, 1e-6, A, A, None, None, 0, None) == -1
+    # zero rows: nothing to do, nothing launched
+    assert twl._lib.twl_prune_top_p(A, None, 0, 16, 0.9, 1e-6, A, A, None, None, 0, None) == 0
+
+
+def test_decode_step_rejects_bad_arguments():
+    kv = _kv()
+    aux = twl._KAux(A, A, A)
+    f = twl._lib.twl_decode_step
+
+    def call(q=A, aux_=aux, p=0.85, eps=1e-6, o=A, lse=A, ws=A, ws_bytes=1 << 40, kvv=kv,
+             max_budget=16):
+        return f(q, 32, C.byref(kvv), C.byref(aux_), 0, 4, max_budget, p, eps, o, lse, None, ws,
+                 ws_bytes, None)
+
+    assert call(p=0.0) == twl.TWL_ERR_INVALID_ARG
+    assert call(eps=0.0) == twl.TWL_ERR_INVALID_ARG
+    assert call(o=0) == twl.TWL_ERR_INVALID_ARG
+    assert call(o=A + 4) == twl.TWL_ERR_INVALID_ARG
+    assert call(aux_=twl._KAux(A, 0, A)) == twl.TWL_ERR_INVALID_ARG
+    assert call(kvv=_kv(v=0)) == twl.TWL_ERR_INVALID_ARG
+    assert call(ws_bytes=100) == twl.TWL_ERR_WORKSPACE
+    assert call(max_budget=3) == twl.TWL_ERR_INVALID_ARG
+    assert call(kvv=_kv(batch=1024)) == twl.TWL_ERR_UNSUPPORTED   # 8192 groups > 4096
+
+
+def test_sparse_decode_rejects_bad_arguments():
+    kv = _kv()
+    f = twl._lib.twl_sparse_decode
+    assert f(A, 32, C.byref(kv), A, A, 0, 0.088, A, A, A, 1 << 30, None) == -1   # tok_stride 0
+    assert f(A, 32, C.byref(kv), A, A, 64, 0.0, A, A, A, 1 << 30, None) == -1    # sm_scale 0
+    assert f(A, 32, C.byref(kv), A, A, 64, 0.088, A, A, A, 16, None) == -5       # workspace
+
+
+def test_cache_calls_reject_bad_arguments():
+    kv = _kv()
+    assert twl._lib.twl_page_bounds(C.byref(kv), 0, None, 0, None) == -1
+    assert twl._lib.twl_page_bounds(C.byref(kv), A + 2, None, 0, None) == -1
+    assert twl._lib.twl_quantize_k(C.byref(kv), A, 0, None, 0, None) == -1
+    assert twl._lib.twl_quantize_k(C.byref(_kv(k=0)), A, A, None, 0, None) == -1
+    assert twl._lib.twl_page_bounds(C.byref(kv), A, A, 16, None) == -5
+
+
+def test_workspace_sizes():
+    wb = twl.twl_workspace_bytes
+    assert wb(twl.TWL_OP_CACHE) == 256
+    assert wb(99) == 0
+    s1 = wb(twl.TWL_OP_DECODE_STEP, 1, 32, 8, 2048, 512)
+    s2 = wb(twl.TWL_OP_DECODE_STEP, 2, 32, 8, 2048, 512)
+    assert 256 < s1 < s2
+    assert s1 % 256 == 0
+    assert wb(twl.TWL_OP_SELECT, 1, 32, 8, 2048) >= 256 + 32 * 2048 * 4
+    assert wb(twl.TWL_OP_SPARSE_DECODE, 1, 32, 8, 0, 0, 0, 4096) > 256
+    assert wb(twl.TWL_OP_DECODE_STEP, -1, 32, 8, 2048, 512) == 0
