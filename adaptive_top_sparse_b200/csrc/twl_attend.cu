@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(512)
                   const int* __restrict__ kept_idx, const int* __restrict__ kept_count,
                   const int* __restrict__ cand_count, int cand_stride, int* __restrict__ union_tok,
                   int* __restrict__ union_count, uint32_t* flags) {
-  extern __shared__ uint32_t bits[];  // [16 * max_pages / 32]
+  extern __shared__ uint32_t bits[];  // [ceil(16 * max_pages / 32)]
   __shared__ int scan_sh[33];
   const int gi = blockIdx.x, b = gi / kv.hkv, kvh = gi % kv.hkv;
   const int g = hq / kv.hkv;
@@ -303,7 +303,7 @@ cudaError_t launch_group_union(int hq, const KV& kv, const int* cand_tok, const 
                                const int* kept_count, const int* cand_count, int cand_stride,
                                int* union_tok, int* union_count, uint32_t* flags,
                                cudaStream_t s) {
-  const size_t smem = (size_t)(kv.max_pages * kPage / 32) * sizeof(uint32_t);
+  const size_t smem = (size_t)((kv.max_pages * kPage + 31) / 32) * sizeof(uint32_t);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k_group_union,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -58,8 +58,8 @@ __global__ void __launch_bounds__(kPruneThreads)
   top = block_max(top, red);
 
   float m;
-  if (n == 0) {
-    m = 0.f;
+  if (n == 0 || p >= 1.f) {
+    m = 0.f;  // p = 1 keeps every candidate: the mass test cannot resolve 1.0 in fp32
   } else if (mass_at_least(row, n, top, red) >= p) {
     m = top;
   } else {

@@ -186,8 +186,8 @@ twl_status twl_estimate(const void* q, int32_t num_q_heads, const twl_paged_kv* 
  * efficient top-p: find m with sum_{W[i] >= m} W[i] >= p in O(log(max W / eps)) rounds of O(n)
  * parallel work, no sort; [Summary] 4.2).  If mass(W >= max W) >= p then m = max W; else
  * lo = 0, hi = max W, mid = lo + (hi - lo)/2 (fp32); mass(W >= mid) >= p sets lo = mid, else
- * hi = mid; stop when hi - lo <= eps or mid no longer splits; m = lo.  Masses are fp32 block
- * sums in a fixed order.
+ * hi = mid; stop when hi - lo <= eps or mid no longer splits; m = lo.  p = 1 keeps every entry
+ * (m = 0).  Masses are fp32 block sums in a fixed order.
  *   m_out      float [rows] out
  *   kept_count int32 [rows] out = |{i : W_i >= m}|
  *   kept_idx   int32 [rows][row_stride] out (ascending indices) or NULL */

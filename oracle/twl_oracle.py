@@ -233,7 +233,8 @@ def top_p_bisect(w: np.ndarray, p: float, eps: float, max_iter: int = 64):
 
     Searches m with mass(w >= m) >= p: lo = 0, hi = max w; mid = lo + (hi - lo) / 2 in the
     dtype of ``w``; mass(>= mid) >= p moves lo up, else hi down; stops once hi - lo <= eps or
-    mid no longer splits the interval.  Masses are exact-ish fp64 sums.  Returns (m, kept).
+    mid no longer splits the interval; p >= 1 keeps every entry.  Masses are fp64 sums.
+    Returns (m, kept).
     """
     w = np.asarray(w)
     dt = w.dtype.type
@@ -243,7 +244,9 @@ def top_p_bisect(w: np.ndarray, p: float, eps: float, max_iter: int = 64):
         return float(w64[w >= t].sum())
 
     top = dt(w.max())
-    if mass(top) >= p:
+    if p >= 1.0:
+        m = dt(0.0)           # p = 1: the whole distribution, every candidate is kept
+    elif mass(top) >= p:
         m = top
     else:
         lo, hi = dt(0.0), top
