@@ -218,6 +218,7 @@ const char* twl_status_string(twl_status s) {
     case TWL_ERR_TIMEOUT: return "a bounded device wait gave up";
     case TWL_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case TWL_ERR_BAD_INDEX: return "page table, sequence length or index list out of range";
+    case TWL_ERR_SCRATCH_LIMIT: return "request exceeds the built-in scratch of the no-allocation call";
     default: return "unknown status";
   }
 }

@@ -27,6 +27,7 @@ TWL_ERR_CUDA = -3
 TWL_ERR_TIMEOUT = -4
 TWL_ERR_WORKSPACE = -5
 TWL_ERR_BAD_INDEX = -6
+TWL_ERR_SCRATCH_LIMIT = -7
 TWL_FLAG_BAD_INDEX = 1
 TWL_FLAG_TIMEOUT = 2
 
@@ -41,7 +42,8 @@ TWL_OP_DECODE_STEP = 7
 EXPORTED = [
     "twl_workspace_bytes", "twl_workspace_init", "twl_device_status", "twl_status_string",
     "twl_page_bounds", "twl_quantize_k", "twl_select_pages", "twl_estimate", "twl_prune_top_p",
-    "twl_group_union", "twl_sparse_decode", "twl_decode_step",
+    "twl_group_union", "twl_sparse_decode", "twl_decode_step", "twl_noalloc_scratch_bytes",
+    "twl_sparse_decode_noalloc",
 ]
 
 
@@ -85,6 +87,9 @@ _sigs = {
                                _sz, _vp]),
     "twl_sparse_decode": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _vp, _vp, _i32, _f32, _vp, _vp,
                                  _vp, _sz, _vp]),
+    "twl_noalloc_scratch_bytes": (_sz, []),
+    "twl_sparse_decode_noalloc": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _vp, _vp, _i32, _f32,
+                                         _vp, _vp, _vp]),
     "twl_decode_step": (_i32, [_vp, _i32, C.POINTER(_PagedKV), C.POINTER(_KAux), _i32, _i32,
                                _i32, _f32, _f32, _vp, _vp, C.POINTER(_StepStats), _vp, _sz,
                                _vp]),
@@ -259,3 +264,18 @@ def twl_decode_step(q, num_q_heads: int, kv: PagedKV, aux: KAux, budget_pages: i
     _check(_lib.twl_decode_step(_ptr(q), num_q_heads, C.byref(ckv), C.byref(caux), budget_pages,
                                 budget_div, max_budget, p, eps, _ptr(o), _ptr(lse), cst,
                                 _ptr(ws), _nbytes(ws), _stream(stream)), "twl_decode_step")
+
+
+def twl_noalloc_scratch_bytes() -> int:
+    return int(_lib.twl_noalloc_scratch_bytes())
+
+
+def twl_sparse_decode_noalloc(q, num_q_heads: int, kv: PagedKV, tok, tok_count, tok_stride: int,
+                              sm_scale: float, o, lse, stream=None) -> None:
+    """twl_sparse_decode without a workspace, for callers that cannot allocate device memory;
+    the scratch is a fixed-size array inside the library (see include/twl.h)."""
+    ckv = kv.c()
+    _check(_lib.twl_sparse_decode_noalloc(_ptr(q), num_q_heads, C.byref(ckv), _ptr(tok),
+                                          _ptr(tok_count), tok_stride, sm_scale, _ptr(o),
+                                          _ptr(lse), _stream(stream)),
+           "twl_sparse_decode_noalloc")

@@ -65,6 +65,7 @@ typedef int32_t twl_status;
 #define TWL_ERR_TIMEOUT (-4)     /* device flag: a bounded wait inside a kernel gave up */
 #define TWL_ERR_WORKSPACE (-5)   /* workspace NULL, misaligned or smaller than required */
 #define TWL_ERR_BAD_INDEX (-6)   /* device flag: page table / seq_lens / index list out of range */
+#define TWL_ERR_SCRATCH_LIMIT (-7) /* request larger than twl_sparse_decode_noalloc's scratch */
 
 /* Device flag bits reported by twl_device_status (sticky until cleared). */
 #define TWL_FLAG_BAD_INDEX 1u
@@ -219,6 +220,24 @@ twl_status twl_sparse_decode(const void* q, int32_t num_q_heads, const twl_paged
                              const int32_t* tok, const int32_t* tok_count, int32_t tok_stride,
                              float sm_scale, float* o, float* lse, void* ws, size_t ws_bytes,
                              twl_stream_t stream);
+
+/* ---------------------------------------------------------------- attend, no allocation
+ * The paper has no counterpart to this call; it serves callers that cannot allocate device
+ * memory for a workspace: plug-ins inside a framework that owns all device memory, real-time
+ * code that may not call cudaMalloc (it can synchronise the device), and deployments whose memory
+ * plan is fixed up front.  Same arguments and results as twl_sparse_decode, minus the workspace:
+ * the split-KV scratch comes from one statically sized device array inside the library
+ * (twl_noalloc_scratch_bytes() bytes, 8 MiB), held by every GPU that loads the library until the
+ * process exits.  A request whose scratch (twl_workspace_bytes(TWL_OP_SPARSE_DECODE, ...)) exceeds
+ * it returns TWL_ERR_SCRATCH_LIMIT and launches nothing.  The first call on a device looks up the
+ * array's device address (once per device, that device current); make it before any stream
+ * capture.  Every call shares the array: calls that overlap on the GPU race.  Device flags are not
+ * reported by this call.  It allocates nothing. */
+size_t twl_noalloc_scratch_bytes(void);
+twl_status twl_sparse_decode_noalloc(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
+                                     const int32_t* tok, const int32_t* tok_count,
+                                     int32_t tok_stride, float sm_scale, float* o, float* lse,
+                                     twl_stream_t stream);
 
 /* ---------------------------------------------------------------- the whole step
  * select -> estimate -> prune (p, eps) -> group union -> attend, with sm_scale = 1/sqrt(128)
