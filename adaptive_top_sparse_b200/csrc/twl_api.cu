@@ -2,7 +2,10 @@
 // Each entry point validates everything it can on the host before launching anything.
 #include <math.h>
 
+#include <mutex>
+
 #include "twl_common.cuh"
+#include "twl_fused.h"
 #include "twl_kernels.h"
 
 namespace twl {
@@ -91,6 +94,26 @@ twl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TWL_OK : TWL_E
 
 uint32_t* flags_of(void* ws) { return ws ? &reinterpret_cast<WsHeader*>(ws)->flags : nullptr; }
 
+// Cluster size for the fused kernel, cached per (device, group size, wanted size, smem).
+int fitted_cluster(int g, int want, int groups, int smem_bytes) {
+  struct Entry {
+    int dev, g, want, groups, smem, c;
+  };
+  static std::mutex mu;
+  static Entry cache[64];
+  static int n = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n; ++i)
+    if (cache[i].dev == dev && cache[i].g == g && cache[i].want == want &&
+        cache[i].groups == groups && cache[i].smem == smem_bytes)
+      return cache[i].c;
+  const int c = fit_cluster(g, want, groups, smem_bytes);
+  if (n < 64) cache[n++] = Entry{dev, g, want, groups, smem_bytes, c};
+  return c;
+}
+
 // ---------------------------------------------------------------- workspace layouts
 struct SelectWs {
   float* scores;
@@ -113,40 +136,6 @@ EstimateWs carve_estimate(Carve& c, int batch, int hq, int hkv, int max_pages) {
   w.union_pages = c.take<int>((size_t)batch * hkv * max_pages);
   w.union_mask = c.take<uint32_t>((size_t)batch * hkv * max_pages);
   w.union_npages = c.take<int>((size_t)batch * hkv);
-  return w;
-}
-
-struct StepWs {
-  SelectWs sel_ws;
-  EstimateWs est_ws;
-  int* sel_pages;
-  int* sel_count;
-  float* weights;
-  int* cand_tok;
-  int* cand_count;
-  float* m;
-  int* kept_count;
-  int* kept_idx;
-  int* union_tok;
-  int* union_count;
-  void* partials;
-};
-StepWs carve_step(Carve& c, int batch, int hq, int hkv, int max_pages, int max_budget) {
-  StepWs w;
-  const size_t bh = (size_t)batch * hq, cs = (size_t)kPage * max_budget;
-  w.sel_ws = carve_select(c, batch, hq, max_pages);
-  w.est_ws = carve_estimate(c, batch, hq, hkv, max_pages);
-  w.sel_pages = c.take<int>(bh * max_budget);
-  w.sel_count = c.take<int>(bh);
-  w.weights = c.take<float>(bh * cs);
-  w.cand_tok = c.take<int>(bh * cs);
-  w.cand_count = c.take<int>(bh);
-  w.m = c.take<float>(bh);
-  w.kept_count = c.take<int>(bh);
-  w.kept_idx = c.take<int>(bh * cs);
-  w.union_tok = c.take<int>((size_t)batch * hkv * kPage * max_pages);
-  w.union_count = c.take<int>((size_t)batch * hkv);
-  w.partials = c.take<char>(attend_partial_bytes(batch, hq, hkv, kPage * max_pages));
   return w;
 }
 
@@ -181,8 +170,10 @@ size_t twl_workspace_bytes(int32_t op, int32_t batch, int32_t num_q_heads, int32
       c.take<char>(attend_partial_bytes(batch, num_q_heads, num_kv_heads, row_stride));
       break;
     case TWL_OP_DECODE_STEP:
-      if (num_kv_heads < 1) return 0;
-      carve_step(c, batch, num_q_heads, num_kv_heads, max_pages, max_budget);
+      if (num_kv_heads < 1 || num_q_heads < num_kv_heads || max_pages < 1 || max_budget < 1)
+        return 0;
+      c.take<char>(fused_workspace_bytes(batch, num_q_heads, num_kv_heads, max_pages,
+                                         max_budget));
       break;
     default:
       return 0;
@@ -369,53 +360,48 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
     return TWL_ERR_INVALID_ARG;
   if (!(p > 0.f && p <= 1.f) || !(eps > 0.f) || isinf(eps)) return TWL_ERR_INVALID_ARG;
   if ((st = check_budget(budget_pages, budget_div, max_budget, k.max_pages)) != TWL_OK) return st;
-  if (k.batch * k.hkv > 4096) return TWL_ERR_UNSUPPORTED;
+  FusedPlan pl = plan_fused(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
+  if (!pl.ok) return TWL_ERR_UNSUPPORTED;
   Carve c{static_cast<char*>(ws)};
-  StepWs w = carve_step(c, k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
+  char* fws = c.take<char>(fused_workspace_bytes(k.batch, num_q_heads, k.hkv, k.max_pages,
+                                                 max_budget));
   if ((st = check_ws(ws, ws_bytes, c.off)) != TWL_OK) return st;
+  pl.cluster = fitted_cluster(num_q_heads / k.hkv, pl.cluster, k.batch * k.hkv, pl.smem_bytes);
   const twl_step_stats none = {};
   const twl_step_stats& so = stats ? *stats : none;
-  int* sel_pages = so.sel_pages ? so.sel_pages : w.sel_pages;
-  int* sel_count = so.sel_count ? so.sel_count : w.sel_count;
-  float* weights = so.weights ? so.weights : w.weights;
-  int* cand_tok = so.cand_tok ? so.cand_tok : w.cand_tok;
-  int* cand_count = so.cand_count ? so.cand_count : w.cand_count;
-  float* m = so.threshold ? so.threshold : w.m;
-  int* kept_count = so.kept_count ? so.kept_count : w.kept_count;
-  int* union_tok = so.union_tok ? so.union_tok : w.union_tok;
-  int* union_count = so.union_count ? so.union_count : w.union_count;
-  const int cs = kPage * max_budget;
-  const uint16_t* qh = static_cast<const uint16_t*>(q);
-  cudaStream_t s = (cudaStream_t)stream;
-  uint32_t* fl = flags_of(ws);
-  cudaError_t e = launch_page_scores(qh, num_q_heads, k,
-                                     static_cast<const uint16_t*>(aux->bounds),
-                                     w.sel_ws.scores, fl, s);
-  if (e == cudaSuccess)
-    e = launch_topk_pages(w.sel_ws.scores, num_q_heads, k, budget_pages, budget_div, max_budget,
-                          sel_pages, sel_count, fl, s);
-  if (e == cudaSuccess)
-    e = launch_union_pages(num_q_heads, k, sel_pages, sel_count, max_budget, w.est_ws.rank,
-                           w.est_ws.union_pages, w.est_ws.union_mask, w.est_ws.union_npages, fl,
-                           s);
-  if (e == cudaSuccess)
-    e = launch_estimate_logits(qh, num_q_heads, k, static_cast<const uint8_t*>(aux->k_int4),
-                               static_cast<const uint16_t*>(aux->k_scale_zero), w.est_ws.rank,
-                               w.est_ws.union_pages, w.est_ws.union_mask, w.est_ws.union_npages,
-                               cs, weights, cand_tok, fl, s);
-  if (e == cudaSuccess)
-    e = launch_softmax_rows(num_q_heads, k, sel_pages, sel_count, max_budget, weights,
-                            cand_count, s);
-  if (e == cudaSuccess)
-    e = launch_prune(weights, cand_count, nullptr, k.batch * num_q_heads, cs, p, eps, m,
-                     kept_count, w.kept_idx, s);
-  if (e == cudaSuccess)
-    e = launch_group_union(num_q_heads, k, cand_tok, w.kept_idx, kept_count, cand_count, cs,
-                           union_tok, union_count, fl, s);
-  if (e == cudaSuccess)
-    e = launch_sparse_decode(qh, num_q_heads, k, union_tok, union_count, kPage * k.max_pages,
-                             0.08838834764831845f, o, lse, w.partials, fl, s);
-  return cuda_status(e);
+  FusedArgs a = {};
+  a.q = static_cast<const uint16_t*>(q);
+  a.hq = num_q_heads;
+  a.kv = k;
+  a.k_int4 = static_cast<const uint8_t*>(aux->k_int4);
+  a.k_sz = static_cast<const uint16_t*>(aux->k_scale_zero);
+  a.bounds = static_cast<const uint16_t*>(aux->bounds);
+  a.budget_pages = budget_pages;
+  a.budget_div = budget_div;
+  a.max_budget = max_budget;
+  a.p = p;
+  a.eps = eps;
+  a.sm_scale = 0.08838834764831845f;
+  a.o = o;
+  a.lse = lse;
+  a.sel_pages = so.sel_pages;
+  a.sel_count = so.sel_count;
+  a.weights_out = so.weights;
+  a.cand_tok = so.cand_tok;
+  a.cand_count = so.cand_count;
+  a.threshold = so.threshold;
+  a.kept_count = so.kept_count;
+  a.union_count = so.union_count;
+  a.union_tok = so.union_tok;
+  a.flags = flags_of(ws);
+  a.sel_words = pl.sel_words;
+  a.cand_stride = pl.cand_stride;
+  a.kept_words = pl.kept_words;
+  a.union_stride = pl.union_stride;
+  a.cluster = pl.cluster;
+  a.smem_bytes = pl.smem_bytes;
+  carve_fused(a, fws, pl, k.batch, num_q_heads, k.hkv, k.max_pages);
+  return cuda_status(launch_fused(a, pl, (cudaStream_t)stream));
 }
 
 }  // extern "C"

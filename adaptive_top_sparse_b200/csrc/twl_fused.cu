@@ -1,0 +1,1525 @@
+// The fused decode step: select -> INT4 estimate -> top-p prune -> group union -> attention in one
+// kernel, one thread-block cluster per (sequence, kv-head) group.
+//
+// "Twilight: Adaptive Attention Sparsity with Hierarchical Top-p Pruning": notes page, "Overall
+// framework" (select-then-prune) and "Key designs" (binary-search top-p, 4-bit K cache, head
+// flattening); summary, sections 4.1-4.3 and appendices B.1-B.2 (INT4 SpGEMV once per GQA group
+// over the union of the heads' pages, group-wise variable-length attention).
+//
+// Every dependency of the path stays inside one GQA group, so a group is processed by one cluster
+// of C CTAs (C = 16 at batch 1, down to 1 when there are enough groups to fill the GPU), and the
+// phases are separated by hardware cluster barriers instead of kernel boundaries:
+//   1 scores   CTA r scores pages [r P/C, (r+1) P/C) of every head of the group  -> L2
+//   2 top-k    one owner CTA per head radix-selects its k pages               -> page bitmap
+//   3 union    every CTA ORs the head bitmaps; ranks come from prefix popcounts
+//   4 estimate CTA r takes an even share of the union pages; one warp per page runs the INT4
+//              dequant-dot on the tensor cores for all heads that selected it    -> logits
+//   5 prune    the owner CTA of each head normalises its weights and bisects the threshold
+//   6 union    CTA r ORs the heads' kept bits on its pages; counts are exchanged, then the
+//              group's kept tokens are written in ascending order
+//   7 attend   CTA r gathers an even share of the kept K/V rows; partial (o, lse) per CTA
+//   8 merge    the owner CTA of each head merges the C partials by log-sum-exp.
+// Data that crosses CTAs goes through global memory (it stays in L2) with L1-bypassing loads;
+// the cluster barrier's release/acquire orders it.  Every CTA executes every barrier: no barrier
+// sits behind a data-dependent branch, and a group whose sequence is invalid exits before the
+// first one, uniformly across its cluster.  Arithmetic and summation orders match the staged
+// kernels, so the selection is bit-identical to twl_select_pages.
+#include <cooperative_groups.h>
+#include <stdlib.h>
+
+#include "twl_common.cuh"
+#include "twl_fused.h"
+#include "twl_kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace twl {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kAttChunk = 64;  // tokens gathered per attention round
+
+__device__ __forceinline__ void cluster_sync() { cg::this_cluster().sync(); }
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+  return n;
+}
+
+// Optional phase timestamps (compile with -DTWL_PHASE_TIMING): thread 0 of the first CTA of the
+// first cluster records %globaltimer at each phase boundary into the workspace header (words
+// 8..63 as 64-bit values; word 1 = the cluster size launched).  Off by default.
+#ifdef TWL_PHASE_TIMING
+__device__ __forceinline__ void stamp(const FusedArgs& a, int slot) {
+  if (blockIdx.x == 0 && threadIdx.x == 0 && a.flags) {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    reinterpret_cast<uint64_t*>(a.flags)[4 + slot] = t;
+    a.flags[1] = cluster_size();
+  }
+}
+#else
+__device__ __forceinline__ void stamp(const FusedArgs&, int) {}
+#endif
+
+__device__ __forceinline__ float ldcg_f(const float* p) { return __ldcg(p); }
+__device__ __forceinline__ int ldcg_i(const int* p) { return __ldcg(p); }
+__device__ __forceinline__ uint32_t ldcg_u(const uint32_t* p) { return __ldcg(p); }
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// Same fragment map as the staged estimate kernel (see twl_estimate.cu).
+__device__ __forceinline__ void q_fragments(const uint16_t* qh, bool valid, uint32_t (&bf)[8][2]) {
+  const int t = threadIdx.x & 3;
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v =
+        valid ? *reinterpret_cast<const uint4*>(qh + 32 * t + 8 * i) : make_uint4(0, 0, 0, 0);
+    w[4 * i + 0] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+  }
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int w8 = ks >> 1, e = ks & 1;
+    bf[ks][0] = __byte_perm(w[4 * w8 + e], w[4 * w8 + e + 2], 0x5410);
+    bf[ks][1] = __byte_perm(w[4 * w8 + e], w[4 * w8 + e + 2], 0x7632);
+  }
+}
+
+__device__ __forceinline__ uint32_t nib_pair(uint32_t x, int i) {
+  uint32_t v = ((x >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&v), __float2half2_rn(1024.f));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// Bytes of the persistent bitmap region, rounded up so the scratch region after it is 128-byte
+// aligned (the attention phase does 16-byte vector and cp.async accesses into it).
+__host__ __device__ constexpr int persistent_bytes(int g, int sel_words) {
+  return ((4 * (2 * g + 2) * sel_words) + 127) & ~127;
+}
+
+// Shared-memory layout: a persistent region for the page bitmaps (phases 3-6) and one scratch
+// region reused by the phases.
+struct Smem {
+  uint32_t* hbits;  // [G][nw]  head page bitmaps
+  int* hpre;        // [G][nw]  exclusive prefix popcounts per word
+  uint32_t* ubits;  // [nw]     union bitmap
+  int* upre;        // [nw]     exclusive prefix popcounts of the union
+  unsigned char* scratch;
+  int scratch_bytes;
+  int nw;
+};
+
+__device__ __forceinline__ int rank_in(const uint32_t* bits, const int* pre, int j) {
+  const int w = j >> 5, b = j & 31;
+  return pre[w] + __popc(bits[w] & ((1u << b) - 1u));
+}
+
+// Position of the k-th (0-based) set bit of w; requires popc(w) > k.
+__device__ __forceinline__ int nth_set_bit(uint32_t w, int k) {
+  int pos = 0;
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) {
+    const int c = __popc(w & ((1u << s) - 1u));
+    if (k >= c) {
+      k -= c;
+      w >>= s;
+      pos += s;
+    }
+  }
+  return pos;
+}
+
+// j of the u-th set bit of the union (u < total), via binary search over the prefix table.
+__device__ __forceinline__ int union_select(const uint32_t* ubits, const int* upre, int nw, int u) {
+  int lo = 0, hi = nw;  // upre[lo] <= u < upre[hi] (upre[nw] = total implied)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (upre[mid] <= u) lo = mid;
+    else hi = mid;
+  }
+  return 32 * lo + nth_set_bit(ubits[lo], u - upre[lo]);
+}
+
+// ------------------------------------------------------------------------- phase 1: scores
+// The CTA's slice of the page table is staged in shared memory first (one coalesced read), so
+// the bounds loads of kIt page pairs per warp are all independent and in flight together.
+template <int G>
+__device__ void phase_scores(const FusedArgs& a, int b, int kvh, int n_pages, int r, int C,
+                             Smem& sm) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = lane >> 4, l = lane & 15;
+  const int p0 = (int)((long)n_pages * r / C), p1 = (int)((long)n_pages * (r + 1) / C);
+  int* phys = reinterpret_cast<int*>(sm.scratch);  // [p1 - p0]
+  for (int j = p0 + (int)threadIdx.x; j < p1; j += kThreads)
+    phys[j - p0] = load_phys(a.kv.page_table, b, j, a.kv.max_pages, a.kv.num_phys, a.flags);
+  float qv[G][8];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(
+        a.q + ((size_t)b * a.hq + kvh * G + h) * kHeadDim + 8 * l);
+    unpack8(raw, qv[h]);
+  }
+  __syncthreads();
+  constexpr int kIt = G <= 4 ? 4 : 2;  // page pairs in flight per warp
+  for (int base = p0; base < p1; base += kWarps * 2 * kIt) {
+    uint4 bmn[kIt], bmx[kIt];
+    bool ok[kIt];
+#pragma unroll
+    for (int it = 0; it < kIt; ++it) {
+      const int j = base + it * kWarps * 2 + 2 * warp + half;
+      const int ph = j < p1 ? phys[j - p0] : -1;
+      ok[it] = ph >= 0;
+      bmn[it] = make_uint4(0, 0, 0, 0);
+      bmx[it] = bmn[it];
+      if (ok[it]) {
+        const uint16_t* src = a.bounds + (((size_t)ph * a.kv.hkv + kvh) * 2) * kHeadDim + 8 * l;
+        bmn[it] = __ldg(reinterpret_cast<const uint4*>(src));
+        bmx[it] = __ldg(reinterpret_cast<const uint4*>(src + kHeadDim));
+      }
+    }
+#pragma unroll
+    for (int it = 0; it < kIt; ++it) {
+      float mn[8], mx[8];
+      unpack8(bmn[it], mn);
+      unpack8(bmx[it], mx);
+      float acc[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float sc = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) sc = __fmaf_rn(qv[h][c], qv[h][c] > 0.f ? mx[c] : mn[c], sc);
+        acc[h] = sc;
+      }
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) {
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+          acc[h] = __fadd_rn(acc[h], __shfl_xor_sync(0xffffffffu, acc[h], off));
+      }
+      const int j = base + it * kWarps * 2 + 2 * warp + half;
+      if (j < p1 && l < G) {
+        float v = acc[0];
+#pragma unroll
+        for (int h = 1; h < G; ++h) v = (l == h) ? acc[h] : v;
+        if (!ok[it]) v = -INFINITY;
+        a.scores[((size_t)b * a.hq + kvh * G + l) * a.kv.max_pages + j] = v;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------- phase 2: top-k
+// Radix select of the kb largest keys (ties to the lower index) -> bitmap of selected pages.
+__device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb, Smem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = sm.nw;
+  uint32_t* out_bits = a.selbits + (size_t)bh * a.sel_words;
+  int* sel_list = a.sel_pages ? a.sel_pages + (size_t)bh * a.max_budget : nullptr;
+  if (n_pages <= kb) {
+    for (int w = tid; w < nw; w += kThreads) {
+      const int lo = 32 * w;
+      uint32_t m = 0xFFFFFFFFu;
+      if (lo + 32 > n_pages) m = n_pages > lo ? ((1u << (n_pages - lo)) - 1u) : 0u;
+      out_bits[w] = m;
+    }
+    if (sel_list)
+      for (int i = tid; i < n_pages; i += kThreads) sel_list[i] = i;
+    if (tid == 0 && a.sel_count) a.sel_count[bh] = n_pages;
+    return;
+  }
+  // keys in shared memory when they fit, else read from L2 on every pass
+  const float* row = a.scores + (size_t)bh * a.kv.max_pages;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sm.scratch);           // 256
+  int* scan_sh = reinterpret_cast<int*>(sm.scratch + 1024);           // 33
+  uint32_t* state = reinterpret_cast<uint32_t*>(sm.scratch + 1200);   // 2
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm.scratch + 1280);
+  const bool staged = 1280 + 4 * n_pages <= sm.scratch_bytes;
+  if (staged) {
+    constexpr int kB = 8;  // independent loads in flight per thread
+    for (int base = 0; base < n_pages; base += kThreads * kB) {
+      float v[kB];
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int i = base + k * kThreads + tid;
+        v[k] = i < n_pages ? ldcg_f(row + i) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int i = base + k * kThreads + tid;
+        if (i < n_pages) keys[i] = f32_key(v[k]);
+      }
+    }
+  }
+  __syncthreads();
+  stamp(a, 23);
+  auto key_at = [&](int i) -> uint32_t { return staged ? keys[i] : f32_key(ldcg_f(row + i)); };
+
+  // Radix select over the bits where this head's keys differ: the common prefix of the smallest
+  // and largest key is known, the rest is split into at most three digits (9 bits each when
+  // that suffices, else 8-bit digits).  Histograms are per warp (no cross-warp atomics).
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int i = tid; i < n_pages; i += kThreads) {
+    const uint32_t k = key_at(i);
+    kmin = min(kmin, k);
+    kmax = max(kmax, k);
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  __syncthreads();
+  if (lane == 0) {
+    hist[2 * warp] = kmin;
+    hist[2 * warp + 1] = kmax;
+  }
+  __syncthreads();
+  kmin = 0xFFFFFFFFu;
+  kmax = 0u;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    kmin = min(kmin, hist[2 * w]);
+    kmax = max(kmax, hist[2 * w + 1]);
+  }
+  const uint32_t diff = kmin ^ kmax;
+  uint32_t prefix, mask;
+  int remaining = kb;
+  int eq_count = n_pages;  // keys equal to the final prefix (all keys when they are all equal)
+  int hi_bit = diff ? 31 - __clz(diff) : -1;
+  mask = hi_bit >= 31 ? 0u : ~((2u << hi_bit) - 1u);
+  if (hi_bit < 0) mask = 0xFFFFFFFFu;
+  prefix = kmax & mask;
+  const int nbits = hi_bit + 1;
+  // per-warp histograms [kWarps][1 << dw] after the staged keys, then the bin totals
+  uint32_t* whist = reinterpret_cast<uint32_t*>(sm.scratch + 1280 + 4 * n_pages);
+  const bool whist_ok =
+      staged && 1280 + 4 * n_pages + 4 * kWarps * 512 + 2048 <= sm.scratch_bytes;
+  // digit width: three digits of up to 9 bits when the per-warp histograms fit, else 8 bits
+  // (the shared 256-bin histogram)
+  const int dw = (whist_ok && nbits <= 27) ? (nbits + 2) / 3 : 8;
+  uint32_t* tot = whist_ok ? whist + kWarps * (1 << dw) : hist;  // [1 << dw] totals
+  const int n_iter = (n_pages + kThreads - 1) / kThreads;
+#pragma unroll 1
+  while (hi_bit >= 0) {
+    const int lo_bit = max(hi_bit - dw + 1, 0);
+    const int width = hi_bit - lo_bit + 1;
+    const int nb = 1 << width;
+    const uint32_t dmask = (uint32_t)nb - 1u;
+    if (whist_ok) {
+      for (int i = tid; i < kWarps * nb; i += kThreads) whist[i] = 0u;
+    } else {
+      for (int i = tid; i < nb; i += kThreads) tot[i] = 0u;
+    }
+    __syncthreads();
+    uint32_t* my = whist_ok ? whist + warp * nb : tot;
+#pragma unroll 1
+    for (int it = 0; it < n_iter; ++it) {
+      const int i = it * kThreads + tid;
+      bool take = false;
+      uint32_t digit = 0;
+      if (i < n_pages) {
+        const uint32_t key = key_at(i);
+        take = (key & mask) == prefix;
+        digit = (key >> lo_bit) & dmask;
+      }
+      const uint32_t tag = take ? digit : 1024u + lane;
+      const uint32_t peers = __match_any_sync(0xffffffffu, tag);
+      if (take && (__ffs(peers) - 1) == lane) atomicAdd(&my[digit], (uint32_t)__popc(peers));
+    }
+    __syncthreads();
+    if (whist_ok) {
+      for (int bin = tid; bin < nb; bin += kThreads) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) t += whist[w * nb + bin];
+        tot[bin] = t;
+      }
+      __syncthreads();
+    }
+    if (warp == 0) {
+      // lane l covers the bins nb-1-l*per .. nb-per-l*per (descending)
+      const int per = (nb + 31) / 32;
+      uint32_t lsum = 0;
+      for (int e = 0; e < per; ++e) {
+        const int bin = nb - 1 - lane * per - e;
+        if (bin >= 0) lsum += tot[bin];
+      }
+      uint32_t incl = lsum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - lsum;
+      if (excl < (uint32_t)remaining && incl >= (uint32_t)remaining) {
+        uint32_t run = excl;
+        for (int e = 0; e < per; ++e) {
+          const int bin = nb - 1 - lane * per - e;
+          if (bin < 0) break;
+          const uint32_t c = tot[bin];
+          if (run + c >= (uint32_t)remaining) {
+            state[0] = prefix | ((uint32_t)bin << lo_bit);
+            state[1] = (uint32_t)remaining - run;
+            state[2] = c;
+            break;
+          }
+          run += c;
+        }
+      }
+    }
+    __syncthreads();
+    prefix = state[0];
+    remaining = (int)state[1];
+    eq_count = (int)state[2];
+    mask |= dmask << lo_bit;
+    hi_bit = lo_bit - 1;
+    __syncthreads();
+  }
+  if (eq_count == remaining && sel_list == nullptr) {
+    // every key equal to the k-th is taken: one ballot per 32-page word, no ordering needed
+    for (int base = 0; base < 32 * nw; base += kThreads) {
+      const int i = base + tid;
+      const bool in = i < n_pages;
+      const uint32_t key = in ? key_at(i) : 0u;
+      const uint32_t sel = __ballot_sync(0xffffffffu, in && key >= prefix);
+      if (lane == 0 && (i >> 5) < nw) out_bits[i >> 5] = sel;
+    }
+    if (tid == 0 && a.sel_count) a.sel_count[bh] = kb;
+    return;
+  }
+  stamp(a, 24);
+  // Keys above the k-th are taken; equal keys are taken in ascending page order.  One element
+  // per thread per round; a warp's ballot is one 32-page word of the bitmap.
+  int* wsum = scan_sh;  // [kWarps] per-warp counts, then their prefix
+  int carry_eq = 0, carry_sel = 0;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int base = 0; base < 32 * nw; base += kThreads) {
+    const int i = base + tid;
+    const bool in = i < n_pages;
+    const uint32_t key = in ? key_at(i) : 0u;
+    const uint32_t gt = __ballot_sync(0xffffffffu, in && key > prefix);
+    const uint32_t eq = __ballot_sync(0xffffffffu, in && key == prefix);
+    if (lane == 0) wsum[warp] = __popc(eq);
+    __syncthreads();
+    int eq_before = carry_eq, eq_round = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      if (w < warp) eq_before += wsum[w];
+      eq_round += wsum[w];
+    }
+    const bool take = in && key == prefix && eq_before + __popc(eq & lt) < remaining;
+    const uint32_t sel = gt | __ballot_sync(0xffffffffu, take);
+    __syncthreads();
+    if (lane == 0) wsum[warp] = __popc(sel);
+    __syncthreads();
+    int sel_before = carry_sel, sel_round = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      if (w < warp) sel_before += wsum[w];
+      sel_round += wsum[w];
+    }
+    const int word = i >> 5;
+    if (lane == 0 && word < nw) out_bits[word] = sel;
+    if (sel_list && ((sel >> lane) & 1u)) sel_list[sel_before + __popc(sel & lt)] = i;
+    carry_eq += eq_round;
+    carry_sel += sel_round;
+    __syncthreads();
+  }
+  if (tid == 0 && a.sel_count) a.sel_count[bh] = kb;
+}
+
+// ------------------------------------------------------------------------- phase 3: bitmaps
+template <int G>
+__device__ void phase_union_bitmaps(const FusedArgs& a, int b, int kvh, Smem& sm, int* s_total,
+                                    int* scan_sh) {
+  const int tid = threadIdx.x, nw = sm.nw;
+  for (int i = tid; i < G * nw; i += kThreads) {
+    const int h = i / nw, w = i % nw;
+    sm.hbits[i] = ldcg_u(a.selbits + (size_t)(b * a.hq + kvh * G + h) * a.sel_words + w);
+  }
+  __syncthreads();
+  for (int w = tid; w < nw; w += kThreads) {
+    uint32_t u = 0;
+#pragma unroll
+    for (int h = 0; h < G; ++h) u |= sm.hbits[h * nw + w];
+    sm.ubits[w] = u;
+  }
+  __syncthreads();
+  // exclusive prefix popcounts of the union and of every head bitmap, in one scan per round
+  // of kThreads words (warp scans, then the warp totals)
+  int* wtot = reinterpret_cast<int*>(sm.scratch);  // [kWarps][G + 1]
+  const int lane = tid & 31, warp = tid >> 5;
+  int carry[G + 1];
+#pragma unroll
+  for (int h = 0; h <= G; ++h) carry[h] = 0;
+  for (int base = 0; base < nw; base += kThreads) {
+    const int w = base + tid;
+    int x[G + 1], v[G + 1];
+#pragma unroll
+    for (int h = 0; h <= G; ++h) {
+      v[h] = w < nw ? __popc(h == 0 ? sm.ubits[w] : sm.hbits[(h - 1) * nw + w]) : 0;
+      x[h] = v[h];
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+      for (int h = 0; h <= G; ++h) {
+        const int y = __shfl_up_sync(0xffffffffu, x[h], o);
+        if (lane >= o) x[h] += y;
+      }
+    }
+    if (lane == 31) {
+#pragma unroll
+      for (int h = 0; h <= G; ++h) wtot[warp * (G + 1) + h] = x[h];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h <= G; ++h) {
+      int before = carry[h], round = 0;
+      for (int ww = 0; ww < kWarps; ++ww) {
+        const int t = wtot[ww * (G + 1) + h];
+        if (ww < warp) before += t;
+        round += t;
+      }
+      if (w < nw) {
+        if (h == 0) sm.upre[w] = before + x[h] - v[h];
+        else sm.hpre[(h - 1) * nw + w] = before + x[h] - v[h];
+      }
+      carry[h] += round;
+    }
+    __syncthreads();
+  }
+  if (tid == 0) *s_total = carry[0];
+  __syncthreads();
+}
+
+// ------------------------------------------------------------------------- phase 4: estimate
+// The CTA's share of the union is processed in chunks of up to kEstChunk pages: first every
+// page's logical id and physical page are staged in shared memory (thread per page), then each
+// warp takes kEstBatch pages at a time and issues all their INT4 loads before computing.
+constexpr int kEstChunk = 1024;
+constexpr int kEstBatch = 4;
+
+template <int G>
+__device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n, int U, int r,
+                               int C, Smem& sm) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gr = lane >> 2, t = lane & 3;
+  const int nw = sm.nw;
+  const float inv_sqrt_d = 0.08838834764831845f;
+  const int u0 = (int)((long)U * r / C), u1 = (int)((long)U * (r + 1) / C);
+  float* red = reinterpret_cast<float*>(sm.scratch);                  // [kWarps][8][2]
+  int* pj = reinterpret_cast<int*>(sm.scratch + 2048);                 // [kEstChunk]
+  int* pph = reinterpret_cast<int*>(sm.scratch + 2048 + 4 * kEstChunk);  // [kEstChunk]
+  uint32_t bf[8][2];
+  const bool head_ok = gr < G;
+  const uint16_t* qh = a.q + ((size_t)b * a.hq + kvh * G + (head_ok ? gr : 0)) * kHeadDim;
+  q_fragments(qh, head_ok, bf);
+  float qs_part = 0.f;
+  if (head_ok) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) qs_part += __half2float(__ushort_as_half(qh[32 * t + i]));
+  }
+  qs_part += __shfl_xor_sync(0xffffffffu, qs_part, 1);
+  qs_part += __shfl_xor_sync(0xffffffffu, qs_part, 2);
+  const float qsum0 = __shfl_sync(0xffffffffu, qs_part, (2 * t) * 4);
+  const float qsum1 = __shfl_sync(0xffffffffu, qs_part, (2 * t + 1) * 4);
+  // running max of this lane's two heads over its rows (the softmax's shift)
+  float rm[2] = {-INFINITY, -INFINITY};
+
+  for (int c0 = u0; c0 < u1; c0 += kEstChunk) {
+    const int cn = min(kEstChunk, u1 - c0);
+    __syncthreads();  // previous chunk's staging fully consumed
+    for (int i = threadIdx.x; i < cn; i += kThreads) {
+      const int j = union_select(sm.ubits, sm.upre, nw, c0 + i);
+      pj[i] = j;
+      pph[i] = load_phys(a.kv.page_table, b, j, a.kv.max_pages, a.kv.num_phys, a.flags);
+    }
+    __syncthreads();
+    for (int i0 = warp * kEstBatch; i0 < cn; i0 += kWarps * kEstBatch) {
+      uint4 x0[kEstBatch], x1[kEstBatch];
+      uint32_t sz0[kEstBatch], sz1[kEstBatch];
+#pragma unroll
+      for (int k = 0; k < kEstBatch; ++k) {
+        const int i = i0 + k;
+        const int ph = i < cn ? pph[i] : -1;
+        x0[k] = make_uint4(0, 0, 0, 0);
+        x1[k] = x0[k];
+        sz0[k] = sz1[k] = 0;
+        if (ph >= 0) {
+          const size_t tile = ((size_t)ph * a.kv.hkv + kvh) * kPage;
+          const uint4* src = reinterpret_cast<const uint4*>(a.k_int4 + tile * (kHeadDim / 2));
+          x0[k] = __ldg(src + lane);
+          x1[k] = __ldg(src + 32 + lane);
+          sz0[k] = __ldg(reinterpret_cast<const uint32_t*>(a.k_sz + tile * 2) + gr);
+          sz1[k] = __ldg(reinterpret_cast<const uint32_t*>(a.k_sz + tile * 2) + gr + 8);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kEstBatch; ++k) {
+        const int i = i0 + k;
+        if (i >= cn) break;  // warp-uniform
+        const int j = pj[i];
+        const bool bad = pph[i] < 0;
+        const uint32_t r0[4] = {x0[k].x, x0[k].y, x0[k].z, x0[k].w};
+        const uint32_t r1[4] = {x1[k].x, x1[k].y, x1[k].z, x1[k].w};
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const int w8 = ks >> 1, e = ks & 1;
+          uint32_t av[4];
+          av[0] = nib_pair(r0[w8], 2 * e);
+          av[1] = nib_pair(r1[w8], 2 * e);
+          av[2] = nib_pair(r0[w8], 2 * e + 1);
+          av[3] = nib_pair(r1[w8], 2 * e + 1);
+          mma_16816(acc, av, bf[ks][0], bf[ks][1]);
+        }
+        const int rows = page_rows(n, j);
+        const float s0 = __half2float(__ushort_as_half((unsigned short)(sz0[k] & 0xFFFFu)));
+        const float z0 = __half2float(__ushort_as_half((unsigned short)(sz0[k] >> 16)));
+        const float s1 = __half2float(__ushort_as_half((unsigned short)(sz1[k] & 0xFFFFu)));
+        const float z1 = __half2float(__ushort_as_half((unsigned short)(sz1[k] >> 16)));
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int hl = 2 * t + e;
+          if (hl >= G) continue;
+          const uint32_t* hb = sm.hbits + hl * nw;
+          if (!((hb[j >> 5] >> (j & 31)) & 1u)) continue;
+          const int bh = b * a.hq + kvh * G + hl;
+          const int rk = rank_in(hb, sm.hpre + hl * nw, j);
+          const float qsum = e ? qsum1 : qsum0;
+          const size_t obase = (size_t)bh * a.cand_stride + (size_t)rk * kPage;
+#pragma unroll
+          for (int rr = 0; rr < 2; ++rr) {
+            const int row = gr + 8 * rr;
+            if (row >= rows) continue;
+            const float sv = rr ? s1 : s0, zv = rr ? z1 : z0;
+            const float lg = bad ? -INFINITY : (sv * acc[2 * rr + e] + zv * qsum) * inv_sqrt_d;
+            a.logits[obase + row] = lg;
+            if (a.cand_tok) a.cand_tok[obase + row] = kPage * j + row;
+            rm[e] = fmaxf(rm[e], lg);
+          }
+        }
+      }
+    }
+  }
+  // combine the maxima over the 8 row-lanes of each head, then over the warps
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) rm[e] = fmaxf(rm[e], __shfl_xor_sync(0xffffffffu, rm[e], off));
+  }
+  __syncthreads();
+  if (lane < 4) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) red[warp * 8 + 2 * lane + e] = rm[e];
+  }
+  __syncthreads();
+  if (threadIdx.x < G) {
+    const int hl = threadIdx.x;
+    float m = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, red[w * 8 + hl]);
+    a.part_ms[((size_t)gi * C * G + r * G + hl) * 2] = m;
+  }
+}
+
+// ------------------------------------------------------------------------- phase 5: prune
+__device__ float block_sum_fixed(float v, float* red) {
+  // sum over the block in a fixed order; every thread receives the total
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) t += red[w];
+  return t;
+}
+
+// Bisection of the notes page's "Key designs" (efficient top-p), three levels per block
+// reduction: the seven midpoints the sequential search could visit next are computed exactly as it
+// would compute them (mid = lo + (hi - lo) * 0.5 in fp32), their masses are summed in one pass, and
+// the search then walks the tree taking the same decisions, stopping rules included.  Each mass is
+// the same per-thread sum and the same block reduction as a one-threshold pass, so every decision
+// is the one the one-midpoint-per-pass loop with this reduction would take.
+__device__ __forceinline__ float mid_of(float lo, float hi) {
+  return __fadd_rn(lo, __fmul_rn(__fsub_rn(hi, lo), 0.5f));
+}
+
+__device__ void phase_prune_head(const FusedArgs& a, int gi, int hl, int G, int bh, int nc, int C,
+                                 Smem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* red = reinterpret_cast<float*>(sm.scratch);                  // [kWarps][8]
+  float* ctl = reinterpret_cast<float*>(sm.scratch + 4 * kWarps * 8);   // thresholds + state
+  float* wbuf = reinterpret_cast<float*>(sm.scratch + 1024);
+  const bool staged = 1024 + 4 * nc <= sm.scratch_bytes;
+  // the group-wide max of this head's logits: merge the C partial maxima (loads in flight together)
+  float pmv[16];
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr)
+    pmv[rr] = rr < C ? ldcg_f(a.part_ms + ((size_t)gi * C * G + rr * G + hl) * 2) : -INFINITY;
+  float M = -INFINITY;
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr) M = fmaxf(M, pmv[rr]);
+  const bool empty = !(M > -INFINITY);
+  stamp(a, 17);
+  float* lrow = a.logits + (size_t)bh * a.cand_stride;
+  float* E = staged ? wbuf : lrow;
+  // pass 1: e = exp(l - M) and its block sum
+  float esum = 0.f;
+  constexpr int kB = 8;
+#pragma unroll 1
+  for (int base = 0; base < nc; base += kThreads * kB) {
+    float v[kB];
+#pragma unroll
+    for (int k = 0; k < kB; ++k) {
+      const int i = base + k * kThreads + tid;
+      v[k] = i < nc ? ldcg_f(lrow + i) : -INFINITY;
+    }
+#pragma unroll
+    for (int k = 0; k < kB; ++k) {
+      const int i = base + k * kThreads + tid;
+      if (i < nc) {
+        const float e = empty ? 0.f : __expf(v[k] - M);
+        E[i] = e;
+        esum += e;
+      }
+    }
+  }
+  const float S = block_sum_fixed(esum, red);
+  const float inv = S > 0.f ? 1.f / S : 0.f;
+  // pass 2: W = e / S (in place), the output copy, the largest weight
+  float* wout = a.weights_out ? a.weights_out + (size_t)bh * a.cand_stride : nullptr;
+  float top = 0.f;
+#pragma unroll 1
+  for (int i = tid; i < nc; i += kThreads) {
+    const float wv = (staged ? E[i] : ldcg_f(E + i)) * inv;
+    E[i] = wv;
+    if (wout) wout[i] = wv;
+    top = fmaxf(top, wv);
+  }
+  const float* W = E;
+  stamp(a, 18);
+  top = warp_max(top);
+  __syncthreads();
+  if (lane == 0) red[warp] = top;
+  __syncthreads();
+  {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) t = fmaxf(t, red[w]);
+    top = t;
+  }
+  const float p = a.p, eps = a.eps;
+  stamp(a, 19);
+  // Decisions at thresholds t <= L = (1 - p) / (2 nc) need no mass: the weights below t sum to
+  // less than nc * t <= (1 - p) / 2, so mass(W >= t) > 1 - (1 - p) / 2 >= p (with margin for fp32
+  // sums, hence the 1e-3 guard).  Above L only weights >= L can count, so the search runs on the
+  // live set {W >= L}; when it is small one warp finishes the bisection from registers.
+  constexpr int kLivePerLane = 8;
+  const bool use_bound = nc > 0 && p < 1.f && (1.f - p) >= 1e-3f;
+  const float L = use_bound ? (1.f - p) / (2.f * (float)nc) : 0.f;
+  float* live = wbuf + (staged ? nc : 0);  // after the staged weights
+  const bool live_fits = staged && 1024 + 4 * nc + 4 * 32 * kLivePerLane <= sm.scratch_bytes;
+  int nlive = 0x7FFFFFFF;
+  if (use_bound && live_fits) {
+    int cntl = 0;
+    for (int i = tid; i < nc; i += kThreads) cntl += W[i] >= L;
+    int* scan_sh2 = reinterpret_cast<int*>(red);  // 33 ints over the reduction area
+    int total_live;
+    int pos = block_exclusive_scan(cntl, scan_sh2, &total_live);
+    nlive = total_live;
+    if (nlive <= 32 * kLivePerLane) {
+      for (int i = tid; i < nc; i += kThreads)
+        if (W[i] >= L) live[pos++] = W[i];
+    }
+    __syncthreads();
+  }
+  int rounds = 0;
+  if (nlive <= 32 * kLivePerLane) {
+    if (warp == 0) {
+      float v[kLivePerLane];
+#pragma unroll
+      for (int k = 0; k < kLivePerLane; ++k) {
+        const int i = k * 32 + lane;
+        v[k] = i < nlive ? live[i] : -1.f;
+      }
+      float mres;
+      // mass over the live set (warp-uniform: xor butterflies give every lane the same bits)
+      auto wmass = [&](float t) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < kLivePerLane; ++k) acc += v[k] >= t ? v[k] : 0.f;
+        return warp_sum(acc);
+      };
+      if (wmass(top) >= p) {
+        mres = top;
+      } else {
+        float lo = 0.f, hi = top;
+        int steps = 0;
+        bool done = false;
+#pragma unroll 1
+        while (!done) {
+          // three bisection levels per round: masses of the 7 candidate midpoints at once
+          float nlo[8], nhi[8], nmid[8];
+          nlo[1] = lo;
+          nhi[1] = hi;
+          nmid[1] = mid_of(lo, hi);
+#pragma unroll
+          for (int n = 2; n < 8; ++n) {
+            const int par = n >> 1;
+            nlo[n] = (n & 1) ? nmid[par] : nlo[par];
+            nhi[n] = (n & 1) ? nhi[par] : nmid[par];
+            nmid[n] = mid_of(nlo[n], nhi[n]);
+          }
+          float acc[8];
+#pragma unroll
+          for (int n = 1; n < 8; ++n) {
+            float s8 = 0.f;
+#pragma unroll
+            for (int k = 0; k < kLivePerLane; ++k) s8 += v[k] >= nmid[n] ? v[k] : 0.f;
+            acc[n] = s8;
+          }
+#pragma unroll
+          for (int n = 1; n < 8; ++n) acc[n] = warp_sum(acc[n]);
+          int node = 1;
+#pragma unroll
+          for (int level = 0; level < 3; ++level) {
+            if (done) break;
+            if (__fsub_rn(hi, lo) <= eps) {
+              done = true;
+              break;
+            }
+            float mid = nmid[1], mass = acc[1];
+#pragma unroll
+            for (int n = 2; n < 8; ++n)
+              if (node == n) {
+                mid = nmid[n];
+                mass = acc[n];
+              }
+            if (!(lo < mid && mid < hi) || steps >= 64) {
+              done = true;
+              break;
+            }
+            const bool ge = mid <= L || mass >= p;
+            if (ge) {
+              lo = mid;
+              node = 2 * node + 1;
+            } else {
+              hi = mid;
+              node = 2 * node;
+            }
+            ++steps;
+          }
+        }
+        mres = lo;
+      }
+      if (lane == 0) ctl[11] = mres;
+    }
+    __syncthreads();
+  } else {
+  // ctl[0..6] thresholds, ctl[8] lo, ctl[9] hi, ctl[10] done (as float), ctl[11] m,
+  // ctl[12] bisection steps taken
+  if (tid == 0) {
+    ctl[10] = (nc == 0 || p >= 1.f) ? 2.f : 0.f;  // 2 = finished with m = 0
+    ctl[0] = top;
+    for (int k = 1; k < 7; ++k) ctl[k] = INFINITY;
+    ctl[8] = 0.f;
+    ctl[9] = top;
+    ctl[11] = 0.f;
+    ctl[12] = 0.f;
+  }
+  __syncthreads();
+  bool first = true;
+#pragma unroll 1
+  while (ctl[10] == 0.f) {
+    float th[7];
+#pragma unroll
+    for (int k = 0; k < 7; ++k) th[k] = ctl[k];
+    float tmin = th[0];
+#pragma unroll
+    for (int k = 1; k < 7; ++k) tmin = fminf(tmin, th[k]);
+    float acc[7];
+#pragma unroll
+    for (int k = 0; k < 7; ++k) acc[k] = 0.f;
+#pragma unroll 1
+    for (int i = tid; i < nc; i += kThreads) {
+      const float x = staged ? W[i] : ldcg_f(W + i);
+      if (x >= tmin) {  // below every threshold of this round: contributes to no mass
+#pragma unroll
+        for (int k = 0; k < 7; ++k) acc[k] += x >= th[k] ? x : 0.f;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 7; ++k) acc[k] = warp_sum(acc[k]);
+    if (lane == 0) {
+#pragma unroll
+      for (int k = 0; k < 7; ++k) red[warp * 8 + k] = acc[k];
+    }
+    __syncthreads();
+    if (warp == 0) {
+      float t = 0.f;
+      if (lane < 7) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) t += red[w * 8 + lane];
+      }
+      float ms[7];
+#pragma unroll
+      for (int k = 0; k < 7; ++k) ms[k] = __shfl_sync(0xffffffffu, t, k);
+      if (lane == 0) {
+        float lo = ctl[8], hi = ctl[9];
+        int steps = (int)ctl[12];
+        int done = 0;
+        if (first) {
+          // the single-threshold test at max W
+          if (ms[0] >= p) {
+            ctl[11] = top;
+            done = 1;
+          }
+        } else {
+          // walk the 3-level tree rooted at (lo, hi); node n's midpoint is th[n - 1]
+          int node = 1;
+#pragma unroll
+          for (int level = 0; level < 3; ++level) {
+            if (done) break;
+            if (__fsub_rn(hi, lo) <= eps) {
+              done = 1;
+              break;
+            }
+            float mid = th[0], mass = ms[0];
+#pragma unroll
+            for (int n = 2; n < 8; ++n)
+              if (node == n) {
+                mid = th[n - 1];
+                mass = ms[n - 1];
+              }
+            if (!(lo < mid && mid < hi) || steps >= 64) {
+              done = 1;
+              break;
+            }
+            if (mass >= p) {
+              lo = mid;
+              node = 2 * node + 1;
+            } else {
+              hi = mid;
+              node = 2 * node;
+            }
+            ++steps;
+          }
+          if (done) ctl[11] = lo;
+        }
+        if (!done) {
+          // next round: the tree of midpoints below (lo, hi), computed as the search would
+          float nlo[8], nhi[8], nmid[8];
+          nlo[1] = lo;
+          nhi[1] = hi;
+          nmid[1] = mid_of(lo, hi);
+#pragma unroll
+          for (int n = 2; n < 8; ++n) {
+            const int par = n >> 1;
+            nlo[n] = (n & 1) ? nmid[par] : nlo[par];
+            nhi[n] = (n & 1) ? nhi[par] : nmid[par];
+            nmid[n] = mid_of(nlo[n], nhi[n]);
+          }
+#pragma unroll
+          for (int n = 1; n < 8; ++n) ctl[n - 1] = nmid[n];
+        }
+        ctl[8] = lo;
+        ctl[9] = hi;
+        ctl[10] = done ? 1.f : 0.f;
+        ctl[12] = (float)steps;
+      }
+    }
+    first = false;
+    ++rounds;
+    __syncthreads();
+  }
+  }
+  const float m = ctl[11];
+  stamp(a, 21);
+#ifdef TWL_PHASE_TIMING
+  if (blockIdx.x == 0 && threadIdx.x == 0 && a.flags) a.flags[2] = rounds;
+#endif
+  (void)rounds;
+  // kept bits over candidate slots
+  uint32_t* kb = a.keptbits + (size_t)bh * a.kept_words;
+  int cnt = 0;
+  const int nword = (nc + 31) >> 5;
+#pragma unroll 1
+  for (int base = 0; base < nword * 32; base += kThreads) {
+    const int i = base + tid;
+    bool keep = false;
+    if (i < nc) {
+      const float x = staged ? W[i] : ldcg_f(W + i);
+      keep = x >= m;
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0 && (i >> 5) < nword) kb[i >> 5] = bal;
+    cnt += keep;
+  }
+  const float total = block_sum_fixed((float)cnt, red);
+  stamp(a, 22);
+  if (tid == 0) {
+    if (a.threshold) a.threshold[bh] = m;
+    if (a.kept_count) a.kept_count[bh] = (int)total;
+    if (a.cand_count) a.cand_count[bh] = nc;
+  }
+}
+
+// ------------------------------------------------------------------------- phase 6: kept union
+// Per page of this CTA's union share: 16-bit mask of rows kept by any head of the group.
+template <int G>
+__device__ int phase_kept_rows(const FusedArgs& a, int b, int kvh, int n, int U, int r, int C,
+                               Smem& sm, uint16_t* rowmask, int* scan_sh) {
+  const int tid = threadIdx.x, nw = sm.nw;
+  const int u0 = (int)((long)U * r / C), u1 = (int)((long)U * (r + 1) / C);
+  int cnt = 0;
+  for (int u = u0 + tid; u < u1; u += kThreads) {
+    const int j = union_select(sm.ubits, sm.upre, nw, u);
+    uint32_t words[G];
+    int shift[G];
+#pragma unroll
+    for (int hl = 0; hl < G; ++hl) {  // issue every head's load before combining
+      const uint32_t* hb = sm.hbits + hl * nw;
+      words[hl] = 0;
+      shift[hl] = 0;
+      if ((hb[j >> 5] >> (j & 31)) & 1u) {
+        const int slot = kPage * rank_in(hb, sm.hpre + hl * nw, j);
+        shift[hl] = slot & 31;
+        words[hl] = ldcg_u(a.keptbits + (size_t)(b * a.hq + kvh * G + hl) * a.kept_words +
+                           (slot >> 5));
+      }
+    }
+    uint32_t m = 0;
+#pragma unroll
+    for (int hl = 0; hl < G; ++hl) m |= (words[hl] >> shift[hl]) & 0xFFFFu;
+    const int rows = page_rows(n, j);
+    m &= rows >= 16 ? 0xFFFFu : ((1u << rows) - 1u);
+    rowmask[u - u0] = (uint16_t)m;
+    cnt += __popc(m);
+  }
+  int total;
+  block_exclusive_scan(cnt, scan_sh, &total);
+  return total;
+}
+
+template <int G>
+__device__ void phase_write_union(const FusedArgs& a, int gi, int U, int r, int C, int base,
+                                  Smem& sm, const uint16_t* rowmask, int* scan_sh) {
+  const int tid = threadIdx.x, nw = sm.nw;
+  const int u0 = (int)((long)U * r / C), u1 = (int)((long)U * (r + 1) / C);
+  int* out = a.union_tok + (size_t)gi * a.union_stride;
+  // pages are handled in rounds of kThreads; thread order = page order
+  int carry = base;
+  for (int ub = u0; ub < u1; ub += kThreads) {
+    const int u = ub + tid;
+    const uint32_t m = u < u1 ? rowmask[u - u0] : 0u;
+    int total;
+    int pos = carry + block_exclusive_scan(__popc(m), scan_sh, &total);
+    carry += total;
+    if (m) {
+      const int j = union_select(sm.ubits, sm.upre, nw, u);
+      uint32_t mm = m;
+      while (mm) {
+        out[pos++] = kPage * j + __ffs(mm) - 1;
+        mm &= mm - 1u;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------- phase 7: attention
+// Thread layout: token slot t = tid / 8 (64 per round), sub-lane s = tid % 8 owns channels
+// [8s, 8s+8) and [64+8s, 64+8s+8).  For P.V: channel d = tid % 128, token quarter = tid / 128.
+template <int G>
+__device__ void phase_attend(const FusedArgs& a, int b, int kvh, int gi, int n, int T, int r, int C,
+                             Smem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ts = tid >> 3, s8 = tid & 7;
+  const int d = tid & 127, quarter = tid >> 7;
+  unsigned char* sp = sm.scratch;
+  uint4* ks = reinterpret_cast<uint4*>(sp);                       // [64][16]
+  uint4* vs = reinterpret_cast<uint4*>(sp + 16384);               // [64][16]
+  float* ps = reinterpret_cast<float*>(sp + 32768);               // [G][64]
+  float* red = reinterpret_cast<float*>(sp + 32768 + G * 256);    // [kWarps][G]
+  uint32_t* rowidx = reinterpret_cast<uint32_t*>(sp + 32768 + G * 256 + kWarps * G * 4);  // 64
+  float* opart = reinterpret_cast<float*>(sp + 32768 + G * 256 + kWarps * G * 4 + 256);  // [4][G][128]
+  const int t0 = (int)((long)T * r / C), t1 = (int)((long)T * (r + 1) / C);
+  const int* ulist = a.union_tok + (size_t)gi * a.union_stride;
+
+  float qv[G][16];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const uint16_t* qh = a.q + ((size_t)b * a.hq + kvh * G + h) * kHeadDim;
+    float f[8];
+    unpack8(*reinterpret_cast<const uint4*>(qh + 8 * s8), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qv[h][i] = f[i];
+    unpack8(*reinterpret_cast<const uint4*>(qh + 64 + 8 * s8), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qv[h][8 + i] = f[i];
+  }
+  float M[G], L[G], O[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    M[h] = -INFINITY;
+    L[h] = 0.f;
+    O[h] = 0.f;
+  }
+  for (int cb = t0; cb < t1; cb += kAttChunk) {
+    const int nt = min(kAttChunk, t1 - cb);
+    if (tid < kAttChunk) {
+      uint32_t ri = 0xFFFFFFFFu;
+      if (tid < nt) {
+        const int tk = ldcg_i(ulist + cb + tid);
+        if (tk >= 0 && tk < n) {
+          const int ph = load_phys(a.kv.page_table, b, tk >> 4, a.kv.max_pages, a.kv.num_phys,
+                                   a.flags);
+          if (ph >= 0) ri = (uint32_t)(((size_t)ph * a.kv.hkv + kvh) * kPage + (tk & 15));
+        } else {
+          raise_flag(a.flags, TWL_FLAG_BAD_INDEX);
+        }
+      }
+      rowidx[tid] = ri;
+    }
+    __syncthreads();
+    // gather 64 rows of K and V: 2048 16-byte chunks, 4 per thread
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int c = tid + it * kThreads;  // 0 .. 1023
+      const int tt = c >> 4, ch = c & 15;
+      const uint32_t ri = rowidx[tt];
+      const bool ok = ri != 0xFFFFFFFFu;
+      const size_t off = ok ? (size_t)ri * kHeadDim + 8 * ch : 0;
+      cp_async16(&ks[tt * 16 + ch], a.kv.k + off, ok);
+      cp_async16(&vs[tt * 16 + ch], a.kv.v + off, ok);
+    }
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncthreads();
+    // scores
+    const bool tok_ok = ts < nt && rowidx[ts] != 0xFFFFFFFFu;
+    float sc[G];
+    {
+      float k0[8], k1[8];
+      unpack8(ks[ts * 16 + s8], k0);
+      unpack8(ks[ts * 16 + 8 + s8], k1);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc = fmaf(qv[h][i], k0[i], acc);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc = fmaf(qv[h][8 + i], k1[i], acc);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        sc[h] = tok_ok ? acc * a.sm_scale : -INFINITY;
+      }
+    }
+    // chunk max per head
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float m = sc[h];
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+      if (lane == 0) red[warp * G + h] = m;
+    }
+    __syncthreads();
+    float scale[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float cm = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) cm = fmaxf(cm, red[w * G + h]);
+      const float nm = fmaxf(M[h], cm);
+      scale[h] = (nm > -INFINITY && M[h] > -INFINITY) ? __expf(M[h] - nm) : (nm > -INFINITY ? 0.f : 1.f);
+      M[h] = nm;
+      const float pv = (tok_ok && nm > -INFINITY) ? __expf(sc[h] - nm) : 0.f;
+      if (s8 == 0) ps[h * kAttChunk + ts] = pv;
+    }
+    __syncthreads();
+    // P.V for channel d over tokens quarter, quarter+4, ...
+    const __half* vh = reinterpret_cast<const __half*>(vs);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float acc = 0.f, lsum = 0.f;
+      for (int tt = quarter; tt < nt; tt += 4) {
+        const float pv = ps[h * kAttChunk + tt];
+        acc = fmaf(pv, __half2float(vh[tt * kHeadDim + d]), acc);
+        lsum += pv;
+      }
+      O[h] = O[h] * scale[h] + acc;
+      L[h] = L[h] * scale[h] + lsum;
+    }
+    __syncthreads();
+  }
+  // combine the 4 quarters, write this CTA's partial: M, L, O (unnormalised)
+#pragma unroll
+  for (int h = 0; h < G; ++h) opart[(quarter * G + h) * kHeadDim + d] = O[h];
+  float* lpart = reinterpret_cast<float*>(ps);  // reuse: [4][G]
+  if (d == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) lpart[quarter * G + h] = L[h];
+  }
+  __syncthreads();
+  float* part = a.part_att + ((size_t)gi * C + r) * G * (kHeadDim + 2);
+  if (quarter == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float o = opart[(0 * G + h) * kHeadDim + d] + opart[(1 * G + h) * kHeadDim + d] +
+                      opart[(2 * G + h) * kHeadDim + d] + opart[(3 * G + h) * kHeadDim + d];
+      part[h * (kHeadDim + 2) + 2 + d] = o;
+      if (d == 0) {
+        part[h * (kHeadDim + 2) + 0] = M[h];
+        part[h * (kHeadDim + 2) + 1] =
+            lpart[0 * G + h] + lpart[1 * G + h] + lpart[2 * G + h] + lpart[3 * G + h];
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------- phase 8: merge
+__device__ void phase_merge_head(const FusedArgs& a, int gi, int bh, int hl, int G, int C) {
+  const int tid = threadIdx.x;
+  if (tid >= kHeadDim) return;
+  float pm[16], pl[16], po[16];
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr) {  // every partial's loads in flight together
+    pm[rr] = -INFINITY;
+    pl[rr] = 0.f;
+    po[rr] = 0.f;
+    if (rr < C) {
+      const float* part =
+          a.part_att + ((size_t)gi * C + rr) * G * (kHeadDim + 2) + hl * (kHeadDim + 2);
+      pm[rr] = ldcg_f(part);
+      pl[rr] = ldcg_f(part + 1);
+      po[rr] = ldcg_f(part + 2 + tid);
+    }
+  }
+  float Mx = -INFINITY;
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr)
+    if (pl[rr] > 0.f) Mx = fmaxf(Mx, pm[rr]);
+  float o = 0.f, l = 0.f;
+  if (Mx > -INFINITY) {
+#pragma unroll
+    for (int rr = 0; rr < 16; ++rr) {
+      if (!(pl[rr] > 0.f)) continue;
+      const float wgt = __expf(pm[rr] - Mx);
+      o = fmaf(wgt, po[rr], o);
+      l = fmaf(wgt, pl[rr], l);
+    }
+  }
+  const bool any = l > 0.f;
+  a.o[(size_t)bh * kHeadDim + tid] = any ? o / l : 0.f;
+  if (tid == 0) a.lse[bh] = any ? Mx + __logf(l) : -INFINITY;
+}
+
+// ------------------------------------------------------------------------- the kernel
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ int scan_sh[33];
+  __shared__ int s_total;
+  const int C = (int)cluster_size();
+  const int r = (int)cluster_rank();
+  const int gi = blockIdx.x / C;
+  const int b = gi / a.kv.hkv, kvh = gi % a.kv.hkv;
+  const int tid = threadIdx.x;
+
+  const Seq sq = load_seq(a.kv.seq_lens, b, a.kv.max_pages, a.flags, r == 0 && tid == 0);
+  const int n_pages = sq.pages;
+  if (n_pages == 0) {  // invalid sequence: uniform across the cluster, before any barrier
+    if (r == 0) {
+      for (int i = tid; i < G * kHeadDim; i += kThreads)
+        a.o[((size_t)b * a.hq + kvh * G) * kHeadDim + i] = 0.f;
+      if (tid < G) {
+        a.lse[(size_t)b * a.hq + kvh * G + tid] = -INFINITY;
+        if (a.sel_count) a.sel_count[b * a.hq + kvh * G + tid] = 0;
+        if (a.cand_count) a.cand_count[b * a.hq + kvh * G + tid] = 0;
+        if (a.kept_count) a.kept_count[b * a.hq + kvh * G + tid] = 0;
+      }
+      if (tid == 0 && a.union_count) a.union_count[gi] = 0;
+    }
+    return;
+  }
+  int kb = a.budget_pages > 0 ? a.budget_pages : (n_pages + a.budget_div - 1) / a.budget_div;
+  kb = min(min(kb, n_pages), a.max_budget);
+
+  Smem sm;
+  sm.nw = (n_pages + 31) >> 5;
+  {
+    unsigned char* p = smem_raw;
+    sm.hbits = reinterpret_cast<uint32_t*>(p);
+    p += 4 * G * a.sel_words;
+    sm.hpre = reinterpret_cast<int*>(p);
+    p += 4 * G * a.sel_words;
+    sm.ubits = reinterpret_cast<uint32_t*>(p);
+    p += 4 * a.sel_words;
+    sm.upre = reinterpret_cast<int*>(p);
+    p = smem_raw + persistent_bytes(G, a.sel_words);  // scratch starts 128-byte aligned
+    sm.scratch = p;
+    sm.scratch_bytes = a.smem_bytes - (int)(p - smem_raw);
+  }
+
+  // 1: scores
+  stamp(a, 0);
+  phase_scores<G>(a, b, kvh, n_pages, r, C, sm);
+  stamp(a, 1);
+  cluster_sync();
+  stamp(a, 2);
+  // 2: top-k of the heads this CTA owns
+  for (int hl = r; hl < G; hl += C) phase_topk_head(a, b * a.hq + kvh * G + hl, n_pages, kb, sm);
+  stamp(a, 3);
+  cluster_sync();
+  stamp(a, 4);
+  // 3: bitmaps, union, ranks (every CTA)
+  phase_union_bitmaps<G>(a, b, kvh, sm, &s_total, scan_sh);
+  const int U = s_total;
+  stamp(a, 5);
+  // 4: INT4 estimate over this CTA's share of the union
+  phase_estimate<G>(a, b, kvh, gi, sq.n, U, r, C, sm);
+  stamp(a, 6);
+  cluster_sync();
+  stamp(a, 7);
+  // 5: top-p of the heads this CTA owns
+  {
+    int nc = 0;
+    if (kb > 0) {
+      // the last selected page is the highest set bit of the head bitmap
+      for (int hl = r; hl < G; hl += C) {
+        const uint32_t* hb = sm.hbits + hl * sm.nw;
+        int jl = -1;
+        for (int w = sm.nw - 1; w >= 0; --w)
+          if (hb[w]) {
+            jl = 32 * w + 31 - __clz(hb[w]);
+            break;
+          }
+        nc = jl >= 0 ? kPage * (kb - 1) + page_rows(sq.n, jl) : 0;
+        phase_prune_head(a, gi, hl, G, b * a.hq + kvh * G + hl, nc, C, sm);
+        __syncthreads();
+      }
+    }
+  }
+  stamp(a, 8);
+  cluster_sync();
+  stamp(a, 9);
+  // 6: kept rows of this CTA's union pages, counts exchanged, ascending union list written
+  uint16_t* rowmask = reinterpret_cast<uint16_t*>(sm.scratch);
+  const int local = phase_kept_rows<G>(a, b, kvh, sq.n, U, r, C, sm, rowmask, scan_sh);
+  if (tid == 0) a.union_part[(size_t)gi * C + r] = local;
+  stamp(a, 10);
+  cluster_sync();
+  stamp(a, 11);
+  int base = 0, T = 0;
+  for (int rr = 0; rr < C; ++rr) {
+    const int c = ldcg_i(a.union_part + (size_t)gi * C + rr);
+    if (rr < r) base += c;
+    T += c;
+  }
+  phase_write_union<G>(a, gi, U, r, C, base, sm, rowmask, scan_sh);
+  if (r == 0 && tid == 0 && a.union_count) a.union_count[gi] = T;
+  stamp(a, 12);
+  cluster_sync();
+  stamp(a, 13);
+  // 7: attention over this CTA's even share of the group's kept tokens
+  phase_attend<G>(a, b, kvh, gi, sq.n, T, r, C, sm);
+  stamp(a, 14);
+  cluster_sync();
+  stamp(a, 15);
+  // 8: merge per head
+  for (int hl = r; hl < G; hl += C) phase_merge_head(a, gi, b * a.hq + kvh * G + hl, hl, G, C);
+  stamp(a, 16);
+}
+
+template <int G>
+size_t attend_smem_bytes() {
+  return 32768 + G * 256 + kWarps * G * 4 + 256 + 4 * G * kHeadDim * 4;
+}
+
+}  // namespace
+
+FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) {
+  FusedPlan pl{};
+  const int g = hq / hkv;
+  const int groups = batch * hkv;
+  pl.sel_words = (max_pages + 31) / 32;
+  pl.cand_stride = kPage * max_budget;
+  pl.kept_words = (pl.cand_stride + 31) / 32;
+  pl.union_stride = kPage * max_pages;
+  // cluster size: enough CTAs to fill the GPU, at most 16
+  const int sms = num_sms();
+  int c = 1;
+  while (c < 16 && groups * c * 2 <= sms) c *= 2;
+  // TWL_FUSED_CLUSTER=1|2|4|8|16 forces the cluster size (used by the tests to cover every size)
+  if (const char* env = getenv("TWL_FUSED_CLUSTER")) {
+    const int f = atoi(env);
+    if (f == 1 || f == 2 || f == 4 || f == 8 || f == 16) c = f;
+  }
+  pl.cluster = c;
+  const size_t persistent = (size_t)persistent_bytes(g, pl.sel_words);
+  size_t scratch = 0;
+  switch (g) {
+    case 1: scratch = attend_smem_bytes<1>(); break;
+    case 2: scratch = attend_smem_bytes<2>(); break;
+    case 4: scratch = attend_smem_bytes<4>(); break;
+    default: scratch = attend_smem_bytes<8>(); break;
+  }
+  // top-k keys and staged weights when they fit in what is left
+  const size_t cap = 220 * 1024;
+  size_t want = scratch;
+  const size_t topk_need = 1280 + (size_t)4 * max_pages + 4 * kWarps * 512 + 2048;
+  want = want > topk_need ? want : topk_need;
+  want = want > 256 + (size_t)4 * pl.cand_stride ? want : 256 + (size_t)4 * pl.cand_stride;
+  want = want > (size_t)2 * pl.union_stride / 16 + 16 ? want : (size_t)2 * pl.union_stride / 16 + 16;
+  if (persistent + want > cap) want = cap - persistent;
+  pl.smem_bytes = (int)(persistent + want);
+  pl.ok = persistent + scratch <= cap && persistent + (size_t)2 * max_pages <= cap;
+  return pl;
+}
+
+size_t fused_workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_budget) {
+  const FusedPlan pl = plan_fused(batch, hq, hkv, max_pages, max_budget);
+  const int g = hq / hkv;
+  const size_t bh = (size_t)batch * hq, groups = (size_t)batch * hkv;
+  // cluster-dependent parts are sized for the largest cluster (16)
+  size_t s = 0;
+  auto add = [&](size_t bytes) { s += (bytes + 255) & ~(size_t)255; };
+  add(bh * max_pages * 4);                    // scores
+  add(bh * pl.sel_words * 4);                 // selected-page bitmaps
+  add(bh * (size_t)pl.cand_stride * 4);       // logits / weights
+  add(bh * (size_t)pl.kept_words * 4);        // kept bits
+  add(groups * 16 * g * 2 * 4);               // partial (max, sum)
+  add(groups * 16 * 4);                       // union counts per CTA
+  add(groups * (size_t)pl.union_stride * 4);  // union token lists
+  add(groups * 16 * g * (kHeadDim + 2) * 4);  // attention partials
+  return s;
+}
+
+void carve_fused(FusedArgs& a, char* ws, const FusedPlan& pl, int batch, int hq, int hkv,
+                 int max_pages) {
+  const int g = hq / hkv;
+  const size_t bh = (size_t)batch * hq, groups = (size_t)batch * hkv;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = ws + off;
+    off += (bytes + 255) & ~(size_t)255;
+    return p;
+  };
+  a.scores = reinterpret_cast<float*>(take(bh * max_pages * 4));
+  a.selbits = reinterpret_cast<uint32_t*>(take(bh * pl.sel_words * 4));
+  a.logits = reinterpret_cast<float*>(take(bh * (size_t)pl.cand_stride * 4));
+  a.keptbits = reinterpret_cast<uint32_t*>(take(bh * (size_t)pl.kept_words * 4));
+  a.part_ms = reinterpret_cast<float*>(take(groups * 16 * g * 2 * 4));
+  a.union_part = reinterpret_cast<int*>(take(groups * 16 * 4));
+  int* ulist = reinterpret_cast<int*>(take(groups * (size_t)pl.union_stride * 4));
+  if (!a.union_tok) a.union_tok = ulist;
+  a.part_att = reinterpret_cast<float*>(take(groups * 16 * g * (kHeadDim + 2) * 4));
+}
+
+cudaError_t launch_fused(const FusedArgs& a, const FusedPlan& pl, cudaStream_t s) {
+  const int g = a.hq / a.kv.hkv;
+  const int groups = a.kv.batch * a.kv.hkv;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(groups * pl.cluster));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)pl.smem_bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)pl.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+#define TWL_FUSED(G)                                                                            \
+  do {                                                                                          \
+    cudaError_t e = cudaFuncSetAttribute(k_decode_fused<G>,                                     \
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,           \
+                                         pl.smem_bytes);                                        \
+    if (e != cudaSuccess) return e;                                                             \
+    if (pl.cluster > 8) {                                                                       \
+      e = cudaFuncSetAttribute(k_decode_fused<G>,                                               \
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);              \
+      if (e != cudaSuccess) return e;                                                           \
+    }                                                                                           \
+    e = cudaLaunchKernelEx(&cfg, k_decode_fused<G>, a);                                         \
+    if (e != cudaSuccess) return e;                                                             \
+  } while (0)
+  switch (g) {
+    case 1: TWL_FUSED(1); break;
+    case 2: TWL_FUSED(2); break;
+    case 4: TWL_FUSED(4); break;
+    case 8: TWL_FUSED(8); break;
+    default: return cudaErrorInvalidValue;
+  }
+#undef TWL_FUSED
+  return cudaGetLastError();
+}
+
+// Active clusters of size c the device can hold at once for this kernel (0 if none / error).
+static int active_clusters(int g, int c, int smem_bytes) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)c);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)smem_bytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)c;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  cudaError_t e = cudaErrorInvalidValue;
+#define TWL_FIT(G)                                                                              \
+  do {                                                                                          \
+    cudaFuncSetAttribute(k_decode_fused<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,        \
+                         smem_bytes);                                                           \
+    if (c > 8)                                                                                  \
+      cudaFuncSetAttribute(k_decode_fused<G>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1); \
+    e = cudaOccupancyMaxActiveClusters(&n, k_decode_fused<G>, &cfg);                            \
+  } while (0)
+  switch (g) {
+    case 1: TWL_FIT(1); break;
+    case 2: TWL_FIT(2); break;
+    case 4: TWL_FIT(4); break;
+    default: TWL_FIT(8); break;
+  }
+#undef TWL_FIT
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+// Cluster size for `groups` groups: the largest c <= want whose clusters for every group can be
+// resident at once; if none can, the c that keeps the most CTAs resident.
+int fit_cluster(int g, int want, int groups, int smem_bytes) {
+  int best = 1, best_ctas = 0;
+  for (int c = want; c >= 1; c >>= 1) {
+    const int n = c == 1 ? groups : active_clusters(g, c, smem_bytes);
+    if (n >= groups) return c;
+    if (n * c > best_ctas) {
+      best_ctas = n * c;
+      best = c;
+    }
+  }
+  return best;
+}
+
+}  // namespace twl

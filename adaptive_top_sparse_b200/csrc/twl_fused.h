@@ -1,0 +1,63 @@
+// The fused decode-step kernel (twl_fused.cu): arguments, launch plan, workspace carving.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "twl_kernels.h"
+
+namespace twl {
+
+struct FusedArgs {
+  // inputs
+  const uint16_t* q;
+  int hq;
+  KV kv;
+  const uint8_t* k_int4;
+  const uint16_t* k_sz;
+  const uint16_t* bounds;
+  int budget_pages, budget_div, max_budget;
+  float p, eps, sm_scale;
+  // outputs
+  float* o;
+  float* lse;
+  // optional outputs (NULL = not written)
+  int* sel_pages;
+  int* sel_count;
+  float* weights_out;
+  int* cand_tok;
+  int* cand_count;
+  float* threshold;
+  int* kept_count;
+  int* union_count;
+  int* union_tok;  // the workspace's list when the caller does not ask for it
+  // workspace
+  float* scores;
+  uint32_t* selbits;
+  float* logits;
+  uint32_t* keptbits;
+  float* part_ms;
+  int* union_part;
+  float* part_att;
+  uint32_t* flags;
+  // strides and launch shape
+  int sel_words, cand_stride, kept_words, union_stride;
+  int cluster;
+  int smem_bytes;
+};
+
+struct FusedPlan {
+  int cluster;
+  int smem_bytes;
+  int sel_words, cand_stride, kept_words, union_stride;
+  bool ok;
+};
+
+FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget);
+size_t fused_workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_budget);
+void carve_fused(FusedArgs& a, char* ws, const FusedPlan& pl, int batch, int hq, int hkv,
+                 int max_pages);
+int fit_cluster(int g, int want, int groups, int smem_bytes);
+cudaError_t launch_fused(const FusedArgs& a, const FusedPlan& pl, cudaStream_t s);
+
+}  // namespace twl

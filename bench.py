@@ -40,7 +40,7 @@ from workloads import synth  # noqa: E402
 METRIC = "decode attn layer-steps/s at 32K ctx (select+prune+attend); % of HBM roofline"
 UNIT = "layer-steps/s"
 LAYERS = 32  # default; --layers overrides (profiling runs use 1)
-KERNELS_PER_LAYER_STEP = 9
+KERNELS_PER_LAYER_STEP = 1  # twl_decode_step is one fused kernel
 FALLBACK_HBM_GBS = 6650.0
 
 

@@ -132,7 +132,8 @@ def test_decode_step_rejects_bad_arguments():
     assert call(kvv=_kv(v=0)) == twl.TWL_ERR_INVALID_ARG
     assert call(ws_bytes=100) == twl.TWL_ERR_WORKSPACE
     assert call(max_budget=3) == twl.TWL_ERR_INVALID_ARG
-    assert call(kvv=_kv(batch=1024)) == twl.TWL_ERR_UNSUPPORTED   # 8192 groups > 4096
+    assert call(kvv=_kv(max_pages=40000)) == twl.TWL_ERR_UNSUPPORTED   # > 512K tokens
+    assert call(kvv=_kv(head_dim=64)) == twl.TWL_ERR_UNSUPPORTED
 
 
 def test_sparse_decode_rejects_bad_arguments():

@@ -330,7 +330,9 @@ def test_decode_step_equals_staged_calls(small):
     twl.twl_sparse_decode(q, wl.num_q_heads, layer.kv, torch.from_numpy(st["union_tok"]).to(dev),
                           torch.from_numpy(st["union_count"]).to(dev), stride, SM_SCALE, o2,
                           lse2, ws)
-    assert np.allclose(np_(o2), o, atol=1e-5) and np.allclose(np_(lse2), lse, atol=1e-5)
+    # two fp32 attention kernels that differ only in chunking and summation order
+    do, dl = float(np.abs(np_(o2) - o).max()), float(np.abs(np_(lse2) - lse).max())
+    assert do <= 2e-4 and dl <= 2e-4, (do, dl)
 
 
 def test_decode_step_dense_limit():
@@ -346,6 +348,19 @@ def test_decode_step_dense_limit():
     for (bb, h), (o_or, lse_or) in ref.items():
         assert st["union_count"][0, h // 4] == 700
         check_attention(o[bb, h], lse[bb, h], o_or, lse_or, f"dense h{h}")
+
+
+@pytest.mark.parametrize("cluster", [1, 2, 4, 8, 16])
+def test_decode_step_every_cluster_size(cluster, monkeypatch):
+    monkeypatch.setenv("TWL_FUSED_CLUSTER", str(cluster))
+    wl = synth.make_decode("clusters", 2, 8, 2, [3001, 515], seed=9)
+    layer = DecodeLayer.from_workload(wl)
+    layer.build_aux()
+    st, o, lse = _run_step(wl, layer)
+    for bb in range(wl.batch):
+        for kvh in range(wl.num_kv_heads):
+            check_step_group(wl, bb, kvh, st, o, lse)
+    assert layer.status()[0] == twl.TWL_OK
 
 
 # -------------------------------------------------------------------------- full-size workloads
