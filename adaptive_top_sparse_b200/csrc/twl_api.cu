@@ -396,7 +396,6 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
   a.flags = flags_of(ws);
   a.sel_words = pl.sel_words;
   a.cand_stride = pl.cand_stride;
-  a.kept_words = pl.kept_words;
   a.union_stride = pl.union_stride;
   a.cluster = pl.cluster;
   a.smem_bytes = pl.smem_bytes;

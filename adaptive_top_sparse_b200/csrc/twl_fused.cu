@@ -302,60 +302,50 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
   mask = hi_bit >= 31 ? 0u : ~((2u << hi_bit) - 1u);
   if (hi_bit < 0) mask = 0xFFFFFFFFu;
   prefix = kmax & mask;
-  const int nbits = hi_bit + 1;
-  // per-warp histograms [kWarps][1 << dw] after the staged keys, then the bin totals
-  uint32_t* whist = reinterpret_cast<uint32_t*>(sm.scratch + 1280 + 4 * n_pages);
-  const bool whist_ok =
-      staged && 1280 + 4 * n_pages + 4 * kWarps * 512 + 2048 <= sm.scratch_bytes;
-  // digit width: three digits of up to 9 bits when the per-warp histograms fit, else 8 bits
-  // (the shared 256-bin histogram)
-  const int dw = (whist_ok && nbits <= 27) ? (nbits + 2) / 3 : 8;
-  uint32_t* tot = whist_ok ? whist + kWarps * (1 << dw) : hist;  // [1 << dw] totals
-  const int n_iter = (n_pages + kThreads - 1) / kThreads;
+  // Narrow the candidate bin with histogram passes over the next (up to) 10 bits of the keys
+  // that still match the prefix, until it holds at most kGatherCap keys; every key above the bin
+  // is selected, and the bin's keys are ranked exactly by (key desc, page asc).  Only when all
+  // bits are resolved and more than kGatherCap keys are exactly equal does the ordered ballot
+  // path below take the first ones by page index.
+  constexpr int kGatherCap = 64;
+  uint32_t* bhist = reinterpret_cast<uint32_t*>(sm.scratch + 1280 + 4 * n_pages);  // [1024]
+  uint32_t* gkey = bhist + 1024;                                                   // [cap]
+  int* gidx = reinterpret_cast<int*>(gkey + kGatherCap);                           // [cap]
+  uint32_t* sbits = reinterpret_cast<uint32_t*>(gidx + kGatherCap);                // [nw]
+  const bool room = staged && 1280 + 4 * (size_t)n_pages + 4 * 1024 + 8 * kGatherCap + 4 * nw +
+                                  16 <= (size_t)sm.scratch_bytes;
+  uint32_t* hh = room ? bhist : hist;  // the 256-bin histogram when there is no room
+  const int max_dw = room ? 10 : 8;
+  int cand = n_pages;
+  const int n_it = (n_pages + kThreads - 1) / kThreads;
 #pragma unroll 1
-  while (hi_bit >= 0) {
-    const int lo_bit = max(hi_bit - dw + 1, 0);
-    const int width = hi_bit - lo_bit + 1;
-    const int nb = 1 << width;
-    const uint32_t dmask = (uint32_t)nb - 1u;
-    if (whist_ok) {
-      for (int i = tid; i < kWarps * nb; i += kThreads) whist[i] = 0u;
-    } else {
-      for (int i = tid; i < nb; i += kThreads) tot[i] = 0u;
-    }
+  while ((cand > kGatherCap || !room) && hi_bit >= 0) {
+    const int dwb = hi_bit + 1 < max_dw ? hi_bit + 1 : max_dw;
+    const int lo_b = hi_bit - dwb + 1;
+    const int nbb = 1 << dwb;
+    const uint32_t dmb = (uint32_t)nbb - 1u;
+    for (int i = tid; i < nbb; i += kThreads) hh[i] = 0u;
     __syncthreads();
-    uint32_t* my = whist_ok ? whist + warp * nb : tot;
 #pragma unroll 1
-    for (int it = 0; it < n_iter; ++it) {
+    for (int it = 0; it < n_it; ++it) {
       const int i = it * kThreads + tid;
       bool take = false;
       uint32_t digit = 0;
       if (i < n_pages) {
         const uint32_t key = key_at(i);
         take = (key & mask) == prefix;
-        digit = (key >> lo_bit) & dmask;
+        digit = (key >> lo_b) & dmb;
       }
-      const uint32_t tag = take ? digit : 1024u + lane;
-      const uint32_t peers = __match_any_sync(0xffffffffu, tag);
-      if (take && (__ffs(peers) - 1) == lane) atomicAdd(&my[digit], (uint32_t)__popc(peers));
+      const uint32_t peers = __match_any_sync(0xffffffffu, take ? digit : 2048u + lane);
+      if (take && (__ffs(peers) - 1) == lane) atomicAdd(&hh[digit], (uint32_t)__popc(peers));
     }
     __syncthreads();
-    if (whist_ok) {
-      for (int bin = tid; bin < nb; bin += kThreads) {
-        uint32_t t = 0;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) t += whist[w * nb + bin];
-        tot[bin] = t;
-      }
-      __syncthreads();
-    }
     if (warp == 0) {
-      // lane l covers the bins nb-1-l*per .. nb-per-l*per (descending)
-      const int per = (nb + 31) / 32;
+      const int per = (nbb + 31) / 32;
       uint32_t lsum = 0;
       for (int e = 0; e < per; ++e) {
-        const int bin = nb - 1 - lane * per - e;
-        if (bin >= 0) lsum += tot[bin];
+        const int bin = nbb - 1 - lane * per - e;
+        if (bin >= 0) lsum += hh[bin];
       }
       uint32_t incl = lsum;
 #pragma unroll
@@ -367,11 +357,11 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
       if (excl < (uint32_t)remaining && incl >= (uint32_t)remaining) {
         uint32_t run = excl;
         for (int e = 0; e < per; ++e) {
-          const int bin = nb - 1 - lane * per - e;
+          const int bin = nbb - 1 - lane * per - e;
           if (bin < 0) break;
-          const uint32_t c = tot[bin];
+          const uint32_t c = hh[bin];
           if (run + c >= (uint32_t)remaining) {
-            state[0] = prefix | ((uint32_t)bin << lo_bit);
+            state[0] = (uint32_t)bin;
             state[1] = (uint32_t)remaining - run;
             state[2] = c;
             break;
@@ -381,25 +371,69 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
       }
     }
     __syncthreads();
-    prefix = state[0];
+    prefix |= state[0] << lo_b;
+    mask |= dmb << lo_b;
     remaining = (int)state[1];
-    eq_count = (int)state[2];
-    mask |= dmask << lo_bit;
-    hi_bit = lo_bit - 1;
+    cand = (int)state[2];
+    hi_bit = lo_b - 1;
     __syncthreads();
   }
-  if (eq_count == remaining && sel_list == nullptr) {
-    // every key equal to the k-th is taken: one ballot per 32-page word, no ordering needed
+  if (room && cand <= kGatherCap) {
+    for (int w = tid; w < nw; w += kThreads) sbits[w] = 0u;
+    // ordered gather of the bin's keys: thread t scans a contiguous range of pages
+    const int per = (n_pages + kThreads - 1) / kThreads;
+    const int beg = min(n_pages, tid * per), end = min(n_pages, beg + per);
+    int mine = 0;
+    for (int i = beg; i < end; ++i) mine += (key_at(i) & mask) == prefix;
+    int slot = block_exclusive_scan(mine, scan_sh, nullptr);
+    for (int i = beg; i < end && mine > 0; ++i) {
+      const uint32_t key = key_at(i);
+      if ((key & mask) == prefix) {
+        gkey[slot] = key;
+        gidx[slot] = i;
+        ++slot;
+        --mine;
+      }
+    }
+    __syncthreads();
+    for (int e = tid; e < cand; e += kThreads) {
+      const uint32_t ke = gkey[e];
+      const int ie = gidx[e];
+      int rank = 0;
+      for (int f = 0; f < cand; ++f) {
+        const uint32_t kf = gkey[f];
+        rank += (kf > ke || (kf == ke && gidx[f] < ie)) ? 1 : 0;
+      }
+      if (rank < remaining) atomicOr(&sbits[ie >> 5], 1u << (ie & 31));
+    }
+    __syncthreads();
     for (int base = 0; base < 32 * nw; base += kThreads) {
       const int i = base + tid;
-      const bool in = i < n_pages;
-      const uint32_t key = in ? key_at(i) : 0u;
-      const uint32_t sel = __ballot_sync(0xffffffffu, in && key >= prefix);
-      if (lane == 0 && (i >> 5) < nw) out_bits[i >> 5] = sel;
+      const bool above = i < n_pages && (key_at(i) & mask) > prefix;
+      const uint32_t bal = __ballot_sync(0xffffffffu, above);
+      if (lane == 0 && (i >> 5) < nw) sbits[i >> 5] |= bal;
+    }
+    __syncthreads();
+    int carry = 0;
+    for (int base = 0; base < nw; base += kThreads) {
+      const int w = base + tid;
+      const uint32_t word = w < nw ? sbits[w] : 0u;
+      if (w < nw) out_bits[w] = word;
+      if (sel_list) {
+        int total;
+        int pos = carry + block_exclusive_scan(__popc(word), scan_sh, &total);
+        carry += total;
+        uint32_t x = word;
+        while (x) {
+          sel_list[pos++] = 32 * w + __ffs(x) - 1;
+          x &= x - 1u;
+        }
+      }
     }
     if (tid == 0 && a.sel_count) a.sel_count[bh] = kb;
     return;
   }
+  // all bits resolved (or no room for the gather): prefix is the k-th key itself
   stamp(a, 24);
   // Keys above the k-th are taken; equal keys are taken in ascending page order.  One element
   // per thread per round; a warp's ballot is one 32-page word of the bitmap.
@@ -953,29 +987,23 @@ __device__ void phase_prune_head(const FusedArgs& a, int gi, int hl, int G, int 
   if (blockIdx.x == 0 && threadIdx.x == 0 && a.flags) a.flags[2] = rounds;
 #endif
   (void)rounds;
-  // kept bits over candidate slots
-  uint32_t* kb = a.keptbits + (size_t)bh * a.kept_words;
-  int cnt = 0;
-  const int nword = (nc + 31) >> 5;
-#pragma unroll 1
-  for (int base = 0; base < nword * 32; base += kThreads) {
-    const int i = base + tid;
-    bool keep = false;
-    if (i < nc) {
-      const float x = staged ? W[i] : ldcg_f(W + i);
-      keep = x >= m;
-    }
-    const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0 && (i >> 5) < nword) kb[i >> 5] = bal;
-    cnt += keep;
-  }
-  const float total = block_sum_fixed((float)cnt, red);
-  stamp(a, 22);
+  // publish what every CTA needs to decide kept rows from its own logits: W = exp(l - M) * inv
+  // (the same two operations as above, so the same bits) and the threshold m
   if (tid == 0) {
+    float* hp = a.head_par + (size_t)bh * 4;
+    hp[0] = M;
+    hp[1] = inv;
+    hp[2] = m;
     if (a.threshold) a.threshold[bh] = m;
-    if (a.kept_count) a.kept_count[bh] = (int)total;
     if (a.cand_count) a.cand_count[bh] = nc;
   }
+  if (a.kept_count) {  // only when the caller asks for it
+    int cnt = 0;
+    for (int i = tid; i < nc; i += kThreads) cnt += (staged ? W[i] : ldcg_f(W + i)) >= m;
+    const float total = block_sum_fixed((float)cnt, red);
+    if (tid == 0) a.kept_count[bh] = (int)total;
+  }
+  stamp(a, 22);
 }
 
 // ------------------------------------------------------------------------- phase 6: kept union
@@ -985,26 +1013,46 @@ __device__ int phase_kept_rows(const FusedArgs& a, int b, int kvh, int n, int U,
                                Smem& sm, uint16_t* rowmask, int* scan_sh) {
   const int tid = threadIdx.x, nw = sm.nw;
   const int u0 = (int)((long)U * r / C), u1 = (int)((long)U * (r + 1) / C);
+  float hM[G], hinv[G], hm[G];
+#pragma unroll
+  for (int hl = 0; hl < G; ++hl) {
+    const float* hp = a.head_par + (size_t)(b * a.hq + kvh * G + hl) * 4;
+    hM[hl] = ldcg_f(hp);
+    hinv[hl] = ldcg_f(hp + 1);
+    hm[hl] = ldcg_f(hp + 2);
+  }
   int cnt = 0;
   for (int u = u0 + tid; u < u1; u += kThreads) {
     const int j = union_select(sm.ubits, sm.upre, nw, u);
-    uint32_t words[G];
-    int shift[G];
+    float4 lg[G][4];
+    bool sel[G];
 #pragma unroll
-    for (int hl = 0; hl < G; ++hl) {  // issue every head's load before combining
+    for (int hl = 0; hl < G; ++hl) {  // every head's 16 logits in flight before deciding
       const uint32_t* hb = sm.hbits + hl * nw;
-      words[hl] = 0;
-      shift[hl] = 0;
-      if ((hb[j >> 5] >> (j & 31)) & 1u) {
-        const int slot = kPage * rank_in(hb, sm.hpre + hl * nw, j);
-        shift[hl] = slot & 31;
-        words[hl] = ldcg_u(a.keptbits + (size_t)(b * a.hq + kvh * G + hl) * a.kept_words +
-                           (slot >> 5));
+      sel[hl] = (hb[j >> 5] >> (j & 31)) & 1u;
+      if (sel[hl]) {
+        const int rk = rank_in(hb, sm.hpre + hl * nw, j);
+        const float4* src = reinterpret_cast<const float4*>(
+            a.logits + (size_t)(b * a.hq + kvh * G + hl) * a.cand_stride + (size_t)rk * kPage);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) lg[hl][q4] = __ldcg(src + q4);
       }
     }
     uint32_t m = 0;
 #pragma unroll
-    for (int hl = 0; hl < G; ++hl) m |= (words[hl] >> shift[hl]) & 0xFFFFu;
+    for (int hl = 0; hl < G; ++hl) {
+      if (!sel[hl]) continue;
+      const bool live = hM[hl] > -INFINITY;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float l4[4] = {lg[hl][q4].x, lg[hl][q4].y, lg[hl][q4].z, lg[hl][q4].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float w = live ? __expf(l4[e] - hM[hl]) * hinv[hl] : 0.f;
+          m |= (w >= hm[hl] ? 1u : 0u) << (4 * q4 + e);
+        }
+      }
+    }
     const int rows = page_rows(n, j);
     m &= rows >= 16 ? 0xFFFFu : ((1u << rows) - 1u);
     rowmask[u - u0] = (uint16_t)m;
@@ -1358,16 +1406,15 @@ FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) 
   const int groups = batch * hkv;
   pl.sel_words = (max_pages + 31) / 32;
   pl.cand_stride = kPage * max_budget;
-  pl.kept_words = (pl.cand_stride + 31) / 32;
   pl.union_stride = kPage * max_pages;
   // cluster size: enough CTAs to fill the GPU, at most 16
   const int sms = num_sms();
   int c = 1;
-  while (c < 16 && groups * c * 2 <= sms) c *= 2;
-  // TWL_FUSED_CLUSTER=1|2|4|8|16 forces the cluster size (used by the tests to cover every size)
+  while (c < 16 && groups * (c + 1) <= sms) ++c;
+  // TWL_FUSED_CLUSTER=1..16 forces the cluster size (used by the tests to cover several sizes)
   if (const char* env = getenv("TWL_FUSED_CLUSTER")) {
     const int f = atoi(env);
-    if (f == 1 || f == 2 || f == 4 || f == 8 || f == 16) c = f;
+    if (f >= 1 && f <= 16) c = f;
   }
   pl.cluster = c;
   const size_t persistent = (size_t)persistent_bytes(g, pl.sel_words);
@@ -1383,7 +1430,8 @@ FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) 
   size_t want = scratch;
   const size_t topk_need = 1280 + (size_t)4 * max_pages + 4 * kWarps * 512 + 2048;
   want = want > topk_need ? want : topk_need;
-  want = want > 256 + (size_t)4 * pl.cand_stride ? want : 256 + (size_t)4 * pl.cand_stride;
+  const size_t prune_need = 1024 + (size_t)4 * pl.cand_stride + 4 * 32 * 8 + 64;
+  want = want > prune_need ? want : prune_need;
   want = want > (size_t)2 * pl.union_stride / 16 + 16 ? want : (size_t)2 * pl.union_stride / 16 + 16;
   if (persistent + want > cap) want = cap - persistent;
   pl.smem_bytes = (int)(persistent + want);
@@ -1401,7 +1449,7 @@ size_t fused_workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_
   add(bh * max_pages * 4);                    // scores
   add(bh * pl.sel_words * 4);                 // selected-page bitmaps
   add(bh * (size_t)pl.cand_stride * 4);       // logits / weights
-  add(bh * (size_t)pl.kept_words * 4);        // kept bits
+  add(bh * 4 * 4);                            // per-head (max, 1/sum, threshold)
   add(groups * 16 * g * 2 * 4);               // partial (max, sum)
   add(groups * 16 * 4);                       // union counts per CTA
   add(groups * (size_t)pl.union_stride * 4);  // union token lists
@@ -1422,7 +1470,7 @@ void carve_fused(FusedArgs& a, char* ws, const FusedPlan& pl, int batch, int hq,
   a.scores = reinterpret_cast<float*>(take(bh * max_pages * 4));
   a.selbits = reinterpret_cast<uint32_t*>(take(bh * pl.sel_words * 4));
   a.logits = reinterpret_cast<float*>(take(bh * (size_t)pl.cand_stride * 4));
-  a.keptbits = reinterpret_cast<uint32_t*>(take(bh * (size_t)pl.kept_words * 4));
+  a.head_par = reinterpret_cast<float*>(take(bh * 4 * 4));
   a.part_ms = reinterpret_cast<float*>(take(groups * 16 * g * 2 * 4));
   a.union_part = reinterpret_cast<int*>(take(groups * 16 * 4));
   int* ulist = reinterpret_cast<int*>(take(groups * (size_t)pl.union_stride * 4));
@@ -1507,11 +1555,11 @@ static int active_clusters(int g, int c, int smem_bytes) {
   return n;
 }
 
-// Cluster size for `groups` groups: the largest c <= want whose clusters for every group can be
-// resident at once; if none can, the c that keeps the most CTAs resident.
+// Cluster size for `groups` groups: the largest c <= want (any size up to 16) whose clusters for
+// every group can be resident at once; if none can, the c that keeps the most CTAs resident.
 int fit_cluster(int g, int want, int groups, int smem_bytes) {
   int best = 1, best_ctas = 0;
-  for (int c = want; c >= 1; c >>= 1) {
+  for (int c = want; c >= 1; --c) {
     const int n = c == 1 ? groups : active_clusters(g, c, smem_bytes);
     if (n >= groups) return c;
     if (n * c > best_ctas) {

@@ -35,13 +35,13 @@ struct FusedArgs {
   float* scores;
   uint32_t* selbits;
   float* logits;
-  uint32_t* keptbits;
+  float* head_par;  // [B * Hq][4]: max logit, 1 / sum of exp, top-p threshold
   float* part_ms;
   int* union_part;
   float* part_att;
   uint32_t* flags;
   // strides and launch shape
-  int sel_words, cand_stride, kept_words, union_stride;
+  int sel_words, cand_stride, union_stride;
   int cluster;
   int smem_bytes;
 };
@@ -49,7 +49,7 @@ struct FusedArgs {
 struct FusedPlan {
   int cluster;
   int smem_bytes;
-  int sel_words, cand_stride, kept_words, union_stride;
+  int sel_words, cand_stride, union_stride;
   bool ok;
 };
 

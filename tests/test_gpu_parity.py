@@ -350,7 +350,7 @@ def test_decode_step_dense_limit():
         check_attention(o[bb, h], lse[bb, h], o_or, lse_or, f"dense h{h}")
 
 
-@pytest.mark.parametrize("cluster", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("cluster", [1, 2, 3, 4, 7, 8, 12, 16])
 def test_decode_step_every_cluster_size(cluster, monkeypatch):
     monkeypatch.setenv("TWL_FUSED_CLUSTER", str(cluster))
     wl = synth.make_decode("clusters", 2, 8, 2, [3001, 515], seed=9)
