@@ -70,6 +70,11 @@ __device__ __forceinline__ void stamp(const FusedArgs&, int) {}
 #endif
 
 __device__ __forceinline__ float ldcg_f(const float* p) { return __ldcg(p); }
+
+// Bulk prefetch of a 16-byte aligned range (size a multiple of 16) into L2.
+__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ int ldcg_i(const int* p) { return __ldcg(p); }
 __device__ __forceinline__ uint32_t ldcg_u(const uint32_t* p) { return __ldcg(p); }
 
@@ -84,7 +89,8 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
 }
 
 // Same fragment map as the staged estimate kernel (see twl_estimate.cu).
-__device__ __forceinline__ void q_fragments(const uint16_t* qh, bool valid, uint32_t (&bf)[8][2]) {
+// Also returns the sum of the lane's 32 query channels (for the zero-point term).
+__device__ __forceinline__ float q_fragments(const uint16_t* qh, bool valid, uint32_t (&bf)[8][2]) {
   const int t = threadIdx.x & 3;
   uint32_t w[16];
 #pragma unroll
@@ -93,12 +99,19 @@ __device__ __forceinline__ void q_fragments(const uint16_t* qh, bool valid, uint
         valid ? *reinterpret_cast<const uint4*>(qh + 32 * t + 8 * i) : make_uint4(0, 0, 0, 0);
     w[4 * i + 0] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
   }
+  float qsum = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    qsum += f.x + f.y;
+  }
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
     const int w8 = ks >> 1, e = ks & 1;
     bf[ks][0] = __byte_perm(w[4 * w8 + e], w[4 * w8 + e + 2], 0x5410);
     bf[ks][1] = __byte_perm(w[4 * w8 + e], w[4 * w8 + e + 2], 0x7632);
   }
+  return qsum;
 }
 
 __device__ __forceinline__ uint32_t nib_pair(uint32_t x, int i) {
@@ -116,6 +129,7 @@ __host__ __device__ constexpr int persistent_bytes(int g, int sel_words) {
 // Shared-memory layout: a persistent region for the page bitmaps (phases 3-6) and one scratch
 // region reused by the phases.
 struct Smem {
+  const int* pt;    // the sequence's page table (validated; -1 = bad entry), or nullptr
   uint32_t* hbits;  // [G][nw]  head page bitmaps
   int* hpre;        // [G][nw]  exclusive prefix popcounts per word
   uint32_t* ubits;  // [nw]     union bitmap
@@ -156,18 +170,22 @@ __device__ __forceinline__ int union_select(const uint32_t* ubits, const int* up
   return 32 * lo + nth_set_bit(ubits[lo], u - upre[lo]);
 }
 
+// Physical page of logical page j: from the staged copy when there is one.
+__device__ __forceinline__ int phys_of(const FusedArgs& a, const Smem& sm, int b, int j) {
+  if (sm.pt) return sm.pt[j];
+  return load_phys(a.kv.page_table, b, j, a.kv.max_pages, a.kv.num_phys, a.flags);
+}
+
 // ------------------------------------------------------------------------- phase 1: scores
-// The CTA's slice of the page table is staged in shared memory first (one coalesced read), so
-// the bounds loads of kIt page pairs per warp are all independent and in flight together.
+// The bounds of the CTA's pages (512 B per page) are copied into shared memory in chunks with
+// 16-byte cp.async spread over all threads (one memory round trip per chunk); a half-warp then
+// scores a page for all G heads.
 template <int G>
 __device__ void phase_scores(const FusedArgs& a, int b, int kvh, int n_pages, int r, int C,
                              Smem& sm) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int half = lane >> 4, l = lane & 15;
   const int p0 = (int)((long)n_pages * r / C), p1 = (int)((long)n_pages * (r + 1) / C);
-  int* phys = reinterpret_cast<int*>(sm.scratch);  // [p1 - p0]
-  for (int j = p0 + (int)threadIdx.x; j < p1; j += kThreads)
-    phys[j - p0] = load_phys(a.kv.page_table, b, j, a.kv.max_pages, a.kv.num_phys, a.flags);
   float qv[G][8];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -175,29 +193,40 @@ __device__ void phase_scores(const FusedArgs& a, int b, int kvh, int n_pages, in
         a.q + ((size_t)b * a.hq + kvh * G + h) * kHeadDim + 8 * l);
     unpack8(raw, qv[h]);
   }
-  __syncthreads();
-  constexpr int kIt = G <= 4 ? 4 : 2;  // page pairs in flight per warp
-  for (int base = p0; base < p1; base += kWarps * 2 * kIt) {
-    uint4 bmn[kIt], bmx[kIt];
-    bool ok[kIt];
-#pragma unroll
-    for (int it = 0; it < kIt; ++it) {
-      const int j = base + it * kWarps * 2 + 2 * warp + half;
-      const int ph = j < p1 ? phys[j - p0] : -1;
-      ok[it] = ph >= 0;
-      bmn[it] = make_uint4(0, 0, 0, 0);
-      bmx[it] = bmn[it];
-      if (ok[it]) {
-        const uint16_t* src = a.bounds + (((size_t)ph * a.kv.hkv + kvh) * 2) * kHeadDim + 8 * l;
-        bmn[it] = __ldg(reinterpret_cast<const uint4*>(src));
-        bmx[it] = __ldg(reinterpret_cast<const uint4*>(src + kHeadDim));
-      }
+  int* phys = reinterpret_cast<int*>(sm.scratch);
+  const int cap = (sm.scratch_bytes - 128) / (4 + 512);
+  const int ch = cap < 1024 ? cap : 1024;
+  unsigned char* buf = sm.scratch + ((4 * ch + 127) & ~127);
+#pragma unroll 1
+  for (int c0 = p0; c0 < p1; c0 += ch) {
+    const int cn = min(ch, p1 - c0);
+    for (int i = threadIdx.x; i < cn; i += kThreads)
+      phys[i] = phys_of(a, sm, b, c0 + i);
+    __syncthreads();
+    // 32 chunks of 16 bytes per page, spread over all threads, all in flight together
+    for (int c = threadIdx.x; c < 32 * cn; c += kThreads) {
+      const int i = c >> 5, k = c & 31;
+      const int ph = phys[i];
+      const uint16_t* src =
+          ph >= 0 ? a.bounds + ((size_t)ph * a.kv.hkv + kvh) * 2 * kHeadDim + 8 * k : a.bounds;
+      cp_async16(buf + 512 * i + 16 * k, src, ph >= 0);
     }
-#pragma unroll
-    for (int it = 0; it < kIt; ++it) {
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncthreads();
+    const bool ok = true;
+    for (int base = 0; base < cn; base += 2 * kWarps) {  // warp-uniform trip count
+      const int i0 = base + 2 * warp + half;
+      const bool in = i0 < cn;
+      const int ph = in ? phys[i0] : -1;
+      uint4 vmn = make_uint4(0, 0, 0, 0), vmx = vmn;
+      if (ph >= 0 && ok) {
+        vmn = *reinterpret_cast<const uint4*>(buf + 512 * i0 + 16 * l);
+        vmx = *reinterpret_cast<const uint4*>(buf + 512 * i0 + 256 + 16 * l);
+      }
       float mn[8], mx[8];
-      unpack8(bmn[it], mn);
-      unpack8(bmx[it], mx);
+      unpack8(vmn, mn);
+      unpack8(vmx, mx);
       float acc[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -212,13 +241,48 @@ __device__ void phase_scores(const FusedArgs& a, int b, int kvh, int n_pages, in
         for (int h = 0; h < G; ++h)
           acc[h] = __fadd_rn(acc[h], __shfl_xor_sync(0xffffffffu, acc[h], off));
       }
-      const int j = base + it * kWarps * 2 + 2 * warp + half;
-      if (j < p1 && l < G) {
+      if (in && l < G) {
         float v = acc[0];
 #pragma unroll
         for (int h = 1; h < G; ++h) v = (l == h) ? acc[h] : v;
-        if (!ok[it]) v = -INFINITY;
-        a.scores[((size_t)b * a.hq + kvh * G + l) * a.kv.max_pages + j] = v;
+        if (ph < 0) v = -INFINITY;
+        a.scores[((size_t)b * a.hq + kvh * G + l) * a.kv.max_pages + c0 + i0] = v;
+      }
+    }
+    __syncthreads();  // the chunk's buffer is read before the next copies land
+  }
+}
+
+// Bitonic sort of 256 keys held by one warp, descending.  Key i*32 + lane lives in v[i] of
+// `lane`; partners at distance >= 32 are in the same lane, smaller distances one shuffle away.
+__device__ __forceinline__ void warp_sort256_desc(uint32_t (&v)[8]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 256; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= 32) {
+        const int rs = stride >> 5;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = i ^ rs;
+          if (j > i) {
+            const bool desc = ((i * 32 + lane) & size) == 0;
+            const uint32_t x = v[i], y = v[j];
+            const bool swap = desc ? (x < y) : (x > y);
+            v[i] = swap ? y : x;
+            v[j] = swap ? x : y;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t other = __shfl_xor_sync(0xffffffffu, v[i], stride);
+          const bool lower = (lane & stride) == 0;
+          const bool desc = ((i * 32 + lane) & size) == 0;
+          const uint32_t hi = max(v[i], other), lo = min(v[i], other);
+          v[i] = (lower == desc) ? hi : lo;
+        }
       }
     }
   }
@@ -270,38 +334,81 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
   stamp(a, 23);
   auto key_at = [&](int i) -> uint32_t { return staged ? keys[i] : f32_key(ldcg_f(row + i)); };
 
-  // Radix select over the bits where this head's keys differ: the common prefix of the smallest
-  // and largest key is known, the rest is split into at most three digits (9 bits each when
-  // that suffices, else 8-bit digits).  Histograms are per warp (no cross-warp atomics).
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (int i = tid; i < n_pages; i += kThreads) {
-    const uint32_t k = key_at(i);
-    kmin = min(kmin, k);
-    kmax = max(kmax, k);
-  }
-  kmin = __reduce_min_sync(0xffffffffu, kmin);
-  kmax = __reduce_max_sync(0xffffffffu, kmax);
-  __syncthreads();
-  if (lane == 0) {
-    hist[2 * warp] = kmin;
-    hist[2 * warp + 1] = kmax;
-  }
-  __syncthreads();
-  kmin = 0xFFFFFFFFu;
-  kmax = 0u;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    kmin = min(kmin, hist[2 * w]);
-    kmax = max(kmax, hist[2 * w + 1]);
-  }
-  const uint32_t diff = kmin ^ kmax;
-  uint32_t prefix, mask;
+  // Where to start narrowing.  A sample of 256 keys (every n/256-th page), sorted by one warp,
+  // brackets the k-th largest key between the sample's ranks r* - 16 and r* + 16
+  // (r* = k * 256 / n); when the keys above and inside the common-prefix block of that bracket
+  // confirm it (above < k <= above + inside), narrowing starts from that block.  Otherwise it
+  // starts from the common prefix of the smallest and largest key.
+  uint32_t prefix = 0u, mask = 0u;
   int remaining = kb;
-  int eq_count = n_pages;  // keys equal to the final prefix (all keys when they are all equal)
-  int hi_bit = diff ? 31 - __clz(diff) : -1;
-  mask = hi_bit >= 31 ? 0u : ~((2u << hi_bit) - 1u);
-  if (hi_bit < 0) mask = 0xFFFFFFFFu;
-  prefix = kmax & mask;
+  int hi_bit = 31;
+  int cand = n_pages;
+  bool bracketed = false;
+  if (staged && n_pages > 512) {
+    if (warp == 0) {
+      uint32_t v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = keys[(int)((long)(i * 32 + lane) * n_pages / 256)];
+      warp_sort256_desc(v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hist[i * 32 + lane] = v[i];
+    }
+    __syncthreads();
+    const int rstar = (int)((long)kb * 256 / n_pages);
+    const uint32_t hi_key = rstar - 16 >= 0 ? hist[rstar - 16] : 0xFFFFFFFFu;
+    const uint32_t lo_key = rstar + 16 <= 255 ? hist[rstar + 16] : 0u;
+    const uint32_t d = lo_key ^ hi_key;
+    const int hb = d ? 31 - __clz(d) : -1;
+    const uint32_t bmask = hb >= 31 ? 0u : (hb < 0 ? 0xFFFFFFFFu : ~((2u << hb) - 1u));
+    const uint32_t bpre = hi_key & bmask;
+    int packed = 0;  // above * 65536 + inside (n <= 32768)
+    for (int i = tid; i < n_pages; i += kThreads) {
+      const uint32_t k = keys[i] & bmask;
+      packed += (k > bpre ? 65536 : 0) + (k == bpre ? 1 : 0);
+    }
+    int tot;
+    block_exclusive_scan(packed, scan_sh, &tot);
+    const int above = tot >> 16, inside = tot & 0xFFFF;
+    if (above < kb && kb <= above + inside) {
+      prefix = bpre;
+      mask = bmask;
+      remaining = kb - above;
+      cand = inside;
+      hi_bit = hb;
+      bracketed = true;
+    }
+  }
+  if (!bracketed) {
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i = tid; i < n_pages; i += kThreads) {
+      const uint32_t k = key_at(i);
+      kmin = min(kmin, k);
+      kmax = max(kmax, k);
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    __syncthreads();
+    if (lane == 0) {
+      hist[2 * warp] = kmin;
+      hist[2 * warp + 1] = kmax;
+    }
+    __syncthreads();
+    kmin = 0xFFFFFFFFu;
+    kmax = 0u;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      kmin = min(kmin, hist[2 * w]);
+      kmax = max(kmax, hist[2 * w + 1]);
+    }
+    const uint32_t diff = kmin ^ kmax;
+    hi_bit = diff ? 31 - __clz(diff) : -1;
+    mask = hi_bit >= 31 ? 0u : ~((2u << hi_bit) - 1u);
+    if (hi_bit < 0) mask = 0xFFFFFFFFu;
+    prefix = kmax & mask;
+    remaining = kb;
+    cand = n_pages;
+  }
+  __syncthreads();
   // Narrow the candidate bin with histogram passes over the next (up to) 10 bits of the keys
   // that still match the prefix, until it holds at most kGatherCap keys; every key above the bin
   // is selected, and the bin's keys are ranked exactly by (key desc, page asc).  Only when all
@@ -316,7 +423,6 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
                                   16 <= (size_t)sm.scratch_bytes;
   uint32_t* hh = room ? bhist : hist;  // the 256-bin histogram when there is no room
   const int max_dw = room ? 10 : 8;
-  int cand = n_pages;
   const int n_it = (n_pages + kThreads - 1) / kThreads;
 #pragma unroll 1
   while ((cand > kGatherCap || !room) && hi_bit >= 0) {
@@ -539,12 +645,9 @@ __device__ void phase_union_bitmaps(const FusedArgs& a, int b, int kvh, Smem& sm
 }
 
 // ------------------------------------------------------------------------- phase 4: estimate
-// The CTA's share of the union is processed in chunks of up to kEstChunk pages: first every
-// page's logical id and physical page are staged in shared memory (thread per page), then each
-// warp takes kEstBatch pages at a time and issues all their INT4 loads before computing.
-constexpr int kEstChunk = 1024;
-constexpr int kEstBatch = 4;
-
+// The CTA's share of the union is processed in chunks: every page's logical id and physical page
+// are staged (thread per page), then its INT4 tile (1 KB) and scale/zero row (64 B) are copied
+// into shared memory with 16-byte cp.async over all threads; one warp then computes a page.
 template <int G>
 __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n, int U, int r,
                                int C, Smem& sm) {
@@ -553,18 +656,17 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
   const int nw = sm.nw;
   const float inv_sqrt_d = 0.08838834764831845f;
   const int u0 = (int)((long)U * r / C), u1 = (int)((long)U * (r + 1) / C);
-  float* red = reinterpret_cast<float*>(sm.scratch);                  // [kWarps][8][2]
-  int* pj = reinterpret_cast<int*>(sm.scratch + 2048);                 // [kEstChunk]
-  int* pph = reinterpret_cast<int*>(sm.scratch + 2048 + 4 * kEstChunk);  // [kEstChunk]
+  float* red = reinterpret_cast<float*>(sm.scratch);  // [kWarps][8]
+  const int cap = (sm.scratch_bytes - 1024 - 256) / (8 + 1088);
+  const int ch = cap < 1024 ? cap : 1024;
+  int* pj = reinterpret_cast<int*>(sm.scratch + 1024);  // [ch]
+  int* pph = pj + ch;                                    // [ch]
+  unsigned char* tiles = sm.scratch + ((1024 + 8 * ch + 127) & ~127);  // [ch][1024] nibbles
+  unsigned char* szs = tiles + 1024 * ch;                              // [ch][64] scale/zero
   uint32_t bf[8][2];
   const bool head_ok = gr < G;
   const uint16_t* qh = a.q + ((size_t)b * a.hq + kvh * G + (head_ok ? gr : 0)) * kHeadDim;
-  q_fragments(qh, head_ok, bf);
-  float qs_part = 0.f;
-  if (head_ok) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) qs_part += __half2float(__ushort_as_half(qh[32 * t + i]));
-  }
+  float qs_part = q_fragments(qh, head_ok, bf);
   qs_part += __shfl_xor_sync(0xffffffffu, qs_part, 1);
   qs_part += __shfl_xor_sync(0xffffffffu, qs_part, 2);
   const float qsum0 = __shfl_sync(0xffffffffu, qs_part, (2 * t) * 4);
@@ -572,42 +674,56 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
   // running max of this lane's two heads over its rows (the softmax's shift)
   float rm[2] = {-INFINITY, -INFINITY};
 
-  for (int c0 = u0; c0 < u1; c0 += kEstChunk) {
-    const int cn = min(kEstChunk, u1 - c0);
-    __syncthreads();  // previous chunk's staging fully consumed
+#pragma unroll 1
+  for (int c0 = u0; c0 < u1; c0 += ch) {
+    const int cn = min(ch, u1 - c0);
     for (int i = threadIdx.x; i < cn; i += kThreads) {
       const int j = union_select(sm.ubits, sm.upre, nw, c0 + i);
       pj[i] = j;
-      pph[i] = load_phys(a.kv.page_table, b, j, a.kv.max_pages, a.kv.num_phys, a.flags);
+      pph[i] = phys_of(a, sm, b, j);
     }
     __syncthreads();
-    for (int i0 = warp * kEstBatch; i0 < cn; i0 += kWarps * kEstBatch) {
-      uint4 x0[kEstBatch], x1[kEstBatch];
-      uint32_t sz0[kEstBatch], sz1[kEstBatch];
+    stamp(a, 25);
+    // 68 chunks of 16 bytes per page (64 of nibbles, 4 of scale/zero), spread over all threads
+    for (int c = threadIdx.x; c < 68 * cn; c += kThreads) {
+      const int i = c / 68, k = c - 68 * i;
+      const int ph = pph[i];
+      const size_t tile = ph >= 0 ? ((size_t)ph * a.kv.hkv + kvh) * kPage : 0;
+      if (k < 64)
+        cp_async16(tiles + 1024 * i + 16 * k, a.k_int4 + tile * (kHeadDim / 2) + 16 * k, ph >= 0);
+      else
+        cp_async16(szs + 64 * i + 16 * (k - 64), a.k_sz + tile * 2 + 8 * (k - 64), ph >= 0);
+    }
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncthreads();
+    stamp(a, 26);
+    const bool ok = true;
+    // two pages per warp iteration: their mma chains and epilogues are independent
+#pragma unroll 1
+    for (int i0 = 2 * warp; i0 < cn; i0 += 2 * kWarps) {
+      float accp[2][4];
+      int jp[2];
+      bool badp[2];
+      uint32_t szp[2][2];
 #pragma unroll
-      for (int k = 0; k < kEstBatch; ++k) {
-        const int i = i0 + k;
-        const int ph = i < cn ? pph[i] : -1;
-        x0[k] = make_uint4(0, 0, 0, 0);
-        x1[k] = x0[k];
-        sz0[k] = sz1[k] = 0;
-        if (ph >= 0) {
-          const size_t tile = ((size_t)ph * a.kv.hkv + kvh) * kPage;
-          const uint4* src = reinterpret_cast<const uint4*>(a.k_int4 + tile * (kHeadDim / 2));
-          x0[k] = __ldg(src + lane);
-          x1[k] = __ldg(src + 32 + lane);
-          sz0[k] = __ldg(reinterpret_cast<const uint32_t*>(a.k_sz + tile * 2) + gr);
-          sz1[k] = __ldg(reinterpret_cast<const uint32_t*>(a.k_sz + tile * 2) + gr + 8);
+      for (int pp = 0; pp < 2; ++pp) {
+        const int i = i0 + pp;
+        const bool in = i < cn;
+        jp[pp] = in ? pj[i] : 0;
+        badp[pp] = !in || pph[i] < 0 || !ok;
+        uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
+        szp[pp][0] = szp[pp][1] = 0;
+        if (!badp[pp]) {
+          const uint4* tp = reinterpret_cast<const uint4*>(tiles + 1024 * i);
+          x0 = tp[lane];
+          x1 = tp[32 + lane];
+          const uint32_t* sp = reinterpret_cast<const uint32_t*>(szs + 64 * i);
+          szp[pp][0] = sp[gr];
+          szp[pp][1] = sp[gr + 8];
         }
-      }
-#pragma unroll
-      for (int k = 0; k < kEstBatch; ++k) {
-        const int i = i0 + k;
-        if (i >= cn) break;  // warp-uniform
-        const int j = pj[i];
-        const bool bad = pph[i] < 0;
-        const uint32_t r0[4] = {x0[k].x, x0[k].y, x0[k].z, x0[k].w};
-        const uint32_t r1[4] = {x1[k].x, x1[k].y, x1[k].z, x1[k].w};
+        const uint32_t r0[4] = {x0.x, x0.y, x0.z, x0.w};
+        const uint32_t r1[4] = {x1.x, x1.y, x1.z, x1.w};
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
@@ -619,11 +735,20 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
           av[3] = nib_pair(r1[w8], 2 * e + 1);
           mma_16816(acc, av, bf[ks][0], bf[ks][1]);
         }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) accp[pp][k] = acc[k];
+      }
+#pragma unroll
+      for (int pp = 0; pp < 2; ++pp) {
+        if (i0 + pp >= cn) break;  // warp-uniform
+        const int j = jp[pp];
+        const bool bad = badp[pp];
         const int rows = page_rows(n, j);
-        const float s0 = __half2float(__ushort_as_half((unsigned short)(sz0[k] & 0xFFFFu)));
-        const float z0 = __half2float(__ushort_as_half((unsigned short)(sz0[k] >> 16)));
-        const float s1 = __half2float(__ushort_as_half((unsigned short)(sz1[k] & 0xFFFFu)));
-        const float z1 = __half2float(__ushort_as_half((unsigned short)(sz1[k] >> 16)));
+        const uint32_t sz0 = szp[pp][0], sz1 = szp[pp][1];
+        const float s0 = __half2float(__ushort_as_half((unsigned short)(sz0 & 0xFFFFu)));
+        const float z0 = __half2float(__ushort_as_half((unsigned short)(sz0 >> 16)));
+        const float s1 = __half2float(__ushort_as_half((unsigned short)(sz1 & 0xFFFFu)));
+        const float z1 = __half2float(__ushort_as_half((unsigned short)(sz1 >> 16)));
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int hl = 2 * t + e;
@@ -639,7 +764,8 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
             const int row = gr + 8 * rr;
             if (row >= rows) continue;
             const float sv = rr ? s1 : s0, zv = rr ? z1 : z0;
-            const float lg = bad ? -INFINITY : (sv * acc[2 * rr + e] + zv * qsum) * inv_sqrt_d;
+            const float lg =
+                bad ? -INFINITY : (sv * accp[pp][2 * rr + e] + zv * qsum) * inv_sqrt_d;
             a.logits[obase + row] = lg;
             if (a.cand_tok) a.cand_tok[obase + row] = kPage * j + row;
             rm[e] = fmaxf(rm[e], lg);
@@ -647,6 +773,8 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
         }
       }
     }
+    __syncthreads();  // the chunk's tiles are read before the next copies land
+    stamp(a, 27);
   }
   // combine the maxima over the 8 row-lanes of each head, then over the warps
 #pragma unroll
@@ -1063,6 +1191,73 @@ __device__ int phase_kept_rows(const FusedArgs& a, int b, int kvh, int n, int U,
   return total;
 }
 
+// Kept rows of this CTA's union share for attention without a global list: per page (in union
+// order) its 16-bit row mask, the exclusive prefix of kept rows, and its physical page.
+// Returns the number of kept rows of the share.
+template <int G>
+__device__ int phase_kept_rows_local(const FusedArgs& a, int b, int kvh, int n, int U, int r,
+                                     int C, Smem& sm, uint16_t* rowmask, int* pfx, int* pph,
+                                     int* scan_sh) {
+  const int tid = threadIdx.x, nw = sm.nw;
+  const int u0 = (int)((long)U * r / C), u1 = (int)((long)U * (r + 1) / C);
+  float hM[G], hinv[G], hm[G];
+#pragma unroll
+  for (int hl = 0; hl < G; ++hl) {
+    const float* hp = a.head_par + (size_t)(b * a.hq + kvh * G + hl) * 4;
+    hM[hl] = ldcg_f(hp);
+    hinv[hl] = ldcg_f(hp + 1);
+    hm[hl] = ldcg_f(hp + 2);
+  }
+  int carry = 0;
+#pragma unroll 1
+  for (int ub = u0; ub < u1; ub += kThreads) {
+    const int u = ub + tid;
+    uint32_t m = 0;
+    if (u < u1) {
+      const int j = union_select(sm.ubits, sm.upre, nw, u);
+      const int ph = phys_of(a, sm, b, j);
+      float4 lg[G][4];
+      bool sel[G];
+#pragma unroll
+      for (int hl = 0; hl < G; ++hl) {
+        const uint32_t* hb = sm.hbits + hl * nw;
+        sel[hl] = (hb[j >> 5] >> (j & 31)) & 1u;
+        if (sel[hl]) {
+          const int rk = rank_in(hb, sm.hpre + hl * nw, j);
+          const float4* src = reinterpret_cast<const float4*>(
+              a.logits + (size_t)(b * a.hq + kvh * G + hl) * a.cand_stride + (size_t)rk * kPage);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) lg[hl][q4] = __ldcg(src + q4);
+        }
+      }
+#pragma unroll
+      for (int hl = 0; hl < G; ++hl) {
+        if (!sel[hl]) continue;
+        const bool live = hM[hl] > -INFINITY;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const float l4[4] = {lg[hl][q4].x, lg[hl][q4].y, lg[hl][q4].z, lg[hl][q4].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float w = live ? __expf(l4[e] - hM[hl]) * hinv[hl] : 0.f;
+            m |= (w >= hm[hl] ? 1u : 0u) << (4 * q4 + e);
+          }
+        }
+      }
+      const int rows = page_rows(n, j);
+      m &= rows >= 16 ? 0xFFFFu : ((1u << rows) - 1u);
+      rowmask[u - u0] = (uint16_t)m;
+      pph[u - u0] = ph;
+    }
+    int total;
+    const int ex = block_exclusive_scan(__popc(m), scan_sh, &total);
+    if (u < u1) pfx[u - u0] = carry + ex;
+    carry += total;
+  }
+  __syncthreads();
+  return carry;
+}
+
 template <int G>
 __device__ void phase_write_union(const FusedArgs& a, int gi, int U, int r, int C, int base,
                                   Smem& sm, const uint16_t* rowmask, int* scan_sh) {
@@ -1091,9 +1286,12 @@ __device__ void phase_write_union(const FusedArgs& a, int gi, int U, int r, int 
 // ------------------------------------------------------------------------- phase 7: attention
 // Thread layout: token slot t = tid / 8 (64 per round), sub-lane s = tid % 8 owns channels
 // [8s, 8s+8) and [64+8s, 64+8s+8).  For P.V: channel d = tid % 128, token quarter = tid / 128.
-template <int G>
+// kLocal: tokens of this CTA's own union share, from (rowmask, pfx, pph) in shared memory;
+// otherwise an even share [T r / C, T (r+1) / C) of the group's global ascending list.
+template <int G, bool kLocal>
 __device__ void phase_attend(const FusedArgs& a, int b, int kvh, int gi, int n, int T, int r, int C,
-                             Smem& sm) {
+                             Smem& sm, const uint16_t* rowmask = nullptr, const int* pfx = nullptr,
+                             const int* pph = nullptr, int npg = 0) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ts = tid >> 3, s8 = tid & 7;
   const int d = tid & 127, quarter = tid >> 7;
@@ -1104,7 +1302,7 @@ __device__ void phase_attend(const FusedArgs& a, int b, int kvh, int gi, int n, 
   float* red = reinterpret_cast<float*>(sp + 32768 + G * 256);    // [kWarps][G]
   uint32_t* rowidx = reinterpret_cast<uint32_t*>(sp + 32768 + G * 256 + kWarps * G * 4);  // 64
   float* opart = reinterpret_cast<float*>(sp + 32768 + G * 256 + kWarps * G * 4 + 256);  // [4][G][128]
-  const int t0 = (int)((long)T * r / C), t1 = (int)((long)T * (r + 1) / C);
+  const int t0 = kLocal ? 0 : (int)((long)T * r / C), t1 = kLocal ? T : (int)((long)T * (r + 1) / C);
   const int* ulist = a.union_tok + (size_t)gi * a.union_stride;
 
   float qv[G][16];
@@ -1131,13 +1329,27 @@ __device__ void phase_attend(const FusedArgs& a, int b, int kvh, int gi, int n, 
     if (tid < kAttChunk) {
       uint32_t ri = 0xFFFFFFFFu;
       if (tid < nt) {
-        const int tk = ldcg_i(ulist + cb + tid);
-        if (tk >= 0 && tk < n) {
-          const int ph = load_phys(a.kv.page_table, b, tk >> 4, a.kv.max_pages, a.kv.num_phys,
-                                   a.flags);
-          if (ph >= 0) ri = (uint32_t)(((size_t)ph * a.kv.hkv + kvh) * kPage + (tk & 15));
+        if (kLocal) {
+          // page of local token t: the last page whose exclusive prefix is <= t
+          const int t = cb + tid;
+          int lo = 0, hi = npg;
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pfx[mid] <= t) lo = mid;
+            else hi = mid;
+          }
+          const int row = nth_set_bit(rowmask[lo], t - pfx[lo]);
+          const int ph = pph[lo];
+          if (ph >= 0) ri = (uint32_t)(((size_t)ph * a.kv.hkv + kvh) * kPage + row);
         } else {
-          raise_flag(a.flags, TWL_FLAG_BAD_INDEX);
+          const int tk = ldcg_i(ulist + cb + tid);
+          if (tk >= 0 && tk < n) {
+            const int ph = load_phys(a.kv.page_table, b, tk >> 4, a.kv.max_pages, a.kv.num_phys,
+                                     a.flags);
+            if (ph >= 0) ri = (uint32_t)(((size_t)ph * a.kv.hkv + kvh) * kPage + (tk & 15));
+          } else {
+            raise_flag(a.flags, TWL_FLAG_BAD_INDEX);
+          }
         }
       }
       rowidx[tid] = ri;
@@ -1276,17 +1488,36 @@ __device__ void phase_merge_head(const FusedArgs& a, int gi, int bh, int hl, int
   if (tid == 0) a.lse[bh] = any ? Mx + __logf(l) : -INFINITY;
 }
 
+template <int G>
+__host__ __device__ constexpr size_t attend_smem_bytes() {
+  return 32768 + G * 256 + kWarps * G * 4 + 256 + 4 * G * kHeadDim * 4;
+}
+
+// The local attention path needs room for the largest share of the cluster (so every CTA takes
+// the same branch and executes the same barriers).
+__device__ __forceinline__ bool local_fits_all(const FusedArgs& a, int U, int C, int att_bytes,
+                                               int scratch_bytes) {
+  (void)a;
+  const int max_share = (U + C - 1) / C;
+  return att_bytes + 10 * max_share + 64 <= scratch_bytes;
+}
+
 // ------------------------------------------------------------------------- the kernel
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ int scan_sh[33];
   __shared__ int s_total;
+
   const int C = (int)cluster_size();
   const int r = (int)cluster_rank();
   const int gi = blockIdx.x / C;
   const int b = gi / a.kv.hkv, kvh = gi % a.kv.hkv;
   const int tid = threadIdx.x;
+  // wait for the previous grid in the stream (launched programmatically), then let the next one
+  // be scheduled: it will in turn wait for this grid to complete before touching memory
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
 
   const Seq sq = load_seq(a.kv.seq_lens, b, a.kv.max_pages, a.flags, r == 0 && tid == 0);
   const int n_pages = sq.pages;
@@ -1318,10 +1549,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
     sm.ubits = reinterpret_cast<uint32_t*>(p);
     p += 4 * a.sel_words;
     sm.upre = reinterpret_cast<int*>(p);
-    p = smem_raw + persistent_bytes(G, a.sel_words);  // scratch starts 128-byte aligned
-    sm.scratch = p;
+    p = smem_raw + persistent_bytes(G, a.sel_words);
+    sm.pt = nullptr;
+    if (a.pt_smem) {  // the sequence's page table, validated once
+      int* pt = reinterpret_cast<int*>(p);
+      for (int j = tid; j < n_pages; j += kThreads)
+        pt[j] = load_phys(a.kv.page_table, b, j, a.kv.max_pages, a.kv.num_phys, a.flags);
+      sm.pt = pt;
+      p += (4 * a.kv.max_pages + 127) & ~127;
+    }
+    sm.scratch = p;  // 128-byte aligned
     sm.scratch_bytes = a.smem_bytes - (int)(p - smem_raw);
   }
+  __syncthreads();
 
   // 1: scores
   stamp(a, 0);
@@ -1365,26 +1605,41 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
   stamp(a, 8);
   cluster_sync();
   stamp(a, 9);
-  // 6: kept rows of this CTA's union pages, counts exchanged, ascending union list written
-  uint16_t* rowmask = reinterpret_cast<uint16_t*>(sm.scratch);
-  const int local = phase_kept_rows<G>(a, b, kvh, sq.n, U, r, C, sm, rowmask, scan_sh);
-  if (tid == 0) a.union_part[(size_t)gi * C + r] = local;
-  stamp(a, 10);
-  cluster_sync();
-  stamp(a, 11);
-  int base = 0, T = 0;
-  for (int rr = 0; rr < C; ++rr) {
-    const int c = ldcg_i(a.union_part + (size_t)gi * C + rr);
-    if (rr < r) base += c;
-    T += c;
+  // 6-7: kept rows of this CTA's union pages, then attention over them.  The group's ordered
+  // union list is only built when the caller asks for it (counts exchanged, list written, then
+  // attention over even shares of it); otherwise every CTA attends over its own kept rows.
+  const int share = (int)((long)U * (r + 1) / C) - (int)((long)U * r / C);
+  const int att_bytes = (int)attend_smem_bytes<G>();
+  const bool local_fits = att_bytes + 10 * share + 64 <= sm.scratch_bytes;
+  if (!a.want_union && local_fits_all(a, U, C, att_bytes, sm.scratch_bytes)) {
+    unsigned char* base = sm.scratch + att_bytes;
+    int* pfx = reinterpret_cast<int*>(base);
+    int* pph = pfx + share;
+    uint16_t* rowmask = reinterpret_cast<uint16_t*>(pph + share);
+    const int T = phase_kept_rows_local<G>(a, b, kvh, sq.n, U, r, C, sm, rowmask, pfx, pph, scan_sh);
+    stamp(a, 10);
+    phase_attend<G, true>(a, b, kvh, gi, sq.n, T, r, C, sm, rowmask, pfx, pph, share);
+  } else {
+    (void)local_fits;
+    uint16_t* rowmask = reinterpret_cast<uint16_t*>(sm.scratch);
+    const int local = phase_kept_rows<G>(a, b, kvh, sq.n, U, r, C, sm, rowmask, scan_sh);
+    if (tid == 0) a.union_part[(size_t)gi * C + r] = local;
+    stamp(a, 10);
+    cluster_sync();
+    stamp(a, 11);
+    int base = 0, T = 0;
+    for (int rr = 0; rr < C; ++rr) {
+      const int c = ldcg_i(a.union_part + (size_t)gi * C + rr);
+      if (rr < r) base += c;
+      T += c;
+    }
+    phase_write_union<G>(a, gi, U, r, C, base, sm, rowmask, scan_sh);
+    if (r == 0 && tid == 0 && a.union_count) a.union_count[gi] = T;
+    stamp(a, 12);
+    cluster_sync();
+    stamp(a, 13);
+    phase_attend<G, false>(a, b, kvh, gi, sq.n, T, r, C, sm);
   }
-  phase_write_union<G>(a, gi, U, r, C, base, sm, rowmask, scan_sh);
-  if (r == 0 && tid == 0 && a.union_count) a.union_count[gi] = T;
-  stamp(a, 12);
-  cluster_sync();
-  stamp(a, 13);
-  // 7: attention over this CTA's even share of the group's kept tokens
-  phase_attend<G>(a, b, kvh, gi, sq.n, T, r, C, sm);
   stamp(a, 14);
   cluster_sync();
   stamp(a, 15);
@@ -1393,10 +1648,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
   stamp(a, 16);
 }
 
-template <int G>
-size_t attend_smem_bytes() {
-  return 32768 + G * 256 + kWarps * G * 4 + 256 + 4 * G * kHeadDim * 4;
-}
 
 }  // namespace
 
@@ -1417,7 +1668,9 @@ FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) 
     if (f >= 1 && f <= 16) c = f;
   }
   pl.cluster = c;
-  const size_t persistent = (size_t)persistent_bytes(g, pl.sel_words);
+  pl.pt_smem = max_pages <= 8192;
+  const size_t persistent = (size_t)persistent_bytes(g, pl.sel_words) +
+                            (pl.pt_smem ? ((size_t)4 * max_pages + 127) / 128 * 128 : 0);
   size_t scratch = 0;
   switch (g) {
     case 1: scratch = attend_smem_bytes<1>(); break;
@@ -1430,10 +1683,14 @@ FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) 
   size_t want = scratch;
   const size_t topk_need = 1280 + (size_t)4 * max_pages + 4 * kWarps * 512 + 2048;
   want = want > topk_need ? want : topk_need;
+  const size_t local_need = scratch + (size_t)10 * max_pages + 64;
+  want = want > local_need ? want : local_need;
   const size_t prune_need = 1024 + (size_t)4 * pl.cand_stride + 4 * 32 * 8 + 64;
   want = want > prune_need ? want : prune_need;
   want = want > (size_t)2 * pl.union_stride / 16 + 16 ? want : (size_t)2 * pl.union_stride / 16 + 16;
-  if (persistent + want > cap) want = cap - persistent;
+  // the bulk-copy chunks of the scoring and estimate phases take whatever is left: ask for the
+  // full capacity (one CTA per SM in any case)
+  want = cap - persistent;
   pl.smem_bytes = (int)(persistent + want);
   pl.ok = persistent + scratch <= cap && persistent + (size_t)2 * max_pages <= cap;
   return pl;
@@ -1486,13 +1743,17 @@ cudaError_t launch_fused(const FusedArgs& a, const FusedPlan& pl, cudaStream_t s
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = (size_t)pl.smem_bytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)pl.cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: this grid may be scheduled while the previous kernel in the
+  // stream finishes; it waits for that kernel (griddepcontrol.wait) before touching memory
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
 #define TWL_FUSED(G)                                                                            \
   do {                                                                                          \
     cudaError_t e = cudaFuncSetAttribute(k_decode_fused<G>,                                     \

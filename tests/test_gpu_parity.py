@@ -299,6 +299,23 @@ def test_decode_step_vs_oracle(small):
     assert layer.status()[0] == twl.TWL_OK
 
 
+def test_decode_step_without_stats_attends_locally(small):
+    # without stats each CTA attends over its own kept rows (no ordered union list); the output
+    # must match the stats run up to summation order, and the oracle over the same union
+    wl, layer = small
+    st, o1, lse1 = _run_step(wl, layer)
+    q = torch.from_numpy(wl.q).to(layer.device)
+    o2, lse2 = layer.decode(q, wl.p, wl.eps, None)
+    o2, lse2 = np_(o2), np_(lse2)
+    assert np.abs(o2 - o1).max() <= 2e-4 and np.abs(lse2 - lse1).max() <= 2e-4
+    for bb in range(wl.batch):
+        for kvh in range(wl.num_kv_heads):
+            uc = int(st["union_count"][bb, kvh])
+            att = O.group_attention(wl, {(bb, kvh): st["union_tok"][bb, kvh, :uc]})
+            for (b2, h), (o_or, lse_or) in att.items():
+                check_attention(o2[b2, h], lse2[b2, h], o_or, lse_or, f"{wl.name} b{b2} h{h}")
+
+
 def test_decode_step_deterministic(small):
     wl, layer = small
     a = _run_step(wl, layer)
@@ -319,7 +336,9 @@ def test_decode_step_equals_staged_calls(small):
     for bb in range(wl.batch):
         for h in range(wl.num_q_heads):
             c = ccn[bb, h]
-            assert np.allclose(wn[bb, h, :c], st["weights"][bb, h, :c], rtol=1e-5, atol=1e-12)
+            # two fp32 logit computations that differ in accumulation order (both are checked
+            # against the oracle at 1e-3): large logits (~270) move W by ~3e-5 relative
+            assert np.allclose(wn[bb, h, :c], st["weights"][bb, h, :c], rtol=5e-4, atol=1e-9)
     dev = layer.device
     stride = 16 * wl.max_pages
     o2 = torch.zeros((wl.batch, wl.num_q_heads, 128), device=dev)
