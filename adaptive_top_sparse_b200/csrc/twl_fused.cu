@@ -334,17 +334,30 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
   stamp(a, 23);
   auto key_at = [&](int i) -> uint32_t { return staged ? keys[i] : f32_key(ldcg_f(row + i)); };
 
-  // Where to start narrowing.  A sample of 256 keys (every n/256-th page), sorted by one warp,
-  // brackets the k-th largest key between the sample's ranks r* - 16 and r* + 16
-  // (r* = k * 256 / n); when the keys above and inside the common-prefix block of that bracket
-  // confirm it (above < k <= above + inside), narrowing starts from that block.  Otherwise it
-  // starts from the common prefix of the smallest and largest key.
-  uint32_t prefix = 0u, mask = 0u;
+  // The k-th largest key is narrowed down to a key interval [blo, bhi] holding `cand` keys, of
+  // which the `remaining` largest are selected (every key above bhi is selected).  Each pass
+  // histograms the keys inside the interval into up to 1024 bins of equal key width (the keys'
+  // offsets from blo, shifted right) and keeps the bin holding the k-th key.
+  //
+  // Start: a sample of 256 keys (every n/256-th page), sorted by one warp, brackets the k-th key
+  // between the sample's ranks r* - 16 and r* + 16 (r* = k * 256 / n).  The first pass also counts
+  // the keys above the bracket; when the count confirms the bracket (above < k <= above +
+  // inside) narrowing goes on from the bin found, otherwise it restarts from [min key, max key].
+  constexpr int kGatherCap = 64;
+  uint32_t* bhist = reinterpret_cast<uint32_t*>(sm.scratch + 1280 + 4 * n_pages);  // [1024]
+  uint32_t* gkey = bhist + 1024;                                                   // [cap]
+  int* gidx = reinterpret_cast<int*>(gkey + kGatherCap);                           // [cap]
+  uint32_t* sbits = reinterpret_cast<uint32_t*>(gidx + kGatherCap);                // [nw]
+  const bool room = staged && 1280 + 4 * (size_t)n_pages + 4 * 1024 + 8 * kGatherCap + 4 * nw +
+                                  16 <= (size_t)sm.scratch_bytes;
+  uint32_t* hh = room ? bhist : hist;  // the 256-bin histogram when there is no room
+  const int nbins = room ? 1024 : 256;
+  const int bin_bits = room ? 10 : 8;
+  uint32_t blo = 0u, bhi = 0xFFFFFFFFu;
   int remaining = kb;
-  int hi_bit = 31;
   int cand = n_pages;
-  bool bracketed = false;
-  if (staged && n_pages > 512) {
+  bool need_above = false;
+  if (room && n_pages > 512) {
     if (warp == 0) {
       uint32_t v[8];
 #pragma unroll
@@ -354,31 +367,12 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
       for (int i = 0; i < 8; ++i) hist[i * 32 + lane] = v[i];
     }
     __syncthreads();
+    stamp(a, 17);
     const int rstar = (int)((long)kb * 256 / n_pages);
-    const uint32_t hi_key = rstar - 16 >= 0 ? hist[rstar - 16] : 0xFFFFFFFFu;
-    const uint32_t lo_key = rstar + 16 <= 255 ? hist[rstar + 16] : 0u;
-    const uint32_t d = lo_key ^ hi_key;
-    const int hb = d ? 31 - __clz(d) : -1;
-    const uint32_t bmask = hb >= 31 ? 0u : (hb < 0 ? 0xFFFFFFFFu : ~((2u << hb) - 1u));
-    const uint32_t bpre = hi_key & bmask;
-    int packed = 0;  // above * 65536 + inside (n <= 32768)
-    for (int i = tid; i < n_pages; i += kThreads) {
-      const uint32_t k = keys[i] & bmask;
-      packed += (k > bpre ? 65536 : 0) + (k == bpre ? 1 : 0);
-    }
-    int tot;
-    block_exclusive_scan(packed, scan_sh, &tot);
-    const int above = tot >> 16, inside = tot & 0xFFFF;
-    if (above < kb && kb <= above + inside) {
-      prefix = bpre;
-      mask = bmask;
-      remaining = kb - above;
-      cand = inside;
-      hi_bit = hb;
-      bracketed = true;
-    }
-  }
-  if (!bracketed) {
+    bhi = rstar - 16 >= 0 ? hist[rstar - 16] : 0xFFFFFFFFu;
+    blo = rstar + 16 <= 255 ? hist[rstar + 16] : 0u;
+    need_above = true;
+  } else {
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
     for (int i = tid; i < n_pages; i += kThreads) {
       const uint32_t k = key_at(i);
@@ -387,7 +381,6 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
     }
     kmin = __reduce_min_sync(0xffffffffu, kmin);
     kmax = __reduce_max_sync(0xffffffffu, kmax);
-    __syncthreads();
     if (lane == 0) {
       hist[2 * warp] = kmin;
       hist[2 * warp + 1] = kmax;
@@ -400,101 +393,109 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
       kmin = min(kmin, hist[2 * w]);
       kmax = max(kmax, hist[2 * w + 1]);
     }
-    const uint32_t diff = kmin ^ kmax;
-    hi_bit = diff ? 31 - __clz(diff) : -1;
-    mask = hi_bit >= 31 ? 0u : ~((2u << hi_bit) - 1u);
-    if (hi_bit < 0) mask = 0xFFFFFFFFu;
-    prefix = kmax & mask;
-    remaining = kb;
-    cand = n_pages;
+    blo = kmin;
+    bhi = kmax;
   }
   __syncthreads();
-  // Narrow the candidate bin with histogram passes over the next (up to) 10 bits of the keys
-  // that still match the prefix, until it holds at most kGatherCap keys; every key above the bin
-  // is selected, and the bin's keys are ranked exactly by (key desc, page asc).  Only when all
-  // bits are resolved and more than kGatherCap keys are exactly equal does the ordered ballot
-  // path below take the first ones by page index.
-  constexpr int kGatherCap = 64;
-  uint32_t* bhist = reinterpret_cast<uint32_t*>(sm.scratch + 1280 + 4 * n_pages);  // [1024]
-  uint32_t* gkey = bhist + 1024;                                                   // [cap]
-  int* gidx = reinterpret_cast<int*>(gkey + kGatherCap);                           // [cap]
-  uint32_t* sbits = reinterpret_cast<uint32_t*>(gidx + kGatherCap);                // [nw]
-  const bool room = staged && 1280 + 4 * (size_t)n_pages + 4 * 1024 + 8 * kGatherCap + 4 * nw +
-                                  16 <= (size_t)sm.scratch_bytes;
-  uint32_t* hh = room ? bhist : hist;  // the 256-bin histogram when there is no room
-  const int max_dw = room ? 10 : 8;
   const int n_it = (n_pages + kThreads - 1) / kThreads;
 #pragma unroll 1
-  while ((cand > kGatherCap || !room) && hi_bit >= 0) {
-    const int dwb = hi_bit + 1 < max_dw ? hi_bit + 1 : max_dw;
-    const int lo_b = hi_bit - dwb + 1;
-    const int nbb = 1 << dwb;
-    const uint32_t dmb = (uint32_t)nbb - 1u;
-    for (int i = tid; i < nbb; i += kThreads) hh[i] = 0u;
+  while (need_above || ((cand > kGatherCap || !room) && blo < bhi)) {
+    const uint32_t range = bhi - blo;
+    const int width = range ? 32 - __clz(range) : 0;
+    const int sh = width > bin_bits ? width - bin_bits : 0;
+    for (int i = tid; i < nbins; i += kThreads) hh[i] = 0u;
     __syncthreads();
+    int above = 0;
 #pragma unroll 1
     for (int it = 0; it < n_it; ++it) {
       const int i = it * kThreads + tid;
-      bool take = false;
-      uint32_t digit = 0;
       if (i < n_pages) {
         const uint32_t key = key_at(i);
-        take = (key & mask) == prefix;
-        digit = (key >> lo_b) & dmb;
+        above += need_above && key > bhi ? 1 : 0;
+        if (key >= blo && key <= bhi) atomicAdd(&hh[(key - blo) >> sh], 1u);
       }
-      const uint32_t peers = __match_any_sync(0xffffffffu, take ? digit : 2048u + lane);
-      if (take && (__ffs(peers) - 1) == lane) atomicAdd(&hh[digit], (uint32_t)__popc(peers));
     }
     __syncthreads();
-    if (warp == 0) {
-      const int per = (nbb + 31) / 32;
-      uint32_t lsum = 0;
-      for (int e = 0; e < per; ++e) {
-        const int bin = nbb - 1 - lane * per - e;
-        if (bin >= 0) lsum += hh[bin];
+    // descending scan over the bins, two per thread; the keys above the interval ride in the
+    // upper 16 bits (n_pages < 65536)
+    const int b0 = nbins - 1 - 2 * tid, b1 = b0 - 1;
+    const uint32_t c0 = b0 >= 0 ? hh[b0] : 0u, c1 = b1 >= 0 ? hh[b1] : 0u;
+    int tot;
+    const int ex = block_exclusive_scan((int)(((uint32_t)above << 16) | (c0 + c1)), scan_sh, &tot);
+    const int excl = ex & 0xFFFF;
+    int base_rank = 0;  // keys above the interval that `remaining` does not yet exclude
+    bool restart = false;
+    if (need_above) {
+      base_rank = tot >> 16;
+      const int inside = tot & 0xFFFF;
+      restart = !(base_rank < kb && kb <= base_rank + inside);
+    }
+    const int want = remaining - base_rank;
+    if (!restart) {
+      if (excl < want && want <= excl + (int)c0) {
+        state[0] = (uint32_t)b0;
+        state[1] = (uint32_t)(want - excl);
+        state[2] = c0;
+      } else if (excl + (int)c0 < want && want <= excl + (int)(c0 + c1)) {
+        state[0] = (uint32_t)b1;
+        state[1] = (uint32_t)(want - excl - (int)c0);
+        state[2] = c1;
       }
-      uint32_t incl = lsum;
+    }
+    __syncthreads();
+    if (restart) {
+      // the sample's bracket missed the k-th key: start again from the whole key range
+      uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+      for (int i = tid; i < n_pages; i += kThreads) {
+        const uint32_t k = key_at(i);
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+      }
+      kmin = __reduce_min_sync(0xffffffffu, kmin);
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      if (lane == 0) {
+        hist[2 * warp] = kmin;
+        hist[2 * warp + 1] = kmax;
+      }
+      __syncthreads();
+      kmin = 0xFFFFFFFFu;
+      kmax = 0u;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+      for (int w = 0; w < kWarps; ++w) {
+        kmin = min(kmin, hist[2 * w]);
+        kmax = max(kmax, hist[2 * w + 1]);
       }
-      const uint32_t excl = incl - lsum;
-      if (excl < (uint32_t)remaining && incl >= (uint32_t)remaining) {
-        uint32_t run = excl;
-        for (int e = 0; e < per; ++e) {
-          const int bin = nbb - 1 - lane * per - e;
-          if (bin < 0) break;
-          const uint32_t c = hh[bin];
-          if (run + c >= (uint32_t)remaining) {
-            state[0] = (uint32_t)bin;
-            state[1] = (uint32_t)remaining - run;
-            state[2] = c;
-            break;
-          }
-          run += c;
-        }
-      }
+      blo = kmin;
+      bhi = kmax;
+      remaining = kb;
+      cand = n_pages;
+    } else {
+      const uint32_t bin = state[0];
+      const uint32_t nlo = blo + (bin << sh);
+      const uint64_t top = (uint64_t)nlo + ((1ull << sh) - 1ull);
+      bhi = top < (uint64_t)bhi ? (uint32_t)top : bhi;
+      blo = nlo;
+      remaining = (int)state[1];
+      cand = (int)state[2];
     }
-    __syncthreads();
-    prefix |= state[0] << lo_b;
-    mask |= dmb << lo_b;
-    remaining = (int)state[1];
-    cand = (int)state[2];
-    hi_bit = lo_b - 1;
+    need_above = false;
     __syncthreads();
   }
+  stamp(a, 19);
   if (room && cand <= kGatherCap) {
     for (int w = tid; w < nw; w += kThreads) sbits[w] = 0u;
     // ordered gather of the bin's keys: thread t scans a contiguous range of pages
     const int per = (n_pages + kThreads - 1) / kThreads;
     const int beg = min(n_pages, tid * per), end = min(n_pages, beg + per);
     int mine = 0;
-    for (int i = beg; i < end; ++i) mine += (key_at(i) & mask) == prefix;
+    for (int i = beg; i < end; ++i) {
+      const uint32_t key = key_at(i);
+      mine += key >= blo && key <= bhi;
+    }
     int slot = block_exclusive_scan(mine, scan_sh, nullptr);
     for (int i = beg; i < end && mine > 0; ++i) {
       const uint32_t key = key_at(i);
-      if ((key & mask) == prefix) {
+      if (key >= blo && key <= bhi) {
         gkey[slot] = key;
         gidx[slot] = i;
         ++slot;
@@ -502,6 +503,7 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
       }
     }
     __syncthreads();
+    stamp(a, 20);
     for (int e = tid; e < cand; e += kThreads) {
       const uint32_t ke = gkey[e];
       const int ie = gidx[e];
@@ -513,9 +515,10 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
       if (rank < remaining) atomicOr(&sbits[ie >> 5], 1u << (ie & 31));
     }
     __syncthreads();
+    stamp(a, 21);
     for (int base = 0; base < 32 * nw; base += kThreads) {
       const int i = base + tid;
-      const bool above = i < n_pages && (key_at(i) & mask) > prefix;
+      const bool above = i < n_pages && key_at(i) > bhi;
       const uint32_t bal = __ballot_sync(0xffffffffu, above);
       if (lane == 0 && (i >> 5) < nw) sbits[i >> 5] |= bal;
     }
@@ -539,7 +542,8 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
     if (tid == 0 && a.sel_count) a.sel_count[bh] = kb;
     return;
   }
-  // all bits resolved (or no room for the gather): prefix is the k-th key itself
+  // the interval is down to one key (or there is no room for the gather): blo == bhi is the
+  // k-th key itself
   stamp(a, 24);
   // Keys above the k-th are taken; equal keys are taken in ascending page order.  One element
   // per thread per round; a warp's ballot is one 32-page word of the bitmap.
@@ -550,8 +554,8 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
     const int i = base + tid;
     const bool in = i < n_pages;
     const uint32_t key = in ? key_at(i) : 0u;
-    const uint32_t gt = __ballot_sync(0xffffffffu, in && key > prefix);
-    const uint32_t eq = __ballot_sync(0xffffffffu, in && key == prefix);
+    const uint32_t gt = __ballot_sync(0xffffffffu, in && key > bhi);
+    const uint32_t eq = __ballot_sync(0xffffffffu, in && key == blo);
     if (lane == 0) wsum[warp] = __popc(eq);
     __syncthreads();
     int eq_before = carry_eq, eq_round = 0;
@@ -559,7 +563,7 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
       if (w < warp) eq_before += wsum[w];
       eq_round += wsum[w];
     }
-    const bool take = in && key == prefix && eq_before + __popc(eq & lt) < remaining;
+    const bool take = in && key == blo && eq_before + __popc(eq & lt) < remaining;
     const uint32_t sel = gt | __ballot_sync(0xffffffffu, take);
     __syncthreads();
     if (lane == 0) wsum[warp] = __popc(sel);
@@ -683,8 +687,7 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
       pph[i] = phys_of(a, sm, b, j);
     }
     __syncthreads();
-    stamp(a, 25);
-    // 68 chunks of 16 bytes per page (64 of nibbles, 4 of scale/zero), spread over all threads
+      // 68 chunks of 16 bytes per page (64 of nibbles, 4 of scale/zero), spread over all threads
     for (int c = threadIdx.x; c < 68 * cn; c += kThreads) {
       const int i = c / 68, k = c - 68 * i;
       const int ph = pph[i];
@@ -697,8 +700,7 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
     cp_async_commit();
     cp_async_wait_all();
     __syncthreads();
-    stamp(a, 26);
-    const bool ok = true;
+      const bool ok = true;
     // two pages per warp iteration: their mma chains and epilogues are independent
 #pragma unroll 1
     for (int i0 = 2 * warp; i0 < cn; i0 += 2 * kWarps) {
@@ -774,8 +776,7 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
       }
     }
     __syncthreads();  // the chunk's tiles are read before the next copies land
-    stamp(a, 27);
-  }
+    }
   // combine the maxima over the 8 row-lanes of each head, then over the warps
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
@@ -836,7 +837,6 @@ __device__ void phase_prune_head(const FusedArgs& a, int gi, int hl, int G, int 
 #pragma unroll
   for (int rr = 0; rr < 16; ++rr) M = fmaxf(M, pmv[rr]);
   const bool empty = !(M > -INFINITY);
-  stamp(a, 17);
   float* lrow = a.logits + (size_t)bh * a.cand_stride;
   float* E = staged ? wbuf : lrow;
   // pass 1: e = exp(l - M) and its block sum
@@ -873,7 +873,6 @@ __device__ void phase_prune_head(const FusedArgs& a, int gi, int hl, int G, int 
     top = fmaxf(top, wv);
   }
   const float* W = E;
-  stamp(a, 18);
   top = warp_max(top);
   __syncthreads();
   if (lane == 0) red[warp] = top;
@@ -885,7 +884,6 @@ __device__ void phase_prune_head(const FusedArgs& a, int gi, int hl, int G, int 
     top = t;
   }
   const float p = a.p, eps = a.eps;
-  stamp(a, 19);
   // Decisions at thresholds t <= L = (1 - p) / (2 nc) need no mass: the weights below t sum to
   // less than nc * t <= (1 - p) / 2, so mass(W >= t) > 1 - (1 - p) / 2 >= p (with margin for fp32
   // sums, hence the 1e-3 guard).  Above L only weights >= L can count, so the search runs on the
@@ -1110,79 +1108,69 @@ __device__ void phase_prune_head(const FusedArgs& a, int gi, int hl, int G, int 
   }
   }
   const float m = ctl[11];
-  stamp(a, 21);
 #ifdef TWL_PHASE_TIMING
   if (blockIdx.x == 0 && threadIdx.x == 0 && a.flags) a.flags[2] = rounds;
 #endif
   (void)rounds;
-  // publish what every CTA needs to decide kept rows from its own logits: W = exp(l - M) * inv
-  // (the same two operations as above, so the same bits) and the threshold m
   if (tid == 0) {
-    float* hp = a.head_par + (size_t)bh * 4;
-    hp[0] = M;
-    hp[1] = inv;
-    hp[2] = m;
     if (a.threshold) a.threshold[bh] = m;
     if (a.cand_count) a.cand_count[bh] = nc;
   }
+  // kept-row bitmap of this head: bit i = (W_i >= m), one 32-row word per warp ballot
+  uint32_t* kb_out = a.keptbits + (size_t)bh * a.kept_words;
+  int cnt = 0;
+#pragma unroll 1
+  for (int base = 0; base < nc; base += kThreads) {
+    const int i = base + tid;
+    const bool keep = i < nc && (staged ? W[i] : ldcg_f(W + i)) >= m;
+    const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0 && base + 32 * warp < nc) kb_out[(base >> 5) + warp] = bal;
+    cnt += keep;
+  }
   if (a.kept_count) {  // only when the caller asks for it
-    int cnt = 0;
-    for (int i = tid; i < nc; i += kThreads) cnt += (staged ? W[i] : ldcg_f(W + i)) >= m;
     const float total = block_sum_fixed((float)cnt, red);
     if (tid == 0) a.kept_count[bh] = (int)total;
   }
-  stamp(a, 22);
 }
 
 // ------------------------------------------------------------------------- phase 6: kept union
 // Per page of this CTA's union share: 16-bit mask of rows kept by any head of the group.
+// The kept rows of union page j: the OR over the group's heads that selected j of their 16-row
+// pieces of the kept-row bitmaps (the candidate rows of a head are its selected pages' rows in
+// ascending page order), cut to the page's valid rows.
+template <int G>
+__device__ __forceinline__ uint32_t union_row_mask(const FusedArgs& a, int b, int kvh, int n, int j,
+                                                   const Smem& sm) {
+  const int nw = sm.nw;
+  uint32_t words[G];
+  int shift[G];
+#pragma unroll
+  for (int hl = 0; hl < G; ++hl) {  // every head's word in flight before combining
+    const uint32_t* hb = sm.hbits + hl * nw;
+    words[hl] = 0u;
+    shift[hl] = 0;
+    if ((hb[j >> 5] >> (j & 31)) & 1u) {
+      const int rk = rank_in(hb, sm.hpre + hl * nw, j);
+      words[hl] = ldcg_u(a.keptbits + (size_t)(b * a.hq + kvh * G + hl) * a.kept_words + (rk >> 1));
+      shift[hl] = 16 * (rk & 1);
+    }
+  }
+  uint32_t m = 0;
+#pragma unroll
+  for (int hl = 0; hl < G; ++hl) m |= (words[hl] >> shift[hl]) & 0xFFFFu;
+  const int rows = page_rows(n, j);
+  return m & (rows >= 16 ? 0xFFFFu : ((1u << rows) - 1u));
+}
+
 template <int G>
 __device__ int phase_kept_rows(const FusedArgs& a, int b, int kvh, int n, int U, int r, int C,
                                Smem& sm, uint16_t* rowmask, int* scan_sh) {
   const int tid = threadIdx.x, nw = sm.nw;
   const int u0 = (int)((long)U * r / C), u1 = (int)((long)U * (r + 1) / C);
-  float hM[G], hinv[G], hm[G];
-#pragma unroll
-  for (int hl = 0; hl < G; ++hl) {
-    const float* hp = a.head_par + (size_t)(b * a.hq + kvh * G + hl) * 4;
-    hM[hl] = ldcg_f(hp);
-    hinv[hl] = ldcg_f(hp + 1);
-    hm[hl] = ldcg_f(hp + 2);
-  }
   int cnt = 0;
   for (int u = u0 + tid; u < u1; u += kThreads) {
     const int j = union_select(sm.ubits, sm.upre, nw, u);
-    float4 lg[G][4];
-    bool sel[G];
-#pragma unroll
-    for (int hl = 0; hl < G; ++hl) {  // every head's 16 logits in flight before deciding
-      const uint32_t* hb = sm.hbits + hl * nw;
-      sel[hl] = (hb[j >> 5] >> (j & 31)) & 1u;
-      if (sel[hl]) {
-        const int rk = rank_in(hb, sm.hpre + hl * nw, j);
-        const float4* src = reinterpret_cast<const float4*>(
-            a.logits + (size_t)(b * a.hq + kvh * G + hl) * a.cand_stride + (size_t)rk * kPage);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) lg[hl][q4] = __ldcg(src + q4);
-      }
-    }
-    uint32_t m = 0;
-#pragma unroll
-    for (int hl = 0; hl < G; ++hl) {
-      if (!sel[hl]) continue;
-      const bool live = hM[hl] > -INFINITY;
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const float l4[4] = {lg[hl][q4].x, lg[hl][q4].y, lg[hl][q4].z, lg[hl][q4].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float w = live ? __expf(l4[e] - hM[hl]) * hinv[hl] : 0.f;
-          m |= (w >= hm[hl] ? 1u : 0u) << (4 * q4 + e);
-        }
-      }
-    }
-    const int rows = page_rows(n, j);
-    m &= rows >= 16 ? 0xFFFFu : ((1u << rows) - 1u);
+    const uint32_t m = union_row_mask<G>(a, b, kvh, n, j, sm);
     rowmask[u - u0] = (uint16_t)m;
     cnt += __popc(m);
   }
@@ -1200,14 +1188,7 @@ __device__ int phase_kept_rows_local(const FusedArgs& a, int b, int kvh, int n, 
                                      int* scan_sh) {
   const int tid = threadIdx.x, nw = sm.nw;
   const int u0 = (int)((long)U * r / C), u1 = (int)((long)U * (r + 1) / C);
-  float hM[G], hinv[G], hm[G];
-#pragma unroll
-  for (int hl = 0; hl < G; ++hl) {
-    const float* hp = a.head_par + (size_t)(b * a.hq + kvh * G + hl) * 4;
-    hM[hl] = ldcg_f(hp);
-    hinv[hl] = ldcg_f(hp + 1);
-    hm[hl] = ldcg_f(hp + 2);
-  }
+  stamp(a, 27);
   int carry = 0;
 #pragma unroll 1
   for (int ub = u0; ub < u1; ub += kThreads) {
@@ -1215,42 +1196,14 @@ __device__ int phase_kept_rows_local(const FusedArgs& a, int b, int kvh, int n, 
     uint32_t m = 0;
     if (u < u1) {
       const int j = union_select(sm.ubits, sm.upre, nw, u);
-      const int ph = phys_of(a, sm, b, j);
-      float4 lg[G][4];
-      bool sel[G];
-#pragma unroll
-      for (int hl = 0; hl < G; ++hl) {
-        const uint32_t* hb = sm.hbits + hl * nw;
-        sel[hl] = (hb[j >> 5] >> (j & 31)) & 1u;
-        if (sel[hl]) {
-          const int rk = rank_in(hb, sm.hpre + hl * nw, j);
-          const float4* src = reinterpret_cast<const float4*>(
-              a.logits + (size_t)(b * a.hq + kvh * G + hl) * a.cand_stride + (size_t)rk * kPage);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) lg[hl][q4] = __ldcg(src + q4);
-        }
-      }
-#pragma unroll
-      for (int hl = 0; hl < G; ++hl) {
-        if (!sel[hl]) continue;
-        const bool live = hM[hl] > -INFINITY;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const float l4[4] = {lg[hl][q4].x, lg[hl][q4].y, lg[hl][q4].z, lg[hl][q4].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float w = live ? __expf(l4[e] - hM[hl]) * hinv[hl] : 0.f;
-            m |= (w >= hm[hl] ? 1u : 0u) << (4 * q4 + e);
-          }
-        }
-      }
-      const int rows = page_rows(n, j);
-      m &= rows >= 16 ? 0xFFFFu : ((1u << rows) - 1u);
+      pph[u - u0] = phys_of(a, sm, b, j);
+      m = union_row_mask<G>(a, b, kvh, n, j, sm);
       rowmask[u - u0] = (uint16_t)m;
-      pph[u - u0] = ph;
     }
+    stamp(a, 25);
     int total;
     const int ex = block_exclusive_scan(__popc(m), scan_sh, &total);
+    stamp(a, 26);
     if (u < u1) pfx[u - u0] = carry + ex;
     carry += total;
   }
@@ -1706,11 +1659,11 @@ size_t fused_workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_
   add(bh * max_pages * 4);                    // scores
   add(bh * pl.sel_words * 4);                 // selected-page bitmaps
   add(bh * (size_t)pl.cand_stride * 4);       // logits / weights
-  add(bh * 4 * 4);                            // per-head (max, 1/sum, threshold)
   add(groups * 16 * g * 2 * 4);               // partial (max, sum)
   add(groups * 16 * 4);                       // union counts per CTA
   add(groups * (size_t)pl.union_stride * 4);  // union token lists
   add(groups * 16 * g * (kHeadDim + 2) * 4);  // attention partials
+  add(bh * (size_t)((pl.cand_stride + 31) / 32) * 4);  // kept-row bitmaps
   return s;
 }
 
@@ -1727,12 +1680,13 @@ void carve_fused(FusedArgs& a, char* ws, const FusedPlan& pl, int batch, int hq,
   a.scores = reinterpret_cast<float*>(take(bh * max_pages * 4));
   a.selbits = reinterpret_cast<uint32_t*>(take(bh * pl.sel_words * 4));
   a.logits = reinterpret_cast<float*>(take(bh * (size_t)pl.cand_stride * 4));
-  a.head_par = reinterpret_cast<float*>(take(bh * 4 * 4));
   a.part_ms = reinterpret_cast<float*>(take(groups * 16 * g * 2 * 4));
   a.union_part = reinterpret_cast<int*>(take(groups * 16 * 4));
   int* ulist = reinterpret_cast<int*>(take(groups * (size_t)pl.union_stride * 4));
   if (!a.union_tok) a.union_tok = ulist;
   a.part_att = reinterpret_cast<float*>(take(groups * 16 * g * (kHeadDim + 2) * 4));
+  a.kept_words = (pl.cand_stride + 31) / 32;
+  a.keptbits = reinterpret_cast<uint32_t*>(take(bh * (size_t)a.kept_words * 4));
 }
 
 cudaError_t launch_fused(const FusedArgs& a, const FusedPlan& pl, cudaStream_t s) {

@@ -38,13 +38,13 @@ struct FusedArgs {
   float* scores;
   uint32_t* selbits;
   float* logits;
-  float* head_par;  // [B * Hq][4]: max logit, 1 / sum of exp, top-p threshold
+  uint32_t* keptbits;  // [B * Hq][kept_words]: bit i = candidate row i passes top-p
   float* part_ms;
   int* union_part;
   float* part_att;
   uint32_t* flags;
   // strides and launch shape
-  int sel_words, cand_stride, union_stride;
+  int sel_words, cand_stride, union_stride, kept_words;
   int cluster;
   int smem_bytes;
 };
