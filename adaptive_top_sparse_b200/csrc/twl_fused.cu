@@ -53,6 +53,25 @@ __device__ __forceinline__ uint32_t cluster_size() {
   return n;
 }
 
+// Distributed shared memory: a CTA's shared address mapped into cluster CTA `rank`, and stores /
+// atomics through such an address.  Ordered for the target CTA by the next cluster barrier
+// (arrive has release, wait has acquire semantics).
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint32_t map_rank(uint32_t addr, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+// Exchange slots (shared memory, written by the other CTAs of the cluster): one per head that the
+// CTA owns (heads r, r + C, ...), holding the C per-CTA maxima of the head's logits.
+constexpr int kXchgSlot = 64;                // [16] floats
+constexpr int kXchgBytes = 8 * kXchgSlot;    // up to 8 owned heads
+
 // Optional phase timestamps (compile with -DTWL_PHASE_TIMING): thread 0 of the first CTA of the
 // first cluster records %globaltimer at each phase boundary into the workspace header (words
 // 8..63 as 64-bit values; word 1 = the cluster size launched).  Off by default.
@@ -122,8 +141,11 @@ __device__ __forceinline__ uint32_t nib_pair(uint32_t x, int i) {
 
 // Bytes of the persistent bitmap region, rounded up so the scratch region after it is 128-byte
 // aligned (the attention phase does 16-byte vector and cp.async accesses into it).
-__host__ __device__ constexpr int persistent_bytes(int g, int sel_words) {
+__host__ __device__ constexpr int bitmap_bytes(int g, int sel_words) {
   return ((4 * (2 * g + 2) * sel_words) + 127) & ~127;
+}
+__host__ __device__ constexpr int persistent_bytes(int g, int sel_words) {
+  return bitmap_bytes(g, sel_words) + kXchgBytes;
 }
 
 // Shared-memory layout: a persistent region for the page bitmaps (phases 3-6) and one scratch
@@ -134,6 +156,7 @@ struct Smem {
   int* hpre;        // [G][nw]  exclusive prefix popcounts per word
   uint32_t* ubits;  // [nw]     union bitmap
   int* upre;        // [nw]     exclusive prefix popcounts of the union
+  unsigned char* xchg;  // exchange slots of the heads this CTA owns
   unsigned char* scratch;
   int scratch_bytes;
   int nw;
@@ -203,6 +226,7 @@ __device__ void phase_scores(const FusedArgs& a, int b, int kvh, int n_pages, in
     for (int i = threadIdx.x; i < cn; i += kThreads)
       phys[i] = phys_of(a, sm, b, c0 + i);
     __syncthreads();
+    if (c0 == p0) stamp(a, 17);
     // 32 chunks of 16 bytes per page, spread over all threads, all in flight together
     for (int c = threadIdx.x; c < 32 * cn; c += kThreads) {
       const int i = c >> 5, k = c & 31;
@@ -214,6 +238,7 @@ __device__ void phase_scores(const FusedArgs& a, int b, int kvh, int n_pages, in
     cp_async_commit();
     cp_async_wait_all();
     __syncthreads();
+    if (c0 == p0) stamp(a, 18);
     const bool ok = true;
     for (int base = 0; base < cn; base += 2 * kWarps) {  // warp-uniform trip count
       const int i0 = base + 2 * warp + half;
@@ -331,7 +356,6 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
     }
   }
   __syncthreads();
-  stamp(a, 23);
   auto key_at = [&](int i) -> uint32_t { return staged ? keys[i] : f32_key(ldcg_f(row + i)); };
 
   // The k-th largest key is narrowed down to a key interval [blo, bhi] holding `cand` keys, of
@@ -367,7 +391,6 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
       for (int i = 0; i < 8; ++i) hist[i * 32 + lane] = v[i];
     }
     __syncthreads();
-    stamp(a, 17);
     const int rstar = (int)((long)kb * 256 / n_pages);
     bhi = rstar - 16 >= 0 ? hist[rstar - 16] : 0xFFFFFFFFu;
     blo = rstar + 16 <= 255 ? hist[rstar + 16] : 0u;
@@ -481,7 +504,6 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
     need_above = false;
     __syncthreads();
   }
-  stamp(a, 19);
   if (room && cand <= kGatherCap) {
     for (int w = tid; w < nw; w += kThreads) sbits[w] = 0u;
     // ordered gather of the bin's keys: thread t scans a contiguous range of pages
@@ -503,7 +525,6 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
       }
     }
     __syncthreads();
-    stamp(a, 20);
     for (int e = tid; e < cand; e += kThreads) {
       const uint32_t ke = gkey[e];
       const int ie = gidx[e];
@@ -515,7 +536,6 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
       if (rank < remaining) atomicOr(&sbits[ie >> 5], 1u << (ie & 31));
     }
     __syncthreads();
-    stamp(a, 21);
     for (int base = 0; base < 32 * nw; base += kThreads) {
       const int i = base + tid;
       const bool above = i < n_pages && key_at(i) > bhi;
@@ -544,7 +564,6 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
   }
   // the interval is down to one key (or there is no room for the gather): blo == bhi is the
   // k-th key itself
-  stamp(a, 24);
   // Keys above the k-th are taken; equal keys are taken in ascending page order.  One element
   // per thread per round; a warp's ballot is one 32-page word of the bitmap.
   int* wsum = scan_sh;  // [kWarps] per-warp counts, then their prefix
@@ -653,8 +672,8 @@ __device__ void phase_union_bitmaps(const FusedArgs& a, int b, int kvh, Smem& sm
 // are staged (thread per page), then its INT4 tile (1 KB) and scale/zero row (64 B) are copied
 // into shared memory with 16-byte cp.async over all threads; one warp then computes a page.
 template <int G>
-__device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n, int U, int r,
-                               int C, Smem& sm) {
+__device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int n, int U, int r, int C,
+                               Smem& sm) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gr = lane >> 2, t = lane & 3;
   const int nw = sm.nw;
@@ -675,7 +694,7 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
   qs_part += __shfl_xor_sync(0xffffffffu, qs_part, 2);
   const float qsum0 = __shfl_sync(0xffffffffu, qs_part, (2 * t) * 4);
   const float qsum1 = __shfl_sync(0xffffffffu, qs_part, (2 * t + 1) * 4);
-  // running max of this lane's two heads over its rows (the softmax's shift)
+  // running max of this lane's two heads over its rows
   float rm[2] = {-INFINITY, -INFINITY};
 
 #pragma unroll 1
@@ -687,6 +706,7 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
       pph[i] = phys_of(a, sm, b, j);
     }
     __syncthreads();
+    if (c0 == u0) stamp(a, 25);
       // 68 chunks of 16 bytes per page (64 of nibbles, 4 of scale/zero), spread over all threads
     for (int c = threadIdx.x; c < 68 * cn; c += kThreads) {
       const int i = c / 68, k = c - 68 * i;
@@ -700,6 +720,7 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
     cp_async_commit();
     cp_async_wait_all();
     __syncthreads();
+    if (c0 == u0) stamp(a, 26);
       const bool ok = true;
     // two pages per warp iteration: their mma chains and epilogues are independent
 #pragma unroll 1
@@ -777,13 +798,15 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
     }
     __syncthreads();  // the chunk's tiles are read before the next copies land
     }
-  // combine the maxima over the 8 row-lanes of each head, then over the warps
+  stamp(a, 21);
+  // the CTA's max per head (over the 8 row-lanes of each head, then over the warps), pushed to
+  // the head's owner
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) rm[e] = fmaxf(rm[e], __shfl_xor_sync(0xffffffffu, rm[e], off));
+    for (int off = 4; off < 32; off <<= 1)
+      rm[e] = fmaxf(rm[e], __shfl_xor_sync(0xffffffffu, rm[e], off));
   }
-  __syncthreads();
   if (lane < 4) {
 #pragma unroll
     for (int e = 0; e < 2; ++e) red[warp * 8 + 2 * lane + e] = rm[e];
@@ -792,8 +815,9 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int gi, int n
   if (threadIdx.x < G) {
     const int hl = threadIdx.x;
     float m = -INFINITY;
+#pragma unroll
     for (int w = 0; w < kWarps; ++w) m = fmaxf(m, red[w * 8 + hl]);
-    a.part_ms[((size_t)gi * C * G + r * G + hl) * 2] = m;
+    st_cluster(map_rank(smem_addr(sm.xchg + (hl / C) * kXchgSlot + 4 * r), hl % C), m);
   }
 }
 
@@ -821,179 +845,68 @@ __device__ __forceinline__ float mid_of(float lo, float hi) {
   return __fadd_rn(lo, __fmul_rn(__fsub_rn(hi, lo), 0.5f));
 }
 
-__device__ void phase_prune_head(const FusedArgs& a, int gi, int hl, int G, int bh, int nc, int C,
-                                 Smem& sm) {
+// Weight in fixed point (units of 2^-48; W <= 1): integer sums are exact up to the conversion and
+// independent of the order of the terms, so the live-set masses do not depend on the order in
+// which the other CTAs pushed the entries.
+__device__ __forceinline__ long long w_fixed(float w) { return __float2ll_rn(w * 281474976710656.f); }
+
+// The search on (0, top]: lo = 0, hi = top; the midpoint test is "mid <= T" (see
+// top_p_from_live); stop when hi - lo <= eps, when the midpoint no longer splits, or after 64
+// steps; the threshold is lo (top when the test passes at top itself).
+__device__ __forceinline__ float bisect_scalar(float top, float T, float eps) {
+  if (top <= T) return top;
+  float lo = 0.f, hi = top;
+#pragma unroll 1
+  for (int steps = 0; steps < 64; ++steps) {
+    if (__fsub_rn(hi, lo) <= eps) break;
+    const float mid = mid_of(lo, hi);
+    if (!(lo < mid && mid < hi)) break;
+    if (mid <= T) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// Threshold from the live set {W >= L} (n <= kThreads values lw, fixed-point copies lq).  Every
+// test of the search at mid > L counts only live weights, and mass(W >= t) is a non-increasing
+// step function of t, so "mid <= L or mass(W >= mid) >= p" is the same test as "mid <= T" with
+// T = max(L, the largest live weight v with mass(W >= v) >= p).  T comes from all pairwise
+// comparisons at once (4, 2 or 1 threads per value); the search itself is then a scalar loop that
+// every thread runs (same inputs, same result).
+__device__ float top_p_from_live(const float* lw, const long long* lq, int n, float L, float p,
+                                 float eps, float top, float* red) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float* red = reinterpret_cast<float*>(sm.scratch);                  // [kWarps][8]
-  float* ctl = reinterpret_cast<float*>(sm.scratch + 4 * kWarps * 8);   // thresholds + state
-  float* wbuf = reinterpret_cast<float*>(sm.scratch + 1024);
-  const bool staged = 1024 + 4 * nc <= sm.scratch_bytes;
-  // the group-wide max of this head's logits: merge the C partial maxima (loads in flight together)
-  float pmv[16];
-#pragma unroll
-  for (int rr = 0; rr < 16; ++rr)
-    pmv[rr] = rr < C ? ldcg_f(a.part_ms + ((size_t)gi * C * G + rr * G + hl) * 2) : -INFINITY;
-  float M = -INFINITY;
-#pragma unroll
-  for (int rr = 0; rr < 16; ++rr) M = fmaxf(M, pmv[rr]);
-  const bool empty = !(M > -INFINITY);
-  float* lrow = a.logits + (size_t)bh * a.cand_stride;
-  float* E = staged ? wbuf : lrow;
-  // pass 1: e = exp(l - M) and its block sum
-  float esum = 0.f;
-  constexpr int kB = 8;
-#pragma unroll 1
-  for (int base = 0; base < nc; base += kThreads * kB) {
-    float v[kB];
-#pragma unroll
-    for (int k = 0; k < kB; ++k) {
-      const int i = base + k * kThreads + tid;
-      v[k] = i < nc ? ldcg_f(lrow + i) : -INFINITY;
-    }
-#pragma unroll
-    for (int k = 0; k < kB; ++k) {
-      const int i = base + k * kThreads + tid;
-      if (i < nc) {
-        const float e = empty ? 0.f : __expf(v[k] - M);
-        E[i] = e;
-        esum += e;
-      }
-    }
+  const long long P = __double2ll_ru((double)p * 281474976710656.0);
+  const int tpv = n <= kThreads / 4 ? 4 : (n <= kThreads / 2 ? 2 : 1);
+  const int i = tid / tpv, part = tid % tpv;
+  long long mass = 0;
+  float vi = 0.f;
+  if (i < n) {
+    vi = lw[i];
+#pragma unroll 4
+    for (int j = part; j < n; j += tpv) mass += lw[j] >= vi ? lq[j] : 0ll;
   }
-  const float S = block_sum_fixed(esum, red);
-  const float inv = S > 0.f ? 1.f / S : 0.f;
-  // pass 2: W = e / S (in place), the output copy, the largest weight
-  float* wout = a.weights_out ? a.weights_out + (size_t)bh * a.cand_stride : nullptr;
-  float top = 0.f;
-#pragma unroll 1
-  for (int i = tid; i < nc; i += kThreads) {
-    const float wv = (staged ? E[i] : ldcg_f(E + i)) * inv;
-    E[i] = wv;
-    if (wout) wout[i] = wv;
-    top = fmaxf(top, wv);
-  }
-  const float* W = E;
-  top = warp_max(top);
+  if (tpv >= 2) mass += __shfl_xor_sync(0xffffffffu, mass, 1);
+  if (tpv >= 4) mass += __shfl_xor_sync(0xffffffffu, mass, 2);
+  float t = (i < n && mass >= P) ? vi : 0.f;
+  t = warp_max(t);
   __syncthreads();
-  if (lane == 0) red[warp] = top;
+  if (lane == 0) red[warp] = t;
   __syncthreads();
-  {
-    float t = 0.f;
+  float Tp = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) t = fmaxf(t, red[w]);
-    top = t;
-  }
-  const float p = a.p, eps = a.eps;
-  // Decisions at thresholds t <= L = (1 - p) / (2 nc) need no mass: the weights below t sum to
-  // less than nc * t <= (1 - p) / 2, so mass(W >= t) > 1 - (1 - p) / 2 >= p (with margin for fp32
-  // sums, hence the 1e-3 guard).  Above L only weights >= L can count, so the search runs on the
-  // live set {W >= L}; when it is small one warp finishes the bisection from registers.
-  constexpr int kLivePerLane = 8;
-  const bool use_bound = nc > 0 && p < 1.f && (1.f - p) >= 1e-3f;
-  const float L = use_bound ? (1.f - p) / (2.f * (float)nc) : 0.f;
-  float* live = wbuf + (staged ? nc : 0);  // after the staged weights
-  const bool live_fits = staged && 1024 + 4 * nc + 4 * 32 * kLivePerLane <= sm.scratch_bytes;
-  int nlive = 0x7FFFFFFF;
-  if (use_bound && live_fits) {
-    int cntl = 0;
-    for (int i = tid; i < nc; i += kThreads) cntl += W[i] >= L;
-    int* scan_sh2 = reinterpret_cast<int*>(red);  // 33 ints over the reduction area
-    int total_live;
-    int pos = block_exclusive_scan(cntl, scan_sh2, &total_live);
-    nlive = total_live;
-    if (nlive <= 32 * kLivePerLane) {
-      for (int i = tid; i < nc; i += kThreads)
-        if (W[i] >= L) live[pos++] = W[i];
-    }
-    __syncthreads();
-  }
-  int rounds = 0;
-  if (nlive <= 32 * kLivePerLane) {
-    if (warp == 0) {
-      float v[kLivePerLane];
-#pragma unroll
-      for (int k = 0; k < kLivePerLane; ++k) {
-        const int i = k * 32 + lane;
-        v[k] = i < nlive ? live[i] : -1.f;
-      }
-      float mres;
-      // mass over the live set (warp-uniform: xor butterflies give every lane the same bits)
-      auto wmass = [&](float t) {
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < kLivePerLane; ++k) acc += v[k] >= t ? v[k] : 0.f;
-        return warp_sum(acc);
-      };
-      if (wmass(top) >= p) {
-        mres = top;
-      } else {
-        float lo = 0.f, hi = top;
-        int steps = 0;
-        bool done = false;
-#pragma unroll 1
-        while (!done) {
-          // three bisection levels per round: masses of the 7 candidate midpoints at once
-          float nlo[8], nhi[8], nmid[8];
-          nlo[1] = lo;
-          nhi[1] = hi;
-          nmid[1] = mid_of(lo, hi);
-#pragma unroll
-          for (int n = 2; n < 8; ++n) {
-            const int par = n >> 1;
-            nlo[n] = (n & 1) ? nmid[par] : nlo[par];
-            nhi[n] = (n & 1) ? nhi[par] : nmid[par];
-            nmid[n] = mid_of(nlo[n], nhi[n]);
-          }
-          float acc[8];
-#pragma unroll
-          for (int n = 1; n < 8; ++n) {
-            float s8 = 0.f;
-#pragma unroll
-            for (int k = 0; k < kLivePerLane; ++k) s8 += v[k] >= nmid[n] ? v[k] : 0.f;
-            acc[n] = s8;
-          }
-#pragma unroll
-          for (int n = 1; n < 8; ++n) acc[n] = warp_sum(acc[n]);
-          int node = 1;
-#pragma unroll
-          for (int level = 0; level < 3; ++level) {
-            if (done) break;
-            if (__fsub_rn(hi, lo) <= eps) {
-              done = true;
-              break;
-            }
-            float mid = nmid[1], mass = acc[1];
-#pragma unroll
-            for (int n = 2; n < 8; ++n)
-              if (node == n) {
-                mid = nmid[n];
-                mass = acc[n];
-              }
-            if (!(lo < mid && mid < hi) || steps >= 64) {
-              done = true;
-              break;
-            }
-            const bool ge = mid <= L || mass >= p;
-            if (ge) {
-              lo = mid;
-              node = 2 * node + 1;
-            } else {
-              hi = mid;
-              node = 2 * node;
-            }
-            ++steps;
-          }
-        }
-        mres = lo;
-      }
-      if (lane == 0) ctl[11] = mres;
-    }
-    __syncthreads();
-  } else {
-  // ctl[0..6] thresholds, ctl[8] lo, ctl[9] hi, ctl[10] done (as float), ctl[11] m,
-  // ctl[12] bisection steps taken
+  for (int w = 0; w < kWarps; ++w) Tp = fmaxf(Tp, red[w]);
+  return bisect_scalar(top, fmaxf(L, Tp), eps);
+}
+
+// The same search over all nc weights (shared memory or global), three levels of the bisection
+// tree per round: every round sums the masses of the 7 candidate midpoints below (lo, hi) at once.
+__device__ float bisect_block(const float* W, bool staged, int nc, float top, float p, float eps,
+                              float* red, float* ctl) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // ctl[0..6] thresholds, ctl[8] lo, ctl[9] hi, ctl[10] done, ctl[11] m, ctl[12] steps taken
   if (tid == 0) {
-    ctl[10] = (nc == 0 || p >= 1.f) ? 2.f : 0.f;  // 2 = finished with m = 0
+    ctl[10] = 0.f;
     ctl[0] = top;
     for (int k = 1; k < 7; ++k) ctl[k] = INFINITY;
     ctl[8] = 0.f;
@@ -1103,29 +1016,202 @@ __device__ void phase_prune_head(const FusedArgs& a, int gi, int hl, int G, int 
       }
     }
     first = false;
-    ++rounds;
     __syncthreads();
   }
-  }
   const float m = ctl[11];
-#ifdef TWL_PHASE_TIMING
-  if (blockIdx.x == 0 && threadIdx.x == 0 && a.flags) a.flags[2] = rounds;
-#endif
-  (void)rounds;
+  __syncthreads();
+  return m;
+}
+
+// Top-p of one head, run by its owner CTA.  M is the largest of the C per-CTA maxima pushed into
+// this CTA's exchange slot; W_i = exp(l_i - M) / S with S summed in a fixed order (per thread over
+// its rows, then over the block).  Only weights >= L = (1 - p) / (2 nc) can decide a test above
+// L (the weights below L sum to less than nc L = (1 - p) / 2, so the mass above any t <= L
+// exceeds p): the threshold comes from that live set when it is small (the common case), else
+// from the three-level search over every weight.
+__device__ void phase_prune_head(const FusedArgs& a, int hl, int bh, int nc, int C, Smem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float* red = reinterpret_cast<float*>(sm.scratch);                  // [kWarps][8]
+  float* ctl = reinterpret_cast<float*>(sm.scratch + 4 * kWarps * 8);   // search state
+  int* scan_sh2 = reinterpret_cast<int*>(sm.scratch + 768);             // 33 ints
+  uint32_t* top_u = reinterpret_cast<uint32_t*>(sm.scratch + 1000);     // block max of W
+  float* lw = reinterpret_cast<float*>(sm.scratch + 1024);              // [kThreads] live W
+  int* li = reinterpret_cast<int*>(sm.scratch + 1024 + 4 * kThreads);   // [kThreads] their rows
+  long long* lq = reinterpret_cast<long long*>(sm.scratch + 1024 + 8 * kThreads);  // fixed point
+  unsigned char* tail = sm.scratch + 1024 + 16 * kThreads;
+  const int tail_off = (int)(tail - sm.scratch);
+  const bool staged = tail_off + 4 * nc <= sm.scratch_bytes;
+
+  const float* part = reinterpret_cast<const float*>(sm.xchg + (hl / C) * kXchgSlot);
+  float pm[16];
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr) pm[rr] = rr < C ? part[rr] : -INFINITY;
+  float M = -INFINITY;
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr) M = fmaxf(M, pm[rr]);
+  const bool empty = !(M > -INFINITY);
+
+  const float p = a.p, eps = a.eps;
+  const bool use_bound = nc > 0 && p < 1.f && (1.f - p) >= 1e-3f;
+  const float L = use_bound ? (1.f - p) / (2.f * (float)nc) : 0.f;
+  float* lrow = a.logits + (size_t)bh * a.cand_stride;
+  float* wout = a.weights_out ? a.weights_out + (size_t)bh * a.cand_stride : nullptr;
+  if (tid == 0) *top_u = 0u;
+
+  // Weights: in registers (row i = k * kThreads + tid) when nc <= kThreads * kR, else in shared
+  // memory (or in place in the logits row when they do not fit).
+  constexpr int kR = 16;
+  const bool in_regs = nc <= kThreads * kR;
+  float wr[kR];
+  float* W = staged ? reinterpret_cast<float*>(tail) : lrow;
+  float esum = 0.f;
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int i = k * kThreads + tid;
+      wr[k] = i < nc ? ldcg_f(lrow + i) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int i = k * kThreads + tid;
+      const float e = (i < nc && !empty) ? __expf(wr[k] - M) : 0.f;
+      wr[k] = e;
+      esum += e;
+    }
+  } else {
+    constexpr int kB = 8;
+#pragma unroll 1
+    for (int base = 0; base < nc; base += kThreads * kB) {
+      float v[kB];
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int i = base + k * kThreads + tid;
+        v[k] = i < nc ? ldcg_f(lrow + i) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int i = base + k * kThreads + tid;
+        if (i < nc) {
+          const float e = empty ? 0.f : __expf(v[k] - M);
+          W[i] = e;
+          esum += e;
+        }
+      }
+    }
+  }
+  const float S = block_sum_fixed(esum, red);
+  const float inv = S > 0.f ? 1.f / S : 0.f;
+  // W = e / S, the largest weight, the live count
+  float top = 0.f;
+  int cntl = 0;
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int i = k * kThreads + tid;
+      wr[k] *= inv;
+      top = fmaxf(top, wr[k]);
+      cntl += (i < nc && wr[k] >= L) ? 1 : 0;
+    }
+  } else {
+#pragma unroll 1
+    for (int i = tid; i < nc; i += kThreads) {
+      const float w = (staged ? W[i] : ldcg_f(W + i)) * inv;
+      W[i] = w;
+      top = fmaxf(top, w);
+      cntl += w >= L ? 1 : 0;
+    }
+  }
+  top = warp_max(top);
+  if (lane == 0) atomicMax(top_u, __float_as_uint(top));  // W >= 0: the bits order as the values
+  int nlive = 0;
+  int pos = block_exclusive_scan(cntl, scan_sh2, &nlive);  // its barriers also publish top_u
+  top = __uint_as_float(*top_u);
+  const bool from_live = use_bound && nlive <= kThreads;
+  if (from_live) {
+    if (in_regs) {
+#pragma unroll
+      for (int k = 0; k < kR; ++k) {
+        const int i = k * kThreads + tid;
+        if (i < nc && wr[k] >= L) {
+          lw[pos] = wr[k];
+          li[pos] = i;
+          lq[pos] = w_fixed(wr[k]);
+          ++pos;
+        }
+      }
+    } else {
+      for (int i = tid; i < nc; i += kThreads) {
+        const float w = staged ? W[i] : ldcg_f(W + i);
+        if (w >= L) {
+          lw[pos] = w;
+          li[pos] = i;
+          lq[pos] = w_fixed(w);
+          ++pos;
+        }
+      }
+    }
+  }
+  if (wout) {  // the weights output: every candidate
+    if (in_regs) {
+#pragma unroll
+      for (int k = 0; k < kR; ++k) {
+        const int i = k * kThreads + tid;
+        if (i < nc) wout[i] = wr[k];
+      }
+    } else {
+      for (int i = tid; i < nc; i += kThreads) wout[i] = staged ? W[i] : ldcg_f(W + i);
+    }
+  }
+  if (in_regs && !from_live && nc > 0 && p < 1.f) {  // the block search reads every weight
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int i = k * kThreads + tid;
+      if (i < nc) W[i] = wr[k];
+    }
+  }
+  __syncthreads();  // the live set (or the weights) complete
+  float m;
+  if (nc == 0 || p >= 1.f) m = 0.f;  // keep every candidate
+  else if (from_live) m = top_p_from_live(lw, lq, nlive, L, p, eps, top, red);
+  else m = bisect_block(W, staged, nc, top, p, eps, red, ctl);
   if (tid == 0) {
     if (a.threshold) a.threshold[bh] = m;
     if (a.cand_count) a.cand_count[bh] = nc;
   }
-  // kept-row bitmap of this head: bit i = (W_i >= m), one 32-row word per warp ballot
+  // kept-row bitmap of this head: bit i = (W_i >= m)
   uint32_t* kb_out = a.keptbits + (size_t)bh * a.kept_words;
+  const int kw = (nc + 31) >> 5;
+  uint32_t* kbits = reinterpret_cast<uint32_t*>(tail);
   int cnt = 0;
+  if (from_live && m >= L && tail_off + 4 * kw <= sm.scratch_bytes) {
+    // every kept candidate is live
+    for (int w = tid; w < kw; w += kThreads) kbits[w] = 0u;
+    __syncthreads();
+    if (tid < nlive && lw[tid] >= m) atomicOr(&kbits[li[tid] >> 5], 1u << (li[tid] & 31));
+    __syncthreads();
+    for (int w = tid; w < kw; w += kThreads) {
+      const uint32_t x = kbits[w];
+      kb_out[w] = x;
+      cnt += __popc(x);
+    }
+  } else if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int i = k * kThreads + tid;
+      const bool keep = i < nc && wr[k] >= m;
+      const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0 && k * kThreads + 32 * warp < nc) kb_out[k * kWarps + warp] = bal;
+      cnt += keep;
+    }
+  } else {
 #pragma unroll 1
-  for (int base = 0; base < nc; base += kThreads) {
-    const int i = base + tid;
-    const bool keep = i < nc && (staged ? W[i] : ldcg_f(W + i)) >= m;
-    const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0 && base + 32 * warp < nc) kb_out[(base >> 5) + warp] = bal;
-    cnt += keep;
+    for (int base = 0; base < nc; base += kThreads) {
+      const int i = base + tid;
+      const bool keep = i < nc && (staged ? W[i] : ldcg_f(W + i)) >= m;
+      const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0 && base + 32 * warp < nc) kb_out[(base >> 5) + warp] = bal;
+      cnt += keep;
+    }
   }
   if (a.kept_count) {  // only when the caller asks for it
     const float total = block_sum_fixed((float)cnt, red);
@@ -1188,7 +1274,6 @@ __device__ int phase_kept_rows_local(const FusedArgs& a, int b, int kvh, int n, 
                                      int* scan_sh) {
   const int tid = threadIdx.x, nw = sm.nw;
   const int u0 = (int)((long)U * r / C), u1 = (int)((long)U * (r + 1) / C);
-  stamp(a, 27);
   int carry = 0;
 #pragma unroll 1
   for (int ub = u0; ub < u1; ub += kThreads) {
@@ -1200,11 +1285,9 @@ __device__ int phase_kept_rows_local(const FusedArgs& a, int b, int kvh, int n, 
       m = union_row_mask<G>(a, b, kvh, n, j, sm);
       rowmask[u - u0] = (uint16_t)m;
     }
-    stamp(a, 25);
-    int total;
+      int total;
     const int ex = block_exclusive_scan(__popc(m), scan_sh, &total);
-    stamp(a, 26);
-    if (u < u1) pfx[u - u0] = carry + ex;
+      if (u < u1) pfx[u - u0] = carry + ex;
     carry += total;
   }
   __syncthreads();
@@ -1461,6 +1544,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ int scan_sh[33];
   __shared__ int s_total;
+  __shared__ int s_nc[8];
 
   const int C = (int)cluster_size();
   const int r = (int)cluster_rank();
@@ -1502,6 +1586,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
     sm.ubits = reinterpret_cast<uint32_t*>(p);
     p += 4 * a.sel_words;
     sm.upre = reinterpret_cast<int*>(p);
+    sm.xchg = smem_raw + bitmap_bytes(G, a.sel_words);
     p = smem_raw + persistent_bytes(G, a.sel_words);
     sm.pt = nullptr;
     if (a.pt_smem) {  // the sequence's page table, validated once
@@ -1530,31 +1615,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
   // 3: bitmaps, union, ranks (every CTA)
   phase_union_bitmaps<G>(a, b, kvh, sm, &s_total, scan_sh);
   const int U = s_total;
+  if (tid < G) {
+    // candidate rows of each head: its kb pages' rows; the last selected page (the highest set
+    // bit of the head bitmap) may be partial
+    const uint32_t* hb = sm.hbits + tid * sm.nw;
+    int jl = -1;
+    for (int w = sm.nw - 1; w >= 0; --w)
+      if (hb[w]) {
+        jl = 32 * w + 31 - __clz(hb[w]);
+        break;
+      }
+    s_nc[tid] = (kb > 0 && jl >= 0) ? kPage * (kb - 1) + page_rows(sq.n, jl) : 0;
+  }
+  __syncthreads();
   stamp(a, 5);
-  // 4: INT4 estimate over this CTA's share of the union
-  phase_estimate<G>(a, b, kvh, gi, sq.n, U, r, C, sm);
+  // 4: INT4 estimate over this CTA's share of the union; partials and candidate lists to owners
+  phase_estimate<G>(a, b, kvh, sq.n, U, r, C, sm);
   stamp(a, 6);
   cluster_sync();
   stamp(a, 7);
   // 5: top-p of the heads this CTA owns
-  {
-    int nc = 0;
-    if (kb > 0) {
-      // the last selected page is the highest set bit of the head bitmap
-      for (int hl = r; hl < G; hl += C) {
-        const uint32_t* hb = sm.hbits + hl * sm.nw;
-        int jl = -1;
-        for (int w = sm.nw - 1; w >= 0; --w)
-          if (hb[w]) {
-            jl = 32 * w + 31 - __clz(hb[w]);
-            break;
-          }
-        nc = jl >= 0 ? kPage * (kb - 1) + page_rows(sq.n, jl) : 0;
-        phase_prune_head(a, gi, hl, G, b * a.hq + kvh * G + hl, nc, C, sm);
-        __syncthreads();
-      }
+  if (kb > 0)
+    for (int hl = r; hl < G; hl += C) {
+      phase_prune_head(a, hl, b * a.hq + kvh * G + hl, s_nc[hl], C, sm);
+      __syncthreads();
     }
-  }
   stamp(a, 8);
   cluster_sync();
   stamp(a, 9);
@@ -1638,7 +1723,7 @@ FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) 
   want = want > topk_need ? want : topk_need;
   const size_t local_need = scratch + (size_t)10 * max_pages + 64;
   want = want > local_need ? want : local_need;
-  const size_t prune_need = 1024 + (size_t)4 * pl.cand_stride + 4 * 32 * 8 + 64;
+  const size_t prune_need = 1024 + (size_t)16 * kThreads + (size_t)4 * pl.cand_stride;
   want = want > prune_need ? want : prune_need;
   want = want > (size_t)2 * pl.union_stride / 16 + 16 ? want : (size_t)2 * pl.union_stride / 16 + 16;
   // the bulk-copy chunks of the scoring and estimate phases take whatever is left: ask for the
@@ -1659,7 +1744,6 @@ size_t fused_workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_
   add(bh * max_pages * 4);                    // scores
   add(bh * pl.sel_words * 4);                 // selected-page bitmaps
   add(bh * (size_t)pl.cand_stride * 4);       // logits / weights
-  add(groups * 16 * g * 2 * 4);               // partial (max, sum)
   add(groups * 16 * 4);                       // union counts per CTA
   add(groups * (size_t)pl.union_stride * 4);  // union token lists
   add(groups * 16 * g * (kHeadDim + 2) * 4);  // attention partials
@@ -1680,7 +1764,6 @@ void carve_fused(FusedArgs& a, char* ws, const FusedPlan& pl, int batch, int hq,
   a.scores = reinterpret_cast<float*>(take(bh * max_pages * 4));
   a.selbits = reinterpret_cast<uint32_t*>(take(bh * pl.sel_words * 4));
   a.logits = reinterpret_cast<float*>(take(bh * (size_t)pl.cand_stride * 4));
-  a.part_ms = reinterpret_cast<float*>(take(groups * 16 * g * 2 * 4));
   a.union_part = reinterpret_cast<int*>(take(groups * 16 * 4));
   int* ulist = reinterpret_cast<int*>(take(groups * (size_t)pl.union_stride * 4));
   if (!a.union_tok) a.union_tok = ulist;

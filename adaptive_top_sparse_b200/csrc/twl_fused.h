@@ -39,7 +39,6 @@ struct FusedArgs {
   uint32_t* selbits;
   float* logits;
   uint32_t* keptbits;  // [B * Hq][kept_words]: bit i = candidate row i passes top-p
-  float* part_ms;
   int* union_part;
   float* part_att;
   uint32_t* flags;
