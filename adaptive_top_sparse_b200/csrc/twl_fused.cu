@@ -24,14 +24,11 @@
 // sits behind a data-dependent branch, and a group whose sequence is invalid exits before the
 // first one, uniformly across its cluster.  Arithmetic and summation orders match the staged
 // kernels, so the selection is bit-identical to twl_select_pages.
-#include <cooperative_groups.h>
 #include <stdlib.h>
 
 #include "twl_common.cuh"
 #include "twl_fused.h"
 #include "twl_kernels.h"
-
-namespace cg = cooperative_groups;
 
 namespace twl {
 namespace {
@@ -40,7 +37,12 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kAttChunk = 64;  // tokens gathered per attention round
 
-__device__ __forceinline__ void cluster_sync() { cg::this_cluster().sync(); }
+// Cluster barrier: arrive with release, wait with acquire semantics (orders shared, distributed
+// shared and global memory accesses of the cluster's CTAs across it).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -107,7 +109,9 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   }
 }
 
-// Same fragment map as the staged estimate kernel (see twl_estimate.cu).
+// B fragments of the query for the m16n8k16 products: lane (g, t) holds the channels
+// c0 = 32 t + 8 w8 (w8 = ks / 2) of its head; k-step ks pairs (c0 + 4e, c0 + 4e + 2) and
+// (c0 + 4e + 1, c0 + 4e + 3), e = ks % 2, the same pairs nibble_pairs() builds from K.
 // Also returns the sum of the lane's 32 query channels (for the zero-point term).
 __device__ __forceinline__ float q_fragments(const uint16_t* qh, bool valid, uint32_t (&bf)[8][2]) {
   const int t = threadIdx.x & 3;
@@ -127,16 +131,40 @@ __device__ __forceinline__ float q_fragments(const uint16_t* qh, bool valid, uin
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
     const int w8 = ks >> 1, e = ks & 1;
-    bf[ks][0] = __byte_perm(w[4 * w8 + e], w[4 * w8 + e + 2], 0x5410);
-    bf[ks][1] = __byte_perm(w[4 * w8 + e], w[4 * w8 + e + 2], 0x7632);
+    bf[ks][0] = __byte_perm(w[4 * w8 + 2 * e], w[4 * w8 + 2 * e + 1], 0x5410);
+    bf[ks][1] = __byte_perm(w[4 * w8 + 2 * e], w[4 * w8 + 2 * e + 1], 0x7632);
   }
   return qsum;
 }
 
-__device__ __forceinline__ uint32_t nib_pair(uint32_t x, int i) {
-  uint32_t v = ((x >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
-  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&v), __float2half2_rn(1024.f));
-  return *reinterpret_cast<const uint32_t*>(&r);
+// Nibbles to fp16 without arithmetic: a byte 0000nnnn read as FP8 E4M3 (sign 0, exponent 000n3,
+// mantissa n2 n1 n0) is n * 2^-9 exactly (subnormal m * 2^-9 for n < 8, (8 + m) * 2^-9 for
+// n >= 8), and that is an exact fp16 value.  A word of 8 nibbles (channels c0..c0+7, low nibble
+// first) gives the bytes (n0, n2, n4, n6) and (n1, n3, n5, n7); each 16-bit half converts to
+// one f16x2 pair.  Products with q are therefore 2^-9 times the integer-nibble products, and the
+// fp32 sums scale exactly; the epilogue multiplies by 512.
+__device__ __forceinline__ uint32_t e4m3x2_lo(uint32_t y) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\t}"
+      : "=r"(r)
+      : "r"(y));
+  return r;
+}
+__device__ __forceinline__ uint32_t e4m3x2_hi(uint32_t y) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, h;\n\t}"
+      : "=r"(r)
+      : "r"(y));
+  return r;
+}
+// The four A registers of k-step (w8, e) for rows g (word x0) and g + 8 (word x1).
+__device__ __forceinline__ void nibble_pairs(uint32_t x0, uint32_t x1, int e, uint32_t (&av)[4]) {
+  const uint32_t e0 = x0 & 0x0F0F0F0Fu, o0 = (x0 >> 4) & 0x0F0F0F0Fu;
+  const uint32_t e1 = x1 & 0x0F0F0F0Fu, o1 = (x1 >> 4) & 0x0F0F0F0Fu;
+  av[0] = e ? e4m3x2_hi(e0) : e4m3x2_lo(e0);
+  av[1] = e ? e4m3x2_hi(e1) : e4m3x2_lo(e1);
+  av[2] = e ? e4m3x2_hi(o0) : e4m3x2_lo(o0);
+  av[3] = e ? e4m3x2_hi(o1) : e4m3x2_lo(o1);
 }
 
 // Bytes of the persistent bitmap region, rounded up so the scratch region after it is 128-byte
@@ -152,6 +180,7 @@ __host__ __device__ constexpr int persistent_bytes(int g, int sel_words) {
 // region reused by the phases.
 struct Smem {
   const int* pt;    // the sequence's page table (validated; -1 = bad entry), or nullptr
+  const uint16_t* q;  // [G][128] the group's queries (fp16), staged once
   uint32_t* hbits;  // [G][nw]  head page bitmaps
   int* hpre;        // [G][nw]  exclusive prefix popcounts per word
   uint32_t* ubits;  // [nw]     union bitmap
@@ -213,7 +242,7 @@ __device__ void phase_scores(const FusedArgs& a, int b, int kvh, int n_pages, in
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     const uint4 raw = *reinterpret_cast<const uint4*>(
-        a.q + ((size_t)b * a.hq + kvh * G + h) * kHeadDim + 8 * l);
+        sm.q + h * kHeadDim + 8 * l);
     unpack8(raw, qv[h]);
   }
   int* phys = reinterpret_cast<int*>(sm.scratch);
@@ -226,7 +255,6 @@ __device__ void phase_scores(const FusedArgs& a, int b, int kvh, int n_pages, in
     for (int i = threadIdx.x; i < cn; i += kThreads)
       phys[i] = phys_of(a, sm, b, c0 + i);
     __syncthreads();
-    if (c0 == p0) stamp(a, 17);
     // 32 chunks of 16 bytes per page, spread over all threads, all in flight together
     for (int c = threadIdx.x; c < 32 * cn; c += kThreads) {
       const int i = c >> 5, k = c & 31;
@@ -238,7 +266,6 @@ __device__ void phase_scores(const FusedArgs& a, int b, int kvh, int n_pages, in
     cp_async_commit();
     cp_async_wait_all();
     __syncthreads();
-    if (c0 == p0) stamp(a, 18);
     const bool ok = true;
     for (int base = 0; base < cn; base += 2 * kWarps) {  // warp-uniform trip count
       const int i0 = base + 2 * warp + half;
@@ -688,7 +715,7 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int n, int U,
   unsigned char* szs = tiles + 1024 * ch;                              // [ch][64] scale/zero
   uint32_t bf[8][2];
   const bool head_ok = gr < G;
-  const uint16_t* qh = a.q + ((size_t)b * a.hq + kvh * G + (head_ok ? gr : 0)) * kHeadDim;
+  const uint16_t* qh = sm.q + (head_ok ? gr : 0) * kHeadDim;
   float qs_part = q_fragments(qh, head_ok, bf);
   qs_part += __shfl_xor_sync(0xffffffffu, qs_part, 1);
   qs_part += __shfl_xor_sync(0xffffffffu, qs_part, 2);
@@ -752,10 +779,7 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int n, int U,
         for (int ks = 0; ks < 8; ++ks) {
           const int w8 = ks >> 1, e = ks & 1;
           uint32_t av[4];
-          av[0] = nib_pair(r0[w8], 2 * e);
-          av[1] = nib_pair(r1[w8], 2 * e);
-          av[2] = nib_pair(r0[w8], 2 * e + 1);
-          av[3] = nib_pair(r1[w8], 2 * e + 1);
+          nibble_pairs(r0[w8], r1[w8], e, av);
           mma_16816(acc, av, bf[ks][0], bf[ks][1]);
         }
 #pragma unroll
@@ -788,7 +812,7 @@ __device__ void phase_estimate(const FusedArgs& a, int b, int kvh, int n, int U,
             if (row >= rows) continue;
             const float sv = rr ? s1 : s0, zv = rr ? z1 : z0;
             const float lg =
-                bad ? -INFINITY : (sv * accp[pp][2 * rr + e] + zv * qsum) * inv_sqrt_d;
+                bad ? -INFINITY : (sv * (accp[pp][2 * rr + e] * 512.f) + zv * qsum) * inv_sqrt_d;
             a.logits[obase + row] = lg;
             if (a.cand_tok) a.cand_tok[obase + row] = kPage * j + row;
             rm[e] = fmaxf(rm[e], lg);
@@ -1050,6 +1074,7 @@ __device__ void phase_prune_head(const FusedArgs& a, int hl, int bh, int nc, int
 #pragma unroll
   for (int rr = 0; rr < 16; ++rr) M = fmaxf(M, pm[rr]);
   const bool empty = !(M > -INFINITY);
+  stamp(a, 17);
 
   const float p = a.p, eps = a.eps;
   const bool use_bound = nc > 0 && p < 1.f && (1.f - p) >= 1e-3f;
@@ -1101,6 +1126,7 @@ __device__ void phase_prune_head(const FusedArgs& a, int hl, int bh, int nc, int
   }
   const float S = block_sum_fixed(esum, red);
   const float inv = S > 0.f ? 1.f / S : 0.f;
+  stamp(a, 18);
   // W = e / S, the largest weight, the live count
   float top = 0.f;
   int cntl = 0;
@@ -1126,6 +1152,7 @@ __device__ void phase_prune_head(const FusedArgs& a, int hl, int bh, int nc, int
   int nlive = 0;
   int pos = block_exclusive_scan(cntl, scan_sh2, &nlive);  // its barriers also publish top_u
   top = __uint_as_float(*top_u);
+  stamp(a, 19);
   const bool from_live = use_bound && nlive <= kThreads;
   if (from_live) {
     if (in_regs) {
@@ -1174,6 +1201,7 @@ __device__ void phase_prune_head(const FusedArgs& a, int hl, int bh, int nc, int
   if (nc == 0 || p >= 1.f) m = 0.f;  // keep every candidate
   else if (from_live) m = top_p_from_live(lw, lq, nlive, L, p, eps, top, red);
   else m = bisect_block(W, staged, nc, top, p, eps, red, ctl);
+  stamp(a, 20);
   if (tid == 0) {
     if (a.threshold) a.threshold[bh] = m;
     if (a.cand_count) a.cand_count[bh] = nc;
@@ -1344,7 +1372,7 @@ __device__ void phase_attend(const FusedArgs& a, int b, int kvh, int gi, int n, 
   float qv[G][16];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    const uint16_t* qh = a.q + ((size_t)b * a.hq + kvh * G + h) * kHeadDim;
+    const uint16_t* qh = sm.q + h * kHeadDim;
     float f[8];
     unpack8(*reinterpret_cast<const uint4*>(qh + 8 * s8), f);
 #pragma unroll
@@ -1577,6 +1605,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
 
   Smem sm;
   sm.nw = (n_pages + 31) >> 5;
+  {
+    __shared__ __align__(16) uint16_t s_q[8 * kHeadDim];
+    const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.hq + kvh * G) * kHeadDim);
+    for (int i = tid; i < G * kHeadDim / 8; i += kThreads) reinterpret_cast<uint4*>(s_q)[i] = src[i];
+    sm.q = s_q;
+  }
   {
     unsigned char* p = smem_raw;
     sm.hbits = reinterpret_cast<uint32_t*>(p);
