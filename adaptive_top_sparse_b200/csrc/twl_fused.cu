@@ -305,41 +305,6 @@ __device__ void phase_scores(const FusedArgs& a, int b, int kvh, int n_pages, in
   }
 }
 
-// Bitonic sort of 256 keys held by one warp, descending.  Key i*32 + lane lives in v[i] of
-// `lane`; partners at distance >= 32 are in the same lane, smaller distances one shuffle away.
-__device__ __forceinline__ void warp_sort256_desc(uint32_t (&v)[8]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int size = 2; size <= 256; size <<= 1) {
-#pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      if (stride >= 32) {
-        const int rs = stride >> 5;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int j = i ^ rs;
-          if (j > i) {
-            const bool desc = ((i * 32 + lane) & size) == 0;
-            const uint32_t x = v[i], y = v[j];
-            const bool swap = desc ? (x < y) : (x > y);
-            v[i] = swap ? y : x;
-            v[j] = swap ? x : y;
-          }
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t other = __shfl_xor_sync(0xffffffffu, v[i], stride);
-          const bool lower = (lane & stride) == 0;
-          const bool desc = ((i * 32 + lane) & size) == 0;
-          const uint32_t hi = max(v[i], other), lo = min(v[i], other);
-          v[i] = (lower == desc) ? hi : lo;
-        }
-      }
-    }
-  }
-}
-
 // ------------------------------------------------------------------------- phase 2: top-k
 // Radix select of the kb largest keys (ties to the lower index) -> bitmap of selected pages.
 __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb, Smem& sm) {
@@ -359,14 +324,13 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
     if (tid == 0 && a.sel_count) a.sel_count[bh] = n_pages;
     return;
   }
-  // keys in shared memory when they fit, else read from L2 on every pass
+  // the keys in shared memory (the launch plan guarantees room for max_pages of them)
   const float* row = a.scores + (size_t)bh * a.kv.max_pages;
   uint32_t* hist = reinterpret_cast<uint32_t*>(sm.scratch);           // 256
   int* scan_sh = reinterpret_cast<int*>(sm.scratch + 1024);           // 33
-  uint32_t* state = reinterpret_cast<uint32_t*>(sm.scratch + 1200);   // 2
+  uint32_t* state = reinterpret_cast<uint32_t*>(sm.scratch + 1200);   // 3
   uint32_t* keys = reinterpret_cast<uint32_t*>(sm.scratch + 1280);
-  const bool staged = 1280 + 4 * n_pages <= sm.scratch_bytes;
-  if (staged) {
+  {
     constexpr int kB = 8;  // independent loads in flight per thread
     for (int base = 0; base < n_pages; base += kThreads * kB) {
       float v[kB];
@@ -383,46 +347,28 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
     }
   }
   __syncthreads();
-  auto key_at = [&](int i) -> uint32_t { return staged ? keys[i] : f32_key(ldcg_f(row + i)); };
+  auto key_at = [&](int i) -> uint32_t { return keys[i]; };
 
   // The k-th largest key is narrowed down to a key interval [blo, bhi] holding `cand` keys, of
-  // which the `remaining` largest are selected (every key above bhi is selected).  Each pass
-  // histograms the keys inside the interval into up to 1024 bins of equal key width (the keys'
-  // offsets from blo, shifted right) and keeps the bin holding the k-th key.
-  //
-  // Start: a sample of 256 keys (every n/256-th page), sorted by one warp, brackets the k-th key
-  // between the sample's ranks r* - 16 and r* + 16 (r* = k * 256 / n).  The first pass also counts
-  // the keys above the bracket; when the count confirms the bracket (above < k <= above +
-  // inside) narrowing goes on from the bin found, otherwise it restarts from [min key, max key].
+  // which the `remaining` largest are selected (every key above bhi is selected).  It starts as
+  // [min key, max key]; each pass histograms the keys inside it into up to 4096 bins of equal key
+  // width (offsets from blo, shifted right) and keeps the bin holding the k-th key.  Keys are
+  // monotone in the score and roughly logarithmic in its magnitude, so one pass usually leaves a
+  // handful of candidates.
   constexpr int kGatherCap = 64;
-  uint32_t* bhist = reinterpret_cast<uint32_t*>(sm.scratch + 1280 + 4 * n_pages);  // [1024]
-  uint32_t* gkey = bhist + 1024;                                                   // [cap]
+  constexpr int kBins = 4096;
+  uint32_t* bhist = reinterpret_cast<uint32_t*>(sm.scratch + 1280 + 4 * n_pages);  // [kBins]
+  uint32_t* gkey = bhist + kBins;                                                  // [cap]
   int* gidx = reinterpret_cast<int*>(gkey + kGatherCap);                           // [cap]
   uint32_t* sbits = reinterpret_cast<uint32_t*>(gidx + kGatherCap);                // [nw]
-  const bool room = staged && 1280 + 4 * (size_t)n_pages + 4 * 1024 + 8 * kGatherCap + 4 * nw +
-                                  16 <= (size_t)sm.scratch_bytes;
+  const bool room = 1280 + 4 * (size_t)n_pages + 4 * kBins + 8 * kGatherCap + 4 * nw + 16 <=
+                    (size_t)sm.scratch_bytes;
   uint32_t* hh = room ? bhist : hist;  // the 256-bin histogram when there is no room
-  const int nbins = room ? 1024 : 256;
-  const int bin_bits = room ? 10 : 8;
-  uint32_t blo = 0u, bhi = 0xFFFFFFFFu;
-  int remaining = kb;
-  int cand = n_pages;
-  bool need_above = false;
-  if (room && n_pages > 512) {
-    if (warp == 0) {
-      uint32_t v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = keys[(int)((long)(i * 32 + lane) * n_pages / 256)];
-      warp_sort256_desc(v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) hist[i * 32 + lane] = v[i];
-    }
-    __syncthreads();
-    const int rstar = (int)((long)kb * 256 / n_pages);
-    bhi = rstar - 16 >= 0 ? hist[rstar - 16] : 0xFFFFFFFFu;
-    blo = rstar + 16 <= 255 ? hist[rstar + 16] : 0u;
-    need_above = true;
-  } else {
+  const int nbins = room ? kBins : 256;
+  const int bin_bits = room ? 12 : 8;
+  const int per = nbins / kThreads > 0 ? nbins / kThreads : 1;  // bins per thread in the scan
+  uint32_t blo, bhi;
+  {
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
     for (int i = tid; i < n_pages; i += kThreads) {
       const uint32_t k = key_at(i);
@@ -446,89 +392,53 @@ __device__ void phase_topk_head(const FusedArgs& a, int bh, int n_pages, int kb,
     blo = kmin;
     bhi = kmax;
   }
+  int remaining = kb;
+  int cand = n_pages;
   __syncthreads();
   const int n_it = (n_pages + kThreads - 1) / kThreads;
 #pragma unroll 1
-  while (need_above || ((cand > kGatherCap || !room) && blo < bhi)) {
+  while ((cand > kGatherCap || !room) && blo < bhi) {
     const uint32_t range = bhi - blo;
-    const int width = range ? 32 - __clz(range) : 0;
+    const int width = 32 - __clz(range);
     const int sh = width > bin_bits ? width - bin_bits : 0;
     for (int i = tid; i < nbins; i += kThreads) hh[i] = 0u;
     __syncthreads();
-    int above = 0;
 #pragma unroll 1
     for (int it = 0; it < n_it; ++it) {
       const int i = it * kThreads + tid;
       if (i < n_pages) {
         const uint32_t key = key_at(i);
-        above += need_above && key > bhi ? 1 : 0;
         if (key >= blo && key <= bhi) atomicAdd(&hh[(key - blo) >> sh], 1u);
       }
     }
     __syncthreads();
-    // descending scan over the bins, two per thread; the keys above the interval ride in the
-    // upper 16 bits (n_pages < 65536)
-    const int b0 = nbins - 1 - 2 * tid, b1 = b0 - 1;
-    const uint32_t c0 = b0 >= 0 ? hh[b0] : 0u, c1 = b1 >= 0 ? hh[b1] : 0u;
-    int tot;
-    const int ex = block_exclusive_scan((int)(((uint32_t)above << 16) | (c0 + c1)), scan_sh, &tot);
-    const int excl = ex & 0xFFFF;
-    int base_rank = 0;  // keys above the interval that `remaining` does not yet exclude
-    bool restart = false;
-    if (need_above) {
-      base_rank = tot >> 16;
-      const int inside = tot & 0xFFFF;
-      restart = !(base_rank < kb && kb <= base_rank + inside);
-    }
-    const int want = remaining - base_rank;
-    if (!restart) {
-      if (excl < want && want <= excl + (int)c0) {
-        state[0] = (uint32_t)b0;
-        state[1] = (uint32_t)(want - excl);
-        state[2] = c0;
-      } else if (excl + (int)c0 < want && want <= excl + (int)(c0 + c1)) {
-        state[0] = (uint32_t)b1;
-        state[1] = (uint32_t)(want - excl - (int)c0);
-        state[2] = c1;
+    // descending scan over the bins: thread t owns bins nbins-1-per*t ... nbins-per*(t+1)
+    const int b0 = nbins - 1 - per * tid;
+    int mine = 0;
+    for (int e = 0; e < per; ++e)
+      if (b0 - e >= 0) mine += (int)hh[b0 - e];
+    const int excl = block_exclusive_scan(mine, scan_sh, nullptr);
+    if (excl < remaining && remaining <= excl + mine) {
+      int run = excl;
+      for (int e = 0; e < per; ++e) {
+        const int c = (int)hh[b0 - e];
+        if (run + c >= remaining) {
+          state[0] = (uint32_t)(b0 - e);
+          state[1] = (uint32_t)(remaining - run);
+          state[2] = (uint32_t)c;
+          break;
+        }
+        run += c;
       }
     }
     __syncthreads();
-    if (restart) {
-      // the sample's bracket missed the k-th key: start again from the whole key range
-      uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-      for (int i = tid; i < n_pages; i += kThreads) {
-        const uint32_t k = key_at(i);
-        kmin = min(kmin, k);
-        kmax = max(kmax, k);
-      }
-      kmin = __reduce_min_sync(0xffffffffu, kmin);
-      kmax = __reduce_max_sync(0xffffffffu, kmax);
-      if (lane == 0) {
-        hist[2 * warp] = kmin;
-        hist[2 * warp + 1] = kmax;
-      }
-      __syncthreads();
-      kmin = 0xFFFFFFFFu;
-      kmax = 0u;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        kmin = min(kmin, hist[2 * w]);
-        kmax = max(kmax, hist[2 * w + 1]);
-      }
-      blo = kmin;
-      bhi = kmax;
-      remaining = kb;
-      cand = n_pages;
-    } else {
-      const uint32_t bin = state[0];
-      const uint32_t nlo = blo + (bin << sh);
-      const uint64_t top = (uint64_t)nlo + ((1ull << sh) - 1ull);
-      bhi = top < (uint64_t)bhi ? (uint32_t)top : bhi;
-      blo = nlo;
-      remaining = (int)state[1];
-      cand = (int)state[2];
-    }
-    need_above = false;
+    const uint32_t bin = state[0];
+    const uint32_t nlo = blo + (bin << sh);
+    const uint64_t top = (uint64_t)nlo + ((1ull << sh) - 1ull);
+    bhi = top < (uint64_t)bhi ? (uint32_t)top : bhi;
+    blo = nlo;
+    remaining = (int)state[1];
+    cand = (int)state[2];
     __syncthreads();
   }
   if (room && cand <= kGatherCap) {
@@ -1764,7 +1674,8 @@ FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) 
   // full capacity (one CTA per SM in any case)
   want = cap - persistent;
   pl.smem_bytes = (int)(persistent + want);
-  pl.ok = persistent + scratch <= cap && persistent + (size_t)2 * max_pages <= cap;
+  pl.ok = persistent + scratch <= cap && persistent + (size_t)2 * max_pages <= cap &&
+          persistent + 1280 + (size_t)4 * max_pages <= cap;  // the top-k keys
   return pl;
 }
 
