@@ -7,22 +7,26 @@
 // over the union of the heads' pages, group-wise variable-length attention).
 //
 // Every dependency of the path stays inside one GQA group, so a group is processed by one cluster
-// of C CTAs (C = 16 at batch 1, down to 1 when there are enough groups to fill the GPU), and the
+// of C CTAs (up to 16 at batch 1, down to 1 when there are enough groups to fill the GPU), and the
 // phases are separated by hardware cluster barriers instead of kernel boundaries:
 //   1 scores   CTA r scores pages [r P/C, (r+1) P/C) of every head of the group  -> L2
-//   2 top-k    one owner CTA per head radix-selects its k pages               -> page bitmap
+//   2 top-k    one owner CTA per head selects its k pages (histogram passes over the keys, then
+//              an exact ranking of the last bin)                                 -> page bitmap
 //   3 union    every CTA ORs the head bitmaps; ranks come from prefix popcounts
-//   4 estimate CTA r takes an even share of the union pages; one warp per page runs the INT4
-//              dequant-dot on the tensor cores for all heads that selected it    -> logits
-//   5 prune    the owner CTA of each head normalises its weights and bisects the threshold
-//   6 union    CTA r ORs the heads' kept bits on its pages; counts are exchanged, then the
-//              group's kept tokens are written in ascending order
-//   7 attend   CTA r gathers an even share of the kept K/V rows; partial (o, lse) per CTA
+//   4 estimate CTA r takes an even share of the union pages; a warp runs the INT4 dequant-dot
+//              of two pages at a time on the tensor cores for all heads that selected them
+//                                                  -> logits; per-CTA maxima -> owners' smem
+//   5 prune    the owner CTA of each head normalises its weights, finds the top-p threshold and
+//              writes the bitmap of kept candidate rows
+//   6 union    CTA r ORs the heads' kept bits on its pages (with stats: counts are exchanged,
+//              then the group's kept tokens are written in ascending order)
+//   7 attend   CTA r gathers its kept K/V rows; partial (o, lse) per CTA
 //   8 merge    the owner CTA of each head merges the C partials by log-sum-exp.
-// Data that crosses CTAs goes through global memory (it stays in L2) with L1-bypassing loads;
-// the cluster barrier's release/acquire orders it.  Every CTA executes every barrier: no barrier
-// sits behind a data-dependent branch, and a group whose sequence is invalid exits before the
-// first one, uniformly across its cluster.  Arithmetic and summation orders match the staged
+// Data that crosses CTAs goes through global memory (it stays in L2) with L1-bypassing loads,
+// except the per-CTA logit maxima, which are stored into the owner's shared memory; the cluster
+// barrier's release/acquire orders both.  Every CTA executes every barrier: no barrier sits
+// behind a data-dependent branch, and a group whose sequence is invalid exits before the first
+// one, uniformly across its cluster.  The score arithmetic and summation order match the staged
 // kernels, so the selection is bit-identical to twl_select_pages.
 #include <stdlib.h>
 
