@@ -238,6 +238,26 @@ twl_status twl_quantize_k(const twl_paged_kv* kv, void* k_int4, void* k_scale_ze
                                        (cudaStream_t)stream));
 }
 
+twl_status twl_append_token(const twl_paged_kv* kv, const twl_k_aux* aux, const void* k_new,
+                            const void* v_new, int32_t advance, void* ws, size_t ws_bytes,
+                            twl_stream_t stream) {
+  KV k;
+  twl_status st = check_kv(kv, true, true, &k);
+  if (st != TWL_OK) return st;
+  if (!aux || !aux->k_int4 || !aux->k_scale_zero || !aux->bounds || !aligned(aux->k_int4, 16) ||
+      !aligned(aux->k_scale_zero, 16) || !aligned(aux->bounds, 16))
+    return TWL_ERR_INVALID_ARG;
+  if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return TWL_ERR_INVALID_ARG;
+  if (ws && (st = check_ws(ws, ws_bytes, kHeaderBytes)) != TWL_OK) return st;
+  // the caller's cache buffers are written through (see the declaration)
+  return cuda_status(launch_append_token(
+      k, const_cast<uint16_t*>(k.k), const_cast<uint16_t*>(k.v),
+      static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new),
+      static_cast<uint8_t*>(aux->k_int4), static_cast<uint16_t*>(aux->k_scale_zero),
+      static_cast<uint16_t*>(aux->bounds), advance ? const_cast<int32_t*>(kv->seq_lens) : nullptr,
+      flags_of(ws), (cudaStream_t)stream));
+}
+
 twl_status twl_select_pages(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
                             const void* bounds, int32_t budget_pages, int32_t budget_div,
                             int32_t max_budget, int32_t* sel_pages, int32_t* sel_count,

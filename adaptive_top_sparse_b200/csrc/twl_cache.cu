@@ -6,8 +6,9 @@
 //   - INT4 K: summary, appendix B.1 (per-head dynamic quantisation, fp16 scale and zero point,
 //     two 4-bit values per byte); notes page, "Key designs" (4-bit K cache, 1/8 extra memory).
 //
-// Both kernels give one warp to one (sequence, logical page, kv-head): the page-head tile is
-// 16 rows x 256 B, contiguous; lane l owns channels 4l .. 4l+3 (8 bytes of every row).
+// The full kernels give one warp to one (sequence, logical page, kv-head): the page-head tile is
+// 16 rows x 256 B, contiguous; lane l owns channels 4l .. 4l+3 (8 bytes of every row).  The
+// append kernel gives one warp to one (sequence, kv-head) of the new token, same lane layout.
 #include "twl_common.cuh"
 #include "twl_kernels.h"
 
@@ -82,6 +83,29 @@ __device__ __forceinline__ uint32_t nibble(uint32_t xbits, float z, float s) {
   return (uint32_t)r;
 }
 
+// INT4 of one token row held by a warp (lane l: channels 4l .. 4l+3): returns the lane's 4
+// nibbles (channel 2j in the low nibble of byte j) and, in *sz, fp16 scale | fp16 zero << 16.
+__device__ __forceinline__ uint16_t quantize_row_warp(const Half4& v, uint32_t* sz) {
+  int k0 = f16_key(v.lo), k1 = f16_key(v.lo >> 16), k2 = f16_key(v.hi), k3 = f16_key(v.hi >> 16);
+  int kmn = min(min(k0, k1), min(k2, k3));
+  int kmx = max(max(k0, k1), max(k2, k3));
+  kmn = __reduce_min_sync(0xffffffffu, kmn);
+  kmx = __reduce_max_sync(0xffffffffu, kmx);
+  const uint32_t mn_bits = f16_from_key(kmn), mx_bits = f16_from_key(kmx);
+  const float mn = __half2float(__ushort_as_half((unsigned short)mn_bits));
+  const float mx = __half2float(__ushort_as_half((unsigned short)mx_bits));
+  const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.f));
+  const float s = __half2float(s16);
+  uint32_t packed = 0;
+  if (s != 0.f) {
+    uint32_t n0 = nibble(v.lo, mn, s), n1 = nibble(v.lo >> 16, mn, s);
+    uint32_t n2 = nibble(v.hi, mn, s), n3 = nibble(v.hi >> 16, mn, s);
+    packed = n0 | (n1 << 4) | (n2 << 8) | (n3 << 12);
+  }
+  *sz = uint32_t(__half_as_ushort(s16)) | (mn_bits << 16);
+  return (uint16_t)packed;
+}
+
 __global__ void __launch_bounds__(256) k_quantize_k(KV kv, uint8_t* __restrict__ k_int4,
                                                     uint16_t* __restrict__ k_sz,
                                                     uint32_t* flags) {
@@ -107,29 +131,96 @@ __global__ void __launch_bounds__(256) k_quantize_k(KV kv, uint8_t* __restrict__
       if (lane == 0) dst_sz[r] = 0u;
       continue;
     }
-    Half4 v = load_half4(src + r * kHeadDim);
-    int k0 = f16_key(v.lo), k1 = f16_key(v.lo >> 16), k2 = f16_key(v.hi), k3 = f16_key(v.hi >> 16);
-    int kmn = min(min(k0, k1), min(k2, k3));
-    int kmx = max(max(k0, k1), max(k2, k3));
-    kmn = __reduce_min_sync(0xffffffffu, kmn);
-    kmx = __reduce_max_sync(0xffffffffu, kmx);
-    const uint32_t mn_bits = f16_from_key(kmn), mx_bits = f16_from_key(kmx);
-    const float mn = __half2float(__ushort_as_half((unsigned short)mn_bits));
-    const float mx = __half2float(__ushort_as_half((unsigned short)mx_bits));
-    const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.f));
-    const float s = __half2float(s16);
-    uint32_t packed = 0;
-    if (s != 0.f) {
-      uint32_t n0 = nibble(v.lo, mn, s), n1 = nibble(v.lo >> 16, mn, s);
-      uint32_t n2 = nibble(v.hi, mn, s), n3 = nibble(v.hi >> 16, mn, s);
-      packed = n0 | (n1 << 4) | (n2 << 8) | (n3 << 12);
+    uint32_t sz;
+    const uint16_t packed = quantize_row_warp(load_half4(src + r * kHeadDim), &sz);
+    dst_q[r * (kHeadDim / 4)] = packed;
+    if (lane == 0) dst_sz[r] = sz;
+  }
+}
+
+// One decode step's append: CTA b writes the new token of sequence b (one warp per kv-head,
+// looping when there are more heads than warps), then advances seq_lens[b].
+__global__ void __launch_bounds__(256) k_append_token(KV kv, uint16_t* __restrict__ k_cache,
+                                                      uint16_t* __restrict__ v_cache,
+                                                      const uint16_t* __restrict__ k_new,
+                                                      const uint16_t* __restrict__ v_new,
+                                                      uint8_t* __restrict__ k_int4,
+                                                      uint16_t* __restrict__ k_sz,
+                                                      uint16_t* __restrict__ bounds,
+                                                      int32_t* seq_lens_out, uint32_t* flags) {
+  __shared__ int s_n, s_ph;
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  if (threadIdx.x == 0) {
+    const int n = kv.seq_lens[b];
+    const int j = n >> 4;
+    int ph = -1;
+    if (n >= 0 && j < kv.max_pages) ph = kv.page_table[(size_t)b * kv.max_pages + j];
+    if (ph < 0 || ph >= kv.num_phys) {
+      raise_flag(flags, TWL_FLAG_BAD_INDEX);
+      ph = -1;
     }
-    dst_q[r * (kHeadDim / 4)] = (uint16_t)packed;
-    if (lane == 0) dst_sz[r] = uint32_t(__half_as_ushort(s16)) | (mn_bits << 16);
+    s_n = n;
+    s_ph = ph;
+  }
+  __syncthreads();
+  const int n = s_n, ph = s_ph;
+  if (ph < 0) return;  // uniform over the CTA
+  const int row = n & (kPage - 1);
+  for (int h = warp; h < kv.hkv; h += nwarps) {
+    const size_t tile = ((size_t)ph * kv.hkv + h) * kPage;
+    const size_t in_off = ((size_t)b * kv.hkv + h) * kHeadDim + lane * 4;
+    const Half4 x = load_half4(k_new + in_off);
+    *reinterpret_cast<uint2*>(k_cache + (tile + row) * kHeadDim + lane * 4) = make_uint2(x.lo, x.hi);
+    *reinterpret_cast<uint2*>(v_cache + (tile + row) * kHeadDim + lane * 4) =
+        *reinterpret_cast<const uint2*>(v_new + in_off);
+    // INT4 row, as k_quantize_k writes it
+    uint32_t sz;
+    const uint16_t packed = quantize_row_warp(x, &sz);
+    reinterpret_cast<uint16_t*>(k_int4 + tile * (kHeadDim / 2))[row * (kHeadDim / 4) + lane] = packed;
+    if (lane == 0) reinterpret_cast<uint32_t*>(k_sz + tile * 2)[row] = sz;
+    // page bounds: the row itself on a fresh page, else min / max with the old bounds
+    int key[4] = {f16_key(x.lo), f16_key(x.lo >> 16), f16_key(x.hi), f16_key(x.hi >> 16)};
+    int mn[4], mx[4];
+    uint16_t* dst = bounds + (((size_t)ph * kv.hkv + h) * 2) * kHeadDim + lane * 4;
+    if (row == 0) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) mn[c] = mx[c] = key[c];
+    } else {
+      const Half4 omn = load_half4(dst), omx = load_half4(dst + kHeadDim);
+      const int okn[4] = {f16_key(omn.lo), f16_key(omn.lo >> 16), f16_key(omn.hi), f16_key(omn.hi >> 16)};
+      const int okx[4] = {f16_key(omx.lo), f16_key(omx.lo >> 16), f16_key(omx.hi), f16_key(omx.hi >> 16)};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        mn[c] = min(okn[c], key[c]);
+        mx[c] = max(okx[c], key[c]);
+      }
+    }
+    uint2 lo, hi;
+    lo.x = f16_from_key(mn[0]) | (f16_from_key(mn[1]) << 16);
+    lo.y = f16_from_key(mn[2]) | (f16_from_key(mn[3]) << 16);
+    hi.x = f16_from_key(mx[0]) | (f16_from_key(mx[1]) << 16);
+    hi.y = f16_from_key(mx[2]) | (f16_from_key(mx[3]) << 16);
+    *reinterpret_cast<uint2*>(dst) = lo;
+    *reinterpret_cast<uint2*>(dst + kHeadDim) = hi;
+  }
+  if (seq_lens_out) {
+    __syncthreads();  // every head of the token is written before the length moves
+    if (threadIdx.x == 0) seq_lens_out[b] = n + 1;
   }
 }
 
 }  // namespace
+
+cudaError_t launch_append_token(const KV& kv, uint16_t* k_cache, uint16_t* v_cache,
+                                const uint16_t* k_new, const uint16_t* v_new, uint8_t* k_int4,
+                                uint16_t* k_sz, uint16_t* bounds, int32_t* seq_lens_out,
+                                uint32_t* flags, cudaStream_t s) {
+  const int threads = kv.hkv >= 8 ? 256 : 32 * kv.hkv;
+  k_append_token<<<kv.batch, threads, 0, s>>>(kv, k_cache, v_cache, k_new, v_new, k_int4, k_sz,
+                                              bounds, seq_lens_out, flags);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_page_bounds(const KV& kv, uint16_t* bounds, uint32_t* flags, cudaStream_t s) {
   long warps = (long)kv.batch * kv.max_pages * kv.hkv;

@@ -17,6 +17,10 @@ struct KV {
 
 // twl_cache.cu
 cudaError_t launch_page_bounds(const KV& kv, uint16_t* bounds, uint32_t* flags, cudaStream_t s);
+cudaError_t launch_append_token(const KV& kv, uint16_t* k_cache, uint16_t* v_cache,
+                                const uint16_t* k_new, const uint16_t* v_new, uint8_t* k_int4,
+                                uint16_t* k_sz, uint16_t* bounds, int32_t* seq_lens_out,
+                                uint32_t* flags, cudaStream_t s);
 cudaError_t launch_quantize_k(const KV& kv, uint8_t* k_int4, uint16_t* k_sz, uint32_t* flags,
                               cudaStream_t s);
 

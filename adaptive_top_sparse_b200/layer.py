@@ -61,6 +61,11 @@ class DecodeLayer:
         twl.twl_quantize_k(self.kv, self.aux.k_int4, self.aux.k_scale_zero, self.ws, stream)
         twl.twl_page_bounds(self.kv, self.aux.bounds, self.ws, stream)
 
+    def append(self, k_new, v_new, stream=None) -> None:
+        """Append one token per sequence at position seq_lens[b] (K, V, INT4 K and page bounds
+        in one launch) and advance seq_lens.  The page for the position must be mapped."""
+        twl.twl_append_token(self.kv, self.aux, k_new, v_new, True, self.ws, stream)
+
     # ------------------------------------------------------------------ stats buffers
     def alloc_stats(self) -> dict:
         b, hq, hkv, mb = self.batch, self.num_q_heads, self.num_kv_heads, self.max_budget

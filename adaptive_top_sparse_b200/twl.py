@@ -41,7 +41,7 @@ TWL_OP_DECODE_STEP = 7
 
 EXPORTED = [
     "twl_workspace_bytes", "twl_workspace_init", "twl_device_status", "twl_status_string",
-    "twl_page_bounds", "twl_quantize_k", "twl_select_pages", "twl_estimate", "twl_prune_top_p",
+    "twl_page_bounds", "twl_quantize_k", "twl_append_token", "twl_select_pages", "twl_estimate", "twl_prune_top_p",
     "twl_group_union", "twl_sparse_decode", "twl_decode_step", "twl_noalloc_scratch_bytes",
     "twl_sparse_decode_noalloc",
 ]
@@ -78,6 +78,8 @@ _sigs = {
     "twl_status_string": (C.c_char_p, [_i32]),
     "twl_page_bounds": (_i32, [C.POINTER(_PagedKV), _vp, _vp, _sz, _vp]),
     "twl_quantize_k": (_i32, [C.POINTER(_PagedKV), _vp, _vp, _vp, _sz, _vp]),
+    "twl_append_token": (_i32, [C.POINTER(_PagedKV), C.POINTER(_KAux), _vp, _vp, _i32, _vp,
+                                _sz, _vp]),
     "twl_select_pages": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _vp, _i32, _i32, _i32, _vp, _vp,
                                 _vp, _vp, _sz, _vp]),
     "twl_estimate": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _vp, _vp, _vp, _vp, _i32, _vp, _vp,
@@ -193,6 +195,14 @@ def twl_quantize_k(kv: PagedKV, k_int4, k_scale_zero, ws=None, stream=None) -> N
     ckv = kv.c()
     _check(_lib.twl_quantize_k(C.byref(ckv), _ptr(k_int4), _ptr(k_scale_zero), _ptr(ws),
                                _nbytes(ws), _stream(stream)), "twl_quantize_k")
+
+
+def twl_append_token(kv: PagedKV, aux: "KAux", k_new, v_new, advance: bool = True, ws=None,
+                     stream=None) -> None:
+    ckv, caux = kv.c(), aux.c()
+    _check(_lib.twl_append_token(C.byref(ckv), C.byref(caux), _ptr(k_new), _ptr(v_new),
+                                 1 if advance else 0, _ptr(ws), _nbytes(ws), _stream(stream)),
+           "twl_append_token")
 
 
 def twl_select_pages(q, num_q_heads: int, kv: PagedKV, bounds, budget_pages: int,

@@ -44,12 +44,27 @@ KERNELS_PER_LAYER_STEP = 1  # twl_decode_step is one fused kernel
 FALLBACK_HBM_GBS = 6650.0
 
 
-def workload_config():
+WORKLOADS = {
+    "c2": ("GQA decode layer, batch 1, 32 q-heads / 8 kv-heads, head_dim 128, 32768-token "
+           "context, 16-token pages, Quest budget 1/4 of pages, INT4 K (group 128), p = 0.85, "
+           "eps = 1e-6, seed 0", dict(batch=1, ctx=32768)),
+    "c3": ("GQA decode layer, batch 16, 32 q-heads / 8 kv-heads, head_dim 128, contexts uniform "
+           "in [8192, 32768] tokens, pages randomly permuted, 16-token pages, Quest budget 1/4, "
+           "INT4 K, p = 0.85, eps = 1e-6, seed 0", dict(batch=16, ctx="U[8192, 32768]")),
+    "c4": ("GQA decode layer, batch 4, 32 q-heads / 8 kv-heads, head_dim 128, 131072-token "
+           "context, heavy tokens in 8 spans of 512 per head, 16-token pages, Quest budget 1/4, "
+           "INT4 K, p = 0.85, eps = 1e-6, seed 0", dict(batch=4, ctx=131072)),
+}
+
+
+def make_workload(name):
+    return {"c2": synth.config2, "c3": synth.config3, "c4": synth.config4}[name]()
+
+
+def workload_config(name="c2"):
+    text, dims = WORKLOADS[name]
     return {
-        "workload": "GQA decode layer, batch 1, 32 q-heads / 8 kv-heads, head_dim 128, "
-                    "32768-token context, 16-token pages, Quest budget 1/4 of pages, INT4 K "
-                    "(group 128), p = 0.85, eps = 1e-6, seed 0",
-        "batch": 1, "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128, "ctx": 32768,
+        "workload": text, **dims, "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128,
         "page_size": 16, "budget": "ceil(P/4) pages", "p": 0.85, "eps": 1e-6,
         "layers_per_step": LAYERS,
         "l2": f"no flush; {LAYERS} distinct layer caches per step, so each layer's touched bytes "
@@ -240,22 +255,23 @@ def max_over_ranks(x: float, world: int) -> float:
 def run_reference(args, world, rank):
     if rank != 0:
         return None
-    wl = synth.config2()
+    wl = make_workload(args.workload)
     groups = [(0, 0), (0, 1)]
     with cpu_threads_guard():
         for _ in range(args.warmup):
             oracle_sample(wl, groups[:1])
         times = [oracle_sample(wl, groups) for _ in range(args.steps)]
-    per_layer = sum(times) / len(times) * (wl.num_kv_heads / len(groups))
+    n_groups = wl.batch * wl.num_kv_heads
+    per_layer = sum(times) / len(times) * (n_groups / len(groups))
     value = 1.0 / per_layer
-    sample = (f"oracle decode path on {len(groups)} of the layer's 8 kv-head groups "
-              f"(4 q-heads each) per step, scaled x{wl.num_kv_heads // len(groups)} to one "
+    sample = (f"oracle decode path on {len(groups)} of the layer's {n_groups} (sequence, kv-head) "
+              f"groups (4 q-heads each) per step, scaled x{n_groups // len(groups)} to one "
               f"layer-step")
     return {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per_layer * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "impl": "reference", "config": workload_config(),
+        "impl": "reference", "config": workload_config(args.workload),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -267,7 +283,7 @@ def run_ours(args, world, rank, local):
     from adaptive_top_sparse_b200.layer import DecodeLayer
 
     dev = torch.device("cuda", local)
-    wl = synth.config2()
+    wl = make_workload(args.workload)
     layers = []
     for _ in range(LAYERS):
         layer = DecodeLayer.from_workload(wl, dev)
@@ -360,12 +376,14 @@ def run_ours(args, world, rank, local):
     peak, peak_kind = hbm_peak()
     layer_step_s = ms_per_step / 1e3 / LAYERS
     achieved = alg_bytes / layer_step_s / 1e9
-    traffic = measured_traffic()
+    traffic = measured_traffic() if args.workload == "c2" else None
+    metric = METRIC if args.workload == "c2" else \
+        f"decode attn layer-steps/s (select+prune+attend), workload {args.workload}; % of HBM roofline"
     out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": metric, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(),
+        "config": workload_config(args.workload),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "twl_decode_step (whole layer-step)",
@@ -387,13 +405,172 @@ def run_ours(args, world, rank, local):
         with cpu_threads_guard():
             oracle_sample(wl, wl_groups)                    # warm
             t = oracle_sample(wl, wl_groups)
-        per_layer = t * wl.num_kv_heads / len(wl_groups)
+        n_groups = wl.batch * wl.num_kv_heads
+        per_layer = t * n_groups / len(wl_groups)
         out["cpu_baseline"] = {
             "value": 1.0 / per_layer, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "oracle decode path (numpy, fp64) on 1 of the layer's 8 kv-head groups, "
-                      "scaled x8 to one layer-step; bounds/INT4 prepared untimed"}
+            "sample": f"oracle decode path (numpy, fp64) on 1 of the layer's {n_groups} "
+                      f"(sequence, kv-head) groups, scaled x{n_groups} to one layer-step; "
+                      f"bounds/INT4 prepared untimed"}
     del graph
     return out
+
+
+# ---------------------------------------------------------------------------------- append step
+
+APPEND_METRIC = "decode-step cache appends/s (K/V + INT4 K + page bounds), batch 16, 8 kv-heads"
+APPEND_UNIT = "layer-appends/s"
+
+
+def append_config():
+    return {"workload": "one decode token appended per sequence: batch 16, 8 kv-heads, head_dim "
+                        "128, 16-token pages, contexts uniform in [256, 2048] tokens, fp16 K/V",
+            "batch": 16, "num_kv_heads": 8, "head_dim": 128, "page_size": 16,
+            "layers_per_step": LAYERS,
+            "l2": "flushed (256 MiB write, outside the events) before every timed replay"}
+
+
+def append_bytes(row_is_first):
+    """Unique bytes of one append per (sequence, kv-head): new K and V rows read (512 B) and
+    written to the cache (512 B), the INT4 row and its scale/zero written (68 B), the page
+    bounds written (512 B) and, unless the row opens the page, read (512 B); plus per sequence
+    the length read and written and the page-table entry read (12 B)."""
+    per_head = 512 + 512 + 68 + 512 + (0 if row_is_first else 512)
+    return per_head
+
+
+def run_append(args, world, rank, local):
+    from adaptive_top_sparse_b200 import twl
+    dev = torch.device("cuda", local)
+    batch, hkv = 16, 8
+    gen = torch.Generator(device="cpu").manual_seed(0)
+    lens0 = torch.randint(256, 2049, (batch,), generator=gen).numpy()
+    total_appends = args.warmup + args.steps + 2
+    need = [-(-(int(n) + total_appends) // 16) for n in lens0]
+    max_pages = max(need)
+    p_phys = sum(need)
+    layers = []
+    for _ in range(LAYERS):
+        k = torch.randn((p_phys, hkv, 16, 128), dtype=torch.float16, device=dev)
+        v = torch.randn((p_phys, hkv, 16, 128), dtype=torch.float16, device=dev)
+        pt = torch.full((batch, max_pages), -1, dtype=torch.int32)
+        off = 0
+        for b, m in enumerate(need):
+            pt[b, :m] = torch.arange(off, off + m, dtype=torch.int32)
+            off += m
+        pt = pt.to(dev)
+        n = torch.from_numpy(lens0.astype(np.int32)).to(dev)
+        kv = twl.PagedKV(k, v, pt, n, hkv, p_phys)
+        aux = twl.KAux(torch.zeros((p_phys, hkv, 16, 64), dtype=torch.uint8, device=dev),
+                       torch.zeros((p_phys, hkv, 16, 2), dtype=torch.float16, device=dev),
+                       torch.zeros((p_phys, hkv, 2, 128), dtype=torch.float16, device=dev))
+        ws = twl.alloc_workspace(twl.TWL_OP_CACHE, dev)
+        twl.twl_quantize_k(kv, aux.k_int4, aux.k_scale_zero, ws)
+        twl.twl_page_bounds(kv, aux.bounds, ws)
+        kn = torch.randn((batch, hkv, 128), dtype=torch.float16, device=dev)
+        vn = torch.randn((batch, hkv, 128), dtype=torch.float16, device=dev)
+        layers.append((kv, aux, ws, kn, vn, (k, v, pt, n)))
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):                     # eager warm-up append (one token)
+        for kv, aux, ws, kn, vn, _ in layers:
+            twl.twl_append_token(kv, aux, kn, vn, True, ws, stream)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for kv, aux, ws, kn, vn, _ in layers:
+            twl.twl_append_token(kv, aux, kn, vn, True, ws, stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    done = 1 + args.warmup                              # tokens appended so far
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(world)
+    clocks.start()
+    ms = 0.0
+    nbytes = 0
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    for step in range(args.steps):
+        with torch.cuda.stream(stream):
+            flush.fill_(step & 0xFF)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+        e1.synchronize()
+        ms += e0.elapsed_time(e1)
+        for b in range(batch):
+            first = (int(lens0[b]) + done + step) % 16 == 0
+            nbytes += LAYERS * (hkv * append_bytes(first) + 12)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier(world)
+    for kv, aux, ws, kn, vn, t in layers:
+        st, fl = twl.twl_device_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device flags set: {fl}")
+        assert int(t[3][0].item()) == int(lens0[0]) + done + args.steps
+    ms_max = max_over_ranks(ms, world)
+    value = world * args.steps * LAYERS / (ms_max / 1e3)
+    peak, peak_kind = hbm_peak()
+    achieved = nbytes / (ms / 1e3) / 1e9
+    out = {
+        "metric": APPEND_METRIC, "value": value, "unit": APPEND_UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic", "config": append_config(),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "twl_append_token (k_append_token)",
+                     "alg_bytes_per_call": nbytes / (args.steps * LAYERS),
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+        "gpu_launches": args.steps * LAYERS, "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = append_oracle_sample(lens0, hkv, reps=20)
+    del graph
+    return out
+
+
+def append_oracle_sample(lens0, hkv, reps):
+    """The oracle's append (numpy) on the same batch and heads, over a cache of just the pages
+    the appended positions touch (the per-call work is the same rows)."""
+    from oracle import twl_oracle as O
+    batch = len(lens0)
+    rng = np.random.default_rng(0)
+    n = np.array([int(x) % 16 for x in lens0], np.int64)     # same rows, one page per sequence
+    pt = np.arange(batch, dtype=np.int32).reshape(batch, 1)
+    k = rng.standard_normal((batch, hkv, 16, 128)).astype(np.float16)
+    v = rng.standard_normal((batch, hkv, 16, 128)).astype(np.float16)
+    bounds = O.page_bounds(k, pt, np.maximum(n, 1))
+    q4, sz = O.quantize_k(k, pt, np.maximum(n, 1))
+    kn = rng.standard_normal((batch, hkv, 128)).astype(np.float16)
+    vn = rng.standard_normal((batch, hkv, 128)).astype(np.float16)
+    with cpu_threads_guard():
+        O.append_token(k, v, bounds, q4, sz, pt, n, kn, vn)
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            O.append_token(k, v, bounds, q4, sz, pt, n, kn, vn)
+        dt = (time.perf_counter() - t0) / reps
+    return {"value": 1.0 / dt, "unit": APPEND_UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"oracle append_token (numpy) for {batch} sequences x {hkv} kv-heads, "
+                      f"{reps} calls on a one-page-per-sequence cache"}
+
+
+def run_append_reference(args, world, rank):
+    if rank != 0:
+        return None
+    gen = torch.Generator(device="cpu").manual_seed(0)
+    lens0 = torch.randint(256, 2049, (16,), generator=gen).numpy()
+    cb = append_oracle_sample(lens0, 8, reps=max(3, args.steps))
+    return {"metric": APPEND_METRIC, "value": cb["value"], "unit": APPEND_UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 / cb["value"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": append_config(), "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": APPEND_UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
 
 
 def main():
@@ -404,15 +581,23 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layer caches per step (default 32 for c2 and append, 4 for c3 / c4)")
+    ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4", "append"],
+                    help="c2 is the headline; c3 / c4 and the append step are extra reports")
     args = ap.parse_args()
     global LAYERS
+    if args.layers is None:
+        args.layers = 4 if args.workload in ("c3", "c4") else 32
     LAYERS = max(1, args.layers)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup(args)
     try:
-        if args.impl == "reference":
+        if args.workload == "append":
+            out = (run_append_reference(args, world, rank) if args.impl == "reference"
+                   else run_append(args, world, rank, local))
+        elif args.impl == "reference":
             out = run_reference(args, world, rank)
         else:
             out = run_ours(args, world, rank, local)

@@ -147,6 +147,28 @@ twl_status twl_page_bounds(const twl_paged_kv* kv, void* bounds, void* ws, size_
 twl_status twl_quantize_k(const twl_paged_kv* kv, void* k_int4, void* k_scale_zero, void* ws,
                           size_t ws_bytes, twl_stream_t stream);
 
+/* twl_append_token: the cache maintenance of one decode step, fused with the KV append (the 4-bit
+ *   K cache and the page metadata are kept current as tokens arrive: [Summary] B.1, 4.3; [Notes]
+ *   "Key designs", 4-bit K cache).  For every sequence b with n_b = seq_lens[b], the new token
+ *   goes to logical position n_b: row n_b % 16 of physical page page_table[b][n_b / 16], which
+ *   the caller has mapped.  Per kv-head h:
+ *     K row = k_new[b][h][:], V row = v_new[b][h][:];
+ *     the INT4 row and its (scale, zero) are written exactly as twl_quantize_k writes them;
+ *     the page bounds become the K row itself when it is the page's first row (n_b % 16 == 0),
+ *     else the channel-wise min / max (total order, -0 < +0) of the old bounds and the row.
+ *   The result equals twl_page_bounds + twl_quantize_k over the extended cache, bit for bit.
+ *   If advance != 0, seq_lens[b] becomes n_b + 1 afterwards (device side, same launch).
+ *   k_new, v_new: device fp16 [batch][num_kv_heads][128], 16-byte aligned.  kv->k, kv->v and
+ *   (with advance) kv->seq_lens are written through: the caller's buffers must be writable.
+ *   A sequence whose position has no mapped page (n_b >= 16 * max_pages, or a negative or
+ *   out-of-range table entry) is left unchanged and not advanced; TWL_FLAG_BAD_INDEX is raised.
+ *   Workspace (TWL_OP_CACHE) may be NULL; it only carries the device flags.
+ *   Returns TWL_ERR_INVALID_ARG for NULL or misaligned pointers, TWL_ERR_UNSUPPORTED for shapes
+ *   the library does not support (head_dim != 128, page_size != 16). */
+twl_status twl_append_token(const twl_paged_kv* kv, const twl_k_aux* aux, const void* k_new,
+                            const void* v_new, int32_t advance, void* ws, size_t ws_bytes,
+                            twl_stream_t stream);
+
 /* ---------------------------------------------------------------- select (a1, a2)
  * Per (b, q-head h): score every page j < P_b = ceil(seq_lens[b]/16) by
  *   score_j = sum_c t_c,  t_c = q_c * max_c if q_c > 0 else q_c * min_c

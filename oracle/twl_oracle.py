@@ -161,6 +161,46 @@ def quantize_k(k, page_table, seq_lens, out_int4=None, out_sz=None):
     return q4, sz
 
 
+def append_token(k, v, bounds, q4, sz, page_table, seq_lens, k_new, v_new):
+    """One decode step of cache maintenance: sequence b's new token goes to logical position
+    n_b = seq_lens[b], i.e. row n_b % 16 of physical page page_table[b][n_b // 16].
+
+    Per kv-head: the K and V rows are written; the page's bounds become the new row itself when
+    it is the page's first row, else the channel-wise (total-order) min and max of the old bounds
+    and the row; the INT4 row and its scale / zero are ``quantize_rows`` of the row.  Then
+    seq_lens[b] = n_b + 1.  A sequence whose position has no mapped page (the table is full or
+    the entry is negative) is left unchanged.  The result equals ``page_bounds`` and
+    ``quantize_k`` recomputed over the extended cache (min and max are associative, and the
+    INT4 scheme is per row).  Returns new arrays (k, v, bounds, q4, sz, seq_lens).
+    """
+    k, v, bounds, q4, sz = (np.array(x, copy=True) for x in (k, v, bounds, q4, sz))
+    seq_lens = np.array(seq_lens, dtype=np.int64, copy=True)
+    max_pages = page_table.shape[1]
+    for b in range(len(seq_lens)):
+        n = int(seq_lens[b])
+        j, row = n // PAGE, n % PAGE
+        if j >= max_pages or int(page_table[b, j]) < 0:
+            continue
+        ph = int(page_table[b, j])
+        x = np.asarray(k_new[b], dtype=F16)                               # [Hkv][D]
+        k[ph, :, row, :] = x
+        v[ph, :, row, :] = np.asarray(v_new[b], dtype=F16)
+        if row == 0:
+            bounds[ph, :, 0, :] = x
+            bounds[ph, :, 1, :] = x
+        else:
+            mn, _ = f16_min_max(np.stack([bounds[ph, :, 0, :], x]), axis=0)
+            _, mx = f16_min_max(np.stack([bounds[ph, :, 1, :], x]), axis=0)
+            bounds[ph, :, 0, :] = mn
+            bounds[ph, :, 1, :] = mx
+        pk, s16, z16 = quantize_rows(x)
+        q4[ph, :, row, :] = pk
+        sz[ph, :, row, 0] = s16
+        sz[ph, :, row, 1] = z16
+        seq_lens[b] = n + 1
+    return k, v, bounds, q4, sz, seq_lens
+
+
 # ----------------------------------------------------------------------------------------------
 # Quest-style page scoring and top-k selection
 # ----------------------------------------------------------------------------------------------
