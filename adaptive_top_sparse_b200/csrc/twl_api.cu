@@ -283,11 +283,12 @@ twl_status twl_select_pages(const void* q, int32_t num_q_heads, const twl_paged_
   return cuda_status(e);
 }
 
-twl_status twl_estimate(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
-                        const void* k_int4, const void* k_scale_zero, const int32_t* sel_pages,
-                        const int32_t* sel_count, int32_t max_budget, float* weights,
-                        int32_t* cand_tok, int32_t* cand_count, void* ws, size_t ws_bytes,
-                        twl_stream_t stream) {
+static twl_status estimate_impl(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
+                                int bits, const void* k_int4, const void* k_scale_zero,
+                                const int32_t* sel_pages, const int32_t* sel_count,
+                                int32_t max_budget, float* weights, int32_t* cand_tok,
+                                int32_t* cand_count, void* ws, size_t ws_bytes,
+                                twl_stream_t stream) {
   KV k;
   twl_status st = check_kv(kv, false, false, &k);
   if (st != TWL_OK) return st;
@@ -304,7 +305,7 @@ twl_status twl_estimate(const void* q, int32_t num_q_heads, const twl_paged_kv* 
   cudaError_t e = launch_union_pages(num_q_heads, k, sel_pages, sel_count, max_budget, w.rank,
                                      w.union_pages, w.union_mask, w.union_npages, fl, s);
   if (e == cudaSuccess)
-    e = launch_estimate_logits(static_cast<const uint16_t*>(q), num_q_heads, k,
+    e = launch_estimate_logits(static_cast<const uint16_t*>(q), num_q_heads, k, bits,
                                static_cast<const uint8_t*>(k_int4),
                                static_cast<const uint16_t*>(k_scale_zero), w.rank, w.union_pages,
                                w.union_mask, w.union_npages, kPage * max_budget, weights,
@@ -313,6 +314,41 @@ twl_status twl_estimate(const void* q, int32_t num_q_heads, const twl_paged_kv* 
     e = launch_softmax_rows(num_q_heads, k, sel_pages, sel_count, max_budget, weights,
                             cand_count, s);
   return cuda_status(e);
+}
+
+twl_status twl_estimate(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
+                        const void* k_int4, const void* k_scale_zero, const int32_t* sel_pages,
+                        const int32_t* sel_count, int32_t max_budget, float* weights,
+                        int32_t* cand_tok, int32_t* cand_count, void* ws, size_t ws_bytes,
+                        twl_stream_t stream) {
+  return estimate_impl(q, num_q_heads, kv, 4, k_int4, k_scale_zero, sel_pages, sel_count,
+                       max_budget, weights, cand_tok, cand_count, ws, ws_bytes, stream);
+}
+
+twl_status twl_estimate_nbit(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
+                             int32_t bits, const void* k_codes, const void* k_scale_zero,
+                             const int32_t* sel_pages, const int32_t* sel_count,
+                             int32_t max_budget, float* weights, int32_t* cand_tok,
+                             int32_t* cand_count, void* ws, size_t ws_bytes,
+                             twl_stream_t stream) {
+  if (bits != 2 && bits != 4 && bits != 8) return TWL_ERR_UNSUPPORTED;
+  return estimate_impl(q, num_q_heads, kv, bits, k_codes, k_scale_zero, sel_pages, sel_count,
+                       max_budget, weights, cand_tok, cand_count, ws, ws_bytes, stream);
+}
+
+twl_status twl_quantize_k_nbit(const twl_paged_kv* kv, int32_t bits, void* k_codes,
+                               void* k_scale_zero, void* ws, size_t ws_bytes,
+                               twl_stream_t stream) {
+  if (bits != 2 && bits != 4 && bits != 8) return TWL_ERR_UNSUPPORTED;
+  KV k;
+  twl_status st = check_kv(kv, true, false, &k);
+  if (st != TWL_OK) return st;
+  if (!k_codes || !k_scale_zero || !aligned(k_codes, 16) || !aligned(k_scale_zero, 16))
+    return TWL_ERR_INVALID_ARG;
+  if (ws && (st = check_ws(ws, ws_bytes, kHeaderBytes)) != TWL_OK) return st;
+  return cuda_status(launch_quantize_k_bits(k, bits, static_cast<uint8_t*>(k_codes),
+                                            static_cast<uint16_t*>(k_scale_zero), flags_of(ws),
+                                            (cudaStream_t)stream));
 }
 
 twl_status twl_prune_top_p(const float* w, const int32_t* row_len, int32_t rows,

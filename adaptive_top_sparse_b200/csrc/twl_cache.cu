@@ -75,12 +75,74 @@ __global__ void __launch_bounds__(256) k_page_bounds(KV kv, uint16_t* __restrict
   *reinterpret_cast<uint2*>(dst + kHeadDim) = hi;
 }
 
-// One nibble: n = min(15, rint_even(fp32(x - z) / s)); x - z >= 0 because z is the row minimum.
-__device__ __forceinline__ uint32_t nibble(uint32_t xbits, float z, float s) {
+// One code: n = min(L, rint_even(fp32(x - z) / s)); x - z >= 0 because z is the row minimum.
+__device__ __forceinline__ uint32_t code_of(uint32_t xbits, float z, float s, float levels) {
   float x = __half2float(__ushort_as_half((unsigned short)(xbits & 0xFFFFu)));
   float r = rintf(__fdiv_rn(__fsub_rn(x, z), s));
-  r = fminf(fmaxf(r, 0.f), 15.f);
+  r = fminf(fmaxf(r, 0.f), levels);
   return (uint32_t)r;
+}
+__device__ __forceinline__ uint32_t nibble(uint32_t xbits, float z, float s) {
+  return code_of(xbits, z, s, 15.f);
+}
+
+// The same scheme at BITS bits (L = 2^BITS - 1 levels): the lane's 4 codes (channel c at bit
+// c * BITS of the row) and, in *sz, fp16 scale | fp16 zero << 16.
+template <int BITS>
+__device__ __forceinline__ uint32_t quantize_row_warp_bits(const uint32_t lo, const uint32_t hi,
+                                                           uint32_t* sz) {
+  constexpr float kLevels = (float)((1 << BITS) - 1);
+  int k0 = f16_key(lo), k1 = f16_key(lo >> 16), k2 = f16_key(hi), k3 = f16_key(hi >> 16);
+  int kmn = __reduce_min_sync(0xffffffffu, min(min(k0, k1), min(k2, k3)));
+  int kmx = __reduce_max_sync(0xffffffffu, max(max(k0, k1), max(k2, k3)));
+  const uint32_t mn_bits = f16_from_key(kmn), mx_bits = f16_from_key(kmx);
+  const float mn = __half2float(__ushort_as_half((unsigned short)mn_bits));
+  const float mx = __half2float(__ushort_as_half((unsigned short)mx_bits));
+  const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), kLevels));
+  const float s = __half2float(s16);
+  uint32_t packed = 0;
+  if (s != 0.f) {
+    packed = code_of(lo, mn, s, kLevels) | (code_of(lo >> 16, mn, s, kLevels) << BITS) |
+             (code_of(hi, mn, s, kLevels) << (2 * BITS)) |
+             (code_of(hi >> 16, mn, s, kLevels) << (3 * BITS));
+  }
+  *sz = uint32_t(__half_as_ushort(s16)) | (mn_bits << 16);
+  return packed;
+}
+
+// 2- and 8-bit copies of K for the estimator bit-width variants: a warp per (sequence, page,
+// kv-head), lane l writes the 4 * BITS bits of channels 4l .. 4l+3 of every row.
+template <int BITS>
+__global__ void __launch_bounds__(256) k_quantize_k_bits(KV kv, uint8_t* __restrict__ k_codes,
+                                                         uint16_t* __restrict__ k_sz,
+                                                         uint32_t* flags) {
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  int b, j, h;
+  if (!decode_warp(warp, kv, &b, &j, &h)) return;
+  Seq sq = load_seq(kv.seq_lens, b, kv.max_pages, flags, j == 0 && h == 0 && lane == 0);
+  if (j >= sq.pages) return;
+  int ph = kv.page_table[(size_t)b * kv.max_pages + j];
+  if (ph < 0 || ph >= kv.num_phys) {
+    if (lane == 0 && h == 0) raise_flag(flags, TWL_FLAG_BAD_INDEX);
+    return;
+  }
+  const int rows = page_rows(sq.n, j);
+  const size_t tile = ((size_t)ph * kv.hkv + h) * kPage;
+  const uint16_t* src = kv.k + tile * kHeadDim + lane * 4;
+  uint8_t* dst = k_codes + tile * (kHeadDim * BITS / 8) + lane * (BITS / 2);
+  uint32_t* dst_sz = reinterpret_cast<uint32_t*>(k_sz + tile * 2);
+  for (int r = 0; r < kPage; ++r) {
+    uint32_t packed = 0, sz = 0;
+    if (r < rows) {
+      const Half4 v = load_half4(src + r * kHeadDim);
+      packed = quantize_row_warp_bits<BITS>(v.lo, v.hi, &sz);
+    }
+    uint8_t* d = dst + r * (kHeadDim * BITS / 8);
+    if constexpr (BITS == 2) *d = (uint8_t)packed;
+    else *reinterpret_cast<uint32_t*>(d) = packed;
+    if (lane == 0) dst_sz[r] = sz;
+  }
 }
 
 // INT4 of one token row held by a warp (lane l: channels 4l .. 4l+3): returns the lane's 4
@@ -219,6 +281,16 @@ cudaError_t launch_append_token(const KV& kv, uint16_t* k_cache, uint16_t* v_cac
   const int threads = kv.hkv >= 8 ? 256 : 32 * kv.hkv;
   k_append_token<<<kv.batch, threads, 0, s>>>(kv, k_cache, v_cache, k_new, v_new, k_int4, k_sz,
                                               bounds, seq_lens_out, flags);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_k_bits(const KV& kv, int bits, uint8_t* k_codes, uint16_t* k_sz,
+                                   uint32_t* flags, cudaStream_t s) {
+  long warps = (long)kv.batch * kv.max_pages * kv.hkv;
+  long blocks = (warps * 32 + 255) / 256;
+  if (bits == 2) k_quantize_k_bits<2><<<(unsigned)blocks, 256, 0, s>>>(kv, k_codes, k_sz, flags);
+  else if (bits == 8) k_quantize_k_bits<8><<<(unsigned)blocks, 256, 0, s>>>(kv, k_codes, k_sz, flags);
+  else return launch_quantize_k(kv, k_codes, k_sz, flags, s);
   return cudaGetLastError();
 }
 

@@ -10,10 +10,11 @@
 // With khat = n * s + z per token row:  q . khat = s * (q . n) + z * sum(q).  The q . n products are
 // computed on the tensor cores: one 16-token page is exactly the M = 16 tile of
 // mma.m16n8k16, the 128 channels are 8 K-steps and the N = 8 columns hold the group's query heads
-// (zero-padded when the group is smaller).  Nibbles become exact fp16 integers with bit
+// (zero-padded when the group is smaller).  Codes become exact fp16 integers with bit
 // arithmetic: the binary16 pattern 0x6400 | n (exponent 10, mantissa n) is the number 1024 + n, so
-// one half2 subtraction of 1024 yields n exactly.  The mma's K index is mapped to channels so that
-// each lane's nibbles unpack with a mask and a shift; the query fragment uses the same map.
+// one half2 subtraction of 1024 yields n exactly (any n < 1024, so 2-, 4- and 8-bit codes alike).
+// The mma's K index is mapped to channels so that each lane's codes unpack with a mask and a
+// shift; the query fragment uses the same map.
 #include "twl_common.cuh"
 #include "twl_kernels.h"
 
@@ -96,18 +97,44 @@ __device__ __forceinline__ void load_q_fragments(const uint16_t* qh, bool valid,
   }
 }
 
-// Nibbles i and i+4 of a packed word as an exact fp16 pair (n_i, n_{i+4}).
-__device__ __forceinline__ uint32_t nib_pair(uint32_t x, int i) {
-  uint32_t v = ((x >> (4 * i)) & 0x000F000Fu) | 0x64006400u;
+// The values of channels ca and cb (within the lane's block of 32 channels, BITS bits each,
+// channel c at bit c * BITS) as an exact fp16 pair: 0x6400 | v is 1024 + v for v < 1024.
+template <int BITS>
+__device__ __forceinline__ uint32_t code_pair(const uint32_t (&w)[BITS], int ca, int cb) {
+  constexpr uint32_t kMask = (1u << BITS) - 1u;
+  const uint32_t va = (w[(ca * BITS) >> 5] >> ((ca * BITS) & 31)) & kMask;
+  const uint32_t vb = (w[(cb * BITS) >> 5] >> ((cb * BITS) & 31)) & kMask;
+  uint32_t v = (va | (vb << 16)) | 0x64006400u;
   const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&v), __float2half2_rn(1024.f));
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
+// The lane's 32 channels of one row: 4 * BITS bytes at byte 4 * BITS * t of the row.
+template <int BITS>
+__device__ __forceinline__ void load_codes(const uint8_t* row, int t, uint32_t (&w)[BITS]) {
+  const uint32_t* p = reinterpret_cast<const uint32_t*>(row + 4 * BITS * t);
+  if constexpr (BITS == 2) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    w[0] = v.x;
+    w[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < BITS; i += 4) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p + i));
+      w[i] = v.x;
+      w[i + 1] = v.y;
+      w[i + 2] = v.z;
+      w[i + 3] = v.w;
+    }
+  }
+}
+
 // grid (ceil(max_pages / 32), Hkv, B).  Each warp handles union pages of group (b, kvh).
-template <int G>
+// BITS = 4 is the INT4 copy; 2 and 8 are the estimator bit-width variants (same scheme).
+template <int G, int BITS>
 __global__ void __launch_bounds__(kEstThreads)
     k_estimate_logits(const uint16_t* __restrict__ q, int hq, KV kv,
-                      const uint8_t* __restrict__ k_int4, const uint16_t* __restrict__ k_sz,
+                      const uint8_t* __restrict__ k_codes, const uint16_t* __restrict__ k_sz,
                       const int* __restrict__ rank, const int* __restrict__ union_pages,
                       const uint32_t* __restrict__ union_mask,
                       const int* __restrict__ union_npages, int cand_stride,
@@ -147,27 +174,27 @@ __global__ void __launch_bounds__(kEstThreads)
     const uint32_t hm = union_mask[ubase + u];
     const int ph = load_phys(kv.page_table, b, j, kv.max_pages, kv.num_phys, flags);
     const bool bad = ph < 0;  // warp-uniform: its candidates get logit -inf
-    uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
+    uint32_t r0[BITS], r1[BITS];
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) r0[i] = r1[i] = 0u;
     uint32_t sz0 = 0, sz1 = 0;
     if (!bad) {
       const size_t tile = ((size_t)ph * kv.hkv + kvh) * kPage;
-      const uint4* src = reinterpret_cast<const uint4*>(k_int4 + tile * (kHeadDim / 2));
-      x0 = __ldg(src + lane);       // row gr,     bytes 16t .. 16t+15
-      x1 = __ldg(src + 32 + lane);  // row gr + 8
+      const uint8_t* src = k_codes + tile * (kHeadDim * BITS / 8);
+      load_codes<BITS>(src + gr * (kHeadDim * BITS / 8), t, r0);        // row gr
+      load_codes<BITS>(src + (gr + 8) * (kHeadDim * BITS / 8), t, r1);  // row gr + 8
       sz0 = __ldg(reinterpret_cast<const uint32_t*>(k_sz + tile * 2) + gr);
       sz1 = __ldg(reinterpret_cast<const uint32_t*>(k_sz + tile * 2) + gr + 8);
     }
-    const uint32_t r0[4] = {x0.x, x0.y, x0.z, x0.w};
-    const uint32_t r1[4] = {x1.x, x1.y, x1.z, x1.w};
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const int w8 = ks >> 1, e = ks & 1;
+      const int c0 = 8 * (ks >> 1) + 2 * (ks & 1);
       uint32_t a[4];
-      a[0] = nib_pair(r0[w8], 2 * e);      // row gr,   K cols 2t, 2t+1
-      a[1] = nib_pair(r1[w8], 2 * e);      // row gr+8
-      a[2] = nib_pair(r0[w8], 2 * e + 1);  // row gr,   K cols 2t+8, 2t+9
-      a[3] = nib_pair(r1[w8], 2 * e + 1);  // row gr+8
+      a[0] = code_pair<BITS>(r0, c0, c0 + 4);      // row gr,   K cols 2t, 2t+1
+      a[1] = code_pair<BITS>(r1, c0, c0 + 4);      // row gr+8
+      a[2] = code_pair<BITS>(r0, c0 + 1, c0 + 5);  // row gr,   K cols 2t+8, 2t+9
+      a[3] = code_pair<BITS>(r1, c0 + 1, c0 + 5);  // row gr+8
       mma_16816(acc, a, bf[ks][0], bf[ks][1]);
     }
     const int rows = page_rows(sq.n, j);
@@ -243,24 +270,31 @@ cudaError_t launch_union_pages(int hq, const KV& kv, const int* sel_pages, const
   return cudaGetLastError();
 }
 
-cudaError_t launch_estimate_logits(const uint16_t* q, int hq, const KV& kv,
-                                   const uint8_t* k_int4, const uint16_t* k_sz, const int* rank,
+cudaError_t launch_estimate_logits(const uint16_t* q, int hq, const KV& kv, int bits,
+                                   const uint8_t* k_codes, const uint16_t* k_sz, const int* rank,
                                    const int* union_pages, const uint32_t* union_mask,
                                    const int* union_npages, int cand_stride, float* logits,
                                    int* cand_tok, uint32_t* flags, cudaStream_t s) {
   const int g = hq / kv.hkv;
   dim3 grid((kv.max_pages + kEstPagesPerBlock - 1) / kEstPagesPerBlock, kv.hkv, kv.batch);
-#define TWL_EST(G)                                                                          \
-  k_estimate_logits<G><<<grid, kEstThreads, 0, s>>>(q, hq, kv, k_int4, k_sz, rank,          \
-                                                    union_pages, union_mask, union_npages,  \
-                                                    cand_stride, logits, cand_tok, flags)
-  switch (g) {
-    case 1: TWL_EST(1); break;
-    case 2: TWL_EST(2); break;
-    case 4: TWL_EST(4); break;
-    case 8: TWL_EST(8); break;
-    default: return cudaErrorInvalidValue;
+#define TWL_EST(G, B)                                                                         \
+  k_estimate_logits<G, B><<<grid, kEstThreads, 0, s>>>(q, hq, kv, k_codes, k_sz, rank,        \
+                                                       union_pages, union_mask, union_npages, \
+                                                       cand_stride, logits, cand_tok, flags)
+#define TWL_EST_G(B)               \
+  switch (g) {                     \
+    case 1: TWL_EST(1, B); break;  \
+    case 2: TWL_EST(2, B); break;  \
+    case 4: TWL_EST(4, B); break;  \
+    case 8: TWL_EST(8, B); break;  \
+    default: return cudaErrorInvalidValue; \
   }
+  switch (bits) {
+    case 2: TWL_EST_G(2); break;
+    case 8: TWL_EST_G(8); break;
+    default: TWL_EST_G(4); break;
+  }
+#undef TWL_EST_G
 #undef TWL_EST
   return cudaGetLastError();
 }

@@ -23,6 +23,8 @@ cudaError_t launch_append_token(const KV& kv, uint16_t* k_cache, uint16_t* v_cac
                                 uint32_t* flags, cudaStream_t s);
 cudaError_t launch_quantize_k(const KV& kv, uint8_t* k_int4, uint16_t* k_sz, uint32_t* flags,
                               cudaStream_t s);
+cudaError_t launch_quantize_k_bits(const KV& kv, int bits, uint8_t* k_codes, uint16_t* k_sz,
+                                   uint32_t* flags, cudaStream_t s);
 
 // twl_select.cu
 cudaError_t launch_page_scores(const uint16_t* q, int hq, const KV& kv, const uint16_t* bounds,
@@ -36,8 +38,8 @@ cudaError_t launch_union_pages(int hq, const KV& kv, const int* sel_pages, const
                                int max_budget, int* rank, int* union_pages,
                                uint32_t* union_mask, int* union_npages, uint32_t* flags,
                                cudaStream_t s);
-cudaError_t launch_estimate_logits(const uint16_t* q, int hq, const KV& kv,
-                                   const uint8_t* k_int4, const uint16_t* k_sz, const int* rank,
+cudaError_t launch_estimate_logits(const uint16_t* q, int hq, const KV& kv, int bits,
+                                   const uint8_t* k_codes, const uint16_t* k_sz, const int* rank,
                                    const int* union_pages, const uint32_t* union_mask,
                                    const int* union_npages, int cand_stride, float* logits,
                                    int* cand_tok, uint32_t* flags, cudaStream_t s);

@@ -41,7 +41,8 @@ TWL_OP_DECODE_STEP = 7
 
 EXPORTED = [
     "twl_workspace_bytes", "twl_workspace_init", "twl_device_status", "twl_status_string",
-    "twl_page_bounds", "twl_quantize_k", "twl_append_token", "twl_select_pages", "twl_estimate", "twl_prune_top_p",
+    "twl_page_bounds", "twl_quantize_k", "twl_append_token", "twl_quantize_k_nbit",
+    "twl_estimate_nbit", "twl_select_pages", "twl_estimate", "twl_prune_top_p",
     "twl_group_union", "twl_sparse_decode", "twl_decode_step", "twl_noalloc_scratch_bytes",
     "twl_sparse_decode_noalloc",
 ]
@@ -84,6 +85,9 @@ _sigs = {
                                 _vp, _vp, _sz, _vp]),
     "twl_estimate": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _vp, _vp, _vp, _vp, _i32, _vp, _vp,
                             _vp, _vp, _sz, _vp]),
+    "twl_quantize_k_nbit": (_i32, [C.POINTER(_PagedKV), _i32, _vp, _vp, _vp, _sz, _vp]),
+    "twl_estimate_nbit": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _i32, _vp, _vp, _vp, _vp, _i32,
+                                 _vp, _vp, _vp, _vp, _sz, _vp]),
     "twl_prune_top_p": (_i32, [_vp, _vp, _i32, _i32, _f32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "twl_group_union": (_i32, [_i32, C.POINTER(_PagedKV), _vp, _vp, _vp, _i32, _vp, _vp, _vp,
                                _sz, _vp]),
@@ -222,6 +226,24 @@ def twl_estimate(q, num_q_heads: int, kv: PagedKV, k_int4, k_scale_zero, sel_pag
                              _ptr(k_scale_zero), _ptr(sel_pages), _ptr(sel_count), max_budget,
                              _ptr(weights), _ptr(cand_tok), _ptr(cand_count), _ptr(ws),
                              _nbytes(ws), _stream(stream)), "twl_estimate")
+
+
+def twl_quantize_k_nbit(kv: PagedKV, bits: int, k_codes, k_scale_zero, ws=None,
+                        stream=None) -> None:
+    ckv = kv.c()
+    _check(_lib.twl_quantize_k_nbit(C.byref(ckv), bits, _ptr(k_codes), _ptr(k_scale_zero),
+                                    _ptr(ws), _nbytes(ws), _stream(stream)),
+           "twl_quantize_k_nbit")
+
+
+def twl_estimate_nbit(q, num_q_heads: int, kv: PagedKV, bits: int, k_codes, k_scale_zero,
+                      sel_pages, sel_count, max_budget: int, weights, cand_tok, cand_count,
+                      ws=None, stream=None) -> None:
+    ckv = kv.c()
+    _check(_lib.twl_estimate_nbit(_ptr(q), num_q_heads, C.byref(ckv), bits, _ptr(k_codes),
+                                  _ptr(k_scale_zero), _ptr(sel_pages), _ptr(sel_count),
+                                  max_budget, _ptr(weights), _ptr(cand_tok), _ptr(cand_count),
+                                  _ptr(ws), _nbytes(ws), _stream(stream)), "twl_estimate_nbit")
 
 
 def twl_prune_top_p(w, row_len, rows: int, row_stride: int, p: float, eps: float, m_out,

@@ -573,6 +573,103 @@ def run_append_reference(args, world, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+# ---------------------------------------------------------------------------------- bit widths
+
+def run_bits(args, world, rank, local):
+    """The staged estimate (union, dequant-dot, softmax) on the 32K-context layer at 2, 4 and 8
+    bits (survey row f2): time per call, and the roofline over the codes + scale/zero of the
+    groups' union pages (16 rows x (16 bits + 4) bytes per page per kv-head)."""
+    from adaptive_top_sparse_b200 import twl
+    from adaptive_top_sparse_b200.layer import DecodeLayer
+    dev = torch.device("cuda", local)
+    wl = synth.config2()
+    b, hq, hkv = wl.batch, wl.num_q_heads, wl.num_kv_heads
+    layers = []
+    for _ in range(LAYERS):
+        layer = DecodeLayer.from_workload(wl, dev)
+        layer.build_aux()
+        mb = layer.max_budget
+        sel = torch.full((b, hq, mb), -1, dtype=torch.int32, device=dev)
+        cnt = torch.zeros((b, hq), dtype=torch.int32, device=dev)
+        ws = twl.alloc_workspace(twl.TWL_OP_ESTIMATE, dev, batch=b, num_q_heads=hq,
+                                 num_kv_heads=hkv, max_pages=layer.max_pages, max_budget=mb)
+        wss = twl.alloc_workspace(twl.TWL_OP_SELECT, dev, batch=b, num_q_heads=hq,
+                                  num_kv_heads=hkv, max_pages=layer.max_pages)
+        q = torch.from_numpy(wl.q).to(dev)
+        twl.twl_select_pages(q, hq, layer.kv, layer.aux.bounds, 0, wl.budget_div, mb, sel, cnt,
+                             None, wss)
+        out = (torch.zeros((b, hq, 16 * mb), dtype=torch.float32, device=dev),
+               torch.zeros((b, hq, 16 * mb), dtype=torch.int32, device=dev),
+               torch.zeros((b, hq), dtype=torch.int32, device=dev))
+        codes = {}
+        for bits in (2, 4, 8):
+            kq = torch.zeros((layer.k.shape[0], hkv, 16, 16 * bits), dtype=torch.uint8,
+                             device=dev)
+            sz = torch.zeros((layer.k.shape[0], hkv, 16, 2), dtype=torch.float16, device=dev)
+            twl.twl_quantize_k_nbit(layer.kv, bits, kq, sz, ws)
+            codes[bits] = (kq, sz)
+        layers.append((layer, q, sel, cnt, ws, out, codes))
+    torch.cuda.synchronize(dev)
+    seln, cntn = layers[0][2].cpu().numpy(), layers[0][3].cpu().numpy()
+    union_pages = 0
+    g = hq // hkv
+    for kvh in range(hkv):
+        pages = set()
+        for h in range(kvh * g, (kvh + 1) * g):
+            pages.update(seln[0, h, :cntn[0, h]].tolist())
+        union_pages += len(pages)
+    stream = torch.cuda.Stream(dev)
+    peak, peak_kind = hbm_peak()
+    variants = {}
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    clocks.start()
+    for bits in (2, 4, 8):
+        def step():
+            for layer, q, sel, cnt, ws, (w, tok, cc), codes in layers:
+                kq, sz = codes[bits]
+                twl.twl_estimate_nbit(q, hq, layer.kv, bits, kq, sz, sel, cnt, layer.max_budget,
+                                      w, tok, cc, ws, stream)
+        with torch.cuda.stream(stream):
+            step()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (args.steps * LAYERS)
+        nbytes = union_pages * 16 * (16 * bits + 4)
+        variants[str(bits)] = {"us_per_layer": us, "layer_steps_per_s": 1e6 / us,
+                               "alg_bytes": nbytes, "achieved_gbs": nbytes / us / 1e3,
+                               "frac": nbytes / us / 1e3 / peak}
+        del graph
+    clk = clocks.stop()
+    v4 = variants["4"]
+    return {
+        "metric": "staged estimate layer-steps/s (union + dequant-dot + softmax), 32K-context "
+                  "layer, INT4 (2- and 8-bit variants beside it)",
+        "value": v4["layer_steps_per_s"], "unit": "layer-steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": v4["us_per_layer"] * LAYERS / 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": workload_config("c2"),
+        "roofline": {"bound": "hbm", "achieved": v4["achieved_gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": v4["frac"], "traffic": None,
+                     "kernel": "twl_estimate_nbit (3 launches)",
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+        "variants": variants, "union_pages": union_pages, "clocks": clk,
+        "gpu_launches": 3 * 3 * args.steps * LAYERS,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -583,7 +680,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="layer caches per step (default 32 for c2 and append, 4 for c3 / c4)")
-    ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4", "append"],
+    ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4", "append", "bits"],
                     help="c2 is the headline; c3 / c4 and the append step are extra reports")
     args = ap.parse_args()
     global LAYERS
@@ -594,7 +691,9 @@ def main():
         args.warmup = 3
     world, rank, local = dist_setup(args)
     try:
-        if args.workload == "append":
+        if args.workload == "bits":
+            out = run_bits(args, world, rank, local) if args.impl == "ours" else None
+        elif args.workload == "append":
             out = (run_append_reference(args, world, rank) if args.impl == "reference"
                    else run_append(args, world, rank, local))
         elif args.impl == "reference":

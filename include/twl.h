@@ -203,6 +203,26 @@ twl_status twl_estimate(const void* q, int32_t num_q_heads, const twl_paged_kv* 
                         int32_t* cand_tok, int32_t* cand_count, void* ws, size_t ws_bytes,
                         twl_stream_t stream);
 
+/* ---------------------------------------------------------------- estimator bit widths (f2)
+ * The estimator ablation ([Notes] "Key designs": a 4-bit K cache suffices for the weight
+ * estimate; [Summary] 4.3 and its bit-width figures): the INT4 scheme of twl_quantize_k at
+ * bits = 2 or 8 (bits = 4 is exactly twl_quantize_k / twl_estimate).  Per token row:
+ * L = 2^bits - 1, s = fp16_rn(fp32(max - min) / L), z = min,
+ * n_c = min(L, rint_even(fp32(x_c - z) / s)) (n_c = 0 when s = 0); channel c occupies bits
+ * [c*bits, (c+1)*bits) of the row, from the low bit of byte 0.
+ *   twl_quantize_k_nbit: k_codes uint8 [P][Hkv][16][128*bits/8], k_scale_zero as twl_quantize_k.
+ *   twl_estimate_nbit: twl_estimate reading that copy (workspace TWL_OP_ESTIMATE).
+ * bits outside {2, 4, 8} returns TWL_ERR_UNSUPPORTED; other errors as the INT4 calls. */
+twl_status twl_quantize_k_nbit(const twl_paged_kv* kv, int32_t bits, void* k_codes,
+                               void* k_scale_zero, void* ws, size_t ws_bytes,
+                               twl_stream_t stream);
+twl_status twl_estimate_nbit(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
+                             int32_t bits, const void* k_codes, const void* k_scale_zero,
+                             const int32_t* sel_pages, const int32_t* sel_count,
+                             int32_t max_budget, float* weights, int32_t* cand_tok,
+                             int32_t* cand_count, void* ws, size_t ws_bytes,
+                             twl_stream_t stream);
+
 /* ---------------------------------------------------------------- prune (a5)
  * Per row r of w (float [rows][row_stride], row length row_len[r] or row_stride if row_len is
  * NULL, weights >= 0 summing to ~1): bisection on the threshold m ([Notes] "Key designs",

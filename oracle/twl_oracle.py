@@ -370,6 +370,91 @@ def estimate_head(q16, k_int4, k_sz, page_table, b, kvh, n, sel_pages, head_dim=
     return cand, softmax64(logits)
 
 
+# ----------------------------------------------------------------------------------------------
+# Estimator bit widths ([Notes] "Key designs": the 4-bit K cache, and lower / higher precisions
+# compared in the ablation; [Summary] 4.3 and the bit-width figures): the same per-row
+# asymmetric scheme with L = 2^bits - 1 levels.
+# ----------------------------------------------------------------------------------------------
+
+def quantize_rows_bits(x16: np.ndarray, bits: int):
+    """Token rows (fp16 [R][D]) -> (packed uint8 [R][D*bits/8], scale fp16 [R], zero fp16 [R]).
+
+    s = fp16(fp32(max - min) / L), z = min, n_c = clamp(rint_even(fp32(x_c - z) / s), 0, L)
+    (n_c = 0 when s = 0), L = 2^bits - 1.  Channel c occupies bits [c*bits, (c+1)*bits) of the
+    row, counted from the low bit of byte 0 (for bits = 4: channel 2j in the low nibble of
+    byte j, as ``quantize_rows``)."""
+    assert bits in (2, 4, 8)
+    levels = (1 << bits) - 1
+    x16 = np.asarray(x16, dtype=F16)
+    mn, mx = f16_min_max(x16, axis=1)
+    s16 = ((mx.astype(F32) - mn.astype(F32)) / F32(levels)).astype(F16)
+    s32 = s16.astype(F32)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = np.rint((x16.astype(F32) - mn.astype(F32)[:, None]) / s32)
+    r = np.where(s32 == F32(0.0), F32(0.0), r)
+    n = np.clip(r, 0, levels).astype(np.uint64)
+    per = 8 // bits                                    # values per byte
+    rows, d = n.shape
+    packed = np.zeros((rows, d // per), dtype=np.uint64)
+    for i in range(per):
+        packed |= n[:, i::per] << np.uint64(bits * i)
+    return packed.astype(np.uint8), s16, mn
+
+
+def unpack_rows_bits(packed: np.ndarray, bits: int) -> np.ndarray:
+    packed = np.asarray(packed, dtype=np.uint8).astype(np.int64)
+    per = 8 // bits
+    mask = (1 << bits) - 1
+    out = np.empty(packed.shape[:-1] + (packed.shape[-1] * per,), dtype=np.int64)
+    for i in range(per):
+        out[..., i::per] = (packed >> (bits * i)) & mask
+    return out
+
+
+def quantize_k_bits(k, page_table, seq_lens, bits: int):
+    """``quantize_k`` at another bit width: (uint8 [P][Hkv][16][D*bits/8], fp16 [P][Hkv][16][2])."""
+    p_phys, hkv, page, d = k.shape
+    q = np.zeros((p_phys, hkv, page, d * bits // 8), dtype=np.uint8)
+    sz = np.zeros((p_phys, hkv, page, 2), dtype=F16)
+    for b in range(len(seq_lens)):
+        n = int(seq_lens[b])
+        pb = num_pages(n)
+        phys = np.asarray(page_table[b, :pb], dtype=np.int64)
+        pk, s16, z16 = quantize_rows_bits(k[phys].reshape(-1, d), bits)
+        pk = pk.reshape(pb, hkv, page, -1)
+        s16 = s16.reshape(pb, hkv, page)
+        z16 = z16.reshape(pb, hkv, page)
+        r_valid = n - PAGE * (pb - 1)
+        pk[pb - 1, :, r_valid:] = 0
+        s16[pb - 1, :, r_valid:] = F16(0.0)
+        z16[pb - 1, :, r_valid:] = F16(0.0)
+        q[phys] = pk
+        sz[phys, :, :, 0] = s16
+        sz[phys, :, :, 1] = z16
+    return q, sz
+
+
+def estimate_head_bits(q16, k_q, k_sz, page_table, b, kvh, n, sel_pages, bits, head_dim=128):
+    """``estimate_head`` from the ``bits``-wide copy of K: khat = n*s + z, fp64 logits."""
+    cand = candidates(sel_pages, n)
+    if cand.size == 0:
+        return cand, np.zeros(0)
+    packed = gather_tokens(k_q, page_table, b, kvh, cand)
+    sz = gather_tokens(k_sz, page_table, b, kvh, cand)
+    khat = unpack_rows_bits(packed, bits).astype(F64) * sz[:, 0:1].astype(F64) \
+        + sz[:, 1:2].astype(F64)
+    logits = (khat @ np.asarray(q16, dtype=F16).astype(F64)) / math.sqrt(head_dim)
+    return cand, softmax64(logits)
+
+
+def exact_weights(q16, k, page_table, b, kvh, cand, head_dim=128):
+    """Softmax of the exact q.k / sqrt(D) (fp16 K, fp64 arithmetic) over the candidates: the
+    weights the estimate stands in for."""
+    kk = gather_tokens(k, page_table, b, kvh, cand).astype(F64)
+    logits = (kk @ np.asarray(q16, dtype=F16).astype(F64)) / math.sqrt(head_dim)
+    return softmax64(logits)
+
+
 def decode_step(wl, bounds=None, k_int4=None, k_sz=None, with_attention=True):
     """Full oracle pass of select -> estimate -> top-p -> group union -> attention.
 

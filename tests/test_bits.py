@@ -1,0 +1,224 @@
+"""Estimator bit widths (survey row f2): the INT4 scheme at 2 and 8 bits, and the ablation's
+weight-mass check (the exact weights' mass over the set kept from the estimate, against p).
+
+CPU: the oracle's bit-width restatement is pinned to the INT4 path at 4 bits, to hand-worked
+exact-grid rows at 2 and 8 bits, and to the quantisation error bound; the C entry points reject
+unsupported widths.  GPU: bit-exact codes, weights against the oracle, and the ablation on the
+32K-context heads.
+"""
+import ctypes as C
+
+import numpy as np
+import pytest
+
+from oracle import twl_oracle as O
+from tests.twl_checks import W_ATOL, W_RTOL, group_workload
+from workloads import synth
+
+D = 128
+
+
+def u16(x):
+    return np.ascontiguousarray(x).view(np.uint16)
+
+
+def test_four_bits_is_the_int4_path():
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((64, D)).astype(np.float16)
+    x[3] = np.float16(1.5)                      # a constant row: s = 0, all codes 0
+    a, b = O.quantize_rows(x), O.quantize_rows_bits(x, 4)
+    assert np.array_equal(a[0], b[0])
+    assert np.array_equal(u16(a[1]), u16(b[1])) and np.array_equal(u16(a[2]), u16(b[2]))
+    wl = synth.make_decode("bits4", 1, 4, 1, [700], seed=3)
+    bounds = O.page_bounds(wl.k, wl.page_table, wl.seq_lens)
+    sel = O.select_pages(wl.q, bounds, wl.page_table, wl.seq_lens, 4, 1, 0, 4)
+    q4, sz = O.quantize_k(wl.k, wl.page_table, wl.seq_lens)
+    qb, szb = O.quantize_k_bits(wl.k, wl.page_table, wl.seq_lens, 4)
+    assert np.array_equal(q4, qb) and np.array_equal(u16(sz), u16(szb))
+    for h in range(4):
+        pages = sel[(0, h)][1]
+        c1, w1 = O.estimate_head(wl.q[0, h], q4, sz, wl.page_table, 0, 0, 700, pages)
+        c2, w2 = O.estimate_head_bits(wl.q[0, h], qb, szb, wl.page_table, 0, 0, 700, pages, 4)
+        assert np.array_equal(c1, c2) and np.array_equal(w1, w2)
+
+
+def test_exact_grid_rows_by_hand():
+    # 2 bits: x_c = (c mod 4) / 2 -> min 0, max 1.5, s = 0.5, codes c mod 4; byte j holds
+    # channels 4j .. 4j+3 from the low bits: 0 | 1 << 2 | 2 << 4 | 3 << 6 = 0xE4
+    x = (np.arange(D) % 4 / 2).astype(np.float16)[None]
+    pk, s, z = O.quantize_rows_bits(x, 2)
+    assert pk.shape == (1, 32) and np.all(pk == 0xE4)
+    assert float(s[0]) == 0.5 and float(z[0]) == 0.0
+    # 8 bits: x_c = n_c / 64 with n_0 = 0 and n_1 = 255 -> s = 1/64 exactly, bytes = n_c
+    n = (37 * np.arange(D) + 11) % 256
+    n[0], n[1] = 0, 255
+    x = (n / 64).astype(np.float16)[None]
+    pk, s, z = O.quantize_rows_bits(x, 8)
+    assert np.array_equal(pk[0], n.astype(np.uint8)) and float(s[0]) == 1 / 64
+    assert np.array_equal(O.unpack_rows_bits(pk, 8)[0], n)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_reconstruction_within_half_a_step(bits):
+    rng = np.random.default_rng(bits)
+    x = (rng.standard_normal((200, D)) * rng.uniform(0.01, 10, (200, 1))).astype(np.float16)
+    pk, s, z = O.quantize_rows_bits(x, bits)
+    levels = (1 << bits) - 1
+    khat = O.unpack_rows_bits(pk, bits) * s.astype(np.float64)[:, None] + \
+        z.astype(np.float64)[:, None]
+    xf = x.astype(np.float64)
+    s64 = s.astype(np.float64)
+    exact_step = (xf.max(1) - xf.min(1)) / levels
+    bound = s64 / 2 + levels * np.abs(exact_step - s64) + 1e-12   # the top code may clamp
+    assert np.all(np.abs(khat - xf).max(1) <= bound)
+    codes = O.unpack_rows_bits(pk, bits)
+    assert codes.min() >= 0 and codes.max() <= levels
+
+
+def test_nbit_calls_reject_unsupported_widths():
+    from adaptive_top_sparse_b200 import twl
+    A = 1 << 20
+    kv = twl._PagedKV(A, A + 4096, A + 8192, A + 12288, 2, 8, 128, 16, 64, 128)
+    for bits in (0, 1, 3, 16):
+        assert twl._lib.twl_quantize_k_nbit(C.byref(kv), bits, A, A, None, 0,
+                                            None) == twl.TWL_ERR_UNSUPPORTED
+        assert twl._lib.twl_estimate_nbit(A, 32, C.byref(kv), bits, A, A, A, A, 16, A, A, A, A,
+                                          1 << 30, None) == twl.TWL_ERR_UNSUPPORTED
+    assert twl._lib.twl_quantize_k_nbit(C.byref(kv), 2, A + 4, A, None, 0,
+                                        None) == twl.TWL_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------ GPU
+
+def _device(wl):
+    from adaptive_top_sparse_b200.layer import DecodeLayer
+    layer = DecodeLayer.from_workload(wl)
+    layer.build_aux()
+    return layer
+
+
+def _codes_on_device(layer, bits):
+    import torch
+    from adaptive_top_sparse_b200 import twl
+    p_phys = layer.k.shape[0]
+    kq = torch.zeros((p_phys, layer.num_kv_heads, 16, D * bits // 8), dtype=torch.uint8,
+                     device=layer.device)
+    sz = torch.zeros((p_phys, layer.num_kv_heads, 16, 2), dtype=torch.float16, device=layer.device)
+    twl.twl_quantize_k_nbit(layer.kv, bits, kq, sz, layer.ws)
+    return kq, sz
+
+
+def _estimate_on_device(layer, wl, bits, kq, sz, sel, cnt):
+    import torch
+    from adaptive_top_sparse_b200 import twl
+    dev = layer.device
+    b, hq, mb = wl.batch, wl.num_q_heads, layer.max_budget
+    w = torch.zeros((b, hq, 16 * mb), dtype=torch.float32, device=dev)
+    tok = torch.full((b, hq, 16 * mb), -1, dtype=torch.int32, device=dev)
+    cc = torch.zeros((b, hq), dtype=torch.int32, device=dev)
+    ws = twl.alloc_workspace(twl.TWL_OP_ESTIMATE, dev, batch=b, num_q_heads=hq,
+                             num_kv_heads=wl.num_kv_heads, max_pages=wl.page_table.shape[1],
+                             max_budget=mb)
+    q = torch.from_numpy(wl.q).to(dev)
+    twl.twl_estimate_nbit(q, hq, layer.kv, bits, kq, sz, sel, cnt, mb, w, tok, cc, ws)
+    return w, tok, cc
+
+
+def _select_on_device(layer, wl):
+    import torch
+    from adaptive_top_sparse_b200 import twl
+    dev = layer.device
+    b, hq, mb = wl.batch, wl.num_q_heads, layer.max_budget
+    sel = torch.full((b, hq, mb), -1, dtype=torch.int32, device=dev)
+    cnt = torch.zeros((b, hq), dtype=torch.int32, device=dev)
+    ws = twl.alloc_workspace(twl.TWL_OP_SELECT, dev, batch=b, num_q_heads=hq,
+                             num_kv_heads=wl.num_kv_heads, max_pages=wl.page_table.shape[1])
+    q = torch.from_numpy(wl.q).to(dev)
+    twl.twl_select_pages(q, hq, layer.kv, layer.aux.bounds, wl.budget_pages, wl.budget_div, mb,
+                         sel, cnt, None, ws)
+    return sel, cnt
+
+
+@pytest.fixture(scope="module")
+def small():
+    wl = synth.make_decode("bits_small", 3, 16, 4, [2001, 777, 16], seed=21, permute_pages=True)
+    return wl, _device(wl)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("bits", [2, 8])
+def test_quantize_nbit_bit_exact(small, bits):
+    wl, layer = small
+    kq, sz = _codes_on_device(layer, bits)
+    rq, rs = O.quantize_k_bits(wl.k, wl.page_table, wl.seq_lens, bits)
+    ref = np.array(sorted({int(p) for b in range(wl.batch)
+                           for p in wl.page_table[b, :O.num_pages(int(wl.seq_lens[b]))]}))
+    assert np.array_equal(kq.cpu().numpy()[ref], rq[ref])
+    assert np.array_equal(u16(sz.cpu().numpy()[ref]), u16(rs[ref]))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_estimate_nbit_vs_oracle(small, bits):
+    wl, layer = small
+    kq, sz = _codes_on_device(layer, bits)
+    sel, cnt = _select_on_device(layer, wl)
+    w, tok, cc = _estimate_on_device(layer, wl, bits, kq, sz, sel, cnt)
+    rq, rs = O.quantize_k_bits(wl.k, wl.page_table, wl.seq_lens, bits)
+    seln, cntn, wn, tokn, ccn = (x.cpu().numpy() for x in (sel, cnt, w, tok, cc))
+    g = wl.num_q_heads // wl.num_kv_heads
+    for b in range(wl.batch):
+        n = int(wl.seq_lens[b])
+        for h in range(wl.num_q_heads):
+            pages = seln[b, h, :cntn[b, h]]
+            cand, w_or = O.estimate_head_bits(wl.q[b, h], rq, rs, wl.page_table, b, h // g, n,
+                                              pages, bits)
+            c = int(ccn[b, h])
+            assert c == cand.size and np.array_equal(tokn[b, h, :c], cand)
+            assert np.all(np.abs(wn[b, h, :c] - w_or) <= W_RTOL * w_or + W_ATOL), (b, h, bits)
+
+
+@pytest.mark.gpu
+def test_bitwidth_mass_ablation():
+    """The exact weights' mass over the set the device keeps from each estimate (device
+    estimate, device bisection), on 4 of the 32K-context layer's groups (16 heads).  On the
+    oracle these heads give mean masses 0.43 / 0.83 / 0.86 at 2 / 4 / 8 bits for p = 0.85
+    (0.86 with exact weights): 4 bits holds the mass near p, 2 bits does not."""
+    import torch
+    from adaptive_top_sparse_b200 import twl
+    wl = synth.config2()
+    layer = _device(wl)
+    sel, cnt = _select_on_device(layer, wl)
+    seln, cntn = sel.cpu().numpy(), cnt.cpu().numpy()
+    n = int(wl.seq_lens[0])
+    g = wl.num_q_heads // wl.num_kv_heads
+    groups = [0, 2, 5, 7]
+    exact = {}
+    for kvh in groups:
+        for hl in range(g):
+            h = kvh * g + hl
+            cand = O.candidates(seln[0, h, :cntn[0, h]], n)
+            exact[h] = (cand, O.exact_weights(wl.q[0, h], wl.k, wl.page_table, 0, kvh, cand))
+    masses = {}
+    for bits in (2, 4, 8):
+        kq, sz = _codes_on_device(layer, bits)
+        w, tok, cc = _estimate_on_device(layer, wl, bits, kq, sz, sel, cnt)
+        rows = wl.num_q_heads
+        stride = w.shape[-1]
+        m_out = torch.zeros(rows, dtype=torch.float32, device=layer.device)
+        kc = torch.zeros(rows, dtype=torch.int32, device=layer.device)
+        kidx = torch.zeros((rows, stride), dtype=torch.int32, device=layer.device)
+        twl.twl_prune_top_p(w.view(rows, stride), cc.view(rows), rows, stride, wl.p, wl.eps,
+                            m_out, kc, kidx)
+        kcn, kidxn, tokn = kc.cpu().numpy(), kidx.cpu().numpy(), tok.cpu().numpy()
+        got = []
+        for h, (cand, wex) in exact.items():
+            kept_tok = tokn[0, h, kidxn[h, :kcn[h]]]
+            pos = np.searchsorted(cand, kept_tok)
+            assert np.array_equal(cand[pos], kept_tok)
+            got.append(float(wex[pos].sum()))
+        masses[bits] = np.array(got)
+    p = wl.p
+    assert masses[8].mean() >= p - 0.01 and masses[8].min() >= p - 0.03, masses[8]
+    assert masses[4].mean() >= p - 0.05, masses[4]
+    assert masses[2].mean() <= masses[4].mean() - 0.1, (masses[2].mean(), masses[4].mean())
