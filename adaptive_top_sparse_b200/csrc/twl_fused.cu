@@ -1665,7 +1665,13 @@ FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) 
     default: scratch = attend_smem_bytes<8>(); break;
   }
   // top-k keys and staged weights when they fit in what is left
-  const size_t cap = 220 * 1024;
+  size_t cap = 220 * 1024;
+  // TWL_FUSED_SMEM_KB=N caps the dynamic shared memory per CTA (N >= 64; below ~110 two CTAs fit
+  // on one SM)
+  if (const char* env = getenv("TWL_FUSED_SMEM_KB")) {
+    const int kb = atoi(env);
+    if (kb >= 64 && kb < 220) cap = (size_t)kb * 1024;
+  }
   size_t want = scratch;
   const size_t topk_need = 1280 + (size_t)4 * max_pages + 4 * kWarps * 512 + 2048;
   want = want > topk_need ? want : topk_need;

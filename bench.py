@@ -54,11 +54,15 @@ WORKLOADS = {
     "c4": ("GQA decode layer, batch 4, 32 q-heads / 8 kv-heads, head_dim 128, 131072-token "
            "context, heavy tokens in 8 spans of 512 per head, 16-token pages, Quest budget 1/4, "
            "INT4 K, p = 0.85, eps = 1e-6, seed 0", dict(batch=4, ctx=131072)),
+    "c6": ("GQA decode layer, batch 64, 32 q-heads / 8 kv-heads, head_dim 128, 8192-token "
+           "context, pages randomly permuted, 16-token pages, Quest budget 1/4, INT4 K, "
+           "p = 0.85, eps = 1e-6, seed 0", dict(batch=64, ctx=8192)),
 }
 
 
 def make_workload(name):
-    return {"c2": synth.config2, "c3": synth.config3, "c4": synth.config4}[name]()
+    return {"c2": synth.config2, "c3": synth.config3, "c4": synth.config4,
+            "c6": synth.config6}[name]()
 
 
 def workload_config(name="c2"):
@@ -573,6 +577,105 @@ def run_append_reference(args, world, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+# ---------------------------------------------------------------------------------- Quest baseline
+
+def run_quest(args, world, rank, local):
+    """Quest alone on the same layer: page selection (same budget) and attention over every
+    valid token of each group's union of selected pages; no INT4 estimate, no top-p.  The union
+    token lists are built once on the host from the (deterministic) selection, so their
+    construction is not timed.  The pages compare this against the pruned path in
+    self-attention time at batch 64."""
+    from adaptive_top_sparse_b200 import twl
+    from adaptive_top_sparse_b200.layer import DecodeLayer, SM_SCALE
+    dev = torch.device("cuda", local)
+    wl = make_workload(args.workload)
+    b_, hq, hkv = wl.batch, wl.num_q_heads, wl.num_kv_heads
+    g = hq // hkv
+    layers = []
+    toks_total = 0
+    for li in range(LAYERS):
+        layer = DecodeLayer.from_workload(wl, dev)
+        layer.build_aux()
+        mb = layer.max_budget
+        sel = torch.full((b_, hq, mb), -1, dtype=torch.int32, device=dev)
+        cnt = torch.zeros((b_, hq), dtype=torch.int32, device=dev)
+        wss = twl.alloc_workspace(twl.TWL_OP_SELECT, dev, batch=b_, num_q_heads=hq,
+                                  num_kv_heads=hkv, max_pages=layer.max_pages)
+        q = torch.from_numpy(wl.q).to(dev)
+        if li == 0:
+            twl.twl_select_pages(q, hq, layer.kv, layer.aux.bounds, wl.budget_pages,
+                                 wl.budget_div, mb, sel, cnt, None, wss)
+            seln, cntn = sel.cpu().numpy(), cnt.cpu().numpy()
+            stride = 16 * layer.max_pages
+            tok = np.full((b_, hkv, stride), -1, np.int32)
+            tcnt = np.zeros((b_, hkv), np.int32)
+            for b in range(b_):
+                n = int(wl.seq_lens[b])
+                for kvh in range(hkv):
+                    pages = sorted(set(int(x) for h in range(kvh * g, (kvh + 1) * g)
+                                       for x in seln[b, h, :cntn[b, h]]))
+                    t = np.concatenate([np.arange(16 * j, min(16 * j + 16, n)) for j in pages])
+                    tok[b, kvh, :t.size] = t
+                    tcnt[b, kvh] = t.size
+            toks_total = int(tcnt.sum())
+        tok_d = torch.from_numpy(tok).to(dev)
+        tcnt_d = torch.from_numpy(tcnt).to(dev)
+        wsa = twl.alloc_workspace(twl.TWL_OP_SPARSE_DECODE, dev, batch=b_, num_q_heads=hq,
+                                  num_kv_heads=hkv, row_stride=stride)
+        layers.append((layer, q, sel, cnt, wss, tok_d, tcnt_d, wsa))
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step():
+        for layer, q, sel, cnt, wss, tok_d, tcnt_d, wsa in layers:
+            twl.twl_select_pages(q, hq, layer.kv, layer.aux.bounds, wl.budget_pages,
+                                 wl.budget_div, layer.max_budget, sel, cnt, None, wss, stream)
+            twl.twl_sparse_decode(q, hq, layer.kv, tok_d, tcnt_d, stride, SM_SCALE, layer.o,
+                                  layer.lse, wsa, stream)
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(world)
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+    e1.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    per_layer_us = ms * 1e3 / (args.steps * LAYERS)
+    n_pages_total = sum((int(n) + 15) // 16 for n in wl.seq_lens)
+    nbytes = n_pages_total * (hkv * 512 + 4) + toks_total * 512 + b_ * hq * (256 + 516)
+    peak, peak_kind = hbm_peak()
+    del graph
+    return {
+        "metric": f"Quest baseline layer-steps/s (select + attention over all selected tokens), "
+                  f"workload {args.workload}",
+        "value": world * args.steps * LAYERS / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": workload_config(args.workload),
+        "roofline": {"bound": "hbm", "achieved": nbytes / per_layer_us / 1e3, "peak": peak,
+                     "unit": "GB/s", "frac": nbytes / per_layer_us / 1e3 / peak,
+                     "traffic": None, "kernel": "twl_select_pages + twl_sparse_decode",
+                     "alg_bytes_per_layer_step": nbytes,
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+        "attended_tokens_per_layer": toks_total, "clocks": clk,
+        "gpu_launches": 4 * args.steps * LAYERS,
+    }
+
+
 # ---------------------------------------------------------------------------------- bit widths
 
 def run_bits(args, world, rank, local):
@@ -678,14 +781,18 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--quest", action="store_true",
+                    help="time the Quest baseline (select + attention over every token of the "
+                         "selected pages, no estimate or top-p) on the workload instead")
     ap.add_argument("--layers", type=int, default=None,
                     help="layer caches per step (default 32 for c2 and append, 4 for c3 / c4)")
-    ap.add_argument("--workload", default="c2", choices=["c2", "c3", "c4", "append", "bits"],
+    ap.add_argument("--workload", default="c2",
+                    choices=["c2", "c3", "c4", "c6", "append", "bits"],
                     help="c2 is the headline; c3 / c4 and the append step are extra reports")
     args = ap.parse_args()
     global LAYERS
     if args.layers is None:
-        args.layers = 4 if args.workload in ("c3", "c4") else 32
+        args.layers = 4 if args.workload in ("c3", "c4", "c6") else 32
     LAYERS = max(1, args.layers)
     if args.warmup < 3:
         args.warmup = 3
@@ -696,6 +803,8 @@ def main():
         elif args.workload == "append":
             out = (run_append_reference(args, world, rank) if args.impl == "reference"
                    else run_append(args, world, rank, local))
+        elif args.quest:
+            out = run_quest(args, world, rank, local)
         elif args.impl == "reference":
             out = run_reference(args, world, rank)
         else:

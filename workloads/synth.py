@@ -201,6 +201,12 @@ def config4(seed: int = 0, n: int = 131072, batch: int = 4, p: float = 0.85) -> 
                        p=p)
 
 
+def config6(seed: int = 0, batch: int = 64, n: int = 8192) -> DecodeWorkload:
+    """Serving batch: 64 sequences of 8192 tokens, 32/8 heads, pages randomly permuted."""
+    return make_decode(f"c6_gqa_b{batch}_{n // 1024}k", batch, 32, 8, [n] * batch, seed=seed,
+                       permute_pages=True)
+
+
 def config5_rows(rows: int, n: int, seed: int = 0, tie_frac: float = 0.01):
     """Standalone pruner input: ``rows`` probability vectors of length n (fp32).
 
