@@ -124,6 +124,19 @@ SelectWs carve_select(Carve& c, int batch, int hq, int max_pages) {
   return w;
 }
 
+struct ClusterWs {
+  float* w;
+  int* row_len;
+  float* m;
+};
+ClusterWs carve_clusters(Carve& c, int batch, int hq, int max_pages) {
+  ClusterWs w;
+  w.w = c.take<float>((size_t)batch * hq * max_pages);
+  w.row_len = c.take<int>((size_t)batch * hq);
+  w.m = c.take<float>((size_t)batch * hq);
+  return w;
+}
+
 struct EstimateWs {
   int* rank;
   int* union_pages;
@@ -164,6 +177,9 @@ size_t twl_workspace_bytes(int32_t op, int32_t batch, int32_t num_q_heads, int32
       break;
     case TWL_OP_ESTIMATE:
       carve_estimate(c, batch, num_q_heads, num_kv_heads, max_pages);
+      break;
+    case TWL_OP_SELECT_CLUSTERS:
+      carve_clusters(c, batch, num_q_heads, max_pages);
       break;
     case TWL_OP_SPARSE_DECODE:
       if (num_kv_heads < 1) return 0;
@@ -256,6 +272,45 @@ twl_status twl_append_token(const twl_paged_kv* kv, const twl_k_aux* aux, const 
       static_cast<uint8_t*>(aux->k_int4), static_cast<uint16_t*>(aux->k_scale_zero),
       static_cast<uint16_t*>(aux->bounds), advance ? const_cast<int32_t*>(kv->seq_lens) : nullptr,
       flags_of(ws), (cudaStream_t)stream));
+}
+
+twl_status twl_page_centroids(const twl_paged_kv* kv, void* centroids, void* ws, size_t ws_bytes,
+                              twl_stream_t stream) {
+  KV k;
+  twl_status st = check_kv(kv, true, false, &k);
+  if (st != TWL_OK) return st;
+  if (!centroids || !aligned(centroids, 16)) return TWL_ERR_INVALID_ARG;
+  if (ws && (st = check_ws(ws, ws_bytes, kHeaderBytes)) != TWL_OK) return st;
+  return cuda_status(launch_page_centroids(k, static_cast<uint16_t*>(centroids), flags_of(ws),
+                                           (cudaStream_t)stream));
+}
+
+twl_status twl_select_clusters_top_p(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
+                                     const void* centroids, float p_cluster, float eps,
+                                     int32_t* sel_pages, int32_t* sel_count,
+                                     float* cluster_weights, void* ws, size_t ws_bytes,
+                                     twl_stream_t stream) {
+  KV k;
+  twl_status st = check_kv(kv, false, false, &k);
+  if (st != TWL_OK) return st;
+  if ((st = check_heads(num_q_heads, k.hkv)) != TWL_OK) return st;
+  if (!q || !centroids || !sel_pages || !sel_count || !aligned(q, 16) || !aligned(centroids, 16))
+    return TWL_ERR_INVALID_ARG;
+  if (cluster_weights && !aligned(cluster_weights, 4)) return TWL_ERR_INVALID_ARG;
+  if (!(p_cluster > 0.f && p_cluster <= 1.f) || !(eps > 0.f) || isinf(eps))
+    return TWL_ERR_INVALID_ARG;
+  Carve c{static_cast<char*>(ws)};
+  ClusterWs w = carve_clusters(c, k.batch, num_q_heads, k.max_pages);
+  if ((st = check_ws(ws, ws_bytes, c.off)) != TWL_OK) return st;
+  float* rows = cluster_weights ? cluster_weights : w.w;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_cluster_weights(static_cast<const uint16_t*>(q), num_q_heads, k,
+                                         static_cast<const uint16_t*>(centroids), rows,
+                                         w.row_len, flags_of(ws), s);
+  if (e == cudaSuccess)
+    e = launch_prune(rows, w.row_len, nullptr, k.batch * num_q_heads, k.max_pages, p_cluster, eps,
+                     w.m, sel_count, sel_pages, s);
+  return cuda_status(e);
 }
 
 twl_status twl_select_pages(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,

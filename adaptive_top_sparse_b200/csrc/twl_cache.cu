@@ -200,6 +200,43 @@ __global__ void __launch_bounds__(256) k_quantize_k(KV kv, uint8_t* __restrict__
   }
 }
 
+// Page centroids for cluster-level selection: per (sequence, page, kv-head) warp, lane l sums
+// channels 4l .. 4l+3 over the valid rows in fp32 from row 0 upwards, divides by the row count
+// (IEEE fp32) and rounds to fp16.
+__global__ void __launch_bounds__(256) k_page_centroids(KV kv, uint16_t* __restrict__ centroids,
+                                                        uint32_t* flags) {
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  int b, j, h;
+  if (!decode_warp(warp, kv, &b, &j, &h)) return;
+  Seq sq = load_seq(kv.seq_lens, b, kv.max_pages, flags, j == 0 && h == 0 && lane == 0);
+  if (j >= sq.pages) return;
+  int ph = kv.page_table[(size_t)b * kv.max_pages + j];
+  if (ph < 0 || ph >= kv.num_phys) {
+    if (lane == 0 && h == 0) raise_flag(flags, TWL_FLAG_BAD_INDEX);
+    return;
+  }
+  const int rows = page_rows(sq.n, j);
+  const uint16_t* src = kv.k + (((size_t)ph * kv.hkv + h) * kPage) * kHeadDim + lane * 4;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int r = 0; r < rows; ++r) {
+    const Half4 v = load_half4(src + r * kHeadDim);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&v.lo));
+    const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&v.hi));
+    acc[0] = __fadd_rn(acc[0], a.x);
+    acc[1] = __fadd_rn(acc[1], a.y);
+    acc[2] = __fadd_rn(acc[2], c.x);
+    acc[3] = __fadd_rn(acc[3], c.y);
+  }
+  const float fr = (float)rows;
+  const __half2 lo = __floats2half2_rn(__fdiv_rn(acc[0], fr), __fdiv_rn(acc[1], fr));
+  const __half2 hi = __floats2half2_rn(__fdiv_rn(acc[2], fr), __fdiv_rn(acc[3], fr));
+  uint2 out;
+  out.x = *reinterpret_cast<const uint32_t*>(&lo);
+  out.y = *reinterpret_cast<const uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(centroids + ((size_t)ph * kv.hkv + h) * kHeadDim + lane * 4) = out;
+}
+
 // One decode step's append: CTA b writes the new token of sequence b (one warp per kv-head,
 // looping when there are more heads than warps), then advances seq_lens[b].
 __global__ void __launch_bounds__(256) k_append_token(KV kv, uint16_t* __restrict__ k_cache,
@@ -291,6 +328,14 @@ cudaError_t launch_quantize_k_bits(const KV& kv, int bits, uint8_t* k_codes, uin
   if (bits == 2) k_quantize_k_bits<2><<<(unsigned)blocks, 256, 0, s>>>(kv, k_codes, k_sz, flags);
   else if (bits == 8) k_quantize_k_bits<8><<<(unsigned)blocks, 256, 0, s>>>(kv, k_codes, k_sz, flags);
   else return launch_quantize_k(kv, k_codes, k_sz, flags, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_page_centroids(const KV& kv, uint16_t* centroids, uint32_t* flags,
+                                  cudaStream_t s) {
+  long warps = (long)kv.batch * kv.max_pages * kv.hkv;
+  long blocks = (warps * 32 + 255) / 256;
+  k_page_centroids<<<(unsigned)blocks, 256, 0, s>>>(kv, centroids, flags);
   return cudaGetLastError();
 }
 

@@ -26,7 +26,12 @@ cudaError_t launch_quantize_k(const KV& kv, uint8_t* k_int4, uint16_t* k_sz, uin
 cudaError_t launch_quantize_k_bits(const KV& kv, int bits, uint8_t* k_codes, uint16_t* k_sz,
                                    uint32_t* flags, cudaStream_t s);
 
+cudaError_t launch_page_centroids(const KV& kv, uint16_t* centroids, uint32_t* flags,
+                                  cudaStream_t s);
+
 // twl_select.cu
+cudaError_t launch_cluster_weights(const uint16_t* q, int hq, const KV& kv, const uint16_t* cen,
+                                   float* w, int* row_len, uint32_t* flags, cudaStream_t s);
 cudaError_t launch_page_scores(const uint16_t* q, int hq, const KV& kv, const uint16_t* bounds,
                                float* scores, uint32_t* flags, cudaStream_t s);
 cudaError_t launch_topk_pages(const float* scores, int hq, const KV& kv, int budget_pages,

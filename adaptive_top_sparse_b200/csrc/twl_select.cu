@@ -220,7 +220,65 @@ __global__ void __launch_bounds__(kTopkThreads)
   if (threadIdx.x == 0) sel_count[bh] = kb;
 }
 
+// Cluster-level weights (size-weighted centroids): one block per (b, q-head).  A warp scores a
+// page at a time: logit_j = ln(n_j) + (q . c_j) / sqrt(128), n_j the page's valid rows; then the
+// row is normalised in place (softmax over the sequence's pages) and its length recorded.
+__global__ void __launch_bounds__(512) k_cluster_weights(const uint16_t* __restrict__ q, int hq,
+                                                         KV kv, const uint16_t* __restrict__ cen,
+                                                         float* __restrict__ w,
+                                                         int* __restrict__ row_len,
+                                                         uint32_t* flags) {
+  __shared__ float red[33];
+  const int bh = blockIdx.x, b = bh / hq, h = bh % hq;
+  const int kvh = h / (hq / kv.hkv);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  Seq sq = load_seq(kv.seq_lens, b, kv.max_pages, flags, h == 0 && threadIdx.x == 0);
+  const int np = sq.pages;
+  float* row = w + (size_t)bh * kv.max_pages;
+  float qv[4];
+  {
+    const uint2 raw = *reinterpret_cast<const uint2*>(q + (size_t)bh * kHeadDim + lane * 4);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+    const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+    qv[0] = a.x; qv[1] = a.y; qv[2] = c.x; qv[3] = c.y;
+  }
+  const float inv_sqrt_d = 0.08838834764831845f;
+  float mx = -INFINITY;
+  for (int j = warp; j < np; j += nwarps) {
+    const int ph = load_phys(kv.page_table, b, j, kv.max_pages, kv.num_phys, flags);
+    float dot = 0.f;
+    if (ph >= 0) {
+      const uint2 raw =
+          *reinterpret_cast<const uint2*>(cen + ((size_t)ph * kv.hkv + kvh) * kHeadDim + lane * 4);
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
+      const float2 c = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
+      dot = qv[0] * a.x + qv[1] * a.y + qv[2] * c.x + qv[3] * c.y;
+    }
+    dot = warp_sum(dot);
+    const float l = ph >= 0 ? logf((float)page_rows(sq.n, j)) + dot * inv_sqrt_d : -INFINITY;
+    if (lane == 0) row[j] = l;
+    mx = fmaxf(mx, l);
+  }
+  mx = block_max(mx, red);  // every warp's lane 0 wrote its pages before the barriers inside
+  float sum = 0.f;
+  for (int j = threadIdx.x; j < np; j += blockDim.x) {
+    const float e = mx > -INFINITY ? __expf(row[j] - mx) : 0.f;
+    row[j] = e;
+    sum += e;
+  }
+  sum = block_sum(sum, red);
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  for (int j = threadIdx.x; j < np; j += blockDim.x) row[j] *= inv;
+  if (threadIdx.x == 0) row_len[bh] = np;
+}
+
 }  // namespace
+
+cudaError_t launch_cluster_weights(const uint16_t* q, int hq, const KV& kv, const uint16_t* cen,
+                                   float* w, int* row_len, uint32_t* flags, cudaStream_t s) {
+  k_cluster_weights<<<kv.batch * hq, 512, 0, s>>>(q, hq, kv, cen, w, row_len, flags);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_page_scores(const uint16_t* q, int hq, const KV& kv, const uint16_t* bounds,
                                float* scores, uint32_t* flags, cudaStream_t s) {

@@ -93,8 +93,69 @@ class DecodeLayer:
                             self.ws, stream)
         return self.o, self.lse
 
+    # ------------------------------------------------------------------ cluster-level selector
+    def double_p(self) -> "DoubleP":
+        """The two-level top-p path on this layer's cache (built on first use)."""
+        if getattr(self, "_double_p", None) is None:
+            self._double_p = DoubleP(self)
+        return self._double_p
+
     def status(self, clear: bool = False):
         return twl.twl_device_status(self.ws, clear)
 
 
 SM_SCALE = 1.0 / math.sqrt(128.0)
+
+
+class DoubleP:
+    """The two-level top-p step: top-p over page clusters scored by size-weighted centroids
+    (twl_select_clusters_top_p), then the token-level path on the kept pages: INT4 estimate,
+    top-p prune, group union, sparse attention.  Five library calls; this class only owns the
+    buffers between them."""
+
+    def __init__(self, layer: DecodeLayer):
+        self.layer = layer
+        L, dev = layer, layer.device
+        b, hq, hkv, mp = L.batch, L.num_q_heads, L.num_kv_heads, L.max_pages
+        i32, f32 = torch.int32, torch.float32
+        self.centroids = torch.zeros((L.k.shape[0], hkv, 128), dtype=torch.float16, device=dev)
+        self.sel = torch.full((b, hq, mp), -1, dtype=i32, device=dev)
+        self.sel_count = torch.zeros((b, hq), dtype=i32, device=dev)
+        self.cluster_w = torch.zeros((b, hq, mp), dtype=f32, device=dev)
+        cs = 16 * mp
+        self.weights = torch.zeros((b, hq, cs), dtype=f32, device=dev)
+        self.cand_tok = torch.full((b, hq, cs), -1, dtype=i32, device=dev)
+        self.cand_count = torch.zeros((b, hq), dtype=i32, device=dev)
+        self.m = torch.zeros(b * hq, dtype=f32, device=dev)
+        self.kept_count = torch.zeros(b * hq, dtype=i32, device=dev)
+        self.kept_idx = torch.zeros((b * hq, cs), dtype=i32, device=dev)
+        self.union_tok = torch.full((b, hkv, cs), -1, dtype=i32, device=dev)
+        self.union_count = torch.zeros((b, hkv), dtype=i32, device=dev)
+        dims = dict(batch=b, num_q_heads=hq, num_kv_heads=hkv, max_pages=mp, max_budget=mp)
+        self.ws_sel = twl.alloc_workspace(twl.TWL_OP_SELECT_CLUSTERS, dev, **dims)
+        self.ws_est = twl.alloc_workspace(twl.TWL_OP_ESTIMATE, dev, **dims)
+        self.ws_att = twl.alloc_workspace(twl.TWL_OP_SPARSE_DECODE, dev, batch=b, num_q_heads=hq,
+                                          num_kv_heads=hkv, row_stride=cs)
+        self.ws_cache = twl.alloc_workspace(twl.TWL_OP_CACHE, dev)
+
+    def build_centroids(self, stream=None) -> None:
+        twl.twl_page_centroids(self.layer.kv, self.centroids, self.ws_cache, stream)
+
+    def decode(self, q, p_cluster: float = 0.95, p: float = 0.85, eps: float = 1e-6,
+               stream=None):
+        L = self.layer
+        hq, mp = L.num_q_heads, L.max_pages
+        cs = 16 * mp
+        twl.twl_select_clusters_top_p(q, hq, L.kv, self.centroids, p_cluster, eps, self.sel,
+                                      self.sel_count, self.cluster_w, self.ws_sel, stream)
+        twl.twl_estimate(q, hq, L.kv, L.aux.k_int4, L.aux.k_scale_zero, self.sel,
+                         self.sel_count, mp, self.weights, self.cand_tok, self.cand_count,
+                         self.ws_est, stream)
+        rows = L.batch * hq
+        twl.twl_prune_top_p(self.weights.view(rows, cs), self.cand_count.view(rows), rows, cs,
+                            p, eps, self.m, self.kept_count, self.kept_idx, None, stream)
+        twl.twl_group_union(hq, L.kv, self.cand_tok, self.kept_idx, self.kept_count, cs,
+                            self.union_tok, self.union_count, None, stream)
+        twl.twl_sparse_decode(q, hq, L.kv, self.union_tok, self.union_count, cs, SM_SCALE, L.o,
+                              L.lse, self.ws_att, stream)
+        return L.o, L.lse

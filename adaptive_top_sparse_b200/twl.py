@@ -38,11 +38,12 @@ TWL_OP_PRUNE = 4
 TWL_OP_UNION = 5
 TWL_OP_SPARSE_DECODE = 6
 TWL_OP_DECODE_STEP = 7
+TWL_OP_SELECT_CLUSTERS = 8
 
 EXPORTED = [
     "twl_workspace_bytes", "twl_workspace_init", "twl_device_status", "twl_status_string",
     "twl_page_bounds", "twl_quantize_k", "twl_append_token", "twl_quantize_k_nbit",
-    "twl_estimate_nbit", "twl_select_pages", "twl_estimate", "twl_prune_top_p",
+    "twl_estimate_nbit", "twl_page_centroids", "twl_select_clusters_top_p", "twl_select_pages", "twl_estimate", "twl_prune_top_p",
     "twl_group_union", "twl_sparse_decode", "twl_decode_step", "twl_noalloc_scratch_bytes",
     "twl_sparse_decode_noalloc",
 ]
@@ -85,6 +86,9 @@ _sigs = {
                                 _vp, _vp, _sz, _vp]),
     "twl_estimate": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _vp, _vp, _vp, _vp, _i32, _vp, _vp,
                             _vp, _vp, _sz, _vp]),
+    "twl_page_centroids": (_i32, [C.POINTER(_PagedKV), _vp, _vp, _sz, _vp]),
+    "twl_select_clusters_top_p": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _vp, _f32, _f32, _vp,
+                                         _vp, _vp, _vp, _sz, _vp]),
     "twl_quantize_k_nbit": (_i32, [C.POINTER(_PagedKV), _i32, _vp, _vp, _vp, _sz, _vp]),
     "twl_estimate_nbit": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _i32, _vp, _vp, _vp, _vp, _i32,
                                  _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -226,6 +230,22 @@ def twl_estimate(q, num_q_heads: int, kv: PagedKV, k_int4, k_scale_zero, sel_pag
                              _ptr(k_scale_zero), _ptr(sel_pages), _ptr(sel_count), max_budget,
                              _ptr(weights), _ptr(cand_tok), _ptr(cand_count), _ptr(ws),
                              _nbytes(ws), _stream(stream)), "twl_estimate")
+
+
+def twl_page_centroids(kv: PagedKV, centroids, ws=None, stream=None) -> None:
+    ckv = kv.c()
+    _check(_lib.twl_page_centroids(C.byref(ckv), _ptr(centroids), _ptr(ws), _nbytes(ws),
+                                   _stream(stream)), "twl_page_centroids")
+
+
+def twl_select_clusters_top_p(q, num_q_heads: int, kv: PagedKV, centroids, p_cluster: float,
+                              eps: float, sel_pages, sel_count, cluster_weights=None, ws=None,
+                              stream=None) -> None:
+    ckv = kv.c()
+    _check(_lib.twl_select_clusters_top_p(_ptr(q), num_q_heads, C.byref(ckv), _ptr(centroids),
+                                          p_cluster, eps, _ptr(sel_pages), _ptr(sel_count),
+                                          _ptr(cluster_weights), _ptr(ws), _nbytes(ws),
+                                          _stream(stream)), "twl_select_clusters_top_p")
 
 
 def twl_quantize_k_nbit(kv: PagedKV, bits: int, k_codes, k_scale_zero, ws=None,

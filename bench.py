@@ -676,6 +676,88 @@ def run_quest(args, world, rank, local):
     }
 
 
+# ---------------------------------------------------------------------------------- Double-P
+
+def run_double_p(args, world, rank, local, p_cluster=0.95):
+    """The two-level top-p step (cluster-level top-p over page centroids, then the token-level
+    path on the kept pages; five library calls, survey row f4) on the workload.  Algorithmic
+    bytes: centroids (256 B per page per kv-head) + page table, INT4 K of each group's union
+    of kept pages, fp16 K/V of the union of kept tokens, q and o/lse."""
+    from adaptive_top_sparse_b200.layer import DecodeLayer
+    dev = torch.device("cuda", local)
+    wl = make_workload(args.workload)
+    b_, hq, hkv = wl.batch, wl.num_q_heads, wl.num_kv_heads
+    g = hq // hkv
+    layers = []
+    for _ in range(LAYERS):
+        layer = DecodeLayer.from_workload(wl, dev)
+        layer.build_aux()
+        dp = layer.double_p()
+        dp.build_centroids()
+        layers.append((dp, torch.from_numpy(wl.q).to(dev)))
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step():
+        for dp, q in layers:
+            dp.decode(q, p_cluster, wl.p, wl.eps, stream)
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    dp0 = layers[0][0]
+    seln, cntn = dp0.sel.cpu().numpy(), dp0.sel_count.cpu().numpy()
+    ucnt = dp0.union_count.cpu().numpy()
+    pages_union = 0
+    for b in range(b_):
+        for kvh in range(hkv):
+            pages = set()
+            for h in range(kvh * g, (kvh + 1) * g):
+                pages.update(seln[b, h, :cntn[b, h]].tolist())
+            pages_union += len(pages)
+    n_pages_total = sum((int(n) + 15) // 16 for n in wl.seq_lens)
+    nbytes = (n_pages_total * (hkv * 256 + 4) + pages_union * 1088 + int(ucnt.sum()) * 512 +
+              b_ * hq * (256 + 516))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(world)
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+    e1.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    per_layer_us = ms * 1e3 / (args.steps * LAYERS)
+    peak, peak_kind = hbm_peak()
+    del graph
+    return {
+        "metric": f"two-level top-p (cluster top-p p_c = {p_cluster}, then token top-p) "
+                  f"layer-steps/s, workload {args.workload}",
+        "value": world * args.steps * LAYERS / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": workload_config(args.workload),
+        "roofline": {"bound": "hbm", "achieved": nbytes / per_layer_us / 1e3, "peak": peak,
+                     "unit": "GB/s", "frac": nbytes / per_layer_us / 1e3 / peak,
+                     "traffic": None, "kernel": "twl_select_clusters_top_p + twl_estimate + "
+                     "twl_prune_top_p + twl_group_union + twl_sparse_decode",
+                     "alg_bytes_per_layer_step": nbytes,
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+        "kept_pages_per_head_mean": float(cntn.mean()), "pages_per_head": n_pages_total // b_,
+        "union_tokens_per_group": ucnt.reshape(-1).tolist(), "clocks": clk,
+        "gpu_launches": 9 * args.steps * LAYERS,
+    }
+
+
 # ---------------------------------------------------------------------------------- bit widths
 
 def run_bits(args, world, rank, local):
@@ -781,6 +863,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--double-p", action="store_true",
+                    help="time the two-level (cluster, then token) top-p path on the workload")
     ap.add_argument("--quest", action="store_true",
                     help="time the Quest baseline (select + attention over every token of the "
                          "selected pages, no estimate or top-p) on the workload instead")
@@ -803,6 +887,8 @@ def main():
         elif args.workload == "append":
             out = (run_append_reference(args, world, rank) if args.impl == "reference"
                    else run_append(args, world, rank, local))
+        elif args.double_p:
+            out = run_double_p(args, world, rank, local)
         elif args.quest:
             out = run_quest(args, world, rank, local)
         elif args.impl == "reference":

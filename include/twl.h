@@ -116,6 +116,7 @@ typedef struct twl_step_stats {
 #define TWL_OP_UNION 5         /* twl_group_union                           */
 #define TWL_OP_SPARSE_DECODE 6 /* twl_sparse_decode (row_stride = tok_stride) */
 #define TWL_OP_DECODE_STEP 7   /* twl_decode_step                           */
+#define TWL_OP_SELECT_CLUSTERS 8 /* twl_select_clusters_top_p                 */
 size_t twl_workspace_bytes(int32_t op, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                            int32_t max_pages, int32_t max_budget, int32_t rows,
                            int32_t row_stride);
@@ -202,6 +203,29 @@ twl_status twl_estimate(const void* q, int32_t num_q_heads, const twl_paged_kv* 
                         const int32_t* sel_count, int32_t max_budget, float* weights,
                         int32_t* cand_tok, int32_t* cand_count, void* ws, size_t ws_bytes,
                         twl_stream_t stream);
+
+/* ---------------------------------------------------------------- cluster-level top-p (f4)
+ * The Double-P selector (Double-P summary page, "Technical framework" and "Key designs": a
+ * top-p over clusters scored by size-weighted centroids, then token-level top-p inside the
+ * kept clusters, which twl_estimate / twl_prune_top_p / twl_group_union / twl_sparse_decode
+ * do with the pages kept here).  The page gives no clustering method: a cluster is one page.
+ *   twl_page_centroids: centroids fp16 [P][Hkv][128]; per referenced page and kv-head the mean
+ *     of the valid K rows (fp32 sum from row 0 upwards, IEEE fp32 division by the row count,
+ *     fp16 round to nearest even).  Workspace (TWL_OP_CACHE) may be NULL.
+ *   twl_select_clusters_top_p: per (b, q-head) A_j = n_j exp(q . c_j / sqrt(128)) over the
+ *     sequence's pages j (n_j valid rows), W_j = A_j / sum A; then the bisection of
+ *     twl_prune_top_p at p_cluster, eps.  sel_pages int32 [B][Hq][max_pages] out (kept pages,
+ *     ascending; pass max_budget = max_pages to twl_estimate), sel_count int32 [B][Hq] out,
+ *     cluster_weights float [B][Hq][max_pages] out (W; slots past P_b unwritten) or NULL.
+ *     Workspace TWL_OP_SELECT_CLUSTERS.  p_cluster outside (0, 1], eps <= 0 or not finite:
+ *     TWL_ERR_INVALID_ARG. */
+twl_status twl_page_centroids(const twl_paged_kv* kv, void* centroids, void* ws, size_t ws_bytes,
+                              twl_stream_t stream);
+twl_status twl_select_clusters_top_p(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
+                                     const void* centroids, float p_cluster, float eps,
+                                     int32_t* sel_pages, int32_t* sel_count,
+                                     float* cluster_weights, void* ws, size_t ws_bytes,
+                                     twl_stream_t stream);
 
 /* ---------------------------------------------------------------- estimator bit widths (f2)
  * The estimator ablation ([Notes] "Key designs": a 4-bit K cache suffices for the weight

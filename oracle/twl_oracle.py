@@ -455,6 +455,56 @@ def exact_weights(q16, k, page_table, b, kvh, cand, head_dim=128):
     return softmax64(logits)
 
 
+# ----------------------------------------------------------------------------------------------
+# Cluster-level top-p selection (the Double-P summary page, "Technical framework" and "Key
+# designs": a first top-p over clusters scored with size-weighted centroids, then token-level
+# top-p inside the kept clusters).  The page gives no clustering method; the reading here takes
+# the page (16 consecutive tokens) as the cluster, its centroid as the mean of its valid K rows,
+# and its size as the number of those rows.
+# ----------------------------------------------------------------------------------------------
+
+def page_centroids(k, page_table, seq_lens, out=None):
+    """fp16 [P][Hkv][D]: per referenced page and kv-head, the mean of the valid K rows, summed
+    in fp32 from row 0 upwards, divided by the row count in fp32, rounded to fp16."""
+    p_phys, hkv, page, d = k.shape
+    cen = np.zeros((p_phys, hkv, d), dtype=F16) if out is None else out.copy()
+    for b in range(len(seq_lens)):
+        n = int(seq_lens[b])
+        for j in range(num_pages(n)):
+            ph = int(page_table[b, j])
+            rows = valid_rows(n, j)
+            acc = np.zeros((hkv, d), dtype=F32)
+            for r in range(rows):                   # left to right, fp32
+                acc = (acc + k[ph, :, r, :].astype(F32)).astype(F32)
+            cen[ph] = (acc / F32(rows)).astype(F16)
+    return cen
+
+
+def cluster_weights(q16, cen, page_table, b, kvh, n, head_dim=128):
+    """Size-weighted centroid estimate of each page's share of the attention mass:
+    A_j = n_j exp(q . c_j / sqrt(D)), normalised over the sequence's pages (fp64)."""
+    pb = num_pages(n)
+    phys = np.asarray(page_table[b, :pb], dtype=np.int64)
+    c = cen[phys, kvh].astype(F64)                                      # [pb][D]
+    sizes = np.array([valid_rows(n, j) for j in range(pb)], dtype=F64)
+    logits = np.log(sizes) + (c @ np.asarray(q16, dtype=F16).astype(F64)) / math.sqrt(head_dim)
+    return softmax64(logits)
+
+
+def select_clusters(q, cen, page_table, seq_lens, num_q_heads, num_kv_heads, p_cluster):
+    """Per (b, head): the pages kept by top-p (sort form) over the cluster weights, ascending.
+    Returns {(b, h): (weights, pages)}."""
+    g = num_q_heads // num_kv_heads
+    out = {}
+    for b in range(len(seq_lens)):
+        n = int(seq_lens[b])
+        for h in range(num_q_heads):
+            w = cluster_weights(q[b, h], cen, page_table, b, h // g, n)
+            _, _, kept = top_p_sort(w, p_cluster)
+            out[(b, h)] = (w, np.sort(np.asarray(kept, dtype=np.int64)))
+    return out
+
+
 def decode_step(wl, bounds=None, k_int4=None, k_sz=None, with_attention=True):
     """Full oracle pass of select -> estimate -> top-p -> group union -> attention.
 
