@@ -3,6 +3,7 @@
 #include <math.h>
 
 #include <mutex>
+#include <stdlib.h>
 
 #include "twl_common.cuh"
 #include "twl_fused.h"
@@ -94,8 +95,13 @@ twl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TWL_OK : TWL_E
 
 uint32_t* flags_of(void* ws) { return ws ? &reinterpret_cast<WsHeader*>(ws)->flags : nullptr; }
 
-// Cluster size for the fused kernel, cached per (device, group size, wanted size, smem).
+// Cluster size for the fused kernel, cached per (device, group size, wanted size, smem).  A size
+// forced through TWL_FUSED_CLUSTER is taken as is (clusters then run in as many waves as needed).
 int fitted_cluster(int g, int want, int groups, int smem_bytes) {
+  if (const char* env = getenv("TWL_FUSED_CLUSTER")) {
+    const int f = atoi(env);
+    if (f >= 1 && f <= 16) return want;
+  }
   struct Entry {
     int dev, g, want, groups, smem, c;
   };
