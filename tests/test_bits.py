@@ -222,3 +222,22 @@ def test_bitwidth_mass_ablation():
     assert masses[8].mean() >= p - 0.01 and masses[8].min() >= p - 0.03, masses[8]
     assert masses[4].mean() >= p - 0.05, masses[4]
     assert masses[2].mean() <= masses[4].mean() - 0.1, (masses[2].mean(), masses[4].mean())
+
+
+def test_exact_weights_closed_forms():
+    """exact_weights is the softmax of the exact q.k / sqrt(D) over the candidates: equal keys
+    give equal weights; one key aligned with q at logit x against zero keys gives
+    e^x / (e^x + n - 1)."""
+    d = D
+    q = np.zeros(d, np.float16)
+    q[:4] = np.float16(1.0)                                   # |q|^2 = 4
+    k = np.zeros((1, 1, 16, d), np.float16)
+    pt = np.array([[0]], np.int32)
+    cand = np.arange(16)
+    w = O.exact_weights(q, k, pt, 0, 0, cand)
+    assert np.allclose(w, 1 / 16, rtol=0, atol=1e-15)
+    k[0, 0, 5, :4] = np.float16(8.0)                         # q.k = 32, logit 32 / sqrt(128)
+    w = O.exact_weights(q, k, pt, 0, 0, cand)
+    x = 32 / np.sqrt(d)
+    assert np.isclose(w[5], np.exp(x) / (np.exp(x) + 15), rtol=1e-12)
+    assert np.allclose(np.delete(w, 5), 1 / (np.exp(x) + 15), rtol=1e-12)
