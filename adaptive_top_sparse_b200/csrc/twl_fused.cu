@@ -588,10 +588,12 @@ __device__ void phase_union_bitmaps(const FusedArgs& a, int b, int kvh, Smem& sm
       for (int h = 0; h <= G; ++h) wtot[warp * (G + 1) + h] = x[h];
     }
     __syncthreads();
+    // only the warps that hold words of this round contribute
+    const int active = min(kWarps, (nw - base + 31) >> 5);
 #pragma unroll
     for (int h = 0; h <= G; ++h) {
       int before = carry[h], round = 0;
-      for (int ww = 0; ww < kWarps; ++ww) {
+      for (int ww = 0; ww < active; ++ww) {
         const int t = wtot[ww * (G + 1) + h];
         if (ww < warp) before += t;
         round += t;
