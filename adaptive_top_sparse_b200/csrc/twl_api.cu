@@ -511,7 +511,6 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
   a.union_count = so.union_count;
   a.union_tok = so.union_tok;
   a.want_union = (so.union_tok != nullptr || so.union_count != nullptr) ? 1 : 0;
-  a.prefetch_int4 = 0;  // measured: the estimate phase is not bound by DRAM latency
   a.pt_smem = pl.pt_smem ? 1 : 0;
   a.flags = flags_of(ws);
   a.sel_words = pl.sel_words;

@@ -96,10 +96,6 @@ __device__ __forceinline__ void stamp(const FusedArgs&, int) {}
 
 __device__ __forceinline__ float ldcg_f(const float* p) { return __ldcg(p); }
 
-// Bulk prefetch of a 16-byte aligned range (size a multiple of 16) into L2.
-__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 __device__ __forceinline__ int ldcg_i(const int* p) { return __ldcg(p); }
 __device__ __forceinline__ uint32_t ldcg_u(const uint32_t* p) { return __ldcg(p); }
 

@@ -32,7 +32,6 @@ struct FusedArgs {
   int* union_count;
   int* union_tok;  // the workspace's list when the caller does not ask for it
   int want_union;  // build the group's ordered union list (the caller asked for it)
-  int prefetch_int4;  // prefetch the INT4 tiles of the scored pages into L2 during scoring
   int pt_smem;        // stage the sequence's page table in shared memory
   // workspace
   float* scores;
