@@ -789,16 +789,35 @@ __device__ __forceinline__ long long w_fixed(float w) { return __float2ll_rn(w *
 // The search on (0, top]: lo = 0, hi = top; the midpoint test is "mid <= T" (see
 // top_p_from_live); stop when hi - lo <= eps, when the midpoint no longer splits, or after 64
 // steps; the threshold is lo (top when the test passes at top itself).
+// Four steps per trip, predicated (the same steps and stops as one step per trip).  While
+// hi - lo >= 2^-100, (hi - lo) * 0.5 is exact, so fma(hi - lo, 0.5, lo) rounds the same sum as
+// lo + (hi - lo) * 0.5; eps >= 2^-100 keeps every tested width there.
 __device__ __forceinline__ float bisect_scalar(float top, float T, float eps) {
   if (top <= T) return top;
   float lo = 0.f, hi = top;
+  if (!(eps >= 0x1p-100f)) {
 #pragma unroll 1
-  for (int steps = 0; steps < 64; ++steps) {
-    if (__fsub_rn(hi, lo) <= eps) break;
-    const float mid = mid_of(lo, hi);
-    if (!(lo < mid && mid < hi)) break;
-    if (mid <= T) lo = mid;
-    else hi = mid;
+    for (int steps = 0; steps < 64; ++steps) {
+      if (__fsub_rn(hi, lo) <= eps) break;
+      const float mid = mid_of(lo, hi);
+      if (!(lo < mid && mid < hi)) break;
+      if (mid <= T) lo = mid;
+      else hi = mid;
+    }
+    return lo;
+  }
+  bool done = false;
+#pragma unroll 1
+  for (int steps = 0; steps < 64 && !done; steps += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float d = __fsub_rn(hi, lo);
+      const float mid = __fmaf_rn(d, 0.5f, lo);
+      done = done || d <= eps || !(lo < mid && mid < hi);
+      const bool down = mid <= T;
+      lo = !done && down ? mid : lo;
+      hi = !done && !down ? mid : hi;
+    }
   }
   return lo;
 }
