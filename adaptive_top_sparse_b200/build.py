@@ -42,6 +42,17 @@ def _headers() -> list[str]:
     return hs
 
 
+def _included_sources(src: str) -> list[str]:
+    """Other .cu files a source #includes (a second build of the same kernel source)."""
+    out = []
+    with open(src) as f:
+        for line in f:
+            line = line.strip()
+            if line.startswith("#include \"") and line.endswith('.cu"'):
+                out.append(os.path.join(CSRC, line.split('"')[1]))
+    return out
+
+
 def _stale(target: str, deps: list[str]) -> bool:
     if not os.path.exists(target):
         return True
@@ -58,7 +69,7 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     for src in sources():
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
-        if force or _stale(obj, [src] + hdrs):
+        if force or _stale(obj, [src] + _included_sources(src) + hdrs):
             cmd = [nvcc, *ARCH, *FLAGS, *(extra or []), "-c", src, "-o", obj]
             jobs.append(cmd)
 

@@ -97,13 +97,13 @@ uint32_t* flags_of(void* ws) { return ws ? &reinterpret_cast<WsHeader*>(ws)->fla
 
 // Cluster size for the fused kernel, cached per (device, group size, wanted size, smem).  A size
 // forced through TWL_FUSED_CLUSTER is taken as is (clusters then run in as many waves as needed).
-int fitted_cluster(int g, int want, int groups, int smem_bytes) {
+int fitted_cluster(int g, int want, int groups, int smem_bytes, bool small) {
   if (const char* env = getenv("TWL_FUSED_CLUSTER")) {
     const int f = atoi(env);
     if (f >= 1 && f <= 16) return want;
   }
   struct Entry {
-    int dev, g, want, groups, smem, c;
+    int dev, g, want, groups, smem, small, c;
   };
   static std::mutex mu;
   static Entry cache[64];
@@ -113,11 +113,29 @@ int fitted_cluster(int g, int want, int groups, int smem_bytes) {
   std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < n; ++i)
     if (cache[i].dev == dev && cache[i].g == g && cache[i].want == want &&
-        cache[i].groups == groups && cache[i].smem == smem_bytes)
+        cache[i].groups == groups && cache[i].smem == smem_bytes && cache[i].small == (int)small)
       return cache[i].c;
-  const int c = fit_cluster(g, want, groups, smem_bytes);
-  if (n < 64) cache[n++] = Entry{dev, g, want, groups, smem_bytes, c};
+  const int c = small ? fused256::fit_cluster(g, want, groups, smem_bytes)
+                      : fused512::fit_cluster(g, want, groups, smem_bytes);
+  if (n < 64) cache[n++] = Entry{dev, g, want, groups, smem_bytes, (int)small, c};
   return c;
+}
+
+// The 256-thread build when there are more groups than SMs (two CTAs share an SM there);
+// TWL_FUSED_THREADS=256 or 512 forces one.
+bool use_small_ctas(int groups) {
+  if (const char* env = getenv("TWL_FUSED_THREADS")) {
+    const int t = atoi(env);
+    if (t == 256) return true;
+    if (t == 512) return false;
+  }
+  return groups > num_sms();
+}
+
+size_t decode_step_ws_bytes(int batch, int hq, int hkv, int max_pages, int max_budget) {
+  const size_t a = fused512::fused_workspace_bytes(batch, hq, hkv, max_pages, max_budget);
+  const size_t b = fused256::fused_workspace_bytes(batch, hq, hkv, max_pages, max_budget);
+  return a > b ? a : b;
 }
 
 // ---------------------------------------------------------------- workspace layouts
@@ -194,7 +212,7 @@ size_t twl_workspace_bytes(int32_t op, int32_t batch, int32_t num_q_heads, int32
     case TWL_OP_DECODE_STEP:
       if (num_kv_heads < 1 || num_q_heads < num_kv_heads || max_pages < 1 || max_budget < 1)
         return 0;
-      c.take<char>(fused_workspace_bytes(batch, num_q_heads, num_kv_heads, max_pages,
+      c.take<char>(decode_step_ws_bytes(batch, num_q_heads, num_kv_heads, max_pages,
                                          max_budget));
       break;
     default:
@@ -477,13 +495,20 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
     return TWL_ERR_INVALID_ARG;
   if (!(p > 0.f && p <= 1.f) || !(eps > 0.f) || isinf(eps)) return TWL_ERR_INVALID_ARG;
   if ((st = check_budget(budget_pages, budget_div, max_budget, k.max_pages)) != TWL_OK) return st;
-  FusedPlan pl = plan_fused(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
+  bool small = use_small_ctas(k.batch * k.hkv);
+  FusedPlan pl{};
+  if (small) {
+    pl = fused256::plan_fused(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
+    if (!pl.ok) small = false;  // too little shared memory at two CTAs per SM
+  }
+  if (!small) pl = fused512::plan_fused(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
   if (!pl.ok) return TWL_ERR_UNSUPPORTED;
   Carve c{static_cast<char*>(ws)};
-  char* fws = c.take<char>(fused_workspace_bytes(k.batch, num_q_heads, k.hkv, k.max_pages,
-                                                 max_budget));
+  char* fws = c.take<char>(decode_step_ws_bytes(k.batch, num_q_heads, k.hkv, k.max_pages,
+                                                max_budget));
   if ((st = check_ws(ws, ws_bytes, c.off)) != TWL_OK) return st;
-  pl.cluster = fitted_cluster(num_q_heads / k.hkv, pl.cluster, k.batch * k.hkv, pl.smem_bytes);
+  pl.cluster =
+      fitted_cluster(num_q_heads / k.hkv, pl.cluster, k.batch * k.hkv, pl.smem_bytes, small);
   const twl_step_stats none = {};
   const twl_step_stats& so = stats ? *stats : none;
   FusedArgs a = {};
@@ -518,8 +543,12 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
   a.union_stride = pl.union_stride;
   a.cluster = pl.cluster;
   a.smem_bytes = pl.smem_bytes;
-  carve_fused(a, fws, pl, k.batch, num_q_heads, k.hkv, k.max_pages);
-  return cuda_status(launch_fused(a, pl, (cudaStream_t)stream));
+  if (small) {
+    fused256::carve_fused(a, fws, pl, k.batch, num_q_heads, k.hkv, k.max_pages);
+    return cuda_status(fused256::launch_fused(a, pl, (cudaStream_t)stream));
+  }
+  fused512::carve_fused(a, fws, pl, k.batch, num_q_heads, k.hkv, k.max_pages);
+  return cuda_status(fused512::launch_fused(a, pl, (cudaStream_t)stream));
 }
 
 }  // extern "C"

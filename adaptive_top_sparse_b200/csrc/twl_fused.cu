@@ -37,9 +37,17 @@
 namespace twl {
 namespace {
 
-constexpr int kThreads = 512;
+#ifndef TWL_FUSED_THREADS
+#define TWL_FUSED_THREADS 512
+#endif
+#ifndef TWL_FUSED_NS
+#define TWL_FUSED_NS fused512
+#endif
+constexpr int kThreads = TWL_FUSED_THREADS;  // 512, or 256 for two CTAs per SM at large batch
+static_assert(kThreads == 512 || kThreads == 256, "512 or 256 threads per CTA");
 constexpr int kWarps = kThreads / 32;
-constexpr int kAttChunk = 64;  // tokens gathered per attention round
+constexpr int kAttChunk = kThreads / 8;   // tokens gathered per attention round
+constexpr int kQuarters = kThreads / 128;  // token groups of the P.V product
 
 // Cluster barrier: arrive with release, wait with acquire semantics (orders shared, distributed
 // shared and global memory accesses of the cluster's CTAs across it).
@@ -1279,8 +1287,8 @@ __device__ void phase_write_union(const FusedArgs& a, int gi, int U, int r, int 
 }
 
 // ------------------------------------------------------------------------- phase 7: attention
-// Thread layout: token slot t = tid / 8 (64 per round), sub-lane s = tid % 8 owns channels
-// [8s, 8s+8) and [64+8s, 64+8s+8).  For P.V: channel d = tid % 128, token quarter = tid / 128.
+// Thread layout: token slot t = tid / 8 (kAttChunk per round), sub-lane s = tid % 8 owns channels
+// [8s, 8s+8) and [64+8s, 64+8s+8).  For P.V: channel d = tid % 128, token group tid / 128.
 // kLocal: tokens of this CTA's own union share, from (rowmask, pfx, pph) in shared memory;
 // otherwise an even share [T r / C, T (r+1) / C) of the group's global ascending list.
 template <int G, bool kLocal>
@@ -1291,12 +1299,15 @@ __device__ void phase_attend(const FusedArgs& a, int b, int kvh, int gi, int n, 
   const int ts = tid >> 3, s8 = tid & 7;
   const int d = tid & 127, quarter = tid >> 7;
   unsigned char* sp = sm.scratch;
-  uint4* ks = reinterpret_cast<uint4*>(sp);                       // [64][16]
-  uint4* vs = reinterpret_cast<uint4*>(sp + 16384);               // [64][16]
-  float* ps = reinterpret_cast<float*>(sp + 32768);               // [G][64]
-  float* red = reinterpret_cast<float*>(sp + 32768 + G * 256);    // [kWarps][G]
-  uint32_t* rowidx = reinterpret_cast<uint32_t*>(sp + 32768 + G * 256 + kWarps * G * 4);  // 64
-  float* opart = reinterpret_cast<float*>(sp + 32768 + G * 256 + kWarps * G * 4 + 256);  // [4][G][128]
+  constexpr int kKV = kAttChunk * 256;  // bytes of one staged K (or V) chunk
+  uint4* ks = reinterpret_cast<uint4*>(sp);                              // [kAttChunk][16]
+  uint4* vs = reinterpret_cast<uint4*>(sp + kKV);                        // [kAttChunk][16]
+  float* ps = reinterpret_cast<float*>(sp + 2 * kKV);                    // [G][kAttChunk]
+  float* red = reinterpret_cast<float*>(sp + 2 * kKV + G * kAttChunk * 4);  // [kWarps][G]
+  uint32_t* rowidx =
+      reinterpret_cast<uint32_t*>(sp + 2 * kKV + G * kAttChunk * 4 + kWarps * G * 4);  // [kAttChunk]
+  float* opart = reinterpret_cast<float*>(sp + 2 * kKV + G * kAttChunk * 4 + kWarps * G * 4 +
+                                          kAttChunk * 4);  // [kQuarters][G][128]
   const int t0 = kLocal ? 0 : (int)((long)T * r / C), t1 = kLocal ? T : (int)((long)T * (r + 1) / C);
   const int* ulist = a.union_tok + (size_t)gi * a.union_stride;
 
@@ -1350,10 +1361,10 @@ __device__ void phase_attend(const FusedArgs& a, int b, int kvh, int gi, int n, 
       rowidx[tid] = ri;
     }
     __syncthreads();
-    // gather 64 rows of K and V: 2048 16-byte chunks, 4 per thread
+    // gather kAttChunk rows of K and V: 2 x 16 x kAttChunk 16-byte chunks, 4 per thread
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
-      const int c = tid + it * kThreads;  // 0 .. 1023
+      const int c = tid + it * kThreads;  // 0 .. 16 kAttChunk - 1
       const int tt = c >> 4, ch = c & 15;
       const uint32_t ri = rowidx[tt];
       const bool ok = ri != 0xFFFFFFFFu;
@@ -1406,12 +1417,12 @@ __device__ void phase_attend(const FusedArgs& a, int b, int kvh, int gi, int n, 
       if (s8 == 0) ps[h * kAttChunk + ts] = pv;
     }
     __syncthreads();
-    // P.V for channel d over tokens quarter, quarter+4, ...
+    // P.V for channel d over tokens quarter, quarter + kQuarters, ...
     const __half* vh = reinterpret_cast<const __half*>(vs);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float acc = 0.f, lsum = 0.f;
-      for (int tt = quarter; tt < nt; tt += 4) {
+      for (int tt = quarter; tt < nt; tt += kQuarters) {
         const float pv = ps[h * kAttChunk + tt];
         acc = fmaf(pv, __half2float(vh[tt * kHeadDim + d]), acc);
         lsum += pv;
@@ -1421,10 +1432,10 @@ __device__ void phase_attend(const FusedArgs& a, int b, int kvh, int gi, int n, 
     }
     __syncthreads();
   }
-  // combine the 4 quarters, write this CTA's partial: M, L, O (unnormalised)
+  // combine the token groups, write this CTA's partial: M, L, O (unnormalised)
 #pragma unroll
   for (int h = 0; h < G; ++h) opart[(quarter * G + h) * kHeadDim + d] = O[h];
-  float* lpart = reinterpret_cast<float*>(ps);  // reuse: [4][G]
+  float* lpart = reinterpret_cast<float*>(ps);  // reuse: [kQuarters][G]
   if (d == 0) {
 #pragma unroll
     for (int h = 0; h < G; ++h) lpart[quarter * G + h] = L[h];
@@ -1434,13 +1445,16 @@ __device__ void phase_attend(const FusedArgs& a, int b, int kvh, int gi, int n, 
   if (quarter == 0) {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const float o = opart[(0 * G + h) * kHeadDim + d] + opart[(1 * G + h) * kHeadDim + d] +
-                      opart[(2 * G + h) * kHeadDim + d] + opart[(3 * G + h) * kHeadDim + d];
+      float o = 0.f, l = 0.f;
+#pragma unroll
+      for (int qq = 0; qq < kQuarters; ++qq) {
+        o += opart[(qq * G + h) * kHeadDim + d];
+        l += lpart[qq * G + h];
+      }
       part[h * (kHeadDim + 2) + 2 + d] = o;
       if (d == 0) {
         part[h * (kHeadDim + 2) + 0] = M[h];
-        part[h * (kHeadDim + 2) + 1] =
-            lpart[0 * G + h] + lpart[1 * G + h] + lpart[2 * G + h] + lpart[3 * G + h];
+        part[h * (kHeadDim + 2) + 1] = l;
       }
     }
   }
@@ -1485,7 +1499,8 @@ __device__ void phase_merge_head(const FusedArgs& a, int gi, int bh, int hl, int
 
 template <int G>
 __host__ __device__ constexpr size_t attend_smem_bytes() {
-  return 32768 + G * 256 + kWarps * G * 4 + 256 + 4 * G * kHeadDim * 4;
+  return 2 * kAttChunk * 256 + G * kAttChunk * 4 + kWarps * G * 4 + kAttChunk * 4 +
+         kQuarters * G * kHeadDim * 4;
 }
 
 // The local attention path needs room for the largest share of the cluster (so every CTA takes
@@ -1499,7 +1514,7 @@ __device__ __forceinline__ bool local_fits_all(const FusedArgs& a, int U, int C,
 
 // ------------------------------------------------------------------------- the kernel
 template <int G>
-__global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
+__global__ void __launch_bounds__(kThreads, 512 / kThreads) k_decode_fused(FusedArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ int scan_sh[33];
   __shared__ int s_total;
@@ -1654,6 +1669,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_decode_fused(FusedArgs a) {
 
 }  // namespace
 
+namespace TWL_FUSED_NS {
+
 FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) {
   FusedPlan pl{};
   const int g = hq / hkv;
@@ -1664,7 +1681,8 @@ FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) 
   // cluster size: enough CTAs to fill the GPU, at most 16
   const int sms = num_sms();
   int c = 1;
-  while (c < 16 && groups * (c + 1) <= sms) ++c;
+  const int per_sm = 512 / kThreads;  // CTAs that fit on one SM
+  while (c < 16 && groups * (c + 1) <= per_sm * sms) ++c;
   // TWL_FUSED_CLUSTER=1..16 forces the cluster size (used by the tests to cover several sizes)
   if (const char* env = getenv("TWL_FUSED_CLUSTER")) {
     const int f = atoi(env);
@@ -1682,7 +1700,7 @@ FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget) 
     default: scratch = attend_smem_bytes<8>(); break;
   }
   // top-k keys and staged weights when they fit in what is left
-  size_t cap = 220 * 1024;
+  size_t cap = (kThreads == 256 ? 110 : 220) * 1024;  // two 256-thread CTAs share an SM
   // TWL_FUSED_SMEM_KB=N caps the dynamic shared memory per CTA (N >= 64; below ~110 two CTAs fit
   // on one SM)
   if (const char* env = getenv("TWL_FUSED_SMEM_KB")) {
@@ -1840,4 +1858,5 @@ int fit_cluster(int g, int want, int groups, int smem_bytes) {
   return best;
 }
 
+}  // namespace TWL_FUSED_NS
 }  // namespace twl

@@ -55,11 +55,21 @@ struct FusedPlan {
   bool ok;
 };
 
-FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget);
-size_t fused_workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_budget);
-void carve_fused(FusedArgs& a, char* ws, const FusedPlan& pl, int batch, int hq, int hkv,
-                 int max_pages);
-int fit_cluster(int g, int want, int groups, int smem_bytes);
-cudaError_t launch_fused(const FusedArgs& a, const FusedPlan& pl, cudaStream_t s);
+// Two builds of twl_fused.cu: 512-thread CTAs (one per SM), and 256-thread CTAs with half the
+// shared memory (two per SM) for batches with more groups than SMs.
+#define TWL_FUSED_DECLS                                                                     \
+  FusedPlan plan_fused(int batch, int hq, int hkv, int max_pages, int max_budget);           \
+  size_t fused_workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_budget);   \
+  void carve_fused(FusedArgs& a, char* ws, const FusedPlan& pl, int batch, int hq, int hkv, \
+                   int max_pages);                                                           \
+  int fit_cluster(int g, int want, int groups, int smem_bytes);                              \
+  cudaError_t launch_fused(const FusedArgs& a, const FusedPlan& pl, cudaStream_t s);
+namespace fused512 {
+TWL_FUSED_DECLS
+}
+namespace fused256 {
+TWL_FUSED_DECLS
+}
+#undef TWL_FUSED_DECLS
 
 }  // namespace twl

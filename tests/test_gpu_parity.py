@@ -382,6 +382,33 @@ def test_decode_step_every_cluster_size(cluster, monkeypatch):
     assert layer.status()[0] == twl.TWL_OK
 
 
+@pytest.mark.parametrize("cluster", [1, 3, 8, 16])
+def test_decode_step_small_ctas(cluster, monkeypatch):
+    """The 256-thread build (two CTAs per SM), forced, over several cluster sizes."""
+    monkeypatch.setenv("TWL_FUSED_THREADS", "256")
+    monkeypatch.setenv("TWL_FUSED_CLUSTER", str(cluster))
+    wl = synth.make_decode("small_ctas", 2, 8, 2, [3001, 515], seed=19)
+    layer = DecodeLayer.from_workload(wl)
+    layer.build_aux()
+    st, o, lse = _run_step(wl, layer)
+    for bb in range(wl.batch):
+        for kvh in range(wl.num_kv_heads):
+            check_step_group(wl, bb, kvh, st, o, lse)
+    assert layer.status()[0] == twl.TWL_OK
+
+
+def test_decode_step_more_groups_than_sms():
+    """320 (sequence, kv-head) groups: the 256-thread build is chosen; sampled groups."""
+    lens = [300 + 37 * i for i in range(40)]
+    wl = synth.make_decode("many_groups", 40, 32, 8, lens, seed=29, permute_pages=True)
+    layer = DecodeLayer.from_workload(wl)
+    layer.build_aux()
+    st, o, lse = _run_step(wl, layer)
+    for bb, kvh in [(0, 0), (7, 3), (21, 5), (39, 7)]:
+        check_step_group(wl, bb, kvh, st, o, lse)
+    assert layer.status()[0] == twl.TWL_OK
+
+
 # -------------------------------------------------------------------------- full-size workloads
 
 def _full_check(wl, groups):
