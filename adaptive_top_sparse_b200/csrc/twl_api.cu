@@ -121,15 +121,18 @@ int fitted_cluster(int g, int want, int groups, int smem_bytes, bool small) {
   return c;
 }
 
-// The 256-thread build when there are more groups than SMs (two CTAs share an SM there);
+// The 256-thread build (two CTAs per SM) when the 512-thread build would give each group a
+// single CTA (more than SMs / 2 groups) and the sequences are at most 2048 pages (32K tokens), so
+// its 110 KB of shared memory holds the top-k keys and histogram; measured faster there (batch
+// 10-64 at 8K-32K), slower for the few large clusters of small batches or long contexts.
 // TWL_FUSED_THREADS=256 or 512 forces one.
-bool use_small_ctas(int groups) {
+bool use_small_ctas(int groups, int max_pages) {
   if (const char* env = getenv("TWL_FUSED_THREADS")) {
     const int t = atoi(env);
     if (t == 256) return true;
     if (t == 512) return false;
   }
-  return groups > num_sms();
+  return 2 * groups > num_sms() && max_pages <= 2048;
 }
 
 size_t decode_step_ws_bytes(int batch, int hq, int hkv, int max_pages, int max_budget) {
@@ -495,7 +498,7 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
     return TWL_ERR_INVALID_ARG;
   if (!(p > 0.f && p <= 1.f) || !(eps > 0.f) || isinf(eps)) return TWL_ERR_INVALID_ARG;
   if ((st = check_budget(budget_pages, budget_div, max_budget, k.max_pages)) != TWL_OK) return st;
-  bool small = use_small_ctas(k.batch * k.hkv);
+  bool small = use_small_ctas(k.batch * k.hkv, k.max_pages);
   FusedPlan pl{};
   if (small) {
     pl = fused256::plan_fused(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
