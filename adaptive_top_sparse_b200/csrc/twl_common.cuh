@@ -150,6 +150,52 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int* total) 
   return r;
 }
 
+// ------------------------------------------------------------------ top-p bisection
+// The midpoint of the bisection on the threshold ([Notes] "Key designs", efficient top-p):
+// mid = lo + (hi - lo) * 0.5 in fp32.
+__device__ __forceinline__ float mid_of(float lo, float hi) {
+  return __fadd_rn(lo, __fmul_rn(__fsub_rn(hi, lo), 0.5f));
+}
+
+// The search on (0, top] when its test "mass(W >= mid) >= p" is known to equal "mid <= T": with
+// exact masses, mass(W >= t) is a non-increasing step function of t that changes only at values
+// of W, so the test passes exactly for t <= T = the largest weight v with mass(W >= v) >= p
+// (T = 0 when no weight qualifies).  lo = 0, hi = top; stop when hi - lo <= eps, when the
+// midpoint no longer splits, or after 64 steps; the threshold is lo (top when the test passes at
+// top itself).
+// Four steps per trip, predicated (the same steps and stops as one step per trip).  While
+// hi - lo >= 2^-100, (hi - lo) * 0.5 is exact, so fma(hi - lo, 0.5, lo) rounds the same sum as
+// lo + (hi - lo) * 0.5; eps >= 2^-100 keeps every tested width there.
+__device__ __forceinline__ float bisect_scalar(float top, float T, float eps) {
+  if (top <= T) return top;
+  float lo = 0.f, hi = top;
+  if (!(eps >= 0x1p-100f)) {
+#pragma unroll 1
+    for (int steps = 0; steps < 64; ++steps) {
+      if (__fsub_rn(hi, lo) <= eps) break;
+      const float mid = mid_of(lo, hi);
+      if (!(lo < mid && mid < hi)) break;
+      if (mid <= T) lo = mid;
+      else hi = mid;
+    }
+    return lo;
+  }
+  bool done = false;
+#pragma unroll 1
+  for (int steps = 0; steps < 64 && !done; steps += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float d = __fsub_rn(hi, lo);
+      const float mid = __fmaf_rn(d, 0.5f, lo);
+      done = done || d <= eps || !(lo < mid && mid < hi);
+      const bool down = mid <= T;
+      lo = !done && down ? mid : lo;
+      hi = !done && !down ? mid : hi;
+    }
+  }
+  return lo;
+}
+
 // ------------------------------------------------------------------ tensor-core helper
 // D = A(16x16 fp16, row) * B(16x8 fp16, col) + C, fp32 accumulate (register operands).
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,

@@ -779,56 +779,10 @@ __device__ float block_sum_fixed(float v, float* red) {
   return t;
 }
 
-// Bisection of the notes page's "Key designs" (efficient top-p), three levels per block
-// reduction: the seven midpoints the sequential search could visit next are computed exactly as it
-// would compute them (mid = lo + (hi - lo) * 0.5 in fp32), their masses are summed in one pass, and
-// the search then walks the tree taking the same decisions, stopping rules included.  Each mass is
-// the same per-thread sum and the same block reduction as a one-threshold pass, so every decision
-// is the one the one-midpoint-per-pass loop with this reduction would take.
-__device__ __forceinline__ float mid_of(float lo, float hi) {
-  return __fadd_rn(lo, __fmul_rn(__fsub_rn(hi, lo), 0.5f));
-}
-
 // Weight in fixed point (units of 2^-48; W <= 1): integer sums are exact up to the conversion and
 // independent of the order of the terms, so the live-set masses do not depend on the order in
 // which the other CTAs pushed the entries.
 __device__ __forceinline__ long long w_fixed(float w) { return __float2ll_rn(w * 281474976710656.f); }
-
-// The search on (0, top]: lo = 0, hi = top; the midpoint test is "mid <= T" (see
-// top_p_from_live); stop when hi - lo <= eps, when the midpoint no longer splits, or after 64
-// steps; the threshold is lo (top when the test passes at top itself).
-// Four steps per trip, predicated (the same steps and stops as one step per trip).  While
-// hi - lo >= 2^-100, (hi - lo) * 0.5 is exact, so fma(hi - lo, 0.5, lo) rounds the same sum as
-// lo + (hi - lo) * 0.5; eps >= 2^-100 keeps every tested width there.
-__device__ __forceinline__ float bisect_scalar(float top, float T, float eps) {
-  if (top <= T) return top;
-  float lo = 0.f, hi = top;
-  if (!(eps >= 0x1p-100f)) {
-#pragma unroll 1
-    for (int steps = 0; steps < 64; ++steps) {
-      if (__fsub_rn(hi, lo) <= eps) break;
-      const float mid = mid_of(lo, hi);
-      if (!(lo < mid && mid < hi)) break;
-      if (mid <= T) lo = mid;
-      else hi = mid;
-    }
-    return lo;
-  }
-  bool done = false;
-#pragma unroll 1
-  for (int steps = 0; steps < 64 && !done; steps += 4) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float d = __fsub_rn(hi, lo);
-      const float mid = __fmaf_rn(d, 0.5f, lo);
-      done = done || d <= eps || !(lo < mid && mid < hi);
-      const bool down = mid <= T;
-      lo = !done && down ? mid : lo;
-      hi = !done && !down ? mid : hi;
-    }
-  }
-  return lo;
-}
 
 // Threshold from the live set {W >= L} (n <= kThreads values lw, fixed-point copies lq).  Every
 // test of the search at mid > L counts only live weights, and mass(W >= t) is a non-increasing
@@ -862,6 +816,12 @@ __device__ float top_p_from_live(const float* lw, const long long* lq, int n, fl
   return bisect_scalar(top, fmaxf(L, Tp), eps);
 }
 
+// Bisection of the notes page's "Key designs" (efficient top-p), three levels per block
+// reduction: the seven midpoints the sequential search could visit next are computed exactly as it
+// would compute them (mid = lo + (hi - lo) * 0.5 in fp32), their masses are summed in one pass, and
+// the search then walks the tree taking the same decisions, stopping rules included.  Each mass is
+// the same per-thread sum and the same block reduction as a one-threshold pass, so every decision
+// is the one the one-midpoint-per-pass loop with this reduction would take.
 // The same search over all nc weights (shared memory or global), three levels of the bisection
 // tree per round: every round sums the masses of the 7 candidate midpoints below (lo, hi) at once.
 __device__ float bisect_block(const float* W, bool staged, int nc, float top, float p, float eps,

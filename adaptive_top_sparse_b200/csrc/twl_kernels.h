@@ -52,6 +52,12 @@ cudaError_t launch_softmax_rows(int hq, const KV& kv, const int* sel_pages, cons
                                 int max_budget, float* weights, int* cand_count,
                                 cudaStream_t s);
 
+// twl_prune_rows.cu: the read-once pruner; cudaErrorNotSupported (nothing launched) when the
+// rows do not fit it
+cudaError_t launch_prune_rows(const float* w, const int* row_len, const int* row_len_cap,
+                              int rows, int row_stride, float p, float eps, float* m_out,
+                              int* kept_count, int* kept_idx, cudaStream_t s);
+
 // twl_prune.cu
 cudaError_t launch_prune(const float* w, const int* row_len, const int* row_len_cap, int rows,
                          int row_stride, float p, float eps, float* m_out, int* kept_count,

@@ -9,6 +9,8 @@
 // from global memory / L2 each round).  Every round is one block reduction of the mass above the
 // midpoint, in a fixed order, so all threads take the same branch.  The kept indices are
 // compacted in ascending order with a block scan.
+#include <stdlib.h>
+
 #include "twl_common.cuh"
 #include "twl_kernels.h"
 
@@ -98,6 +100,12 @@ __global__ void __launch_bounds__(kPruneThreads)
 cudaError_t launch_prune(const float* w, const int* row_len, const int* row_len_cap, int rows,
                          int row_stride, float p, float eps, float* m_out, int* kept_count,
                          int* kept_idx, cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  if (!getenv("TWL_PRUNE_BISECT")) {
+    const cudaError_t e = launch_prune_rows(w, row_len, row_len_cap, rows, row_stride, p, eps,
+                                            m_out, kept_count, kept_idx, s);
+    if (e != cudaErrorNotSupported) return e;
+  }
   const int staged = row_stride <= kPruneSmemFloats;
   const size_t smem = staged ? (size_t)row_stride * sizeof(float) : 0;
   if (smem > 48 * 1024) {

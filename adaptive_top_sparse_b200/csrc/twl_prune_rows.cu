@@ -1,0 +1,916 @@
+// Top-p thresholds of many independent weight rows, each row read from HBM once.
+//
+// "Twilight: Adaptive Attention Sparsity with Hierarchical Top-p Pruning", notes page, "Key
+// designs" (efficient top-p): the threshold m is found by bisection, each step testing
+// mass(W >= mid) >= p, with no sort; summary, section 4.2.
+//
+// mass(W >= t) is a non-increasing step function of t that only changes at values of W.  The
+// bisection's test at t is therefore the same as "t <= T", where T is the largest weight value v
+// with mass(W >= v) >= p (T = 0 when the row's mass stays below p).  This kernel finds T, then
+// bisect_scalar replays the bisection's midpoints, stopping rules and result as scalar arithmetic.
+// T is a mass-weighted order statistic, found over the row held in registers with shared-memory
+// atomics for a small share of the weights only (one shared atomic costs about as much issue
+// bandwidth as the rest of a weight's work):
+//   bracket  a count histogram of the fp32 bit patterns over [L, max W] (1024 log-spaced bins)
+//            holding every heavy weight (>= 16 x the mean) and one in four of the others; its
+//            estimated mass profile gives a key range that holds T with high probability.
+//            L = (sum W - p) / (2 n): the weights below L sum to less than (sum - p) / 2, so T >= L.
+//   exact    one pass: the weights above the range add up to the mass above it (fp32 pairwise per
+//            thread, fp64 across threads); the weights inside it go to an exact histogram (count
+//            and sum of low mantissa bits per bin, so a bin's mass is an exact fp64 value).  If T
+//            lies outside the range, the range moves and the pass repeats.
+//   levels   the crossing bin's weights are histogrammed again on the next bits, until one value
+//            (or one weight, whose bits follow from the bin's sums) remains.
+// The fp32 part of the mass above the range is off by at most 2^-21 of it.  When the decision
+// that fixed T is closer than that to p, the pass repeats with that mass summed in fp64, so the
+// result is the one fp64 sums give.
+//
+// Layout: a CTA holds a slice of up to 32 * blockDim.x weights of a row in registers (32 per
+// thread, as 8 float4 chunks strided by the block); rows longer than 32768 weights are split over
+// a thread-block cluster whose CTAs merge their histograms through distributed shared memory.  The
+// grid is persistent: each CTA (cluster) walks rows r, r + G, ..., and while it works on one row
+// its threads' cp.async copies of the next row land in shared memory (every thread copies and
+// later reads back only its own chunks, so the hand-off needs no barrier).
+#include "twl_common.cuh"
+#include "twl_kernels.h"
+
+namespace twl {
+namespace {
+
+typedef unsigned __int128 u128;
+
+constexpr int kRE = 32;                     // weights per thread
+constexpr int kRMaxThreads = 1024;
+constexpr int kRSlice = kRE * kRMaxThreads;  // weights per CTA, at most
+constexpr int kRMaxCluster = 8;
+constexpr int kNB = 1024;                   // bins per histogram
+constexpr float kHeavy = 4.f;               // weights >= kHeavy * sum / n are always counted
+constexpr int kSample = 2;                  // one in kSample of the other weights is counted
+constexpr int kMaxBinShift = 17;            // exact bins: count * 2^shift < 2^32 per CTA
+constexpr uint32_t kNaNBits = 0xFFFFFFFFu;  // weights past the row's length
+
+// Optional phase clock (a probe build defines TWL_PRUNE_STAMP(slot) to record it); off by default.
+#ifndef TWL_PRUNE_STAMP
+#define TWL_PRUNE_STAMP(slot)
+#endif
+
+// ------------------------------------------------------------------ cluster helpers
+__device__ __forceinline__ void csync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ uint32_t crank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cnum() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+  return n;
+}
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ uint64_t ldc64(uint32_t addr) {
+  uint64_t v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ldc32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void stc32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+// the sum over the cluster's CTAs of the shared u32 at `ad` (this CTA's own when C == 1)
+__device__ __forceinline__ uint64_t csum32(uint32_t ad, int C) {
+  if (C == 1) return lds32(ad);
+  uint64_t s = 0;
+#pragma unroll
+  for (int q = 0; q < kRMaxCluster; ++q)
+    if (q < C) s += ldc32(mapa(ad, q));
+  return s;
+}
+
+// Shared-memory add and store at a shared address.
+__device__ __forceinline__ void red_add_u(uint32_t ad, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(ad), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts32(uint32_t ad, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(ad), "r"(v) : "memory");
+}
+// Predicated shared-memory add.
+__device__ __forceinline__ void red_add(uint32_t ad, uint32_t v, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q red.shared.add.u32 [%0], %1;\n\t}" ::"r"(
+          ad),
+      "r"(v), "r"((uint32_t)pred)
+      : "memory");
+}
+
+// Copy 16 bytes, of which `bytes` (0..16) are read from global memory and the rest zero-filled.
+__device__ __forceinline__ void cp_async_n(void* smem, const void* gmem, int bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr(smem)), "l"(gmem),
+               "r"(bytes));
+}
+
+// ------------------------------------------------------------------ exact masses
+__device__ __forceinline__ double pow2d(int k) {  // k in [-1022, 1023]
+  return __longlong_as_double((long long)(k + 1023) << 52);
+}
+// Mass of `cnt` weights whose bit patterns share the prefix of base_key above bit sh (sh <= 23,
+// so they share one exponent), `sum` the sum of their low sh bits: exact (the integer is below
+// 2^53).
+__device__ __forceinline__ double bin_mass(uint32_t base_key, uint64_t cnt, uint64_t sum) {
+  const int e = (int)(base_key >> 23);
+  const uint64_t lead = (base_key & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+  return (double)(cnt * lead + sum) * pow2d(max(e, 1) - 150);
+}
+
+// Smallest shift with (hi >> s) - (lo >> s) < kNB.
+__device__ __forceinline__ int span_shift(uint32_t lo, uint32_t hi) {
+  int s = 0;
+  while ((hi >> s) - (lo >> s) >= (uint32_t)kNB) ++s;
+  return s;
+}
+
+// ------------------------------------------------------------------ block scans
+// Exclusive prefix (thread order) and total; one fixed order.  sh: 33 entries.  Three barriers.
+__device__ double block_excl_d(double v, double* sh, double* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  double x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    double tt = lane < nw ? sh[lane] : 0.0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, tt, o);
+      if (lane >= o) tt += y;
+    }
+    if (lane < nw) sh[lane] = tt;
+  }
+  __syncthreads();
+  const double base = warp ? sh[warp - 1] : 0.0;
+  *total = sh[nw - 1];
+  const double prev = __shfl_up_sync(0xffffffffu, x, 1);
+  __syncthreads();
+  return base + (lane ? prev : 0.0);
+}
+__device__ float block_excl_f2(float a, float b, float* sh, float* tot_a, float* tot_b) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  float x = a;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  const float bs = warp_sum(b);
+  if (lane == 31) {
+    sh[warp] = x;
+    sh[33 + warp] = bs;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float tt = lane < nw ? sh[lane] : 0.f, tb = lane < nw ? sh[33 + lane] : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, tt, o);
+      if (lane >= o) tt += y;
+    }
+    tb = warp_sum(tb);
+    if (lane < nw) sh[lane] = tt;
+    if (lane == 0) sh[65] = tb;
+  }
+  __syncthreads();
+  const float base = warp ? sh[warp - 1] : 0.f;
+  *tot_a = sh[nw - 1];
+  *tot_b = sh[65];
+  const float prev = __shfl_up_sync(0xffffffffu, x, 1);
+  __syncthreads();
+  return base + (lane ? prev : 0.f);
+}
+// Exclusive prefix of 128-bit values (8 packed 16-bit counts in pass D).  sh: 33 entries.
+__device__ __forceinline__ u128 shfl_up_u128(u128 v, int o) {
+  const uint64_t lo = __shfl_up_sync(0xffffffffu, (uint64_t)v, o);
+  const uint64_t hi = __shfl_up_sync(0xffffffffu, (uint64_t)(v >> 64), o);
+  return ((u128)hi << 64) | lo;
+}
+__device__ u128 block_excl_u128(u128 v, u128* sh, u128* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  u128 x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const u128 y = shfl_up_u128(x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    u128 tt = lane < nw ? sh[lane] : (u128)0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const u128 y = shfl_up_u128(tt, o);
+      if (lane >= o) tt += y;
+    }
+    if (lane < nw) sh[lane] = tt;
+  }
+  __syncthreads();
+  const u128 base = warp ? sh[warp - 1] : (u128)0;
+  *total = sh[nw - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
+// ------------------------------------------------------------------ shared state
+struct RowSh {
+  u128 ush[33];
+  double dsh[33];
+  float fsh[66];
+  double cr_above;   // crossing of the last level: mass of every weight above its bin,
+  double cr_mass;    // the bin's mass,
+  uint64_t cr_cnt;   // its weight count
+  uint64_t cr_sum;   // and low-bit sum;
+  int cr_bin;        // the bin (-1: the mass never reaches p)
+  int cb;            // claims (atomicMax)
+  double cta_above;  // this CTA's mass above the key range (read by the cluster)
+  float wsum[32];
+  float cta_sum;
+  uint32_t top_key;  // f32_key of this CTA's largest weight (atomicMax)
+  int bhi, blo;      // bracket bins (atomicMax)
+  uint32_t cta_count[kRMaxCluster];  // kept weights per CTA of the cluster (written remotely)
+};
+
+// One level: bins nb-1 (largest values) .. 0, each thread a contiguous run of ceil(nb / threads);
+// `mass_of(b, &cnt, &sum)` gives the bin's exact mass.  Finds the first bin, from the top, at
+// which base + (the mass of the bins above and including it) reaches P.  Every thread walking
+// its run from its prefix claims its first such bin; the largest claim is the crossing (which
+// keeps the result deterministic when fp64 rounding makes neighbouring prefixes disagree).
+template <class F>
+__device__ void level_cross(int nb, double base, double P, F mass_of, RowSh& sh) {
+  const int per = (nb + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int b0 = nb - 1 - (int)threadIdx.x * per;
+  if (threadIdx.x == 0) sh.cb = -1;
+  double local = 0.0;
+  for (int e = 0; e < per && b0 - e >= 0; ++e) {
+    uint64_t c, s;
+    local += mass_of(b0 - e, &c, &s);
+  }
+  double total;
+  const double start = base + block_excl_d(local, sh.dsh, &total);
+  int claim = -1;
+  {
+    double run = start;
+    for (int e = 0; e < per && b0 - e >= 0; ++e) {
+      uint64_t c, s;
+      const double mb = mass_of(b0 - e, &c, &s);
+      if (run + mb >= P) {
+        claim = b0 - e;
+        break;
+      }
+      run += mb;
+    }
+  }
+  if (claim >= 0) atomicMax(&sh.cb, claim);
+  __syncthreads();
+  const int cb = sh.cb;
+  if (claim >= 0 && claim == cb) {  // the owner records the crossing
+    double run = start;
+    for (int e = 0; e < per && b0 - e >= 0; ++e) {
+      uint64_t c, s;
+      const double mb = mass_of(b0 - e, &c, &s);
+      if (b0 - e == cb) {
+        sh.cr_above = run;
+        sh.cr_mass = mb;
+        sh.cr_cnt = c;
+        sh.cr_sum = s;
+        break;
+      }
+      run += mb;
+    }
+  }
+  if (threadIdx.x == 0) sh.cr_bin = cb;
+  __syncthreads();
+}
+
+struct PruneRowsArgs {
+  const float* w;
+  const int* row_len;
+  const int* row_len_cap;
+  int rows, stride;
+  float p, eps;
+  float* m_out;
+  int* kept_count;
+  int* kept_idx;
+  int list_cap;  // per-thread entries of the exact pass's list
+};
+
+__device__ __forceinline__ int row_length(const PruneRowsArgs& a, int r) {
+  int n = a.row_len ? a.row_len[r] : a.stride;
+  if (a.row_len_cap) n = min(n, a.row_len_cap[r]);
+  return max(0, min(n, a.stride));
+}
+
+// This thread's chunks of row r's slice into shared memory (zero-filled past the row's end).
+__device__ __forceinline__ void prefetch_row(const PruneRowsArgs& a, int r, int q, float4* buf) {
+  const int T = blockDim.x, t = threadIdx.x;
+  const int len = row_length(a, r);
+  const float* row = a.w + (size_t)r * a.stride;
+  const int s0 = q * kRE * T;
+#pragma unroll
+  for (int k = 0; k < kRE / 4; ++k) {
+    const int o = s0 + 4 * (k * T + t);
+    const int bytes = 4 * max(0, min(4, len - o));
+    cp_async_n(buf + k * T + t, bytes > 0 ? row + o : row, bytes);
+  }
+  cp_async_commit();
+}
+
+__device__ __forceinline__ void clear_u32(uint32_t* h, int n) {
+  for (int i = threadIdx.x; i < n / 4; i += blockDim.x)
+    reinterpret_cast<uint4*>(h)[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Histogram of the weights whose bit pattern u has (u >> hs) == pre, binned by the next
+// hs - ls bits (count, and sum of the low ls bits), and the level's crossing.  `cnt`: shared
+// address of kNB u32 counts, then kNB u32 sums; zero on entry.
+// The weights come from this thread's list (lst: shared address of entry 0, entries T words
+// apart, nl of them) when the exact pass kept one, else from the registers.
+__device__ __forceinline__ void prefix_level(const float (&x)[kRE], bool use_list, uint32_t lst,
+                                             int nl, uint32_t pre, int hs, int ls, uint32_t cnt,
+                                             double base, double P, int C, RowSh& sh) {
+  const uint32_t nbm = (1u << (hs - ls)) - 1u, lm = (1u << ls) - 1u;
+  if (use_list) {
+    for (int j = 0; j < nl; ++j) {
+      const uint32_t u = lds32(lst + 4u * blockDim.x * j);
+      if ((u >> hs) == pre) {
+        const uint32_t ad = cnt + 4u * ((u >> ls) & nbm);
+        red_add_u(ad, 1u);
+        red_add_u(ad + 4u * kNB, u & lm);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kRE; ++i) {
+      const uint32_t u = __float_as_uint(x[i]);
+      const bool in = (u >> hs) == pre;  // pre is a prefix of a finite key: NaN never matches
+      const uint32_t ad = cnt + 4u * ((u >> ls) & nbm);
+      red_add(ad, 1u, in);
+      red_add(ad + 4u * kNB, u & lm, in && lm);
+    }
+  }
+  __syncthreads();
+  if (C > 1) csync();
+  auto mass = [&](int b, uint64_t* c, uint64_t* s) -> double {
+    *c = csum32(cnt + 4u * b, C);
+    *s = ls ? csum32(cnt + 4u * (kNB + b), C) : 0ull;
+    const uint32_t key = ((pre << (hs - ls)) | (uint32_t)b) << ls;
+    return bin_mass(key, *c, *s);
+  };
+  level_cross((int)nbm + 1, base, P, mass, sh);
+}
+
+__global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ RowSh sh;
+  const int T = blockDim.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int C = (int)cnum(), q = (int)crank();
+  const int cid = blockIdx.x / C, ncl = gridDim.x / C;
+  float4* buf = reinterpret_cast<float4*>(smem);  // [8][T]
+  // histogram regions of 2 x kNB u32: A (bracket counts), B (exact bins), and for a cluster C
+  // (first refinement level; one CTA alone uses A, which is dead by then); the second refinement
+  // level takes B (one CTA) or A (cluster: after the barrier that ends every read of A)
+  uint32_t* rA = reinterpret_cast<uint32_t*>(smem + (size_t)16 * (kRE / 4) * T);
+  uint32_t* rB = rA + 2 * kNB;
+  uint32_t* rC = C > 1 ? rB + 2 * kNB : rA;
+  uint32_t* rD = C > 1 ? rA : rB;
+  const int nreg = C > 1 ? 3 : 2;
+  // after the regions: 32 words that absorb the sampled adds of weights outside the window, then
+  // the per-thread lists of the exact pass ((list_cap + 1) rows of T words; the last row absorbs
+  // the stores of weights outside the range)
+  const uint32_t a_dummy = saddr(rA + 2 * kNB * nreg) + 4u * (t & 31);
+  const uint32_t a_list = saddr(rA + 2 * kNB * nreg + 32) + 4u * t;
+
+  clear_u32(rA, 2 * kNB * nreg);
+  if (t == 0) sh.top_key = 0u;
+  if (cid < a.rows) prefetch_row(a, cid, q, buf);
+  __syncthreads();
+
+#pragma unroll 1
+  for (int r = cid; r < a.rows; r += ncl) {
+    const int len = row_length(a, r);
+    const int s0 = q * kRE * T;
+    TWL_PRUNE_STAMP(0);
+    cp_async_wait_all();
+    float x[kRE];
+#pragma unroll
+    for (int k = 0; k < kRE / 4; ++k) {
+      const float4 v = buf[k * T + t];
+      x[4 * k + 0] = v.x;
+      x[4 * k + 1] = v.y;
+      x[4 * k + 2] = v.z;
+      x[4 * k + 3] = v.w;
+    }
+    // weights past the end become NaN, which no comparison keeps and no histogram counts (nor
+    // negative, infinite or NaN weights)
+    if (s0 + kRE * T > len) {
+#pragma unroll
+      for (int k = 0; k < kRE / 4; ++k)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (s0 + 4 * (k * T + t) + j >= len) x[4 * k + j] = __uint_as_float(kNaNBits);
+    }
+    // pass 0: largest weight and the weight sum
+    float top = -INFINITY, tsum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kRE; ++i) {
+      top = fmaxf(top, x[i]);
+      tsum += fmaxf(x[i], 0.f);
+    }
+    top = warp_max(top);
+    tsum = warp_sum(tsum);
+    if (lane == 0) {
+      atomicMax(&sh.top_key, f32_key(top));
+      sh.wsum[warp] = tsum;
+    }
+    __syncthreads();  // every read of buf is done
+    if (r + ncl < a.rows) prefetch_row(a, r + ncl, q, buf);
+    if (t == 0) {
+      float sm = 0.f;
+      for (int w = 0; w < (T >> 5); ++w) sm += sh.wsum[w];
+      sh.cta_sum = sm;
+    }
+    if (C > 1) csync();
+    else __syncthreads();
+    uint32_t tk = 0u;
+    float total = 0.f;
+    for (int qq = 0; qq < C; ++qq) {
+      tk = max(tk, C > 1 ? ldc32(mapa(saddr(&sh.top_key), qq)) : sh.top_key);
+      total += C > 1 ? __uint_as_float(ldc32(mapa(saddr(&sh.cta_sum), qq))) : sh.cta_sum;
+    }
+    // back from the order key to the float (keys of non-negative values have the top bit set)
+    top = (tk & 0x80000000u) ? __uint_as_float(tk & 0x7FFFFFFFu) : __uint_as_float(~tk);
+
+    TWL_PRUNE_STAMP(1);
+    float m;
+    if (len == 0 || a.p >= 1.f || !(top > 0.f)) {
+      m = 0.f;  // p = 1 keeps every weight: an fp32 mass cannot resolve 1.0
+    } else if (isinf(top)) {
+      m = top;  // mass(W >= inf) is infinite
+    } else {
+      const uint32_t kt = __float_as_uint(top);
+      const double P = (double)a.p;
+      TWL_PRUNE_STAMP(2);
+      // ---- bracket: sampled count histogram over [L, top]
+      const float tot_lo = total * (1.f - 0x1p-16f);
+      const float L = tot_lo > a.p ? (tot_lo - a.p) / (2.f * (float)len) : 0.f;
+      const uint32_t kL = __float_as_uint(L);
+      const uint32_t kH = __float_as_uint(kHeavy * (total / (float)len));
+      const int s = span_shift(kL, kt);
+      const uint32_t win = (kt >> s) - (uint32_t)(kNB - 1);  // bin b <-> key prefix win + b
+      {
+        // heavy weights: all, behind one warp vote per chunk (they are rare); sampled ones: an
+        // add that every thread makes, to its own dummy word when the weight is not counted
+        const uint32_t aH = saddr(rA);
+#pragma unroll
+        for (int k = 0; k < kRE / 4; ++k) {
+          uint32_t ad[4];
+          bool hv[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t u = __float_as_uint(x[4 * k + j]);
+            const bool in = u - kL <= kt - kL;
+            hv[j] = in && u >= kH;
+            ad[j] = aH + 4u * ((u >> s) - win);
+            if ((j % kSample) == 0) red_add_u(in && !hv[j] ? ad[j] + 4u * kNB : a_dummy, 1u);
+          }
+          if (__any_sync(0xffffffffu, hv[0] || hv[1] || hv[2] || hv[3])) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) red_add(ad[j], 1u, hv[j]);
+          }
+        }
+      }
+      if (t == 0) {
+        sh.bhi = -1;
+        sh.blo = -1;
+      }
+      __syncthreads();
+      if (C > 1) csync();
+      const float pf = a.p;
+      {
+        // estimated mass per bin: (heavy + kSample x sampled) x the bin's middle value; the
+        // variance of the sampled part sets the margin
+        const int per = kNB / T;
+        const int b0 = kNB - 1 - t * per;
+        float le = 0.f, lv = 0.f;
+        for (int e = 0; e < per; ++e) {
+          const int b = b0 - e;
+          const int pk = (int)win + b;
+          const float ch = (float)csum32(saddr(rA + b), C);
+          const float cl = (float)csum32(saddr(rA + kNB + b), C);
+          if (pk >= 0 && ch + cl > 0.f) {
+            const float v = __uint_as_float(((uint32_t)pk << s) + ((1u << s) >> 1));
+            le += (ch + (float)kSample * cl) * v;
+            lv += (float)(kSample * (kSample - 1)) * cl * v * v;
+          }
+        }
+        float te, tv;
+        const float ex = block_excl_f2(le, lv, sh.fsh, &te, &tv);
+        const float delta = 3.f * sqrtf(tv) + te * ldexpf(1.f, s - 24) + 1e-7f * pf;
+        float run = ex;
+        bool got_hi = false, got_lo = false;
+        for (int e = 0; e < per; ++e) {
+          const int b = b0 - e;
+          const int pk = (int)win + b;
+          const float ch = (float)csum32(saddr(rA + b), C);
+          const float cl = (float)csum32(saddr(rA + kNB + b), C);
+          if (pk >= 0 && ch + cl > 0.f) {
+            const float v = __uint_as_float(((uint32_t)pk << s) + ((1u << s) >> 1));
+            run += (ch + (float)kSample * cl) * v;
+          }
+          if (!got_hi && run >= pf - delta) {
+            atomicMax(&sh.bhi, b);
+            got_hi = true;
+          }
+          if (!got_lo && run >= pf + delta) {
+            atomicMax(&sh.blo, b);
+            got_lo = true;
+          }
+        }
+      }
+      __syncthreads();
+      // key range [lo_key, hi_key], then aligned to whole bins of the exact histogram
+      const int bhi = min(kNB - 1, max(sh.bhi, 0) + 1), blo = max(0, sh.blo - 1);
+      long long lo_key = max((long long)kL, (long long)((int)win + blo) << s);
+      long long hi_key = ((((long long)((int)win + bhi)) + 1) << s) - 1;
+      if (hi_key > (long long)kt) hi_key = kt;
+      if (lo_key > hi_key) lo_key = hi_key;
+      if (C == 1) clear_u32(rC, 2 * kNB);  // rC = rA: its last reads were behind the barrier
+      uint32_t Tbits = 0u;
+      bool found = false, exact_above = false, use_list = false;
+      int nlist = 0;
+#pragma unroll 1
+      for (int tries = 0; tries < 64 && !found; ++tries) {
+        TWL_PRUNE_STAMP(3);
+        // ---- exact pass over [klo, khi]
+        int sb = span_shift((uint32_t)lo_key, (uint32_t)hi_key);
+        if (sb > kMaxBinShift) {  // keep the upper part; a miss moves the range down
+          lo_key = hi_key - ((long long)kNB << kMaxBinShift) + 1;
+          sb = span_shift((uint32_t)lo_key, (uint32_t)hi_key);
+        }
+        const uint32_t klo = ((uint32_t)lo_key >> sb) << sb;
+        const uint32_t khi = (((uint32_t)hi_key >> sb) << sb) | ((1u << sb) - 1u);
+        const float fkhi = __uint_as_float(khi);  // khi lies below the first infinite pattern
+        const uint32_t fc = saddr(rB);
+        double above_t;
+        if (!exact_above) {
+          // pairwise: quads, then a tree over the 8 quads (depth 5)
+          float c[kRE / 4];
+#pragma unroll
+          for (int k = 0; k < kRE / 4; ++k) {
+            const float y0 = x[4 * k] > fkhi ? x[4 * k] : 0.f;
+            const float y1 = x[4 * k + 1] > fkhi ? x[4 * k + 1] : 0.f;
+            const float y2 = x[4 * k + 2] > fkhi ? x[4 * k + 2] : 0.f;
+            const float y3 = x[4 * k + 3] > fkhi ? x[4 * k + 3] : 0.f;
+            c[k] = (y0 + y1) + (y2 + y3);
+          }
+          above_t = (double)(((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7])));
+        } else {
+          above_t = 0.0;
+#pragma unroll
+          for (int i = 0; i < kRE; ++i) above_t += x[i] > fkhi ? (double)x[i] : 0.0;
+        }
+        const uint32_t lm = (1u << sb) - 1u, k0 = klo >> sb;
+        // the weights in range go to this thread's list (a store per weight, no branch)
+        const int cap = a.list_cap;
+        nlist = 0;
+#pragma unroll
+        for (int i = 0; i < kRE; ++i) {
+          const uint32_t u = __float_as_uint(x[i]);
+          const bool in = u - klo <= khi - klo;
+          sts32(a_list + 4u * T * (in ? min(nlist, cap) : cap), u);
+          nlist += in ? 1 : 0;
+        }
+        use_list = !__syncthreads_or(nlist > cap);
+        if (use_list) {
+          for (int j = 0; j < nlist; ++j) {
+            const uint32_t u = lds32(a_list + 4u * T * j);
+            const uint32_t ad = fc + 4u * ((u >> sb) - k0);
+            red_add_u(ad, 1u);
+            red_add_u(ad + 4u * kNB, u & lm);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < kRE; ++i) {
+            const uint32_t u = __float_as_uint(x[i]);
+            const bool in = u - klo <= khi - klo;
+            const uint32_t ad = fc + 4u * ((u >> sb) - k0);
+            red_add(ad, 1u, in);
+            red_add(ad + 4u * kNB, u & lm, in && lm);
+          }
+        }
+        double above;
+        block_excl_d(above_t, sh.dsh, &above);  // its barriers also complete the histogram
+        if (C > 1) {
+          if (t == 0) sh.cta_above = above;
+          csync();
+          above = 0.0;
+          for (int qq = 0; qq < C; ++qq) {
+            const uint32_t ad = mapa(saddr(&sh.cta_above), qq);
+            above += __longlong_as_double((long long)ldc64(ad));
+          }
+        }
+        // bound on the fp32 pairwise sums (depth 5): 5 * 2^-24 of the mass, rounded up
+        const double err = exact_above ? 0.0 : above * 0x1p-21;
+        bool up = false, redo = false, used_levels = false;
+        double a_gt = 0.0, a_ge = 0.0;
+        if (above - err >= P) {
+          up = true;  // T lies above the range
+        } else if (above >= P || above + err >= P) {
+          redo = true;  // too close to call with the fp32 part
+        } else {
+          auto mass = [&](int b, uint64_t* c, uint64_t* sm) -> double {
+            *c = csum32(fc + 4u * b, C);
+            *sm = sb ? csum32(fc + 4u * (kNB + b), C) : 0ull;
+            return bin_mass(klo + ((uint32_t)b << sb), *c, *sm);
+          };
+          level_cross((int)((khi >> sb) - (klo >> sb)) + 1, above, P, mass, sh);
+          const int F = sh.cr_bin;
+          if (F >= 0) {
+            found = true;
+            const uint64_t cF = sh.cr_cnt, sF = sh.cr_sum;
+            const double aF = sh.cr_above, mF = sh.cr_mass;
+            const uint32_t pf0 = (klo >> sb) + (uint32_t)F;  // prefix of the crossing bin at sb
+            if (cF == 1 || sb == 0) {
+              Tbits = (pf0 << sb) | (uint32_t)sF;
+              a_gt = aF;
+              a_ge = aF + mF;
+            } else {
+              TWL_PRUNE_STAMP(4);
+              // ---- refinement levels on the crossing bin's weights
+              used_levels = true;
+              if (C > 1) csync();  // after this no CTA reads A, which may serve level 2
+              clear_u32(rD, 2 * kNB);
+              const int s2 = max(0, sb - 10);
+              prefix_level(x, use_list, a_list, nlist, pf0, sb, s2, saddr(rC), aF, P, C, sh);
+              const int S = sh.cr_bin;
+              const uint64_t cS = sh.cr_cnt, sS = sh.cr_sum;
+              const double aS = sh.cr_above, mS = sh.cr_mass;
+              const uint32_t pf1 = (pf0 << (sb - s2)) | (uint32_t)max(S, 0);
+              if (S < 0) {  // fp64 rounding: the finer bins fell short of the bin's sum
+                Tbits = (pf0 << sb);
+                a_gt = aF;
+                a_ge = aF + mF;
+              } else if (cS == 1 || s2 == 0) {
+                Tbits = (pf1 << s2) | (uint32_t)sS;
+                a_gt = aS;
+                a_ge = aS + mS;
+              } else {
+                prefix_level(x, use_list, a_list, nlist, pf1, s2, 0, saddr(rD), aS, P, C, sh);
+                const int V = sh.cr_bin;
+                Tbits = (pf1 << s2) | (uint32_t)max(V, 0);
+                a_gt = V < 0 ? aS : sh.cr_above;
+                a_ge = V < 0 ? aS + mS : sh.cr_above + sh.cr_mass;
+              }
+            }
+            // T is certain unless p lies within the fp32 bound of the masses that decided it
+            if (!exact_above && !(P - a_gt > err && a_ge - P >= err)) {
+              found = false;
+              redo = true;
+            }
+          }
+        }
+        if (!found) {
+          // prepare the next pass: the same range with fp64 sums, or the range moved (up when the
+          // mass above it reaches p, else down)
+          if (C > 1) csync();  // every CTA is done reading this pass's histograms
+          clear_u32(rB, 2 * kNB);
+          if (used_levels) clear_u32(rC, 2 * kNB);
+          if (redo) {
+            exact_above = true;
+          } else {
+            const long long span = 2 * ((long long)khi - (long long)klo + 1);
+            if (up) {
+              lo_key = (long long)khi + 1;
+              hi_key = min((long long)kt, (long long)khi + span);
+              if (lo_key > (long long)kt) {  // cannot happen: the mass above top is zero
+                found = true;
+                Tbits = kt;
+              }
+            } else if (klo == 0u) {  // the whole row's mass is below p
+              found = true;
+              Tbits = 0u;
+            } else {
+              hi_key = (long long)klo - 1;
+              lo_key = max(0ll, hi_key - span + 1);
+            }
+          }
+          __syncthreads();
+        }
+      }
+      TWL_PRUNE_STAMP(5);
+      m = bisect_scalar(top, __uint_as_float(Tbits), a.eps);
+    }
+
+    TWL_PRUNE_STAMP(6);
+    // pass D: kept = {W >= m}
+    uint32_t keepmask = 0u;
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int i = 0; i < kRE; ++i) {
+      const bool keep = x[i] >= m;
+      keepmask |= (keep ? 1u : 0u) << i;
+    }
+    cnt = __popc(keepmask);
+    uint32_t rbase[kRE / 4];
+    uint32_t cta_total = 0;
+    u128 pre = 0;
+    if (a.kept_idx) {
+      // ascending indices: per round k (8 chunks of 4 weights) the thread's count takes a 16-bit
+      // field of one 128-bit word; one exclusive scan places them all
+      u128 packed = 0;
+#pragma unroll
+      for (int k = 0; k < kRE / 4; ++k)
+        packed |= (u128)__popc((keepmask >> (4 * k)) & 0xFu) << (16 * k);
+      u128 tot;
+      pre = block_excl_u128(packed, sh.ush, &tot);
+#pragma unroll
+      for (int k = 0; k < kRE / 4; ++k) {
+        rbase[k] = cta_total;
+        cta_total += (uint32_t)(tot >> (16 * k)) & 0xFFFFu;
+      }
+    } else {
+      double tot;
+      block_excl_d((double)cnt, sh.dsh, &tot);
+      cta_total = (uint32_t)tot;
+    }
+    uint32_t cta_base = 0, row_total = cta_total;
+    if (C > 1) {
+      if (t == 0)
+        for (int qq = 0; qq < C; ++qq) stc32(mapa(saddr(&sh.cta_count[q]), qq), cta_total);
+      csync();  // also: every CTA has finished reading this CTA's histograms
+      row_total = 0;
+      for (int qq = 0; qq < C; ++qq) {
+        const uint32_t c = sh.cta_count[qq];
+        if (qq < q) cta_base += c;
+        row_total += c;
+      }
+    }
+    // Every read of this row's histograms and top (this CTA's and, in a cluster, the others')
+    // happened before the scan's barriers (and the cluster barrier): clear them for the next row.
+    clear_u32(rA, 2 * kNB * nreg);
+    if (t == 0) sh.top_key = 0u;
+    __syncthreads();  // cleared before the next row's histograms
+    if (a.kept_idx && keepmask) {
+      int* out = a.kept_idx + (size_t)r * a.stride;
+#pragma unroll
+      for (int k = 0; k < kRE / 4; ++k) {
+        uint32_t pos = cta_base + rbase[k] + ((uint32_t)(pre >> (16 * k)) & 0xFFFFu);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if ((keepmask >> (4 * k + j)) & 1u) out[pos++] = s0 + 4 * (k * T + t) + j;
+      }
+    }
+    TWL_PRUNE_STAMP(7);
+    if (q == 0 && t == 0) {
+      a.m_out[r] = m;
+      a.kept_count[r] = (int)row_total;
+    }
+  }
+  cp_async_wait_all();  // nothing is in flight at exit
+}
+
+struct RowsPlan {
+  int threads, cluster, grid, list_cap;
+  size_t smem;
+};
+
+// Dynamic shared memory: the prefetch buffer, the histogram regions, 32 dummy words, and the
+// exact pass's lists ((list_cap + 1) x threads words).
+size_t rows_smem(int threads, int cluster, int list_cap) {
+  return (size_t)16 * (kRE / 4) * threads + (size_t)4 * 2 * kNB * (cluster > 1 ? 3 : 2) + 128 +
+         (size_t)4 * (list_cap + 1) * threads;
+}
+
+// List entries per thread: what fits beside the CTAs an SM holds at 64 registers per thread
+// (1024 / threads of them), between 4 and 16.
+int rows_list_cap(int threads, int cluster) {
+  const int ctas = max(1, kRMaxThreads / threads);
+  const size_t per_cta = (size_t)(227 * 1024) / ctas - 2048;  // static shared memory and reserve
+  const size_t fixed = rows_smem(threads, cluster, -1);
+  const long long cap = per_cta > fixed ? (long long)((per_cta - fixed) / (4 * threads)) - 1 : 0;
+  return (int)min(16ll, cap);
+}
+
+}  // namespace
+
+// Plan for rows of `stride` weights: 0 threads when this kernel does not apply.
+static RowsPlan plan_rows(int rows, int stride) {
+  RowsPlan pl{0, 0, 0, 0, 0};
+  if (stride < 1 || stride > kRSlice * kRMaxCluster || (stride & 3)) return pl;
+  int threads = 32;
+  while (threads < kRMaxThreads && threads * kRE < stride) threads <<= 1;
+  const int cluster = (stride + threads * kRE - 1) / (threads * kRE);
+  pl.threads = threads;
+  pl.cluster = cluster;
+  pl.list_cap = max(4, rows_list_cap(threads, cluster));
+  pl.smem = rows_smem(threads, cluster, pl.list_cap);
+  // persistent grid: as many CTAs (clusters) as are resident at once, at most one per row
+  static int cache_key[32], cache_val[32];
+  static int cache_n = 0;
+  const int key = threads * 16 + cluster;
+  int per = -1;
+  for (int i = 0; i < cache_n; ++i)
+    if (cache_key[i] == key) per = cache_val[i];
+  if (per < 0) {
+    cudaFuncSetAttribute(k_prune_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)pl.smem);
+    if (cluster == 1) {
+      int nb = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_prune_rows, threads, pl.smem) !=
+          cudaSuccess)
+        nb = 0;
+      per = nb * num_sms();
+    } else {
+      if (cluster > 8)
+        cudaFuncSetAttribute(k_prune_rows, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)cluster);
+      cfg.blockDim = dim3((unsigned)threads);
+      cfg.dynamicSmemBytes = pl.smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)cluster;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, k_prune_rows, &cfg) != cudaSuccess) n = 0;
+      per = n;
+    }
+    cudaGetLastError();
+    if (cache_n < 32) {
+      cache_key[cache_n] = key;
+      cache_val[cache_n] = per;
+      ++cache_n;
+    }
+  }
+  if (per <= 0) {
+    pl.threads = 0;
+    return pl;
+  }
+  pl.grid = min(rows, per) * cluster;
+  return pl;
+}
+
+// Returns cudaErrorNotSupported (launching nothing) when the rows do not fit this kernel:
+// a row stride that is not a multiple of 4 weights or above 262144, or a base that is not
+// 16-byte aligned.
+cudaError_t launch_prune_rows(const float* w, const int* row_len, const int* row_len_cap,
+                              int rows, int row_stride, float p, float eps, float* m_out,
+                              int* kept_count, int* kept_idx, cudaStream_t s) {
+  if ((reinterpret_cast<uintptr_t>(w) & 15u) != 0) return cudaErrorNotSupported;
+  const RowsPlan pl = plan_rows(rows, row_stride);
+  if (pl.threads == 0) return cudaErrorNotSupported;
+  PruneRowsArgs a{w,   row_len, row_len_cap, rows,     row_stride,
+                  p,   eps,     m_out,       kept_count, kept_idx, pl.list_cap};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)pl.grid);
+  cfg.blockDim = dim3((unsigned)pl.threads);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)pl.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaFuncSetAttribute(k_prune_rows, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)pl.smem);
+  if (e != cudaSuccess) return e;
+  e = cudaLaunchKernelEx(&cfg, k_prune_rows, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace twl

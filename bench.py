@@ -758,6 +758,194 @@ def run_double_p(args, world, rank, local, p_cluster=0.95):
     }
 
 
+# ---------------------------------------------------------------------------------- pruner rows
+
+PRUNE_ROWS = 4096
+PRUNE_EPS = 1e-6
+L2_BYTES = 126 * 1024 * 1024
+
+
+def prune_rows_config(ns, copies):
+    return {"workload": "standalone top-p pruner: 4096 fp32 weight rows of length n (half "
+                        "Gaussian logits, sigma log-uniform in [0.1, 6]; half Zipf rank profiles, "
+                        "s in [0.5, 2]; 1% of rows with exact ties), softmax-normalised, "
+                        "p in {0.8, 0.9}, eps = 1e-6, seed 0",
+            "rows": PRUNE_ROWS, "n": ns, "p": [0.8, 0.9], "eps": PRUNE_EPS,
+            "l2": "no flush; each timed launch reads a copy of the rows not read since "
+                  f">= 4 x L2 bytes (copies per n: {copies})"}
+
+
+def prune_rows_bytes(n, rows, kept_total, with_idx):
+    """Read-once bytes of one launch: every weight (4 B), m and the kept count out (8 B per
+    row), and 4 B per kept index when the indices are written."""
+    return rows * (4 * n + 8) + (4 * kept_total if with_idx else 0)
+
+
+def run_prune_rows(args, world, rank, local):
+    """twl_prune_top_p alone on the standalone-pruner workload (4096 rows x n, survey config 5),
+    against its read-once HBM bound."""
+    from adaptive_top_sparse_b200 import twl
+    dev = torch.device("cuda", local)
+    ns = [int(x) for x in args.prune_n.split(",")]
+    peak, peak_kind = hbm_peak()
+    stream = torch.cuda.Stream(dev)
+    sweep = []
+    copies_by_n = {}
+    launches = 0
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    e2e = None
+    for n in ns:
+        w_np, _ = synth.config5_rows(PRUNE_ROWS, n, seed=0)
+        nbytes_in = w_np.nbytes
+        copies = max(1, -(-4 * L2_BYTES // nbytes_in))
+        copies_by_n[n] = copies
+        ws = [torch.from_numpy(w_np).to(dev) for _ in range(copies)]
+        sample = np.linspace(0, PRUNE_ROWS - 1, 8).astype(int)
+        w_sample = w_np[sample].copy()
+        m = torch.zeros(PRUNE_ROWS, dtype=torch.float32, device=dev)
+        kc = torch.zeros(PRUNE_ROWS, dtype=torch.int32, device=dev)
+        ki = torch.empty((PRUNE_ROWS, n), dtype=torch.int32, device=dev)
+        for p in (0.8, 0.9):
+            for with_idx in (False, True):
+                def step():
+                    for w in ws:
+                        twl.twl_prune_top_p(w, None, PRUNE_ROWS, n, p, PRUNE_EPS, m, kc,
+                                            ki if with_idx else None, stream=stream)
+                with torch.cuda.stream(stream):
+                    step()
+                stream.synchronize()
+                # properties that hold at any size: kept = {W >= m}, mass >= p (up to fp32 sums)
+                mn, kcn = m.cpu().numpy(), kc.cpu().numpy()
+                kin = ki[torch.from_numpy(sample).to(dev)].cpu().numpy() if with_idx else None
+                for j, r in enumerate(sample):
+                    keep = np.nonzero(w_sample[j] >= mn[r])[0]
+                    assert keep.size == kcn[r], f"n={n} row {r}: count"
+                    assert float(w_sample[j][keep].astype(np.float64).sum()) >= p - 1e-5
+                    if with_idx:
+                        assert np.array_equal(kin[j, : keep.size], keep), f"n={n} row {r}: ids"
+                kept_total = int(kcn.astype(np.int64).sum())
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=stream):
+                    step()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    for _ in range(args.warmup):
+                        graph.replay()
+                    e1.record(stream)
+                e1.synchronize()
+                # at least K replays, and at least half a second so the clock record has samples
+                per_replay = e0.elapsed_time(e1) / args.warmup
+                reps = int(max(args.steps, math.ceil(500.0 / max(per_replay, 1e-3))))
+                reps = int(max_over_ranks(float(reps), world))
+                torch.cuda.synchronize(dev)
+                barrier(world)
+                clocks.start()
+                with torch.cuda.stream(stream):
+                    e0.record(stream)
+                    for _ in range(reps):
+                        graph.replay()
+                    e1.record(stream)
+                e1.synchronize()
+                clk = clocks.stop()
+                ms = max_over_ranks(e0.elapsed_time(e1), world)
+                launches += reps * copies
+                us = ms * 1e3 / (reps * copies)
+                nb = prune_rows_bytes(n, PRUNE_ROWS, kept_total, with_idx)
+                sweep.append({"n": n, "p": p, "kept_idx": with_idx, "replays": reps,
+                              "launches_per_replay": copies, "us_per_launch": us,
+                              "rows_per_s": world * PRUNE_ROWS / (us / 1e6),
+                              "alg_bytes": nb, "achieved_gbs": nb / us / 1e3,
+                              "frac": nb / us / 1e3 / peak,
+                              "kept_fraction": kept_total / (PRUNE_ROWS * n), "clocks": clk})
+                del graph
+        if n == ns[-1] and not args.no_e2e:
+            # end to end through the C ABI: pinned host rows in, m and counts out, every step
+            w_host = torch.from_numpy(w_np).pin_memory()
+            m_host = torch.empty(PRUNE_ROWS, dtype=torch.float32).pin_memory()
+            kc_host = torch.empty(PRUNE_ROWS, dtype=torch.int32).pin_memory()
+            e2e_steps = 3
+            with torch.cuda.stream(stream):
+                ws[0].copy_(w_host, non_blocking=True)
+                twl.twl_prune_top_p(ws[0], None, PRUNE_ROWS, n, 0.9, PRUNE_EPS, m, kc,
+                                    None, stream=stream)
+                stream.synchronize()
+                barrier(world)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for _ in range(e2e_steps):
+                    ws[0].copy_(w_host, non_blocking=True)
+                    twl.twl_prune_top_p(ws[0], None, PRUNE_ROWS, n, 0.9, PRUNE_EPS, m, kc,
+                                        None, stream=stream)
+                    m_host.copy_(m, non_blocking=True)
+                    kc_host.copy_(kc, non_blocking=True)
+                e1.record(stream)
+            e1.synchronize()
+            launches += e2e_steps
+            ms = max_over_ranks(e0.elapsed_time(e1), world)
+            e2e = {"value": world * e2e_steps * PRUNE_ROWS / (ms / 1e3), "unit": "rows/s",
+                   "h2d_bytes_per_step": nbytes_in, "d2h_bytes_per_step": 8 * PRUNE_ROWS,
+                   "steps": e2e_steps, "n": n, "p": 0.9}
+            del w_host
+        del ws, ki
+        torch.cuda.empty_cache()
+    head = [r for r in sweep if r["n"] == ns[-1] and r["p"] == 0.9 and not r["kept_idx"]][0]
+    out = {
+        "metric": f"top-p pruner rows/s, 4096 fp32 rows of n = {ns[-1]}, p = 0.9, threshold and "
+                  "kept count (twl_prune_top_p); % of the read-once HBM roofline",
+        "value": head["rows_per_s"], "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["us_per_launch"] / 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": prune_rows_config(ns, copies_by_n),
+        "roofline": {"bound": "hbm", "achieved": head["achieved_gbs"], "peak": peak,
+                     "unit": "GB/s", "frac": head["frac"], "traffic": None,
+                     "kernel": "k_prune_rows (twl_prune_top_p)",
+                     "alg_bytes_per_launch": head["alg_bytes"],
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+        "e2e": e2e, "gpu_launches": launches, "clocks": head["clocks"], "sweep": sweep,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = prune_rows_cpu(ns[-1], 0.9)
+    return out
+
+
+def prune_rows_cpu(n, p, budget_s=10.0):
+    """The oracle's sort-based top-p (one host core) on rows of the same workload, until about
+    budget_s seconds of work; rows/s."""
+    from oracle import twl_oracle as O
+    w_np, _ = synth.config5_rows(64, n, seed=0)
+    done, t = 0, 0.0
+    with cpu_threads_guard():
+        while t < budget_s and done < w_np.shape[0]:
+            t0 = time.perf_counter()
+            O.top_p_sort(w_np[done], p)
+            t += time.perf_counter() - t0
+            done += 1
+    return {"value": done / t, "unit": "rows/s", "cores": 1, "kind": "oracle",
+            "sample": f"oracle sort + cumulative-sum top-p (numpy, fp64 sums) on {done} rows of "
+                      f"the n = {n} workload (same generator, seed 0), p = {p}, one host core"}
+
+
+def run_prune_rows_reference(args, world, rank):
+    if rank != 0:
+        return None
+    ns = [int(x) for x in args.prune_n.split(",")]
+    cb = prune_rows_cpu(ns[-1], 0.9, budget_s=min(60.0, 2.0 * max(1, args.steps)))
+    return {
+        "metric": f"top-p pruner rows/s, 4096 fp32 rows of n = {ns[-1]}, p = 0.9, threshold and "
+                  "kept count (twl_prune_top_p); % of the read-once HBM roofline",
+        "value": cb["value"], "unit": "rows/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * PRUNE_ROWS / cb["value"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference", "config": prune_rows_config(ns, {}),
+        "cpu_baseline": cb,
+        "e2e": {"value": cb["value"], "unit": "rows/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
 # ---------------------------------------------------------------------------------- bit widths
 
 def run_bits(args, world, rank, local):
@@ -871,8 +1059,11 @@ def main():
     ap.add_argument("--layers", type=int, default=None,
                     help="layer caches per step (default 32 for c2 and append, 4 for c3 / c4)")
     ap.add_argument("--workload", default="c2",
-                    choices=["c2", "c3", "c4", "c6", "append", "bits"],
-                    help="c2 is the headline; c3 / c4 and the append step are extra reports")
+                    choices=["c2", "c3", "c4", "c6", "append", "bits", "c5"],
+                    help="c2 is the headline; c3 / c4 / c6, the append step, the estimator bit "
+                         "widths and the standalone pruner (c5) are extra reports")
+    ap.add_argument("--prune-n", default="8192,32768,131072",
+                    help="row lengths of the c5 pruner workload (the last one is the headline)")
     args = ap.parse_args()
     global LAYERS
     if args.layers is None:
@@ -882,7 +1073,10 @@ def main():
         args.warmup = 3
     world, rank, local = dist_setup(args)
     try:
-        if args.workload == "bits":
+        if args.workload == "c5":
+            out = (run_prune_rows_reference(args, world, rank) if args.impl == "reference"
+                   else run_prune_rows(args, world, rank, local))
+        elif args.workload == "bits":
             out = run_bits(args, world, rank, local) if args.impl == "ours" else None
         elif args.workload == "append":
             out = (run_append_reference(args, world, rank) if args.impl == "reference"

@@ -184,6 +184,70 @@ def test_prune_rows(n, p):
         check_prune_row(w_np[r], m[r], int(kc[r]), ki[r], p, 1e-6, f"n{n} row {r}")
 
 
+def _hard_rows(n, seed):
+    """Rows that stress the threshold search: mass carried by many mid-sized weights, unnormalised
+    rows (sum far above or below 1, weights above 1), a geometric profile spanning the fp32 range,
+    near-uniform rows, a flat power law, and mostly-zero rows."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    r = np.full(n, 1e-9)
+    idx = rng.choice(n, size=max(8, n // 16), replace=False)
+    r[idx] = rng.uniform(0.9, 1.0, size=idx.size)
+    rows.append(r / r.sum())
+    rows.append(np.ones(n))                                     # sum n, every weight 1
+    rows.append(rng.uniform(0.0, 100.0, size=n))                # weights above 1
+    rows.append(0.5 * rng.dirichlet(np.ones(n)))                # sum 0.5 < p
+    g = 2.0 ** -np.arange(1, n + 1, dtype=np.float64)
+    rows.append(rng.permutation(np.maximum(g, 2.0 ** -140) / g.sum()))
+    u = np.exp(0.01 * rng.standard_normal(n))
+    rows.append(u / u.sum())                                    # near-uniform
+    z = np.arange(1, n + 1, dtype=np.float64) ** -0.3
+    rows.append(rng.permutation(z / z.sum()))                   # flat power law
+    sp = np.where(rng.random(n) < 0.9, 0.0, np.exp(rng.standard_normal(n)))
+    rows.append(sp / sp.sum())                                  # mostly zeros
+    return np.stack(rows).astype(np.float32)
+
+
+@pytest.mark.parametrize("n", [4096, 32768, 131072])
+@pytest.mark.parametrize("p", [0.5, 0.9, 0.999])
+def test_prune_hard_rows(n, p):
+    w_np = _hard_rows(n, seed=n + int(p * 1000))
+    rows = w_np.shape[0]
+    w = torch.from_numpy(w_np).cuda()
+    m = torch.zeros(rows, dtype=torch.float32, device="cuda")
+    kc = torch.zeros(rows, dtype=torch.int32, device="cuda")
+    ki = torch.full((rows, n), -1, dtype=torch.int32, device="cuda")
+    twl.twl_prune_top_p(w, None, rows, n, p, 1e-6, m, kc, ki)
+    m, kc, ki = np_(m), np_(kc), np_(ki)
+    for r in range(rows):
+        check_prune_row(w_np[r], m[r], int(kc[r]), ki[r], p, 1e-6, f"n{n} p{p} hard row {r}")
+
+
+@pytest.mark.parametrize("n", [8192, 131072])
+def test_prune_rows_ragged_lengths(n):
+    """Per-row lengths (row_len) shorter than the stride, including 0, 1 and non-multiples of 4."""
+    rows = 12
+    w_np, _ = synth.config5_rows(rows, n, seed=7)
+    lens_np = np.array([0, 1, 3, 5, 17, 1000, n // 2 + 1, n - 3, n - 1, n, 4097, 33], np.int32)
+    for r in range(rows):  # renormalise over the valid prefix
+        L = int(lens_np[r])
+        if L:
+            w_np[r, :L] /= w_np[r, :L].astype(np.float64).sum()
+    w = torch.from_numpy(w_np).cuda()
+    lens = torch.from_numpy(lens_np).cuda()
+    m = torch.zeros(rows, dtype=torch.float32, device="cuda")
+    kc = torch.zeros(rows, dtype=torch.int32, device="cuda")
+    ki = torch.full((rows, n), -1, dtype=torch.int32, device="cuda")
+    twl.twl_prune_top_p(w, lens, rows, n, 0.9, 1e-6, m, kc, ki)
+    m, kc, ki = np_(m), np_(kc), np_(ki)
+    for r in range(rows):
+        L = int(lens_np[r])
+        if L == 0:
+            assert kc[r] == 0
+            continue
+        check_prune_row(w_np[r, :L], m[r], int(kc[r]), ki[r], 0.9, 1e-6, f"n{n} len {L}")
+
+
 def test_prune_special_rows():
     n = 40
     rows = np.zeros((5, n), dtype=np.float32)
