@@ -40,7 +40,10 @@ namespace {
 typedef unsigned __int128 u128;
 
 constexpr int kRE = 32;                     // weights per thread
-constexpr int kRMaxThreads = 1024;
+#ifndef TWL_PRUNE_MAX_THREADS
+#define TWL_PRUNE_MAX_THREADS 1024
+#endif
+constexpr int kRMaxThreads = TWL_PRUNE_MAX_THREADS;
 constexpr int kRSlice = kRE * kRMaxThreads;  // weights per CTA, at most
 constexpr int kRMaxCluster = 8;
 constexpr int kNB = 1024;                   // bins per histogram
@@ -131,15 +134,6 @@ __device__ __forceinline__ void cp_async_n(void* smem, const void* gmem, int byt
 __device__ __forceinline__ double pow2d(int k) {  // k in [-1022, 1023]
   return __longlong_as_double((long long)(k + 1023) << 52);
 }
-// Mass of `cnt` weights whose bit patterns share the prefix of base_key above bit sh (sh <= 23,
-// so they share one exponent), `sum` the sum of their low sh bits: exact (the integer is below
-// 2^53).
-__device__ __forceinline__ double bin_mass(uint32_t base_key, uint64_t cnt, uint64_t sum) {
-  const int e = (int)(base_key >> 23);
-  const uint64_t lead = (base_key & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-  return (double)(cnt * lead + sum) * pow2d(max(e, 1) - 150);
-}
-
 // Smallest shift with (hi >> s) - (lo >> s) < kNB.
 __device__ __forceinline__ int span_shift(uint32_t lo, uint32_t hi) {
   int s = 0;
@@ -148,66 +142,6 @@ __device__ __forceinline__ int span_shift(uint32_t lo, uint32_t hi) {
 }
 
 // ------------------------------------------------------------------ block scans
-// Exclusive prefix (thread order) and total; one fixed order.  sh: 33 entries.  Three barriers.
-__device__ double block_excl_d(double v, double* sh, double* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  double x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sh[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    double tt = lane < nw ? sh[lane] : 0.0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double y = __shfl_up_sync(0xffffffffu, tt, o);
-      if (lane >= o) tt += y;
-    }
-    if (lane < nw) sh[lane] = tt;
-  }
-  __syncthreads();
-  const double base = warp ? sh[warp - 1] : 0.0;
-  *total = sh[nw - 1];
-  const double prev = __shfl_up_sync(0xffffffffu, x, 1);
-  __syncthreads();
-  return base + (lane ? prev : 0.0);
-}
-__device__ float block_excl_f2(float a, float b, float* sh, float* tot_a, float* tot_b) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  float x = a;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const float y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  const float bs = warp_sum(b);
-  if (lane == 31) {
-    sh[warp] = x;
-    sh[33 + warp] = bs;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    float tt = lane < nw ? sh[lane] : 0.f, tb = lane < nw ? sh[33 + lane] : 0.f;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, tt, o);
-      if (lane >= o) tt += y;
-    }
-    tb = warp_sum(tb);
-    if (lane < nw) sh[lane] = tt;
-    if (lane == 0) sh[65] = tb;
-  }
-  __syncthreads();
-  const float base = warp ? sh[warp - 1] : 0.f;
-  *tot_a = sh[nw - 1];
-  *tot_b = sh[65];
-  const float prev = __shfl_up_sync(0xffffffffu, x, 1);
-  __syncthreads();
-  return base + (lane ? prev : 0.f);
-}
 // Exclusive prefix of 128-bit values (8 packed 16-bit counts in pass D).  sh: 33 entries.
 __device__ __forceinline__ u128 shfl_up_u128(u128 v, int o) {
   const uint64_t lo = __shfl_up_sync(0xffffffffu, (uint64_t)v, o);
@@ -241,74 +175,96 @@ __device__ u128 block_excl_u128(u128 v, u128* sh, u128* total) {
 }
 
 // ------------------------------------------------------------------ shared state
+struct Cross {
+  uint64_t above;  // mass (level units) of the level's bins above the crossing bin
+  uint64_t mass;   // the crossing bin's mass
+  uint64_t cnt;    // its weight count
+  uint64_t sum;    // and low-bit sum
+  int bin;         // the bin (-1: the level's mass stays below what is needed)
+  int pad;
+};
+
 struct RowSh {
   u128 ush[33];
-  double dsh[33];
-  float fsh[66];
-  double cr_above;   // crossing of the last level: mass of every weight above its bin,
-  double cr_mass;    // the bin's mass,
-  uint64_t cr_cnt;   // its weight count
-  uint64_t cr_sum;   // and low-bit sum;
-  int cr_bin;        // the bin (-1: the mass never reaches p)
-  int cb;            // claims (atomicMax)
-  double cta_above;  // this CTA's mass above the key range (read by the cluster)
+  uint64_t wtot[32];  // per-warp totals of a level scan
+  double wpart[32];   // per-warp partial sums of the mass above the exact range
+  float fw[32], fv[32];
+  Cross cr;
+  double cta_above;   // this CTA's mass above the exact range (read by the cluster)
+  float m;            // the row's threshold (written by the owner of the last crossing)
+  int certain;        // the last crossing is certain under the fp32 bound
   float wsum[32];
   float cta_sum;
-  uint32_t top_key;  // f32_key of this CTA's largest weight (atomicMax)
-  int bhi, blo;      // bracket bins (atomicMax)
+  uint32_t top_key;   // f32_key of this CTA's largest weight (atomicMax)
+  uint32_t wcnt[32];  // per-warp kept counts
+  int bhi, blo;       // bracket bins (atomicMax)
   uint32_t cta_count[kRMaxCluster];  // kept weights per CTA of the cluster (written remotely)
 };
 
-// One level: bins nb-1 (largest values) .. 0, each thread a contiguous run of ceil(nb / threads);
-// `mass_of(b, &cnt, &sum)` gives the bin's exact mass.  Finds the first bin, from the top, at
-// which base + (the mass of the bins above and including it) reaches P.  Every thread walking
-// its run from its prefix claims its first such bin; the largest claim is the crossing (which
-// keeps the result deterministic when fp64 rounding makes neighbouring prefixes disagree).
+__device__ __forceinline__ uint64_t shfl_up_u64(uint64_t v, int o) {
+  return __shfl_up_sync(0xffffffffu, v, o);
+}
+
+// One level in exact integer masses: bins nb-1 (largest values) .. 0; thread t owns the run
+// [b0 - per + 1, b0], b0 = nb - 1 - t * per.  mass_of(b, &cnt, &sum) gives bin b's mass in the
+// level's unit.  Finds the first bin, from the top, at which the mass of the bins above and
+// including it reaches R (>= 1); the one thread whose run holds it records it in sh.cr (bin -1
+// when the level's total stays below R).  The integer sums are exact, so exactly one thread's
+// run [start, end) contains R.  Two barriers; the caller's barrier completes the histogram.
 template <class F>
-__device__ void level_cross(int nb, double base, double P, F mass_of, RowSh& sh) {
+__device__ void level_cross(int nb, uint64_t R, F mass_of, RowSh& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int per = (nb + (int)blockDim.x - 1) / (int)blockDim.x;
   const int b0 = nb - 1 - (int)threadIdx.x * per;
-  if (threadIdx.x == 0) sh.cb = -1;
-  double local = 0.0;
+  uint64_t local = 0;
   for (int e = 0; e < per && b0 - e >= 0; ++e) {
     uint64_t c, s;
     local += mass_of(b0 - e, &c, &s);
   }
-  double total;
-  const double start = base + block_excl_d(local, sh.dsh, &total);
-  int claim = -1;
-  {
-    double run = start;
+  uint64_t x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = shfl_up_u64(x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh.wtot[warp] = x;
+  if (threadIdx.x == 0) sh.cr.bin = -1;
+  __syncthreads();
+  uint64_t wt = lane < nw ? sh.wtot[lane] : 0ull;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = shfl_up_u64(wt, o);
+    if (lane >= o) wt += y;
+  }
+  const uint64_t wp = __shfl_sync(0xffffffffu, wt, (warp + 31) & 31);
+  const uint64_t start = (warp ? wp : 0ull) + x - local;
+  if (start < R && R <= start + local) {
+    uint64_t run = start;
     for (int e = 0; e < per && b0 - e >= 0; ++e) {
       uint64_t c, s;
-      const double mb = mass_of(b0 - e, &c, &s);
-      if (run + mb >= P) {
-        claim = b0 - e;
+      const uint64_t mb = mass_of(b0 - e, &c, &s);
+      if (run + mb >= R) {
+        sh.cr.above = run;
+        sh.cr.mass = mb;
+        sh.cr.cnt = c;
+        sh.cr.sum = s;
+        sh.cr.bin = b0 - e;
         break;
       }
       run += mb;
     }
   }
-  if (claim >= 0) atomicMax(&sh.cb, claim);
   __syncthreads();
-  const int cb = sh.cb;
-  if (claim >= 0 && claim == cb) {  // the owner records the crossing
-    double run = start;
-    for (int e = 0; e < per && b0 - e >= 0; ++e) {
-      uint64_t c, s;
-      const double mb = mass_of(b0 - e, &c, &s);
-      if (b0 - e == cb) {
-        sh.cr_above = run;
-        sh.cr_mass = mb;
-        sh.cr_cnt = c;
-        sh.cr_sum = s;
-        break;
-      }
-      run += mb;
-    }
-  }
-  if (threadIdx.x == 0) sh.cr_bin = cb;
-  __syncthreads();
+}
+
+// Integer mass of `cnt` weights whose bit patterns share the prefix of base_key above bit sh
+// (one exponent, as sh <= 23), `sum` the sum of their low sh bits, in units 2^(e_unit - 150):
+// (cnt * lead + sum) << (e - e_unit), e_unit <= e (callers keep the shift small).
+__device__ __forceinline__ uint64_t bin_units(uint32_t base_key, uint64_t cnt, uint64_t sum,
+                                              int e_unit) {
+  const int e = (int)(base_key >> 23);
+  const uint64_t lead = (base_key & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+  return (cnt * lead + sum) << (max(e, 1) - e_unit);
 }
 
 struct PruneRowsArgs {
@@ -350,13 +306,13 @@ __device__ __forceinline__ void clear_u32(uint32_t* h, int n) {
 }
 
 // Histogram of the weights whose bit pattern u has (u >> hs) == pre, binned by the next
-// hs - ls bits (count, and sum of the low ls bits), and the level's crossing.  `cnt`: shared
-// address of kNB u32 counts, then kNB u32 sums; zero on entry.
-// The weights come from this thread's list (lst: shared address of entry 0, entries T words
-// apart, nl of them) when the exact pass kept one, else from the registers.
+// hs - ls bits (count, and sum of the low ls bits), and the level's crossing (masses in units of
+// the prefix's exponent, so no shift).  The weights come from this thread's list (lst: shared
+// address of entry 0, entries T words apart, nl of them) when the exact pass kept one, else from
+// the registers.  `cnt`: shared address of kNB u32 counts, then kNB u32 sums; zero on entry.
 __device__ __forceinline__ void prefix_level(const float (&x)[kRE], bool use_list, uint32_t lst,
                                              int nl, uint32_t pre, int hs, int ls, uint32_t cnt,
-                                             double base, double P, int C, RowSh& sh) {
+                                             uint64_t R, int C, RowSh& sh) {
   const uint32_t nbm = (1u << (hs - ls)) - 1u, lm = (1u << ls) - 1u;
   if (use_list) {
     for (int j = 0; j < nl; ++j) {
@@ -379,19 +335,20 @@ __device__ __forceinline__ void prefix_level(const float (&x)[kRE], bool use_lis
   }
   __syncthreads();
   if (C > 1) csync();
-  auto mass = [&](int b, uint64_t* c, uint64_t* s) -> double {
+  const int e_unit = max((int)((pre << hs) >> 23), 1);
+  auto mass = [&](int b, uint64_t* c, uint64_t* s) -> uint64_t {
     *c = csum32(cnt + 4u * b, C);
     *s = ls ? csum32(cnt + 4u * (kNB + b), C) : 0ull;
     const uint32_t key = ((pre << (hs - ls)) | (uint32_t)b) << ls;
-    return bin_mass(key, *c, *s);
+    return bin_units(key, *c, *s, e_unit);
   };
-  level_cross((int)nbm + 1, base, P, mass, sh);
+  level_cross((int)nbm + 1, R, mass, sh);
 }
 
 __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ RowSh sh;
-  const int T = blockDim.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int T = blockDim.x, t = threadIdx.x, lane = t & 31, warp = t >> 5, nw = T >> 5;
   const int C = (int)cnum(), q = (int)crank();
   const int cid = blockIdx.x / C, ncl = gridDim.x / C;
   float4* buf = reinterpret_cast<float4*>(smem);  // [8][T]
@@ -453,23 +410,27 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
     }
     __syncthreads();  // every read of buf is done
     if (r + ncl < a.rows) prefetch_row(a, r + ncl, q, buf);
-    if (t == 0) {
-      float sm = 0.f;
-      for (int w = 0; w < (T >> 5); ++w) sm += sh.wsum[w];
-      sh.cta_sum = sm;
-    }
-    if (C > 1) csync();
-    else __syncthreads();
-    uint32_t tk = 0u;
     float total = 0.f;
-    for (int qq = 0; qq < C; ++qq) {
-      tk = max(tk, C > 1 ? ldc32(mapa(saddr(&sh.top_key), qq)) : sh.top_key);
-      total += C > 1 ? __uint_as_float(ldc32(mapa(saddr(&sh.cta_sum), qq))) : sh.cta_sum;
+    uint32_t tk = 0u;
+    if (C == 1) {
+      for (int w = 0; w < nw; ++w) total += sh.wsum[w];
+      tk = sh.top_key;
+    } else {
+      if (t == 0) {
+        float sm = 0.f;
+        for (int w = 0; w < nw; ++w) sm += sh.wsum[w];
+        sh.cta_sum = sm;
+      }
+      csync();
+      for (int qq = 0; qq < C; ++qq) {
+        tk = max(tk, ldc32(mapa(saddr(&sh.top_key), qq)));
+        total += __uint_as_float(ldc32(mapa(saddr(&sh.cta_sum), qq)));
+      }
     }
     // back from the order key to the float (keys of non-negative values have the top bit set)
     top = (tk & 0x80000000u) ? __uint_as_float(tk & 0x7FFFFFFFu) : __uint_as_float(~tk);
-
     TWL_PRUNE_STAMP(1);
+
     float m;
     if (len == 0 || a.p >= 1.f || !(top > 0.f)) {
       m = 0.f;  // p = 1 keeps every weight: an fp32 mass cannot resolve 1.0
@@ -514,10 +475,9 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
       }
       __syncthreads();
       if (C > 1) csync();
-      const float pf = a.p;
       {
         // estimated mass per bin: (heavy + kSample x sampled) x the bin's middle value; the
-        // variance of the sampled part sets the margin
+        // variance of the sampled part sets the margin.  Thread t holds bins b0 .. b0 - per + 1.
         const int per = kNB / T;
         const int b0 = kNB - 1 - t * per;
         float le = 0.f, lv = 0.f;
@@ -532,10 +492,28 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
             lv += (float)(kSample * (kSample - 1)) * cl * v * v;
           }
         }
-        float te, tv;
-        const float ex = block_excl_f2(le, lv, sh.fsh, &te, &tv);
+        float xs = le;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, xs, o);
+          if (lane >= o) xs += y;
+        }
+        const float wv = warp_sum(lv);
+        if (lane == 31) sh.fw[warp] = xs;
+        if (lane == 0) sh.fv[warp] = wv;
+        __syncthreads();
+        float ft = lane < nw ? sh.fw[lane] : 0.f;
+        const float tv = warp_sum(lane < nw ? sh.fv[lane] : 0.f);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, ft, o);
+          if (lane >= o) ft += y;
+        }
+        const float te = __shfl_sync(0xffffffffu, ft, 31);
+        const float wpf = __shfl_sync(0xffffffffu, ft, (warp + 31) & 31);
+        const float pf = a.p;
         const float delta = 3.f * sqrtf(tv) + te * ldexpf(1.f, s - 24) + 1e-7f * pf;
-        float run = ex;
+        float run = (warp ? wpf : 0.f) + (xs - le);
         bool got_hi = false, got_lo = false;
         for (int e = 0; e < per; ++e) {
           const int b = b0 - e;
@@ -564,9 +542,10 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
       if (hi_key > (long long)kt) hi_key = kt;
       if (lo_key > hi_key) lo_key = hi_key;
       if (C == 1) clear_u32(rC, 2 * kNB);  // rC = rA: its last reads were behind the barrier
-      uint32_t Tbits = 0u;
-      bool found = false, exact_above = false, use_list = false;
+      bool found = false, exact_above = false, use_list = false, m_pending = false;
       int nlist = 0;
+      uint32_t t_found = 0u;
+      m = 0.f;
 #pragma unroll 1
       for (int tries = 0; tries < 64 && !found; ++tries) {
         TWL_PRUNE_STAMP(3);
@@ -609,6 +588,10 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
           sts32(a_list + 4u * T * (in ? min(nlist, cap) : cap), u);
           nlist += in ? 1 : 0;
         }
+        // per-warp partial sums of the mass above (fixed order)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) above_t += __shfl_xor_sync(0xffffffffu, above_t, o);
+        if (lane == 0) sh.wpart[warp] = above_t;
         use_list = !__syncthreads_or(nlist > cap);
         if (use_list) {
           for (int j = 0; j < nlist; ++j) {
@@ -627,8 +610,9 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
             red_add(ad + 4u * kNB, u & lm, in && lm);
           }
         }
-        double above;
-        block_excl_d(above_t, sh.dsh, &above);  // its barriers also complete the histogram
+        double above = 0.0;
+        for (int w = 0; w < nw; ++w) above += sh.wpart[w];
+        __syncthreads();  // the exact histogram is complete
         if (C > 1) {
           if (t == 0) sh.cta_above = above;
           csync();
@@ -641,60 +625,73 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
         // bound on the fp32 pairwise sums (depth 5): 5 * 2^-24 of the mass, rounded up
         const double err = exact_above ? 0.0 : above * 0x1p-21;
         bool up = false, redo = false, used_levels = false;
-        double a_gt = 0.0, a_ge = 0.0;
+        TWL_PRUNE_STAMP(4);
         if (above - err >= P) {
           up = true;  // T lies above the range
         } else if (above >= P || above + err >= P) {
           redo = true;  // too close to call with the fp32 part
         } else {
-          auto mass = [&](int b, uint64_t* c, uint64_t* sm) -> double {
+          // masses of the exact bins in units of the range's lowest exponent (the range spans at
+          // most 1024 x 2^17 patterns = 16 binades, so a bin's mass stays below 2^59)
+          const int e_lo = max((int)(klo >> 23), 1);
+          const double unit = pow2d(e_lo - 150);
+          const double need = (P - above) / unit;
+          const uint64_t R = need >= 1.8e19 ? ~0ull : (uint64_t)ceil(need);
+          auto mass = [&](int b, uint64_t* c, uint64_t* sm) -> uint64_t {
             *c = csum32(fc + 4u * b, C);
             *sm = sb ? csum32(fc + 4u * (kNB + b), C) : 0ull;
-            return bin_mass(klo + ((uint32_t)b << sb), *c, *sm);
+            return bin_units(klo + ((uint32_t)b << sb), *c, *sm, e_lo);
           };
-          level_cross((int)((khi >> sb) - (klo >> sb)) + 1, above, P, mass, sh);
-          const int F = sh.cr_bin;
-          if (F >= 0) {
+          level_cross((int)((khi >> sb) - (klo >> sb)) + 1, max(R, (uint64_t)1), mass, sh);
+          const Cross F = sh.cr;
+          if (F.bin >= 0) {
             found = true;
-            const uint64_t cF = sh.cr_cnt, sF = sh.cr_sum;
-            const double aF = sh.cr_above, mF = sh.cr_mass;
-            const uint32_t pf0 = (klo >> sb) + (uint32_t)F;  // prefix of the crossing bin at sb
-            if (cF == 1 || sb == 0) {
-              Tbits = (pf0 << sb) | (uint32_t)sF;
-              a_gt = aF;
-              a_ge = aF + mF;
+            const uint32_t pf0 = (klo >> sb) + (uint32_t)F.bin;  // prefix of the bin at sb
+            uint32_t Tbits;
+            double a_gt = above + (double)F.above * unit, a_mass = (double)F.mass * unit;
+            if (F.cnt == 1 || sb == 0) {
+              Tbits = (pf0 << sb) | (uint32_t)F.sum;
             } else {
-              TWL_PRUNE_STAMP(4);
-              // ---- refinement levels on the crossing bin's weights
+              // ---- refinement levels on the crossing bin's weights (one exponent: unit 2^(e-150))
+              TWL_PRUNE_STAMP(5);
               used_levels = true;
               if (C > 1) csync();  // after this no CTA reads A, which may serve level 2
               clear_u32(rD, 2 * kNB);
+              const int e_f = max((int)((pf0 << sb) >> 23), 1);
+              const int sh_f = e_f - e_lo;  // fine units per bin unit: 2^sh_f
+              const double unit_f = pow2d(e_f - 150);
+              const uint64_t R1 = ((max(R, (uint64_t)1) - F.above) + ((1ull << sh_f) - 1ull)) >> sh_f;
               const int s2 = max(0, sb - 10);
-              prefix_level(x, use_list, a_list, nlist, pf0, sb, s2, saddr(rC), aF, P, C, sh);
-              const int S = sh.cr_bin;
-              const uint64_t cS = sh.cr_cnt, sS = sh.cr_sum;
-              const double aS = sh.cr_above, mS = sh.cr_mass;
-              const uint32_t pf1 = (pf0 << (sb - s2)) | (uint32_t)max(S, 0);
-              if (S < 0) {  // fp64 rounding: the finer bins fell short of the bin's sum
-                Tbits = (pf0 << sb);
-                a_gt = aF;
-                a_ge = aF + mF;
-              } else if (cS == 1 || s2 == 0) {
-                Tbits = (pf1 << s2) | (uint32_t)sS;
-                a_gt = aS;
-                a_ge = aS + mS;
+              prefix_level(x, use_list, a_list, nlist, pf0, sb, s2, saddr(rC), max(R1, (uint64_t)1), C,
+                           sh);
+              const Cross S = sh.cr;
+              const uint32_t pf1 = (pf0 << (sb - s2)) | (uint32_t)max(S.bin, 0);
+              if (S.bin < 0) {  // unreachable: the finer bins sum exactly to the crossing bin
+                Tbits = pf0 << sb;
+              } else if (S.cnt == 1 || s2 == 0) {
+                Tbits = (pf1 << s2) | (uint32_t)S.sum;
+                a_gt += (double)S.above * unit_f;
+                a_mass = (double)S.mass * unit_f;
               } else {
-                prefix_level(x, use_list, a_list, nlist, pf1, s2, 0, saddr(rD), aS, P, C, sh);
-                const int V = sh.cr_bin;
-                Tbits = (pf1 << s2) | (uint32_t)max(V, 0);
-                a_gt = V < 0 ? aS : sh.cr_above;
-                a_ge = V < 0 ? aS + mS : sh.cr_above + sh.cr_mass;
+                prefix_level(x, use_list, a_list, nlist, pf1, s2, 0, saddr(rD),
+                             max(R1 - S.above, (uint64_t)1), C, sh);
+                const Cross V = sh.cr;
+                Tbits = (pf1 << s2) | (uint32_t)max(V.bin, 0);
+                a_gt += (double)S.above * unit_f;
+                a_mass = (double)S.mass * unit_f;
+                if (V.bin >= 0) {
+                  a_gt += (double)V.above * unit_f;
+                  a_mass = (double)V.mass * unit_f;
+                }
               }
             }
             // T is certain unless p lies within the fp32 bound of the masses that decided it
-            if (!exact_above && !(P - a_gt > err && a_ge - P >= err)) {
+            if (!exact_above && !(P - a_gt > err && a_gt + a_mass - P >= err)) {
               found = false;
               redo = true;
+            } else {
+              t_found = Tbits;
+              m_pending = true;
             }
           }
         }
@@ -713,11 +710,11 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
               hi_key = min((long long)kt, (long long)khi + span);
               if (lo_key > (long long)kt) {  // cannot happen: the mass above top is zero
                 found = true;
-                Tbits = kt;
+                m = top;
               }
             } else if (klo == 0u) {  // the whole row's mass is below p
               found = true;
-              Tbits = 0u;
+              m = 0.f;
             } else {
               hi_key = (long long)klo - 1;
               lo_key = max(0ll, hi_key - span + 1);
@@ -726,20 +723,18 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
           __syncthreads();
         }
       }
-      TWL_PRUNE_STAMP(5);
-      m = bisect_scalar(top, __uint_as_float(Tbits), a.eps);
+      if (m_pending) {  // the scalar replay of the bisection, once per CTA
+        if (t == 0) sh.m = bisect_scalar(top, __uint_as_float(t_found), a.eps);
+        __syncthreads();
+        m = sh.m;
+      }
     }
-
     TWL_PRUNE_STAMP(6);
+
     // pass D: kept = {W >= m}
     uint32_t keepmask = 0u;
-    uint32_t cnt = 0;
 #pragma unroll
-    for (int i = 0; i < kRE; ++i) {
-      const bool keep = x[i] >= m;
-      keepmask |= (keep ? 1u : 0u) << i;
-    }
-    cnt = __popc(keepmask);
+    for (int i = 0; i < kRE; ++i) keepmask |= (x[i] >= m ? 1u : 0u) << i;
     uint32_t rbase[kRE / 4];
     uint32_t cta_total = 0;
     u128 pre = 0;
@@ -758,9 +753,10 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
         cta_total += (uint32_t)(tot >> (16 * k)) & 0xFFFFu;
       }
     } else {
-      double tot;
-      block_excl_d((double)cnt, sh.dsh, &tot);
-      cta_total = (uint32_t)tot;
+      const uint32_t wc = __reduce_add_sync(0xffffffffu, (uint32_t)__popc(keepmask));
+      if (lane == 0) sh.wcnt[warp] = wc;
+      __syncthreads();
+      for (int w = 0; w < nw; ++w) cta_total += sh.wcnt[w];
     }
     uint32_t cta_base = 0, row_total = cta_total;
     if (C > 1) {
@@ -775,7 +771,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
       }
     }
     // Every read of this row's histograms and top (this CTA's and, in a cluster, the others')
-    // happened before the scan's barriers (and the cluster barrier): clear them for the next row.
+    // happened before the barriers above: clear them for the next row.
     clear_u32(rA, 2 * kNB * nreg);
     if (t == 0) sh.top_key = 0u;
     __syncthreads();  // cleared before the next row's histograms

@@ -105,27 +105,36 @@ def algorithmic_bytes(page_table, seq_lens, num_q_heads, num_kv_heads, sel_pages
     return total, parts
 
 
-def source_hash() -> str:
+KERNEL_SOURCES = {
+    "decode_step": ["twl_fused.cu", "twl_fused_256.cu", "twl_fused.h", "twl_common.cuh",
+                    "twl_kernels.h"],
+    "prune_rows": ["twl_prune_rows.cu", "twl_common.cuh", "twl_kernels.h"],
+}
+
+
+def source_hash(kernel: str = "decode_step") -> str:
+    """Hash of the sources one kernel is built from (a profile's traffic is reported only while
+    they are unchanged)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "adaptive_top_sparse_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def measured_traffic():
-    """DRAM bytes per layer-step from the committed ncu summary, if it matches these sources."""
-    path = os.path.join(ROOT, "profiles", "decode_step_traffic.json")
+def measured_traffic(kernel: str = "decode_step", key: str = "dram_bytes_per_layer_step"):
+    """DRAM bytes per launch from the committed ncu summary, if it matches these sources."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return None
-    if d.get("source_hash") != source_hash():
+    if d.get("source_hash") != source_hash(kernel):
         return None
-    return d.get("dram_bytes_per_layer_step")
+    return d.get(key)
 
 
 def hbm_peak():
@@ -900,7 +909,8 @@ def run_prune_rows(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "config": prune_rows_config(ns, copies_by_n),
         "roofline": {"bound": "hbm", "achieved": head["achieved_gbs"], "peak": peak,
-                     "unit": "GB/s", "frac": head["frac"], "traffic": None,
+                     "unit": "GB/s", "frac": head["frac"],
+                     "traffic": measured_traffic("prune_rows", f"dram_bytes_per_launch_n{ns[-1]}"),
                      "kernel": "k_prune_rows (twl_prune_top_p)",
                      "alg_bytes_per_launch": head["alg_bytes"],
                      "peak_kind": f"{peak_kind} HBM copy bandwidth"},

@@ -254,7 +254,13 @@ twl_status twl_estimate_nbit(const void* q, int32_t num_q_heads, const twl_paged
  * parallel work, no sort; [Summary] 4.2).  If mass(W >= max W) >= p then m = max W; else
  * lo = 0, hi = max W, mid = lo + (hi - lo)/2 (fp32); mass(W >= mid) >= p sets lo = mid, else
  * hi = mid; stop when hi - lo <= eps or mid no longer splits; m = lo.  p = 1 keeps every entry
- * (m = 0).  Masses are fp32 block sums in a fixed order.
+ * (m = 0).
+ * Rows whose stride is a multiple of 4 (at most 262144) on a 16-byte aligned base are read once:
+ * the test at mid equals "mid <= T" for T = the largest weight v with mass(W >= v) >= p, so T is
+ * found from bit-pattern histograms with exact per-bin masses and the bisection is replayed on
+ * it; the mass of the weights above the final histogram's range is an fp32-pairwise / fp64 sum
+ * (redone in fp64 when the decision falls within its error bound).  Other rows run the direct
+ * bisection with fp32 block sums.  Negative weights carry no mass; NaN weights are never kept.
  *   m_out      float [rows] out
  *   kept_count int32 [rows] out = |{i : W_i >= m}|
  *   kept_idx   int32 [rows][row_stride] out (ascending indices) or NULL */

@@ -30,5 +30,13 @@ def test_algorithmic_bytes_by_hand():
 
 def test_traffic_only_for_matching_sources(tmp_path, monkeypatch):
     assert bench.measured_traffic() in (None,) or isinstance(bench.measured_traffic(), int)
-    monkeypatch.setattr(bench, "source_hash", lambda: "not-the-captured-sources")
+    monkeypatch.setattr(bench, "source_hash", lambda kernel="decode_step": "not-the-sources")
     assert bench.measured_traffic() is None
+    assert bench.measured_traffic("prune_rows", "dram_bytes_per_launch_n131072") is None
+
+
+def test_prune_rows_bytes_by_hand():
+    # 3 rows of 8 weights: 4 B per weight read, m and the count written (8 B per row), 4 B per
+    # kept index when the indices are written
+    assert bench.prune_rows_bytes(8, 3, 5, False) == 3 * (32 + 8)
+    assert bench.prune_rows_bytes(8, 3, 5, True) == 3 * (32 + 8) + 20
