@@ -413,6 +413,44 @@ def run_ours(args, world, rank, local):
             "union_tokens_per_group": st["union_count"].reshape(-1).tolist(),
         },
     }
+    if args.p_sweep:
+        # the same layers at other p: per-head kept fractions beside the time (the config's sweep)
+        sweep = []
+        for p in (0.70, 0.85, 0.95):
+            layers[0].decode(qs[0], p, wl.eps, stats)
+            torch.cuda.synchronize(dev)
+            sp = {k: v.cpu().numpy() for k, v in stats.items()}
+            nb, _ = algorithmic_bytes(wl.page_table, wl.seq_lens, wl.num_q_heads,
+                                      wl.num_kv_heads, sp["sel_pages"], sp["sel_count"],
+                                      sp["union_count"])
+            frac = sp["kept_count"].reshape(-1) / np.maximum(sp["cand_count"].reshape(-1), 1)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for layer, q in zip(layers, qs):
+                    layer.decode(q, p, wl.eps, None, stream)
+            for _ in range(args.warmup):
+                g.replay()
+            torch.cuda.synchronize(dev)
+            barrier(world)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(args.steps):
+                    g.replay()
+                e1.record(stream)
+            e1.synchronize()
+            msp = max_over_ranks(e0.elapsed_time(e1), world)
+            us = msp * 1e3 / (args.steps * LAYERS)
+            sweep.append({
+                "p": p, "us_per_layer_step": us, "layer_steps_per_s": world * 1e6 / us,
+                "alg_bytes_per_layer_step": nb, "achieved_gbs": nb / us / 1e3,
+                "frac": nb / us / 1e3 / peak,
+                "kept_fraction_per_head": {
+                    "min": float(frac.min()), "mean": float(frac.mean()),
+                    "max": float(frac.max()),
+                    "quartiles": [float(v) for v in np.quantile(frac, [0.25, 0.5, 0.75])]},
+                "kept_tokens_per_head_mean": float(sp["kept_count"].mean())})
+            del g
+        out["p_sweep"] = sweep
     if rank == 0 and not args.no_cpu_baseline:
         wl_groups = [(0, 0)]
         with cpu_threads_guard():
@@ -1072,6 +1110,9 @@ def main():
                     choices=["c2", "c3", "c4", "c6", "append", "bits", "c5"],
                     help="c2 is the headline; c3 / c4 / c6, the append step, the estimator bit "
                          "widths and the standalone pruner (c5) are extra reports")
+    ap.add_argument("--p-sweep", action="store_true",
+                    help="also time the decode workload at p = 0.70, 0.85, 0.95 and report the "
+                         "per-head kept fractions (the long-context config's sweep)")
     ap.add_argument("--prune-n", default="8192,32768,131072",
                     help="row lengths of the c5 pruner workload (the last one is the headline)")
     args = ap.parse_args()
