@@ -248,6 +248,30 @@ def test_prune_rows_ragged_lengths(n):
         check_prune_row(w_np[r, :L], m[r], int(kc[r]), ki[r], 0.9, 1e-6, f"n{n} len {L}")
 
 
+@pytest.mark.parametrize("n", [8192, 32768, 131072])
+def test_prune_rows_full_size(n):
+    """The standalone-pruner workload at its full size (4096 rows, the launch the bench times:
+    persistent CTAs or clusters that each walk many rows).  Every row: kept = {W >= m} and the
+    kept mass reaches p; 48 sampled rows (spread over the launch): the full criteria against the
+    oracle, including the ascending index list."""
+    rows = 4096
+    w_np, _ = synth.config5_rows(rows, n, seed=11)
+    w = torch.from_numpy(w_np).cuda()
+    m = torch.zeros(rows, dtype=torch.float32, device="cuda")
+    kc = torch.zeros(rows, dtype=torch.int32, device="cuda")
+    ki = torch.full((rows, n), -1, dtype=torch.int32, device="cuda")
+    twl.twl_prune_top_p(w, None, rows, n, 0.9, 1e-6, m, kc, ki)
+    m, kc = np_(m), np_(kc)
+    keep = w >= torch.from_numpy(m).cuda()[:, None]
+    assert np.array_equal(keep.sum(dim=1).cpu().numpy(), kc), "kept counts"
+    mass = torch.where(keep, w, torch.zeros_like(w)).sum(dim=1, dtype=torch.float64).cpu().numpy()
+    assert np.all(mass >= 0.9 - 1e-5), f"kept mass below p: {mass.min()}"
+    sample = np.unique(np.concatenate([np.arange(8), np.linspace(0, rows - 1, 40).astype(int)]))
+    ki_s = ki[torch.from_numpy(sample).cuda()].cpu().numpy()
+    for j, r in enumerate(sample):
+        check_prune_row(w_np[r], m[r], int(kc[r]), ki_s[j], 0.9, 1e-6, f"n{n} row {r}")
+
+
 def test_prune_special_rows():
     n = 40
     rows = np.zeros((5, n), dtype=np.float32)
