@@ -345,7 +345,8 @@ __device__ __forceinline__ void prefix_level(const float (&x)[kRE], bool use_lis
   level_cross((int)nbm + 1, R, mass, sh);
 }
 
-__global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a) {
+// 64 registers per thread: 1024 threads per SM, in 1024 / kRMaxThreads CTAs of the largest size
+__global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_rows(PruneRowsArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ RowSh sh;
   const int T = blockDim.x, t = threadIdx.x, lane = t & 31, warp = t >> 5, nw = T >> 5;
@@ -412,15 +413,13 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
     if (r + ncl < a.rows) prefetch_row(a, r + ncl, q, buf);
     float total = 0.f;
     uint32_t tk = 0u;
+    // the per-warp sums, added by one warp-wide reduction (the same order in every warp)
+    const float cta_sum = warp_sum(lane < nw ? sh.wsum[lane] : 0.f);
     if (C == 1) {
-      for (int w = 0; w < nw; ++w) total += sh.wsum[w];
+      total = cta_sum;
       tk = sh.top_key;
     } else {
-      if (t == 0) {
-        float sm = 0.f;
-        for (int w = 0; w < nw; ++w) sm += sh.wsum[w];
-        sh.cta_sum = sm;
-      }
+      if (t == 0) sh.cta_sum = cta_sum;
       csync();
       for (int qq = 0; qq < C; ++qq) {
         tk = max(tk, ldc32(mapa(saddr(&sh.top_key), qq)));
@@ -453,19 +452,22 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
         const uint32_t aH = saddr(rA);
 #pragma unroll
         for (int k = 0; k < kRE / 4; ++k) {
-          uint32_t ad[4];
           bool hv[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint32_t u = __float_as_uint(x[4 * k + j]);
-            const bool in = u - kL <= kt - kL;
-            hv[j] = in && u >= kH;
-            ad[j] = aH + 4u * ((u >> s) - win);
-            if ((j % kSample) == 0) red_add_u(in && !hv[j] ? ad[j] + 4u * kNB : a_dummy, 1u);
+            hv[j] = u >= kH && u <= kt;  // heavy (kH >= kL: 4x the mean is above L)
+            if ((j % kSample) == 0) {
+              const bool in = u - kL <= kt - kL;
+              red_add_u(in && !hv[j] ? aH + 4u * ((u >> s) - win) + 4u * kNB : a_dummy, 1u);
+            }
           }
           if (__any_sync(0xffffffffu, hv[0] || hv[1] || hv[2] || hv[3])) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) red_add(ad[j], 1u, hv[j]);
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t u = __float_as_uint(x[4 * k + j]);
+              red_add(aH + 4u * ((u >> s) - win), 1u, hv[j]);
+            }
           }
         }
       }
@@ -610,8 +612,9 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
             red_add(ad + 4u * kNB, u & lm, in && lm);
           }
         }
-        double above = 0.0;
-        for (int w = 0; w < nw; ++w) above += sh.wpart[w];
+        double above = lane < nw ? sh.wpart[lane] : 0.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
         __syncthreads();  // the exact histogram is complete
         if (C > 1) {
           if (t == 0) sh.cta_above = above;
@@ -756,7 +759,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1) k_prune_rows(PruneRowsArgs a)
       const uint32_t wc = __reduce_add_sync(0xffffffffu, (uint32_t)__popc(keepmask));
       if (lane == 0) sh.wcnt[warp] = wc;
       __syncthreads();
-      for (int w = 0; w < nw; ++w) cta_total += sh.wcnt[w];
+      cta_total = __reduce_add_sync(0xffffffffu, lane < nw ? sh.wcnt[lane] : 0u);
     }
     uint32_t cta_base = 0, row_total = cta_total;
     if (C > 1) {
@@ -809,7 +812,7 @@ size_t rows_smem(int threads, int cluster, int list_cap) {
 // List entries per thread: what fits beside the CTAs an SM holds at 64 registers per thread
 // (1024 / threads of them), between 4 and 16.
 int rows_list_cap(int threads, int cluster) {
-  const int ctas = max(1, kRMaxThreads / threads);
+  const int ctas = max(1, 1024 / threads);  // CTAs per SM at 64 registers per thread
   const size_t per_cta = (size_t)(227 * 1024) / ctas - 2048;  // static shared memory and reserve
   const size_t fixed = rows_smem(threads, cluster, -1);
   const long long cap = per_cta > fixed ? (long long)((per_cta - fixed) / (4 * threads)) - 1 : 0;
