@@ -199,6 +199,10 @@ struct RowSh {
   uint32_t wcnt[32];  // per-warp kept counts
   int bhi, blo;       // bracket bins (atomicMax)
   uint32_t cta_count[kRMaxCluster];  // kept weights per CTA of the cluster (written remotely)
+  uint32_t gather[32];  // the crossing bin's weights, when it holds at most 32 (one CTA)
+  int gcount;
+  uint32_t g_t;         // their solve: T's bit pattern,
+  uint64_t g_gt, g_eq;  // the mass above T and at T (units of the bin's exponent)
 };
 
 __device__ __forceinline__ uint64_t shfl_up_u64(uint64_t v, int o) {
@@ -471,12 +475,14 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
           }
         }
       }
+      TWL_PRUNE_STAMP(8);
       if (t == 0) {
         sh.bhi = -1;
         sh.blo = -1;
       }
       __syncthreads();
       if (C > 1) csync();
+      TWL_PRUNE_STAMP(9);
       {
         // estimated mass per bin: (heavy + kSample x sampled) x the bin's middle value; the
         // variance of the sampled part sets the margin.  Thread t holds bins b0 .. b0 - per + 1.
@@ -543,6 +549,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
       long long hi_key = ((((long long)((int)win + bhi)) + 1) << s) - 1;
       if (hi_key > (long long)kt) hi_key = kt;
       if (lo_key > hi_key) lo_key = hi_key;
+      TWL_PRUNE_STAMP(10);
       if (C == 1) clear_u32(rC, 2 * kNB);  // rC = rA: its last reads were behind the barrier
       bool found = false, exact_above = false, use_list = false, m_pending = false;
       int nlist = 0;
@@ -594,6 +601,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) above_t += __shfl_xor_sync(0xffffffffu, above_t, o);
         if (lane == 0) sh.wpart[warp] = above_t;
+        TWL_PRUNE_STAMP(11);
         use_list = !__syncthreads_or(nlist > cap);
         if (use_list) {
           for (int j = 0; j < nlist; ++j) {
@@ -616,6 +624,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
         __syncthreads();  // the exact histogram is complete
+        TWL_PRUNE_STAMP(12);
         if (C > 1) {
           if (t == 0) sh.cta_above = above;
           csync();
@@ -645,6 +654,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
             *sm = sb ? csum32(fc + 4u * (kNB + b), C) : 0ull;
             return bin_units(klo + ((uint32_t)b << sb), *c, *sm, e_lo);
           };
+          if (t == 0) sh.gcount = 0;  // published by the level's barriers
           level_cross((int)((khi >> sb) - (klo >> sb)) + 1, max(R, (uint64_t)1), mass, sh);
           const Cross F = sh.cr;
           if (F.bin >= 0) {
@@ -654,6 +664,47 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
             double a_gt = above + (double)F.above * unit, a_mass = (double)F.mass * unit;
             if (F.cnt == 1 || sb == 0) {
               Tbits = (pf0 << sb) | (uint32_t)F.sum;
+            } else if (C == 1 && use_list && F.cnt <= 32) {
+              // ---- few weights in the crossing bin: gather them from the lists and rank them
+              // in one warp (exact integer masses in units of the bin's exponent)
+              const int e_f = max((int)((pf0 << sb) >> 23), 1);
+              const int sh_f = e_f - e_lo;
+              const double unit_f = pow2d(e_f - 150);
+              const uint64_t R1 = ((max(R, (uint64_t)1) - F.above) + ((1ull << sh_f) - 1ull)) >> sh_f;
+              for (int j = 0; j < nlist; ++j) {
+                const uint32_t u = lds32(a_list + 4u * T * j);
+                if ((u >> sb) == pf0) {
+                  const int g = atomicAdd(&sh.gcount, 1);
+                  if (g < 32) sh.gather[g] = u;
+                }
+              }
+              __syncthreads();
+              if (warp == 0) {
+                const int gc = min(sh.gcount, 32);
+                const uint32_t v = lane < gc ? sh.gather[lane] : 0u;
+                const bool ok = lane < gc;
+                // mass of the gathered weights >= v, and > v
+                uint64_t ge = 0, gt = 0;
+                for (int j = 0; j < gc; ++j) {
+                  const uint32_t w = __shfl_sync(0xffffffffu, v, j);
+                  const uint64_t mw = (w & 0x7FFFFFu) | ((w >> 23) ? 0x800000u : 0u);
+                  ge += w >= v ? mw : 0ull;
+                  gt += w > v ? mw : 0ull;
+                }
+                // T = the largest gathered value whose mass from the top reaches R1
+                const uint32_t cand = (ok && ge >= R1) ? v : 0u;
+                const uint32_t tv = __reduce_max_sync(0xffffffffu, cand);
+                const uint32_t at_t = __ballot_sync(0xffffffffu, ok && v == tv);  // every lane
+                if (ok && v == tv && lane == __ffs(at_t) - 1) {
+                  sh.g_t = tv;
+                  sh.g_gt = gt;
+                  sh.g_eq = ge - gt;
+                }
+              }
+              __syncthreads();
+              Tbits = sh.g_t;
+              a_gt += (double)sh.g_gt * unit_f;
+              a_mass = (double)sh.g_eq * unit_f;
             } else {
               // ---- refinement levels on the crossing bin's weights (one exponent: unit 2^(e-150))
               TWL_PRUNE_STAMP(5);
@@ -726,6 +777,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
           __syncthreads();
         }
       }
+      TWL_PRUNE_STAMP(13);
       if (m_pending) {  // the scalar replay of the bisection, once per CTA
         if (t == 0) sh.m = bisect_scalar(top, __uint_as_float(t_found), a.eps);
         __syncthreads();
