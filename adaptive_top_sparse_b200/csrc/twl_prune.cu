@@ -5,10 +5,13 @@
 // sum_{W[i] >= m} W[i] >= p; each round is one O(n) parallel pass, and O(log(max W / eps)) rounds
 // suffice.  Summary, section 4.2: the search is fused with the other top-p operations.
 //
-// One block per row.  The row is staged once in shared memory when it fits (else it is re-read
-// from global memory / L2 each round).  Every round is one block reduction of the mass above the
-// midpoint, in a fixed order, so all threads take the same branch.  The kept indices are
-// compacted in ascending order with a block scan.
+// This is the direct form of the search, used for rows that the read-once kernel of
+// twl_prune_rows.cu does not take (a stride that is not a multiple of 4 weights or above 262144,
+// or a base that is not 16-byte aligned); TWL_PRUNE_BISECT=1 selects it for every row.  One block
+// per row.  The row is staged once in shared memory when it fits (else it is re-read from global
+// memory / L2 each round).  Every round is one block reduction of the mass above the midpoint, in
+// a fixed order, so all threads take the same branch.  The kept indices are compacted in
+// ascending order with a block scan.
 #include <stdlib.h>
 
 #include "twl_common.cuh"
