@@ -52,11 +52,18 @@ cudaError_t launch_softmax_rows(int hq, const KV& kv, const int* sel_pages, cons
                                 int max_budget, float* weights, int* cand_count,
                                 cudaStream_t s);
 
-// twl_prune_rows.cu: the read-once pruner; cudaErrorNotSupported (nothing launched) when the
-// rows do not fit it
+// twl_prune_rows.cu (32 weights per thread) and twl_prune_rows64.cu (64): the read-once pruner;
+// cudaErrorNotSupported (nothing launched) when the rows do not fit it
+namespace rows32 {
 cudaError_t launch_prune_rows(const float* w, const int* row_len, const int* row_len_cap,
                               int rows, int row_stride, float p, float eps, float* m_out,
                               int* kept_count, int* kept_idx, cudaStream_t s);
+}
+namespace rows64 {
+cudaError_t launch_prune_rows(const float* w, const int* row_len, const int* row_len_cap,
+                              int rows, int row_stride, float p, float eps, float* m_out,
+                              int* kept_count, int* kept_idx, cudaStream_t s);
+}
 
 // twl_prune.cu
 cudaError_t launch_prune(const float* w, const int* row_len, const int* row_len_cap, int rows,

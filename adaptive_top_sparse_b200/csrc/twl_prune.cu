@@ -105,8 +105,13 @@ cudaError_t launch_prune(const float* w, const int* row_len, const int* row_len_
                          int* kept_idx, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
   if (!getenv("TWL_PRUNE_BISECT")) {
-    const cudaError_t e = launch_prune_rows(w, row_len, row_len_cap, rows, row_stride, p, eps,
-                                            m_out, kept_count, kept_idx, s);
+    // 64 weights per thread above 16384 weights per row (no cluster up to 32768), else 32
+    const cudaError_t e =
+        row_stride > 16384
+            ? rows64::launch_prune_rows(w, row_len, row_len_cap, rows, row_stride, p, eps, m_out,
+                                        kept_count, kept_idx, s)
+            : rows32::launch_prune_rows(w, row_len, row_len_cap, rows, row_stride, p, eps, m_out,
+                                        kept_count, kept_idx, s);
     if (e != cudaErrorNotSupported) return e;
   }
   const int staged = row_stride <= kPruneSmemFloats;

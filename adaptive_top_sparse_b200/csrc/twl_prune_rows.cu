@@ -25,9 +25,12 @@
 // that fixed T is closer than that to p, the pass repeats with that mass summed in fp64, so the
 // result is the one fp64 sums give.
 //
-// Layout: a CTA holds a slice of up to 32 * blockDim.x weights of a row in registers (32 per
-// thread, as 8 float4 chunks strided by the block); rows longer than 32768 weights are split over
-// a thread-block cluster whose CTAs merge their histograms through distributed shared memory.  The
+// Layout: a CTA holds a slice of kRE * blockDim.x weights of a row in registers (kRE per
+// thread, as float4 chunks strided by the block); rows longer than 32768 weights are split over
+// a thread-block cluster whose CTAs merge their histograms through distributed shared memory.
+// (This file is built twice: 32 weights per thread in CTAs of up to 1024 threads at 64 registers,
+// and 64 weights per thread in CTAs of up to 512 threads at 128 registers (twl_prune_rows64.cu),
+// which halves the per-row work that every warp repeats and suits rows above 16384 weights.)  The
 // grid is persistent: each CTA (cluster) walks rows r, r + G, ..., and while it works on one row
 // its threads' cp.async copies of the next row land in shared memory (every thread copies and
 // later reads back only its own chunks, so the hand-off needs no barrier).
@@ -39,7 +42,12 @@ namespace {
 
 typedef unsigned __int128 u128;
 
-constexpr int kRE = 32;                     // weights per thread
+#ifndef TWL_PRUNE_RE
+#define TWL_PRUNE_RE 32
+#endif
+constexpr int kRE = TWL_PRUNE_RE;           // weights per thread (32 or 64)
+static_assert(kRE == 32 || kRE == 64, "32 or 64 weights per thread");
+constexpr int kRounds = kRE / 4;            // float4 chunks per thread
 #ifndef TWL_PRUNE_MAX_THREADS
 #define TWL_PRUNE_MAX_THREADS 1024
 #endif
@@ -143,6 +151,7 @@ __device__ __forceinline__ int span_shift(uint32_t lo, uint32_t hi) {
 
 // ------------------------------------------------------------------ block scans
 // Exclusive prefix of 128-bit values (8 packed 16-bit counts in pass D).  sh: 33 entries.
+// Two of them at once (16 rounds of counts): the same scan on a pair.
 __device__ __forceinline__ u128 shfl_up_u128(u128 v, int o) {
   const uint64_t lo = __shfl_up_sync(0xffffffffu, (uint64_t)v, o);
   const uint64_t hi = __shfl_up_sync(0xffffffffu, (uint64_t)(v >> 64), o);
@@ -296,7 +305,7 @@ __device__ __forceinline__ void prefetch_row(const PruneRowsArgs& a, int r, int 
   const float* row = a.w + (size_t)r * a.stride;
   const int s0 = q * kRE * T;
 #pragma unroll
-  for (int k = 0; k < kRE / 4; ++k) {
+  for (int k = 0; k < kRounds; ++k) {
     const int o = s0 + 4 * (k * T + t);
     const int bytes = 4 * max(0, min(4, len - o));
     cp_async_n(buf + k * T + t, bytes > 0 ? row + o : row, bytes);
@@ -349,8 +358,8 @@ __device__ __forceinline__ void prefix_level(const float (&x)[kRE], bool use_lis
   level_cross((int)nbm + 1, R, mass, sh);
 }
 
-// 64 registers per thread: 1024 threads per SM, in 1024 / kRMaxThreads CTAs of the largest size
-__global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_rows(PruneRowsArgs a) {
+// 2 kRE registers per thread: 32768 / kRE threads per SM, in CTAs of up to kRMaxThreads
+__global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_prune_rows(PruneRowsArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ RowSh sh;
   const int T = blockDim.x, t = threadIdx.x, lane = t & 31, warp = t >> 5, nw = T >> 5;
@@ -360,7 +369,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
   // histogram regions of 2 x kNB u32: A (bracket counts), B (exact bins), and for a cluster C
   // (first refinement level; one CTA alone uses A, which is dead by then); the second refinement
   // level takes B (one CTA) or A (cluster: after the barrier that ends every read of A)
-  uint32_t* rA = reinterpret_cast<uint32_t*>(smem + (size_t)16 * (kRE / 4) * T);
+  uint32_t* rA = reinterpret_cast<uint32_t*>(smem + (size_t)16 * kRounds * T);
   uint32_t* rB = rA + 2 * kNB;
   uint32_t* rC = C > 1 ? rB + 2 * kNB : rA;
   uint32_t* rD = C > 1 ? rA : rB;
@@ -384,7 +393,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
     cp_async_wait_all();
     float x[kRE];
 #pragma unroll
-    for (int k = 0; k < kRE / 4; ++k) {
+    for (int k = 0; k < kRounds; ++k) {
       const float4 v = buf[k * T + t];
       x[4 * k + 0] = v.x;
       x[4 * k + 1] = v.y;
@@ -395,7 +404,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
     // negative, infinite or NaN weights)
     if (s0 + kRE * T > len) {
 #pragma unroll
-      for (int k = 0; k < kRE / 4; ++k)
+      for (int k = 0; k < kRounds; ++k)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           if (s0 + 4 * (k * T + t) + j >= len) x[4 * k + j] = __uint_as_float(kNaNBits);
@@ -455,7 +464,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
         // add that every thread makes, to its own dummy word when the weight is not counted
         const uint32_t aH = saddr(rA);
 #pragma unroll
-        for (int k = 0; k < kRE / 4; ++k) {
+        for (int k = 0; k < kRounds; ++k) {
           bool hv[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -571,16 +580,20 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
         double above_t;
         if (!exact_above) {
           // pairwise: quads, then a tree over the 8 quads (depth 5)
-          float c[kRE / 4];
+          float c[kRounds];
 #pragma unroll
-          for (int k = 0; k < kRE / 4; ++k) {
+          for (int k = 0; k < kRounds; ++k) {
             const float y0 = x[4 * k] > fkhi ? x[4 * k] : 0.f;
             const float y1 = x[4 * k + 1] > fkhi ? x[4 * k + 1] : 0.f;
             const float y2 = x[4 * k + 2] > fkhi ? x[4 * k + 2] : 0.f;
             const float y3 = x[4 * k + 3] > fkhi ? x[4 * k + 3] : 0.f;
             c[k] = (y0 + y1) + (y2 + y3);
           }
-          above_t = (double)(((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7])));
+#pragma unroll
+          for (int w = kRounds / 2; w >= 1; w >>= 1)
+#pragma unroll
+            for (int i = 0; i < w; ++i) c[i] += c[i + w];
+          above_t = (double)c[0];
         } else {
           above_t = 0.0;
 #pragma unroll
@@ -787,28 +800,32 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
     TWL_PRUNE_STAMP(6);
 
     // pass D: kept = {W >= m}
-    uint32_t keepmask = 0u;
+    uint64_t keepmask = 0ull;
 #pragma unroll
-    for (int i = 0; i < kRE; ++i) keepmask |= (x[i] >= m ? 1u : 0u) << i;
-    uint32_t rbase[kRE / 4];
+    for (int i = 0; i < kRE; ++i) keepmask |= (x[i] >= m ? 1ull : 0ull) << i;
+    uint32_t rbase[kRounds];
     uint32_t cta_total = 0;
-    u128 pre = 0;
+    u128 pre[(kRounds + 7) / 8];
     if (a.kept_idx) {
-      // ascending indices: per round k (8 chunks of 4 weights) the thread's count takes a 16-bit
-      // field of one 128-bit word; one exclusive scan places them all
-      u128 packed = 0;
+      // ascending indices: per round k (chunks of 4 weights) the thread's count takes a 16-bit
+      // field of a 128-bit word (8 rounds per word); one exclusive scan places them all
+      constexpr int kWords = (kRounds + 7) / 8;
+      u128 packed[kWords];
 #pragma unroll
-      for (int k = 0; k < kRE / 4; ++k)
-        packed |= (u128)__popc((keepmask >> (4 * k)) & 0xFu) << (16 * k);
-      u128 tot;
-      pre = block_excl_u128(packed, sh.ush, &tot);
+      for (int w = 0; w < kWords; ++w) packed[w] = 0;
 #pragma unroll
-      for (int k = 0; k < kRE / 4; ++k) {
+      for (int k = 0; k < kRounds; ++k)
+        packed[k / 8] |= (u128)__popcll((keepmask >> (4 * k)) & 0xFull) << (16 * (k % 8));
+      u128 tot[kWords];
+#pragma unroll
+      for (int w = 0; w < kWords; ++w) pre[w] = block_excl_u128(packed[w], sh.ush, &tot[w]);
+#pragma unroll
+      for (int k = 0; k < kRounds; ++k) {
         rbase[k] = cta_total;
-        cta_total += (uint32_t)(tot >> (16 * k)) & 0xFFFFu;
+        cta_total += (uint32_t)(tot[k / 8] >> (16 * (k % 8))) & 0xFFFFu;
       }
     } else {
-      const uint32_t wc = __reduce_add_sync(0xffffffffu, (uint32_t)__popc(keepmask));
+      const uint32_t wc = __reduce_add_sync(0xffffffffu, (uint32_t)__popcll(keepmask));
       if (lane == 0) sh.wcnt[warp] = wc;
       __syncthreads();
       cta_total = __reduce_add_sync(0xffffffffu, lane < nw ? sh.wcnt[lane] : 0u);
@@ -833,11 +850,11 @@ __global__ void __launch_bounds__(kRMaxThreads, 1024 / kRMaxThreads) k_prune_row
     if (a.kept_idx && keepmask) {
       int* out = a.kept_idx + (size_t)r * a.stride;
 #pragma unroll
-      for (int k = 0; k < kRE / 4; ++k) {
-        uint32_t pos = cta_base + rbase[k] + ((uint32_t)(pre >> (16 * k)) & 0xFFFFu);
+      for (int k = 0; k < kRounds; ++k) {
+        uint32_t pos = cta_base + rbase[k] + ((uint32_t)(pre[k / 8] >> (16 * (k % 8))) & 0xFFFFu);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          if ((keepmask >> (4 * k + j)) & 1u) out[pos++] = s0 + 4 * (k * T + t) + j;
+          if ((keepmask >> (4 * k + j)) & 1ull) out[pos++] = s0 + 4 * (k * T + t) + j;
       }
     }
     TWL_PRUNE_STAMP(7);
@@ -857,14 +874,14 @@ struct RowsPlan {
 // Dynamic shared memory: the prefetch buffer, the histogram regions, 32 dummy words, and the
 // exact pass's lists ((list_cap + 1) x threads words).
 size_t rows_smem(int threads, int cluster, int list_cap) {
-  return (size_t)16 * (kRE / 4) * threads + (size_t)4 * 2 * kNB * (cluster > 1 ? 3 : 2) + 128 +
+  return (size_t)16 * kRounds * threads + (size_t)4 * 2 * kNB * (cluster > 1 ? 3 : 2) + 128 +
          (size_t)4 * (list_cap + 1) * threads;
 }
 
 // List entries per thread: what fits beside the CTAs an SM holds at 64 registers per thread
 // (1024 / threads of them), between 4 and 16.
 int rows_list_cap(int threads, int cluster) {
-  const int ctas = max(1, 1024 / threads);  // CTAs per SM at 64 registers per thread
+  const int ctas = max(1, 32768 / kRE / threads);  // CTAs per SM at 2 kRE registers per thread
   const size_t per_cta = (size_t)(227 * 1024) / ctas - 2048;  // static shared memory and reserve
   const size_t fixed = rows_smem(threads, cluster, -1);
   const long long cap = per_cta > fixed ? (long long)((per_cta - fixed) / (4 * threads)) - 1 : 0;
@@ -872,6 +889,11 @@ int rows_list_cap(int threads, int cluster) {
 }
 
 }  // namespace
+
+#ifndef TWL_PRUNE_NS
+#define TWL_PRUNE_NS rows32
+#endif
+namespace TWL_PRUNE_NS {
 
 // Plan for rows of `stride` weights: 0 threads when this kernel does not apply.
 static RowsPlan plan_rows(int rows, int stride) {
@@ -964,4 +986,5 @@ cudaError_t launch_prune_rows(const float* w, const int* row_len, const int* row
   return cudaGetLastError();
 }
 
+}  // namespace TWL_PRUNE_NS
 }  // namespace twl

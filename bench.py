@@ -108,7 +108,7 @@ def algorithmic_bytes(page_table, seq_lens, num_q_heads, num_kv_heads, sel_pages
 KERNEL_SOURCES = {
     "decode_step": ["twl_fused.cu", "twl_fused_256.cu", "twl_fused.h", "twl_common.cuh",
                     "twl_kernels.h"],
-    "prune_rows": ["twl_prune_rows.cu", "twl_common.cuh", "twl_kernels.h"],
+    "prune_rows": ["twl_prune_rows.cu", "twl_prune_rows64.cu", "twl_common.cuh", "twl_kernels.h"],
 }
 
 
