@@ -615,7 +615,9 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
         for (int o = 16; o > 0; o >>= 1) above_t += __shfl_xor_sync(0xffffffffu, above_t, o);
         if (lane == 0) sh.wpart[warp] = above_t;
         TWL_PRUNE_STAMP(11);
-        use_list = !__syncthreads_or(nlist > cap);
+        // each thread takes its histogram adds from its list, or from its registers when its list
+        // overflowed (the histogram is the same either way)
+        use_list = nlist <= cap;
         if (use_list) {
           for (int j = 0; j < nlist; ++j) {
             const uint32_t u = lds32(a_list + 4u * T * j);
@@ -633,11 +635,11 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
             red_add(ad + 4u * kNB, u & lm, in && lm);
           }
         }
+        __syncthreads();  // the exact histogram and the per-warp sums are complete
+        TWL_PRUNE_STAMP(12);
         double above = lane < nw ? sh.wpart[lane] : 0.0;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
-        __syncthreads();  // the exact histogram is complete
-        TWL_PRUNE_STAMP(12);
         if (C > 1) {
           if (t == 0) sh.cta_above = above;
           csync();
@@ -677,18 +679,29 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
             double a_gt = above + (double)F.above * unit, a_mass = (double)F.mass * unit;
             if (F.cnt == 1 || sb == 0) {
               Tbits = (pf0 << sb) | (uint32_t)F.sum;
-            } else if (C == 1 && use_list && F.cnt <= 32) {
+            } else if (C == 1 && F.cnt <= 32) {
               // ---- few weights in the crossing bin: gather them from the lists and rank them
               // in one warp (exact integer masses in units of the bin's exponent)
               const int e_f = max((int)((pf0 << sb) >> 23), 1);
               const int sh_f = e_f - e_lo;
               const double unit_f = pow2d(e_f - 150);
               const uint64_t R1 = ((max(R, (uint64_t)1) - F.above) + ((1ull << sh_f) - 1ull)) >> sh_f;
-              for (int j = 0; j < nlist; ++j) {
-                const uint32_t u = lds32(a_list + 4u * T * j);
-                if ((u >> sb) == pf0) {
-                  const int g = atomicAdd(&sh.gcount, 1);
-                  if (g < 32) sh.gather[g] = u;
+              if (use_list) {
+                for (int j = 0; j < nlist; ++j) {
+                  const uint32_t u = lds32(a_list + 4u * T * j);
+                  if ((u >> sb) == pf0) {
+                    const int g = atomicAdd(&sh.gcount, 1);
+                    if (g < 32) sh.gather[g] = u;
+                  }
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < kRE; ++i) {
+                  const uint32_t u = __float_as_uint(x[i]);
+                  if ((u >> sb) == pf0) {  // a finite prefix: NaN never matches
+                    const int g = atomicAdd(&sh.gcount, 1);
+                    if (g < 32) sh.gather[g] = u;
+                  }
                 }
               }
               __syncthreads();
