@@ -816,6 +816,12 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
     uint64_t keepmask = 0ull;
 #pragma unroll
     for (int i = 0; i < kRE; ++i) keepmask |= (x[i] >= m ? 1ull : 0ull) << i;
+    if (C == 1) {
+      // every read of this row's histograms and top happened before the barriers above; the
+      // barriers of the count below publish the clears before the next row's adds
+      clear_u32(rA, 2 * kNB * nreg);
+      if (t == 0) sh.top_key = 0u;
+    }
     uint32_t rbase[kRounds];
     uint32_t cta_total = 0;
     u128 pre[(kRounds + 7) / 8];
@@ -855,11 +861,13 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
         row_total += c;
       }
     }
-    // Every read of this row's histograms and top (this CTA's and, in a cluster, the others')
-    // happened before the barriers above: clear them for the next row.
-    clear_u32(rA, 2 * kNB * nreg);
-    if (t == 0) sh.top_key = 0u;
-    __syncthreads();  // cleared before the next row's histograms
+    if (C > 1) {
+      // every read of this CTA's histograms and top, its own and the other CTAs', happened
+      // before the cluster barrier above: clear them for the next row
+      clear_u32(rA, 2 * kNB * nreg);
+      if (t == 0) sh.top_key = 0u;
+      __syncthreads();  // cleared before the next row's histograms
+    }
     if (a.kept_idx && keepmask) {
       int* out = a.kept_idx + (size_t)r * a.stride;
 #pragma unroll
