@@ -12,15 +12,17 @@
 // atomics for a small share of the weights only (one shared atomic costs about as much issue
 // bandwidth as the rest of a weight's work):
 //   bracket  a count histogram of the fp32 bit patterns over [L, max W] (1024 log-spaced bins)
-//            holding every heavy weight (>= 16 x the mean) and one in four of the others; its
+//            holding every heavy weight (>= 4 x the mean) and one in two of the others; its
 //            estimated mass profile gives a key range that holds T with high probability.
 //            L = (sum W - p) / (2 n): the weights below L sum to less than (sum - p) / 2, so T >= L.
 //   exact    one pass: the weights above the range add up to the mass above it (fp32 pairwise per
-//            thread, fp64 across threads); the weights inside it go to an exact histogram (count
-//            and sum of low mantissa bits per bin, so a bin's mass is an exact fp64 value).  If T
-//            lies outside the range, the range moves and the pass repeats.
-//   levels   the crossing bin's weights are histogrammed again on the next bits, until one value
-//            (or one weight, whose bits follow from the bin's sums) remains.
+//            thread, fp64 across threads); the weights inside it go to per-thread lists, then to
+//            an exact histogram (count and sum of low mantissa bits per bin, so a bin's mass is an
+//            exact integer in units of the range's lowest exponent).  If T lies outside the range,
+//            the range moves and the pass repeats.
+//   levels   a crossing bin of at most 32 weights (one CTA) is ranked by one warp; otherwise its
+//            weights are histogrammed again on the next bits, until one value (or one weight,
+//            whose bits follow from the bin's sums) remains.
 // The fp32 part of the mass above the range is off by at most 2^-21 of it.  When the decision
 // that fixed T is closer than that to p, the pass repeats with that mass summed in fp64, so the
 // result is the one fp64 sums give.

@@ -310,6 +310,47 @@ def test_bisect_band_criterion():
         assert check_bisect_band(O.top_p_bisect, rows, p, 1e-6)
 
 
+def _bisect_replay_from_threshold(w, p, eps):
+    """The pages' bisection (lo = 0, hi = max W, fp32 midpoints) with its test mass(W >= mid) >= p
+    replaced by mid <= T, T = the largest weight v with mass(W >= v) >= p (0 if none), T read off
+    the descending cumulative sum.  The standalone pruner computes m this way."""
+    w = np.asarray(w, dtype=F32)
+    order = np.argsort(-w.astype(F64), kind="stable")
+    cs = np.cumsum(w[order].astype(F64))
+    hit = np.nonzero(cs >= F64(p))[0]
+    T = w[order[hit[0]]] if hit.size else F32(0.0)
+    top = F32(w.max())
+    if p >= 1.0:
+        return F32(0.0)
+    if top <= T:
+        return top
+    lo, hi = F32(0.0), top
+    for _ in range(64):
+        if F64(hi) - F64(lo) <= eps:
+            break
+        mid = F32(lo + (hi - lo) / F32(2.0))
+        if not (lo < mid < hi):
+            break
+        if mid <= T:
+            lo = mid
+        else:
+            hi = mid
+    return lo
+
+
+def test_bisect_equals_threshold_replay():
+    """mass(W >= t) only changes at weight values, so each test of the bisection is mid <= T; the
+    replay gives the oracle's bisection result exactly (normalised rows with ties, an
+    unnormalised row, uniform and one-hot rows)."""
+    rows, _ = synth.config5_rows(24, 3000, seed=9, tie_frac=0.3)
+    extra = [np.full(100, 0.01, dtype=F32), np.eye(1, 64, 5, dtype=F32)[0],
+             (np.arange(1, 201, dtype=F32) / 40.0).astype(F32)]
+    for w in list(rows) + extra:
+        for p in (0.5, 0.8, 0.9, 0.999):
+            m, _ = O.top_p_bisect(w, p, 1e-6)
+            assert _bisect_replay_from_threshold(w, p, 1e-6) == m
+
+
 def test_bisect_one_hot_and_keep_all():
     w = np.zeros(64, dtype=F32)
     w[11] = 1.0
