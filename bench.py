@@ -42,6 +42,7 @@ UNIT = "layer-steps/s"
 LAYERS = 32  # default; --layers overrides (profiling runs use 1)
 KERNELS_PER_LAYER_STEP = 1  # twl_decode_step is one fused kernel
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200's nominal HBM3e bandwidth, beside the measured peak
 
 
 WORKLOADS = {
@@ -401,7 +402,8 @@ def run_ours(args, world, rank, local):
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "twl_decode_step (whole layer-step)",
                      "alg_bytes_per_layer_step": alg_bytes, "alg_bytes_parts": parts,
-                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "frac_of_nominal_8tbs": None},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": args.steps * LAYERS * KERNELS_PER_LAYER_STEP,
@@ -575,7 +577,8 @@ def run_append(args, world, rank, local):
                      "frac": achieved / peak, "traffic": None,
                      "kernel": "twl_append_token (k_append_token)",
                      "alg_bytes_per_call": nbytes / (args.steps * LAYERS),
-                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "frac_of_nominal_8tbs": None},
         "gpu_launches": args.steps * LAYERS, "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -717,7 +720,8 @@ def run_quest(args, world, rank, local):
                      "unit": "GB/s", "frac": nbytes / per_layer_us / 1e3 / peak,
                      "traffic": None, "kernel": "twl_select_pages + twl_sparse_decode",
                      "alg_bytes_per_layer_step": nbytes,
-                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "frac_of_nominal_8tbs": None},
         "attended_tokens_per_layer": toks_total, "clocks": clk,
         "gpu_launches": 4 * args.steps * LAYERS,
     }
@@ -798,7 +802,8 @@ def run_double_p(args, world, rank, local, p_cluster=0.95):
                      "traffic": None, "kernel": "twl_select_clusters_top_p + twl_estimate + "
                      "twl_prune_top_p + twl_group_union + twl_sparse_decode",
                      "alg_bytes_per_layer_step": nbytes,
-                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "frac_of_nominal_8tbs": None},
         "kept_pages_per_head_mean": float(cntn.mean()), "pages_per_head": n_pages_total // b_,
         "union_tokens_per_group": ucnt.reshape(-1).tolist(), "clocks": clk,
         "gpu_launches": 9 * args.steps * LAYERS,
@@ -951,7 +956,8 @@ def run_prune_rows(args, world, rank, local):
                      "traffic": measured_traffic("prune_rows", f"dram_bytes_per_launch_n{ns[-1]}"),
                      "kernel": "k_prune_rows (twl_prune_top_p)",
                      "alg_bytes_per_launch": head["alg_bytes"],
-                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "frac_of_nominal_8tbs": None},
         "e2e": e2e, "gpu_launches": launches, "clocks": head["clocks"], "sweep": sweep,
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -1085,7 +1091,8 @@ def run_bits(args, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": v4["achieved_gbs"], "peak": peak, "unit": "GB/s",
                      "frac": v4["frac"], "traffic": None,
                      "kernel": "twl_estimate_nbit (3 launches)",
-                     "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "frac_of_nominal_8tbs": None},
         "variants": variants, "union_pages": union_pages, "clocks": clk,
         "gpu_launches": 3 * 3 * args.steps * LAYERS,
     }
@@ -1141,6 +1148,9 @@ def main():
         else:
             out = run_ours(args, world, rank, local)
         if rank == 0 and out is not None:
+            roof = out.get("roofline")
+            if roof and roof.get("unit") == "GB/s" and roof.get("achieved") is not None:
+                roof["frac_of_nominal_8tbs"] = roof["achieved"] / NOMINAL_HBM_GBS
             print(json.dumps(out), flush=True)
     finally:
         if world > 1:
