@@ -272,6 +272,43 @@ def test_prune_rows_full_size(n):
         check_prune_row(w_np[r], m[r], int(kc[r]), ki_s[j], 0.9, 1e-6, f"n{n} row {r}")
 
 
+@pytest.mark.parametrize("n", [4096, 32768])
+def test_prune_rows_nonfinite_and_extreme_parameters(n):
+    """Weights outside the method's domain and extreme (p, eps).  NaN weights are never kept and
+    carry no mass, negative weights carry none; a row holding +inf keeps exactly its infinite
+    entries; a tiny p keeps the largest weight (and its ties); a wide eps stops the bisection
+    early, so more is kept, but kept = {W >= m} and the mass condition still hold."""
+    rng = np.random.default_rng(n)
+    base = rng.dirichlet(np.ones(n)).astype(np.float32)
+    rows = np.stack([base.copy() for _ in range(4)])
+    rows[0, rng.choice(n, 7, replace=False)] = np.nan
+    rows[1, rng.choice(n, 9, replace=False)] = -rng.random(9).astype(np.float32)
+    rows[2, [3, 11]] = np.inf
+    rows[3, 5] = 0.5
+    w = torch.from_numpy(rows).cuda()
+    for p, eps in ((0.85, 1e-6), (0.01, 1e-6), (0.85, 0.1)):
+        m = torch.zeros(4, dtype=torch.float32, device="cuda")
+        kc = torch.zeros(4, dtype=torch.int32, device="cuda")
+        ki = torch.full((4, n), -1, dtype=torch.int32, device="cuda")
+        twl.twl_prune_top_p(w, None, 4, n, p, eps, m, kc, ki)
+        mn, kcn, kin = np_(m), np_(kc), np_(ki)
+        for r in range(4):
+            with np.errstate(invalid="ignore"):
+                keep = np.nonzero(rows[r] >= mn[r])[0]
+            assert kcn[r] == keep.size and np.array_equal(kin[r, : keep.size], keep), (p, eps, r)
+            if r == 2:
+                assert np.isinf(mn[r]) and list(keep) == [3, 11]
+                continue
+            finite = np.where(np.isfinite(rows[r]) & (rows[r] > 0), rows[r], 0).astype(np.float64)
+            assert finite[keep].sum() >= min(p, finite.sum()) - 1e-5, (p, eps, r)
+            if eps < 1e-3:
+                k_star, m_star, _ = O.top_p_sort(finite, p)
+                band = int(np.count_nonzero((finite >= float(m_star) - eps) & (finite <= m_star)))
+                assert keep.size <= k_star + band, (p, eps, r)
+        if p == 0.01:
+            assert kcn[3] == 1 and kin[3, 0] == 5      # the one weight of 0.5
+
+
 def test_prune_special_rows():
     n = 40
     rows = np.zeros((5, n), dtype=np.float32)
