@@ -103,6 +103,11 @@ __device__ __forceinline__ uint32_t ldc32(uint32_t addr) {
 __device__ __forceinline__ void stc32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
+__device__ __forceinline__ uint32_t atomc_add32(uint32_t addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+  return old;
+}
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
@@ -569,6 +574,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
 #pragma unroll 1
       for (int tries = 0; tries < 64 && !found; ++tries) {
         TWL_PRUNE_STAMP(3);
+        if (t == 0) sh.gcount = 0;  // published by the exact pass's barriers (cluster: its csync)
         // ---- exact pass over [klo, khi]
         int sb = span_shift((uint32_t)lo_key, (uint32_t)hi_key);
         if (sb > kMaxBinShift) {  // keep the upper part; a miss moves the range down
@@ -671,7 +677,6 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
             *sm = sb ? csum32(fc + 4u * (kNB + b), C) : 0ull;
             return bin_units(klo + ((uint32_t)b << sb), *c, *sm, e_lo);
           };
-          if (t == 0) sh.gcount = 0;  // published by the level's barriers
           level_cross((int)((khi >> sb) - (klo >> sb)) + 1, max(R, (uint64_t)1), mass, sh);
           const Cross F = sh.cr;
           if (F.bin >= 0) {
@@ -681,19 +686,21 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
             double a_gt = above + (double)F.above * unit, a_mass = (double)F.mass * unit;
             if (F.cnt == 1 || sb == 0) {
               Tbits = (pf0 << sb) | (uint32_t)F.sum;
-            } else if (C == 1 && F.cnt <= 32) {
-              // ---- few weights in the crossing bin: gather them from the lists and rank them
-              // in one warp (exact integer masses in units of the bin's exponent)
+            } else if (F.cnt <= 32) {
+              // ---- few weights in the crossing bin: gather them (from the lists, into the first
+              // CTA of the cluster) and rank them in one warp (exact integer masses in units of
+              // the bin's exponent)
               const int e_f = max((int)((pf0 << sb) >> 23), 1);
               const int sh_f = e_f - e_lo;
               const double unit_f = pow2d(e_f - 150);
               const uint64_t R1 = ((max(R, (uint64_t)1) - F.above) + ((1ull << sh_f) - 1ull)) >> sh_f;
+              const uint32_t a_gc = mapa(saddr(&sh.gcount), 0), a_ga = mapa(saddr(sh.gather), 0);
               if (use_list) {
                 for (int j = 0; j < nlist; ++j) {
                   const uint32_t u = lds32(a_list + 4u * T * j);
                   if ((u >> sb) == pf0) {
-                    const int g = atomicAdd(&sh.gcount, 1);
-                    if (g < 32) sh.gather[g] = u;
+                    const uint32_t g = atomc_add32(a_gc, 1u);
+                    if (g < 32u) stc32(a_ga + 4u * g, u);
                   }
                 }
               } else {
@@ -701,13 +708,14 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
                 for (int i = 0; i < kRE; ++i) {
                   const uint32_t u = __float_as_uint(x[i]);
                   if ((u >> sb) == pf0) {  // a finite prefix: NaN never matches
-                    const int g = atomicAdd(&sh.gcount, 1);
-                    if (g < 32) sh.gather[g] = u;
+                    const uint32_t g = atomc_add32(a_gc, 1u);
+                    if (g < 32u) stc32(a_ga + 4u * g, u);
                   }
                 }
               }
               __syncthreads();
-              if (warp == 0) {
+              if (C > 1) csync();
+              if (q == 0 && warp == 0) {
                 const int gc = min(sh.gcount, 32);
                 const uint32_t v = lane < gc ? sh.gather[lane] : 0u;
                 const bool ok = lane < gc;
@@ -730,9 +738,19 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
                 }
               }
               __syncthreads();
-              Tbits = sh.g_t;
-              a_gt += (double)sh.g_gt * unit_f;
-              a_mass = (double)sh.g_eq * unit_f;
+              if (C > 1) {
+                csync();
+                const uint32_t a0 = mapa(saddr(&sh.g_t), 0);
+                Tbits = ldc32(a0);
+                const uint64_t g_gt = ldc64(mapa(saddr(&sh.g_gt), 0));
+                const uint64_t g_eq = ldc64(mapa(saddr(&sh.g_eq), 0));
+                a_gt += (double)g_gt * unit_f;
+                a_mass = (double)g_eq * unit_f;
+              } else {
+                Tbits = sh.g_t;
+                a_gt += (double)sh.g_gt * unit_f;
+                a_mass = (double)sh.g_eq * unit_f;
+              }
             } else {
               // ---- refinement levels on the crossing bin's weights (one exponent: unit 2^(e-150))
               TWL_PRUNE_STAMP(5);
