@@ -731,7 +731,7 @@ def run_quest(args, world, rank, local):
 
 def run_double_p(args, world, rank, local, p_cluster=0.95):
     """The two-level top-p step (cluster-level top-p over page centroids, then the token-level
-    path on the kept pages; five library calls, survey row f4) on the workload.  Algorithmic
+    path on the kept pages; five library calls) on the workload.  Algorithmic
     bytes: centroids (256 B per page per kv-head) + page table, INT4 K of each group's union
     of kept pages, fp16 K/V of the union of kept tokens, q and o/lse."""
     from adaptive_top_sparse_b200.layer import DecodeLayer
@@ -834,7 +834,7 @@ def prune_rows_bytes(n, rows, kept_total, with_idx):
 
 
 def run_prune_rows(args, world, rank, local):
-    """twl_prune_top_p alone on the standalone-pruner workload (4096 rows x n, survey config 5),
+    """twl_prune_top_p alone on the standalone-pruner workload (4096 rows x n fp32 weights),
     against its read-once HBM bound."""
     from adaptive_top_sparse_b200 import twl
     dev = torch.device("cuda", local)
@@ -1004,7 +1004,7 @@ def run_prune_rows_reference(args, world, rank):
 
 def run_bits(args, world, rank, local):
     """The staged estimate (union, dequant-dot, softmax) on the 32K-context layer at 2, 4 and 8
-    bits (survey row f2): time per call, and the roofline over the codes + scale/zero of the
+    bits: time per call, and the roofline over the codes + scale/zero of the
     groups' union pages (16 rows x (16 bits + 4) bytes per page per kv-head)."""
     from adaptive_top_sparse_b200 import twl
     from adaptive_top_sparse_b200.layer import DecodeLayer

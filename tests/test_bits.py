@@ -1,4 +1,4 @@
-"""Estimator bit widths (survey row f2): the INT4 scheme at 2 and 8 bits, and the ablation's
+"""Estimator bit widths: the INT4 scheme at 2 and 8 bits, and the ablation's
 weight-mass check (the exact weights' mass over the set kept from the estimate, against p).
 
 CPU: the oracle's bit-width restatement is pinned to the INT4 path at 4 bits, to hand-worked

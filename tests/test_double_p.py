@@ -1,4 +1,4 @@
-"""Cluster-level top-p selection (survey row f4, the Double-P selector): page centroids,
+"""Cluster-level top-p selection (the Double-P selector): page centroids,
 size-weighted cluster weights, top-p over pages, then the token-level path on the kept pages.
 
 CPU pins: the centroid is the plain mean where fp32 sums are exact; a page whose rows are
