@@ -11,9 +11,11 @@
 // T is a mass-weighted order statistic, found over the row held in registers with shared-memory
 // atomics for a small share of the weights only (one shared atomic costs about as much issue
 // bandwidth as the rest of a weight's work):
-//   bracket  a count histogram of the fp32 bit patterns over [L, max W] (1024 log-spaced bins)
-//            holding every heavy weight (>= 4 x the mean) and one in two of the others; its
-//            estimated mass profile gives a key range that holds T with high probability.
+//   bracket  a count histogram of the fp32 bit patterns over [L, max W] (kNB log-spaced bins);
+//            its estimated mass profile (bin middle values) gives a key range that holds T.
+//            Heavy weights (>= 4 x the mean) are always counted; TWL_PRUNE_SAMPLE = k > 1 counts
+//            one in k of the others and widens the range by the sampling variance (fewer shared
+//            atomics, but the wider range costs more than it saves on the rows measured).
 //            L = (sum W - p) / (2 n): the weights below L sum to less than (sum - p) / 2, so T >= L.
 //   exact    one pass: the weights above the range add up to the mass above it (fp32 pairwise per
 //            thread, fp64 across threads); the weights inside it go to per-thread lists, then to
@@ -56,10 +58,23 @@ constexpr int kRounds = kRE / 4;            // float4 chunks per thread
 constexpr int kRMaxThreads = TWL_PRUNE_MAX_THREADS;
 constexpr int kRSlice = kRE * kRMaxThreads;  // weights per CTA, at most
 constexpr int kRMaxCluster = 8;
-constexpr int kNB = 1024;                   // bins per histogram
+#ifndef TWL_PRUNE_NB_BITS
+#define TWL_PRUNE_NB_BITS 10
+#endif
+#ifndef TWL_PRUNE_SAMPLE
+#define TWL_PRUNE_SAMPLE 1
+#endif
+constexpr int kNBBits = TWL_PRUNE_NB_BITS;
+constexpr int kNB = 1 << kNBBits;           // bins per histogram
+static_assert(kNB >= kRMaxThreads, "the bracket scan gives every thread at least one bin");
 constexpr float kHeavy = 4.f;               // weights >= kHeavy * sum / n are always counted
-constexpr int kSample = 2;                  // one in kSample of the other weights is counted
-constexpr int kMaxBinShift = 17;            // exact bins: count * 2^shift < 2^32 per CTA
+constexpr int kSample = TWL_PRUNE_SAMPLE;   // one in kSample of the other weights is counted
+static_assert(kSample == 1 || kSample == 2 || kSample == 4, "a divisor of the 4-weight chunk");
+// exact bins: count * 2^shift < 2^32 per CTA (count <= 2^15), and a range of at most
+// kNB * 2^shift <= 2^27 bit patterns (16 binades) keeps a bin's integer mass below 2^59
+constexpr int kMaxBinShift = kNBBits <= 10 ? 17 : 27 - kNBBits;
+static_assert(kNBBits + kMaxBinShift <= 27, "exact masses fit in 64 bits");
+static_assert(2 * kNBBits >= kMaxBinShift, "two refinement levels resolve an exact bin");
 constexpr uint32_t kNaNBits = 0xFFFFFFFFu;  // weights past the row's length
 
 // Optional phase clock (a probe build defines TWL_PRUNE_STAMP(slot) to record it); off by default.
@@ -366,7 +381,10 @@ __device__ __forceinline__ void prefix_level(const float (&x)[kRE], bool use_lis
 }
 
 // 2 kRE registers per thread: 32768 / kRE threads per SM, in CTAs of up to kRMaxThreads
-__global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_prune_rows(PruneRowsArgs a) {
+#ifndef TWL_PRUNE_MIN_BLOCKS
+#define TWL_PRUNE_MIN_BLOCKS (32768 / kRE / kRMaxThreads)
+#endif
+__global__ void __launch_bounds__(kRMaxThreads, TWL_PRUNE_MIN_BLOCKS) k_prune_rows(PruneRowsArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ RowSh sh;
   const int T = blockDim.x, t = threadIdx.x, lane = t & 31, warp = t >> 5, nw = T >> 5;
@@ -459,7 +477,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
       const uint32_t kt = __float_as_uint(top);
       const double P = (double)a.p;
       TWL_PRUNE_STAMP(2);
-      // ---- bracket: sampled count histogram over [L, top]
+      // ---- bracket: count histogram over [L, top] (non-heavy weights: one in kSample)
       const float tot_lo = total * (1.f - 0x1p-16f);
       const float L = tot_lo > a.p ? (tot_lo - a.p) / (2.f * (float)len) : 0.f;
       const uint32_t kL = __float_as_uint(L);
@@ -538,7 +556,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
         const float pf = a.p;
         const float delta = 3.f * sqrtf(tv) + te * ldexpf(1.f, s - 24) + 1e-7f * pf;
         float run = (warp ? wpf : 0.f) + (xs - le);
-        bool got_hi = false, got_lo = false;
+        int b_hi = -1, b_lo = -1;  // this thread's first bin reaching p - delta, p + delta
         for (int e = 0; e < per; ++e) {
           const int b = b0 - e;
           const int pk = (int)win + b;
@@ -548,14 +566,16 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
             const float v = __uint_as_float(((uint32_t)pk << s) + ((1u << s) >> 1));
             run += (ch + (float)kSample * cl) * v;
           }
-          if (!got_hi && run >= pf - delta) {
-            atomicMax(&sh.bhi, b);
-            got_hi = true;
-          }
-          if (!got_lo && run >= pf + delta) {
-            atomicMax(&sh.blo, b);
-            got_lo = true;
-          }
+          if (b_hi < 0 && run >= pf - delta) b_hi = b;
+          if (b_lo < 0 && run >= pf + delta) b_lo = b;
+        }
+        // the highest such bin over the block: one shared atomic per warp (every thread past the
+        // crossing has one, so a per-thread atomic would serialise on one word)
+        b_hi = __reduce_max_sync(0xffffffffu, b_hi);
+        b_lo = __reduce_max_sync(0xffffffffu, b_lo);
+        if (lane == 0) {
+          if (b_hi >= 0) atomicMax(&sh.bhi, b_hi);
+          if (b_lo >= 0) atomicMax(&sh.blo, b_lo);
         }
       }
       __syncthreads();
@@ -667,7 +687,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
           redo = true;  // too close to call with the fp32 part
         } else {
           // masses of the exact bins in units of the range's lowest exponent (the range spans at
-          // most 1024 x 2^17 patterns = 16 binades, so a bin's mass stays below 2^59)
+          // most kNB x 2^kMaxBinShift <= 2^27 patterns = 16 binades: below 2^59 per bin)
           const int e_lo = max((int)(klo >> 23), 1);
           const double unit = pow2d(e_lo - 150);
           const double need = (P - above) / unit;
@@ -761,7 +781,7 @@ __global__ void __launch_bounds__(kRMaxThreads, 32768 / kRE / kRMaxThreads) k_pr
               const int sh_f = e_f - e_lo;  // fine units per bin unit: 2^sh_f
               const double unit_f = pow2d(e_f - 150);
               const uint64_t R1 = ((max(R, (uint64_t)1) - F.above) + ((1ull << sh_f) - 1ull)) >> sh_f;
-              const int s2 = max(0, sb - 10);
+              const int s2 = max(0, sb - kNBBits);
               prefix_level(x, use_list, a_list, nlist, pf0, sb, s2, saddr(rC), max(R1, (uint64_t)1), C,
                            sh);
               const Cross S = sh.cr;
