@@ -2,6 +2,7 @@
 // Each entry point validates everything it can on the host before launching anything.
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 #include <stdlib.h>
 
@@ -12,16 +13,16 @@
 namespace twl {
 
 int num_sms() {
-  static int cache[128] = {0};
+  static std::atomic<int> cache[128];  // zero-initialised: not yet queried
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 namespace {

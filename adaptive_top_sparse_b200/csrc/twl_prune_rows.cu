@@ -38,6 +38,8 @@
 // grid is persistent: each CTA (cluster) walks rows r, r + G, ..., and while it works on one row
 // its threads' cp.async copies of the next row land in shared memory (every thread copies and
 // later reads back only its own chunks, so the hand-off needs no barrier).
+#include <mutex>
+
 #include "twl_common.cuh"
 #include "twl_kernels.h"
 
@@ -967,10 +969,16 @@ static RowsPlan plan_rows(int rows, int stride) {
   pl.cluster = cluster;
   pl.list_cap = max(4, rows_list_cap(threads, cluster));
   pl.smem = rows_smem(threads, cluster, pl.list_cap);
-  // persistent grid: as many CTAs (clusters) as are resident at once, at most one per row
-  static int cache_key[32], cache_val[32];
+  // persistent grid: as many CTAs (clusters) as are resident at once, at most one per row;
+  // the residency is cached per (device, threads, cluster), under a lock for concurrent callers
+  static std::mutex mu;
+  static long long cache_key[32];
+  static int cache_val[32];
   static int cache_n = 0;
-  const int key = threads * 16 + cluster;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const long long key = ((long long)dev << 32) | (long long)(threads * 16 + cluster);
+  std::lock_guard<std::mutex> lock(mu);
   int per = -1;
   for (int i = 0; i < cache_n; ++i)
     if (cache_key[i] == key) per = cache_val[i];
