@@ -12,6 +12,9 @@ What pins what:
   scores      unit queries give the bound rows themselves; upper-bound property against every
               token of the page (fp64); equality for a page of identical tokens.
   top-k       brute-force full sort.
+  order key   every non-NaN fp16 bit pattern: keys rise strictly with the value, -0 before +0.
+  softmax     closed forms (uniform; logits 0 and ln 3 give 1/4 and 3/4, also at +1000) and the
+              definition term by term with math.fsum.
   estimate    K on the 16-level grid makes the dequantised K exact, so the estimate must equal
               torch's softmax of q.K/sqrt(D) computed from the raw fp16 K.
   top-p       hand examples (tests/golden/top_p_examples.json, [Notes] "Key designs");
@@ -528,3 +531,75 @@ def test_pins_catch_planted_mistakes():
 
     assert check_bisect_band(O.top_p_bisect, rows, 0.9, 1e-6)
     assert not check_bisect_band(bisect_returns_hi, rows, 0.9, 1e-6)
+
+
+
+def check_order_key(key_fn):
+    """Every non-NaN fp16 bit pattern, ordered by value with -0 before +0: the keys must rise
+    strictly along that order (so min/max by key are min/max by value, and -0 < +0)."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = bits.view(F16)
+    ok = ~np.isnan(vals)
+    bits, vals = bits[ok], vals[ok]
+    neg_zero = bits == 0x8000
+    order = np.lexsort((~neg_zero, vals.astype(F64)))  # by value, then -0 first
+    keys = np.asarray(key_fn(vals[order])).astype(np.int64)
+    return bool(np.all(np.diff(keys) > 0))
+
+
+def check_softmax(fn):
+    """Closed forms: uniform logits give 1/n; logits (0, ln 3) give (1/4, 3/4), also shifted by
+    1000 (no overflow); a random row against the definition term by term (math.fsum)."""
+    try:
+        with np.errstate(all="ignore"):
+            for n in (1, 2, 7, 1000):
+                if not np.allclose(fn(np.zeros(n)), np.full(n, 1.0 / n), rtol=1e-15, atol=0):
+                    return False
+            for c in (0.0, 1000.0):
+                if not np.allclose(fn([c, c + math.log(3.0)]), [0.25, 0.75], rtol=1e-12, atol=0):
+                    return False
+            x = np.random.default_rng(3).normal(0.0, 4.0, 257)
+            w = np.asarray(fn(x), dtype=F64)
+    except (FloatingPointError, OverflowError, ValueError):
+        return False
+    e = [math.exp(v - 10.0) for v in x]
+    ref = np.array(e) / math.fsum(e)
+    return bool(np.allclose(w, ref, rtol=1e-13, atol=0)) and abs(math.fsum(w) - 1.0) < 1e-15
+
+
+def test_f16_order_key_orders_every_fp16_value():
+    assert check_order_key(O.f16_order_key)
+    z = O.f16_order_key(np.array([-0.0, 0.0], F16))
+    assert z[0] < z[1]
+
+    def key_magnitude_only(x16):           # drops the sign
+        return np.ascontiguousarray(x16, dtype=F16).view(np.uint16).astype(np.int32) & 0x7FFF
+
+    def key_no_minus_one(x16):             # -0 and +0 collide
+        b = np.ascontiguousarray(x16, dtype=F16).view(np.uint16).astype(np.int32)
+        return np.where(b & 0x8000, -(b & 0x7FFF), b)
+
+    assert not check_order_key(key_magnitude_only)
+    assert not check_order_key(key_no_minus_one)
+
+
+def test_softmax64_closed_forms():
+    assert check_softmax(O.softmax64)
+
+    def softmax_unshifted(x):               # no max subtraction: overflows at logits near 1000
+        e = np.exp(np.asarray(x, dtype=F64))
+        return e / e.sum()
+
+    def softmax_fp32(x):                    # single precision
+        x = np.asarray(x, dtype=F32)
+        e = np.exp(x - x.max())
+        return e / e.sum()
+
+    def softmax_dropped_term(x):            # the normaliser misses the last term
+        x = np.asarray(x, dtype=F64)
+        e = np.exp(x - x.max())
+        return e / (e.sum() - e[-1] if e.size > 1 else e.sum())
+
+    assert not check_softmax(softmax_unshifted)
+    assert not check_softmax(softmax_fp32)
+    assert not check_softmax(softmax_dropped_term)
