@@ -11,7 +11,8 @@ What pins what:
               designs", 4-bit K cache; [Summary] 4.3).
   scores      unit queries give the bound rows themselves; upper-bound property against every
               token of the page (fp64); equality for a page of identical tokens.
-  top-k       brute-force full sort.
+  top-k       brute-force full sort; whole page selection (GQA head map, budget rule, ties) by
+              brute force in Python integers on integer-valued q and K.
   order key   every non-NaN fp16 bit pattern: keys rise strictly with the value, -0 before +0.
   softmax     closed forms (uniform; logits 0 and ln 3 give 1/4 and 3/4, also at +1000) and the
               definition term by term with math.fsum.
@@ -207,6 +208,90 @@ def test_budget_rule():
     assert O.budget_for(2048, 0, 4) == 512
     assert O.budget_for(3, 0, 4) == 1 and O.budget_for(5, 0, 4) == 2
     assert O.budget_for(10, 64, 4) == 10 and O.budget_for(100, 64, 4) == 64
+
+
+def _integer_gqa_case(seed=21):
+    """Integer-valued fp16 q and K (|values| <= 3), so every product and every sum of a page
+    score is exact in fp32 and in Python integers; ragged lengths, a permuted page table, many
+    tied scores."""
+    rng = np.random.default_rng(seed)
+    hq, hkv, d = 8, 2, 128
+    lens = np.array([1, 37, 16 * 9, 16 * 11 + 5])
+    pages = [O.num_pages(n) for n in lens]
+    p_phys = sum(pages) + 3
+    perm = rng.permutation(p_phys)
+    pt = np.full((len(lens), max(pages)), -1, dtype=np.int64)
+    o = 0
+    for b, pb in enumerate(pages):
+        pt[b, :pb] = perm[o:o + pb]
+        o += pb
+    k = rng.integers(-3, 4, size=(p_phys, hkv, 16, d)).astype(F16)
+    q = rng.integers(-3, 4, size=(len(lens), hq, d)).astype(F16)
+    return q, k, pt, lens, hq, hkv
+
+
+def check_select_pages(select_fn, budget_pages=0):
+    """Brute force in Python integers: q-head h reads kv-head h // (Hq / Hkv); score of page j =
+    sum over channels of max(q_c mn_jc, q_c mx_jc) over the page's valid tokens; keep
+    ceil(P / 4) pages (or the fixed budget), highest score first, ties to the lower page."""
+    q, k, pt, lens, hq, hkv = _integer_gqa_case()
+    bounds = O.page_bounds(k, pt, lens)
+    got = select_fn(q, bounds, pt, lens, hq, hkv, budget_pages, 4)
+    for b, n in enumerate(lens):
+        n = int(n)
+        pb = -(-n // 16)
+        kb = min(pb, budget_pages) if budget_pages > 0 else -(-pb // 4)
+        for h in range(hq):
+            kvh = h // (hq // hkv)
+            qi = [int(v) for v in q[b, h]]
+            sc = []
+            for j in range(pb):
+                rows = k[pt[b, j], kvh, : min(16, n - 16 * j)].astype(np.int64)
+                mn, mx = rows.min(axis=0), rows.max(axis=0)
+                sc.append(sum(max(qc * int(a), qc * int(c)) for qc, a, c in zip(qi, mn, mx)))
+            want = sorted(sorted(range(pb), key=lambda j: (-sc[j], j))[:kb])
+            g_sc, g_sel = got[(b, h)]
+            if list(np.asarray(g_sc, dtype=F64)) != [float(v) for v in sc]:
+                return False
+            if list(g_sel) != want:
+                return False
+    return True
+
+
+def test_select_pages_bruteforce_integer_gqa():
+    assert check_select_pages(O.select_pages)
+    assert check_select_pages(O.select_pages, budget_pages=3)
+
+    def kv_head_modulo(q, bounds, pt, lens, hq, hkv, budget_pages=0, budget_div=4):
+        out = {}
+        for b in range(len(lens)):
+            pb = O.num_pages(lens[b])
+            phys = pt[b, :pb]
+            kb = O.budget_for(pb, budget_pages, budget_div)
+            for h in range(hq):
+                sc = O.page_scores(q[b, h], bounds[phys, h % hkv, 0], bounds[phys, h % hkv, 1])
+                out[(b, h)] = (sc, O.select_top_k(sc, kb))
+        return out
+
+    def budget_floor(q, bounds, pt, lens, hq, hkv, budget_pages=0, budget_div=4):
+        out = O.select_pages(q, bounds, pt, lens, hq, hkv, budget_pages, budget_div)
+        res = {}
+        for (b, h), (sc, _) in out.items():
+            kb = max(1, len(sc) // budget_div) if budget_pages == 0 else min(len(sc), budget_pages)
+            res[(b, h)] = (sc, O.select_top_k(sc, kb))
+        return res
+
+    def ties_to_higher(q, bounds, pt, lens, hq, hkv, budget_pages=0, budget_div=4):
+        out = O.select_pages(q, bounds, pt, lens, hq, hkv, budget_pages, budget_div)
+        res = {}
+        for (b, h), (sc, sel) in out.items():
+            order = sorted(range(len(sc)), key=lambda j: (-float(sc[j]), -j))
+            res[(b, h)] = (sc, np.array(sorted(order[:len(sel)])))
+        return res
+
+    assert not check_select_pages(kv_head_modulo)
+    assert not check_select_pages(budget_floor)
+    assert not check_select_pages(ties_to_higher)
 
 
 # ------------------------------------------------------------------------------------- estimate
