@@ -21,6 +21,8 @@ What pins what:
   top-p       hand examples (tests/golden/top_p_examples.json, [Notes] "Key designs");
               brute-force subset search for n <= 14; mass(W >= m*) >= p > mass(W > m*);
               bisection result inside the epsilon band ([Notes] "Key designs", efficient top-p).
+  gather      rows that carry their own (token, head, sequence) address, behind a permuted
+              page table.
   attention   all tokens kept -> torch scaled_dot_product_attention in fp64; one token kept ->
               o = v_i, lse = q.k_i/sqrt(D); the error bound (1-p)*||V||_F ([Notes] "Key
               designs", oracle top-p guarantee).
@@ -517,6 +519,46 @@ def test_decode_step_small_consistency():
         assert sorted(want) == grp["union"].tolist()
         # p = 1 style check: all kept tokens of the group are inside the sequence
         assert grp["union"].max() < wl.seq_lens[b]
+
+
+def check_gather(gather_fn):
+    """Paged rows that carry their own address: the row of logical token t of sequence b in
+    kv-head h holds (t, h, b) in its first three channels, written while walking the sequences'
+    pages in logical order (a permuted page table puts them anywhere).  A gather must return
+    exactly the rows it was asked for."""
+    _, _, pt, lens, _, hkv = _integer_gqa_case(seed=5)
+    p_phys = int(pt.max()) + 4
+    arr = np.full((p_phys, hkv, 16, 8), -1.0, dtype=F16)
+    for b, n in enumerate(lens):
+        for t in range(int(n)):
+            for h in range(hkv):
+                arr[pt[b, t // 16], h, t % 16, :3] = (t, h, b)
+    rng = np.random.default_rng(6)
+    for b, n in enumerate(lens):
+        for h in range(hkv):
+            toks = np.sort(rng.choice(int(n), size=min(int(n), 23), replace=False))
+            rows = np.asarray(gather_fn(arr, pt, b, h, toks)).astype(F64)
+            if rows.shape[0] != toks.size:
+                return False
+            if not (np.array_equal(rows[:, 0], toks) and np.all(rows[:, 1] == h)
+                    and np.all(rows[:, 2] == b)):
+                return False
+    return True
+
+
+def test_gather_tokens_returns_the_addressed_rows():
+    assert check_gather(O.gather_tokens)
+
+    def gather_no_page_table(arr, pt, b, kvh, toks):     # treats logical pages as physical
+        toks = np.asarray(toks, dtype=np.int64)
+        return arr[toks // 16, kvh, toks % 16]
+
+    def gather_wrong_row(arr, pt, b, kvh, toks):         # row index from the page, not the token
+        toks = np.asarray(toks, dtype=np.int64)
+        return arr[pt[b, toks // 16], kvh, (toks // 16) % 16]
+
+    assert not check_gather(gather_no_page_table)
+    assert not check_gather(gather_wrong_row)
 
 
 def test_dense_limit_equals_full_attention():
