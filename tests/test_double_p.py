@@ -3,7 +3,8 @@ size-weighted cluster weights, top-p over pages, then the token-level path on th
 
 CPU pins: the centroid is the plain mean where fp32 sums are exact; a page whose rows are
 identical has a cluster weight equal to its exact share of the attention mass (the size
-weighting is exact there); p = 1 keeps every page; the entry points reject bad arguments.
+weighting is exact there); p = 1 keeps every page; each q-head keeps its own group's dominant
+page behind a permuted page table; the entry points reject bad arguments.
 GPU: centroids bit-exact, cluster weights and kept pages against the oracle's criteria, and the
 whole two-level step against the oracle over the device's sets.
 """
@@ -72,6 +73,36 @@ def test_select_clusters_p_one_keeps_every_page():
     sel = O.select_clusters(wl.q, cen, wl.page_table, wl.seq_lens, 4, 1, 1.0)
     for h in range(4):
         assert np.array_equal(sel[(0, h)][1], np.arange(O.num_pages(300)))
+
+
+def test_select_clusters_follows_each_groups_dominant_page():
+    """Four pages behind a permuted page table; kv-head 0 has one page aligned with the query
+    (logical page 1), kv-head 1 another (logical page 2), every other row is zero.  That page's
+    cluster weight is about 287 / 290, so p = 0.9 keeps it alone, and each q-head keeps the page
+    of its own group (q-head h reads kv-head h // 2)."""
+    pt = np.array([[2, 0, 3, 1]], np.int32)
+    k = np.zeros((4, 2, 16, D), np.float16)
+    k[pt[0, 1], 0, :, 0] = 8.0
+    k[pt[0, 2], 1, :, 0] = 8.0
+    q = np.zeros((1, 4, D), np.float16)
+    q[0, :, 0] = 8.0
+    lens = np.array([64])
+    cen = O.page_centroids(k, pt, lens)
+
+    def kept(select_fn):
+        sel = select_fn(q, cen, pt, lens, 4, 2, 0.9)
+        return [sel[(0, h)][1].tolist() for h in range(4)]
+
+    assert kept(O.select_clusters) == [[1], [1], [2], [2]]
+
+    def head_modulo(q, cen, pt, lens, hq, hkv, p_cluster):    # q-head h reads kv-head h % hkv
+        out = {}
+        for h in range(hq):
+            w = O.cluster_weights(q[0, h], cen, pt, 0, h % hkv, int(lens[0]))
+            out[(0, h)] = (w, np.sort(O.top_p_sort(w, p_cluster)[2]))
+        return out
+
+    assert kept(head_modulo) != [[1], [1], [2], [2]]
 
 
 def test_cluster_calls_reject_bad_arguments():
