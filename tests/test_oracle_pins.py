@@ -561,6 +561,31 @@ def test_gather_tokens_returns_the_addressed_rows():
     assert not check_gather(gather_wrong_row)
 
 
+def check_candidates(cand_fn):
+    """The candidates of a page set are the tokens whose page is selected and whose id is below
+    the sequence length, ascending; checked against a scan of every token id."""
+    rng = np.random.default_rng(9)
+    for n in (1, 15, 16, 17, 100, 16 * 9):
+        pb = -(-n // 16)
+        for _ in range(6):
+            sel = np.sort(rng.choice(pb, size=int(rng.integers(0, pb + 1)), replace=False))
+            want = [t for t in range(16 * pb) if t < n and (t // 16) in set(sel.tolist())]
+            got = np.asarray(cand_fn(sel, n)).tolist()
+            if got != want:
+                return False
+    return True
+
+
+def test_candidates_by_scan():
+    assert check_candidates(O.candidates)
+
+    def cand_full_pages(sel, n):             # keeps the unused rows of a partial last page
+        return np.concatenate([np.arange(16 * j, 16 * j + 16) for j in sorted(sel)]) \
+            if len(sel) else np.zeros(0, np.int64)
+
+    assert not check_candidates(cand_full_pages)
+
+
 def test_dense_limit_equals_full_attention():
     # budget = all pages and p = 1: the pipeline reduces to dense attention
     wl = synth.config2(seed=2, n=300, batch=1)
