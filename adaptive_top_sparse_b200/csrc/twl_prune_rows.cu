@@ -486,7 +486,17 @@ __global__ void __launch_bounds__(kRMaxThreads, TWL_PRUNE_MIN_BLOCKS) k_prune_ro
       const uint32_t kH = __float_as_uint(kHeavy * (total / (float)len));
       const int s = span_shift(kL, kt);
       const uint32_t win = (kt >> s) - (uint32_t)(kNB - 1);  // bin b <-> key prefix win + b
-      {
+      if constexpr (kSample == 1) {
+        // every weight: one add, to its bin when it lies in [L, top], else to this lane's dummy
+        // word (no branch)
+        const uint32_t aH = saddr(rA);
+#pragma unroll
+        for (int i = 0; i < kRE; ++i) {
+          const uint32_t u = __float_as_uint(x[i]);
+          const bool in = u - kL <= kt - kL;
+          red_add_u(in ? aH + 4u * ((u >> s) - win) : a_dummy, 1u);
+        }
+      } else {
         // heavy weights: all, behind one warp vote per chunk (they are rare); sampled ones: an
         // add that every thread makes, to its own dummy word when the weight is not counted
         const uint32_t aH = saddr(rA);
@@ -529,7 +539,7 @@ __global__ void __launch_bounds__(kRMaxThreads, TWL_PRUNE_MIN_BLOCKS) k_prune_ro
           const int b = b0 - e;
           const int pk = (int)win + b;
           const float ch = (float)csum32(saddr(rA + b), C);
-          const float cl = (float)csum32(saddr(rA + kNB + b), C);
+          const float cl = kSample > 1 ? (float)csum32(saddr(rA + kNB + b), C) : 0.f;
           if (pk >= 0 && ch + cl > 0.f) {
             const float v = __uint_as_float(((uint32_t)pk << s) + ((1u << s) >> 1));
             le += (ch + (float)kSample * cl) * v;
@@ -563,7 +573,7 @@ __global__ void __launch_bounds__(kRMaxThreads, TWL_PRUNE_MIN_BLOCKS) k_prune_ro
           const int b = b0 - e;
           const int pk = (int)win + b;
           const float ch = (float)csum32(saddr(rA + b), C);
-          const float cl = (float)csum32(saddr(rA + kNB + b), C);
+          const float cl = kSample > 1 ? (float)csum32(saddr(rA + kNB + b), C) : 0.f;
           if (pk >= 0 && ch + cl > 0.f) {
             const float v = __uint_as_float(((uint32_t)pk << s) + ((1u << s) >> 1));
             run += (ch + (float)kSample * cl) * v;
