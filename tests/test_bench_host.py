@@ -1,4 +1,5 @@
-"""Host logic of bench.py: the roofline's algorithmic bytes, counted by hand on a tiny case."""
+"""Host logic of bench.py: the roofline's algorithmic bytes counted by hand on tiny cases, the
+profile-traffic match, the clock summary of nvidia-smi rows, and the HBM peak's source."""
 import os
 import sys
 
@@ -40,3 +41,27 @@ def test_prune_rows_bytes_by_hand():
     # kept index when the indices are written
     assert bench.prune_rows_bytes(8, 3, 5, False) == 3 * (32 + 8)
     assert bench.prune_rows_bytes(8, 3, 5, True) == 3 * (32 + 8) + 20
+
+
+def test_clock_summary_from_nvidia_smi_rows():
+    rows = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1905, 1965, 990.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1950, 1965, 980.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, [N/A], 1965, 10.0, 0x0, Not Active, Not Active, Not Active, Not Active",  # skipped
+        "garbage",
+    ]
+    out = bench.ClockSampler.summarise(rows)
+    assert out == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                   "samples": 3}
+    hot = rows[:1] + ["0, 1200, 1965, 800, 0x8, Active, Not Active, Active, Not Active"]
+    assert bench.ClockSampler.summarise(hot)["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert bench.ClockSampler.summarise([])["sm_mhz"] is None
+
+
+def test_hbm_peak_measured_or_fallback(tmp_path, monkeypatch):
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6554.9, "bf16_tflops": 1500}')
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.hbm_peak() == (6554.9, "measured")
+    (tmp_path / "MEASURED_PEAKS.json").unlink()
+    assert bench.hbm_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
