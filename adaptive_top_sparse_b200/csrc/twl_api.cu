@@ -81,8 +81,9 @@ twl_status check_heads(int hq, int hkv) {
 twl_status check_budget(int budget_pages, int budget_div, int max_budget, int max_pages) {
   if (budget_pages < 0 || max_budget < 1) return TWL_ERR_INVALID_ARG;
   if (budget_pages == 0 && budget_div < 1) return TWL_ERR_INVALID_ARG;
-  const int bound = budget_pages > 0 ? (budget_pages < max_pages ? budget_pages : max_pages)
-                                     : (max_pages + budget_div - 1) / budget_div;
+  const long long bound = budget_pages > 0
+                              ? (budget_pages < max_pages ? budget_pages : max_pages)
+                              : ((long long)max_pages + budget_div - 1) / budget_div;
   if (max_budget < bound || max_budget > max_pages) return TWL_ERR_INVALID_ARG;
   return TWL_OK;
 }
@@ -327,6 +328,7 @@ twl_status twl_select_clusters_top_p(const void* q, int32_t num_q_heads, const t
   if (cluster_weights && !aligned(cluster_weights, 4)) return TWL_ERR_INVALID_ARG;
   if (!(p_cluster > 0.f && p_cluster <= 1.f) || !(eps > 0.f) || isinf(eps))
     return TWL_ERR_INVALID_ARG;
+  if ((long long)k.batch * num_q_heads > 0x7FFFFFFFll) return TWL_ERR_UNSUPPORTED;  // rows
   Carve c{static_cast<char*>(ws)};
   ClusterWs w = carve_clusters(c, k.batch, num_q_heads, k.max_pages);
   if ((st = check_ws(ws, ws_bytes, c.off)) != TWL_OK) return st;
@@ -475,7 +477,7 @@ twl_status twl_sparse_decode(const void* q, int32_t num_q_heads, const twl_paged
   if (!q || !tok || !tok_count || !o || !lse || tok_stride < 1 || !aligned(q, 16) ||
       !aligned(o, 16) || !(sm_scale > 0.f) || isinf(sm_scale))
     return TWL_ERR_INVALID_ARG;
-  if (k.batch * k.hkv > 4096) return TWL_ERR_UNSUPPORTED;
+  if ((long long)k.batch * k.hkv > 4096) return TWL_ERR_UNSUPPORTED;
   Carve c{static_cast<char*>(ws)};
   void* partials = c.take<char>(attend_partial_bytes(k.batch, num_q_heads, k.hkv, tok_stride));
   if ((st = check_ws(ws, ws_bytes, c.off)) != TWL_OK) return st;
