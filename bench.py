@@ -146,6 +146,20 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def host_info(cpuinfo="/proc/cpuinfo"):
+    """The host the CPU baseline ran on: logical CPUs and the CPU model name."""
+    model = None
+    try:
+        with open(cpuinfo) as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "model": model}
+
+
 # ---------------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -1158,6 +1172,8 @@ def main():
             roof = out.get("roofline")
             if roof and roof.get("unit") == "GB/s" and roof.get("achieved") is not None:
                 roof["frac_of_nominal_8tbs"] = roof["achieved"] / NOMINAL_HBM_GBS
+            if isinstance(out.get("cpu_baseline"), dict):
+                out["cpu_baseline"]["host"] = host_info()
             print(json.dumps(out), flush=True)
     finally:
         if world > 1:

@@ -65,3 +65,11 @@ def test_hbm_peak_measured_or_fallback(tmp_path, monkeypatch):
     assert bench.hbm_peak() == (6554.9, "measured")
     (tmp_path / "MEASURED_PEAKS.json").unlink()
     assert bench.hbm_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
+
+
+def test_host_info_reads_the_model_name(tmp_path):
+    f = tmp_path / "cpuinfo"
+    f.write_text("processor\t: 0\nvendor_id\t: X\nmodel name\t: Some CPU @ 2.0GHz\nflags\t: a\n")
+    info = bench.host_info(str(f))
+    assert info["model"] == "Some CPU @ 2.0GHz" and info["nproc"] == os.cpu_count()
+    assert bench.host_info(str(tmp_path / "missing"))["model"] is None
