@@ -8,14 +8,15 @@
 // bisection's test at t is therefore the same as "t <= T", where T is the largest weight value v
 // with mass(W >= v) >= p (T = 0 when the row's mass stays below p).  This kernel finds T, then
 // bisect_scalar replays the bisection's midpoints, stopping rules and result as scalar arithmetic.
-// T is a mass-weighted order statistic, found over the row held in registers with shared-memory
-// atomics for a small share of the weights only (one shared atomic costs about as much issue
-// bandwidth as the rest of a weight's work):
-//   bracket  a count histogram of the fp32 bit patterns over [L, max W] (kNB log-spaced bins);
-//            its estimated mass profile (bin middle values) gives a key range that holds T.
-//            Heavy weights (>= 4 x the mean) are always counted; TWL_PRUNE_SAMPLE = k > 1 counts
-//            one in k of the others and widens the range by the sampling variance (fewer shared
-//            atomics, but the wider range costs more than it saves on the rows measured).
+// T is a mass-weighted order statistic, found over the row held in registers; shared-memory
+// atomics count every weight once for the bracket and only the few weights inside its range after
+// that:
+//   bracket  a count histogram of the fp32 bit patterns over [L, max W] (kNB log-spaced bins), one
+//            shared add per weight (to a dummy word when outside); its estimated mass profile
+//            (bin middle values) gives a key range that holds T.  A build with
+//            TWL_PRUNE_SAMPLE = k > 1 counts every weight >= 4 x the mean but only one in k of
+//            the others, and widens the range by the sampling variance (fewer shared adds, but
+//            the wider range costs more than it saves on the rows measured).
 //            L = (sum W - p) / (2 n): the weights below L sum to less than (sum - p) / 2, so T >= L.
 //   exact    one pass: the weights above the range add up to the mass above it (fp32 pairwise per
 //            thread, fp64 across threads); the weights inside it go to per-thread lists, then to
