@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 from oracle import twl_oracle as O
-from tests.twl_checks import W_ATOL, W_RTOL, group_workload
+from tests.twl_checks import W_ATOL, W_RTOL
 from workloads import synth
 
 D = 128

@@ -4,7 +4,6 @@ Small workloads span several tiles and ragged tails (partial last pages, group s
 permuted page tables); the full-size workloads are checked on sampled (b, kv-head) groups that the
 oracle recomputes one by one.  Criteria: see tests/twl_checks.py.
 """
-import math
 
 import numpy as np
 import pytest
