@@ -73,3 +73,19 @@ def test_host_info_reads_the_model_name(tmp_path):
     info = bench.host_info(str(f))
     assert info["model"] == "Some CPU @ 2.0GHz" and info["nproc"] == os.cpu_count()
     assert bench.host_info(str(tmp_path / "missing"))["model"] is None
+
+
+def test_configs_name_their_workload_and_l2_policy():
+    for name in bench.WORKLOADS:
+        cfg = bench.workload_config(name)
+        assert cfg["workload"] and "l2" in cfg and "model" not in cfg
+    cfg = bench.prune_rows_config([8192, 131072], {8192: 4, 131072: 1})
+    assert cfg["rows"] == 4096 and cfg["n"] == [8192, 131072] and "l2" in cfg
+    assert bench.append_config()["workload"]
+
+
+def test_bench_help_runs_without_a_gpu():
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "--workload" in r.stdout and "--impl" in r.stdout
