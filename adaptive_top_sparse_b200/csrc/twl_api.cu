@@ -182,6 +182,20 @@ EstimateWs carve_estimate(Carve& c, int batch, int hq, int hkv, int max_pages) {
 }
 
 }  // namespace
+
+twl_status check_sparse_decode_args(const void* q, int num_q_heads, const twl_paged_kv* kv,
+                                    const int32_t* tok, const int32_t* tok_count, int tok_stride,
+                                    float sm_scale, const float* o, const float* lse, KV* out) {
+  twl_status st = check_kv(kv, true, true, out);
+  if (st != TWL_OK) return st;
+  if ((st = check_heads(num_q_heads, out->hkv)) != TWL_OK) return st;
+  if (!q || !tok || !tok_count || !o || !lse || tok_stride < 1 || !aligned(q, 16) ||
+      !aligned(o, 16) || !(sm_scale > 0.f) || isinf(sm_scale))
+    return TWL_ERR_INVALID_ARG;
+  if ((long long)out->batch * out->hkv > 4096) return TWL_ERR_UNSUPPORTED;
+  return TWL_OK;
+}
+
 }  // namespace twl
 
 using namespace twl;
@@ -471,13 +485,9 @@ twl_status twl_sparse_decode(const void* q, int32_t num_q_heads, const twl_paged
                              float sm_scale, float* o, float* lse, void* ws, size_t ws_bytes,
                              twl_stream_t stream) {
   KV k;
-  twl_status st = check_kv(kv, true, true, &k);
+  twl_status st = check_sparse_decode_args(q, num_q_heads, kv, tok, tok_count, tok_stride,
+                                           sm_scale, o, lse, &k);
   if (st != TWL_OK) return st;
-  if ((st = check_heads(num_q_heads, k.hkv)) != TWL_OK) return st;
-  if (!q || !tok || !tok_count || !o || !lse || tok_stride < 1 || !aligned(q, 16) ||
-      !aligned(o, 16) || !(sm_scale > 0.f) || isinf(sm_scale))
-    return TWL_ERR_INVALID_ARG;
-  if ((long long)k.batch * k.hkv > 4096) return TWL_ERR_UNSUPPORTED;
   Carve c{static_cast<char*>(ws)};
   void* partials = c.take<char>(attend_partial_bytes(k.batch, num_q_heads, k.hkv, tok_stride));
   if ((st = check_ws(ws, ws_bytes, c.off)) != TWL_OK) return st;

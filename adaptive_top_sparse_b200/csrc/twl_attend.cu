@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(256)
 
 size_t attend_partial_bytes(int batch, int hq, int hkv, int tok_stride) {
   const int g = hq / hkv;
-  const size_t items = (size_t)batch * hkv * ((tok_stride + kChunk - 1) / kChunk);
+  const size_t items = (size_t)batch * hkv * (((size_t)tok_stride + kChunk - 1) / kChunk);
   size_t bytes = items * g * (kHeadDim + 1) * sizeof(float);
   bytes += ((size_t)batch * hkv + 1) * sizeof(int);
   return (bytes + 255) & ~(size_t)255;

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "twl.h"
+
 namespace twl {
 
 struct KV {
@@ -82,5 +84,11 @@ cudaError_t launch_sparse_decode(const uint16_t* q, int hq, const KV& kv, const 
                                  float* lse, void* partials, uint32_t* flags, cudaStream_t s);
 
 int num_sms();
+
+// twl_api.cu: the argument checks of twl_sparse_decode (also run by its no-allocation variant
+// before it sizes the request); fills *out on success.
+twl_status check_sparse_decode_args(const void* q, int num_q_heads, const twl_paged_kv* kv,
+                                    const int32_t* tok, const int32_t* tok_count, int tok_stride,
+                                    float sm_scale, const float* o, const float* lse, KV* out);
 
 }  // namespace twl

@@ -11,6 +11,10 @@
 // not fit are rejected with TWL_ERR_SCRATCH_LIMIT before anything is launched.  The device
 // address of the array is looked up once per device (cudaGetSymbolAddress, with that device
 // current) on the first call made on that device; make that first call before any stream capture.
+// The looked-up address belongs to the device's primary context as it was at that first call: it
+// does not survive cudaDeviceReset (which unloads the library image from the device), nor does it
+// serve a different context made current on the same device; such callers must not use this entry
+// point afterwards.
 // All calls share the array, so calls that overlap on the GPU (different streams, or different
 // host threads) race on it.  Nothing in it needs to start at zero: the partials are written before
 // they are read, and the device flags of its 256-byte header are not reported to the caller.
@@ -20,6 +24,7 @@
 #include <mutex>
 
 #include "twl.h"
+#include "twl_kernels.h"
 
 namespace {
 
@@ -58,9 +63,12 @@ extern "C" twl_status twl_sparse_decode_noalloc(const void* q, int32_t num_q_hea
                                                 const int32_t* tok_count, int32_t tok_stride,
                                                 float sm_scale, float* o, float* lse,
                                                 twl_stream_t stream) {
-  if (kv == nullptr || num_q_heads < 1 || kv->num_kv_heads < 1 || kv->batch < 1 ||
-      tok_stride < 1)
-    return TWL_ERR_INVALID_ARG;
+  // the argument checks of twl_sparse_decode first, so a malformed request gets the same
+  // status as there (not TWL_ERR_SCRATCH_LIMIT)
+  twl::KV k;
+  const twl_status chk = twl::check_sparse_decode_args(q, num_q_heads, kv, tok, tok_count,
+                                                       tok_stride, sm_scale, o, lse, &k);
+  if (chk != TWL_OK) return chk;
   const size_t need = twl_workspace_bytes(TWL_OP_SPARSE_DECODE, kv->batch, num_q_heads,
                                           kv->num_kv_heads, 0, 0, 0, tok_stride);
   if (need == 0) return TWL_ERR_INVALID_ARG;

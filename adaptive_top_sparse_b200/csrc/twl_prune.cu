@@ -104,7 +104,8 @@ cudaError_t launch_prune(const float* w, const int* row_len, const int* row_len_
                          int row_stride, float p, float eps, float* m_out, int* kept_count,
                          int* kept_idx, cudaStream_t s) {
   if (rows <= 0) return cudaSuccess;
-  if (!getenv("TWL_PRUNE_BISECT")) {
+#ifndef TWL_PRUNE_BISECT_ONLY  // a build option (never a run-time switch): direct bisection only
+  {
     // 64 weights per thread above 16384 weights per row (no cluster up to 32768), else 32
     const cudaError_t e =
         row_stride > 16384
@@ -114,6 +115,7 @@ cudaError_t launch_prune(const float* w, const int* row_len, const int* row_len_
                                         kept_count, kept_idx, s);
     if (e != cudaErrorNotSupported) return e;
   }
+#endif
   const int staged = row_stride <= kPruneSmemFloats;
   const size_t smem = staged ? (size_t)row_stride * sizeof(float) : 0;
   if (smem > 48 * 1024) {

@@ -476,6 +476,11 @@ __global__ void __launch_bounds__(kRMaxThreads, TWL_PRUNE_MIN_BLOCKS) k_prune_ro
       m = 0.f;  // p = 1 keeps every weight: an fp32 mass cannot resolve 1.0
     } else if (isinf(top)) {
       m = top;  // mass(W >= inf) is infinite
+    } else if (total * (1.f + 0x1p-16f) < a.p) {
+      // the whole row weighs less than p: no threshold reaches p, so T = 0 and the bisection
+      // ends at m = 0.  The fp32 row sum is within ~80 roundings (< 2^-16 relative) of the exact
+      // one, so the exact mass is below p too; every thread holds the same total.
+      m = 0.f;
     } else {
       const uint32_t kt = __float_as_uint(top);
       const double P = (double)a.p;

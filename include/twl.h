@@ -306,8 +306,11 @@ twl_status twl_sparse_decode(const void* q, int32_t num_q_heads, const twl_paged
  * process exits.  A request whose scratch (twl_workspace_bytes(TWL_OP_SPARSE_DECODE, ...)) exceeds
  * it returns TWL_ERR_SCRATCH_LIMIT and launches nothing.  The first call on a device looks up the
  * array's device address (once per device, that device current); make it before any stream
- * capture.  Every call shares the array: calls that overlap on the GPU race.  Device flags are not
- * reported by this call.  It allocates nothing. */
+ * capture.  That address is kept for the life of the process: it does not survive cudaDeviceReset
+ * or serve another context made current on the same device, so do not call this entry point after
+ * either.  Every call shares the array: calls that overlap on the GPU race.  Device flags are not
+ * reported by this call.  Arguments are checked as by twl_sparse_decode before the scratch size.
+ * It allocates nothing. */
 size_t twl_noalloc_scratch_bytes(void);
 twl_status twl_sparse_decode_noalloc(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
                                      const int32_t* tok, const int32_t* tok_count,

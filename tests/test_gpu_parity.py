@@ -222,6 +222,35 @@ def test_prune_hard_rows(n, p):
         check_prune_row(w_np[r], m[r], int(kc[r]), ki[r], p, 1e-6, f"n{n} p{p} hard row {r}")
 
 
+@pytest.mark.parametrize("n", [8192, 32768, 131072])
+def test_prune_rows_mass_below_p(n):
+    """Rows whose whole mass is below p: no threshold reaches p, so m = 0 and every weight is
+    kept.  Rows whose mass sits just above p (by 1e-6 or 1e-4 relative) must still be searched."""
+    rng = np.random.default_rng(n + 5)
+    p = 0.9
+    base = [rng.dirichlet(np.ones(n)), rng.dirichlet(np.full(n, 0.05))]
+    rows = []
+    for w in base:
+        for scale in (0.5, p * (1 - 1e-4), p * (1 + 1e-6), p * (1 + 1e-4)):
+            rows.append(w * scale)
+    w_np = np.stack(rows).astype(np.float32)
+    nr = w_np.shape[0]
+    w = torch.from_numpy(w_np).cuda()
+    m = torch.zeros(nr, dtype=torch.float32, device="cuda")
+    kc = torch.zeros(nr, dtype=torch.int32, device="cuda")
+    ki = torch.full((nr, n), -1, dtype=torch.int32, device="cuda")
+    twl.twl_prune_top_p(w, None, nr, n, p, 1e-6, m, kc, ki)
+    m, kc, ki = np_(m), np_(kc), np_(ki)
+    for r in range(nr):
+        total = float(w_np[r].astype(np.float64).sum())
+        check_prune_row(w_np[r], m[r], int(kc[r]), ki[r], p, 1e-6, f"n{n} row {r} sum {total}")
+        if total < p:
+            assert m[r] == 0 and kc[r] == n, (r, total)
+        else:   # searched: the bisection's own threshold (fp64 masses in the oracle)
+            m_or, _ = O.top_p_bisect(w_np[r], p, 1e-6)
+            assert m[r] == m_or, (r, total, float(m[r]), float(m_or))
+
+
 @pytest.mark.parametrize("n", [8192, 131072])
 def test_prune_rows_ragged_lengths(n):
     """Per-row lengths (row_len) shorter than the stride, including 0, 1 and non-multiples of 4."""
@@ -563,6 +592,61 @@ def test_full_batch16_sampled():
     _full_check(wl, [(0, 0), (5, 3), (15, 7)])
 
 
-def test_full_128k_sampled():
+@pytest.fixture(scope="module")
+def c4_layer():
     wl = synth.config4()
-    _full_check(wl, [(0, 1), (3, 6)])
+    layer = DecodeLayer.from_workload(wl)
+    layer.build_aux()
+    torch.cuda.synchronize()
+    return wl, layer
+
+
+@pytest.mark.parametrize("p", [0.70, 0.85, 0.95])
+def test_full_128k_sampled(c4_layer, p):
+    """The long-context layer at every p of its sweep (the bench times all three)."""
+    wl, layer = c4_layer
+    wl.p = p
+    try:
+        st, o, lse = _run_step(wl, layer)
+        for b, kvh in [(0, 1), (1, 4), (3, 6)]:
+            check_step_group(wl, b, kvh, st, o, lse)
+        assert layer.status()[0] == twl.TWL_OK
+    finally:
+        wl.p = 0.85
+
+
+def _live_counts(wl, b, kvh, p):
+    """Per head of the group: the oracle's candidate count and the size of the live set
+    {W >= (1 - p) / (2 nc)} that a threshold search over live weights would have to rank."""
+    from twl_checks import group_workload
+    sub = group_workload(wl, b, kvh)
+    sub.p = p
+    r = O.decode_step(sub, with_attention=False)
+    out = []
+    for d in r["heads"].values():
+        nc = d["cand"].size
+        out.append((nc, int(np.count_nonzero(d["w"] >= (1 - p) / (2 * nc)))))
+    return out
+
+
+@pytest.mark.parametrize("n", [8192, 40000])
+@pytest.mark.parametrize("p", [0.85, 0.9995])
+def test_decode_step_diffuse_heads(n, p):
+    """Diffuse heads (no heavy tokens, logit temperature 2-8): most candidates survive top-p, so
+    the threshold search runs over thousands of live weights (more than any CTA has threads) and,
+    at 40000 tokens, over more candidates than a CTA holds in registers; p within 1e-3 of 1 also
+    turns off the live-set bound.  Every group against the oracle."""
+    wl = synth.config_diffuse(n=n)
+    wl.p = p
+    layer = DecodeLayer.from_workload(wl)
+    layer.build_aux()
+    st, o, lse = _run_step(wl, layer)
+    for kvh in range(wl.num_kv_heads):
+        check_step_group(wl, 0, kvh, st, o, lse)
+    assert layer.status()[0] == twl.TWL_OK
+    live = _live_counts(wl, 0, 0, p)
+    assert min(l for _, l in live) > 1024, live
+    if n == 40000:
+        assert min(nc for nc, _ in live) > 16 * 512, live
+    kept = st["kept_count"].reshape(-1) / np.maximum(st["cand_count"].reshape(-1), 1)
+    assert kept.min() > 0.5, kept

@@ -183,6 +183,33 @@ def test_scores_pins():
     assert check_scores(O.page_scores, np.random.default_rng(5))
 
 
+def _score_order_case():
+    case = _golden("score_order.json")
+
+    def vec(spec):
+        v = np.full(128, spec["default"], dtype=F16)
+        for c, x in spec["set"].items():
+            v[int(c)] = F16(x)
+        return v
+
+    return case, vec(case["q"]), vec(case["min"]), vec(case["max"])
+
+
+def check_score_order(score_fn):
+    """The hand-worked case of tests/golden/score_order.json: only the fixed summation order
+    (16 left-to-right partials of 8 channels, then pairs (l, l+8), (l, l+4), (l, l+2), (l, l+1))
+    gives its bits."""
+    case, q, mn, mx = _score_order_case()
+    got = F32(score_fn(q, mn[None], mx[None])[0])
+    return int(np.array([got], dtype=F32).view(np.uint32)[0]) == int(case["score_bits"], 16)
+
+
+def test_scores_summation_order_golden():
+    assert check_score_order(O.page_scores)
+    case, q, mn, mx = _score_order_case()
+    assert float(O.page_scores(q, mn[None], mx[None])[0]) == case["score"]
+
+
 def test_scores_fixed_order_is_deterministic_fp32():
     rng = np.random.default_rng(6)
     q = rng.standard_normal(128).astype(F16)
@@ -638,6 +665,49 @@ def test_pins_catch_planted_mistakes():
 
     assert not check_scores(scores_wrong_sign, np.random.default_rng(5))
     assert not check_scores(scores_dropped_term, np.random.default_rng(5))
+
+    # summation orders other than the fixed one (each term is exact, only the order differs)
+    def terms(q, mn, mx):
+        q = np.asarray(q, dtype=F16).astype(F32)
+        return np.where(q > 0, q * np.asarray(mx, F16).astype(F32)[0],
+                        q * np.asarray(mn, F16).astype(F32)[0]).astype(F32)
+
+    def seq_sum(vals):
+        acc = F32(0)
+        for v in vals:
+            acc = F32(acc + F32(v))
+        return acc
+
+    def tree_sum(vals):                      # adjacent pairs (0,1), (2,3), ...
+        v = [F32(x) for x in vals]
+        while len(v) > 1:
+            v = [F32(v[i] + v[i + 1]) for i in range(0, len(v), 2)]
+        return v[0]
+
+    def fixed_tree(part):                    # the pairs (l, l+8), (l, l+4), (l, l+2), (l, l+1)
+        part = [F32(x) for x in part]
+        while len(part) > 1:
+            h = len(part) // 2
+            part = [F32(part[l] + part[l + h]) for l in range(h)]
+        return part[0]
+
+    wrong_orders = {
+        "sequential_128": lambda t: seq_sum(t),
+        "adjacent_pairs_over_channels": lambda t: tree_sum(t),
+        "partials_paired_adjacent": lambda t: tree_sum([seq_sum(t[8 * l:8 * l + 8])
+                                                         for l in range(16)]),
+        "strided_lane_partials": lambda t: fixed_tree([seq_sum(t[l::16]) for l in range(16)]),
+        "partials_right_to_left": lambda t: fixed_tree([seq_sum(t[8 * l:8 * l + 8][::-1])
+                                                         for l in range(16)]),
+        "exact_then_rounded": lambda t: F32(math.fsum(float(x) for x in t)),
+    }
+    want = _golden("score_order.json")["wrong_order_bits"]
+    for name, order in wrong_orders.items():
+        fn = lambda q, mn, mx, order=order: np.array([order(terms(q, mn, mx))], dtype=F32)
+        assert not check_score_order(fn), name
+        case, q, mn, mx = _score_order_case()
+        got = np.array([fn(q, mn[None], mx[None])[0]], dtype=F32).view(np.uint32)[0]
+        assert int(got) == int(want[name], 16), name     # the hand-worked wrong results
 
     def top_p_strict(w, p):              # '>' instead of '>=' on the mass
         order = np.argsort(-w, kind="stable")

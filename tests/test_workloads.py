@@ -81,3 +81,35 @@ def test_pruner_rows_follow_the_recipe():
             assert np.allclose(ratio, np.arange(1, 9) ** (-s), rtol=1e-5)
     again, _ = synth.config5_rows(200, 1024, seed=2, tie_frac=0.05)
     assert np.array_equal(w, again)
+
+
+def test_temperature_recipe_divides_the_query():
+    # q_h = g_h / tau_h: tau_h * q_h has unit-variance channels whatever tau_h is
+    wl = synth.make_decode("t", 2, 16, 4, [64, 64], seed=5, temperature=True)
+    taus = wl.extra["tau"]
+    assert taus.min() >= 0.25 and taus.max() <= 8.0
+    g = wl.q.astype(np.float64) * taus[:, :, None]
+    assert abs(g.std() - 1.0) < 0.05 and abs(g.mean()) < 0.05
+    plain = synth.make_decode("t", 2, 16, 4, [64, 64], seed=5)
+    # the same draws g_h as the scaled recipe (q_h = tau_h g_h), up to fp16 rounding
+    assert np.allclose(plain.q.astype(np.float64) / taus[:, :, None], g, rtol=2e-3, atol=2e-3)
+
+
+def test_multi_head_layers_mix_focused_and_diffuse_heads():
+    """With tau as a logit temperature the 32K layer's heads span focused and diffuse regimes
+    (oracle kept fractions on an 8K-context copy of the layer, same seed); the diffuse variant
+    keeps most candidates in every head."""
+    from oracle import twl_oracle as O
+    from tests.twl_checks import group_workload
+
+    def kept_fractions(wl):
+        out = []
+        for kvh in range(wl.num_kv_heads):
+            r = O.decode_step(group_workload(wl, 0, kvh), with_attention=False)
+            out += [d["kept"].size / d["cand"].size for d in r["heads"].values()]
+        return np.array(out)
+
+    fr = kept_fractions(synth.config2(n=8192))
+    assert np.median(fr) < 0.02 and fr.max() > 0.2, fr
+    fd = kept_fractions(synth.config_diffuse(n=8192))
+    assert fd.min() > 0.5, fd

@@ -74,11 +74,12 @@ def make_decode(name: str, batch: int, num_q_heads: int, num_kv_heads: int, seq_
                 sink_coef: float = 2.0, spans: int = 0, span_len: int = 512,
                 permute_pages: bool = False, max_pages: int | None = None,
                 p: float = 0.85, eps: float = 1e-6, budget_div: int = 4,
-                budget_pages: int = 0) -> DecodeWorkload:
+                budget_pages: int = 0, temperature: bool = False) -> DecodeWorkload:
     """Draw one decode layer.
 
-    K, V ~ N(0, 1) per channel.  Query q_h = tau_h * g_h with g_h ~ N(0, I_D); tau_h is fixed
-    (``tau``) or log-uniform in ``tau_range``.  Per (b, kv-head): ``heavy_count`` (default
+    K, V ~ N(0, 1) per channel.  Query q_h = tau_h * g_h with g_h ~ N(0, I_D), or, with
+    ``temperature``, q_h = g_h / tau_h (tau_h is then a logit temperature: every logit of head h
+    is divided by it); tau_h is fixed (``tau``) or log-uniform in ``tau_range``.  Per (b, kv-head): ``heavy_count`` (default
     round(heavy_frac * N_b)) heavy tokens, each aimed at one q-head h* of the group,
     K_i = heavy_coef * sqrt(D) * q_h*/|q_h*| + xi; positions uniform in [num_sinks, N_b) or, with
     ``spans`` > 0, uniform inside that head's spans of ``span_len`` tokens.  Sink tokens 0..3:
@@ -109,7 +110,7 @@ def make_decode(name: str, batch: int, num_q_heads: int, num_kv_heads: int, seq_
         taus = np.exp(rng.uniform(lo, hi, size=(batch, num_q_heads)))
     else:
         taus = np.full((batch, num_q_heads), float(tau))
-    q64 = gq * taus[:, :, None]
+    q64 = gq / taus[:, :, None] if temperature else gq * taus[:, :, None]
     q = q64.astype(np.float16)
 
     # base K, V in physical layout (bulk normals from a seeded torch CPU generator: faster
@@ -180,8 +181,10 @@ def config1(seed: int = 0, n: int = 4096) -> DecodeWorkload:
 
 
 def config2(seed: int = 0, n: int = 32768, batch: int = 1) -> DecodeWorkload:
-    """Llama-3.1-8B-shaped GQA layer (32 q-heads / 8 kv-heads), batch 1, 32K context."""
-    return make_decode(f"c2_gqa_b{batch}_{n // 1024}k", batch, 32, 8, [n] * batch, seed=seed)
+    """Llama-3.1-8B-shaped GQA layer (32 q-heads / 8 kv-heads), batch 1, 32K context; per-head
+    logit temperature log-uniform in [0.25, 8] (focused and diffuse heads)."""
+    return make_decode(f"c2_gqa_b{batch}_{n // 1024}k", batch, 32, 8, [n] * batch, seed=seed,
+                       temperature=True)
 
 
 def config3(seed: int = 0, batch: int = 16, n_lo: int = 8192, n_hi: int = 32768,
@@ -191,20 +194,28 @@ def config3(seed: int = 0, batch: int = 16, n_lo: int = 8192, n_hi: int = 32768,
     lens = rng.integers(n_lo, n_hi + 1, size=batch)
     max_pages = _pages(n_hi)
     return make_decode(f"c3_gqa_b{batch}_{n_lo // 1024}k-{n_hi // 1024}k", batch, num_q_heads,
-                       num_kv_heads, lens, seed=seed, permute_pages=True, max_pages=max_pages)
+                       num_kv_heads, lens, seed=seed, permute_pages=True, max_pages=max_pages,
+                       temperature=True)
 
 
 def config4(seed: int = 0, n: int = 131072, batch: int = 4, p: float = 0.85) -> DecodeWorkload:
     """Long context, batch 4, heavy tokens clustered in 8 spans of 512 tokens per head."""
     return make_decode(f"c4_gqa_b{batch}_{n // 1024}k_p{int(round(p * 100))}", batch, 32, 8,
                        [n] * batch, seed=seed, spans=8, span_len=min(512, max(16, n // 16)),
-                       p=p)
+                       p=p, temperature=True)
 
 
 def config6(seed: int = 0, batch: int = 64, n: int = 8192) -> DecodeWorkload:
     """Serving batch: 64 sequences of 8192 tokens, 32/8 heads, pages randomly permuted."""
     return make_decode(f"c6_gqa_b{batch}_{n // 1024}k", batch, 32, 8, [n] * batch, seed=seed,
-                       permute_pages=True)
+                       permute_pages=True, temperature=True)
+
+
+def config_diffuse(seed: int = 0, n: int = 32768, batch: int = 1) -> DecodeWorkload:
+    """The 32K GQA layer with diffuse heads only: no heavy tokens (sinks kept), logit temperature
+    log-uniform in [2, 8], so every head spreads its weight over most of its candidates."""
+    return make_decode(f"c2_diffuse_b{batch}_{n // 1024}k", batch, 32, 8, [n] * batch,
+                       seed=seed, temperature=True, heavy_frac=0.0, tau_range=(2.0, 8.0))
 
 
 def config5_rows(rows: int, n: int, seed: int = 0, tie_frac: float = 0.01):
