@@ -7,8 +7,8 @@
 #include <stdlib.h>
 
 #include "twl_common.cuh"
-#include "twl_fused.h"
 #include "twl_kernels.h"
+#include "twl_step.h"
 
 namespace twl {
 
@@ -97,50 +97,8 @@ twl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TWL_OK : TWL_E
 
 uint32_t* flags_of(void* ws) { return ws ? &reinterpret_cast<WsHeader*>(ws)->flags : nullptr; }
 
-// Cluster size for the fused kernel, cached per (device, group size, wanted size, smem).  A size
-// forced through TWL_FUSED_CLUSTER is taken as is (clusters then run in as many waves as needed).
-int fitted_cluster(int g, int want, int groups, int smem_bytes, bool small) {
-  if (const char* env = getenv("TWL_FUSED_CLUSTER")) {
-    const int f = atoi(env);
-    if (f >= 1 && f <= 16) return want;
-  }
-  struct Entry {
-    int dev, g, want, groups, smem, small, c;
-  };
-  static std::mutex mu;
-  static Entry cache[64];
-  static int n = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  std::lock_guard<std::mutex> lock(mu);
-  for (int i = 0; i < n; ++i)
-    if (cache[i].dev == dev && cache[i].g == g && cache[i].want == want &&
-        cache[i].groups == groups && cache[i].smem == smem_bytes && cache[i].small == (int)small)
-      return cache[i].c;
-  const int c = small ? fused256::fit_cluster(g, want, groups, smem_bytes)
-                      : fused512::fit_cluster(g, want, groups, smem_bytes);
-  if (n < 64) cache[n++] = Entry{dev, g, want, groups, smem_bytes, (int)small, c};
-  return c;
-}
-
-// The 256-thread build (two CTAs per SM) when the 512-thread build would give each group a
-// single CTA (more than SMs / 2 groups) and the sequences are at most 2048 pages (32K tokens), so
-// its 110 KB of shared memory holds the top-k keys and histogram; measured faster there (batch
-// 10-64 at 8K-32K), slower for the few large clusters of small batches or long contexts.
-// TWL_FUSED_THREADS=256 or 512 forces one.
-bool use_small_ctas(int groups, int max_pages) {
-  if (const char* env = getenv("TWL_FUSED_THREADS")) {
-    const int t = atoi(env);
-    if (t == 256) return true;
-    if (t == 512) return false;
-  }
-  return 2 * groups > num_sms() && max_pages <= 2048;
-}
-
 size_t decode_step_ws_bytes(int batch, int hq, int hkv, int max_pages, int max_budget) {
-  const size_t a = fused512::fused_workspace_bytes(batch, hq, hkv, max_pages, max_budget);
-  const size_t b = fused256::fused_workspace_bytes(batch, hq, hkv, max_pages, max_budget);
-  return a > b ? a : b;
+  return step::workspace_bytes(batch, hq, hkv, max_pages, max_budget);
 }
 
 // ---------------------------------------------------------------- workspace layouts
@@ -242,7 +200,7 @@ size_t twl_workspace_bytes(int32_t op, int32_t batch, int32_t num_q_heads, int32
 
 twl_status twl_workspace_init(void* ws, size_t ws_bytes, twl_stream_t stream) {
   if (!ws || ws_bytes < (size_t)kHeaderBytes || !aligned(ws, kAlign)) return TWL_ERR_WORKSPACE;
-  return cuda_status(cudaMemsetAsync(ws, 0, kHeaderBytes, (cudaStream_t)stream));
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
 }
 
 twl_status twl_device_status(void* ws, uint32_t* flags, int32_t clear, twl_stream_t stream) {
@@ -511,23 +469,15 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
     return TWL_ERR_INVALID_ARG;
   if (!(p > 0.f && p <= 1.f) || !(eps > 0.f) || isinf(eps)) return TWL_ERR_INVALID_ARG;
   if ((st = check_budget(budget_pages, budget_div, max_budget, k.max_pages)) != TWL_OK) return st;
-  bool small = use_small_ctas(k.batch * k.hkv, k.max_pages);
-  FusedPlan pl{};
-  if (small) {
-    pl = fused256::plan_fused(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
-    if (!pl.ok) small = false;  // too little shared memory at two CTAs per SM
-  }
-  if (!small) pl = fused512::plan_fused(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
+  const step::Plan pl = step::plan(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
   if (!pl.ok) return TWL_ERR_UNSUPPORTED;
   Carve c{static_cast<char*>(ws)};
-  char* fws = c.take<char>(decode_step_ws_bytes(k.batch, num_q_heads, k.hkv, k.max_pages,
+  char* sws = c.take<char>(decode_step_ws_bytes(k.batch, num_q_heads, k.hkv, k.max_pages,
                                                 max_budget));
   if ((st = check_ws(ws, ws_bytes, c.off)) != TWL_OK) return st;
-  pl.cluster =
-      fitted_cluster(num_q_heads / k.hkv, pl.cluster, k.batch * k.hkv, pl.smem_bytes, small);
   const twl_step_stats none = {};
   const twl_step_stats& so = stats ? *stats : none;
-  FusedArgs a = {};
+  step::Args a = {};
   a.q = static_cast<const uint16_t*>(q);
   a.hq = num_q_heads;
   a.kv = k;
@@ -549,22 +499,11 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
   a.cand_count = so.cand_count;
   a.threshold = so.threshold;
   a.kept_count = so.kept_count;
-  a.union_count = so.union_count;
   a.union_tok = so.union_tok;
-  a.want_union = (so.union_tok != nullptr || so.union_count != nullptr) ? 1 : 0;
-  a.pt_smem = pl.pt_smem ? 1 : 0;
+  a.union_count = so.union_count;
   a.flags = flags_of(ws);
-  a.sel_words = pl.sel_words;
-  a.cand_stride = pl.cand_stride;
-  a.union_stride = pl.union_stride;
-  a.cluster = pl.cluster;
-  a.smem_bytes = pl.smem_bytes;
-  if (small) {
-    fused256::carve_fused(a, fws, pl, k.batch, num_q_heads, k.hkv, k.max_pages);
-    return cuda_status(fused256::launch_fused(a, pl, (cudaStream_t)stream));
-  }
-  fused512::carve_fused(a, fws, pl, k.batch, num_q_heads, k.hkv, k.max_pages);
-  return cuda_status(fused512::launch_fused(a, pl, (cudaStream_t)stream));
+  step::carve(a, sws, pl, k.batch, num_q_heads, k.hkv, k.max_pages);
+  return cuda_status(step::launch(a, pl, (cudaStream_t)stream));
 }
 
 }  // extern "C"

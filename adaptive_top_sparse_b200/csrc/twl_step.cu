@@ -1,0 +1,1969 @@
+// The decode step of hierarchical top-p sparse attention as ONE persistent grid over every SM.
+//
+// "Twilight: Adaptive Attention Sparsity with Hierarchical Top-p Pruning": notes page, "Overall
+// framework" (a conservative selector, then top-p pruning of its tokens) and "Key designs"
+// (binary-search top-p, 4-bit K cache, head flattening for load balancing); summary, sections
+// 4.1-4.3 and appendices B.1-B.2 (INT4 SpGEMV once per GQA group over the union of the heads'
+// pages, group-wise variable-length attention).
+//
+// Every dependency of the path stays inside one (sequence, kv-head) group, but the work of a group
+// is far from uniform: page scoring and the INT4 estimate stream megabytes, top-k and top-p are
+// per-head searches over a few kilobytes, attention scales with the kept tokens (which differ
+// ~50x between heads).  So the step is cut into work items, each a job for one CTA:
+//   score   a chunk of a group's pages, scored for all G heads       -> order keys  (L2)
+//   top-k   one q-head's k best pages                                -> page bitmap (L2)
+//           the last top-k item of a group forms the union of its heads' pages and, per union
+//           page, its physical page and its rank in each head's selection
+//   est     a slice of the union: INT4 dequant-dot on the tensor cores -> logits per head (L2)
+//   prune   one q-head: softmax, top-p threshold m by bisection     -> kept-row bitmap (L2)
+//           the last prune item of a group lists the group's kept tokens (the union over heads)
+//   attend  a slice of that list: fp16 K/V rows gathered, partial (max, sum, o) per head
+//           the last attend item of a group merges the partials by log-sum-exp -> o, lse
+// Items are numbered so that an item depends only on lower-numbered items; the grid is launched
+// with every CTA resident, and each CTA takes the next free number (one atomic).  The lowest
+// unfinished item therefore always has a CTA working on it, so the waits below always end; each
+// is still bounded (TWL_FLAG_TIMEOUT), after which the launch finishes without the missing work.
+// A dependency is a per-group counter in the workspace: producers add to it after a release
+// fence, consumers poll it with acquire loads and read the produced data through L2.  The last
+// CTA to leave clears the counters for the next launch on the workspace.
+//
+// The arithmetic (score order, INT4 products, softmax and threshold search, attention) is the
+// same as the staged kernels', so the selections are bit-identical to twl_select_pages.
+#include "twl_common.cuh"
+#include "twl_step.h"
+
+namespace twl {
+namespace step {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr uint32_t kSpinLimit = 1u << 22;  // polls (>= 64 ns apart) before a wait gives up
+
+struct Shared {
+  int flag;
+  int next;
+  int total;
+  int jlast;
+  int scan[64];
+  uint32_t state[4];
+  unsigned long long t_ready;  // trace builds: when the item's wait ended
+  unsigned long long marks[7];  // trace builds: points inside the item
+};
+
+// Trace build (compile with -DTWL_STEP_TRACE; never in the shipped library): thread 0 of every CTA
+// records, per item, (index, CTA, start, wait end, 7 marks, end) in %globaltimer nanoseconds and
+// the SM clock at start and end into a region
+// at the start of the step's workspace region (before its other arrays).
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#ifdef TWL_STEP_TRACE
+#define TRACE_MARK(sh, k)                                  \
+  do {                                                     \
+    if (threadIdx.x == 0) (sh).marks[(k)] = now_ns();      \
+  } while (0)
+#else
+#define TRACE_MARK(sh, k) \
+  do {                    \
+  } while (0)
+#endif
+
+// ------------------------------------------------------------------------------ synchronisation
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t* counter(const Args& a, int which, int g) {
+  return a.sync + kSyncHead + which * a.groups + g;
+}
+
+// Wait (whole CTA) until *ctr >= target.  False when the wait gave up: the launch was aborted
+// by another CTA's timeout, or this one timed out (it then raises the flag and aborts).
+__device__ bool block_wait(const Args& a, Shared& sh, const uint32_t* ctr, uint32_t target) {
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    uint32_t it = 0;
+    while (ld_acquire(ctr) < target) {
+      if ((++it & 31u) == 0u) {
+        if (ld_acquire(a.sync + kAbort) != 0u) {
+          ok = 0;
+          break;
+        }
+        if (it >= kSpinLimit) {
+          raise_flag(a.flags, TWL_FLAG_TIMEOUT);
+          atomicExch(a.sync + kAbort, 1u);
+          ok = 0;
+          break;
+        }
+      }
+      __nanosleep(64);
+    }
+    sh.flag = ok;
+#ifdef TWL_STEP_TRACE
+    sh.t_ready = now_ns();
+#endif
+  }
+  __syncthreads();
+  const bool ok = sh.flag != 0;
+  __syncthreads();
+  return ok;
+}
+
+// The CTA's results are complete: count this item with a release reduction.  The block barrier
+// orders every thread's writes before thread 0's release (release is cumulative), so a consumer
+// that acquires the counter sees them.
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
+__device__ void block_signal(uint32_t* ctr) {
+  __syncthreads();
+  if (threadIdx.x == 0) red_release_add(ctr, 1u);
+}
+
+// As block_signal; true in every thread of the CTA whose item brought the count to `total`.  Its
+// atomic is acquire-release, so that CTA then sees every other item's results.
+__device__ bool block_signal_last(Shared& sh, uint32_t* ctr, uint32_t total) {
+  __syncthreads();
+  if (threadIdx.x == 0) sh.flag = atom_acq_rel_add(ctr, 1u) + 1u == total;
+  __syncthreads();
+  const bool last = sh.flag != 0;
+  __syncthreads();
+  return last;
+}
+
+__device__ void block_set_ready(uint32_t* f) {
+  __syncthreads();
+  if (threadIdx.x == 0) red_release_add(f, 1u);
+}
+
+__device__ __forceinline__ float ldcg_f(const float* p) { return __ldcg(p); }
+__device__ __forceinline__ int ldcg_i(const int* p) { return __ldcg(p); }
+__device__ __forceinline__ uint32_t ldcg_u(const uint32_t* p) { return __ldcg(p); }
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// Position of the k-th (0-based) set bit of w; requires popc(w) > k.
+__device__ __forceinline__ int nth_set_bit(uint32_t w, int k) {
+  int pos = 0;
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) {
+    const int c = __popc(w & ((1u << s) - 1u));
+    if (k >= c) {
+      k -= c;
+      w >>= s;
+      pos += s;
+    }
+  }
+  return pos;
+}
+
+__device__ __forceinline__ int group_of(const Args& a, int bh) {
+  return (bh / a.hq) * a.kv.hkv + (bh % a.hq) / a.g;
+}
+
+// ------------------------------------------------------------------------------ scores
+// Pages [c * chunk, (c + 1) * chunk) of the group's sequence, scored for every head of the group.
+// The chunk's page-table entries are staged first; the page bounds (512 B per page) are then
+// copied with 16-byte cp.async in passes of up to kScorePass pages, two passes in flight (every
+// copy of a pass is issued at once: measured the fastest way to pull tens of kilobytes per SM).
+// A half-warp scores a page: lane l holds channels 8l..8l+7 of the min and max rows and of each
+// head's query, so the score is the fixed order of the staged selector (8 channels per lane left
+// to right, then the pairs (l, l+8), (l, l+4), (l, l+2), (l, l+1)).
+constexpr int kScorePass = 176;
+
+template <int G>
+__device__ void item_score(const Args& a, Shared& sh, int g, int c, unsigned char* smem) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int half = lane >> 4, l = lane & 15;
+  const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
+  // the chunk's page-table entries are read before the sequence length is known (entries past
+  // the sequence are in the table, only ignored), so the two loads overlap
+  const int p0 = c * a.s_chunk, pmax = min(a.kv.max_pages, p0 + a.s_chunk);
+  int* pt = reinterpret_cast<int*>(smem);
+  unsigned char* buf = smem + ((4 * a.s_chunk + 127) & ~127);
+  for (int i = tid; i < pmax - p0; i += kThreads)
+    pt[i] = a.kv.page_table[(size_t)b * a.kv.max_pages + p0 + i];
+  const Seq sq = load_seq(a.kv.seq_lens, b, a.kv.max_pages, a.flags, c == 0 && tid == 0);
+  const int p1 = min(sq.pages, pmax);
+  const int n = p1 - p0;
+  if (n > 0) {
+    for (int i = tid; i < n; i += kThreads) {
+      const int ph = pt[i];
+      if (ph < 0 || ph >= a.kv.num_phys) {
+        raise_flag(a.flags, TWL_FLAG_BAD_INDEX);
+        pt[i] = -1;
+      }
+    }
+    float qv[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
+                                  a.q + ((size_t)b * a.hq + kvh * G + h) * kHeadDim) + l);
+      unpack8(raw, qv[h]);
+    }
+    __syncthreads();
+    TRACE_MARK(sh, 0);
+    const int npass = (n + kScorePass - 1) / kScorePass;
+    auto issue = [&](int k) {
+      unsigned char* dst = buf + (k & 1) * kScorePass * 512;
+      const int i0 = k * kScorePass, cn = min(kScorePass, n - i0);
+      for (int q = tid; q < 32 * cn; q += kThreads) {
+        const int i = q >> 5, part = q & 31;
+        const int ph = pt[i0 + i];
+        const uint16_t* src = a.bounds + ((size_t)(ph < 0 ? 0 : ph) * a.kv.hkv + kvh) * 2 * kHeadDim;
+        cp_async16(dst + 512 * i + 16 * part, src + 8 * part, ph >= 0);
+      }
+      cp_async_commit();
+    };
+    issue(0);
+    if (npass > 1) issue(1);
+    uint32_t* krow = a.keys + ((size_t)b * a.hq + kvh * G) * a.kv.max_pages + p0;
+#pragma unroll 1
+    for (int k = 0; k < npass; ++k) {
+      if (k + 1 < npass) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+      else cp_async_wait_all();
+      __syncthreads();
+      TRACE_MARK(sh, 1);
+      const unsigned char* src = buf + (k & 1) * kScorePass * 512;
+      const int i0 = k * kScorePass, cn = min(kScorePass, n - i0);
+#pragma unroll 1
+      for (int base = 0; base < cn; base += 2 * kWarps) {  // warp-uniform trip count
+        const int ip = base + 2 * warp + half;
+        const bool in = ip < cn;
+        const int ph = in ? pt[i0 + ip] : -1;
+        const uint4* rowp = reinterpret_cast<const uint4*>(src + 512 * ip);
+        uint4 vmn = make_uint4(0, 0, 0, 0), vmx = vmn;
+        if (ph >= 0) {
+          vmn = rowp[l];
+          vmx = rowp[16 + l];
+        }
+        float mn[8], mx[8];
+        unpack8(vmn, mn);
+        unpack8(vmx, mx);
+        float acc[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float sc = 0.f;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            sc = __fmaf_rn(qv[h][kk], qv[h][kk] > 0.f ? mx[kk] : mn[kk], sc);
+          acc[h] = sc;
+        }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) {
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            acc[h] = __fadd_rn(acc[h], __shfl_xor_sync(0xffffffffu, acc[h], off));
+        }
+        if (in && l < G) {
+          float v = acc[0];
+#pragma unroll
+          for (int h = 1; h < G; ++h) v = (l == h) ? acc[h] : v;
+          if (ph < 0) v = -INFINITY;
+          krow[(size_t)l * a.kv.max_pages + i0 + ip] = f32_key(v);
+        }
+      }
+      __syncthreads();  // the pass's buffer is read before it is refilled
+      if (k + 2 < npass) issue(k + 2);
+    }
+  }
+  block_signal(counter(a, kCntScore, g));
+}
+
+// ------------------------------------------------------------------------------ top-k
+// The kb largest keys of one head (ties to the lower page) -> bitmap of its selected pages.
+// The k-th largest key is narrowed to a key interval [blo, bhi] holding `cand` keys, of which the
+// `remaining` largest are selected (every key above bhi is).  Each pass histograms the keys inside
+// the interval into up to 4096 bins of equal key width and keeps the bin holding the k-th key;
+// float keys are roughly logarithmic in the score, so one pass usually leaves a handful.  A bin of
+// at most 64 keys is ranked exactly; an interval down to one key takes its equal keys in page
+// order.  Writes the bitmap (sbits, shared) and returns nothing; sh.jlast = the last selected page.
+__device__ void topk_bits(const uint32_t* keys, int n_pages, int kb, uint32_t* sbits,
+                          unsigned char* scratch, int scratch_bytes, Shared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = (n_pages + 31) >> 5;
+  constexpr int kGatherCap = 64;
+  constexpr int kBins = 4096;
+  uint32_t* hh = reinterpret_cast<uint32_t*>(scratch);  // [kBins]
+  uint32_t* gkey = hh + kBins;                          // [kGatherCap]
+  int* gidx = reinterpret_cast<int*>(gkey + kGatherCap);  // [kGatherCap]
+  (void)scratch_bytes;
+  uint32_t blo, bhi;
+  {
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i = tid; i < n_pages; i += kThreads) {
+      const uint32_t k = keys[i];
+      kmin = min(kmin, k);
+      kmax = max(kmax, k);
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+      hh[2 * warp] = kmin;
+      hh[2 * warp + 1] = kmax;
+    }
+    __syncthreads();
+    kmin = 0xFFFFFFFFu;
+    kmax = 0u;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      kmin = min(kmin, hh[2 * w]);
+      kmax = max(kmax, hh[2 * w + 1]);
+    }
+    blo = kmin;
+    bhi = kmax;
+  }
+  int remaining = kb;
+  int cand = n_pages;
+  __syncthreads();
+  constexpr int kPerT = kBins / kThreads;  // bins per thread in the scan
+#pragma unroll 1
+  while (cand > kGatherCap && blo < bhi) {
+    const uint32_t range = bhi - blo;
+    const int width = 32 - __clz(range);
+    const int sh_ = width > 12 ? width - 12 : 0;
+    for (int i = tid; i < kBins; i += kThreads) hh[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n_pages; i += kThreads) {
+      const uint32_t key = keys[i];
+      if (key >= blo && key <= bhi) atomicAdd(&hh[(key - blo) >> sh_], 1u);
+    }
+    __syncthreads();
+    // descending scan over the bins: thread t owns bins kBins-1-kPerT*t ... kBins-kPerT*(t+1)
+    const int b0 = kBins - 1 - kPerT * tid;
+    int mine = 0;
+#pragma unroll
+    for (int e = 0; e < kPerT; ++e) mine += (int)hh[b0 - e];
+    const int excl = block_exclusive_scan(mine, sh.scan, nullptr);
+    if (excl < remaining && remaining <= excl + mine) {
+      int run = excl;
+      for (int e = 0; e < kPerT; ++e) {
+        const int c = (int)hh[b0 - e];
+        if (run + c >= remaining) {
+          sh.state[0] = (uint32_t)(b0 - e);
+          sh.state[1] = (uint32_t)(remaining - run);
+          sh.state[2] = (uint32_t)c;
+          break;
+        }
+        run += c;
+      }
+    }
+    __syncthreads();
+    const uint32_t bin = sh.state[0];
+    const uint32_t nlo = blo + (bin << sh_);
+    const uint64_t top = (uint64_t)nlo + ((1ull << sh_) - 1ull);
+    bhi = top < (uint64_t)bhi ? (uint32_t)top : bhi;
+    blo = nlo;
+    remaining = (int)sh.state[1];
+    cand = (int)sh.state[2];
+    __syncthreads();
+  }
+  for (int w = tid; w < nw; w += kThreads) sbits[w] = 0u;
+  if (cand <= kGatherCap) {
+    // ordered gather of the interval's keys: thread t scans a contiguous range of pages
+    const int per = (n_pages + kThreads - 1) / kThreads;
+    const int beg = min(n_pages, tid * per), end = min(n_pages, beg + per);
+    int mine = 0;
+    for (int i = beg; i < end; ++i) {
+      const uint32_t key = keys[i];
+      mine += key >= blo && key <= bhi;
+    }
+    int slot = block_exclusive_scan(mine, sh.scan, nullptr);
+    for (int i = beg; i < end && mine > 0; ++i) {
+      const uint32_t key = keys[i];
+      if (key >= blo && key <= bhi) {
+        gkey[slot] = key;
+        gidx[slot] = i;
+        ++slot;
+        --mine;
+      }
+    }
+    __syncthreads();
+    for (int e = tid; e < cand; e += kThreads) {
+      const uint32_t ke = gkey[e];
+      const int ie = gidx[e];
+      int rank = 0;
+      for (int f = 0; f < cand; ++f) {
+        const uint32_t kf = gkey[f];
+        rank += (kf > ke || (kf == ke && gidx[f] < ie)) ? 1 : 0;
+      }
+      if (rank < remaining) atomicOr(&sbits[ie >> 5], 1u << (ie & 31));
+    }
+    __syncthreads();
+    for (int base = 0; base < 32 * nw; base += kThreads) {
+      const int i = base + tid;
+      const bool above = i < n_pages && keys[i] > bhi;
+      const uint32_t bal = __ballot_sync(0xffffffffu, above);
+      if (lane == 0 && (i >> 5) < nw) atomicOr(&sbits[i >> 5], bal);
+    }
+    __syncthreads();
+    return;
+  }
+  // the interval is down to one key (blo == bhi, the k-th key itself): keys above it are taken,
+  // equal keys in ascending page order.  One element per thread per round; a warp's ballot is
+  // one 32-page word of the bitmap.
+  int* wsum = sh.scan;
+  int carry_eq = 0;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int base = 0; base < 32 * nw; base += kThreads) {
+    const int i = base + tid;
+    const bool in = i < n_pages;
+    const uint32_t key = in ? keys[i] : 0u;
+    const uint32_t gt = __ballot_sync(0xffffffffu, in && key > bhi);
+    const uint32_t eq = __ballot_sync(0xffffffffu, in && key == blo);
+    if (lane == 0) wsum[warp] = __popc(eq);
+    __syncthreads();
+    int eq_before = carry_eq, eq_round = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      if (w < warp) eq_before += wsum[w];
+      eq_round += wsum[w];
+    }
+    const bool take = in && key == blo && eq_before + __popc(eq & lt) < remaining;
+    const uint32_t sel = gt | __ballot_sync(0xffffffffu, take);
+    if (lane == 0 && (i >> 5) < nw) sbits[i >> 5] = sel;
+    carry_eq += eq_round;
+    __syncthreads();
+  }
+}
+
+// One q-head's selection: bitmap -> workspace, candidate count, optional stats.
+template <int G>
+__device__ void item_topk(const Args& a, Shared& sh, int bh, unsigned char* smem, int smem_bytes) {
+  const int tid = threadIdx.x;
+  const int g = group_of(a, bh);
+  const bool ready = block_wait(a, sh, counter(a, kCntScore, g), (uint32_t)a.s_per);
+  const int b = bh / a.hq;
+  uint32_t* sbits = reinterpret_cast<uint32_t*>(smem);                            // [sel_words]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + 4 * ((a.sel_words + 31) & ~31));
+  unsigned char* scratch = reinterpret_cast<unsigned char*>(keys) + 4 * ((a.kv.max_pages + 31) & ~31);
+  const int scratch_bytes = smem_bytes - (int)(scratch - smem);
+  // the key row is loaded up to max_pages while the sequence length is read (keys past the
+  // sequence are never used)
+  {
+    const uint32_t* row = a.keys + (size_t)bh * a.kv.max_pages;
+    constexpr int kB = 8;  // independent loads in flight per thread
+    for (int base = 0; base < a.kv.max_pages; base += kThreads * kB) {
+      uint32_t v[kB];
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int i = base + k * kThreads + tid;
+        v[k] = i < a.kv.max_pages ? ldcg_u(row + i) : 0u;
+      }
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int i = base + k * kThreads + tid;
+        if (i < a.kv.max_pages) keys[i] = v[k];
+      }
+    }
+  }
+  const Seq sq = load_seq(a.kv.seq_lens, b, a.kv.max_pages, a.flags, false);
+  const int n_pages = ready ? sq.pages : 0;
+  int kb = a.budget_pages > 0 ? a.budget_pages : (n_pages + a.budget_div - 1) / a.budget_div;
+  kb = min(min(kb, n_pages), a.max_budget);
+  const int nw = (n_pages + 31) >> 5;
+  __syncthreads();
+  TRACE_MARK(sh, 0);
+  if (n_pages > 0 && n_pages <= kb) {
+    for (int w = tid; w < nw; w += kThreads) {
+      const int lo = 32 * w;
+      sbits[w] = lo + 32 <= n_pages ? 0xFFFFFFFFu : ((1u << (n_pages - lo)) - 1u);
+    }
+    __syncthreads();
+  } else if (n_pages > 0) {
+    topk_bits(keys, n_pages, kb, sbits, scratch, scratch_bytes, sh);
+  }
+  TRACE_MARK(sh, 1);
+  // bitmap and per-word exclusive prefix counts out (a page's rank in the selection is
+  // hpre[w] + popc(bits[w] below it)); the last selected page fixes the candidate count (only it
+  // can be partial); the ascending list when asked
+  uint32_t* out = a.selbits + (size_t)bh * a.sel_words;
+  int* pre = a.hpre + (size_t)bh * a.sel_words;
+  int* list = a.sel_pages ? a.sel_pages + (size_t)bh * a.max_budget : nullptr;
+  int carry = 0, jlast = -1;
+  for (int base = 0; base < nw; base += kThreads) {
+    const int w = base + tid;
+    const uint32_t x = w < nw ? sbits[w] : 0u;
+    int total;
+    int pos = carry + block_exclusive_scan(__popc(x), sh.scan, &total);
+    carry += total;
+    if (w < nw) {
+      out[w] = x;
+      pre[w] = pos;
+      if (x) jlast = 32 * w + 31 - __clz(x);
+    }
+    if (list) {
+      uint32_t y = x;
+      while (y) {
+        list[pos++] = 32 * w + __ffs(y) - 1;
+        y &= y - 1u;
+      }
+    }
+  }
+  if (tid == 0) sh.jlast = -1;
+  __syncthreads();
+  if (jlast >= 0) atomicMax(&sh.jlast, jlast);
+  __syncthreads();
+  if (tid == 0) {
+    const int jl = sh.jlast;
+    const int nc = (kb > 0 && jl >= 0) ? kPage * (kb - 1) + page_rows(sq.n, jl) : 0;
+    a.ncand[bh] = nc;
+    if (a.sel_count) a.sel_count[bh] = kb;
+  }
+}
+
+// ------------------------------------------------------------------------------ INT4 estimate
+// B fragments of the query for the m16n8k16 products: lane (gr, t) holds the channels
+// c0 = 32 t + 8 w8 (w8 = ks / 2) of head gr; k-step ks pairs (c0 + 4e, c0 + 4e + 2) and
+// (c0 + 4e + 1, c0 + 4e + 3), e = ks % 2, the same pairs nibble_pairs() builds from K.
+// Returns the sum of the lane's 32 query channels (for the zero-point term).
+__device__ __forceinline__ float q_fragments(const uint16_t* qh, bool valid, uint32_t (&bf)[8][2]) {
+  const int t = threadIdx.x & 3;
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 v = valid ? __ldg(reinterpret_cast<const uint4*>(qh + 32 * t + 8 * i))
+                          : make_uint4(0, 0, 0, 0);
+    w[4 * i + 0] = v.x;
+    w[4 * i + 1] = v.y;
+    w[4 * i + 2] = v.z;
+    w[4 * i + 3] = v.w;
+  }
+  float qsum = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    qsum += f.x + f.y;
+  }
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int w8 = ks >> 1, e = ks & 1;
+    bf[ks][0] = __byte_perm(w[4 * w8 + 2 * e], w[4 * w8 + 2 * e + 1], 0x5410);
+    bf[ks][1] = __byte_perm(w[4 * w8 + 2 * e], w[4 * w8 + 2 * e + 1], 0x7632);
+  }
+  return qsum;
+}
+
+// Nibbles to fp16 without arithmetic: a byte 0000nnnn read as FP8 E4M3 (sign 0, exponent 000n3,
+// mantissa n2 n1 n0) is n * 2^-9 exactly (subnormal m * 2^-9 for n < 8, (8 + m) * 2^-9 for
+// n >= 8), and that is an exact fp16 value.  A word of 8 nibbles (channels c0..c0+7, low nibble
+// first) gives the bytes (n0, n2, n4, n6) and (n1, n3, n5, n7); each 16-bit half converts to one
+// f16x2 pair.  Products with q are 2^-9 times the integer-nibble products and the fp32 sums scale
+// exactly; the epilogue multiplies by 512.
+__device__ __forceinline__ uint32_t e4m3x2_lo(uint32_t y) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\t}"
+      : "=r"(r)
+      : "r"(y));
+  return r;
+}
+__device__ __forceinline__ uint32_t e4m3x2_hi(uint32_t y) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, h;\n\t}"
+      : "=r"(r)
+      : "r"(y));
+  return r;
+}
+// The four A registers of k-step (w8, e) for rows gr (word x0) and gr + 8 (word x1).
+__device__ __forceinline__ void nibble_pairs(uint32_t x0, uint32_t x1, int e, uint32_t (&av)[4]) {
+  const uint32_t e0 = x0 & 0x0F0F0F0Fu, o0 = (x0 >> 4) & 0x0F0F0F0Fu;
+  const uint32_t e1 = x1 & 0x0F0F0F0Fu, o1 = (x1 >> 4) & 0x0F0F0F0Fu;
+  av[0] = e ? e4m3x2_hi(e0) : e4m3x2_lo(e0);
+  av[1] = e ? e4m3x2_hi(e1) : e4m3x2_lo(e1);
+  av[2] = e ? e4m3x2_hi(o0) : e4m3x2_lo(o0);
+  av[3] = e ? e4m3x2_hi(o1) : e4m3x2_lo(o1);
+}
+
+// Logical pages [c * chunk, (c + 1) * chunk) of group g, in sub-ranges of up to kEstMeta pages:
+// the union of the heads' selections over the sub-range comes from their bitmaps, and every union
+// page's (logical page, physical page, rank in each head's selection) is staged; the rank is the
+// head's published prefix count of its bitmap word plus the set bits below the page.  The INT4
+// tiles (1 KB) and scale/zero rows (64 B) of those pages are then copied with 16-byte cp.async in
+// passes of kEstPass pages, two in flight.  A warp computes two pages at a time, the page as the
+// M = 16 tile of m16n8k16 and the group's heads as N.  Logit slot of (head h, page j, row r) =
+// 16 * (rank of j in h's selection) + r.
+constexpr int kEstPass = 80;
+constexpr int kEstMeta = 480;  // a multiple of kEstPass, and of 32
+
+template <int G>
+__device__ void item_estimate(const Args& a, Shared& sh, int g, int e, unsigned char* smem) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gr = lane >> 2, t = lane & 3;
+  const bool ready = block_wait(a, sh, counter(a, kCntTopK, g), (uint32_t)a.g);
+  const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
+  const Seq sq = load_seq(a.kv.seq_lens, b, a.kv.max_pages, a.flags, false);
+  const int p0 = e * a.e_chunk, p1 = ready ? min(sq.pages, p0 + a.e_chunk) : 0;
+  if (p0 < p1) {
+    const float inv_sqrt_d = 0.08838834764831845f;
+    constexpr int kM = 2 + G;  // ints of metadata per page
+    constexpr int kW = kEstMeta / 32 + 1;  // bitmap words a sub-range touches
+    int* meta = reinterpret_cast<int*>(smem);
+    uint32_t* hb = reinterpret_cast<uint32_t*>(meta + kM * kEstMeta);  // [G][kW]
+    int* hp = reinterpret_cast<int*>(hb + G * kW);                     // [G][kW]
+    uint32_t* ub = reinterpret_cast<uint32_t*>(hp + G * kW);           // [kW]
+    int* upre = reinterpret_cast<int*>(ub + kW);                       // [kW + 1]
+    unsigned char* buf = smem + ((4 * (kM * kEstMeta + (2 * G + 2) * kW + 1) + 127) & ~127);
+    const size_t row0 = (size_t)b * a.hq + kvh * G;
+    uint32_t bf[8][2];
+    const bool head_ok = gr < G;
+    const uint16_t* qh = a.q + ((size_t)b * a.hq + kvh * G + (head_ok ? gr : 0)) * kHeadDim;
+    float qs_part = q_fragments(qh, head_ok, bf);
+    qs_part += __shfl_xor_sync(0xffffffffu, qs_part, 1);
+    qs_part += __shfl_xor_sync(0xffffffffu, qs_part, 2);
+    const float qsum0 = __shfl_sync(0xffffffffu, qs_part, (2 * t) * 4);
+    const float qsum1 = __shfl_sync(0xffffffffu, qs_part, (2 * t + 1) * 4);
+#pragma unroll 1
+    for (int j0 = p0; j0 < p1; j0 += kEstMeta) {
+      const int j1 = min(p1, j0 + kEstMeta);
+      const int w0 = j0 >> 5, nwr = ((j1 - 1) >> 5) - w0 + 1;
+      for (int i = tid; i < G * nwr; i += kThreads) {
+        const int h = i / nwr, wi = i - h * nwr;
+        hb[h * kW + wi] = ldcg_u(a.selbits + (row0 + h) * a.sel_words + w0 + wi);
+        hp[h * kW + wi] = ldcg_i(a.hpre + (row0 + h) * a.sel_words + w0 + wi);
+      }
+      __syncthreads();
+      if (warp == 0) {  // union words cut to [j0, j1), and their exclusive prefix counts
+        uint32_t u = 0;
+        if (lane < nwr) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) u |= hb[h * kW + lane];
+          const int lo = 32 * (w0 + lane);
+          if (lo < j0) u &= ~((1u << (j0 - lo)) - 1u);
+          if (lo + 32 > j1) u &= j1 - lo >= 32 ? 0xFFFFFFFFu : ((1u << (j1 - lo)) - 1u);
+          ub[lane] = u;
+        }
+        int x = __popc(u);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (lane < nwr) upre[lane] = x - __popc(u);
+        if (lane == 31) upre[kW] = x;
+      }
+      __syncthreads();
+      const int n = upre[kW];
+      for (int jj = j0 + tid; jj < j1; jj += kThreads) {
+        const int wi = (jj >> 5) - w0, bit = jj & 31;
+        const uint32_t below = (1u << bit) - 1u;
+        const uint32_t uw = ub[wi];
+        if ((uw >> bit) & 1u) {
+          int* mm = meta + kM * (upre[wi] + __popc(uw & below));
+          mm[0] = jj;
+          mm[1] = load_phys(a.kv.page_table, b, jj, a.kv.max_pages, a.kv.num_phys, a.flags);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const uint32_t x = hb[h * kW + wi];
+            mm[2 + h] = ((x >> bit) & 1u) ? hp[h * kW + wi] + __popc(x & below) : -1;
+          }
+        }
+      }
+      __syncthreads();
+      TRACE_MARK(sh, 0);
+      const int npass = (n + kEstPass - 1) / kEstPass;
+      auto issue = [&](int k) {
+        unsigned char* tl = buf + (k & 1) * kEstPass * 1088;
+        unsigned char* sz = tl + kEstPass * 1024;
+        const int i0 = k * kEstPass, cn = min(kEstPass, n - i0);
+        // 68 chunks of 16 bytes per page (64 of nibbles, 4 of scale/zero)
+        for (int q = tid; q < 68 * cn; q += kThreads) {
+          const int i = q / 68, kk = q - 68 * i;
+          const int ph = meta[(i0 + i) * kM + 1];
+          const size_t tile = ph >= 0 ? ((size_t)ph * a.kv.hkv + kvh) * kPage : 0;
+          if (kk < 64)
+            cp_async16(tl + 1024 * i + 16 * kk, a.k_int4 + tile * (kHeadDim / 2) + 16 * kk, ph >= 0);
+          else
+            cp_async16(sz + 64 * i + 16 * (kk - 64), a.k_sz + tile * 2 + 8 * (kk - 64), ph >= 0);
+        }
+        cp_async_commit();
+      };
+      issue(0);
+      if (npass > 1) issue(1);
+#pragma unroll 1
+      for (int k = 0; k < npass; ++k) {
+        if (k + 1 < npass) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+        else cp_async_wait_all();
+        __syncthreads();
+        TRACE_MARK(sh, 1);
+        const unsigned char* tl = buf + (k & 1) * kEstPass * 1088;
+        const unsigned char* sz = tl + kEstPass * 1024;
+        const int i0 = k * kEstPass, cn = min(kEstPass, n - i0);
+#pragma unroll 1
+        for (int ib = 2 * warp; ib < cn; ib += 2 * kWarps) {  // warp-uniform
+          float accp[2][4];
+          uint32_t szp[2][2];
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp) {
+            const int ip = ib + pp;
+            uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0;
+            szp[pp][0] = szp[pp][1] = 0;
+            if (ip < cn && meta[(i0 + ip) * kM + 1] >= 0) {
+              const uint4* tp = reinterpret_cast<const uint4*>(tl + 1024 * ip);
+              x0 = tp[lane];
+              x1 = tp[32 + lane];
+              const uint32_t* sp = reinterpret_cast<const uint32_t*>(sz + 64 * ip);
+              szp[pp][0] = sp[gr];
+              szp[pp][1] = sp[gr + 8];
+            }
+            const uint32_t r0[4] = {x0.x, x0.y, x0.z, x0.w};
+            const uint32_t r1[4] = {x1.x, x1.y, x1.z, x1.w};
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const int w8 = ks >> 1, e2 = ks & 1;
+              uint32_t av[4];
+              nibble_pairs(r0[w8], r1[w8], e2, av);
+              mma_16816(acc, av, bf[ks][0], bf[ks][1]);
+            }
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) accp[pp][k2] = acc[k2];
+          }
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp) {
+            const int ip = ib + pp;
+            if (ip >= cn) break;  // warp-uniform
+            const int* mm = meta + (i0 + ip) * kM;
+            const int j = mm[0];
+            const bool bad = mm[1] < 0;
+            const int rows = page_rows(sq.n, j);
+            const uint32_t sz0 = szp[pp][0], sz1 = szp[pp][1];
+            const float s0 = __half2float(__ushort_as_half((unsigned short)(sz0 & 0xFFFFu)));
+            const float z0 = __half2float(__ushort_as_half((unsigned short)(sz0 >> 16)));
+            const float s1 = __half2float(__ushort_as_half((unsigned short)(sz1 & 0xFFFFu)));
+            const float z1 = __half2float(__ushort_as_half((unsigned short)(sz1 >> 16)));
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+              const int hl = 2 * t + e2;
+              if (hl >= G) continue;
+              const int rk = mm[2 + hl];
+              if (rk < 0) continue;
+              const int bh = b * a.hq + kvh * G + hl;
+              const float qsum = e2 ? qsum1 : qsum0;
+              const size_t obase = (size_t)bh * a.cand_stride + (size_t)rk * kPage;
+#pragma unroll
+              for (int rr = 0; rr < 2; ++rr) {
+                const int row = gr + 8 * rr;
+                if (row >= rows) continue;
+                const float sv = rr ? s1 : s0, zv = rr ? z1 : z0;
+                const float lg =
+                    bad ? -INFINITY
+                        : (sv * (accp[pp][2 * rr + e2] * 512.f) + zv * qsum) * inv_sqrt_d;
+                a.logits[obase + row] = lg;
+                if (a.cand_tok) a.cand_tok[obase + row] = kPage * j + row;
+              }
+            }
+          }
+        }
+        __syncthreads();  // the pass's buffer is read before it is refilled
+        if (k + 2 < npass) issue(k + 2);
+      }
+    }
+  }
+  block_signal(counter(a, kCntEst, g));
+}
+
+// ------------------------------------------------------------------------------ prune
+__device__ float block_sum_fixed(float v, float* red) {
+  // sum over the block in a fixed order; every thread receives the total
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) t += red[w];
+  return t;
+}
+
+// Weight in fixed point (units of 2^-48; W <= 1): integer sums are exact up to the conversion and
+// do not depend on the order of the terms.
+__device__ __forceinline__ long long w_fixed(float w) { return __float2ll_rn(w * 281474976710656.f); }
+
+// Threshold from the live set {W >= L} (n <= kThreads values lw, fixed-point copies lq).  Every
+// test of the search at mid > L counts only live weights, and mass(W >= t) is a non-increasing
+// step function of t, so "mid <= L or mass(W >= mid) >= p" is the same test as "mid <= T" with
+// T = max(L, the largest live weight v with mass(W >= v) >= p).  T comes from all pairwise
+// comparisons at once (4, 2 or 1 threads per value); the search itself is then a scalar loop that
+// every thread runs (same inputs, same result).
+__device__ float top_p_from_live(const float* lw, const long long* lq, int n, float L, float p,
+                                 float eps, float top, float* red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long P = __double2ll_ru((double)p * 281474976710656.0);
+  const int tpv = n <= kThreads / 4 ? 4 : (n <= kThreads / 2 ? 2 : 1);
+  const int i = tid / tpv, part = tid % tpv;
+  long long mass = 0;
+  float vi = 0.f;
+  if (i < n) {
+    vi = lw[i];
+#pragma unroll 4
+    for (int j = part; j < n; j += tpv) mass += lw[j] >= vi ? lq[j] : 0ll;
+  }
+  if (tpv >= 2) mass += __shfl_xor_sync(0xffffffffu, mass, 1);
+  if (tpv >= 4) mass += __shfl_xor_sync(0xffffffffu, mass, 2);
+  float t = (i < n && mass >= P) ? vi : 0.f;
+  t = warp_max(t);
+  __syncthreads();
+  if (lane == 0) red[warp] = t;
+  __syncthreads();
+  float Tp = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) Tp = fmaxf(Tp, red[w]);
+  return bisect_scalar(top, fmaxf(L, Tp), eps);
+}
+
+// Exclusive prefix sum over the block of one 64-bit value per thread (thread order); *total gets
+// the block total.  `sh64` needs kWarps + 1 words.
+__device__ unsigned long long block_excl_u64(unsigned long long v, unsigned long long* sh64,
+                                             unsigned long long* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) sh64[warp] = x;
+  __syncthreads();
+  unsigned long long before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const unsigned long long t = sh64[w];
+    if (w < warp) before += t;
+    all += t;
+  }
+  if (total) *total = all;
+  return before + x - v;
+}
+
+// T for a large live set: the largest weight value v with mass(W >= v) >= p, masses exact in
+// fixed point (units of 2^-48).  The masses of the weights with float bit patterns in [lo, hi]
+// are summed into up to 2048 bins of equal key width, exactly and independently of the order of
+// the adds: each fixed-point weight is split into four 12-bit parts summed in 32-bit shared
+// atomics (no overflow for up to 2^20 weights; measured faster than one 64-bit atomic).  A descending scan finds the bin where the mass from
+// the top first reaches p, and T lies in it.  If that bin holds at most kThreads weights they are
+// ranked exactly (pairwise, as for the live set), a single-key bin is T itself, and otherwise the
+// bin is histogrammed again on its finer bits.  Returns 0 when even all counted weights fall
+// short of p.  Weights come from registers (row k * kThreads + tid) or from W (shared or global);
+// `mass` needs 4 * 2048 32-bit words, gv / gq kThreads entries each.
+constexpr int kHBins = 2048;
+template <int kR>
+__device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const float* W,
+                                   bool staged, int nc, uint32_t lo, uint32_t hi, long long P,
+                                   unsigned long long* mass, float* gv, long long* gq, Shared& sh,
+                                   unsigned long long* sh64, float* red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned long long above = 0;  // exact mass of the weights with keys above hi
+// BODY runs with `w` bound to each of this thread's weights (registers or W)
+#define TWL_FOR_EACH_WEIGHT(BODY)                                           \
+  do {                                                                      \
+    if (in_regs) {                                                          \
+      _Pragma("unroll") for (int k_ = 0; k_ < kR; ++k_) {                   \
+        if (k_ * kThreads + tid < nc) {                                     \
+          const float w = wr[k_];                                           \
+          BODY;                                                             \
+        }                                                                   \
+      }                                                                     \
+    } else {                                                                \
+      for (int i_ = tid; i_ < nc; i_ += kThreads) {                         \
+        const float w = staged ? W[i_] : __ldcg(W + i_);                    \
+        BODY;                                                               \
+      }                                                                     \
+    }                                                                       \
+  } while (0)
+  int n = 0;
+#pragma unroll 1
+  for (int level = 0; level < 4; ++level) {
+    const uint32_t width = hi - lo;
+    const int bits = 32 - __clz(width);
+    const int s = bits > 11 ? bits - 11 : 0;
+    const int nb = (int)(width >> s) + 1;
+    uint32_t* part = reinterpret_cast<uint32_t*>(mass);  // [4][kHBins] 12-bit part sums
+    for (int i = tid; i < 4 * kHBins; i += kThreads) part[i] = 0u;
+    __syncthreads();
+    TWL_FOR_EACH_WEIGHT({
+      const uint32_t u = __float_as_uint(w);
+      if (u >= lo && u <= hi) {
+        const int b = (int)((u - lo) >> s);
+        const unsigned long long q = (unsigned long long)w_fixed(w);
+        atomicAdd(&part[b], (uint32_t)(q & 0xFFFu));
+        atomicAdd(&part[kHBins + b], (uint32_t)((q >> 12) & 0xFFFu));
+        atomicAdd(&part[2 * kHBins + b], (uint32_t)((q >> 24) & 0xFFFu));
+        atomicAdd(&part[3 * kHBins + b], (uint32_t)(q >> 36));
+      }
+    });
+    __syncthreads();
+    // descending scan: thread t holds bins nb-1-4t .. nb-4-4t
+    unsigned long long mb[4], mine = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int b = nb - 1 - 4 * tid - e;
+      mb[e] = 0ull;
+      if (b >= 0)
+        mb[e] = (unsigned long long)part[b] + ((unsigned long long)part[kHBins + b] << 12) +
+                ((unsigned long long)part[2 * kHBins + b] << 24) +
+                ((unsigned long long)part[3 * kHBins + b] << 36);
+      mine += mb[e];
+    }
+    if (tid == 0) sh.state[3] = 0xFFFFFFFFu;
+    unsigned long long run = above + block_excl_u64(mine, sh64, nullptr);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int b = nb - 1 - 4 * tid - e;
+      if (b >= 0 && run < (unsigned long long)P && run + mb[e] >= (unsigned long long)P) {
+        sh.state[3] = (uint32_t)b;
+        sh64[kWarps] = run;  // mass above the crossing bin
+      }
+      run += mb[e];
+    }
+    __syncthreads();
+    const uint32_t bx = sh.state[3];
+    if (bx == 0xFFFFFFFFu) return 0.f;  // the counted weights never reach p
+    above = sh64[kWarps];
+    const uint32_t nlo = lo + (bx << s);
+    const uint64_t top_key = (uint64_t)nlo + ((1ull << s) - 1ull);
+    hi = top_key < (uint64_t)hi ? (uint32_t)top_key : hi;
+    lo = nlo;
+    if (lo == hi) return __uint_as_float(lo);  // one key value: T itself
+    int c = 0;
+    TWL_FOR_EACH_WEIGHT({
+      const uint32_t u = __float_as_uint(w);
+      c += (u >= lo && u <= hi) ? 1 : 0;
+    });
+    int pos = block_exclusive_scan(c, sh.scan, &n);
+    if (n <= kThreads) {  // gather the crossing bin's weights and rank them exactly
+      TWL_FOR_EACH_WEIGHT({
+        const uint32_t u = __float_as_uint(w);
+        if (u >= lo && u <= hi) {
+          gv[pos] = w;
+          gq[pos] = w_fixed(w);
+          ++pos;
+        }
+      });
+      break;
+    }
+  }
+  __syncthreads();
+  float t = 0.f;
+  if (tid < n && n <= kThreads) {
+    const float vi = gv[tid];
+    unsigned long long m = above;
+    for (int j = 0; j < n; ++j) m += gv[j] >= vi ? (unsigned long long)gq[j] : 0ull;
+    t = m >= (unsigned long long)P ? vi : 0.f;
+  }
+  t = warp_max(t);
+  __syncthreads();
+  if (lane == 0) red[warp] = t;
+  __syncthreads();
+  float T = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) T = fmaxf(T, red[w]);
+  __syncthreads();
+  return T;
+#undef TWL_FOR_EACH_WEIGHT
+}
+
+// Top-p of one q-head over its nc candidates.  W_i = exp(l_i - M) / S with M the largest logit
+// and S summed in a fixed order (per thread over its rows, then over the block).  Only weights
+// >= L = (1 - p) / (2 nc) can decide a test above L (the weights below L sum to less than
+// nc L = (1 - p) / 2, so the mass above any t <= L exceeds p): the threshold comes from that
+// live set when it fits one value per thread, else from the three-level search over every
+// weight.  Output: the kept-row bitmap of the head (bit i = W_i >= m) and the optional stats.
+__device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* smem,
+                           int smem_bytes) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = group_of(a, bh);
+  const bool ready = block_wait(a, sh, counter(a, kCntEst, g), (uint32_t)a.e_per);
+  const int nc = ready ? ldcg_i(a.ncand + bh) : 0;
+  float* red = reinterpret_cast<float*>(smem);                       // [kWarps][8]
+  uint32_t* top_u = reinterpret_cast<uint32_t*>(smem + 4 * kWarps * 8);
+  unsigned long long* sh64 = reinterpret_cast<unsigned long long*>(smem + 640);  // [kWarps + 1]
+  float* lw = reinterpret_cast<float*>(smem + 1024);                 // [kThreads] live W
+  int* li = reinterpret_cast<int*>(smem + 1024 + 4 * kThreads);      // [kThreads] their rows
+  long long* lq = reinterpret_cast<long long*>(smem + 1024 + 8 * kThreads);  // fixed point
+  unsigned char* tail = smem + 1024 + 16 * kThreads;
+  const int tail_off = (int)(tail - smem);
+  // weights staged in shared memory when they fit beside the histogram scratch of the large
+  // live-set search (5 * 2048 words)
+  const bool staged = tail_off + ((4 * nc + 127) & ~127) + 16 * kHBins <= smem_bytes;
+
+  const float p = a.p, eps = a.eps;
+  const bool use_bound = nc > 0 && p < 1.f && (1.f - p) >= 1e-3f;
+  const float L = use_bound ? (1.f - p) / (2.f * (float)nc) : 0.f;
+  float* lrow = a.logits + (size_t)bh * a.cand_stride;
+  float* wout = a.weights_out ? a.weights_out + (size_t)bh * a.cand_stride : nullptr;
+  if (tid == 0) *top_u = 0u;
+
+  // Weights: in registers (row i = k * kThreads + tid) when nc <= kThreads * kR, else in shared
+  // memory (or in place in the logits row when they do not fit).
+  constexpr int kR = 16;
+  const bool in_regs = nc <= kThreads * kR;
+  float wr[kR];
+  float* W = staged ? reinterpret_cast<float*>(tail) : lrow;
+  float mloc = -INFINITY;
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int i = k * kThreads + tid;
+      wr[k] = i < nc ? ldcg_f(lrow + i) : -INFINITY;
+      mloc = fmaxf(mloc, wr[k]);
+    }
+  } else {
+    constexpr int kB = 8;
+#pragma unroll 1
+    for (int base = 0; base < nc; base += kThreads * kB) {
+      float v[kB];
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int i = base + k * kThreads + tid;
+        v[k] = i < nc ? ldcg_f(lrow + i) : -INFINITY;
+      }
+#pragma unroll
+      for (int k = 0; k < kB; ++k) {
+        const int i = base + k * kThreads + tid;
+        if (i < nc) {
+          if (staged) W[i] = v[k];
+          mloc = fmaxf(mloc, v[k]);
+        }
+      }
+    }
+  }
+  TRACE_MARK(sh, 0);
+  const float M = block_max(mloc, red);
+  const bool empty = !(M > -INFINITY);
+  float esum = 0.f;
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int i = k * kThreads + tid;
+      const float e = (i < nc && !empty) ? __expf(wr[k] - M) : 0.f;
+      wr[k] = e;
+      esum += e;
+    }
+  } else {
+#pragma unroll 1
+    for (int i = tid; i < nc; i += kThreads) {
+      const float e = empty ? 0.f : __expf((staged ? W[i] : ldcg_f(lrow + i)) - M);
+      W[i] = e;
+      esum += e;
+    }
+  }
+  const float S = block_sum_fixed(esum, red);
+  const float inv = S > 0.f ? 1.f / S : 0.f;
+  TRACE_MARK(sh, 1);
+  // W = e / S, the largest weight, the live count
+  float top = 0.f;
+  int cntl = 0;
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int i = k * kThreads + tid;
+      wr[k] *= inv;
+      top = fmaxf(top, wr[k]);
+      cntl += (i < nc && wr[k] >= L) ? 1 : 0;
+    }
+  } else {
+#pragma unroll 1
+    for (int i = tid; i < nc; i += kThreads) {
+      const float w = (staged ? W[i] : ldcg_f(W + i)) * inv;
+      W[i] = w;
+      top = fmaxf(top, w);
+      cntl += w >= L ? 1 : 0;
+    }
+  }
+  top = warp_max(top);
+  if (lane == 0) atomicMax(top_u, __float_as_uint(top));  // W >= 0: the bits order as the values
+  int nlive = 0;
+  int pos = block_exclusive_scan(cntl, sh.scan, &nlive);  // its barriers also publish top_u
+  top = __uint_as_float(*top_u);
+  TRACE_MARK(sh, 2);
+  const bool from_live = use_bound && nlive <= kThreads;
+  if (from_live) {
+    if (in_regs) {
+#pragma unroll
+      for (int k = 0; k < kR; ++k) {
+        const int i = k * kThreads + tid;
+        if (i < nc && wr[k] >= L) {
+          lw[pos] = wr[k];
+          li[pos] = i;
+          lq[pos] = w_fixed(wr[k]);
+          ++pos;
+        }
+      }
+    } else {
+      for (int i = tid; i < nc; i += kThreads) {
+        const float w = staged ? W[i] : ldcg_f(W + i);
+        if (w >= L) {
+          lw[pos] = w;
+          li[pos] = i;
+          lq[pos] = w_fixed(w);
+          ++pos;
+        }
+      }
+    }
+  }
+  if (wout) {  // the weights output: every candidate
+    if (in_regs) {
+#pragma unroll
+      for (int k = 0; k < kR; ++k) {
+        const int i = k * kThreads + tid;
+        if (i < nc) wout[i] = wr[k];
+      }
+    } else {
+      for (int i = tid; i < nc; i += kThreads) wout[i] = staged ? W[i] : ldcg_f(W + i);
+    }
+  }
+  __syncthreads();  // the live set (or the weights) complete
+  float m;
+  if (nc == 0 || p >= 1.f) {
+    m = 0.f;  // keep every candidate
+  } else if (from_live) {
+    m = top_p_from_live(lw, lq, nlive, L, p, eps, top, red);
+  } else {
+    // the threshold from exact bin masses over the weights >= L (histogram scratch after the
+    // staged weights)
+    const long long P = __double2ll_ru((double)p * 281474976710656.0);
+    unsigned long long* hist =
+        reinterpret_cast<unsigned long long*>(tail + (staged ? ((4 * nc + 127) & ~127) : 0));
+    const float T = threshold_by_bins<kR>(wr, in_regs, W, staged, nc, __float_as_uint(L),
+                                          __float_as_uint(top), P, hist, lw, lq, sh,
+                                          sh64, red);
+    m = bisect_scalar(top, fmaxf(L, T), eps);
+  }
+  TRACE_MARK(sh, 3);
+  if (tid == 0) {
+    if (a.threshold) a.threshold[bh] = m;
+    if (a.cand_count) a.cand_count[bh] = nc;
+  }
+  // kept-row bitmap of this head: bit i = (W_i >= m)
+  uint32_t* kb_out = a.keptbits + (size_t)bh * a.kept_words;
+  const int kw = (nc + 31) >> 5;
+  uint32_t* kbits = reinterpret_cast<uint32_t*>(tail);
+  int cnt = 0;
+  if (from_live && m >= L && tail_off + 4 * kw <= smem_bytes) {
+    // every kept candidate is live
+    for (int w = tid; w < kw; w += kThreads) kbits[w] = 0u;
+    __syncthreads();
+    if (tid < nlive && lw[tid] >= m) atomicOr(&kbits[li[tid] >> 5], 1u << (li[tid] & 31));
+    __syncthreads();
+    for (int w = tid; w < kw; w += kThreads) {
+      const uint32_t x = kbits[w];
+      kb_out[w] = x;
+      cnt += __popc(x);
+    }
+  } else if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int i = k * kThreads + tid;
+      const bool keep = i < nc && wr[k] >= m;
+      const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0 && k * kThreads + 32 * warp < nc) kb_out[k * kWarps + warp] = bal;
+      cnt += keep;
+    }
+  } else {
+#pragma unroll 1
+    for (int base = 0; base < nc; base += kThreads) {
+      const int i = base + tid;
+      const bool keep = i < nc && (staged ? W[i] : ldcg_f(W + i)) >= m;
+      const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0 && base + 32 * warp < nc) kb_out[(base >> 5) + warp] = bal;
+      cnt += keep;
+    }
+  }
+  if (a.kept_count) {  // only when the caller asks for it
+    const float total = block_sum_fixed((float)cnt, red);
+    if (tid == 0) a.kept_count[bh] = (int)total;
+  }
+}
+
+// ------------------------------------------------------------------------------ kept tokens
+// Run by the CTA whose prune item completed its group: for every union page (ascending) the OR of
+// the 16-row pieces of the kept bitmaps of the heads that selected it, cut to the page's valid
+// rows; the kept rows are listed in ascending token order as K/V row indices (and token ids when
+// the caller asks for the union).
+template <int G>
+__device__ void build_kept(const Args& a, Shared& sh, int g) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
+  const Seq sq = load_seq(a.kv.seq_lens, b, a.kv.max_pages, a.flags, false);
+  const bool aborted = ld_acquire(a.sync + kAbort) != 0u;
+  const int n_pages = aborted ? 0 : sq.pages;
+  const size_t kbase = (size_t)g * kPage * a.kv.max_pages;
+  const size_t row0 = (size_t)b * a.hq + kvh * G;
+  TRACE_MARK(sh, 4);
+  // four logical pages per thread (j = base + tid + kThreads * r), every load in flight together:
+  // the heads' bitmap words and prefix counts (shared by 32 pages) and the page-table entry, then
+  // the kept-row words of the heads that selected the page; the list is in page order, so the
+  // scan is over (r, tid)
+  constexpr int kR = 4;
+  int* wsum = sh.scan;  // [kR][kWarps] per-warp totals
+  int carry = 0;
+#pragma unroll 1
+  for (int base = 0; base < n_pages; base += kR * kThreads) {
+    int ph[kR], rk[kR][G];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      const int j = base + tid + kThreads * r;
+      ph[r] = -1;
+#pragma unroll
+      for (int h = 0; h < G; ++h) rk[r][h] = -1;
+      if (j < n_pages) {
+        const int w = j >> 5, bit = j & 31;
+        uint32_t x[G];
+        int pre[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          x[h] = ldcg_u(a.selbits + (row0 + h) * a.sel_words + w);
+          pre[h] = ldcg_i(a.hpre + (row0 + h) * a.sel_words + w);
+        }
+        ph[r] = a.kv.page_table[(size_t)b * a.kv.max_pages + j];
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+          rk[r][h] = ((x[h] >> bit) & 1u) ? pre[h] + __popc(x[h] & ((1u << bit) - 1u)) : -1;
+      }
+    }
+    uint32_t mask[kR];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      uint32_t w[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        w[h] = rk[r][h] >= 0 ? ldcg_u(a.keptbits + (row0 + h) * a.kept_words + (rk[r][h] >> 1))
+                             : 0u;
+      uint32_t m = 0;
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        if (rk[r][h] >= 0) m |= (w[h] >> (16 * (rk[r][h] & 1))) & 0xFFFFu;
+      const int j = base + tid + kThreads * r;
+      if (m) {
+        const int rows = page_rows(sq.n, j);
+        m &= rows >= 16 ? 0xFFFFu : ((1u << rows) - 1u);
+        if (ph[r] < 0 || ph[r] >= a.kv.num_phys) {  // never attended; the estimate flagged it
+          ph[r] = -1;
+          m = 0u;
+        }
+      }
+      mask[r] = m;
+    }
+    TRACE_MARK(sh, 5);
+    int pos[kR], incl[kR];
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      int x = __popc(mask[r]);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      incl[r] = x;
+    }
+    __syncthreads();
+    if (lane == 31) {
+#pragma unroll
+      for (int r = 0; r < kR; ++r) wsum[r * kWarps + warp] = incl[r];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      int before = carry, all = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const int tt = wsum[r * kWarps + w];
+        if (w < warp) before += tt;
+        all += tt;
+      }
+      pos[r] = before + incl[r] - __popc(mask[r]);
+      carry += all;
+    }
+#pragma unroll
+    for (int r = 0; r < kR; ++r) {
+      const int j = base + tid + kThreads * r;
+      const uint32_t rbase = (uint32_t)(((size_t)(ph[r] < 0 ? 0 : ph[r]) * a.kv.hkv + kvh) * kPage);
+      uint32_t mm = mask[r];
+      int q = pos[r];
+      while (mm) {
+        const int row = __ffs(mm) - 1;
+        a.krow[kbase + q] = rbase + (uint32_t)row;
+        if (a.union_tok) a.union_tok[kbase + q] = kPage * j + row;
+        ++q;
+        mm &= mm - 1u;
+      }
+    }
+  }
+  // publish the group's kept tokens to the attention queue: chunks of up to kAttChunkTok tokens
+  // (one empty chunk when nothing is kept, so the merge still writes the outputs)
+  const int nch = carry > 0 ? (carry + kAttChunkTok - 1) / kAttChunkTok : 1;
+  if (tid == 0) {
+    if (a.union_count) a.union_count[g] = carry;
+    sh.total = (int)atomicAdd(a.sync + kQAlloc, (uint32_t)nch);
+  }
+  __syncthreads();
+  const int base = sh.total;
+  for (int c = tid; c < nch; c += kThreads) {
+    if (base + c >= a.q_cap) break;
+    int* e = a.qtab + 4 * (size_t)(base + c);
+    e[0] = g;
+    e[1] = (int)((long long)carry * c / nch);
+    e[2] = (int)((long long)carry * (c + 1) / nch);
+  }
+  if (tid == 0) {
+    a.cbase[2 * g] = base;
+    a.cbase[2 * g + 1] = nch;
+  }
+  __syncthreads();  // the chunk entries, counts and kept list before the valid flags
+  if (tid == 0) {
+    // one release fence for everything the block wrote (it observed all of it at the barrier),
+    // then plain stores of the flags
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    for (int c = 0; c < nch && base + c < a.q_cap; ++c)
+      asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(a.qvalid + base + c), "r"(1u)
+                   : "memory");
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(a.sync + kQGroups), "r"(1u)
+                 : "memory");
+  }
+  TRACE_MARK(sh, 6);
+}
+
+// ------------------------------------------------------------------------------ attention
+// Kept tokens [t0, t1) of group g (one chunk of the attention work list).  Their K/V row indices
+// are staged in passes of up to kAttIdx; the rows (256 B of K and of V each) are copied with
+// 16-byte cp.async in passes of kAttPass tokens, two in flight, each row's 16-byte pieces XOR-
+// swizzled by the row number so that ldmatrix reads are free of bank conflicts.
+// The contraction runs on the tensor cores (mma.m16n8k16, fp16 in, fp32 accumulate).  S = Q K^T
+// takes the group's heads as the M rows (padded to 16 with zeros) and 8 tokens as N; its output
+// fragments are exactly the B operand of O^T += V^T P^T, which takes 16 channels as M, the tile's
+// 16 tokens as K and the heads as N, so no fragment is moved between the two products.  Warp w
+// takes the 16-token tile w / 2 of a pass for QK^T (both warps of a pair compute it) and the 64
+// channels (w % 2) of P.V.  P is split into an fp16 head and an fp16 tail (p - head), two
+// products, so its rounding stays near 2^-22 of the weights.  Each warp keeps its own running
+// (max, sum, o) per head; the warps' states are merged at the end into the chunk's partial.
+constexpr int kAttPass = 128;
+constexpr int kAttIdx = 3840;  // a multiple of kAttPass
+
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int G>
+__device__ void attend_chunk(const Args& a, Shared& sh, int g, int t0, int t1, int slot,
+                             unsigned char* smem) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gr = lane >> 2, t = lane & 3;  // mma fragment row / column pair
+  const int tile = warp >> 1, hh = warp & 1;
+  const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
+  uint32_t* idx = reinterpret_cast<uint32_t*>(smem);
+  unsigned char* buf = smem + 4 * kAttIdx;
+  const uint32_t* klist = a.krow + (size_t)g * kPage * a.kv.max_pages;
+  // A fragments of the queries (rows = heads; rows >= G and the upper 8 rows are zero)
+  uint32_t qa[8][2];
+  {
+    const bool head_ok = gr < G;
+    const uint16_t* qh = a.q + ((size_t)b * a.hq + kvh * G + (head_ok ? gr : 0)) * kHeadDim;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qa[ks][0] = head_ok ? __ldg(reinterpret_cast<const uint32_t*>(qh + 16 * ks + 2 * t)) : 0u;
+      qa[ks][1] = head_ok ? __ldg(reinterpret_cast<const uint32_t*>(qh + 16 * ks + 8 + 2 * t)) : 0u;
+    }
+  }
+  float M = -INFINITY, L = 0.f;  // softmax state of head gr (the QK^T row of this lane)
+  float ot[4][4];                // O^T: channels 64 hh + 16 mt + (gr, gr + 8), heads (2t, 2t+1)
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) ot[mt][c] = 0.f;
+  const float sc_scale = a.sm_scale;
+#pragma unroll 1
+  for (int m0 = t0; m0 < t1; m0 += kAttIdx) {
+    const int n = min(kAttIdx, t1 - m0);
+    for (int i = tid; i < n; i += kThreads) idx[i] = ldcg_u(klist + m0 + i);
+    __syncthreads();
+    TRACE_MARK(sh, 0);
+    const int npass = (n + kAttPass - 1) / kAttPass;
+    auto issue = [&](int k) {
+      unsigned char* kb = buf + (k & 1) * kAttPass * 512;
+      unsigned char* vb = kb + kAttPass * 256;
+      const int i0 = k * kAttPass, cn = min(kAttPass, n - i0);
+      for (int q = tid; q < 32 * kAttPass; q += kThreads) {
+        const int i = q >> 5, part = q & 31;
+        const uint32_t r = i < cn ? idx[i0 + i] : 0xFFFFFFFFu;
+        const bool okr = r != 0xFFFFFFFFu;
+        const size_t off = okr ? (size_t)r * kHeadDim : 0;
+        // a slot without a row reads zeros (its scores are masked; its V must not be inf)
+        if (part < 16)
+          cp_async16(kb + 256 * i + 16 * (part ^ (i & 7)), a.kv.k + off + 8 * part, okr);
+        else
+          cp_async16(vb + 256 * i + 16 * ((part - 16) ^ (i & 7)), a.kv.v + off + 8 * (part - 16),
+                     okr);
+      }
+      cp_async_commit();
+    };
+    issue(0);
+    if (npass > 1) issue(1);
+#pragma unroll 1
+    for (int k = 0; k < npass; ++k) {
+      if (k + 1 < npass) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+      else cp_async_wait_all();
+      __syncthreads();
+      TRACE_MARK(sh, 1);
+      const unsigned char* kb = buf + (k & 1) * kAttPass * 512;
+      const unsigned char* vb = kb + kAttPass * 256;
+      const int i0 = k * kAttPass, cn = min(kAttPass, n - i0);
+      const int tok0 = 16 * tile;  // this warp's tile
+      if (tok0 < cn) {             // warp-uniform
+        // S = Q K^T for the tile's two 8-token halves (rows = heads)
+        float s[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
+        const int mrow = lane & 7, mat = lane >> 3;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const int tk = tok0 + mrow + 8 * (mat >> 1), ch = 2 * ks + (mat & 1);
+          uint32_t kf[4];
+          ldsm_x4(kf, saddr(kb + 256 * tk + 16 * (ch ^ (tk & 7))));
+          const uint32_t av[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
+          mma_16816(s[0], av, kf[0], kf[1]);
+          mma_16816(s[1], av, kf[2], kf[3]);
+        }
+        // mask, scale, online softmax of head gr over the tile's 16 tokens
+        float pv[2][2];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int tk = tok0 + 8 * nt + 2 * t + c;
+            const bool valid = tk < cn && idx[i0 + (tk < cn ? tk : 0)] != 0xFFFFFFFFu;
+            pv[nt][c] = valid ? s[nt][c] * sc_scale : -INFINITY;
+            mx = fmaxf(mx, pv[nt][c]);
+          }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float nm = fmaxf(M, mx);
+        float scale = 1.f;
+        if (nm > -INFINITY) {  // the same in the four lanes of a row
+          scale = M > -INFINITY ? __expf(M - nm) : 0.f;
+          float rs = 0.f;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              pv[nt][c] = __expf(pv[nt][c] - nm);
+              rs += pv[nt][c];
+            }
+          rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+          rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+          L = L * scale + rs;
+          M = nm;
+        } else {
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) pv[nt][c] = 0.f;
+        }
+        // rescale O^T: this lane's columns are heads 2t and 2t+1, whose factors are held by the
+        // lanes of rows 2t (lane 8t) and 2t+1 (lane 8t+4)
+        const float f0 = __shfl_sync(0xffffffffu, scale, 8 * t);
+        const float f1 = __shfl_sync(0xffffffffu, scale, 8 * t + 4);
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          ot[mt][0] *= f0;
+          ot[mt][1] *= f1;
+          ot[mt][2] *= f0;
+          ot[mt][3] *= f1;
+        }
+        // P^T as the B operand (k = the tile's 16 tokens, n = head gr): fp16 head and tail
+        const uint32_t bh0 = pack_f16x2(pv[0][0], pv[0][1]);
+        const uint32_t bh1 = pack_f16x2(pv[1][0], pv[1][1]);
+        const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&bh0));
+        const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&bh1));
+        const uint32_t bl0 = pack_f16x2(pv[0][0] - h0.x, pv[0][1] - h0.y);
+        const uint32_t bl1 = pack_f16x2(pv[1][0] - h1.x, pv[1][1] - h1.y);
+        // O^T += V^T P^T over this warp's 64 channels (four 16-channel M tiles; A from
+        // ldmatrix.trans of the V rows)
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          const int tk = tok0 + mrow + 8 * (mat >> 1);
+          const int ch = 8 * hh + 2 * mt + (mat & 1);
+          uint32_t va[4];
+          ldsm_x4_t(va, saddr(vb + 256 * tk + 16 * (ch ^ (tk & 7))));
+          mma_16816(ot[mt], va, bh0, bh1);
+          mma_16816(ot[mt], va, bl0, bl1);
+        }
+      }
+      __syncthreads();  // the pass's buffer is read before it is refilled
+      if (k + 2 < npass) issue(k + 2);
+    }
+  }
+  TRACE_MARK(sh, 2);
+  // merge the warps' states: smem [kWarps][16] (max, sum) and [kWarps][G][64] o
+  float* wm = reinterpret_cast<float*>(buf);
+  float* wl = wm + kWarps * 16;
+  float* wo = wl + kWarps * 16;
+  if (t == 0) {
+    wm[warp * 16 + gr] = M;
+    wl[warp * 16 + gr] = L;
+  }
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+    const int c0 = 16 * mt + gr;  // channel within the warp's half
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * t + e;
+      if (h < G) {
+        wo[((size_t)warp * G + h) * 64 + c0] = ot[mt][e];
+        wo[((size_t)warp * G + h) * 64 + c0 + 8] = ot[mt][2 + e];
+      }
+    }
+  }
+  __syncthreads();
+  float* part = a.part + (size_t)slot * G * (kHeadDim + 2);
+  for (int i = tid; i < G * kHeadDim; i += kThreads) {
+    const int h = i / kHeadDim, d = i - h * kHeadDim;
+    const int half = d >> 6, dd = d & 63;
+    float mxw = -INFINITY;
+#pragma unroll
+    for (int tl = 0; tl < kWarps / 2; ++tl) mxw = fmaxf(mxw, wm[(2 * tl + half) * 16 + h]);
+    float ov = 0.f, lv = 0.f;
+    if (mxw > -INFINITY) {
+#pragma unroll
+      for (int tl = 0; tl < kWarps / 2; ++tl) {
+        const int w = 2 * tl + half;
+        const float mw = wm[w * 16 + h];
+        if (!(mw > -INFINITY)) continue;
+        const float f = __expf(mw - mxw);
+        ov = fmaf(f, wo[((size_t)w * G + h) * 64 + dd], ov);
+        lv = fmaf(f, wl[w * 16 + h], lv);
+      }
+    }
+    part[h * (kHeadDim + 2) + 2 + d] = ov;
+    if (d == 0) {
+      part[h * (kHeadDim + 2) + 0] = mxw;
+      part[h * (kHeadDim + 2) + 1] = lv;
+    }
+  }
+}
+
+// Run by the CTA whose chunk completed its group: log-sum-exp merge of the group's chunk
+// partials, in chunk order -> o, lse of every head (o = 0, lse = -inf when nothing was kept).
+template <int G>
+__device__ void merge_group(const Args& a, int g, int c0, int nch) {
+  const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
+  for (int i = threadIdx.x; i < G * kHeadDim; i += kThreads) {
+    const int h = i / kHeadDim, d = i - h * kHeadDim;
+    const float* base = a.part + (size_t)c0 * G * (kHeadDim + 2) + h * (kHeadDim + 2);
+    const size_t stride = (size_t)G * (kHeadDim + 2);
+    float Mx = -INFINITY;
+    for (int ai = 0; ai < nch; ++ai) {
+      const float* pp = base + ai * stride;
+      if (ldcg_f(pp + 1) > 0.f) Mx = fmaxf(Mx, ldcg_f(pp));
+    }
+    float o = 0.f, l = 0.f;
+    if (Mx > -INFINITY) {
+      for (int ai = 0; ai < nch; ++ai) {
+        const float* pp = base + ai * stride;
+        const float la = ldcg_f(pp + 1);
+        if (!(la > 0.f)) continue;
+        const float wgt = __expf(ldcg_f(pp) - Mx);
+        o = fmaf(wgt, ldcg_f(pp + 2 + d), o);
+        l = fmaf(wgt, la, l);
+      }
+    }
+    const size_t bh = (size_t)b * a.hq + kvh * G + h;
+    const bool any = l > 0.f;
+    a.o[bh * kHeadDim + d] = any ? o / l : 0.f;
+    if (d == 0) a.lse[bh] = any ? Mx + __logf(l) : -INFINITY;
+  }
+}
+
+// One worker of the flattened attention work list ([Notes] "Key designs", load balancing: the
+// heads' kept tokens differ ~50x, so they are cut into equal chunks that any CTA takes): take the
+// next chunk number, wait until it is published (or until every group has published and the
+// number is past the end), attend over it, and merge the group when its last chunk is done.
+template <int G>
+__device__ void attend_worker(const Args& a, Shared& sh, unsigned char* smem) {
+#pragma unroll 1
+  for (;;) {
+    if (threadIdx.x == 0) {
+      const int c = (int)atomicAdd(a.sync + kQNext, 1u);
+      int got = -1;
+      uint32_t it = 0;
+      for (;;) {
+        if (c < a.q_cap && ld_acquire(a.qvalid + c) != 0u) {
+          got = c;
+          break;
+        }
+        if (ld_acquire(a.sync + kQGroups) >= (uint32_t)a.groups &&
+            (uint32_t)c >= ld_acquire(a.sync + kQAlloc))
+          break;  // every group published and this number is past the end
+        if ((++it & 31u) == 0u) {
+          if (ld_acquire(a.sync + kAbort) != 0u) break;
+          if (it >= kSpinLimit) {
+            raise_flag(a.flags, TWL_FLAG_TIMEOUT);
+            atomicExch(a.sync + kAbort, 1u);
+            break;
+          }
+        }
+        __nanosleep(64);
+      }
+      sh.flag = got;
+#ifdef TWL_STEP_TRACE
+      sh.t_ready = now_ns();
+#endif
+    }
+    __syncthreads();
+    const int c = sh.flag;
+    __syncthreads();
+    if (c < 0) break;
+    const int* e = a.qtab + 4 * (size_t)c;
+    const int g = ldcg_i(e), t0 = ldcg_i(e + 1), t1 = ldcg_i(e + 2);
+    const int c0 = ldcg_i(a.cbase + 2 * g), nch = ldcg_i(a.cbase + 2 * g + 1);
+    attend_chunk<G>(a, sh, g, t0, t1, c, smem);
+    if (block_signal_last(sh, counter(a, kCntAttend, g), (uint32_t)nch)) {
+      TRACE_MARK(sh, 5);
+      merge_group<G>(a, g, c0, nch);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------ the kernel
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1) k_step(const __grid_constant__ Args a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ Shared sh;
+  // wait for the previous grid in the stream (launched programmatically), then let the next one
+  // be scheduled: it will in turn wait for this grid to complete before touching memory
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
+  int idx = blockIdx.x;
+#pragma unroll 1
+  while (idx < a.n_items) {
+#ifdef TWL_STEP_TRACE
+    unsigned long long t_start = 0, c_start = 0;
+    if (threadIdx.x == 0) {
+      t_start = now_ns();
+      c_start = clock64();
+      sh.t_ready = 0;
+      for (int m = 0; m < 7; ++m) sh.marks[m] = 0;
+    }
+#endif
+    int phase = -1, g = 0, sub = 0;
+#pragma unroll 1
+    for (int s = 0; s < a.nseg; ++s) {
+      const Segment& sg = a.seg[s];
+      const int cnt = (sg.g1 - sg.g0) * sg.per;
+      if (idx < sg.first + cnt) {
+        const int l = idx - sg.first;
+        phase = sg.phase;
+        g = sg.g0 + l / sg.per;
+        sub = l - (l / sg.per) * sg.per;
+        break;
+      }
+    }
+    const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
+    switch (phase) {
+      case kScore:
+        item_score<G>(a, sh, g, sub, smem);
+        break;
+      case kTopK:
+        item_topk<G>(a, sh, b * a.hq + kvh * G + sub, smem, a.smem_bytes);
+        block_signal(counter(a, kCntTopK, g));
+        break;
+      case kEst:
+        item_estimate<G>(a, sh, g, sub, smem);
+        break;
+      case kPrune:
+        item_prune(a, sh, b * a.hq + kvh * G + sub, smem, a.smem_bytes);
+        if (block_signal_last(sh, counter(a, kCntPrune, g), (uint32_t)G)) build_kept<G>(a, sh, g);
+        break;
+      case kAttend:
+        attend_worker<G>(a, sh, smem);
+        break;
+      default:
+        break;
+    }
+#ifdef TWL_STEP_TRACE
+    __syncthreads();
+    if (threadIdx.x == 0 && a.trace) {
+      unsigned long long* tr = a.trace + 14 * (size_t)idx;
+      tr[0] = (unsigned long long)idx;
+      tr[1] = blockIdx.x;
+      tr[2] = t_start;
+      tr[3] = sh.t_ready;
+      for (int m = 0; m < 7; ++m) tr[4 + m] = sh.marks[m];
+      tr[11] = now_ns();
+      tr[12] = c_start;
+      tr[13] = clock64();
+    }
+#endif
+    // the next free item, taken only now: a CTA never holds an item it cannot start
+    if (threadIdx.x == 0) sh.next = (int)(gridDim.x + atomicAdd(a.sync + kNext, 1u));
+    __syncthreads();
+    idx = sh.next;
+    __syncthreads();
+  }
+  // leaving: the last CTA out clears the synchronisation words for the next launch
+  __syncthreads();
+  if (threadIdx.x == 0) sh.flag = atom_acq_rel_add(a.sync + kExit, 1u) + 1u == gridDim.x;
+  __syncthreads();
+  if (sh.flag) {
+    const int used = min(a.q_cap, (int)ldcg_u(a.sync + kQAlloc));
+    for (int i = threadIdx.x; i < used; i += kThreads) a.qvalid[i] = 0u;
+    const int nwords = kSyncHead + kCounters * a.groups;
+    for (int i = threadIdx.x; i < nwords; i += kThreads) a.sync[i] = 0u;
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------- host side
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+int round32(int x) { return (x + 31) & ~31; }
+
+template <int G>
+const void* kernel_of() {
+  return reinterpret_cast<const void*>(&k_step<G>);
+}
+const void* kernel_for(int g) {
+  switch (g) {
+    case 1: return kernel_of<1>();
+    case 2: return kernel_of<2>();
+    case 4: return kernel_of<4>();
+    case 8: return kernel_of<8>();
+    default: return nullptr;
+  }
+}
+
+// Shared memory each item kind needs (bytes).
+int smem_need(int g, int max_pages, int max_budget, int s_chunk) {
+  const int sw = round32((max_pages + 31) / 32);
+  const int topk = 4 * sw + 4 * round32(max_pages) + 4 * 4096 + 8 * 64 + 64;
+  const int prune = 1024 + 16 * kThreads + 16 * kHBins;  // + staged weights when they fit
+  const int score = ((4 * s_chunk + 127) & ~127) + 2 * kScorePass * 512;
+  const int est_kw = kEstMeta / 32 + 1;
+  const int est = ((4 * ((2 + g) * kEstMeta + (2 * g + 2) * est_kw + 1) + 127) & ~127) +
+                  2 * kEstPass * 1088;
+  const int att = 4 * kAttIdx + 2 * kAttPass * 512;
+  const int att_merge = 4 * kAttIdx + 4 * (2 * kWarps * 16 + kWarps * g * 64);
+  int need = topk;
+  for (int x : {prune, score, est, att, att_merge}) need = need > x ? need : x;
+  return need;
+}
+
+// Dynamic shared memory per CTA: everything the device grants one block beyond the static part
+// (the estimate's stages and the staged weights use what the minimum leaves).
+int smem_avail(int g) {
+  int dev = 0, optin = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    optin = 227 * 1024;
+  cudaFuncAttributes fa{};
+  const void* k = kernel_for(g);
+  size_t stat = 1024;
+  if (k && cudaFuncGetAttributes(&fa, k) == cudaSuccess) stat = fa.sharedSizeBytes;
+  cudaGetLastError();
+  return (int)((size_t)optin - stat - 1024) & ~127;
+}
+
+}  // namespace
+
+Plan plan(int batch, int hq, int hkv, int max_pages, int max_budget) {
+  Plan pl{};
+  const int g = hq / hkv;
+  const int groups = batch * hkv;
+  pl.sel_words = (max_pages + 31) / 32;
+  pl.cand_stride = kPage * max_budget;
+  pl.kept_words = (pl.cand_stride + 31) / 32;
+  const int sms = num_sms();
+  pl.grid = sms;  // one 512-thread CTA per SM, every CTA resident
+  pl.smem_bytes = smem_avail(g);
+  // work list: score chunks so the pages fill every CTA (one wave when the groups are few and
+  // short, about four otherwise); estimate and attention slices likewise per group
+  const long long total_pages = (long long)groups * max_pages;
+  if (groups <= sms / 2 && total_pages <= (long long)sms * 512) {
+    pl.s_per = sms / groups;
+  } else {
+    const long long chunk = (total_pages + 4ll * sms - 1) / (4ll * sms);
+    pl.s_per = (int)((max_pages + chunk - 1) / chunk);
+  }
+  pl.s_per = pl.s_per < 1 ? 1 : (pl.s_per > max_pages ? max_pages : pl.s_per);
+  if ((max_pages + pl.s_per - 1) / pl.s_per > 4096) pl.s_per = (max_pages + 4095) / 4096;
+  pl.s_chunk = (max_pages + pl.s_per - 1) / pl.s_per;
+  pl.s_per = (max_pages + pl.s_chunk - 1) / pl.s_chunk;
+  pl.ok = smem_need(g, max_pages, max_budget, pl.s_chunk) <= pl.smem_bytes;
+  const long long est_pages = (long long)groups * (max_pages < 2 * max_budget ? max_pages
+                                                                             : 2 * max_budget);
+  long long waves = (est_pages + (long long)sms * 128 - 1) / ((long long)sms * 128);
+  waves = waves < 1 ? 1 : (waves > 4 ? 4 : waves);
+  if (waves == 1 && groups <= sms) pl.e_per = sms / groups;
+  else pl.e_per = (int)((waves * sms + groups - 1) / groups);
+  pl.e_per = pl.e_per < 1 ? 1 : (pl.e_per > 64 ? 64 : pl.e_per);
+  pl.e_chunk = (max_pages + pl.e_per - 1) / pl.e_per;  // logical pages per estimate item
+  pl.e_per = (max_pages + pl.e_chunk - 1) / pl.e_chunk;
+  // attention chunks: at most one per kAttChunkTok kept tokens of each group plus one, and the
+  // numbers the workers take past the end
+  pl.q_cap = groups * (1 + (kPage * max_pages + kAttChunkTok - 1) / kAttChunkTok) + sms + 32;
+  return pl;
+}
+
+namespace {
+struct Layout {
+  size_t sync, keys, selbits, ncand, hpre, logits, keptbits, krow,
+      qtab, qvalid, cbase, part, trace, total;
+};
+Layout layout(const Plan& pl, int batch, int hq, int hkv, int max_pages) {
+  const int g = hq / hkv;
+  const size_t bh = (size_t)batch * hq, groups = (size_t)batch * hkv;
+  Layout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align_up(bytes);
+    return o;
+  };
+#ifdef TWL_STEP_TRACE
+  L.trace = take(8 * 14 * (size_t)(groups * (pl.s_per + 2 * g + pl.e_per) + pl.grid));
+#endif
+  L.sync = take(4 * (kSyncHead + kCounters * groups));
+  L.keys = take(4 * bh * max_pages);
+  L.selbits = take(4 * bh * pl.sel_words);
+  L.ncand = take(4 * bh);
+  L.hpre = take(4 * bh * pl.sel_words);
+  L.logits = take(4 * bh * pl.cand_stride);
+  L.keptbits = take(4 * bh * pl.kept_words);
+  L.krow = take(4 * groups * kPage * (size_t)max_pages);
+  L.qtab = take(16 * (size_t)pl.q_cap);
+  L.qvalid = take(4 * (size_t)pl.q_cap);
+  L.cbase = take(8 * groups);
+  L.part = take(4 * (size_t)pl.q_cap * g * (kHeadDim + 2));
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+size_t workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_budget) {
+  const Plan pl = plan(batch, hq, hkv, max_pages, max_budget);
+  return layout(pl, batch, hq, hkv, max_pages).total;
+}
+
+void carve(Args& a, char* ws, const Plan& pl, int batch, int hq, int hkv, int max_pages) {
+  const Layout L = layout(pl, batch, hq, hkv, max_pages);
+  a.sync = reinterpret_cast<uint32_t*>(ws + L.sync);
+  a.keys = reinterpret_cast<uint32_t*>(ws + L.keys);
+  a.selbits = reinterpret_cast<uint32_t*>(ws + L.selbits);
+  a.ncand = reinterpret_cast<int*>(ws + L.ncand);
+  a.hpre = reinterpret_cast<int*>(ws + L.hpre);
+  a.logits = reinterpret_cast<float*>(ws + L.logits);
+  a.keptbits = reinterpret_cast<uint32_t*>(ws + L.keptbits);
+  a.krow = reinterpret_cast<uint32_t*>(ws + L.krow);
+  a.qtab = reinterpret_cast<int*>(ws + L.qtab);
+  a.qvalid = reinterpret_cast<uint32_t*>(ws + L.qvalid);
+  a.cbase = reinterpret_cast<int*>(ws + L.cbase);
+  a.part = reinterpret_cast<float*>(ws + L.part);
+#ifdef TWL_STEP_TRACE
+  a.trace = reinterpret_cast<unsigned long long*>(ws + L.trace);
+#endif
+  const int g = hq / hkv;
+  a.g = g;
+  a.groups = batch * hkv;
+  a.sel_words = pl.sel_words;
+  a.cand_stride = pl.cand_stride;
+  a.kept_words = pl.kept_words;
+  a.s_per = pl.s_per;
+  a.s_chunk = pl.s_chunk;
+  a.e_per = pl.e_per;
+  a.e_chunk = pl.e_chunk;
+  a.q_cap = pl.q_cap;
+  a.smem_bytes = pl.smem_bytes;
+  // the work list, kind by kind (every item depends only on items of earlier kinds)
+  // the work list, kind by kind (every item depends only on items of earlier kinds); the last
+  // kind is one attention worker per CTA
+  const int per[4] = {pl.s_per, g, pl.e_per, g};
+  int first = 0;
+  a.nseg = 0;
+  for (int ph = kScore; ph <= kPrune; ++ph) {
+    Segment& s = a.seg[a.nseg++];
+    s.phase = ph;
+    s.g0 = 0;
+    s.g1 = a.groups;
+    s.per = per[ph];
+    s.first = first;
+    first += a.groups * per[ph];
+  }
+  Segment& w = a.seg[a.nseg++];
+  w.phase = kAttend;
+  w.g0 = 0;
+  w.g1 = 1;
+  w.per = pl.grid;
+  w.first = first;
+  a.n_items = first + pl.grid;
+}
+
+cudaError_t launch(const Args& a, const Plan& pl, cudaStream_t s) {
+  const void* k = kernel_for(a.g);
+  if (!k) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       pl.smem_bytes);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, pl.smem_bytes);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;  // the grid could not all be resident
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)pl.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)pl.smem_bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  // programmatic dependent launch: this grid may be scheduled while the previous kernel in the
+  // stream finishes; it waits for that kernel (griddepcontrol.wait) before touching memory
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  void* params[] = {const_cast<Args*>(&a)};
+  e = cudaLaunchKernelExC(&cfg, k, params);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace step
+}  // namespace twl

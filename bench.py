@@ -58,12 +58,16 @@ WORKLOADS = {
     "c6": ("GQA decode layer, batch 64, 32 q-heads / 8 kv-heads, head_dim 128, 8192-token "
            "context, pages randomly permuted, 16-token pages, Quest budget 1/4, INT4 K, "
            "p = 0.85, eps = 1e-6, seed 0", dict(batch=64, ctx=8192)),
+    "diffuse": ("GQA decode layer with diffuse heads only, batch 1, 32 q-heads / 8 kv-heads, "
+                "head_dim 128, 32768-token context, no heavy tokens (sinks kept), logit "
+                "temperature log-uniform in [2, 8], 16-token pages, Quest budget 1/4, INT4 K, "
+                "p = 0.85, eps = 1e-6, seed 0", dict(batch=1, ctx=32768)),
 }
 
 
 def make_workload(name):
     return {"c2": synth.config2, "c3": synth.config3, "c4": synth.config4,
-            "c6": synth.config6}[name]()
+            "c6": synth.config6, "diffuse": synth.config_diffuse}[name]()
 
 
 def workload_config(name="c2"):
@@ -107,8 +111,7 @@ def algorithmic_bytes(page_table, seq_lens, num_q_heads, num_kv_heads, sel_pages
 
 
 KERNEL_SOURCES = {
-    "decode_step": ["twl_fused.cu", "twl_fused_256.cu", "twl_fused.h", "twl_common.cuh",
-                    "twl_kernels.h"],
+    "decode_step": ["twl_step.cu", "twl_step.h", "twl_common.cuh", "twl_kernels.h"],
     "prune_rows": ["twl_prune_rows.cu", "twl_prune_rows64.cu", "twl_common.cuh", "twl_kernels.h"],
 }
 
@@ -242,6 +245,53 @@ def oracle_sample(wl, groups):
     for sub, bounds, q4, sz in subs:
         O.decode_step(sub, bounds=bounds, k_int4=q4, k_sz=sz)
     return time.perf_counter() - t0
+
+
+def _oracle_worker(name, groups, reps, barrier, results):
+    """One process of the all-core CPU baseline: build the workload (seeded, identical in every
+    process), prepare its groups' bounds / INT4 untimed, wait for the others, then time `reps`
+    passes of the oracle's decode path over its groups."""
+    with cpu_threads_guard():
+        from oracle import twl_oracle as O
+        from tests.twl_checks import group_workload
+        wl = make_workload(name)
+        subs = []
+        for b, kvh in groups:
+            sub = group_workload(wl, b, kvh)
+            subs.append((sub, O.page_bounds(sub.k, sub.page_table, sub.seq_lens),
+                         *O.quantize_k(sub.k, sub.page_table, sub.seq_lens)))
+        barrier.wait()
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            for sub, bounds, q4, sz in subs:
+                O.decode_step(sub, bounds=bounds, k_int4=q4, k_sz=sz)
+        results.put((time.perf_counter() - t0) / reps)
+
+
+def oracle_all_cores(name, n_groups_total, batch, hkv, max_groups=None, reps=3):
+    """The oracle's decode path split over the host's cores: one spawned process per core (BLAS
+    at one thread each), each with a fixed share of the layer's (sequence, kv-head) groups, all
+    started together; a layer-step takes as long as the slowest process.  At most `max_groups`
+    groups are timed (the per-layer time is scaled by n_groups_total / timed groups).  Returns
+    (seconds per layer-step, processes used, groups timed)."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")      # never fork a process that has touched the GPU
+    all_groups = [(b, kvh) for b in range(batch) for kvh in range(hkv)]
+    if max_groups is not None:
+        all_groups = all_groups[:max_groups]
+    nproc = max(1, min(os.cpu_count() or 1, len(all_groups)))
+    shares = [all_groups[i::nproc] for i in range(nproc)]
+    barrier = ctx.Barrier(nproc)
+    results = ctx.Queue()
+    procs = [ctx.Process(target=_oracle_worker, args=(name, sh_, reps, barrier, results))
+             for sh_ in shares]
+    for p_ in procs:
+        p_.start()
+    times = [results.get() for _ in procs]
+    for p_ in procs:
+        p_.join()
+    per_layer = max(times) * n_groups_total / len(all_groups)
+    return per_layer, nproc, len(all_groups)
 
 
 def cpu_threads_guard():
@@ -481,11 +531,21 @@ def run_ours(args, world, rank, local):
             t = oracle_sample(wl, wl_groups)
         n_groups = wl.batch * wl.num_kv_heads
         per_layer = t * n_groups / len(wl_groups)
-        out["cpu_baseline"] = {
-            "value": 1.0 / per_layer, "unit": UNIT, "cores": 1, "kind": "oracle",
+        single = {
+            "value": 1.0 / per_layer, "unit": UNIT, "cores": 1,
             "sample": f"oracle decode path (numpy, fp64) on 1 of the layer's {n_groups} "
                       f"(sequence, kv-head) groups, scaled x{n_groups} to one layer-step; "
                       f"bounds/INT4 prepared untimed"}
+        cap = 16 if args.workload in ("c2", "diffuse") else 8
+        per_all, nproc, timed = oracle_all_cores(args.workload, n_groups, wl.batch,
+                                                 wl.num_kv_heads, max_groups=cap)
+        out["cpu_baseline"] = {
+            "value": 1.0 / per_all, "unit": UNIT, "cores": nproc, "kind": "oracle",
+            "sample": f"oracle decode path (numpy, fp64) over {timed} of the layer's {n_groups} "
+                      f"(sequence, kv-head) groups split across {nproc} spawned processes (BLAS "
+                      f"one thread each, common start), scaled x{n_groups / timed:g} to one "
+                      f"layer-step; bounds/INT4 prepared untimed",
+            "single_core": single}
     del graph
     return out
 
@@ -1135,7 +1195,7 @@ def main():
     ap.add_argument("--layers", type=int, default=None,
                     help="layer caches per step (default 32 for c2 and append, 4 for c3 / c4)")
     ap.add_argument("--workload", default="c2",
-                    choices=["c2", "c3", "c4", "c6", "append", "bits", "c5"],
+                    choices=["c2", "c3", "c4", "c6", "diffuse", "append", "bits", "c5"],
                     help="c2 is the headline; c3 / c4 / c6, the append step, the estimator bit "
                          "widths and the standalone pruner (c5) are extra reports")
     ap.add_argument("--p-sweep", action="store_true",

@@ -522,10 +522,19 @@ def test_decode_step_dense_limit():
         check_attention(o[bb, h], lse[bb, h], o_or, lse_or, f"dense h{h}")
 
 
-@pytest.mark.parametrize("cluster", [1, 2, 3, 4, 7, 8, 12, 16])
-def test_decode_step_every_cluster_size(cluster, monkeypatch):
-    monkeypatch.setenv("TWL_FUSED_CLUSTER", str(cluster))
-    wl = synth.make_decode("clusters", 2, 8, 2, [3001, 515], seed=9)
+@pytest.mark.parametrize("shape", [
+    (1, 8, 1, [3001]),                      # one group: ~90 one-page score items, 64 slices
+    (2, 8, 2, [3001, 515]),                 # 4 groups
+    (5, 16, 8, [1999, 17, 4100, 700, 1]),   # 40 groups, ragged, a one-token sequence
+    (12, 8, 8, [2500] * 12),                # 96 groups: several items per CTA in every kind
+], ids=["1grp", "4grp", "40grp", "96grp"])
+def test_decode_step_work_list_shapes(shape):
+    """The persistent step cuts each group into score chunks and estimate / attention slices
+    sized from the group count; these shapes cover every branch of that plan (one group spread
+    over the whole GPU, a few groups, more groups than half the SMs)."""
+    batch, hq, hkv, lens = shape
+    wl = synth.make_decode("shapes", batch, hq, hkv, lens, seed=9 + batch, permute_pages=True,
+                           temperature=True)
     layer = DecodeLayer.from_workload(wl)
     layer.build_aux()
     st, o, lse = _run_step(wl, layer)
@@ -535,18 +544,19 @@ def test_decode_step_every_cluster_size(cluster, monkeypatch):
     assert layer.status()[0] == twl.TWL_OK
 
 
-@pytest.mark.parametrize("cluster", [1, 3, 8, 16])
-def test_decode_step_small_ctas(cluster, monkeypatch):
-    """The 256-thread build (two CTAs per SM), forced, over several cluster sizes."""
-    monkeypatch.setenv("TWL_FUSED_THREADS", "256")
-    monkeypatch.setenv("TWL_FUSED_CLUSTER", str(cluster))
-    wl = synth.make_decode("small_ctas", 2, 8, 2, [3001, 515], seed=19)
+def test_decode_step_repeated_launches_on_one_workspace():
+    """Back-to-back steps on one workspace (its synchronisation words are cleared by each launch
+    for the next), including a different p in between: every launch equals a fresh one."""
+    wl = synth.make_decode("repeat", 3, 16, 4, [2000, 900, 3100], seed=41, temperature=True)
     layer = DecodeLayer.from_workload(wl)
     layer.build_aux()
-    st, o, lse = _run_step(wl, layer)
-    for bb in range(wl.batch):
-        for kvh in range(wl.num_kv_heads):
-            check_step_group(wl, bb, kvh, st, o, lse)
+    q = torch.from_numpy(wl.q).cuda()
+    first = [t.clone() for t in layer.decode(q, wl.p, wl.eps)]
+    for p in (0.9, 0.85, 0.7, 0.85):
+        for _ in range(5):
+            layer.decode(q, p, wl.eps)
+    again = layer.decode(q, wl.p, wl.eps)
+    assert torch.equal(first[0], again[0]) and torch.equal(first[1], again[1])
     assert layer.status()[0] == twl.TWL_OK
 
 
