@@ -48,11 +48,11 @@ struct Shared {
   int scan[64];
   uint32_t state[4];
   unsigned long long t_ready;  // trace builds: when the item's wait ended
-  unsigned long long marks[7];  // trace builds: points inside the item
+  unsigned long long marks[10];  // trace builds: points inside the item
 };
 
 // Trace build (compile with -DTWL_STEP_TRACE; never in the shipped library): thread 0 of every CTA
-// records, per item, (index, CTA, start, wait end, 7 marks, end) in %globaltimer nanoseconds and
+// records, per item, (index, CTA, start, wait end, 10 marks, end) in %globaltimer nanoseconds and
 // the SM clock at start and end into a region
 // at the start of the step's workspace region (before its other arrays).
 __device__ __forceinline__ unsigned long long now_ns() {
@@ -151,6 +151,7 @@ __device__ void block_set_ready(uint32_t* f) {
 __device__ __forceinline__ float ldcg_f(const float* p) { return __ldcg(p); }
 __device__ __forceinline__ int ldcg_i(const int* p) { return __ldcg(p); }
 __device__ __forceinline__ uint32_t ldcg_u(const uint32_t* p) { return __ldcg(p); }
+__device__ __forceinline__ int4 ldcg_i4(const int4* p) { return __ldcg(p); }
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -191,6 +192,84 @@ __device__ __forceinline__ int group_of(const Args& a, int bh) {
 // to right, then the pairs (l, l+8), (l, l+4), (l, l+2), (l, l+1)).
 constexpr int kScorePass = 176;
 
+// Packed fp32 FMA on two lanes (a.x*b.x + c.x, a.y*b.y + c.y), each lane rounded as fmaf.
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long pack2(float x, float y) {
+  return (unsigned long long)__float_as_uint(x) | ((unsigned long long)__float_as_uint(y) << 32);
+}
+
+// The score of the half-warp's page for every head, in the fixed order: lane l's partial sum of
+// channels 8l..8l+7 (from +0, left to right), then the pairs (l, l^8), (l, l^4), (l, l^2),
+// (l, l^1).  Each term is q_c * max_c (q_c > 0) or q_c * min_c: written as fma(q+, max, acc)
+// followed by fma(q-, min, acc), one of which adds an exact zero, so the sum rounds exactly as
+// acc + t_c.  Two heads share each packed FMA.  The tree exchanges halves of the head set at
+// each level (every sum still pairs the same two partial sums), so lane l ends with the score of
+// head l / (16 / G) when l is a multiple of 16 / G.
+template <int G, int NV>
+__device__ __forceinline__ float score_tree(float (&v)[NV], int l) {
+  // exchange tree over offsets 8, 4, 2, 1 (within the half-warp)
+  int n = G;
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) {
+    if (n > 1) {
+      const bool up = (l & o) != 0;
+      const int half = n / 2;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (i < half) {
+          const float send = up ? v[i] : v[i + half];
+          const float keep = up ? v[i + half] : v[i];
+          v[i] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, o));
+        }
+      }
+      n = half;
+    } else {
+      v[0] = __fadd_rn(v[0], __shfl_xor_sync(0xffffffffu, v[0], o));
+    }
+  }
+  return v[0];
+}
+
+template <int G>
+__device__ __forceinline__ float page_score(const unsigned long long (&qp)[(G + 1) / 2][8],
+                                            const unsigned long long (&qn)[(G + 1) / 2][8],
+                                            const float (&mn)[8], const float (&mx)[8], int l) {
+  constexpr int GP = (G + 1) / 2;
+  float v[2 * GP];
+#pragma unroll
+  for (int hp = 0; hp < GP; ++hp) {
+    unsigned long long acc = 0ull;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      acc = fma2(qp[hp][k], pack2(mx[k], mx[k]), acc);
+      acc = fma2(qn[hp][k], pack2(mn[k], mn[k]), acc);
+    }
+    v[2 * hp] = __uint_as_float((uint32_t)acc);
+    v[2 * hp + 1] = __uint_as_float((uint32_t)(acc >> 32));
+  }
+  return score_tree<G>(v, l);
+}
+
+// The same for eight heads (the packed (q+, q-) pairs would take 128 registers): the term is
+// selected per head and added with one scalar FMA (the same rounding).
+__device__ __forceinline__ float page_score8(const float (&qv)[8][8], const float (&mn)[8],
+                                             const float (&mx)[8], int l) {
+  float v[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc = __fmaf_rn(qv[h][k], qv[h][k] > 0.f ? mx[k] : mn[k], acc);
+    v[h] = acc;
+  }
+  return score_tree<8>(v, l);
+}
+
 template <int G>
 __device__ void item_score(const Args& a, Shared& sh, int g, int c, unsigned char* smem) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -214,13 +293,43 @@ __device__ void item_score(const Args& a, Shared& sh, int g, int c, unsigned cha
         pt[i] = -1;
       }
     }
-    float qv[G][8];
+    constexpr int GP = (G + 1) / 2;
+    constexpr bool kPacked = G <= 4;
+    // (q+, q-) of heads (2i, 2i+1), channels 8l..8l+7 (packed form), or q itself (eight heads)
+    unsigned long long qp[kPacked ? GP : 1][8], qn[kPacked ? GP : 1][8];
+    float q8[kPacked ? 1 : 8][8];
+    if constexpr (!kPacked) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
-                                  a.q + ((size_t)b * a.hq + kvh * G + h) * kHeadDim) + l);
-      unpack8(raw, qv[h]);
+      for (int h = 0; h < 8; ++h) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
+                                    a.q + ((size_t)b * a.hq + kvh * G + h) * kHeadDim) + l);
+        unpack8(raw, q8[h]);
+      }
+    } else {
+      float qv[2 * GP][8];
+#pragma unroll
+      for (int h = 0; h < 2 * GP; ++h) {
+        if (h < G) {
+          const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
+                                      a.q + ((size_t)b * a.hq + kvh * G + h) * kHeadDim) + l);
+          unpack8(raw, qv[h]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) qv[h][k] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int hp = 0; hp < GP; ++hp)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float x = qv[2 * hp][k], y = qv[2 * hp + 1][k];
+          qp[hp][k] = pack2(x > 0.f ? x : 0.f, y > 0.f ? y : 0.f);
+          qn[hp][k] = pack2(x > 0.f ? 0.f : x, y > 0.f ? 0.f : y);
+        }
     }
+    (void)qp;
+    (void)qn;
+    (void)q8;
     __syncthreads();
     TRACE_MARK(sh, 0);
     const int npass = (n + kScorePass - 1) / kScorePass;
@@ -260,27 +369,13 @@ __device__ void item_score(const Args& a, Shared& sh, int g, int c, unsigned cha
         float mn[8], mx[8];
         unpack8(vmn, mn);
         unpack8(vmx, mx);
-        float acc[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float sc = 0.f;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            sc = __fmaf_rn(qv[h][kk], qv[h][kk] > 0.f ? mx[kk] : mn[kk], sc);
-          acc[h] = sc;
-        }
-#pragma unroll
-        for (int off = 8; off > 0; off >>= 1) {
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-            acc[h] = __fadd_rn(acc[h], __shfl_xor_sync(0xffffffffu, acc[h], off));
-        }
-        if (in && l < G) {
-          float v = acc[0];
-#pragma unroll
-          for (int h = 1; h < G; ++h) v = (l == h) ? acc[h] : v;
+        float v;
+        if constexpr (kPacked) v = page_score<G>(qp, qn, mn, mx, l);
+        else v = page_score8(q8, mn, mx, l);
+        constexpr int kStride = 16 / G;  // lanes per head after the exchange tree
+        if (in && (l % kStride) == 0) {
           if (ph < 0) v = -INFINITY;
-          krow[(size_t)l * a.kv.max_pages + i0 + ip] = f32_key(v);
+          krow[(size_t)(l / kStride) * a.kv.max_pages + i0 + ip] = f32_key(v);
         }
       }
       __syncthreads();  // the pass's buffer is read before it is refilled
@@ -983,6 +1078,134 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
 #undef TWL_FOR_EACH_WEIGHT
 }
 
+// The same T, located first with approximate bin masses (one shared integer atomic per weight,
+// the weight truncated to units of 2^-30) and then
+// proven exactly: with the bin where the approximate mass from the top first reaches p, the band of
+// that bin and its two neighbours is checked in fixed point (the exact mass above the band is below p
+// and, with the band, reaches p), and the band's weights are ranked pairwise.  The approximate
+// sums only choose where to look; the threshold is exact or the exact histogram search runs
+// instead.
+// Returns false when the check fails (or the band holds more than kThreads weights).
+template <int kR>
+__device__ bool threshold_by_band(const float (&wr)[kR], bool in_regs, const float* W,
+                                  bool staged, int nc, uint32_t lo, uint32_t hi, long long P,
+                                  float* fmass, float* gv, long long* gq, Shared& sh,
+                                  unsigned long long* sh64, float* red, float* T_out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// BODY runs with `w` bound to each of this thread's weights (registers or W)
+#define TWL_FOR_EACH_WEIGHT(BODY)                                           \
+  do {                                                                      \
+    if (in_regs) {                                                          \
+      _Pragma("unroll") for (int k_ = 0; k_ < kR; ++k_) {                   \
+        if (k_ * kThreads + tid < nc) {                                     \
+          const float w = wr[k_];                                           \
+          BODY;                                                             \
+        }                                                                   \
+      }                                                                     \
+    } else {                                                                \
+      for (int i_ = tid; i_ < nc; i_ += kThreads) {                         \
+        const float w = staged ? W[i_] : __ldcg(W + i_);                    \
+        BODY;                                                               \
+      }                                                                     \
+    }                                                                       \
+  } while (0)
+  const uint32_t width = hi - lo;
+  const int bits = 32 - __clz(width);
+  const int s = bits > 11 ? bits - 11 : 0;
+  const int nb = (int)(width >> s) + 1;
+  uint32_t* imass = reinterpret_cast<uint32_t*>(fmass);
+  for (int i = tid; i < kHBins; i += kThreads) imass[i] = 0u;
+  __syncthreads();
+  // bin masses in units of 2^-30, truncated (a weight loses < 2^-30; the sums stay below 2^32)
+  TWL_FOR_EACH_WEIGHT({
+    const uint32_t u = __float_as_uint(w);
+    if (u >= lo && u <= hi) atomicAdd(&imass[(u - lo) >> s], (uint32_t)(w * 1073741824.f));
+  });
+  __syncthreads();
+  // descending scan (thread t holds bins nb-1-4t .. nb-4-4t): the crossing bin
+  float mb[4], mine = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int b = nb - 1 - 4 * tid - e;
+    mb[e] = b >= 0 ? (float)imass[b] * 9.313225746154785e-10f : 0.f;
+    mine += mb[e];
+  }
+  float x = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (tid == 0) sh.state[3] = 0xFFFFFFFFu;
+  __syncthreads();
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  float run = x - mine;
+  for (int w2 = 0; w2 < warp; ++w2) run += red[w2];
+  const float pf = (float)((double)P * 3.552713678800501e-15);  // P * 2^-48
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int b = nb - 1 - 4 * tid - e;
+    if (b >= 0 && run < pf && run + mb[e] >= pf) sh.state[3] = (uint32_t)b;
+    run += mb[e];
+  }
+  __syncthreads();
+  const uint32_t bx = sh.state[3];
+  bool ok = bx != 0xFFFFFFFFu;
+  float T = 0.f;
+  if (ok) {
+    // the band: the crossing bin and its two neighbours
+    const uint32_t blo_bin = bx > 0 ? bx - 1 : 0, bhi_bin = bx + 1;
+    const uint32_t band_lo = lo + (blo_bin << s);
+    const uint64_t bh_top = (uint64_t)lo + ((uint64_t)(bhi_bin + 1) << s) - 1;
+    const uint32_t band_hi = bh_top < (uint64_t)hi ? (uint32_t)bh_top : hi;
+    // exact: the mass above the band, and the band's weights
+    unsigned long long above_t = 0;
+    int c = 0;
+    TWL_FOR_EACH_WEIGHT({
+      const uint32_t u = __float_as_uint(w);
+      if (u > band_hi && u <= hi) above_t += (unsigned long long)w_fixed(w);
+      c += (u >= band_lo && u <= band_hi) ? 1 : 0;
+    });
+    unsigned long long above = 0;
+    block_excl_u64(above_t, sh64, &above);
+    int n = 0;
+    int pos = block_exclusive_scan(c, sh.scan, &n);
+    ok = n <= kThreads && above < (unsigned long long)P;  // uniform
+    TRACE_MARK(sh, 8);
+    if (ok) {
+      TWL_FOR_EACH_WEIGHT({
+        const uint32_t u = __float_as_uint(w);
+        if (u >= band_lo && u <= band_hi) {
+          gv[pos] = w;
+          gq[pos] = w_fixed(w);
+          ++pos;
+        }
+      });
+      __syncthreads();
+      float t = 0.f;
+      if (tid < n) {
+        const float vi = gv[tid];
+        unsigned long long m = above;
+        for (int j = 0; j < n; ++j) m += gv[j] >= vi ? (unsigned long long)gq[j] : 0ull;
+        t = m >= (unsigned long long)P ? vi : 0.f;
+      }
+      t = warp_max(t);
+      __syncthreads();
+      if (lane == 0) red[warp] = t;
+      __syncthreads();
+#pragma unroll
+      for (int w2 = 0; w2 < kWarps; ++w2) T = fmaxf(T, red[w2]);
+      // no band weight reaching p means T lies below the band
+      ok = T > 0.f;
+    }
+  }
+  __syncthreads();
+#undef TWL_FOR_EACH_WEIGHT
+  *T_out = T;
+  return ok;
+}
+
 // Top-p of one q-head over its nc candidates.  W_i = exp(l_i - M) / S with M the largest logit
 // and S summed in a fixed order (per thread over its rows, then over the block).  Only weights
 // >= L = (1 - p) / (2 nc) can decide a test above L (the weights below L sum to less than
@@ -1005,7 +1228,9 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
   const int tail_off = (int)(tail - smem);
   // weights staged in shared memory when they fit beside the histogram scratch of the large
   // live-set search (5 * 2048 words)
-  const bool staged = tail_off + ((4 * nc + 127) & ~127) + 16 * kHBins <= smem_bytes;
+  const bool staged = tail_off + ((4 * nc + 127) & ~127) + 16 * kHBins +
+                          4 * (((nc + 31) >> 5) + 32) + 8 * (a.sel_words + 32) <=
+                      smem_bytes;
 
   const float p = a.p, eps = a.eps;
   const bool use_bound = nc > 0 && p < 1.f && (1.f - p) >= 1e-3f;
@@ -1145,9 +1370,15 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
     const long long P = __double2ll_ru((double)p * 281474976710656.0);
     unsigned long long* hist =
         reinterpret_cast<unsigned long long*>(tail + (staged ? ((4 * nc + 127) & ~127) : 0));
-    const float T = threshold_by_bins<kR>(wr, in_regs, W, staged, nc, __float_as_uint(L),
-                                          __float_as_uint(top), P, hist, lw, lq, sh,
-                                          sh64, red);
+    float T = 0.f;
+    if (!threshold_by_band<kR>(wr, in_regs, W, staged, nc, __float_as_uint(L),
+                               __float_as_uint(top), P, reinterpret_cast<float*>(hist), lw, lq,
+                               sh, sh64, red, &T))
+    {
+      TRACE_MARK(sh, 9);
+      T = threshold_by_bins<kR>(wr, in_regs, W, staged, nc, __float_as_uint(L),
+                                __float_as_uint(top), P, hist, lw, lq, sh, sh64, red);
+    }
     m = bisect_scalar(top, fmaxf(L, T), eps);
   }
   TRACE_MARK(sh, 3);
@@ -1155,29 +1386,26 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
     if (a.threshold) a.threshold[bh] = m;
     if (a.cand_count) a.cand_count[bh] = nc;
   }
-  // kept-row bitmap of this head: bit i = (W_i >= m)
-  uint32_t* kb_out = a.keptbits + (size_t)bh * a.kept_words;
+  // kept-row bitmap of this head: bit i = (W_i >= m), in shared memory (after the staged
+  // weights and the histogram scratch)
   const int kw = (nc + 31) >> 5;
-  uint32_t* kbits = reinterpret_cast<uint32_t*>(tail);
+  uint32_t* kws = reinterpret_cast<uint32_t*>(tail + (staged ? ((4 * nc + 127) & ~127) : 0) +
+                                              16 * kHBins);
   int cnt = 0;
-  if (from_live && m >= L && tail_off + 4 * kw <= smem_bytes) {
+  if (from_live && m >= L) {
     // every kept candidate is live
-    for (int w = tid; w < kw; w += kThreads) kbits[w] = 0u;
+    for (int w = tid; w < kw; w += kThreads) kws[w] = 0u;
     __syncthreads();
-    if (tid < nlive && lw[tid] >= m) atomicOr(&kbits[li[tid] >> 5], 1u << (li[tid] & 31));
+    if (tid < nlive && lw[tid] >= m) atomicOr(&kws[li[tid] >> 5], 1u << (li[tid] & 31));
     __syncthreads();
-    for (int w = tid; w < kw; w += kThreads) {
-      const uint32_t x = kbits[w];
-      kb_out[w] = x;
-      cnt += __popc(x);
-    }
+    for (int w = tid; w < kw; w += kThreads) cnt += __popc(kws[w]);
   } else if (in_regs) {
 #pragma unroll
     for (int k = 0; k < kR; ++k) {
       const int i = k * kThreads + tid;
       const bool keep = i < nc && wr[k] >= m;
       const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-      if (lane == 0 && k * kThreads + 32 * warp < nc) kb_out[k * kWarps + warp] = bal;
+      if (lane == 0 && k * kThreads + 32 * warp < nc) kws[k * kWarps + warp] = bal;
       cnt += keep;
     }
   } else {
@@ -1186,13 +1414,39 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
       const int i = base + tid;
       const bool keep = i < nc && (staged ? W[i] : ldcg_f(W + i)) >= m;
       const uint32_t bal = __ballot_sync(0xffffffffu, keep);
-      if (lane == 0 && base + 32 * warp < nc) kb_out[(base >> 5) + warp] = bal;
+      if (lane == 0 && base + 32 * warp < nc) kws[(base >> 5) + warp] = bal;
       cnt += keep;
     }
   }
   if (a.kept_count) {  // only when the caller asks for it
     const float total = block_sum_fixed((float)cnt, red);
     if (tid == 0) a.kept_count[bh] = (int)total;
+  }
+  // the head's kept rows of each selected page, ORed into the group's page masks (two pages per
+  // word); the page of selection rank r is the r-th set bit of the head's bitmap, found from its
+  // per-word prefix counts
+  const Seq sq = load_seq(a.kv.seq_lens, bh / a.hq, a.kv.max_pages, a.flags, false);
+  const int nw = (sq.pages + 31) >> 5;
+  uint32_t* sb = kws + ((kw + 31) & ~31);
+  int* sp = reinterpret_cast<int*>(sb + ((nw + 31) & ~31));
+  for (int w = tid; w < nw; w += kThreads) {
+    sb[w] = ldcg_u(a.selbits + (size_t)bh * a.sel_words + w);
+    sp[w] = ldcg_i(a.hpre + (size_t)bh * a.sel_words + w);
+  }
+  __syncthreads();
+  uint32_t* pm = a.pmask + (size_t)g * a.pm_words;
+  const int kbp = (nc + kPage - 1) / kPage;  // selected pages of the head
+  for (int r = tid; r < kbp; r += kThreads) {
+    const uint32_t mk = (kws[r >> 1] >> (16 * (r & 1))) & 0xFFFFu;
+    if (mk == 0u) continue;
+    int lo = 0, hi = nw;  // the last word whose prefix is <= r
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (sp[mid] <= r) lo = mid;
+      else hi = mid;
+    }
+    const int j = 32 * lo + nth_set_bit(sb[lo], r - sp[lo]);
+    atomicOr(pm + (j >> 1), mk << (16 * (j & 1)));
   }
 }
 
@@ -1202,135 +1456,134 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
 // rows; the kept rows are listed in ascending token order as K/V row indices (and token ids when
 // the caller asks for the union).
 template <int G>
-__device__ void build_kept(const Args& a, Shared& sh, int g) {
+__device__ void build_kept(const Args& a, Shared& sh, int g, unsigned char* smem) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
   const Seq sq = load_seq(a.kv.seq_lens, b, a.kv.max_pages, a.flags, false);
   const bool aborted = ld_acquire(a.sync + kAbort) != 0u;
   const int n_pages = aborted ? 0 : sq.pages;
-  const size_t kbase = (size_t)g * kPage * a.kv.max_pages;
-  const size_t row0 = (size_t)b * a.hq + kvh * G;
+  const int nw2 = (n_pages + 1) >> 1;
+  int4* kp = a.kpages + (size_t)g * a.kv.max_pages;
+  uint32_t* pm = a.pmask + (size_t)g * a.pm_words;
   TRACE_MARK(sh, 4);
-  // four logical pages per thread (j = base + tid + kThreads * r), every load in flight together:
-  // the heads' bitmap words and prefix counts (shared by 32 pages) and the page-table entry, then
-  // the kept-row words of the heads that selected the page; the list is in page order, so the
-  // scan is over (r, tid)
-  constexpr int kR = 4;
-  int* wsum = sh.scan;  // [kR][kWarps] per-warp totals
-  int carry = 0;
+  // thread per mask word (two logical pages): the kept rows of the group's heads, cut to the valid
+  // rows of pages the table can place (the word is cleared for the next launch); every page with
+  // a kept row becomes one entry (K/V row index of its row 0, row mask, logical page, kept tokens
+  // before it), in page order
+  const int* ptab = a.kv.page_table + (size_t)b * a.kv.max_pages;
+  int* spre = reinterpret_cast<int*>(smem);  // kept tokens before each kept page
+  int npg = 0, ntok = 0;
 #pragma unroll 1
-  for (int base = 0; base < n_pages; base += kR * kThreads) {
-    int ph[kR], rk[kR][G];
-#pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      const int j = base + tid + kThreads * r;
-      ph[r] = -1;
-#pragma unroll
-      for (int h = 0; h < G; ++h) rk[r][h] = -1;
-      if (j < n_pages) {
-        const int w = j >> 5, bit = j & 31;
-        uint32_t x[G];
-        int pre[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          x[h] = ldcg_u(a.selbits + (row0 + h) * a.sel_words + w);
-          pre[h] = ldcg_i(a.hpre + (row0 + h) * a.sel_words + w);
-        }
-        ph[r] = a.kv.page_table[(size_t)b * a.kv.max_pages + j];
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-          rk[r][h] = ((x[h] >> bit) & 1u) ? pre[h] + __popc(x[h] & ((1u << bit) - 1u)) : -1;
-      }
+  for (int base = 0; base < nw2; base += kThreads) {
+    const int w2 = base + tid;
+    uint32_t m32 = 0;
+    int ph[2] = {-1, -1};
+    if (w2 < nw2) {
+      m32 = ldcg_u(pm + w2);
+      ph[0] = ptab[2 * w2];
+      ph[1] = 2 * w2 + 1 < n_pages ? ptab[2 * w2 + 1] : -1;
     }
-    uint32_t mask[kR];
+    if (m32) pm[w2] = 0u;
+    uint32_t mk[2] = {m32 & 0xFFFFu, m32 >> 16};
 #pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      uint32_t w[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-        w[h] = rk[r][h] >= 0 ? ldcg_u(a.keptbits + (row0 + h) * a.kept_words + (rk[r][h] >> 1))
-                             : 0u;
-      uint32_t m = 0;
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-        if (rk[r][h] >= 0) m |= (w[h] >> (16 * (rk[r][h] & 1))) & 0xFFFFu;
-      const int j = base + tid + kThreads * r;
-      if (m) {
+    for (int e = 0; e < 2; ++e) {
+      const int j = 2 * w2 + e;
+      if (mk[e]) {
         const int rows = page_rows(sq.n, j);
-        m &= rows >= 16 ? 0xFFFFu : ((1u << rows) - 1u);
-        if (ph[r] < 0 || ph[r] >= a.kv.num_phys) {  // never attended; the estimate flagged it
-          ph[r] = -1;
-          m = 0u;
-        }
+        mk[e] &= rows >= 16 ? 0xFFFFu : ((1u << rows) - 1u);
+        if (ph[e] < 0 || ph[e] >= a.kv.num_phys) mk[e] = 0u;  // never attended (flagged before)
       }
-      mask[r] = m;
     }
     TRACE_MARK(sh, 5);
-    int pos[kR], incl[kR];
+    // two scans at once (pages, tokens): warp shuffles, then the warp totals
+    int cp = (mk[0] != 0u) + (mk[1] != 0u), ct = __popc(mk[0]) + __popc(mk[1]);
+    int xp = cp, xt = ct;
 #pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      int x = __popc(mask[r]);
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yp = __shfl_up_sync(0xffffffffu, xp, o);
+      const int yt = __shfl_up_sync(0xffffffffu, xt, o);
+      if (lane >= o) {
+        xp += yp;
+        xt += yt;
       }
-      incl[r] = x;
     }
     __syncthreads();
     if (lane == 31) {
-#pragma unroll
-      for (int r = 0; r < kR; ++r) wsum[r * kWarps + warp] = incl[r];
+      sh.scan[warp] = xp;
+      sh.scan[kWarps + warp] = xt;
     }
     __syncthreads();
+    int bp = npg, bt = ntok, ap = 0, at = 0;
 #pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      int before = carry, all = 0;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const int tt = wsum[r * kWarps + w];
-        if (w < warp) before += tt;
-        all += tt;
+    for (int w = 0; w < kWarps; ++w) {
+      const int vp = sh.scan[w], vt = sh.scan[kWarps + w];
+      if (w < warp) {
+        bp += vp;
+        bt += vt;
       }
-      pos[r] = before + incl[r] - __popc(mask[r]);
-      carry += all;
+      ap += vp;
+      at += vt;
     }
+    int q = bp + xp - cp, tq = bt + xt - ct;
 #pragma unroll
-    for (int r = 0; r < kR; ++r) {
-      const int j = base + tid + kThreads * r;
-      const uint32_t rbase = (uint32_t)(((size_t)(ph[r] < 0 ? 0 : ph[r]) * a.kv.hkv + kvh) * kPage);
-      uint32_t mm = mask[r];
-      int q = pos[r];
-      while (mm) {
-        const int row = __ffs(mm) - 1;
-        a.krow[kbase + q] = rbase + (uint32_t)row;
-        if (a.union_tok) a.union_tok[kbase + q] = kPage * j + row;
+    for (int e = 0; e < 2; ++e) {
+      if (mk[e]) {
+        const int j = 2 * w2 + e;
+        kp[q] = make_int4((int)(((size_t)ph[e] * a.kv.hkv + kvh) * kPage), (int)mk[e], j, tq);
+        spre[q] = tq;
+        if (a.union_tok) {  // the ascending union of kept tokens, when the caller asks for it
+          uint32_t mm = mk[e];
+          int t = tq;
+          while (mm) {
+            a.union_tok[(size_t)g * kPage * a.kv.max_pages + t++] = kPage * j + __ffs(mm) - 1;
+            mm &= mm - 1u;
+          }
+        }
         ++q;
-        mm &= mm - 1u;
+        tq += __popc(mk[e]);
       }
     }
+    npg += ap;
+    ntok += at;
   }
-  // publish the group's kept tokens to the attention queue: chunks of up to kAttChunkTok tokens
-  // (one empty chunk when nothing is kept, so the merge still writes the outputs)
-  const int nch = carry > 0 ? (carry + kAttChunkTok - 1) / kAttChunkTok : 1;
+  TRACE_MARK(sh, 7);
+  // publish the group's kept pages to the attention queue in nch chunks of about equal token
+  // counts (at most kAttChunkTok + 15 tokens each): page q opens chunk floor(pre(q) nch / ntok).
+  // As a page holds at most 16 tokens and a chunk about kAttChunkTok, consecutive pages open
+  // consecutive chunks and none is empty.  One empty chunk when nothing is kept, so the merge
+  // still writes the outputs.
+  const int nch = ntok > 0 ? (ntok + kAttChunkTok - 1) / kAttChunkTok : 1;
   if (tid == 0) {
-    if (a.union_count) a.union_count[g] = carry;
+    if (a.union_count) a.union_count[g] = ntok;
     sh.total = (int)atomicAdd(a.sync + kQAlloc, (uint32_t)nch);
   }
-  __syncthreads();
+  __syncthreads();  // also orders the staged prefix counts
   const int base = sh.total;
-  for (int c = tid; c < nch; c += kThreads) {
-    if (base + c >= a.q_cap) break;
-    int* e = a.qtab + 4 * (size_t)(base + c);
-    e[0] = g;
-    e[1] = (int)((long long)carry * c / nch);
-    e[2] = (int)((long long)carry * (c + 1) / nch);
+  for (int q = tid; q < npg; q += kThreads) {
+    const int c = (int)((long long)spre[q] * nch / ntok);
+    const int cp = q > 0 ? (int)((long long)spre[q - 1] * nch / ntok) : -1;
+    if (c != cp) {
+      if (base + c < a.q_cap) {
+        int* e = a.qtab + 4 * (size_t)(base + c);
+        e[0] = g;
+        e[1] = q;
+      }
+      if (c > 0 && base + c - 1 < a.q_cap) a.qtab[4 * (size_t)(base + c - 1) + 2] = q;
+    }
   }
   if (tid == 0) {
+    if (base + nch - 1 < a.q_cap) {
+      int* e = a.qtab + 4 * (size_t)(base + nch - 1);
+      e[2] = npg;
+      if (npg == 0) {
+        e[0] = g;
+        e[1] = 0;
+      }
+    }
     a.cbase[2 * g] = base;
     a.cbase[2 * g + 1] = nch;
   }
-  __syncthreads();  // the chunk entries, counts and kept list before the valid flags
+  __syncthreads();  // the chunk entries, counts and kept pages before the valid flags
   if (tid == 0) {
     // one release fence for everything the block wrote (it observed all of it at the barrier),
     // then plain stores of the flags
@@ -1345,8 +1598,8 @@ __device__ void build_kept(const Args& a, Shared& sh, int g) {
 }
 
 // ------------------------------------------------------------------------------ attention
-// Kept tokens [t0, t1) of group g (one chunk of the attention work list).  Their K/V row indices
-// are staged in passes of up to kAttIdx; the rows (256 B of K and of V each) are copied with
+// Kept pages [t0, t1) of group g (one chunk of the attention work list).  Their row masks are
+// expanded to the K/V row index of every kept token in shared memory; the rows (256 B of K and of V each) are copied with
 // 16-byte cp.async in passes of kAttPass tokens, two in flight, each row's 16-byte pieces XOR-
 // swizzled by the row number so that ldmatrix reads are free of bank conflicts.
 // The contraction runs on the tensor cores (mma.m16n8k16, fp16 in, fp32 accumulate).  S = Q K^T
@@ -1358,7 +1611,7 @@ __device__ void build_kept(const Args& a, Shared& sh, int g) {
 // products, so its rounding stays near 2^-22 of the weights.  Each warp keeps its own running
 // (max, sum, o) per head; the warps' states are merged at the end into the chunk's partial.
 constexpr int kAttPass = 128;
-constexpr int kAttIdx = 3840;  // a multiple of kAttPass
+constexpr int kAttIdx = 384;  // >= the tokens of a chunk (kAttChunkTok + 15)
 
 __device__ __forceinline__ uint32_t saddr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -1387,7 +1640,7 @@ __device__ void attend_chunk(const Args& a, Shared& sh, int g, int t0, int t1, i
   const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
   uint32_t* idx = reinterpret_cast<uint32_t*>(smem);
   unsigned char* buf = smem + 4 * kAttIdx;
-  const uint32_t* klist = a.krow + (size_t)g * kPage * a.kv.max_pages;
+  const int4* kp = a.kpages + (size_t)g * a.kv.max_pages;
   // A fragments of the queries (rows = heads; rows >= G and the upper 8 rows are zero)
   uint32_t qa[8][2];
   {
@@ -1406,10 +1659,23 @@ __device__ void attend_chunk(const Args& a, Shared& sh, int g, int t0, int t1, i
 #pragma unroll
     for (int c = 0; c < 4; ++c) ot[mt][c] = 0.f;
   const float sc_scale = a.sm_scale;
-#pragma unroll 1
-  for (int m0 = t0; m0 < t1; m0 += kAttIdx) {
-    const int n = min(kAttIdx, t1 - m0);
-    for (int i = tid; i < n; i += kThreads) idx[i] = ldcg_u(klist + m0 + i);
+  {
+    // the chunk's kept pages [t0, t1) expanded to K/V row indices, thread per page, in token order
+    int n = 0, tb = 0;
+    if (t1 > t0) {
+      const int4 f = ldcg_i4(kp + t0), l = ldcg_i4(kp + t1 - 1);
+      tb = f.w;
+      n = l.w + __popc((uint32_t)l.y) - tb;
+    }
+    for (int q = t0 + tid; q < t1; q += kThreads) {
+      const int4 e = ldcg_i4(kp + q);
+      uint32_t m = (uint32_t)e.y;
+      int pos = e.w - tb;
+      while (m) {
+        idx[pos++] = (uint32_t)e.x + (uint32_t)(__ffs(m) - 1);
+        m &= m - 1u;
+      }
+    }
     __syncthreads();
     TRACE_MARK(sh, 0);
     const int npass = (n + kAttPass - 1) / kAttPass;
@@ -1679,7 +1945,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_step(const __grid_constant__ Ar
       t_start = now_ns();
       c_start = clock64();
       sh.t_ready = 0;
-      for (int m = 0; m < 7; ++m) sh.marks[m] = 0;
+      for (int m = 0; m < 10; ++m) sh.marks[m] = 0;
     }
 #endif
     int phase = -1, g = 0, sub = 0;
@@ -1709,7 +1975,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_step(const __grid_constant__ Ar
         break;
       case kPrune:
         item_prune(a, sh, b * a.hq + kvh * G + sub, smem, a.smem_bytes);
-        if (block_signal_last(sh, counter(a, kCntPrune, g), (uint32_t)G)) build_kept<G>(a, sh, g);
+        if (block_signal_last(sh, counter(a, kCntPrune, g), (uint32_t)G))
+          build_kept<G>(a, sh, g, smem);
         break;
       case kAttend:
         attend_worker<G>(a, sh, smem);
@@ -1720,15 +1987,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_step(const __grid_constant__ Ar
 #ifdef TWL_STEP_TRACE
     __syncthreads();
     if (threadIdx.x == 0 && a.trace) {
-      unsigned long long* tr = a.trace + 14 * (size_t)idx;
+      unsigned long long* tr = a.trace + 17 * (size_t)idx;
       tr[0] = (unsigned long long)idx;
       tr[1] = blockIdx.x;
       tr[2] = t_start;
       tr[3] = sh.t_ready;
-      for (int m = 0; m < 7; ++m) tr[4 + m] = sh.marks[m];
-      tr[11] = now_ns();
-      tr[12] = c_start;
-      tr[13] = clock64();
+      for (int m = 0; m < 10; ++m) tr[4 + m] = sh.marks[m];
+      tr[14] = now_ns();
+      tr[15] = c_start;
+      tr[16] = clock64();
     }
 #endif
     // the next free item, taken only now: a CTA never holds an item it cannot start
@@ -1776,7 +2043,9 @@ const void* kernel_for(int g) {
 int smem_need(int g, int max_pages, int max_budget, int s_chunk) {
   const int sw = round32((max_pages + 31) / 32);
   const int topk = 4 * sw + 4 * round32(max_pages) + 4 * 4096 + 8 * 64 + 64;
-  const int prune = 1024 + 16 * kThreads + 16 * kHBins;  // + staged weights when they fit
+  const int kept_words = (16 * max_budget + 31) / 32;
+  const int prune = 1024 + 16 * kThreads + 16 * kHBins + 4 * round32(kept_words) +
+                    8 * round32(sw) + 128;  // + staged weights when they fit
   const int score = ((4 * s_chunk + 127) & ~127) + 2 * kScorePass * 512;
   const int est_kw = kEstMeta / 32 + 1;
   const int est = ((4 * ((2 + g) * kEstMeta + (2 * g + 2) * est_kw + 1) + 127) & ~127) +
@@ -1846,7 +2115,7 @@ Plan plan(int batch, int hq, int hkv, int max_pages, int max_budget) {
 
 namespace {
 struct Layout {
-  size_t sync, keys, selbits, ncand, hpre, logits, keptbits, krow,
+  size_t sync, keys, selbits, ncand, hpre, logits, pmask, kpages,
       qtab, qvalid, cbase, part, trace, total;
 };
 Layout layout(const Plan& pl, int batch, int hq, int hkv, int max_pages) {
@@ -1860,7 +2129,7 @@ Layout layout(const Plan& pl, int batch, int hq, int hkv, int max_pages) {
     return o;
   };
 #ifdef TWL_STEP_TRACE
-  L.trace = take(8 * 14 * (size_t)(groups * (pl.s_per + 2 * g + pl.e_per) + pl.grid));
+  L.trace = take(8 * 17 * (size_t)(groups * (pl.s_per + 2 * g + pl.e_per) + pl.grid));
 #endif
   L.sync = take(4 * (kSyncHead + kCounters * groups));
   L.keys = take(4 * bh * max_pages);
@@ -1868,8 +2137,8 @@ Layout layout(const Plan& pl, int batch, int hq, int hkv, int max_pages) {
   L.ncand = take(4 * bh);
   L.hpre = take(4 * bh * pl.sel_words);
   L.logits = take(4 * bh * pl.cand_stride);
-  L.keptbits = take(4 * bh * pl.kept_words);
-  L.krow = take(4 * groups * kPage * (size_t)max_pages);
+  L.pmask = take(4 * groups * (size_t)((max_pages + 1) / 2));
+  L.kpages = take(16 * groups * (size_t)max_pages);
   L.qtab = take(16 * (size_t)pl.q_cap);
   L.qvalid = take(4 * (size_t)pl.q_cap);
   L.cbase = take(8 * groups);
@@ -1892,8 +2161,9 @@ void carve(Args& a, char* ws, const Plan& pl, int batch, int hq, int hkv, int ma
   a.ncand = reinterpret_cast<int*>(ws + L.ncand);
   a.hpre = reinterpret_cast<int*>(ws + L.hpre);
   a.logits = reinterpret_cast<float*>(ws + L.logits);
-  a.keptbits = reinterpret_cast<uint32_t*>(ws + L.keptbits);
-  a.krow = reinterpret_cast<uint32_t*>(ws + L.krow);
+  a.pmask = reinterpret_cast<uint32_t*>(ws + L.pmask);
+  a.pm_words = (max_pages + 1) / 2;
+  a.kpages = reinterpret_cast<int4*>(ws + L.kpages);
   a.qtab = reinterpret_cast<int*>(ws + L.qtab);
   a.qvalid = reinterpret_cast<uint32_t*>(ws + L.qvalid);
   a.cbase = reinterpret_cast<int*>(ws + L.cbase);

@@ -15,8 +15,8 @@ enum Phase : int {
   kScore = 0,   // page scores of a chunk of the group's pages (all G heads)
   kTopK = 1,    // top-k pages of one q-head
   kEst = 2,     // INT4 estimate over the union pages in a range of the group's logical pages
-  kPrune = 3,   // softmax + top-p threshold of one q-head; the last builds the kept-token list
-  kAttend = 4,  // a worker of the attention queue: takes chunks of kept tokens from every group
+  kPrune = 3,   // softmax + top-p threshold of one q-head; the last builds the kept-page list
+  kAttend = 4,  // a worker of the attention queue: takes chunks of kept pages from every group
 };
 
 // A run of consecutive item indices: groups [g0, g1), `per` items per group, group-major.
@@ -31,7 +31,8 @@ constexpr int kMaxSegments = 40;
 //   kQAlloc  attention chunks published (allocated)    kQNext  chunks taken by workers
 //   kQGroups groups whose chunks are published
 enum { kNext = 0, kExit = 1, kAbort = 2, kQAlloc = 3, kQNext = 4, kQGroups = 5, kSyncHead = 8 };
-// Kept tokens per attention chunk of the flattened work list.
+// Kept tokens per attention chunk of the flattened work list (chunks are cut at page bounds into
+// pieces of about this many tokens).
 constexpr int kAttChunkTok = 256;
 enum { kCntScore = 0, kCntTopK, kCntEst, kCntPrune, kCntAttend, kCounters };
 
@@ -66,15 +67,17 @@ struct Args {
   int* ncand;          // [B*Hq]              candidate rows of each head
   int* hpre;           // [B*Hq][sel_words]   exclusive prefix counts of the selected-page bitmaps
   float* logits;       // [B*Hq][cand_stride] estimated logits, then weights
-  uint32_t* keptbits;  // [B*Hq][kept_words]  bit i = candidate row i passes top-p
-  uint32_t* krow;      // [groups][16*max_pages] K/V row index of each kept token, ascending
-  int* qtab;           // [q_cap][4] attention chunks: (group, first token, end token, -)
+  uint32_t* pmask;     // [groups][pm_words]  kept rows of two logical pages per word (OR over
+                       //                     the group's heads); zero between launches
+  int4* kpages;        // [groups][max_pages] kept pages, ascending: (K/V row index of row 0, row
+                       //                     mask, logical page, kept tokens before the page)
+  int* qtab;           // [q_cap][4] attention chunks: (group, first kept page, end page, -)
   uint32_t* qvalid;    // [q_cap] 1 once the chunk is published
   int* cbase;          // [groups][2] first chunk and chunk count of each group
   float* part;         // [q_cap][G][2 + 128] attention partials per chunk (max, sum, o)
-  unsigned long long* trace;  // trace builds only (-DTWL_STEP_TRACE): 14 words per item
+  unsigned long long* trace;  // trace builds only (-DTWL_STEP_TRACE): 17 words per item
   // strides and the work list
-  int groups, sel_words, cand_stride, kept_words;
+  int groups, sel_words, cand_stride, kept_words, pm_words;
   int s_per, s_chunk, e_per, e_chunk, q_cap;
   int n_items;
   int smem_bytes;  // dynamic shared memory of each CTA

@@ -190,10 +190,27 @@ class ClockSampler:
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return
+        # nvidia-smi takes a few hundred ms to print its first row: wait for it, so that a short
+        # timed region still has samples around it
+        self._wait_rows(1, 5.0)
+
+    def _rows(self) -> int:
+        try:
+            with open(self.path) as f:
+                return sum(1 for _ in f)
+        except OSError:
+            return 0
+
+    def _wait_rows(self, n: int, limit: float):
+        t_end = time.monotonic() + limit
+        while self._rows() < n and time.monotonic() < t_end and self.proc.poll() is None:
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self._wait_rows(self._rows() + 1, 1.0)  # one row after the timed region ends
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
