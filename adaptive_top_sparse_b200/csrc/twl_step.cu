@@ -47,7 +47,13 @@ struct Shared {
   int jlast;
   int scan[64];
   uint32_t state[4];
-  unsigned long long t_ready;  // trace builds: when the item's wait ended
+  int att[2][4];       // attention producers: the chunk taken (slot, group, first, end page)
+  int att_desc[3][4];  // attention ring: per buffer (tokens, slot, group, flags)
+  int att_last;        // attention consumers: this chunk completed its group
+  int att_prod_ok;     // attention producers: the wait for a free buffer succeeded
+  __align__(8) uint64_t att_full[3];   // attention ring: buffer filled (producers -> consumers)
+  __align__(8) uint64_t att_empty[3];  // attention ring: buffer consumed (consumers -> producers)
+  unsigned long long t_ready;    // trace builds: when the item's wait ended
   unsigned long long marks[10];  // trace builds: points inside the item
 };
 
@@ -55,12 +61,12 @@ struct Shared {
 // records, per item, (index, CTA, start, wait end, 10 marks, end) in %globaltimer nanoseconds and
 // the SM clock at start and end into a region
 // at the start of the step's workspace region (before its other arrays).
+#ifdef TWL_STEP_TRACE
 __device__ __forceinline__ unsigned long long now_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-#ifdef TWL_STEP_TRACE
 #define TRACE_MARK(sh, k)                                  \
   do {                                                     \
     if (threadIdx.x == 0) (sh).marks[(k)] = now_ns();      \
@@ -143,15 +149,13 @@ __device__ bool block_signal_last(Shared& sh, uint32_t* ctr, uint32_t total) {
   return last;
 }
 
-__device__ void block_set_ready(uint32_t* f) {
-  __syncthreads();
-  if (threadIdx.x == 0) red_release_add(f, 1u);
-}
-
 __device__ __forceinline__ float ldcg_f(const float* p) { return __ldcg(p); }
 __device__ __forceinline__ int ldcg_i(const int* p) { return __ldcg(p); }
 __device__ __forceinline__ uint32_t ldcg_u(const uint32_t* p) { return __ldcg(p); }
 __device__ __forceinline__ int4 ldcg_i4(const int4* p) { return __ldcg(p); }
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
 
 __device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -894,36 +898,19 @@ __device__ float block_sum_fixed(float v, float* red) {
 // do not depend on the order of the terms.
 __device__ __forceinline__ long long w_fixed(float w) { return __float2ll_rn(w * 281474976710656.f); }
 
-// Threshold from the live set {W >= L} (n <= kThreads values lw, fixed-point copies lq).  Every
-// test of the search at mid > L counts only live weights, and mass(W >= t) is a non-increasing
-// step function of t, so "mid <= L or mass(W >= mid) >= p" is the same test as "mid <= T" with
-// T = max(L, the largest live weight v with mass(W >= v) >= p).  T comes from all pairwise
-// comparisons at once (4, 2 or 1 threads per value); the search itself is then a scalar loop that
-// every thread runs (same inputs, same result).
-__device__ float top_p_from_live(const float* lw, const long long* lq, int n, float L, float p,
-                                 float eps, float top, float* red) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long long P = __double2ll_ru((double)p * 281474976710656.0);
-  const int tpv = n <= kThreads / 4 ? 4 : (n <= kThreads / 2 ? 2 : 1);
-  const int i = tid / tpv, part = tid % tpv;
-  long long mass = 0;
-  float vi = 0.f;
-  if (i < n) {
-    vi = lw[i];
-#pragma unroll 4
-    for (int j = part; j < n; j += tpv) mass += lw[j] >= vi ? lq[j] : 0ll;
-  }
-  if (tpv >= 2) mass += __shfl_xor_sync(0xffffffffu, mass, 1);
-  if (tpv >= 4) mass += __shfl_xor_sync(0xffffffffu, mass, 2);
-  float t = (i < n && mass >= P) ? vi : 0.f;
-  t = warp_max(t);
-  __syncthreads();
-  if (lane == 0) red[warp] = t;
-  __syncthreads();
-  float Tp = 0.f;
+// Sum over the block of one 64-bit value per thread (exact; every thread receives the total).
+// `sh64` needs kWarps words.
+__device__ unsigned long long block_sum_u64(unsigned long long v, unsigned long long* sh64) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) Tp = fmaxf(Tp, red[w]);
-  return bisect_scalar(top, fmaxf(L, Tp), eps);
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) sh64[warp] = v;
+  __syncthreads();
+  unsigned long long t = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) t += sh64[w];
+  return t;
 }
 
 // Exclusive prefix sum over the block of one 64-bit value per thread (thread order); *total gets
@@ -951,14 +938,116 @@ __device__ unsigned long long block_excl_u64(unsigned long long v, unsigned long
   return before + x - v;
 }
 
+// T among n <= kThreads weights gv (fixed-point copies gq) given the exact mass `above` of the
+// weights above them: the largest v with above + mass(gv >= v) >= P (0 when none), by comparing
+// all pairs at once (4, 2 or 1 threads per value).  Cheaper than refine_threshold up to a few
+// hundred weights (its cost grows as n^2; the refinement's is about three block scans).
+__device__ float rank_pairwise(const float* gv, const long long* gq, int n,
+                               unsigned long long above, long long P, float* red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tpv = n <= kThreads / 4 ? 4 : (n <= kThreads / 2 ? 2 : 1);
+  const int i = tid / tpv, part = tid % tpv;
+  unsigned long long mass = 0;
+  float vi = 0.f;
+  if (i < n) {
+    vi = gv[i];
+#pragma unroll 4
+    for (int j = part; j < n; j += tpv) mass += gv[j] >= vi ? (unsigned long long)gq[j] : 0ull;
+  }
+  if (tpv >= 2) mass += __shfl_xor_sync(0xffffffffu, mass, 1);
+  if (tpv >= 4) mass += __shfl_xor_sync(0xffffffffu, mass, 2);
+  float t = (i < n && above + mass >= (unsigned long long)P) ? vi : 0.f;
+  t = warp_max(t);
+  __syncthreads();
+  if (lane == 0) red[warp] = t;
+  __syncthreads();
+  float T = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) T = fmaxf(T, red[w]);
+  __syncthreads();  // red is read before it is reused
+  return T;
+}
+constexpr int kPairwiseMax = 384;  // rank_pairwise up to this many weights, refine_threshold above
+
+// T among n <= kThreads weights gv (fixed-point copies gq, units of 2^-48) whose keys (float
+// bits) lie in [lo, hi], given the exact mass `above` of the weights with keys above hi: the
+// largest value v with above + mass(gv >= v) >= P, or 0 when even all of them fall short.  The
+// keys are histogrammed into up to kHBins bins of equal key width with exact masses (each
+// fixed-point weight, < 2^49, summed as three 16-bit parts in 32-bit shared atomics: no overflow
+// for n <= 2^15); a descending scan finds the bin where the mass from the top first reaches P, and
+// the search narrows to that bin until it is a single key: at most three levels for 32-bit keys.
+// A crossing bin holds mass, so the key found is one of the weights.  `bins` needs 3 * kHBins
+// 32-bit words, `sh64` kWarps + 1.
+__device__ float refine_threshold(const float* gv, const long long* gq, int n, uint32_t lo,
+                                  uint32_t hi, unsigned long long above, long long P,
+                                  uint32_t* bins, Shared& sh, unsigned long long* sh64) {
+  const int tid = threadIdx.x;
+  const bool mine = tid < n;
+  const uint32_t u = mine ? __float_as_uint(gv[tid]) : 0u;
+  const unsigned long long q = mine ? (unsigned long long)gq[tid] : 0ull;
+#pragma unroll 1
+  for (int level = 0; level < 4; ++level) {
+    const uint32_t width = hi - lo;
+    const int bits = 32 - __clz(width);
+    const int s = bits > 11 ? bits - 11 : 0;
+    const int nb = (int)(width >> s) + 1;
+    for (int i = tid; i < nb; i += kThreads) {
+      bins[i] = 0u;
+      bins[2048 + i] = 0u;
+      bins[4096 + i] = 0u;
+    }
+    __syncthreads();
+    if (mine && u >= lo && u <= hi) {
+      const int b = (int)((u - lo) >> s);
+      atomicAdd(&bins[b], (uint32_t)(q & 0xFFFFu));
+      atomicAdd(&bins[2048 + b], (uint32_t)((q >> 16) & 0xFFFFu));
+      atomicAdd(&bins[4096 + b], (uint32_t)(q >> 32));
+    }
+    __syncthreads();
+    // descending scan: thread t holds bins nb-1-4t .. nb-4-4t
+    unsigned long long mb[4], tot = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int b = nb - 1 - 4 * tid - e;
+      mb[e] = b >= 0 ? (unsigned long long)bins[b] + ((unsigned long long)bins[2048 + b] << 16) +
+                           ((unsigned long long)bins[4096 + b] << 32)
+                     : 0ull;
+      tot += mb[e];
+    }
+    if (tid == 0) sh.state[3] = 0xFFFFFFFFu;
+    unsigned long long run = above + block_excl_u64(tot, sh64, nullptr);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int b = nb - 1 - 4 * tid - e;
+      if (b >= 0 && run < (unsigned long long)P && run + mb[e] >= (unsigned long long)P) {
+        sh.state[3] = (uint32_t)b;
+        sh64[kWarps] = run;  // mass above the crossing bin
+      }
+      run += mb[e];
+    }
+    __syncthreads();
+    const uint32_t bx = sh.state[3];
+    const unsigned long long ab = sh64[kWarps];
+    __syncthreads();  // read before the next level (or the caller) writes them
+    if (bx == 0xFFFFFFFFu) return 0.f;
+    above = ab;
+    lo = lo + (bx << s);
+    const uint64_t top_key = (uint64_t)lo + ((1ull << s) - 1ull);
+    hi = top_key < (uint64_t)hi ? (uint32_t)top_key : hi;
+    if (lo == hi) return __uint_as_float(lo);
+  }
+  return 0.f;
+}
+
 // T for a large live set: the largest weight value v with mass(W >= v) >= p, masses exact in
 // fixed point (units of 2^-48).  The masses of the weights with float bit patterns in [lo, hi]
 // are summed into up to 2048 bins of equal key width, exactly and independently of the order of
 // the adds: each fixed-point weight is split into four 12-bit parts summed in 32-bit shared
-// atomics (no overflow for up to 2^20 weights; measured faster than one 64-bit atomic).  A descending scan finds the bin where the mass from
-// the top first reaches p, and T lies in it.  If that bin holds at most kThreads weights they are
-// ranked exactly (pairwise, as for the live set), a single-key bin is T itself, and otherwise the
-// bin is histogrammed again on its finer bits.  Returns 0 when even all counted weights fall
+// atomics (no overflow for up to 2^20 weights; measured faster than one 64-bit atomic).  A
+// descending scan finds the bin where the mass from the top first reaches p, and T lies in it.
+// If that bin holds at most kThreads weights they are gathered and refined exactly
+// (refine_threshold), a single-key bin is T itself, and otherwise the bin is histogrammed again
+// on its finer bits.  Returns 0 when even all counted weights fall
 // short of p.  Weights come from registers (row k * kThreads + tid) or from W (shared or global);
 // `mass` needs 4 * 2048 32-bit words, gv / gq kThreads entries each.
 constexpr int kHBins = 2048;
@@ -967,7 +1056,7 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
                                    bool staged, int nc, uint32_t lo, uint32_t hi, long long P,
                                    unsigned long long* mass, float* gv, long long* gq, Shared& sh,
                                    unsigned long long* sh64, float* red) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   unsigned long long above = 0;  // exact mass of the weights with keys above hi
 // BODY runs with `w` bound to each of this thread's weights (registers or W)
 #define TWL_FOR_EACH_WEIGHT(BODY)                                           \
@@ -1059,30 +1148,19 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
     }
   }
   __syncthreads();
-  float t = 0.f;
-  if (tid < n && n <= kThreads) {
-    const float vi = gv[tid];
-    unsigned long long m = above;
-    for (int j = 0; j < n; ++j) m += gv[j] >= vi ? (unsigned long long)gq[j] : 0ull;
-    t = m >= (unsigned long long)P ? vi : 0.f;
-  }
-  t = warp_max(t);
-  __syncthreads();
-  if (lane == 0) red[warp] = t;
-  __syncthreads();
-  float T = 0.f;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) T = fmaxf(T, red[w]);
-  __syncthreads();
-  return T;
+  if (n > kThreads) return 0.f;  // not reached: four levels narrow any 32-bit key range
+  return n <= kPairwiseMax ? rank_pairwise(gv, gq, n, above, P, red)
+                           : refine_threshold(gv, gq, n, lo, hi, above, P,
+                                              reinterpret_cast<uint32_t*>(mass), sh, sh64);
 #undef TWL_FOR_EACH_WEIGHT
 }
 
-// The same T, located first with approximate bin masses (one shared integer atomic per weight,
-// the weight truncated to units of 2^-30) and then
+constexpr int kBandBins = 8192;
+// The same T, located first with approximate bin masses (kBandBins bins, one shared integer
+// atomic per weight, the weight truncated to units of 2^-30) and then
 // proven exactly: with the bin where the approximate mass from the top first reaches p, the band of
 // that bin and its two neighbours is checked in fixed point (the exact mass above the band is below p
-// and, with the band, reaches p), and the band's weights are ranked pairwise.  The approximate
+// and, with the band, reaches p), and the band's weights are refined exactly (refine_threshold).  The approximate
 // sums only choose where to look; the threshold is exact or the exact histogram search runs
 // instead.
 // Returns false when the check fails (or the band holds more than kThreads weights).
@@ -1091,7 +1169,7 @@ __device__ bool threshold_by_band(const float (&wr)[kR], bool in_regs, const flo
                                   bool staged, int nc, uint32_t lo, uint32_t hi, long long P,
                                   float* fmass, float* gv, long long* gq, Shared& sh,
                                   unsigned long long* sh64, float* red, float* T_out) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
 // BODY runs with `w` bound to each of this thread's weights (registers or W)
 #define TWL_FOR_EACH_WEIGHT(BODY)                                           \
   do {                                                                      \
@@ -1109,44 +1187,37 @@ __device__ bool threshold_by_band(const float (&wr)[kR], bool in_regs, const flo
       }                                                                     \
     }                                                                       \
   } while (0)
+  // kBandBins bins of equal key width (16 per thread in the scan)
+  static_assert(kBandBins == 16 * kThreads, "the scan holds 16 bins per thread");
   const uint32_t width = hi - lo;
   const int bits = 32 - __clz(width);
-  const int s = bits > 11 ? bits - 11 : 0;
+  const int s = bits > 13 ? bits - 13 : 0;
   const int nb = (int)(width >> s) + 1;
   uint32_t* imass = reinterpret_cast<uint32_t*>(fmass);
-  for (int i = tid; i < kHBins; i += kThreads) imass[i] = 0u;
+  for (int i = tid; i < nb; i += kThreads) imass[i] = 0u;
   __syncthreads();
-  // bin masses in units of 2^-30, truncated (a weight loses < 2^-30; the sums stay below 2^32)
+  // bin masses in units of 2^-30, truncated (a weight loses < 2^-30; W <= 1 and the weights sum
+  // to about 1, so the sums and their prefix stay below 2^31)
   TWL_FOR_EACH_WEIGHT({
     const uint32_t u = __float_as_uint(w);
     if (u >= lo && u <= hi) atomicAdd(&imass[(u - lo) >> s], (uint32_t)(w * 1073741824.f));
   });
   __syncthreads();
-  // descending scan (thread t holds bins nb-1-4t .. nb-4-4t): the crossing bin
-  float mb[4], mine = 0.f;
+  // descending integer scan (thread t holds bins nb-1-16t .. nb-16-16t): the crossing bin
+  int mb[16], mine = 0;
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int b = nb - 1 - 4 * tid - e;
-    mb[e] = b >= 0 ? (float)imass[b] * 9.313225746154785e-10f : 0.f;
+  for (int e = 0; e < 16; ++e) {
+    const int b = nb - 1 - 16 * tid - e;
+    mb[e] = b >= 0 ? (int)imass[b] : 0;
     mine += mb[e];
   }
-  float x = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const float y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
   if (tid == 0) sh.state[3] = 0xFFFFFFFFu;
-  __syncthreads();
-  if (lane == 31) red[warp] = x;
-  __syncthreads();
-  float run = x - mine;
-  for (int w2 = 0; w2 < warp; ++w2) run += red[w2];
-  const float pf = (float)((double)P * 3.552713678800501e-15);  // P * 2^-48
+  int run = block_exclusive_scan(mine, sh.scan, nullptr);
+  const int p30 = (int)(P >> 18);  // P in units of 2^-30
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int b = nb - 1 - 4 * tid - e;
-    if (b >= 0 && run < pf && run + mb[e] >= pf) sh.state[3] = (uint32_t)b;
+  for (int e = 0; e < 16; ++e) {
+    const int b = nb - 1 - 16 * tid - e;
+    if (b >= 0 && run < p30 && run + mb[e] >= p30) sh.state[3] = (uint32_t)b;
     run += mb[e];
   }
   __syncthreads();
@@ -1168,7 +1239,7 @@ __device__ bool threshold_by_band(const float (&wr)[kR], bool in_regs, const flo
       c += (u >= band_lo && u <= band_hi) ? 1 : 0;
     });
     unsigned long long above = 0;
-    block_excl_u64(above_t, sh64, &above);
+    above = block_sum_u64(above_t, sh64);
     int n = 0;
     int pos = block_exclusive_scan(c, sh.scan, &n);
     ok = n <= kThreads && above < (unsigned long long)P;  // uniform
@@ -1183,19 +1254,10 @@ __device__ bool threshold_by_band(const float (&wr)[kR], bool in_regs, const flo
         }
       });
       __syncthreads();
-      float t = 0.f;
-      if (tid < n) {
-        const float vi = gv[tid];
-        unsigned long long m = above;
-        for (int j = 0; j < n; ++j) m += gv[j] >= vi ? (unsigned long long)gq[j] : 0ull;
-        t = m >= (unsigned long long)P ? vi : 0.f;
-      }
-      t = warp_max(t);
-      __syncthreads();
-      if (lane == 0) red[warp] = t;
-      __syncthreads();
-#pragma unroll
-      for (int w2 = 0; w2 < kWarps; ++w2) T = fmaxf(T, red[w2]);
+      // rank the band exactly (the approximate bins are no longer needed: their space is reused)
+      T = n <= kPairwiseMax ? rank_pairwise(gv, gq, n, above, P, red)
+                            : refine_threshold(gv, gq, n, band_lo, band_hi, above, P,
+                                               reinterpret_cast<uint32_t*>(fmass), sh, sh64);
       // no band weight reaching p means T lies below the band
       ok = T > 0.f;
     }
@@ -1231,6 +1293,27 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
   const bool staged = tail_off + ((4 * nc + 127) & ~127) + 16 * kHBins +
                           4 * (((nc + 31) >> 5) + 32) + 8 * (a.sel_words + 32) <=
                       smem_bytes;
+
+  // the head's selected-page bitmap and its prefix counts (for the page masks at the end), copied
+  // into shared memory now so that their latency overlaps the softmax
+  const Seq sq = load_seq(a.kv.seq_lens, bh / a.hq, a.kv.max_pages, a.flags, false);
+  const int nw = (sq.pages + 31) >> 5;
+  const int kw = (nc + 31) >> 5;
+  uint32_t* kws = reinterpret_cast<uint32_t*>(tail + (staged ? ((4 * nc + 127) & ~127) : 0) +
+                                              16 * kHBins);
+  uint32_t* sb = kws + ((kw + 31) & ~31);
+  int* sp = reinterpret_cast<int*>(sb + ((nw + 31) & ~31));
+  {
+    const int n4 = (nw + 3) >> 2;  // 16-byte pieces (rows are sel_words, a multiple of 4, long)
+    for (int w = tid; w < 2 * n4; w += kThreads) {
+      const bool second = w >= n4;
+      const int ww = 4 * (second ? w - n4 : w);
+      const void* src = second ? (const void*)(a.hpre + (size_t)bh * a.sel_words + ww)
+                               : (const void*)(a.selbits + (size_t)bh * a.sel_words + ww);
+      cp_async16(second ? (void*)(sp + ww) : (void*)(sb + ww), src, true);
+    }
+    cp_async_commit();
+  }
 
   const float p = a.p, eps = a.eps;
   const bool use_bound = nc > 0 && p < 1.f && (1.f - p) >= 1e-3f;
@@ -1359,17 +1442,26 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
     }
   }
   __syncthreads();  // the live set (or the weights) complete
+  // histogram scratch, after the staged weights
+  unsigned long long* hist =
+      reinterpret_cast<unsigned long long*>(tail + (staged ? ((4 * nc + 127) & ~127) : 0));
   float m;
   if (nc == 0 || p >= 1.f) {
     m = 0.f;  // keep every candidate
   } else if (from_live) {
-    m = top_p_from_live(lw, lq, nlive, L, p, eps, top, red);
-  } else {
-    // the threshold from exact bin masses over the weights >= L (histogram scratch after the
-    // staged weights)
+    // Every test of the search at mid > L counts only live weights, and mass(W >= t) is a
+    // non-increasing step function of t, so "mid <= L or mass(W >= mid) >= p" is the same test
+    // as "mid <= T" with T = max(L, the largest live weight v with mass(W >= v) >= p).
     const long long P = __double2ll_ru((double)p * 281474976710656.0);
-    unsigned long long* hist =
-        reinterpret_cast<unsigned long long*>(tail + (staged ? ((4 * nc + 127) & ~127) : 0));
+    const float T =
+        nlive <= kPairwiseMax
+            ? rank_pairwise(lw, lq, nlive, 0ull, P, red)
+            : refine_threshold(lw, lq, nlive, __float_as_uint(L), __float_as_uint(top), 0ull, P,
+                               reinterpret_cast<uint32_t*>(hist), sh, sh64);
+    m = bisect_scalar(top, fmaxf(L, T), eps);
+  } else {
+    // the threshold from exact bin masses over the weights >= L
+    const long long P = __double2ll_ru((double)p * 281474976710656.0);
     float T = 0.f;
     if (!threshold_by_band<kR>(wr, in_regs, W, staged, nc, __float_as_uint(L),
                                __float_as_uint(top), P, reinterpret_cast<float*>(hist), lw, lq,
@@ -1386,11 +1478,8 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
     if (a.threshold) a.threshold[bh] = m;
     if (a.cand_count) a.cand_count[bh] = nc;
   }
-  // kept-row bitmap of this head: bit i = (W_i >= m), in shared memory (after the staged
+  // kept-row bitmap of this head (kws): bit i = (W_i >= m), in shared memory (after the staged
   // weights and the histogram scratch)
-  const int kw = (nc + 31) >> 5;
-  uint32_t* kws = reinterpret_cast<uint32_t*>(tail + (staged ? ((4 * nc + 127) & ~127) : 0) +
-                                              16 * kHBins);
   int cnt = 0;
   if (from_live && m >= L) {
     // every kept candidate is live
@@ -1425,14 +1514,7 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
   // the head's kept rows of each selected page, ORed into the group's page masks (two pages per
   // word); the page of selection rank r is the r-th set bit of the head's bitmap, found from its
   // per-word prefix counts
-  const Seq sq = load_seq(a.kv.seq_lens, bh / a.hq, a.kv.max_pages, a.flags, false);
-  const int nw = (sq.pages + 31) >> 5;
-  uint32_t* sb = kws + ((kw + 31) & ~31);
-  int* sp = reinterpret_cast<int*>(sb + ((nw + 31) & ~31));
-  for (int w = tid; w < nw; w += kThreads) {
-    sb[w] = ldcg_u(a.selbits + (size_t)bh * a.sel_words + w);
-    sp[w] = ldcg_i(a.hpre + (size_t)bh * a.sel_words + w);
-  }
+  cp_async_wait_all();  // the bitmap and prefix counts copied at the start
   __syncthreads();
   uint32_t* pm = a.pmask + (size_t)g * a.pm_words;
   const int kbp = (nc + kPage - 1) / kPage;  // selected pages of the head
@@ -1548,11 +1630,14 @@ __device__ void build_kept(const Args& a, Shared& sh, int g, unsigned char* smem
   }
   TRACE_MARK(sh, 7);
   // publish the group's kept pages to the attention queue in nch chunks of about equal token
-  // counts (at most kAttChunkTok + 15 tokens each): page q opens chunk floor(pre(q) nch / ntok).
-  // As a page holds at most 16 tokens and a chunk about kAttChunkTok, consecutive pages open
-  // consecutive chunks and none is empty.  One empty chunk when nothing is kept, so the merge
-  // still writes the outputs.
-  const int nch = ntok > 0 ? (ntok + kAttChunkTok - 1) / kAttChunkTok : 1;
+  // counts: page q opens chunk floor(pre(q) nch / ntok).  A chunk is cut to about ntok /
+  // att_chunks tokens (the group's share of the workers, twice over), at least kAttChunkTok and
+  // at most kAttChunkMax (+15 at a page edge).  As a page holds at most 16 tokens and a chunk
+  // about ntok / nch >= kAttChunkTok / 2 = 64, consecutive pages open consecutive chunks and none
+  // is empty.  One empty chunk when nothing is kept, so the merge still writes the outputs.
+  int tgt = (ntok + a.att_chunks - 1) / a.att_chunks;
+  tgt = tgt < kAttChunkTok ? kAttChunkTok : (tgt > kAttChunkMax ? kAttChunkMax : tgt);
+  const int nch = ntok > 0 ? (ntok + tgt - 1) / tgt : 1;
   if (tid == 0) {
     if (a.union_count) a.union_count[g] = ntok;
     sh.total = (int)atomicAdd(a.sync + kQAlloc, (uint32_t)nch);
@@ -1598,24 +1683,52 @@ __device__ void build_kept(const Args& a, Shared& sh, int g, unsigned char* smem
 }
 
 // ------------------------------------------------------------------------------ attention
-// Kept pages [t0, t1) of group g (one chunk of the attention work list).  Their row masks are
-// expanded to the K/V row index of every kept token in shared memory; the rows (256 B of K and of V each) are copied with
-// 16-byte cp.async in passes of kAttPass tokens, two in flight, each row's 16-byte pieces XOR-
-// swizzled by the row number so that ldmatrix reads are free of bank conflicts.
-// The contraction runs on the tensor cores (mma.m16n8k16, fp16 in, fp32 accumulate).  S = Q K^T
-// takes the group's heads as the M rows (padded to 16 with zeros) and 8 tokens as N; its output
-// fragments are exactly the B operand of O^T += V^T P^T, which takes 16 channels as M, the tile's
-// 16 tokens as K and the heads as N, so no fragment is moved between the two products.  Warp w
-// takes the 16-token tile w / 2 of a pass for QK^T (both warps of a pair compute it) and the 64
-// channels (w % 2) of P.V.  P is split into an fp16 head and an fp16 tail (p - head), two
-// products, so its rounding stays near 2^-22 of the weights.  Each warp keeps its own running
-// (max, sum, o) per head; the warps' states are merged at the end into the chunk's partial.
+// The attention work list ([Notes] "Key designs", load balancing: the heads' kept tokens differ
+// ~50x, so each group's kept pages are cut into chunks that any CTA takes).  A worker is warp-
+// specialised: warps 8-15 produce, warps 0-7 consume, and the two sides meet only at mbarriers
+// on a ring of pass buffers, so that the copies of later passes are issued while earlier ones are
+// computed.
+//   * Producers take the chunks from the queue (ticket, wait until published), expand a chunk's
+//     kept pages to the K/V row index of every kept token (thread per page), and copy each pass
+//     of up to kAttPass tokens (256 B of K and of V per token, with 16-byte cp.async, each row's
+//     16-byte pieces XOR-swizzled by the row number so that ldmatrix reads are free of bank
+//     conflicts; the group's query rows too) into the next free buffer, with a descriptor (tokens,
+//     chunk, group, first / last pass of the chunk).  The buffer's full barrier completes when
+//     every producer thread's copies have landed.
+//   * Consumer warp w takes the 16-token tile w of a pass, on the tensor cores (mma.m16n8k16,
+//     fp16 in, fp32 accumulate): S^T = K Q^T takes the tile's tokens as the M rows and the heads
+//     (G <= 8) as N; the weights are moved by shuffles into the B operand of O^T += V^T P^T, which
+//     takes 16 channels as M (eight tiles), the 16 tokens as K and the heads as N.  P is split into
+//     an fp16 head and an fp16 tail (p - head), two products, so its rounding stays near 2^-22 of
+//     the weights.  Each warp keeps its own running (max, sum, o) of its lanes' heads (2t, 2t+1),
+//     and frees the buffer through its empty barrier.
+//   * At a chunk's last pass the consumers merge the warps' states into the chunk's partial
+//     [G][128 o, max, sum, -, -]; the chunk that completes its group merges the group's
+//     partials (log-sum-exp, in chunk order) into o and lse.
 constexpr int kAttPass = 128;
-constexpr int kAttIdx = 384;  // >= the tokens of a chunk (kAttChunkTok + 15)
-
-__device__ __forceinline__ uint32_t saddr(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
+constexpr int kAttIdx = kAttChunkMax + 16;
+constexpr int kAttPartStride = kHeadDim + 4;  // floats per head of a chunk partial
+constexpr int kAttCons = 256;                 // consumer threads (warps 0-7)
+constexpr int kAttProd = kThreads - kAttCons;  // producer threads (warps 8-15)
+constexpr int kAttBufBytes = kAttPass * 512 + 8 * 256;  // K rows | V rows | query rows
+constexpr uint32_t kMbarLimit = 1u << 22;      // polls of an mbarrier before a wait gives up
+// pass buffers in the ring (three when the merge scratch leaves room for them)
+template <int G>
+constexpr int att_bufs() {
+  return G >= 8 ? 2 : 3;
 }
+// shared memory of a worker: [bufs][kAttBufBytes] | [kAttIdx] row indices | scratch of the
+// consumers ([8 warps][2 G] max, sum | [8 warps][G][128] o)
+template <int G>
+constexpr int att_scratch_off() {
+  return att_bufs<G>() * kAttBufBytes + ((4 * kAttIdx + 127) & ~127);
+}
+template <int G>
+constexpr int att_smem() {
+  return att_scratch_off<G>() + 4 * 8 * (2 * G + G * kHeadDim);
+}
+enum { kDescEnd = 1, kDescFirst = 2, kDescLast = 4 };
+
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -1630,301 +1743,479 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
-
-template <int G>
-__device__ void attend_chunk(const Args& a, Shared& sh, int g, int t0, int t1, int slot,
-                             unsigned char* smem) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gr = lane >> 2, t = lane & 3;  // mma fragment row / column pair
-  const int tile = warp >> 1, hh = warp & 1;
-  const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
-  uint32_t* idx = reinterpret_cast<uint32_t*>(smem);
-  unsigned char* buf = smem + 4 * kAttIdx;
-  const int4* kp = a.kpages + (size_t)g * a.kv.max_pages;
-  // A fragments of the queries (rows = heads; rows >= G and the upper 8 rows are zero)
-  uint32_t qa[8][2];
-  {
-    const bool head_ok = gr < G;
-    const uint16_t* qh = a.q + ((size_t)b * a.hq + kvh * G + (head_ok ? gr : 0)) * kHeadDim;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      qa[ks][0] = head_ok ? __ldg(reinterpret_cast<const uint32_t*>(qh + 16 * ks + 2 * t)) : 0u;
-      qa[ks][1] = head_ok ? __ldg(reinterpret_cast<const uint32_t*>(qh + 16 * ks + 8 + 2 * t)) : 0u;
-    }
-  }
-  float M = -INFINITY, L = 0.f;  // softmax state of head gr (the QK^T row of this lane)
-  float ot[4][4];                // O^T: channels 64 hh + 16 mt + (gr, gr + 8), heads (2t, 2t+1)
-#pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) ot[mt][c] = 0.f;
-  const float sc_scale = a.sm_scale;
-  {
-    // the chunk's kept pages [t0, t1) expanded to K/V row indices, thread per page, in token order
-    int n = 0, tb = 0;
-    if (t1 > t0) {
-      const int4 f = ldcg_i4(kp + t0), l = ldcg_i4(kp + t1 - 1);
-      tb = f.w;
-      n = l.w + __popc((uint32_t)l.y) - tb;
-    }
-    for (int q = t0 + tid; q < t1; q += kThreads) {
-      const int4 e = ldcg_i4(kp + q);
-      uint32_t m = (uint32_t)e.y;
-      int pos = e.w - tb;
-      while (m) {
-        idx[pos++] = (uint32_t)e.x + (uint32_t)(__ffs(m) - 1);
-        m &= m - 1u;
-      }
-    }
-    __syncthreads();
-    TRACE_MARK(sh, 0);
-    const int npass = (n + kAttPass - 1) / kAttPass;
-    auto issue = [&](int k) {
-      unsigned char* kb = buf + (k & 1) * kAttPass * 512;
-      unsigned char* vb = kb + kAttPass * 256;
-      const int i0 = k * kAttPass, cn = min(kAttPass, n - i0);
-      for (int q = tid; q < 32 * kAttPass; q += kThreads) {
-        const int i = q >> 5, part = q & 31;
-        const uint32_t r = i < cn ? idx[i0 + i] : 0xFFFFFFFFu;
-        const bool okr = r != 0xFFFFFFFFu;
-        const size_t off = okr ? (size_t)r * kHeadDim : 0;
-        // a slot without a row reads zeros (its scores are masked; its V must not be inf)
-        if (part < 16)
-          cp_async16(kb + 256 * i + 16 * (part ^ (i & 7)), a.kv.k + off + 8 * part, okr);
-        else
-          cp_async16(vb + 256 * i + 16 * ((part - 16) ^ (i & 7)), a.kv.v + off + 8 * (part - 16),
-                     okr);
-      }
-      cp_async_commit();
-    };
-    issue(0);
-    if (npass > 1) issue(1);
+__device__ __forceinline__ void bar_named(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_inval(uint64_t* b) {
+  asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(saddr(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
+}
+// arrives once every cp.async this thread issued before has landed
+__device__ __forceinline__ void mbar_arrive_cp(uint64_t* b) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(saddr(b)) : "memory");
+}
+// one bounded poll (the thread may be suspended up to about a microsecond inside it)
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(saddr(b)), "r"(parity), "r"(1000u)
+      : "memory");
+  return ok != 0u;
+}
+// One thread: wait (bounded) for the phase of parity `parity` of b; false when the wait gave up
+// (which flags a timeout and aborts the step).  The ring's waits do not give up on an abort of
+// the step by others: the producers end the ring themselves (an end descriptor), so that every
+// consumer warp leaves at the same pass and the consumers' named barriers stay matched.
+__device__ bool mbar_wait(const Args& a, uint64_t* b, uint32_t parity) {
 #pragma unroll 1
-    for (int k = 0; k < npass; ++k) {
-      if (k + 1 < npass) asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-      else cp_async_wait_all();
-      __syncthreads();
-      TRACE_MARK(sh, 1);
-      const unsigned char* kb = buf + (k & 1) * kAttPass * 512;
-      const unsigned char* vb = kb + kAttPass * 256;
-      const int i0 = k * kAttPass, cn = min(kAttPass, n - i0);
-      const int tok0 = 16 * tile;  // this warp's tile
-      if (tok0 < cn) {             // warp-uniform
-        // S = Q K^T for the tile's two 8-token halves (rows = heads)
-        float s[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) s[nt][c] = 0.f;
-        const int mrow = lane & 7, mat = lane >> 3;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const int tk = tok0 + mrow + 8 * (mat >> 1), ch = 2 * ks + (mat & 1);
-          uint32_t kf[4];
-          ldsm_x4(kf, saddr(kb + 256 * tk + 16 * (ch ^ (tk & 7))));
-          const uint32_t av[4] = {qa[ks][0], 0u, qa[ks][1], 0u};
-          mma_16816(s[0], av, kf[0], kf[1]);
-          mma_16816(s[1], av, kf[2], kf[3]);
-        }
-        // mask, scale, online softmax of head gr over the tile's 16 tokens
-        float pv[2][2];
-        float mx = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int tk = tok0 + 8 * nt + 2 * t + c;
-            const bool valid = tk < cn && idx[i0 + (tk < cn ? tk : 0)] != 0xFFFFFFFFu;
-            pv[nt][c] = valid ? s[nt][c] * sc_scale : -INFINITY;
-            mx = fmaxf(mx, pv[nt][c]);
-          }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float nm = fmaxf(M, mx);
-        float scale = 1.f;
-        if (nm > -INFINITY) {  // the same in the four lanes of a row
-          scale = M > -INFINITY ? __expf(M - nm) : 0.f;
-          float rs = 0.f;
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              pv[nt][c] = __expf(pv[nt][c] - nm);
-              rs += pv[nt][c];
-            }
-          rs += __shfl_xor_sync(0xffffffffu, rs, 1);
-          rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-          L = L * scale + rs;
-          M = nm;
-        } else {
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) pv[nt][c] = 0.f;
-        }
-        // rescale O^T: this lane's columns are heads 2t and 2t+1, whose factors are held by the
-        // lanes of rows 2t (lane 8t) and 2t+1 (lane 8t+4)
-        const float f0 = __shfl_sync(0xffffffffu, scale, 8 * t);
-        const float f1 = __shfl_sync(0xffffffffu, scale, 8 * t + 4);
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
-          ot[mt][0] *= f0;
-          ot[mt][1] *= f1;
-          ot[mt][2] *= f0;
-          ot[mt][3] *= f1;
-        }
-        // P^T as the B operand (k = the tile's 16 tokens, n = head gr): fp16 head and tail
-        const uint32_t bh0 = pack_f16x2(pv[0][0], pv[0][1]);
-        const uint32_t bh1 = pack_f16x2(pv[1][0], pv[1][1]);
-        const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&bh0));
-        const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&bh1));
-        const uint32_t bl0 = pack_f16x2(pv[0][0] - h0.x, pv[0][1] - h0.y);
-        const uint32_t bl1 = pack_f16x2(pv[1][0] - h1.x, pv[1][1] - h1.y);
-        // O^T += V^T P^T over this warp's 64 channels (four 16-channel M tiles; A from
-        // ldmatrix.trans of the V rows)
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
-          const int tk = tok0 + mrow + 8 * (mat >> 1);
-          const int ch = 8 * hh + 2 * mt + (mat & 1);
-          uint32_t va[4];
-          ldsm_x4_t(va, saddr(vb + 256 * tk + 16 * (ch ^ (tk & 7))));
-          mma_16816(ot[mt], va, bh0, bh1);
-          mma_16816(ot[mt], va, bl0, bl1);
-        }
-      }
-      __syncthreads();  // the pass's buffer is read before it is refilled
-      if (k + 2 < npass) issue(k + 2);
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_test(b, parity)) return true;
+    if (it >= kMbarLimit) {
+      raise_flag(a.flags, TWL_FLAG_TIMEOUT);
+      atomicExch(a.sync + kAbort, 1u);
+      return false;
     }
   }
-  TRACE_MARK(sh, 2);
-  // merge the warps' states: smem [kWarps][16] (max, sum) and [kWarps][G][64] o
-  float* wm = reinterpret_cast<float*>(buf);
-  float* wl = wm + kWarps * 16;
-  float* wo = wl + kWarps * 16;
-  if (t == 0) {
-    wm[warp * 16 + gr] = M;
-    wl[warp * 16 + gr] = L;
+}
+
+// Consumer warp: one 16-token tile of a pass (cn tokens; K rows at kb, V rows at vb, the query
+// rows at qs) folded into the warp's running state of its lanes' heads (2t, 2t+1): max m[], sum
+// l[] (of this lane's tokens only) and O^T (channels 16 mt + gr (+8), heads 2t, 2t+1).
+template <int G>
+__device__ __forceinline__ void attend_tile(const unsigned char* kb, const unsigned char* vb,
+                                            const unsigned char* qs, int cn, float sc_scale,
+                                            float (&m)[2], float (&l)[2], float (&ot)[8][4]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gr = lane >> 2, t = lane & 3;  // mma fragment row / column pair
+  const int tok0 = 16 * warp;
+  if (tok0 >= cn) return;  // warp-uniform
+  const int mrow = lane & 7, mat = lane >> 3;
+  // S^T = K Q^T: A = the tile's K rows (ldmatrix), B = the query rows (head gr; zero for heads
+  // >= G)
+  const bool head_ok = gr < G;
+  const unsigned char* qh = qs + 256 * (head_ok ? gr : 0);
+  float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int tk = tok0 + mrow + 8 * (mat >> 1), ch = 2 * ks + (mat & 1);
+    uint32_t kf[4];
+    ldsm_x4(kf, saddr(kb + 256 * tk + 16 * (ch ^ (tk & 7))));
+    const uint32_t ka[4] = {kf[0], kf[2], kf[1], kf[3]};
+    const uint32_t q0 = head_ok ? *reinterpret_cast<const uint32_t*>(qh + 32 * ks + 4 * t) : 0u;
+    const uint32_t q1 = head_ok ? *reinterpret_cast<const uint32_t*>(qh + 32 * ks + 16 + 4 * t) : 0u;
+    mma_16816(s, ka, q0, q1);
+  }
+  // s[0], s[1]: token tok0 + gr, heads 2t, 2t + 1; s[2], s[3]: token tok0 + gr + 8
+  const bool v0 = tok0 + gr < cn, v1 = tok0 + gr + 8 < cn;
+  float x[4];
+  x[0] = v0 ? s[0] * sc_scale : -INFINITY;
+  x[1] = v0 ? s[1] * sc_scale : -INFINITY;
+  x[2] = v1 ? s[2] * sc_scale : -INFINITY;
+  x[3] = v1 ? s[3] * sc_scale : -INFINITY;
+  float f[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    float mx = fmaxf(x[e], x[2 + e]);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    const float nm = fmaxf(m[e], mx);  // finite: token tok0 is valid
+    f[e] = m[e] > -INFINITY ? __expf(m[e] - nm) : 0.f;
+    m[e] = nm;
+    x[e] = v0 ? __expf(x[e] - nm) : 0.f;
+    x[2 + e] = v1 ? __expf(x[2 + e] - nm) : 0.f;
+    l[e] = l[e] * f[e] + (x[e] + x[2 + e]);
   }
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt) {
-    const int c0 = 16 * mt + gr;  // channel within the warp's half
+  for (int mt = 0; mt < 8; ++mt) {
+    ot[mt][0] *= f[0];
+    ot[mt][1] *= f[1];
+    ot[mt][2] *= f[0];
+    ot[mt][3] *= f[1];
+  }
+  // P^T as the B operand (k = tokens, n = head gr): tokens 2t, 2t + 8 of head gr are held by
+  // lane 8t + gr / 2, tokens 2t + 1, 2t + 9 by lane 8t + 4 + gr / 2 (component gr & 1)
+  const int sa = 8 * t + (gr >> 1), sb = sa + 4;
+  const bool odd = gr & 1;
+  float pa0 = __shfl_sync(0xffffffffu, x[0], sa), pa1 = __shfl_sync(0xffffffffu, x[1], sa);
+  float pa2 = __shfl_sync(0xffffffffu, x[2], sa), pa3 = __shfl_sync(0xffffffffu, x[3], sa);
+  float pb0 = __shfl_sync(0xffffffffu, x[0], sb), pb1 = __shfl_sync(0xffffffffu, x[1], sb);
+  float pb2 = __shfl_sync(0xffffffffu, x[2], sb), pb3 = __shfl_sync(0xffffffffu, x[3], sb);
+  const float p_t0 = odd ? pa1 : pa0, p_t8 = odd ? pa3 : pa2;  // tokens 2t, 2t + 8
+  const float p_t1 = odd ? pb1 : pb0, p_t9 = odd ? pb3 : pb2;  // tokens 2t + 1, 2t + 9
+  const uint32_t bh0 = pack_f16x2(p_t0, p_t1), bh1 = pack_f16x2(p_t8, p_t9);
+  const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&bh0));
+  const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&bh1));
+  const uint32_t bl0 = pack_f16x2(p_t0 - h0.x, p_t1 - h0.y);
+  const uint32_t bl1 = pack_f16x2(p_t8 - h1.x, p_t9 - h1.y);
+  // O^T += V^T P^T over the eight 16-channel tiles (A from ldmatrix.trans of the V rows)
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int h = 2 * t + e;
-      if (h < G) {
-        wo[((size_t)warp * G + h) * 64 + c0] = ot[mt][e];
-        wo[((size_t)warp * G + h) * 64 + c0 + 8] = ot[mt][2 + e];
-      }
+  for (int mt = 0; mt < 8; ++mt) {
+    const int tk = tok0 + mrow + 8 * (mat >> 1);
+    const int ch = 2 * mt + (mat & 1);
+    uint32_t va[4];
+    ldsm_x4_t(va, saddr(vb + 256 * tk + 16 * (ch ^ (tk & 7))));
+    mma_16816(ot[mt], va, bh0, bh1);
+    mma_16816(ot[mt], va, bl0, bl1);
+  }
+}
+
+// Consumers (256 threads): the warps' states of a finished chunk -> its partial [G][o(128), max,
+// sum] in a.part (slot c).  scr: the consumers' scratch.
+template <int G>
+__device__ void attend_finish(const Args& a, int c, const float (&m)[2], float (&l)[2],
+                              const float (&ot)[8][4], float* scr) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gr = lane >> 2, t = lane & 3;
+  float* wm = scr;               // [8][G]
+  float* wl = wm + 8 * G;        // [8][G]
+  float* wo = wl + 8 * G;        // [8][G][128]
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    l[e] += __shfl_xor_sync(0xffffffffu, l[e], 4);
+    l[e] += __shfl_xor_sync(0xffffffffu, l[e], 8);
+    l[e] += __shfl_xor_sync(0xffffffffu, l[e], 16);
+    const int h = 2 * t + e;
+    if (gr == 0 && h < G) {
+      wm[warp * G + h] = m[e];
+      wl[warp * G + h] = l[e];
     }
   }
-  __syncthreads();
-  float* part = a.part + (size_t)slot * G * (kHeadDim + 2);
-  for (int i = tid; i < G * kHeadDim; i += kThreads) {
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int h = 2 * t + (e & 1), ch = 16 * mt + gr + 8 * (e >> 1);
+      if (h < G) wo[(warp * G + h) * kHeadDim + ch] = ot[mt][e];
+    }
+  bar_named(2, kAttCons);
+  float* part = a.part + (size_t)c * G * kAttPartStride;
+  for (int i = tid; i < G * kHeadDim; i += kAttCons) {
     const int h = i / kHeadDim, d = i - h * kHeadDim;
-    const int half = d >> 6, dd = d & 63;
     float mxw = -INFINITY;
 #pragma unroll
-    for (int tl = 0; tl < kWarps / 2; ++tl) mxw = fmaxf(mxw, wm[(2 * tl + half) * 16 + h]);
+    for (int w = 0; w < 8; ++w) mxw = fmaxf(mxw, wm[w * G + h]);
     float ov = 0.f, lv = 0.f;
     if (mxw > -INFINITY) {
 #pragma unroll
-      for (int tl = 0; tl < kWarps / 2; ++tl) {
-        const int w = 2 * tl + half;
-        const float mw = wm[w * 16 + h];
+      for (int w = 0; w < 8; ++w) {
+        const float mw = wm[w * G + h];
         if (!(mw > -INFINITY)) continue;
-        const float f = __expf(mw - mxw);
-        ov = fmaf(f, wo[((size_t)w * G + h) * 64 + dd], ov);
-        lv = fmaf(f, wl[w * 16 + h], lv);
+        const float fw = __expf(mw - mxw);
+        ov = fmaf(fw, wo[(w * G + h) * kHeadDim + d], ov);
+        lv = fmaf(fw, wl[w * G + h], lv);
       }
     }
-    part[h * (kHeadDim + 2) + 2 + d] = ov;
+    part[h * kAttPartStride + d] = ov;
     if (d == 0) {
-      part[h * (kHeadDim + 2) + 0] = mxw;
-      part[h * (kHeadDim + 2) + 1] = lv;
+      part[h * kAttPartStride + kHeadDim] = mxw;
+      part[h * kAttPartStride + kHeadDim + 1] = lv;
     }
   }
 }
 
-// Run by the CTA whose chunk completed its group: log-sum-exp merge of the group's chunk
-// partials, in chunk order -> o, lse of every head (o = 0, lse = -inf when nothing was kept).
+// Consumers (256 threads), in the CTA whose chunk completed group g: log-sum-exp merge of the
+// group's nch chunk partials (slots c0 ...) -> o, lse of every head (o = 0, lse = -inf when
+// nothing was kept).  Warp h finds head h's max and total; then each float4 of o is summed by
+// 8 / G threads over interleaved chunks (loads independent of the sums, so they stay in flight
+// together) and their sums are added in a fixed order.  scr: the consumers' scratch.
 template <int G>
-__device__ void merge_group(const Args& a, int g, int c0, int nch) {
+__device__ void merge_group(const Args& a, int g, int c0, int nch, float* scr) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
-  for (int i = threadIdx.x; i < G * kHeadDim; i += kThreads) {
-    const int h = i / kHeadDim, d = i - h * kHeadDim;
-    const float* base = a.part + (size_t)c0 * G * (kHeadDim + 2) + h * (kHeadDim + 2);
-    const size_t stride = (size_t)G * (kHeadDim + 2);
-    float Mx = -INFINITY;
-    for (int ai = 0; ai < nch; ++ai) {
-      const float* pp = base + ai * stride;
-      if (ldcg_f(pp + 1) > 0.f) Mx = fmaxf(Mx, ldcg_f(pp));
+  const float* part = a.part + (size_t)c0 * G * kAttPartStride;
+  float* hs = scr;                                      // [G] head max, [G] head total
+  float4* red = reinterpret_cast<float4*>(scr + 16);    // [kAttCons]
+  if (warp < G) {
+    float mx = -INFINITY;
+    for (int c = lane; c < nch; c += 32) {
+      const float* pp = part + (size_t)(c * G + warp) * kAttPartStride + kHeadDim;
+      if (ldcg_f(pp + 1) > 0.f) mx = fmaxf(mx, ldcg_f(pp));
     }
-    float o = 0.f, l = 0.f;
-    if (Mx > -INFINITY) {
-      for (int ai = 0; ai < nch; ++ai) {
-        const float* pp = base + ai * stride;
-        const float la = ldcg_f(pp + 1);
-        if (!(la > 0.f)) continue;
-        const float wgt = __expf(ldcg_f(pp) - Mx);
-        o = fmaf(wgt, ldcg_f(pp + 2 + d), o);
-        l = fmaf(wgt, la, l);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float tot = 0.f;
+    if (mx > -INFINITY)
+      for (int c = lane; c < nch; c += 32) {
+        const float* pp = part + (size_t)(c * G + warp) * kAttPartStride + kHeadDim;
+        const float lc = ldcg_f(pp + 1);
+        if (lc > 0.f) tot = fmaf(__expf(ldcg_f(pp) - mx), lc, tot);
       }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    if (lane == 0) {
+      hs[warp] = mx;
+      hs[G + warp] = tot;
     }
+  }
+  bar_named(2, kAttCons);
+  constexpr int kCols = G * kHeadDim / 4, kPer = kAttCons / kCols;
+  const int col = tid % kCols, r = tid / kCols, h = col / (kHeadDim / 4);
+  const float mx = hs[h];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (mx > -INFINITY) {
+#pragma unroll 8
+    for (int c = r; c < nch; c += kPer) {
+      const float* pp = part + (size_t)(c * G + h) * kAttPartStride;
+      const float lc = ldcg_f(pp + kHeadDim + 1);
+      const float w = lc > 0.f ? __expf(ldcg_f(pp + kHeadDim) - mx) : 0.f;
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(pp) + (col % (kHeadDim / 4)));
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+  }
+  red[tid] = acc;
+  bar_named(2, kAttCons);
+  if (r == 0) {
+#pragma unroll
+    for (int k = 1; k < kPer; ++k) {
+      const float4 v = red[k * kCols + col];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    const float lt = hs[G + h];
+    const bool any = lt > 0.f;
     const size_t bh = (size_t)b * a.hq + kvh * G + h;
-    const bool any = l > 0.f;
-    a.o[bh * kHeadDim + d] = any ? o / l : 0.f;
-    if (d == 0) a.lse[bh] = any ? Mx + __logf(l) : -INFINITY;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (any) o = make_float4(acc.x / lt, acc.y / lt, acc.z / lt, acc.w / lt);
+    reinterpret_cast<float4*>(a.o + bh * kHeadDim)[col % (kHeadDim / 4)] = o;
+    if (col % (kHeadDim / 4) == 0) a.lse[bh] = any ? mx + __logf(lt) : -INFINITY;
+  }
+  bar_named(2, kAttCons);  // the scratch is reused
+}
+
+// Thread 0: the state of queue ticket c: 1 = its chunk is published, -1 = there is none (every
+// group has published and c is past the end, or the step was aborted), 0 = not yet.
+__device__ __forceinline__ int ticket_state(const Args& a, int c) {
+  if (c < a.q_cap && ld_acquire(a.qvalid + c) != 0u) return 1;
+  if (ld_acquire(a.sync + kQGroups) >= (uint32_t)a.groups &&
+      (uint32_t)c >= ld_acquire(a.sync + kQAlloc))
+    return -1;
+  if (ld_acquire(a.sync + kAbort) != 0u) return -1;
+  return 0;
+}
+
+// Thread 0: wait (bounded) until ticket c is decided; 1 = published, -1 = none.
+__device__ int ticket_wait(const Args& a, int c) {
+#pragma unroll 1
+  for (uint32_t it = 0;; ++it) {
+    const int st = ticket_state(a, c);
+    if (st != 0) return st;
+    if (it >= kSpinLimit) {
+      raise_flag(a.flags, TWL_FLAG_TIMEOUT);
+      atomicExch(a.sync + kAbort, 1u);
+      return -1;
+    }
+    __nanosleep(64);
   }
 }
 
-// One worker of the flattened attention work list ([Notes] "Key designs", load balancing: the
-// heads' kept tokens differ ~50x, so they are cut into equal chunks that any CTA takes): take the
-// next chunk number, wait until it is published (or until every group has published and the
-// number is past the end), attend over it, and merge the group when its last chunk is done.
+// Producers (warps 8-15): take chunks until the queue is done, copy their passes into the ring,
+// then post the end.
 template <int G>
-__device__ void attend_worker(const Args& a, Shared& sh, unsigned char* smem) {
+__device__ void attend_produce(const Args& a, Shared& sh, unsigned char* smem) {
+  constexpr int NB = att_bufs<G>();
+  const int pt = threadIdx.x - kAttCons;
+  uint32_t* idx = reinterpret_cast<uint32_t*>(smem + NB * kAttBufBytes);
+  int j = 0;  // passes posted
+  bool ok = true;
 #pragma unroll 1
   for (;;) {
-    if (threadIdx.x == 0) {
+    // the next chunk
+    if (pt == 0) {
       const int c = (int)atomicAdd(a.sync + kQNext, 1u);
-      int got = -1;
-      uint32_t it = 0;
-      for (;;) {
-        if (c < a.q_cap && ld_acquire(a.qvalid + c) != 0u) {
-          got = c;
-          break;
-        }
-        if (ld_acquire(a.sync + kQGroups) >= (uint32_t)a.groups &&
-            (uint32_t)c >= ld_acquire(a.sync + kQAlloc))
-          break;  // every group published and this number is past the end
-        if ((++it & 31u) == 0u) {
-          if (ld_acquire(a.sync + kAbort) != 0u) break;
-          if (it >= kSpinLimit) {
-            raise_flag(a.flags, TWL_FLAG_TIMEOUT);
-            atomicExch(a.sync + kAbort, 1u);
-            break;
-          }
-        }
-        __nanosleep(64);
+      const int st = ticket_wait(a, c);
+      sh.att[0][0] = st > 0 ? c : -1;
+      if (st > 0) {
+        const int* e = a.qtab + 4 * (size_t)c;
+        sh.att[0][1] = ldcg_i(e);
+        sh.att[0][2] = ldcg_i(e + 1);
+        sh.att[0][3] = ldcg_i(e + 2);
       }
-      sh.flag = got;
+    }
+    bar_named(1, kAttProd);
+    const int c = sh.att[0][0], g = sh.att[0][1], p0 = sh.att[0][2], p1 = sh.att[0][3];
+    bar_named(1, kAttProd);  // read before the next chunk's entry is written
+    int n = 0, np = 1;
+    if (c >= 0) {
+      // expand the chunk's pages to row indices (token order)
+      const int4* kp = a.kpages + (size_t)g * a.kv.max_pages;
+      int tb = 0;
+      if (p1 > p0) {
+        const int4 f = ldcg_i4(kp + p0), ls = ldcg_i4(kp + p1 - 1);
+        tb = f.w;
+        n = ls.w + __popc((uint32_t)ls.y) - tb;
+      }
+      for (int q = p0 + pt; q < p1; q += kAttProd) {
+        const int4 en = ldcg_i4(kp + q);
+        uint32_t mk = (uint32_t)en.y;
+        int pos = en.w - tb;
+        while (mk) {
+          idx[pos++] = (uint32_t)en.x + (uint32_t)(__ffs(mk) - 1);
+          mk &= mk - 1u;
+        }
+      }
+      bar_named(1, kAttProd);
+      np = n > 0 ? (n + kAttPass - 1) / kAttPass : 1;
+    }
+    const int b_ = g / a.kv.hkv, kvh = g - b_ * a.kv.hkv;
+#pragma unroll 1
+    for (int k = 0; k < np; ++k, ++j) {
+      const int bs = j % NB, u = j / NB;
 #ifdef TWL_STEP_TRACE
-      sh.t_ready = now_ns();
+      const unsigned long long tp0 = now_ns();
+#endif
+      if (u > 0) {  // the buffer's previous pass consumed (thread 0 waits for all)
+        if (pt == 0) sh.att_prod_ok = mbar_wait(a, &sh.att_empty[bs], (uint32_t)((u - 1) & 1));
+        bar_named(1, kAttProd);
+        ok = sh.att_prod_ok != 0;
+        bar_named(1, kAttProd);
+        if (!ok) break;
+      }
+#ifdef TWL_STEP_TRACE
+      const unsigned long long tp1 = now_ns();
+#endif
+      unsigned char* kb = smem + bs * kAttBufBytes;
+      unsigned char* vb = kb + kAttPass * 256;
+      unsigned char* qb = kb + kAttPass * 512;
+      if (c >= 0) {
+        const int cn = min(kAttPass, n - k * kAttPass);
+        const int rows = (cn + 15) & ~15;  // rows past cn in the last tile read zeros
+        const uint32_t* ix = idx + k * kAttPass;
+        for (int q = pt; q < 32 * rows; q += kAttProd) {
+          const int i = q >> 5, part = q & 31;
+          const bool okr = i < cn;
+          const size_t off = okr ? (size_t)ix[i] * kHeadDim : 0;
+          if (part < 16)
+            cp_async16(kb + 256 * i + 16 * (part ^ (i & 7)), a.kv.k + off + 8 * part, okr);
+          else
+            cp_async16(vb + 256 * i + 16 * ((part - 16) ^ (i & 7)),
+                       a.kv.v + off + 8 * (part - 16), okr);
+        }
+        if (pt < G * 16) {
+          const int row = pt >> 4, piece = pt & 15;
+          cp_async16(qb + 256 * row + 16 * piece,
+                     a.q + ((size_t)b_ * a.hq + kvh * G + row) * kHeadDim + 8 * piece, true);
+        }
+        if (pt == 0) {
+          sh.att_desc[bs][0] = cn;
+          sh.att_desc[bs][1] = c;
+          sh.att_desc[bs][2] = g;
+          sh.att_desc[bs][3] = (k == 0 ? kDescFirst : 0) | (k == np - 1 ? kDescLast : 0);
+        }
+      } else if (pt == 0) {
+        sh.att_desc[bs][3] = kDescEnd;
+      }
+      mbar_arrive_cp(&sh.att_full[bs]);
+      if (pt == 0) mbar_arrive(&sh.att_full[bs]);
+#ifdef TWL_STEP_TRACE
+      if (pt == 0 && a.trace && j < 16) {
+        unsigned long long* pr = a.trace + 17 * (size_t)a.n_items + 96 * (size_t)blockIdx.x + 6 * j;
+        pr[0] = tp0;
+        pr[1] = tp1;
+        pr[2] = now_ns();
+      }
 #endif
     }
-    __syncthreads();
-    const int c = sh.flag;
-    __syncthreads();
-    if (c < 0) break;
-    const int* e = a.qtab + 4 * (size_t)c;
-    const int g = ldcg_i(e), t0 = ldcg_i(e + 1), t1 = ldcg_i(e + 2);
-    const int c0 = ldcg_i(a.cbase + 2 * g), nch = ldcg_i(a.cbase + 2 * g + 1);
-    attend_chunk<G>(a, sh, g, t0, t1, c, smem);
-    if (block_signal_last(sh, counter(a, kCntAttend, g), (uint32_t)nch)) {
-      TRACE_MARK(sh, 5);
-      merge_group<G>(a, g, c0, nch);
-    }
+    if (c < 0 || !ok) break;
   }
+  cp_async_wait_all();
+}
+
+// Consumers (warps 0-7): compute the posted passes until the end; at a chunk's last pass write
+// its partial, count it, and merge the group when it is the last.
+template <int G>
+__device__ void attend_consume(const Args& a, Shared& sh, unsigned char* smem) {
+  constexpr int NB = att_bufs<G>();
+  const int tid = threadIdx.x, lane = tid & 31;
+  float* scr = reinterpret_cast<float*>(smem + att_scratch_off<G>());
+  const float sc_scale = a.sm_scale;
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+  float ot[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) ot[mt][e] = 0.f;
+#pragma unroll 1
+  for (int j = 0;; ++j) {
+    const int bs = j % NB, u = j / NB;
+#ifdef TWL_STEP_TRACE
+    const unsigned long long tc0 = now_ns();
+#endif
+    int got = 0;
+    if (lane == 0) got = mbar_wait(a, &sh.att_full[bs], (uint32_t)(u & 1));
+    got = __shfl_sync(0xffffffffu, got, 0);
+    if (!got) break;
+    // the other lanes acquire the phase too (it is complete: the poll returns at once)
+    if (lane != 0) mbar_test(&sh.att_full[bs], (uint32_t)(u & 1));
+    const int flags = sh.att_desc[bs][3];
+    if (flags & kDescEnd) break;
+    const int cn = sh.att_desc[bs][0], c = sh.att_desc[bs][1], g = sh.att_desc[bs][2];
+#ifdef TWL_STEP_TRACE
+    const unsigned long long tc1 = now_ns();
+#endif
+    if (flags & kDescFirst) {
+      m[0] = m[1] = -INFINITY;
+      l[0] = l[1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ot[mt][e] = 0.f;
+    }
+    const unsigned char* kb = smem + bs * kAttBufBytes;
+    attend_tile<G>(kb, kb + kAttPass * 256, kb + kAttPass * 512, cn, sc_scale, m, l, ot);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.att_empty[bs]);
+#ifdef TWL_STEP_TRACE
+    if (tid == 0 && a.trace && j < 16) {
+      unsigned long long* pr = a.trace + 17 * (size_t)a.n_items + 96 * (size_t)blockIdx.x + 6 * j;
+      pr[3] = tc0;
+      pr[4] = tc1;
+      pr[5] = now_ns();
+    }
+#endif
+    if (!(flags & kDescLast)) continue;
+    attend_finish<G>(a, c, m, l, ot, scr);
+    const int c0 = ldcg_i(a.cbase + 2 * g), nch = ldcg_i(a.cbase + 2 * g + 1);
+    bar_named(2, kAttCons);  // every consumer's partial writes before the count
+    if (tid == 0) sh.att_last = atom_acq_rel_add(counter(a, kCntAttend, g), 1u) + 1u == (uint32_t)nch;
+    bar_named(2, kAttCons);
+    if (sh.att_last) merge_group<G>(a, g, c0, nch, scr);
+  }
+}
+
+// A worker of the attention queue (one per CTA, after its other items).
+template <int G>
+__device__ void attend_worker(const Args& a, Shared& sh, unsigned char* smem) {
+  constexpr int NB = att_bufs<G>();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NB; ++i) {
+      mbar_init(&sh.att_full[i], kAttProd + 1);
+      mbar_init(&sh.att_empty[i], kAttCons / 32);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x >= kAttCons) attend_produce<G>(a, sh, smem);
+  else attend_consume<G>(a, sh, smem);
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int i = 0; i < NB; ++i) {
+      mbar_inval(&sh.att_full[i]);
+      mbar_inval(&sh.att_empty[i]);
+    }
 }
 
 // ------------------------------------------------------------------------------ the kernel
@@ -2050,10 +2341,10 @@ int smem_need(int g, int max_pages, int max_budget, int s_chunk) {
   const int est_kw = kEstMeta / 32 + 1;
   const int est = ((4 * ((2 + g) * kEstMeta + (2 * g + 2) * est_kw + 1) + 127) & ~127) +
                   2 * kEstPass * 1088;
-  const int att = 4 * kAttIdx + 2 * kAttPass * 512;
-  const int att_merge = 4 * kAttIdx + 4 * (2 * kWarps * 16 + kWarps * g * 64);
   int need = topk;
-  for (int x : {prune, score, est, att, att_merge}) need = need > x ? need : x;
+  const int att = g == 1 ? att_smem<1>() : g == 2 ? att_smem<2>() : g == 4 ? att_smem<4>()
+                                                                        : att_smem<8>();
+  for (int x : {prune, score, est, att}) need = need > x ? need : x;
   return need;
 }
 
@@ -2078,7 +2369,7 @@ Plan plan(int batch, int hq, int hkv, int max_pages, int max_budget) {
   Plan pl{};
   const int g = hq / hkv;
   const int groups = batch * hkv;
-  pl.sel_words = (max_pages + 31) / 32;
+  pl.sel_words = ((max_pages + 31) / 32 + 3) & ~3;  // rows of whole 16-byte pieces
   pl.cand_stride = kPage * max_budget;
   pl.kept_words = (pl.cand_stride + 31) / 32;
   const int sms = num_sms();
@@ -2110,6 +2401,8 @@ Plan plan(int batch, int hq, int hkv, int max_pages, int max_budget) {
   // attention chunks: at most one per kAttChunkTok kept tokens of each group plus one, and the
   // numbers the workers take past the end
   pl.q_cap = groups * (1 + (kPage * max_pages + kAttChunkTok - 1) / kAttChunkTok) + sms + 32;
+  pl.att_chunks = 2 * sms / groups;
+  pl.att_chunks = pl.att_chunks < 1 ? 1 : pl.att_chunks;
   return pl;
 }
 
@@ -2129,7 +2422,8 @@ Layout layout(const Plan& pl, int batch, int hq, int hkv, int max_pages) {
     return o;
   };
 #ifdef TWL_STEP_TRACE
-  L.trace = take(8 * 17 * (size_t)(groups * (pl.s_per + 2 * g + pl.e_per) + pl.grid));
+  L.trace = take(8 * 17 * (size_t)(groups * (pl.s_per + 2 * g + pl.e_per) + pl.grid) +
+                 8 * 96 * (size_t)pl.grid);
 #endif
   L.sync = take(4 * (kSyncHead + kCounters * groups));
   L.keys = take(4 * bh * max_pages);
@@ -2142,7 +2436,7 @@ Layout layout(const Plan& pl, int batch, int hq, int hkv, int max_pages) {
   L.qtab = take(16 * (size_t)pl.q_cap);
   L.qvalid = take(4 * (size_t)pl.q_cap);
   L.cbase = take(8 * groups);
-  L.part = take(4 * (size_t)pl.q_cap * g * (kHeadDim + 2));
+  L.part = take(4 * (size_t)pl.q_cap * g * kAttPartStride);
   L.total = off;
   return L;
 }
@@ -2182,6 +2476,7 @@ void carve(Args& a, char* ws, const Plan& pl, int batch, int hq, int hkv, int ma
   a.e_per = pl.e_per;
   a.e_chunk = pl.e_chunk;
   a.q_cap = pl.q_cap;
+  a.att_chunks = pl.att_chunks;
   a.smem_bytes = pl.smem_bytes;
   // the work list, kind by kind (every item depends only on items of earlier kinds)
   // the work list, kind by kind (every item depends only on items of earlier kinds); the last

@@ -31,9 +31,10 @@ constexpr int kMaxSegments = 40;
 //   kQAlloc  attention chunks published (allocated)    kQNext  chunks taken by workers
 //   kQGroups groups whose chunks are published
 enum { kNext = 0, kExit = 1, kAbort = 2, kQAlloc = 3, kQNext = 4, kQGroups = 5, kSyncHead = 8 };
-// Kept tokens per attention chunk of the flattened work list (chunks are cut at page bounds into
-// pieces of about this many tokens).
-constexpr int kAttChunkTok = 256;
+// Kept tokens per attention chunk of the flattened work list: chunks are cut at page bounds, to
+// at least kAttChunkTok and at most kAttChunkMax tokens (+15 at a page edge).
+constexpr int kAttChunkTok = 128;
+constexpr int kAttChunkMax = 1024;
 enum { kCntScore = 0, kCntTopK, kCntEst, kCntPrune, kCntAttend, kCounters };
 
 struct Args {
@@ -79,6 +80,7 @@ struct Args {
   // strides and the work list
   int groups, sel_words, cand_stride, kept_words, pm_words;
   int s_per, s_chunk, e_per, e_chunk, q_cap;
+  int att_chunks;  // chunks a group's kept tokens are cut into, before the size limits
   int n_items;
   int smem_bytes;  // dynamic shared memory of each CTA
   int nseg;
@@ -88,7 +90,7 @@ struct Args {
 struct Plan {
   int grid;        // CTAs (all resident at once)
   int smem_bytes;  // dynamic shared memory per CTA
-  int s_per, s_chunk, e_per, e_chunk, q_cap;
+  int s_per, s_chunk, e_per, e_chunk, q_cap, att_chunks;
   int sel_words, cand_stride, kept_words;
   bool ok;
 };
