@@ -319,9 +319,19 @@ twl_status twl_sparse_decode_noalloc(const void* q, int32_t num_q_heads, const t
 
 /* ---------------------------------------------------------------- the whole step
  * select -> estimate -> prune (p, eps) -> group union -> attend, with sm_scale = 1/sqrt(128)
- * ([Notes] "Overall framework"; [Summary] 4.1 and Figure 5).  Results equal running the five
- * calls above in sequence.  max_budget: as for twl_select_pages (>= every k_b).
- *   o float [B][Hq][128] out; lse float [B][Hq] out; stats optional (see twl_step_stats). */
+ * ([Notes] "Overall framework"; [Summary] 4.1 and Figure 5), as one persistent launch over every
+ * SM.  The selections, candidates and weights equal those of the five calls above in sequence;
+ * the threshold m is the bisection's result computed from exact fixed-point masses (units of
+ * 2^-48, each weight rounded to that unit), so it can differ from twl_prune_top_p's only when p
+ * is within that rounding (n * 2^-49 for n candidates) of a prefix mass.
+ * max_budget: as for twl_select_pages (>= every k_b).
+ *   o float [B][Hq][128] out; lse float [B][Hq] out; stats optional (see twl_step_stats).
+ * The workspace (TWL_OP_DECODE_STEP bytes, zeroed once by twl_workspace_init) carries the
+ * launch's synchronisation words, which every launch leaves cleared for the next; launches on
+ * one workspace must be stream-ordered.  Device-side errors are reported through the workspace
+ * flags (twl_device_status): page-table entries outside the pool and bad sequence lengths are
+ * skipped (TWL_FLAG_BAD_INDEX); a wait between work items that gives up after its bounded number
+ * of polls aborts the launch (TWL_FLAG_TIMEOUT, outputs undefined). */
 twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
                            const twl_k_aux* aux, int32_t budget_pages, int32_t budget_div,
                            int32_t max_budget, float p, float eps, float* o, float* lse,

@@ -561,7 +561,8 @@ def test_decode_step_repeated_launches_on_one_workspace():
 
 
 def test_decode_step_more_groups_than_sms():
-    """320 (sequence, kv-head) groups: the 256-thread build is chosen; sampled groups."""
+    """320 (sequence, kv-head) groups, more than twice the SMs: several items of every kind per
+    CTA; sampled groups."""
     lens = [300 + 37 * i for i in range(40)]
     wl = synth.make_decode("many_groups", 40, 32, 8, lens, seed=29, permute_pages=True)
     layer = DecodeLayer.from_workload(wl)
