@@ -403,8 +403,10 @@ __device__ void topk_bits(const uint32_t* keys, int n_pages, int kb, uint32_t* s
   const int nw = (n_pages + 31) >> 5;
   constexpr int kGatherCap = 64;
   constexpr int kBins = 4096;
-  uint32_t* hh = reinterpret_cast<uint32_t*>(scratch);  // [kBins]
-  uint32_t* gkey = hh + kBins;                          // [kGatherCap]
+  // the bins, one padding word after every 8 (bin b at word b + b / 8), so that the scan's
+  // per-thread runs of 8 bins start 9 words apart and load free of bank conflicts
+  uint32_t* hh = reinterpret_cast<uint32_t*>(scratch);  // [kBins + kBins / 8]
+  uint32_t* gkey = hh + kBins + kBins / 8;              // [kGatherCap]
   int* gidx = reinterpret_cast<int*>(gkey + kGatherCap);  // [kGatherCap]
   (void)scratch_bytes;
   uint32_t blo, bhi;
@@ -441,23 +443,26 @@ __device__ void topk_bits(const uint32_t* keys, int n_pages, int kb, uint32_t* s
     const uint32_t range = bhi - blo;
     const int width = 32 - __clz(range);
     const int sh_ = width > 12 ? width - 12 : 0;
-    for (int i = tid; i < kBins; i += kThreads) hh[i] = 0u;
+    for (int i = tid; i < kBins + kBins / 8; i += kThreads) hh[i] = 0u;
     __syncthreads();
     for (int i = tid; i < n_pages; i += kThreads) {
       const uint32_t key = keys[i];
-      if (key >= blo && key <= bhi) atomicAdd(&hh[(key - blo) >> sh_], 1u);
+      if (key >= blo && key <= bhi) {
+        const uint32_t b = (key - blo) >> sh_;
+        atomicAdd(&hh[b + (b >> 3)], 1u);
+      }
     }
     __syncthreads();
     // descending scan over the bins: thread t owns bins kBins-1-kPerT*t ... kBins-kPerT*(t+1)
     const int b0 = kBins - 1 - kPerT * tid;
     int mine = 0;
 #pragma unroll
-    for (int e = 0; e < kPerT; ++e) mine += (int)hh[b0 - e];
+    for (int e = 0; e < kPerT; ++e) mine += (int)hh[(b0 - e) + ((b0 - e) >> 3)];
     const int excl = block_exclusive_scan(mine, sh.scan, nullptr);
     if (excl < remaining && remaining <= excl + mine) {
       int run = excl;
       for (int e = 0; e < kPerT; ++e) {
-        const int c = (int)hh[b0 - e];
+        const int c = (int)hh[(b0 - e) + ((b0 - e) >> 3)];
         if (run + c >= remaining) {
           sh.state[0] = (uint32_t)(b0 - e);
           sh.state[1] = (uint32_t)(remaining - run);
@@ -968,6 +973,8 @@ __device__ float rank_pairwise(const float* gv, const long long* gq, int n,
   return T;
 }
 constexpr int kPairwiseMax = 384;  // rank_pairwise up to this many weights, refine_threshold above
+constexpr int kHBins = 2048;                 // bins of the exact histograms
+constexpr int kPadBins = kHBins + kHBins / 4;  // words per part of a padded kHBins histogram
 
 // T among n <= kThreads weights gv (fixed-point copies gq, units of 2^-48) whose keys (float
 // bits) lie in [lo, hi], given the exact mass `above` of the weights with keys above hi: the
@@ -991,26 +998,28 @@ __device__ float refine_threshold(const float* gv, const long long* gq, int n, u
     const int bits = 32 - __clz(width);
     const int s = bits > 11 ? bits - 11 : 0;
     const int nb = (int)(width >> s) + 1;
-    for (int i = tid; i < nb; i += kThreads) {
+    // bin b at word b + b / 4 of each part (the scan's runs of 4 bins load conflict-free)
+    for (int i = tid; i < kPadBins; i += kThreads) {
       bins[i] = 0u;
-      bins[2048 + i] = 0u;
-      bins[4096 + i] = 0u;
+      bins[kPadBins + i] = 0u;
+      bins[2 * kPadBins + i] = 0u;
     }
     __syncthreads();
     if (mine && u >= lo && u <= hi) {
       const int b = (int)((u - lo) >> s);
-      atomicAdd(&bins[b], (uint32_t)(q & 0xFFFFu));
-      atomicAdd(&bins[2048 + b], (uint32_t)((q >> 16) & 0xFFFFu));
-      atomicAdd(&bins[4096 + b], (uint32_t)(q >> 32));
+      const int bp = b + (b >> 2);
+      atomicAdd(&bins[bp], (uint32_t)(q & 0xFFFFu));
+      atomicAdd(&bins[kPadBins + bp], (uint32_t)((q >> 16) & 0xFFFFu));
+      atomicAdd(&bins[2 * kPadBins + bp], (uint32_t)(q >> 32));
     }
     __syncthreads();
     // descending scan: thread t holds bins nb-1-4t .. nb-4-4t
     unsigned long long mb[4], tot = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int b = nb - 1 - 4 * tid - e;
-      mb[e] = b >= 0 ? (unsigned long long)bins[b] + ((unsigned long long)bins[2048 + b] << 16) +
-                           ((unsigned long long)bins[4096 + b] << 32)
+      const int b = nb - 1 - 4 * tid - e, bp = b + (b >> 2);
+      mb[e] = b >= 0 ? (unsigned long long)bins[bp] + ((unsigned long long)bins[kPadBins + bp] << 16) +
+                           ((unsigned long long)bins[2 * kPadBins + bp] << 32)
                      : 0ull;
       tot += mb[e];
     }
@@ -1050,7 +1059,6 @@ __device__ float refine_threshold(const float* gv, const long long* gq, int n, u
 // on its finer bits.  Returns 0 when even all counted weights fall
 // short of p.  Weights come from registers (row k * kThreads + tid) or from W (shared or global);
 // `mass` needs 4 * 2048 32-bit words, gv / gq kThreads entries each.
-constexpr int kHBins = 2048;
 template <int kR>
 __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const float* W,
                                    bool staged, int nc, uint32_t lo, uint32_t hi, long long P,
@@ -1082,18 +1090,21 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
     const int bits = 32 - __clz(width);
     const int s = bits > 11 ? bits - 11 : 0;
     const int nb = (int)(width >> s) + 1;
-    uint32_t* part = reinterpret_cast<uint32_t*>(mass);  // [4][kHBins] 12-bit part sums
-    for (int i = tid; i < 4 * kHBins; i += kThreads) part[i] = 0u;
+    // [4][kPadBins] 12-bit part sums; bin b at word b + b / 4 of each part (the scan's runs of 4
+    // bins load conflict-free)
+    uint32_t* part = reinterpret_cast<uint32_t*>(mass);
+    for (int i = tid; i < 4 * kPadBins; i += kThreads) part[i] = 0u;
     __syncthreads();
     TWL_FOR_EACH_WEIGHT({
       const uint32_t u = __float_as_uint(w);
       if (u >= lo && u <= hi) {
         const int b = (int)((u - lo) >> s);
+        const int bp = b + (b >> 2);
         const unsigned long long q = (unsigned long long)w_fixed(w);
-        atomicAdd(&part[b], (uint32_t)(q & 0xFFFu));
-        atomicAdd(&part[kHBins + b], (uint32_t)((q >> 12) & 0xFFFu));
-        atomicAdd(&part[2 * kHBins + b], (uint32_t)((q >> 24) & 0xFFFu));
-        atomicAdd(&part[3 * kHBins + b], (uint32_t)(q >> 36));
+        atomicAdd(&part[bp], (uint32_t)(q & 0xFFFu));
+        atomicAdd(&part[kPadBins + bp], (uint32_t)((q >> 12) & 0xFFFu));
+        atomicAdd(&part[2 * kPadBins + bp], (uint32_t)((q >> 24) & 0xFFFu));
+        atomicAdd(&part[3 * kPadBins + bp], (uint32_t)(q >> 36));
       }
     });
     __syncthreads();
@@ -1101,12 +1112,12 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
     unsigned long long mb[4], mine = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int b = nb - 1 - 4 * tid - e;
+      const int b = nb - 1 - 4 * tid - e, bp = b + (b >> 2);
       mb[e] = 0ull;
       if (b >= 0)
-        mb[e] = (unsigned long long)part[b] + ((unsigned long long)part[kHBins + b] << 12) +
-                ((unsigned long long)part[2 * kHBins + b] << 24) +
-                ((unsigned long long)part[3 * kHBins + b] << 36);
+        mb[e] = (unsigned long long)part[bp] + ((unsigned long long)part[kPadBins + bp] << 12) +
+                ((unsigned long long)part[2 * kPadBins + bp] << 24) +
+                ((unsigned long long)part[3 * kPadBins + bp] << 36);
       mine += mb[e];
     }
     if (tid == 0) sh.state[3] = 0xFFFFFFFFu;
@@ -1156,6 +1167,9 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
 }
 
 constexpr int kBandBins = 8192;
+// the histogram scratch of the prune item: the band's padded bins (kBandBins + kBandBins / 16
+// words), the exact bins' 4 x kHBins parts, or the refinement's 3 x kHBins, whichever is used
+constexpr int kHistBytes = 4 * 4 * kPadBins;  // >= 4 * (kBandBins + kBandBins / 16 + 1)
 // The same T, located first with approximate bin masses (kBandBins bins, one shared integer
 // atomic per weight, the weight truncated to units of 2^-30) and then
 // proven exactly: with the bin where the approximate mass from the top first reaches p, the band of
@@ -1194,13 +1208,18 @@ __device__ bool threshold_by_band(const float (&wr)[kR], bool in_regs, const flo
   const int s = bits > 13 ? bits - 13 : 0;
   const int nb = (int)(width >> s) + 1;
   uint32_t* imass = reinterpret_cast<uint32_t*>(fmass);
-  for (int i = tid; i < nb; i += kThreads) imass[i] = 0u;
+  // bin b lives at word b + b / 16: a thread's 16 bins of the scan below then start 17 words
+  // after the previous thread's, so the scan's loads are free of bank conflicts
+  for (int i = tid; i < nb + (nb >> 4) + 1; i += kThreads) imass[i] = 0u;
   __syncthreads();
   // bin masses in units of 2^-30, truncated (a weight loses < 2^-30; W <= 1 and the weights sum
   // to about 1, so the sums and their prefix stay below 2^31)
   TWL_FOR_EACH_WEIGHT({
     const uint32_t u = __float_as_uint(w);
-    if (u >= lo && u <= hi) atomicAdd(&imass[(u - lo) >> s], (uint32_t)(w * 1073741824.f));
+    if (u >= lo && u <= hi) {
+      const uint32_t b = (u - lo) >> s;
+      atomicAdd(&imass[b + (b >> 4)], (uint32_t)(w * 1073741824.f));
+    }
   });
   __syncthreads();
   // descending integer scan (thread t holds bins nb-1-16t .. nb-16-16t): the crossing bin
@@ -1208,7 +1227,7 @@ __device__ bool threshold_by_band(const float (&wr)[kR], bool in_regs, const flo
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
     const int b = nb - 1 - 16 * tid - e;
-    mb[e] = b >= 0 ? (int)imass[b] : 0;
+    mb[e] = b >= 0 ? (int)imass[b + (b >> 4)] : 0;
     mine += mb[e];
   }
   if (tid == 0) sh.state[3] = 0xFFFFFFFFu;
@@ -1290,7 +1309,7 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
   const int tail_off = (int)(tail - smem);
   // weights staged in shared memory when they fit beside the histogram scratch of the large
   // live-set search (5 * 2048 words)
-  const bool staged = tail_off + ((4 * nc + 127) & ~127) + 16 * kHBins +
+  const bool staged = tail_off + ((4 * nc + 127) & ~127) + kHistBytes +
                           4 * (((nc + 31) >> 5) + 32) + 8 * (a.sel_words + 32) <=
                       smem_bytes;
 
@@ -1300,7 +1319,7 @@ __device__ void item_prune(const Args& a, Shared& sh, int bh, unsigned char* sme
   const int nw = (sq.pages + 31) >> 5;
   const int kw = (nc + 31) >> 5;
   uint32_t* kws = reinterpret_cast<uint32_t*>(tail + (staged ? ((4 * nc + 127) & ~127) : 0) +
-                                              16 * kHBins);
+                                              kHistBytes);
   uint32_t* sb = kws + ((kw + 31) & ~31);
   int* sp = reinterpret_cast<int*>(sb + ((nw + 31) & ~31));
   {
@@ -2333,9 +2352,9 @@ const void* kernel_for(int g) {
 // Shared memory each item kind needs (bytes).
 int smem_need(int g, int max_pages, int max_budget, int s_chunk) {
   const int sw = round32((max_pages + 31) / 32);
-  const int topk = 4 * sw + 4 * round32(max_pages) + 4 * 4096 + 8 * 64 + 64;
+  const int topk = 4 * sw + 4 * round32(max_pages) + 4 * (4096 + 512) + 8 * 64 + 64;
   const int kept_words = (16 * max_budget + 31) / 32;
-  const int prune = 1024 + 16 * kThreads + 16 * kHBins + 4 * round32(kept_words) +
+  const int prune = 1024 + 16 * kThreads + kHistBytes + 4 * round32(kept_words) +
                     8 * round32(sw) + 128;  // + staged weights when they fit
   const int score = ((4 * s_chunk + 127) & ~127) + 2 * kScorePass * 512;
   const int est_kw = kEstMeta / 32 + 1;
