@@ -506,4 +506,8 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
   return cuda_status(step::launch(a, pl, (cudaStream_t)stream));
 }
 
+void twl_test_set_waits(uint32_t max_polls, int32_t stall_estimate) {
+  step::set_test_waits(max_polls, stall_estimate);
+}
+
 }  // extern "C"

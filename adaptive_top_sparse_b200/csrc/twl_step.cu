@@ -39,6 +39,7 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr uint32_t kSpinLimit = 1u << 22;  // polls (>= 64 ns apart) before a wait gives up
+                                           // (the default of Args::spin_limit)
 
 struct Shared {
   int flag;
@@ -100,7 +101,7 @@ __device__ bool block_wait(const Args& a, Shared& sh, const uint32_t* ctr, uint3
           ok = 0;
           break;
         }
-        if (it >= kSpinLimit) {
+        if (it >= a.spin_limit) {
           raise_flag(a.flags, TWL_FLAG_TIMEOUT);
           atomicExch(a.sync + kAbort, 1u);
           ok = 0;
@@ -712,7 +713,9 @@ template <int G>
 __device__ void item_estimate(const Args& a, Shared& sh, int g, int e, unsigned char* smem) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = lane >> 2, t = lane & 3;
-  const bool ready = block_wait(a, sh, counter(a, kCntTopK, g), (uint32_t)a.g);
+  // (a test of the timeout path makes this wait unreachable: stall_estimate)
+  const bool ready = block_wait(a, sh, counter(a, kCntTopK, g),
+                                a.stall_estimate ? 0xFFFFFFFFu : (uint32_t)a.g);
   const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
   const Seq sq = load_seq(a.kv.seq_lens, b, a.kv.max_pages, a.flags, false);
   const int p0 = e * a.e_chunk, p1 = ready ? min(sq.pages, p0 + a.e_chunk) : 0;
@@ -2032,7 +2035,7 @@ __device__ int ticket_wait(const Args& a, int c) {
   for (uint32_t it = 0;; ++it) {
     const int st = ticket_state(a, c);
     if (st != 0) return st;
-    if (it >= kSpinLimit) {
+    if (it >= a.spin_limit) {
       raise_flag(a.flags, TWL_FLAG_TIMEOUT);
       atomicExch(a.sync + kAbort, 1u);
       return -1;
@@ -2321,6 +2324,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_step(const __grid_constant__ Ar
   if (sh.flag) {
     const int used = min(a.q_cap, (int)ldcg_u(a.sync + kQAlloc));
     for (int i = threadIdx.x; i < used; i += kThreads) a.qvalid[i] = 0u;
+    // an aborted launch may leave page masks that no kept-list build consumed
+    if (ldcg_u(a.sync + kAbort) != 0u)
+      for (size_t i = threadIdx.x; i < (size_t)a.groups * a.pm_words; i += kThreads)
+        a.pmask[i] = 0u;
     const int nwords = kSyncHead + kCounters * a.groups;
     for (int i = threadIdx.x; i < nwords; i += kThreads) a.sync[i] = 0u;
   }
@@ -2466,6 +2473,16 @@ size_t workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_budget
   return layout(pl, batch, hq, hkv, max_pages).total;
 }
 
+namespace {
+uint32_t g_spin_limit = kSpinLimit;  // test knobs (twl_test_set_waits)
+int g_stall_estimate = 0;
+}  // namespace
+
+void set_test_waits(uint32_t spin_limit, int stall_estimate) {
+  g_spin_limit = spin_limit > 0 ? spin_limit : kSpinLimit;
+  g_stall_estimate = stall_estimate != 0;
+}
+
 void carve(Args& a, char* ws, const Plan& pl, int batch, int hq, int hkv, int max_pages) {
   const Layout L = layout(pl, batch, hq, hkv, max_pages);
   a.sync = reinterpret_cast<uint32_t*>(ws + L.sync);
@@ -2496,6 +2513,8 @@ void carve(Args& a, char* ws, const Plan& pl, int batch, int hq, int hkv, int ma
   a.e_chunk = pl.e_chunk;
   a.q_cap = pl.q_cap;
   a.att_chunks = pl.att_chunks;
+  a.spin_limit = g_spin_limit;
+  a.stall_estimate = g_stall_estimate;
   a.smem_bytes = pl.smem_bytes;
   // the work list, kind by kind (every item depends only on items of earlier kinds)
   // the work list, kind by kind (every item depends only on items of earlier kinds); the last

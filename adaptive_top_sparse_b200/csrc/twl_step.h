@@ -81,6 +81,8 @@ struct Args {
   int groups, sel_words, cand_stride, kept_words, pm_words;
   int s_per, s_chunk, e_per, e_chunk, q_cap;
   int att_chunks;  // chunks a group's kept tokens are cut into, before the size limits
+  uint32_t spin_limit;  // polls before a wait between items gives up (TWL_FLAG_TIMEOUT)
+  int stall_estimate;   // test of the timeout path: the estimate items wait for a count never reached
   int n_items;
   int smem_bytes;  // dynamic shared memory of each CTA
   int nseg;
@@ -101,6 +103,9 @@ size_t workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_budget
 // the strides and the work list from the plan.
 void carve(Args& a, char* ws, const Plan& pl, int batch, int hq, int hkv, int max_pages);
 cudaError_t launch(const Args& a, const Plan& pl, cudaStream_t s);
+// Test knobs for the bounded waits (twl_test_set_waits): the polls before a wait gives up (0 =
+// the default) and whether the estimate items wait for a count that is never reached.
+void set_test_waits(uint32_t spin_limit, int stall_estimate);
 
 }  // namespace step
 }  // namespace twl

@@ -45,7 +45,7 @@ EXPORTED = [
     "twl_page_bounds", "twl_quantize_k", "twl_append_token", "twl_quantize_k_nbit",
     "twl_estimate_nbit", "twl_page_centroids", "twl_select_clusters_top_p", "twl_select_pages", "twl_estimate", "twl_prune_top_p",
     "twl_group_union", "twl_sparse_decode", "twl_decode_step", "twl_noalloc_scratch_bytes",
-    "twl_sparse_decode_noalloc",
+    "twl_sparse_decode_noalloc", "twl_test_set_waits",
 ]
 
 
@@ -98,6 +98,7 @@ _sigs = {
     "twl_sparse_decode": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _vp, _vp, _i32, _f32, _vp, _vp,
                                  _vp, _sz, _vp]),
     "twl_noalloc_scratch_bytes": (_sz, []),
+    "twl_test_set_waits": (None, [C.c_uint32, _i32]),
     "twl_sparse_decode_noalloc": (_i32, [_vp, _i32, C.POINTER(_PagedKV), _vp, _vp, _i32, _f32,
                                          _vp, _vp, _vp]),
     "twl_decode_step": (_i32, [_vp, _i32, C.POINTER(_PagedKV), C.POINTER(_KAux), _i32, _i32,
@@ -320,6 +321,11 @@ def twl_decode_step(q, num_q_heads: int, kv: PagedKV, aux: KAux, budget_pages: i
 
 def twl_noalloc_scratch_bytes() -> int:
     return int(_lib.twl_noalloc_scratch_bytes())
+
+
+def twl_test_set_waits(max_polls: int = 0, stall_estimate: bool = False) -> None:
+    """Test hook of the decode step's bounded waits (see include/twl.h)."""
+    _lib.twl_test_set_waits(int(max_polls), 1 if stall_estimate else 0)
 
 
 def twl_sparse_decode_noalloc(q, num_q_heads: int, kv: PagedKV, tok, tok_count, tok_stride: int,

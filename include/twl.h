@@ -338,6 +338,16 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
                            const twl_step_stats* stats, void* ws, size_t ws_bytes,
                            twl_stream_t stream);
 
+/* ---------------------------------------------------------------- test hook of the bounded waits
+ * twl_decode_step's work items wait for one another by polling counters in the workspace; each
+ * wait gives up after a bounded number of polls, raises TWL_FLAG_TIMEOUT and aborts the launch
+ * (the kernel returns; the context stays usable; the next launch on the workspace is valid).
+ * This hook exists so that a test can make that happen without a device fault: max_polls sets
+ * the polls before a wait gives up for later launches (0 = the default, 2^22), and
+ * stall_estimate != 0 makes the INT4-estimate items wait for a count that is never reached.
+ * Process-wide, read at each twl_decode_step call; not for production use. */
+void twl_test_set_waits(uint32_t max_polls, int32_t stall_estimate);
+
 #ifdef __cplusplus
 }
 #endif

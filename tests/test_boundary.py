@@ -18,7 +18,7 @@ A = 1 << 20          # a fake, 256-byte aligned address
 
 def declared_symbols():
     src = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*(?:twl_status|size_t|const char\*)\s+(twl_\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:twl_status|size_t|const char\*|void)\s+(twl_\w+)\s*\(",
                                  src, flags=re.M)))
 
 
