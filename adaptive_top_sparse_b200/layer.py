@@ -94,6 +94,10 @@ class DecodeLayer:
         return self.o, self.lse
 
     # ------------------------------------------------------------------ cluster-level selector
+    def staged(self) -> "Staged":
+        """The same step as five separate library calls (see Staged)."""
+        return Staged(self)
+
     def double_p(self) -> "DoubleP":
         """The two-level top-p path on this layer's cache (built on first use)."""
         if getattr(self, "_double_p", None) is None:
@@ -158,4 +162,52 @@ class DoubleP:
                             self.union_tok, self.union_count, None, stream)
         twl.twl_sparse_decode(q, hq, L.kv, self.union_tok, self.union_count, cs, SM_SCALE, L.o,
                               L.lse, self.ws_att, stream)
+        return L.o, L.lse
+
+
+class Staged:
+    """The decode step as its five staged library calls (twl_select_pages, twl_estimate,
+    twl_prune_top_p, twl_group_union, twl_sparse_decode) instead of the one fused launch: the
+    comparison the flattened per-stage work lists give.  Only owns the buffers between calls."""
+
+    def __init__(self, layer: DecodeLayer):
+        self.layer = layer
+        L, dev = layer, layer.device
+        b, hq, hkv, mb = L.batch, L.num_q_heads, L.num_kv_heads, L.max_budget
+        i32, f32 = torch.int32, torch.float32
+        cs = 16 * mb
+        self.sel = torch.full((b, hq, mb), -1, dtype=i32, device=dev)
+        self.sel_count = torch.zeros((b, hq), dtype=i32, device=dev)
+        self.weights = torch.zeros((b, hq, cs), dtype=f32, device=dev)
+        self.cand_tok = torch.full((b, hq, cs), -1, dtype=i32, device=dev)
+        self.cand_count = torch.zeros((b, hq), dtype=i32, device=dev)
+        self.m = torch.zeros(b * hq, dtype=f32, device=dev)
+        self.kept_count = torch.zeros(b * hq, dtype=i32, device=dev)
+        self.kept_idx = torch.zeros((b * hq, cs), dtype=i32, device=dev)
+        us = 16 * L.max_pages  # union rows: up to every token of the sequence
+        self.union_tok = torch.full((b, hkv, us), -1, dtype=i32, device=dev)
+        self.union_count = torch.zeros((b, hkv), dtype=i32, device=dev)
+        dims = dict(batch=b, num_q_heads=hq, num_kv_heads=hkv, max_pages=L.max_pages,
+                    max_budget=mb)
+        self.ws_sel = twl.alloc_workspace(twl.TWL_OP_SELECT, dev, **dims)
+        self.ws_est = twl.alloc_workspace(twl.TWL_OP_ESTIMATE, dev, **dims)
+        self.ws_att = twl.alloc_workspace(twl.TWL_OP_SPARSE_DECODE, dev, batch=b, num_q_heads=hq,
+                                          num_kv_heads=hkv, row_stride=us)
+
+    def decode(self, q, p: float = 0.85, eps: float = 1e-6, stream=None):
+        L = self.layer
+        hq, mb = L.num_q_heads, L.max_budget
+        cs = 16 * mb
+        twl.twl_select_pages(q, hq, L.kv, L.aux.bounds, L.budget_pages, L.budget_div, mb,
+                             self.sel, self.sel_count, None, self.ws_sel, stream)
+        twl.twl_estimate(q, hq, L.kv, L.aux.k_int4, L.aux.k_scale_zero, self.sel,
+                         self.sel_count, mb, self.weights, self.cand_tok, self.cand_count,
+                         self.ws_est, stream)
+        rows = L.batch * hq
+        twl.twl_prune_top_p(self.weights.view(rows, cs), self.cand_count.view(rows), rows, cs,
+                            p, eps, self.m, self.kept_count, self.kept_idx, None, stream)
+        twl.twl_group_union(hq, L.kv, self.cand_tok, self.kept_idx, self.kept_count, cs,
+                            self.union_tok, self.union_count, None, stream)
+        twl.twl_sparse_decode(q, hq, L.kv, self.union_tok, self.union_count, 16 * L.max_pages,
+                              SM_SCALE, L.o, L.lse, self.ws_att, stream)
         return L.o, L.lse

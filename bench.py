@@ -825,6 +825,73 @@ def run_quest(args, world, rank, local):
     }
 
 
+# ---------------------------------------------------------------------------------- staged
+
+def run_staged(args, world, rank, local):
+    """The same step as five separate library calls (select, estimate, prune, union, attention;
+    each a flattened work list over its own grid) on the workload: the comparison against the
+    one fused launch.  Algorithmic bytes as for the fused step, from the staged selections."""
+    from adaptive_top_sparse_b200.layer import DecodeLayer
+    dev = torch.device("cuda", local)
+    wl = make_workload(args.workload)
+    layers = []
+    for _ in range(LAYERS):
+        layer = DecodeLayer.from_workload(wl, dev)
+        layer.build_aux()
+        layers.append((layer.staged(), torch.from_numpy(wl.q).to(dev)))
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step():
+        for stg, q in layers:
+            stg.decode(q, wl.p, wl.eps, stream)
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    s0 = layers[0][0]
+    nbytes, _ = algorithmic_bytes(wl.page_table, wl.seq_lens, wl.num_q_heads, wl.num_kv_heads,
+                                  s0.sel.cpu().numpy(), s0.sel_count.cpu().numpy(),
+                                  s0.union_count.cpu().numpy())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(world)
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+    e1.synchronize()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    per_layer_us = ms * 1e3 / (args.steps * LAYERS)
+    peak, peak_kind = hbm_peak()
+    del graph
+    return {
+        "metric": f"staged path layer-steps/s (five library calls per layer-step), "
+                  f"workload {args.workload}",
+        "value": world * args.steps * LAYERS / (ms / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": workload_config(args.workload),
+        "roofline": {"bound": "hbm", "achieved": nbytes / per_layer_us / 1e3, "peak": peak,
+                     "unit": "GB/s", "frac": nbytes / per_layer_us / 1e3 / peak,
+                     "traffic": None, "kernel": "twl_select_pages + twl_estimate + "
+                     "twl_prune_top_p + twl_group_union + twl_sparse_decode",
+                     "alg_bytes_per_layer_step": nbytes,
+                     "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "frac_of_nominal_8tbs": None},
+        "clocks": clk,
+    }
+
+
 # ---------------------------------------------------------------------------------- Double-P
 
 def run_double_p(args, world, rank, local, p_cluster=0.95):
@@ -1206,6 +1273,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--double-p", action="store_true",
                     help="time the two-level (cluster, then token) top-p path on the workload")
+    ap.add_argument("--staged", action="store_true",
+                    help="time the step as its five staged library calls instead of the fused "
+                         "launch (a comparison, not the headline)")
     ap.add_argument("--quest", action="store_true",
                     help="time the Quest baseline (select + attention over every token of the "
                          "selected pages, no estimate or top-p) on the workload instead")
@@ -1239,6 +1309,8 @@ def main():
                    else run_append(args, world, rank, local))
         elif args.double_p:
             out = run_double_p(args, world, rank, local)
+        elif args.staged:
+            out = run_staged(args, world, rank, local)
         elif args.quest:
             out = run_quest(args, world, rank, local)
         elif args.impl == "reference":

@@ -507,6 +507,30 @@ def test_decode_step_equals_staged_calls(small):
     assert do <= 2e-4 and dl <= 2e-4, (do, dl)
 
 
+def test_staged_wrapper_matches_the_oracle(small):
+    """The five staged calls through layer.Staged (the bench's staged comparison): every group's
+    selection, candidates, weights, kept sets and output against the oracle."""
+    wl, layer = small
+    stg = layer.staged()
+    q = torch.from_numpy(wl.q).to(layer.device)
+    o, lse = stg.decode(q, wl.p, wl.eps)
+    rows = wl.batch * wl.num_q_heads
+    st = {
+        "sel_pages": np_(stg.sel), "sel_count": np_(stg.sel_count),
+        "weights": np_(stg.weights), "cand_tok": np_(stg.cand_tok),
+        "cand_count": np_(stg.cand_count),
+        "threshold": np_(stg.m).reshape(wl.batch, wl.num_q_heads),
+        "kept_count": np_(stg.kept_count).reshape(wl.batch, wl.num_q_heads),
+        "union_tok": np_(stg.union_tok), "union_count": np_(stg.union_count),
+    }
+    assert rows == st["kept_count"].size
+    o, lse = np_(o), np_(lse)
+    for bb in range(wl.batch):
+        for kvh in range(wl.num_kv_heads):
+            check_step_group(wl, bb, kvh, st, o, lse)
+    assert twl.twl_device_status(stg.ws_sel)[0] == twl.TWL_OK
+
+
 def test_decode_step_dense_limit():
     # budget = every page and p = 1: the step is exact dense attention
     wl = synth.make_decode("dense", 1, 8, 2, [700], seed=8)
