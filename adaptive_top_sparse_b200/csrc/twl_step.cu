@@ -1653,7 +1653,7 @@ __device__ void build_kept(const Args& a, Shared& sh, int g, unsigned char* smem
   TRACE_MARK(sh, 7);
   // publish the group's kept pages to the attention queue in nch chunks of about equal token
   // counts: page q opens chunk floor(pre(q) nch / ntok).  A chunk is cut to about ntok /
-  // att_chunks tokens (the group's share of the workers, twice over), at least kAttChunkTok and
+  // att_chunks tokens (the group's share of the workers), at least kAttChunkTok and
   // at most kAttChunkMax (+15 at a page edge).  As a page holds at most 16 tokens and a chunk
   // about ntok / nch >= kAttChunkTok / 2 = 64, consecutive pages open consecutive chunks and none
   // is empty.  One empty chunk when nothing is kept, so the merge still writes the outputs.
@@ -1739,15 +1739,19 @@ template <int G>
 constexpr int att_bufs() {
   return G >= 8 ? 2 : 3;
 }
-// shared memory of a worker: [bufs][kAttBufBytes] | [kAttIdx] row indices | scratch of the
+// shared memory of a worker: [bufs][kAttBufBytes] | [2][kAttIdx] row indices | scratch of the
 // consumers ([8 warps][2 G] max, sum | [8 warps][G][128] o)
 template <int G>
 constexpr int att_scratch_off() {
-  return att_bufs<G>() * kAttBufBytes + ((4 * kAttIdx + 127) & ~127);
+  return att_bufs<G>() * kAttBufBytes + 2 * ((4 * kAttIdx + 127) & ~127);
 }
 template <int G>
+constexpr int att_merge_floats();
+template <int G>
 constexpr int att_smem() {
-  return att_scratch_off<G>() + 4 * 8 * (2 * G + G * kHeadDim);
+  return att_scratch_off<G>() + 4 * (8 * (2 * G + G * kHeadDim) > att_merge_floats<G>()
+                                         ? 8 * (2 * G + G * kHeadDim)
+                                         : att_merge_floats<G>());
 }
 enum { kDescEnd = 1, kDescFirst = 2, kDescLast = 4 };
 
@@ -1946,31 +1950,43 @@ __device__ void attend_finish(const Args& a, int c, const float (&m)[2], float (
 
 // Consumers (256 threads), in the CTA whose chunk completed group g: log-sum-exp merge of the
 // group's nch chunk partials (slots c0 ...) -> o, lse of every head (o = 0, lse = -inf when
-// nothing was kept).  Warp h finds head h's max and total; then each float4 of o is summed by
-// 8 / G threads over interleaved chunks (loads independent of the sums, so they stay in flight
-// together) and their sums are added in a fixed order.  scr: the consumers' scratch.
+// nothing was kept).  The max of every (chunk, head) is staged in shared memory in one round of
+// loads; warp h turns head h's into chunk weights exp(max_c - max) and the head's total;
+// then each float4 of o is summed by 8 / G threads over interleaved chunks (their loads are
+// independent of the sums, so they stay in flight together) and their sums are added in a fixed
+// order.  scr: the consumers' scratch (kAttMergeFloats floats at least).
+constexpr int kAttMaxChunks = 512;  // chunks of one group at most (16 * kMaxPages / kAttChunkMax)
+template <int G>
+constexpr int att_merge_floats() {
+  return kAttMaxChunks * G + 16 + 4 * kAttCons;
+}
 template <int G>
 __device__ void merge_group(const Args& a, int g, int c0, int nch, float* scr) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int b = g / a.kv.hkv, kvh = g - b * a.kv.hkv;
   const float* part = a.part + (size_t)c0 * G * kAttPartStride;
-  float* hs = scr;                                      // [G] head max, [G] head total
-  float4* red = reinterpret_cast<float4*>(scr + 16);    // [kAttCons]
+  float4* red = reinterpret_cast<float4*>(scr);      // [kAttCons]
+  float* hs = scr + 4 * kAttCons;                    // [G] head max, [G] head total
+  float* wm = hs + 16;                               // [nch][G] chunk max, then its weight
+  for (int i = tid; i < nch * G; i += kAttCons) {
+    const float* pp = part + (size_t)i * kAttPartStride + kHeadDim;
+    const float l = ldcg_f(pp + 1), m = ldcg_f(pp);
+    wm[i] = l > 0.f ? m : -INFINITY;
+  }
+  bar_named(2, kAttCons);
   if (warp < G) {
     float mx = -INFINITY;
-    for (int c = lane; c < nch; c += 32) {
-      const float* pp = part + (size_t)(c * G + warp) * kAttPartStride + kHeadDim;
-      if (ldcg_f(pp + 1) > 0.f) mx = fmaxf(mx, ldcg_f(pp));
-    }
+    for (int c = lane; c < nch; c += 32) mx = fmaxf(mx, wm[c * G + warp]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float tot = 0.f;
-    if (mx > -INFINITY)
-      for (int c = lane; c < nch; c += 32) {
-        const float* pp = part + (size_t)(c * G + warp) * kAttPartStride + kHeadDim;
-        const float lc = ldcg_f(pp + 1);
-        if (lc > 0.f) tot = fmaf(__expf(ldcg_f(pp) - mx), lc, tot);
-      }
+    for (int c = lane; c < nch; c += 32) {
+      const float m = wm[c * G + warp];
+      const float w = m > -INFINITY ? __expf(m - mx) : 0.f;
+      wm[c * G + warp] = w;
+      if (w > 0.f)
+        tot = fmaf(w, ldcg_f(part + (size_t)(c * G + warp) * kAttPartStride + kHeadDim + 1), tot);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
     if (lane == 0) {
@@ -1981,20 +1997,17 @@ __device__ void merge_group(const Args& a, int g, int c0, int nch, float* scr) {
   bar_named(2, kAttCons);
   constexpr int kCols = G * kHeadDim / 4, kPer = kAttCons / kCols;
   const int col = tid % kCols, r = tid / kCols, h = col / (kHeadDim / 4);
-  const float mx = hs[h];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (mx > -INFINITY) {
 #pragma unroll 8
-    for (int c = r; c < nch; c += kPer) {
-      const float* pp = part + (size_t)(c * G + h) * kAttPartStride;
-      const float lc = ldcg_f(pp + kHeadDim + 1);
-      const float w = lc > 0.f ? __expf(ldcg_f(pp + kHeadDim) - mx) : 0.f;
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(pp) + (col % (kHeadDim / 4)));
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
-    }
+  for (int c = r; c < nch; c += kPer) {
+    const float w = wm[c * G + h];
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(part + (size_t)(c * G + h) *
+                                                                      kAttPartStride) +
+                            (col % (kHeadDim / 4)));
+    acc.x = fmaf(w, v.x, acc.x);
+    acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z);
+    acc.w = fmaf(w, v.w, acc.w);
   }
   red[tid] = acc;
   bar_named(2, kAttCons);
@@ -2013,7 +2026,7 @@ __device__ void merge_group(const Args& a, int g, int c0, int nch, float* scr) {
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     if (any) o = make_float4(acc.x / lt, acc.y / lt, acc.z / lt, acc.w / lt);
     reinterpret_cast<float4*>(a.o + bh * kHeadDim)[col % (kHeadDim / 4)] = o;
-    if (col % (kHeadDim / 4) == 0) a.lse[bh] = any ? mx + __logf(lt) : -INFINITY;
+    if (col % (kHeadDim / 4) == 0) a.lse[bh] = any ? hs[h] + __logf(lt) : -INFINITY;
   }
   bar_named(2, kAttCons);  // the scratch is reused
 }
@@ -2045,54 +2058,100 @@ __device__ int ticket_wait(const Args& a, int c) {
 }
 
 // Producers (warps 8-15): take chunks until the queue is done, copy their passes into the ring,
-// then post the end.
+// then post the end.  The next chunk is prepared while the current one's passes are issued, one
+// step per pass (take its queue ticket; see it published and read its entry; expand its pages
+// into the other row-index stage), so a chunk switch leaves no gap in the copies.
 template <int G>
 __device__ void attend_produce(const Args& a, Shared& sh, unsigned char* smem) {
   constexpr int NB = att_bufs<G>();
   const int pt = threadIdx.x - kAttCons;
-  uint32_t* idx = reinterpret_cast<uint32_t*>(smem + NB * kAttBufBytes);
+  uint32_t* idx_base = reinterpret_cast<uint32_t*>(smem + NB * kAttBufBytes);  // [2][kAttIdx]
+  int ticket = -1;  // thread pt == 0: the ticket of the chunk being prepared
+  // expand chunk (group g, pages [p0, p1)) into stage s; returns its token count
+  auto expand = [&](int s, int g, int p0, int p1) {
+    uint32_t* idx = idx_base + s * kAttIdx;
+    const int4* kp = a.kpages + (size_t)g * a.kv.max_pages;
+    int n = 0, tb = 0;
+    if (p1 > p0) {
+      const int4 f = ldcg_i4(kp + p0), ls = ldcg_i4(kp + p1 - 1);
+      tb = f.w;
+      n = ls.w + __popc((uint32_t)ls.y) - tb;
+    }
+    for (int q = p0 + pt; q < p1; q += kAttProd) {
+      const int4 en = ldcg_i4(kp + q);
+      uint32_t mk = (uint32_t)en.y;
+      int pos = en.w - tb;
+      while (mk) {
+        idx[pos++] = (uint32_t)en.x + (uint32_t)(__ffs(mk) - 1);
+        mk &= mk - 1u;
+      }
+    }
+    bar_named(1, kAttProd);
+    return n;
+  };
+  // thread 0 has the ticket's state st (1 published, -1 none, 0 not yet): share it and, when
+  // published, the chunk's entry (slot, group, first page, end page) through stage s
+  auto share = [&](int s, int st) {
+    if (pt == 0) {
+      sh.att[s][0] = st > 0 ? ticket : (st < 0 ? -1 : -2);
+      if (st > 0) {
+        const int* e = a.qtab + 4 * (size_t)ticket;
+        sh.att[s][1] = ldcg_i(e);
+        sh.att[s][2] = ldcg_i(e + 1);
+        sh.att[s][3] = ldcg_i(e + 2);
+      }
+    }
+    bar_named(1, kAttProd);
+  };
+  // the first chunk, waited for
+  if (pt == 0) {
+    ticket = (int)atomicAdd(a.sync + kQNext, 1u);
+  }
+  share(0, pt == 0 ? ticket_wait(a, ticket) : 0);
+  int cs = 0;                 // stage of the current chunk
+  int c = sh.att[0][0], g = sh.att[0][1];
+  int n = c >= 0 ? expand(0, g, sh.att[0][2], sh.att[0][3]) : 0;
+  // preparation of the next chunk (stage cs ^ 1): 0 nothing yet, 1 ticket taken, 2 published and
+  // entry read, 3 expanded, -1 none left (the same value in every producer thread)
+  int prep = 0, c2 = -1, g2 = 0, n2 = 0;
+  auto prep_step = [&](bool wait) {
+    const int s = cs ^ 1;
+    if (prep == 0) {
+      if (pt == 0) ticket = (int)atomicAdd(a.sync + kQNext, 1u);
+      prep = 1;
+      if (!wait) return;
+    }
+    if (prep == 1) {
+      int st = 0;
+      if (pt == 0) st = wait ? ticket_wait(a, ticket) : ticket_state(a, ticket);
+      share(s, st);
+      const int v = sh.att[s][0];
+      bar_named(1, kAttProd);  // read before stage s's entry can be written again
+      if (v == -2) return;     // not published yet
+      if (v < 0) {
+        prep = -1;
+        return;
+      }
+      c2 = v;
+      g2 = sh.att[s][1];
+      prep = 2;
+      if (!wait) {
+        // the entry stays in stage s until the expansion below
+        return;
+      }
+    }
+    if (prep == 2) {
+      n2 = expand(s, g2, sh.att[s][2], sh.att[s][3]);
+      prep = 3;
+    }
+  };
   int j = 0;  // passes posted
   bool ok = true;
 #pragma unroll 1
   for (;;) {
-    // the next chunk
-    if (pt == 0) {
-      const int c = (int)atomicAdd(a.sync + kQNext, 1u);
-      const int st = ticket_wait(a, c);
-      sh.att[0][0] = st > 0 ? c : -1;
-      if (st > 0) {
-        const int* e = a.qtab + 4 * (size_t)c;
-        sh.att[0][1] = ldcg_i(e);
-        sh.att[0][2] = ldcg_i(e + 1);
-        sh.att[0][3] = ldcg_i(e + 2);
-      }
-    }
-    bar_named(1, kAttProd);
-    const int c = sh.att[0][0], g = sh.att[0][1], p0 = sh.att[0][2], p1 = sh.att[0][3];
-    bar_named(1, kAttProd);  // read before the next chunk's entry is written
-    int n = 0, np = 1;
-    if (c >= 0) {
-      // expand the chunk's pages to row indices (token order)
-      const int4* kp = a.kpages + (size_t)g * a.kv.max_pages;
-      int tb = 0;
-      if (p1 > p0) {
-        const int4 f = ldcg_i4(kp + p0), ls = ldcg_i4(kp + p1 - 1);
-        tb = f.w;
-        n = ls.w + __popc((uint32_t)ls.y) - tb;
-      }
-      for (int q = p0 + pt; q < p1; q += kAttProd) {
-        const int4 en = ldcg_i4(kp + q);
-        uint32_t mk = (uint32_t)en.y;
-        int pos = en.w - tb;
-        while (mk) {
-          idx[pos++] = (uint32_t)en.x + (uint32_t)(__ffs(mk) - 1);
-          mk &= mk - 1u;
-        }
-      }
-      bar_named(1, kAttProd);
-      np = n > 0 ? (n + kAttPass - 1) / kAttPass : 1;
-    }
+    const int np = c >= 0 ? (n > 0 ? (n + kAttPass - 1) / kAttPass : 1) : 1;
     const int b_ = g / a.kv.hkv, kvh = g - b_ * a.kv.hkv;
+    const uint32_t* idx = idx_base + cs * kAttIdx;
 #pragma unroll 1
     for (int k = 0; k < np; ++k, ++j) {
       const int bs = j % NB, u = j / NB;
@@ -2150,8 +2209,18 @@ __device__ void attend_produce(const Args& a, Shared& sh, unsigned char* smem) {
         pr[2] = now_ns();
       }
 #endif
+      // one step of the next chunk's preparation while this pass's copies fly
+      if (c >= 0 && prep >= 0 && prep < 3) prep_step(false);
     }
     if (c < 0 || !ok) break;
+    // switch to the next chunk, finishing its preparation (waiting now if it must)
+#pragma unroll 1
+    while (prep >= 0 && prep < 3) prep_step(true);
+    cs ^= 1;
+    c = prep == 3 ? c2 : -1;
+    g = g2;
+    n = n2;
+    prep = 0;
   }
   cp_async_wait_all();
 }
@@ -2427,7 +2496,7 @@ Plan plan(int batch, int hq, int hkv, int max_pages, int max_budget) {
   // attention chunks: at most one per kAttChunkTok kept tokens of each group plus one, and the
   // numbers the workers take past the end
   pl.q_cap = groups * (1 + (kPage * max_pages + kAttChunkTok - 1) / kAttChunkTok) + sms + 32;
-  pl.att_chunks = 2 * sms / groups;
+  pl.att_chunks = sms / groups;
   pl.att_chunks = pl.att_chunks < 1 ? 1 : pl.att_chunks;
   return pl;
 }
