@@ -98,7 +98,9 @@ twl_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TWL_OK : TWL_E
 uint32_t* flags_of(void* ws) { return ws ? &reinterpret_cast<WsHeader*>(ws)->flags : nullptr; }
 
 size_t decode_step_ws_bytes(int batch, int hq, int hkv, int max_pages, int max_budget) {
-  return step::workspace_bytes(batch, hq, hkv, max_pages, max_budget);
+  return step_wide(batch * hkv, num_sms())
+             ? step256::workspace_bytes(batch, hq, hkv, max_pages, max_budget)
+             : step::workspace_bytes(batch, hq, hkv, max_pages, max_budget);
 }
 
 // ---------------------------------------------------------------- workspace layouts
@@ -469,7 +471,10 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
     return TWL_ERR_INVALID_ARG;
   if (!(p > 0.f && p <= 1.f) || !(eps > 0.f) || isinf(eps)) return TWL_ERR_INVALID_ARG;
   if ((st = check_budget(budget_pages, budget_div, max_budget, k.max_pages)) != TWL_OK) return st;
-  const step::Plan pl = step::plan(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
+  const bool wide = step_wide(k.batch * k.hkv, num_sms());
+  const step::Plan pl =
+      wide ? step256::plan(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget)
+           : step::plan(k.batch, num_q_heads, k.hkv, k.max_pages, max_budget);
   if (!pl.ok) return TWL_ERR_UNSUPPORTED;
   Carve c{static_cast<char*>(ws)};
   char* sws = c.take<char>(decode_step_ws_bytes(k.batch, num_q_heads, k.hkv, k.max_pages,
@@ -502,12 +507,17 @@ twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_k
   a.union_tok = so.union_tok;
   a.union_count = so.union_count;
   a.flags = flags_of(ws);
+  if (wide) {
+    step256::carve(a, sws, pl, k.batch, num_q_heads, k.hkv, k.max_pages);
+    return cuda_status(step256::launch(a, pl, (cudaStream_t)stream));
+  }
   step::carve(a, sws, pl, k.batch, num_q_heads, k.hkv, k.max_pages);
   return cuda_status(step::launch(a, pl, (cudaStream_t)stream));
 }
 
 void twl_test_set_waits(uint32_t max_polls, int32_t stall_estimate) {
   step::set_test_waits(max_polls, stall_estimate);
+  step256::set_test_waits(max_polls, stall_estimate);
 }
 
 }  // extern "C"

@@ -29,14 +29,28 @@
 //
 // The arithmetic (score order, INT4 products, softmax and threshold search, attention) is the
 // same as the staged kernels', so the selections are bit-identical to twl_select_pages.
+//
+// This file is built twice: with 512-thread CTAs, one per SM (namespace step, the default), and
+// with 256-thread CTAs, two per SM (twl_step_256.cu: namespace step256), for batches with more
+// groups than SMs, where two resident items per SM hide each other's latency.
 #include "twl_common.cuh"
 #include "twl_step.h"
 
+#ifndef TWL_STEP_THREADS
+#define TWL_STEP_THREADS 512
+#endif
+#ifndef TWL_STEP_NS
+#define TWL_STEP_NS step
+#endif
+
 namespace twl {
-namespace step {
+namespace TWL_STEP_NS {
+using namespace ::twl::step;  // the argument types and constants of twl_step.h
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = TWL_STEP_THREADS;
+static_assert(kThreads == 512 || kThreads == 256, "512 or 256 threads per CTA");
+constexpr int kCtasPerSm = 512 / kThreads;  // resident CTAs per SM the build is sized for
 constexpr int kWarps = kThreads / 32;
 constexpr uint32_t kSpinLimit = 1u << 22;  // polls (>= 64 ns apart) before a wait gives up
                                            // (the default of Args::spin_limit)
@@ -195,7 +209,7 @@ __device__ __forceinline__ int group_of(const Args& a, int bh) {
 // A half-warp scores a page: lane l holds channels 8l..8l+7 of the min and max rows and of each
 // head's query, so the score is the fixed order of the staged selector (8 channels per lane left
 // to right, then the pairs (l, l+8), (l, l+4), (l, l+2), (l, l+1)).
-constexpr int kScorePass = 176;
+constexpr int kScorePass = kThreads == 512 ? 176 : 64;
 
 // Packed fp32 FMA on two lanes (a.x*b.x + c.x, a.y*b.y + c.y), each lane rounded as fmaf.
 __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
@@ -404,10 +418,12 @@ __device__ void topk_bits(const uint32_t* keys, int n_pages, int kb, uint32_t* s
   const int nw = (n_pages + 31) >> 5;
   constexpr int kGatherCap = 64;
   constexpr int kBins = 4096;
-  // the bins, one padding word after every 8 (bin b at word b + b / 8), so that the scan's
-  // per-thread runs of 8 bins start 9 words apart and load free of bank conflicts
-  uint32_t* hh = reinterpret_cast<uint32_t*>(scratch);  // [kBins + kBins / 8]
-  uint32_t* gkey = hh + kBins + kBins / 8;              // [kGatherCap]
+  constexpr int kPerT = kBins / kThreads;  // bins per thread in the scan (8 or 16)
+  // the bins, one padding word after every kPerT (bin b at word b + b / kPerT), so that the
+  // scan's per-thread runs of kPerT bins start kPerT + 1 words apart and load free of bank
+  // conflicts
+  uint32_t* hh = reinterpret_cast<uint32_t*>(scratch);  // [kBins + kBins / kPerT]
+  uint32_t* gkey = hh + kBins + kBins / kPerT;          // [kGatherCap]
   int* gidx = reinterpret_cast<int*>(gkey + kGatherCap);  // [kGatherCap]
   (void)scratch_bytes;
   uint32_t blo, bhi;
@@ -438,19 +454,18 @@ __device__ void topk_bits(const uint32_t* keys, int n_pages, int kb, uint32_t* s
   int remaining = kb;
   int cand = n_pages;
   __syncthreads();
-  constexpr int kPerT = kBins / kThreads;  // bins per thread in the scan
 #pragma unroll 1
   while (cand > kGatherCap && blo < bhi) {
     const uint32_t range = bhi - blo;
     const int width = 32 - __clz(range);
     const int sh_ = width > 12 ? width - 12 : 0;
-    for (int i = tid; i < kBins + kBins / 8; i += kThreads) hh[i] = 0u;
+    for (int i = tid; i < kBins + kBins / kPerT; i += kThreads) hh[i] = 0u;
     __syncthreads();
     for (int i = tid; i < n_pages; i += kThreads) {
       const uint32_t key = keys[i];
       if (key >= blo && key <= bhi) {
         const uint32_t b = (key - blo) >> sh_;
-        atomicAdd(&hh[b + (b >> 3)], 1u);
+        atomicAdd(&hh[b + b / kPerT], 1u);
       }
     }
     __syncthreads();
@@ -458,12 +473,12 @@ __device__ void topk_bits(const uint32_t* keys, int n_pages, int kb, uint32_t* s
     const int b0 = kBins - 1 - kPerT * tid;
     int mine = 0;
 #pragma unroll
-    for (int e = 0; e < kPerT; ++e) mine += (int)hh[(b0 - e) + ((b0 - e) >> 3)];
+    for (int e = 0; e < kPerT; ++e) mine += (int)hh[(b0 - e) + (b0 - e) / kPerT];
     const int excl = block_exclusive_scan(mine, sh.scan, nullptr);
     if (excl < remaining && remaining <= excl + mine) {
       int run = excl;
       for (int e = 0; e < kPerT; ++e) {
-        const int c = (int)hh[(b0 - e) + ((b0 - e) >> 3)];
+        const int c = (int)hh[(b0 - e) + (b0 - e) / kPerT];
         if (run + c >= remaining) {
           sh.state[0] = (uint32_t)(b0 - e);
           sh.state[1] = (uint32_t)(remaining - run);
@@ -706,8 +721,9 @@ __device__ __forceinline__ void nibble_pairs(uint32_t x0, uint32_t x1, int e, ui
 // passes of kEstPass pages, two in flight.  A warp computes two pages at a time, the page as the
 // M = 16 tile of m16n8k16 and the group's heads as N.  Logit slot of (head h, page j, row r) =
 // 16 * (rank of j in h's selection) + r.
-constexpr int kEstPass = 80;
+constexpr int kEstPass = kThreads == 512 ? 80 : 32;
 constexpr int kEstMeta = 480;  // a multiple of kEstPass, and of 32
+static_assert(kEstMeta % kEstPass == 0 && kEstMeta % 32 == 0, "estimate sub-range");
 
 template <int G>
 __device__ void item_estimate(const Args& a, Shared& sh, int g, int e, unsigned char* smem) {
@@ -977,7 +993,8 @@ __device__ float rank_pairwise(const float* gv, const long long* gq, int n,
 }
 constexpr int kPairwiseMax = 384;  // rank_pairwise up to this many weights, refine_threshold above
 constexpr int kHBins = 2048;                 // bins of the exact histograms
-constexpr int kPadBins = kHBins + kHBins / 4;  // words per part of a padded kHBins histogram
+constexpr int kHPer = kHBins / kThreads;     // bins per thread in their scans (4 or 8)
+constexpr int kPadBins = kHBins + kHBins / kHPer;  // words per part of a padded histogram
 
 // T among n <= kThreads weights gv (fixed-point copies gq, units of 2^-48) whose keys (float
 // bits) lie in [lo, hi], given the exact mass `above` of the weights with keys above hi: the
@@ -1001,7 +1018,8 @@ __device__ float refine_threshold(const float* gv, const long long* gq, int n, u
     const int bits = 32 - __clz(width);
     const int s = bits > 11 ? bits - 11 : 0;
     const int nb = (int)(width >> s) + 1;
-    // bin b at word b + b / 4 of each part (the scan's runs of 4 bins load conflict-free)
+    // bin b at word b + b / kHPer of each part (the scan's runs of kHPer bins load
+    // conflict-free)
     for (int i = tid; i < kPadBins; i += kThreads) {
       bins[i] = 0u;
       bins[kPadBins + i] = 0u;
@@ -1010,17 +1028,17 @@ __device__ float refine_threshold(const float* gv, const long long* gq, int n, u
     __syncthreads();
     if (mine && u >= lo && u <= hi) {
       const int b = (int)((u - lo) >> s);
-      const int bp = b + (b >> 2);
+      const int bp = b + b / kHPer;
       atomicAdd(&bins[bp], (uint32_t)(q & 0xFFFFu));
       atomicAdd(&bins[kPadBins + bp], (uint32_t)((q >> 16) & 0xFFFFu));
       atomicAdd(&bins[2 * kPadBins + bp], (uint32_t)(q >> 32));
     }
     __syncthreads();
-    // descending scan: thread t holds bins nb-1-4t .. nb-4-4t
-    unsigned long long mb[4], tot = 0;
+    // descending scan: thread t holds bins nb-1-kHPer t .. nb-kHPer(t+1)
+    unsigned long long mb[kHPer], tot = 0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int b = nb - 1 - 4 * tid - e, bp = b + (b >> 2);
+    for (int e = 0; e < kHPer; ++e) {
+      const int b = nb - 1 - kHPer * tid - e, bp = b + b / kHPer;
       mb[e] = b >= 0 ? (unsigned long long)bins[bp] + ((unsigned long long)bins[kPadBins + bp] << 16) +
                            ((unsigned long long)bins[2 * kPadBins + bp] << 32)
                      : 0ull;
@@ -1029,8 +1047,8 @@ __device__ float refine_threshold(const float* gv, const long long* gq, int n, u
     if (tid == 0) sh.state[3] = 0xFFFFFFFFu;
     unsigned long long run = above + block_excl_u64(tot, sh64, nullptr);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int b = nb - 1 - 4 * tid - e;
+    for (int e = 0; e < kHPer; ++e) {
+      const int b = nb - 1 - kHPer * tid - e;
       if (b >= 0 && run < (unsigned long long)P && run + mb[e] >= (unsigned long long)P) {
         sh.state[3] = (uint32_t)b;
         sh64[kWarps] = run;  // mass above the crossing bin
@@ -1093,8 +1111,8 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
     const int bits = 32 - __clz(width);
     const int s = bits > 11 ? bits - 11 : 0;
     const int nb = (int)(width >> s) + 1;
-    // [4][kPadBins] 12-bit part sums; bin b at word b + b / 4 of each part (the scan's runs of 4
-    // bins load conflict-free)
+    // [4][kPadBins] 12-bit part sums; bin b at word b + b / kHPer of each part (the scan's runs
+    // of kHPer bins load conflict-free)
     uint32_t* part = reinterpret_cast<uint32_t*>(mass);
     for (int i = tid; i < 4 * kPadBins; i += kThreads) part[i] = 0u;
     __syncthreads();
@@ -1102,7 +1120,7 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
       const uint32_t u = __float_as_uint(w);
       if (u >= lo && u <= hi) {
         const int b = (int)((u - lo) >> s);
-        const int bp = b + (b >> 2);
+        const int bp = b + b / kHPer;
         const unsigned long long q = (unsigned long long)w_fixed(w);
         atomicAdd(&part[bp], (uint32_t)(q & 0xFFFu));
         atomicAdd(&part[kPadBins + bp], (uint32_t)((q >> 12) & 0xFFFu));
@@ -1111,11 +1129,11 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
       }
     });
     __syncthreads();
-    // descending scan: thread t holds bins nb-1-4t .. nb-4-4t
-    unsigned long long mb[4], mine = 0;
+    // descending scan: thread t holds bins nb-1-kHPer t .. nb-kHPer(t+1)
+    unsigned long long mb[kHPer], mine = 0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int b = nb - 1 - 4 * tid - e, bp = b + (b >> 2);
+    for (int e = 0; e < kHPer; ++e) {
+      const int b = nb - 1 - kHPer * tid - e, bp = b + b / kHPer;
       mb[e] = 0ull;
       if (b >= 0)
         mb[e] = (unsigned long long)part[bp] + ((unsigned long long)part[kPadBins + bp] << 12) +
@@ -1126,8 +1144,8 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
     if (tid == 0) sh.state[3] = 0xFFFFFFFFu;
     unsigned long long run = above + block_excl_u64(mine, sh64, nullptr);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int b = nb - 1 - 4 * tid - e;
+    for (int e = 0; e < kHPer; ++e) {
+      const int b = nb - 1 - kHPer * tid - e;
       if (b >= 0 && run < (unsigned long long)P && run + mb[e] >= (unsigned long long)P) {
         sh.state[3] = (uint32_t)b;
         sh64[kWarps] = run;  // mass above the crossing bin
@@ -1170,9 +1188,12 @@ __device__ float threshold_by_bins(const float (&wr)[kR], bool in_regs, const fl
 }
 
 constexpr int kBandBins = 8192;
-// the histogram scratch of the prune item: the band's padded bins (kBandBins + kBandBins / 16
-// words), the exact bins' 4 x kHBins parts, or the refinement's 3 x kHBins, whichever is used
-constexpr int kHistBytes = 4 * 4 * kPadBins;  // >= 4 * (kBandBins + kBandBins / 16 + 1)
+constexpr int kBandPer = kBandBins / kThreads;  // bins per thread in the band's scan (16 or 32)
+// the histogram scratch of the prune item: the band's padded bins (kBandBins + kBandBins /
+// kBandPer words), the exact bins' 4 x kPadBins parts, or the refinement's 3 x kPadBins
+constexpr int kHistBytes =
+    4 * (4 * kPadBins > kBandBins + kBandBins / kBandPer + 32 ? 4 * kPadBins
+                                                             : kBandBins + kBandBins / kBandPer + 32);
 // The same T, located first with approximate bin masses (kBandBins bins, one shared integer
 // atomic per weight, the weight truncated to units of 2^-30) and then
 // proven exactly: with the bin where the approximate mass from the top first reaches p, the band of
@@ -1204,16 +1225,16 @@ __device__ bool threshold_by_band(const float (&wr)[kR], bool in_regs, const flo
       }                                                                     \
     }                                                                       \
   } while (0)
-  // kBandBins bins of equal key width (16 per thread in the scan)
-  static_assert(kBandBins == 16 * kThreads, "the scan holds 16 bins per thread");
+  // kBandBins bins of equal key width (kBandPer per thread in the scan)
   const uint32_t width = hi - lo;
   const int bits = 32 - __clz(width);
   const int s = bits > 13 ? bits - 13 : 0;
   const int nb = (int)(width >> s) + 1;
   uint32_t* imass = reinterpret_cast<uint32_t*>(fmass);
-  // bin b lives at word b + b / 16: a thread's 16 bins of the scan below then start 17 words
-  // after the previous thread's, so the scan's loads are free of bank conflicts
-  for (int i = tid; i < nb + (nb >> 4) + 1; i += kThreads) imass[i] = 0u;
+  // bin b lives at word b + b / kBandPer: a thread's kBandPer bins of the scan below then start
+  // kBandPer + 1 words after the previous thread's, so the scan's loads are free of bank
+  // conflicts
+  for (int i = tid; i < nb + nb / kBandPer + 1; i += kThreads) imass[i] = 0u;
   __syncthreads();
   // bin masses in units of 2^-30, truncated (a weight loses < 2^-30; W <= 1 and the weights sum
   // to about 1, so the sums and their prefix stay below 2^31)
@@ -1221,24 +1242,25 @@ __device__ bool threshold_by_band(const float (&wr)[kR], bool in_regs, const flo
     const uint32_t u = __float_as_uint(w);
     if (u >= lo && u <= hi) {
       const uint32_t b = (u - lo) >> s;
-      atomicAdd(&imass[b + (b >> 4)], (uint32_t)(w * 1073741824.f));
+      atomicAdd(&imass[b + b / kBandPer], (uint32_t)(w * 1073741824.f));
     }
   });
   __syncthreads();
-  // descending integer scan (thread t holds bins nb-1-16t .. nb-16-16t): the crossing bin
-  int mb[16], mine = 0;
+  // descending integer scan (thread t holds bins nb-1-kBandPer t .. nb-kBandPer(t+1)): the
+  // crossing bin
+  int mb[kBandPer], mine = 0;
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const int b = nb - 1 - 16 * tid - e;
-    mb[e] = b >= 0 ? (int)imass[b + (b >> 4)] : 0;
+  for (int e = 0; e < kBandPer; ++e) {
+    const int b = nb - 1 - kBandPer * tid - e;
+    mb[e] = b >= 0 ? (int)imass[b + b / kBandPer] : 0;
     mine += mb[e];
   }
   if (tid == 0) sh.state[3] = 0xFFFFFFFFu;
   int run = block_exclusive_scan(mine, sh.scan, nullptr);
   const int p30 = (int)(P >> 18);  // P in units of 2^-30
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const int b = nb - 1 - 16 * tid - e;
+  for (int e = 0; e < kBandPer; ++e) {
+    const int b = nb - 1 - kBandPer * tid - e;
     if (b >= 0 && run < p30 && run + mb[e] >= p30) sh.state[3] = (uint32_t)b;
     run += mb[e];
   }
@@ -1727,20 +1749,21 @@ __device__ void build_kept(const Args& a, Shared& sh, int g, unsigned char* smem
 //   * At a chunk's last pass the consumers merge the warps' states into the chunk's partial
 //     [G][128 o, max, sum, -, -]; the chunk that completes its group merges the group's
 //     partials (log-sum-exp, in chunk order) into o and lse.
-constexpr int kAttPass = 128;
+constexpr int kAttCons = kThreads / 2;          // consumer threads (the first half of the warps)
+constexpr int kAttProd = kThreads - kAttCons;    // producer threads (the second half)
+constexpr int kAttConsWarps = kAttCons / 32;
+constexpr int kAttPass = 16 * kAttConsWarps;     // tokens per pass: one 16-token tile per consumer
 constexpr int kAttIdx = kAttChunkMax + 16;
 constexpr int kAttPartStride = kHeadDim + 4;  // floats per head of a chunk partial
-constexpr int kAttCons = 256;                 // consumer threads (warps 0-7)
-constexpr int kAttProd = kThreads - kAttCons;  // producer threads (warps 8-15)
 constexpr int kAttBufBytes = kAttPass * 512 + 8 * 256;  // K rows | V rows | query rows
 constexpr uint32_t kMbarLimit = 1u << 22;      // polls of an mbarrier before a wait gives up
-// pass buffers in the ring (three when the merge scratch leaves room for them)
+// pass buffers in the ring (three when the merge scratch and the CTAs an SM holds leave room)
 template <int G>
 constexpr int att_bufs() {
-  return G >= 8 ? 2 : 3;
+  return (G >= 8 || kThreads < 512) ? 2 : 3;
 }
 // shared memory of a worker: [bufs][kAttBufBytes] | [2][kAttIdx] row indices | scratch of the
-// consumers ([8 warps][2 G] max, sum | [8 warps][G][128] o)
+// consumers ([warps][2 G] max, sum | [warps][G][128] o)
 template <int G>
 constexpr int att_scratch_off() {
   return att_bufs<G>() * kAttBufBytes + 2 * ((4 * kAttIdx + 127) & ~127);
@@ -1749,9 +1772,10 @@ template <int G>
 constexpr int att_merge_floats();
 template <int G>
 constexpr int att_smem() {
-  return att_scratch_off<G>() + 4 * (8 * (2 * G + G * kHeadDim) > att_merge_floats<G>()
-                                         ? 8 * (2 * G + G * kHeadDim)
-                                         : att_merge_floats<G>());
+  return att_scratch_off<G>() +
+         4 * (kAttConsWarps * (2 * G + G * kHeadDim) > att_merge_floats<G>()
+                  ? kAttConsWarps * (2 * G + G * kHeadDim)
+                  : att_merge_floats<G>());
 }
 enum { kDescEnd = 1, kDescFirst = 2, kDescLast = 4 };
 
@@ -1901,9 +1925,9 @@ __device__ void attend_finish(const Args& a, int c, const float (&m)[2], float (
                               const float (&ot)[8][4], float* scr) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gr = lane >> 2, t = lane & 3;
-  float* wm = scr;               // [8][G]
-  float* wl = wm + 8 * G;        // [8][G]
-  float* wo = wl + 8 * G;        // [8][G][128]
+  float* wm = scr;                           // [kAttConsWarps][G]
+  float* wl = wm + kAttConsWarps * G;        // [kAttConsWarps][G]
+  float* wo = wl + kAttConsWarps * G;        // [kAttConsWarps][G][128]
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     l[e] += __shfl_xor_sync(0xffffffffu, l[e], 4);
@@ -1928,11 +1952,11 @@ __device__ void attend_finish(const Args& a, int c, const float (&m)[2], float (
     const int h = i / kHeadDim, d = i - h * kHeadDim;
     float mxw = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) mxw = fmaxf(mxw, wm[w * G + h]);
+    for (int w = 0; w < kAttConsWarps; ++w) mxw = fmaxf(mxw, wm[w * G + h]);
     float ov = 0.f, lv = 0.f;
     if (mxw > -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
+      for (int w = 0; w < kAttConsWarps; ++w) {
         const float mw = wm[w * G + h];
         if (!(mw > -INFINITY)) continue;
         const float fw = __expf(mw - mxw);
@@ -1960,6 +1984,20 @@ template <int G>
 constexpr int att_merge_floats() {
   return kAttMaxChunks * G + 16 + 4 * kAttCons;
 }
+// o and lse of head h of group (b, kvh) from the merged float4 column c4 of o (sum acc of the
+// weighted chunk partials) and the head's max and total in hs.
+template <int G>
+__device__ __forceinline__ void merge_store(const Args& a, int b, int kvh, int h, int c4,
+                                            const float4& acc, const float* hs) {
+  const float lt = hs[G + h];
+  const bool any = lt > 0.f;
+  const size_t bh = (size_t)b * a.hq + kvh * G + h;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (any) o = make_float4(acc.x / lt, acc.y / lt, acc.z / lt, acc.w / lt);
+  reinterpret_cast<float4*>(a.o + bh * kHeadDim)[c4] = o;
+  if (c4 == 0) a.lse[bh] = any ? hs[h] + __logf(lt) : -INFINITY;
+}
+
 template <int G>
 __device__ void merge_group(const Args& a, int g, int c0, int nch, float* scr) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1974,59 +2012,74 @@ __device__ void merge_group(const Args& a, int g, int c0, int nch, float* scr) {
     wm[i] = l > 0.f ? m : -INFINITY;
   }
   bar_named(2, kAttCons);
-  if (warp < G) {
+  for (int hw = warp; hw < G; hw += kAttConsWarps) {  // warp hw: head hw
     float mx = -INFINITY;
-    for (int c = lane; c < nch; c += 32) mx = fmaxf(mx, wm[c * G + warp]);
+    for (int c = lane; c < nch; c += 32) mx = fmaxf(mx, wm[c * G + hw]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float tot = 0.f;
     for (int c = lane; c < nch; c += 32) {
-      const float m = wm[c * G + warp];
+      const float m = wm[c * G + hw];
       const float w = m > -INFINITY ? __expf(m - mx) : 0.f;
-      wm[c * G + warp] = w;
+      wm[c * G + hw] = w;
       if (w > 0.f)
-        tot = fmaf(w, ldcg_f(part + (size_t)(c * G + warp) * kAttPartStride + kHeadDim + 1), tot);
+        tot = fmaf(w, ldcg_f(part + (size_t)(c * G + hw) * kAttPartStride + kHeadDim + 1), tot);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
     if (lane == 0) {
-      hs[warp] = mx;
-      hs[G + warp] = tot;
+      hs[hw] = mx;
+      hs[G + hw] = tot;
     }
   }
   bar_named(2, kAttCons);
-  constexpr int kCols = G * kHeadDim / 4, kPer = kAttCons / kCols;
-  const int col = tid % kCols, r = tid / kCols, h = col / (kHeadDim / 4);
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr int kCols = G * kHeadDim / 4;
+  if constexpr (kAttCons >= kCols) {
+    constexpr int kPer = kAttCons / kCols;
+    const int col = tid % kCols, r = tid / kCols, h = col / (kHeadDim / 4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
-  for (int c = r; c < nch; c += kPer) {
-    const float w = wm[c * G + h];
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(part + (size_t)(c * G + h) *
-                                                                      kAttPartStride) +
-                            (col % (kHeadDim / 4)));
-    acc.x = fmaf(w, v.x, acc.x);
-    acc.y = fmaf(w, v.y, acc.y);
-    acc.z = fmaf(w, v.z, acc.z);
-    acc.w = fmaf(w, v.w, acc.w);
-  }
-  red[tid] = acc;
-  bar_named(2, kAttCons);
-  if (r == 0) {
-#pragma unroll
-    for (int k = 1; k < kPer; ++k) {
-      const float4 v = red[k * kCols + col];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+    for (int c = r; c < nch; c += kPer) {
+      const float w = wm[c * G + h];
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(part + (size_t)(c * G + h) *
+                                                                        kAttPartStride) +
+                              (col % (kHeadDim / 4)));
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
     }
-    const float lt = hs[G + h];
-    const bool any = lt > 0.f;
-    const size_t bh = (size_t)b * a.hq + kvh * G + h;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (any) o = make_float4(acc.x / lt, acc.y / lt, acc.z / lt, acc.w / lt);
-    reinterpret_cast<float4*>(a.o + bh * kHeadDim)[col % (kHeadDim / 4)] = o;
-    if (col % (kHeadDim / 4) == 0) a.lse[bh] = any ? hs[h] + __logf(lt) : -INFINITY;
+    red[tid] = acc;
+    bar_named(2, kAttCons);
+    if (r == 0) {
+#pragma unroll
+      for (int k = 1; k < kPer; ++k) {
+        const float4 v = red[k * kCols + col];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      merge_store<G>(a, b, kvh, h, col % (kHeadDim / 4), acc, hs);
+    }
+  } else {
+    // more float4 columns than consumer threads: each thread sums whole columns
+    for (int col = tid; col < kCols; col += kAttCons) {
+      const int h = col / (kHeadDim / 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+      for (int c = 0; c < nch; ++c) {
+        const float w = wm[c * G + h];
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(part + (size_t)(c * G + h) *
+                                                                          kAttPartStride) +
+                                (col % (kHeadDim / 4)));
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
+      }
+      merge_store<G>(a, b, kvh, h, col % (kHeadDim / 4), acc, hs);
+    }
   }
   bar_named(2, kAttCons);  // the scratch is reused
 }
@@ -2311,7 +2364,7 @@ __device__ void attend_worker(const Args& a, Shared& sh, unsigned char* smem) {
 
 // ------------------------------------------------------------------------------ the kernel
 template <int G>
-__global__ void __launch_bounds__(kThreads, 1) k_step(const __grid_constant__ Args a) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) k_step(const __grid_constant__ Args a) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ Shared sh;
   // wait for the previous grid in the stream (launched programmatically), then let the next one
@@ -2446,16 +2499,22 @@ int smem_need(int g, int max_pages, int max_budget, int s_chunk) {
 // Dynamic shared memory per CTA: everything the device grants one block beyond the static part
 // (the estimate's stages and the staged weights use what the minimum leaves).
 int smem_avail(int g) {
-  int dev = 0, optin = 0;
+  int dev = 0, optin = 0, per_sm = 0;
   cudaGetDevice(&dev);
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     optin = 227 * 1024;
+  if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+      cudaSuccess)
+    per_sm = 228 * 1024;
   cudaFuncAttributes fa{};
   const void* k = kernel_for(g);
   size_t stat = 1024;
   if (k && cudaFuncGetAttributes(&fa, k) == cudaSuccess) stat = fa.sharedSizeBytes;
   cudaGetLastError();
-  return (int)((size_t)optin - stat - 1024) & ~127;
+  // kCtasPerSm CTAs share the SM's shared memory, 1 KB of it reserved per CTA
+  long long avail = (long long)per_sm / kCtasPerSm - 1024;
+  avail = avail < optin ? avail : optin;
+  return (int)(avail - (long long)stat - (kCtasPerSm == 1 ? 1024 : 0)) & ~127;
 }
 
 }  // namespace
@@ -2467,8 +2526,9 @@ Plan plan(int batch, int hq, int hkv, int max_pages, int max_budget) {
   pl.sel_words = ((max_pages + 31) / 32 + 3) & ~3;  // rows of whole 16-byte pieces
   pl.cand_stride = kPage * max_budget;
   pl.kept_words = (pl.cand_stride + 31) / 32;
-  const int sms = num_sms();
-  pl.grid = sms;  // one 512-thread CTA per SM, every CTA resident
+  // the CTAs of the grid: kCtasPerSm per SM, every CTA resident ("sms" below counts CTAs)
+  const int sms = num_sms() * kCtasPerSm;
+  pl.grid = sms;
   pl.smem_bytes = smem_avail(g);
   // work list: score chunks so the pages fill every CTA (one wave when the groups are few and
   // short, about four otherwise); estimate and attention slices likewise per group
@@ -2618,7 +2678,7 @@ cudaError_t launch(const Args& a, const Plan& pl, cudaStream_t s) {
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, pl.smem_bytes);
   if (e != cudaSuccess) return e;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;  // the grid could not all be resident
+  if (per_sm < kCtasPerSm) return cudaErrorInvalidConfiguration;  // not every CTA resident
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)pl.grid);
   cfg.blockDim = dim3(kThreads);
@@ -2637,5 +2697,5 @@ cudaError_t launch(const Args& a, const Plan& pl, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-}  // namespace step
+}  // namespace TWL_STEP_NS
 }  // namespace twl

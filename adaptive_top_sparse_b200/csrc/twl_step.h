@@ -108,4 +108,19 @@ cudaError_t launch(const Args& a, const Plan& pl, cudaStream_t s);
 void set_test_waits(uint32_t spin_limit, int stall_estimate);
 
 }  // namespace step
+
+// The same kernel built with 256-thread CTAs, two per SM (twl_step_256.cu), for batches with
+// more (sequence, kv-head) groups than SMs.  Same arguments and workspace contents.
+namespace step256 {
+step::Plan plan(int batch, int hq, int hkv, int max_pages, int max_budget);
+size_t workspace_bytes(int batch, int hq, int hkv, int max_pages, int max_budget);
+void carve(step::Args& a, char* ws, const step::Plan& pl, int batch, int hq, int hkv,
+           int max_pages);
+cudaError_t launch(const step::Args& a, const step::Plan& pl, cudaStream_t s);
+void set_test_waits(uint32_t spin_limit, int stall_estimate);
+}  // namespace step256
+
+// Whether the decode step of `groups` (sequence, kv-head) groups runs the 256-thread build
+// (measured: 306 vs 424 us per layer-step at 512 groups; no gain at 128 groups on 148 SMs).
+inline bool step_wide(int groups, int sms) { return groups > sms; }
 }  // namespace twl

@@ -584,6 +584,26 @@ def test_decode_step_repeated_launches_on_one_workspace():
     assert layer.status()[0] == twl.TWL_OK
 
 
+@pytest.mark.parametrize("shape", [
+    (20, 8, 8, 700),     # 160 groups, group size 1
+    (40, 16, 8, 500),    # 320 groups, group size 2
+    (80, 16, 2, 300),    # 160 groups, group size 8
+], ids=["g1", "g2", "g8"])
+def test_decode_step_two_ctas_per_sm(shape):
+    """More groups than SMs: the 256-thread build (two CTAs per SM) runs; every group size it is
+    built for, sampled groups against the oracle."""
+    batch, hq, hkv, n = shape
+    lens = [n + 29 * i for i in range(batch)]
+    wl = synth.make_decode("wide", batch, hq, hkv, lens, seed=51 + hkv, permute_pages=True,
+                           temperature=True)
+    layer = DecodeLayer.from_workload(wl)
+    layer.build_aux()
+    st, o, lse = _run_step(wl, layer)
+    for bb, kvh in [(0, 0), (batch // 3, hkv - 1), (batch - 1, hkv // 2)]:
+        check_step_group(wl, bb, kvh, st, o, lse)
+    assert layer.status()[0] == twl.TWL_OK
+
+
 def test_decode_step_more_groups_than_sms():
     """320 (sequence, kv-head) groups, more than twice the SMs: several items of every kind per
     CTA; sampled groups."""
