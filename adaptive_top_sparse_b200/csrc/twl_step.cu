@@ -1729,7 +1729,8 @@ __device__ void build_kept(const Args& a, Shared& sh, int g, unsigned char* smem
 // ------------------------------------------------------------------------------ attention
 // The attention work list ([Notes] "Key designs", load balancing: the heads' kept tokens differ
 // ~50x, so each group's kept pages are cut into chunks that any CTA takes).  A worker is warp-
-// specialised: warps 8-15 produce, warps 0-7 consume, and the two sides meet only at mbarriers
+// specialised: the upper half of the warps produce, the lower half consume (8 and 8 in the
+// 512-thread build, 4 and 4 in the 256-thread one), and the two sides meet only at mbarriers
 // on a ring of pass buffers, so that the copies of later passes are issued while earlier ones are
 // computed.
 //   * Producers take the chunks from the queue (ticket, wait until published), expand a chunk's
@@ -1976,7 +1977,8 @@ __device__ void attend_finish(const Args& a, int c, const float (&m)[2], float (
 // group's nch chunk partials (slots c0 ...) -> o, lse of every head (o = 0, lse = -inf when
 // nothing was kept).  The max of every (chunk, head) is staged in shared memory in one round of
 // loads; warp h turns head h's into chunk weights exp(max_c - max) and the head's total;
-// then each float4 of o is summed by 8 / G threads over interleaved chunks (their loads are
+// then each float4 of o is summed by kAttCons / (32 G) threads over interleaved chunks, or each
+// thread sums whole float4 columns when there are more columns than threads (their loads are
 // independent of the sums, so they stay in flight together) and their sums are added in a fixed
 // order.  scr: the consumers' scratch (kAttMergeFloats floats at least).
 constexpr int kAttMaxChunks = 512;  // chunks of one group at most (16 * kMaxPages / kAttChunkMax)
@@ -2110,8 +2112,8 @@ __device__ int ticket_wait(const Args& a, int c) {
   }
 }
 
-// Producers (warps 8-15): take chunks until the queue is done, copy their passes into the ring,
-// then post the end.  The next chunk is prepared while the current one's passes are issued, one
+// Producers (the upper half of the warps): take chunks until the queue is done, copy their
+// passes into the ring, then post the end.  The next chunk is prepared while the current one's passes are issued, one
 // step per pass (take its queue ticket; see it published and read its entry; expand its pages
 // into the other row-index stage), so a chunk switch leaves no gap in the copies.
 template <int G>
@@ -2278,8 +2280,8 @@ __device__ void attend_produce(const Args& a, Shared& sh, unsigned char* smem) {
   cp_async_wait_all();
 }
 
-// Consumers (warps 0-7): compute the posted passes until the end; at a chunk's last pass write
-// its partial, count it, and merge the group when it is the last.
+// Consumers (the lower half of the warps): compute the posted passes until the end; at a
+// chunk's last pass write its partial, count it, and merge the group when it is the last.
 template <int G>
 __device__ void attend_consume(const Args& a, Shared& sh, unsigned char* smem) {
   constexpr int NB = att_bufs<G>();
