@@ -86,14 +86,16 @@ class DecodeLayer:
     def decode(self, q, p: float = 0.85, eps: float = 1e-6, stats: dict | None = None,
                stream=None):
         """One select -> estimate -> prune -> union -> attend step for query q [B][Hq][128] fp16
-        (device tensor).  Returns (o, lse) device tensors owned by the layer."""
+        (device tensor), one launch of the library's persistent step kernel.  Returns the
+        layer's (o, lse) device tensors (o and lse are attributes a caller may point at slices
+        of its own buffers)."""
         st = twl.make_stats(**stats) if stats is not None else None
         twl.twl_decode_step(q, self.num_q_heads, self.kv, self.aux, self.budget_pages,
                             self.budget_div, self.max_budget, p, eps, self.o, self.lse, st,
                             self.ws, stream)
         return self.o, self.lse
 
-    # ------------------------------------------------------------------ cluster-level selector
+    # ------------------------------------------------------------------ other paths
     def staged(self) -> "Staged":
         """The same step as five separate library calls (see Staged)."""
         return Staged(self)
