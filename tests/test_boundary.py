@@ -5,6 +5,9 @@ before any CUDA call, so nothing is dereferenced."""
 import ctypes as C
 import os
 import re
+import shutil
+import subprocess
+import sys
 
 import pytest
 
@@ -41,9 +44,36 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(-6, 1):
+    for code in range(twl.TWL_ERR_SCRATCH_LIMIT, 1):
         assert twl.twl_status_string(code) != "unknown status"
     assert twl.twl_status_string(-99) == "unknown status"
+
+
+def test_package_without_the_library_fails_at_import(tmp_path):
+    """The Python side has no fallback: a copy of the package without libtwl.so refuses to
+    import, both the binding and the layer wrapper built on it."""
+    src = os.path.join(ROOT, "adaptive_top_sparse_b200")
+    dst = tmp_path / "adaptive_top_sparse_b200"
+    dst.mkdir()
+    for name in os.listdir(src):
+        if name.endswith(".py"):
+            shutil.copy(os.path.join(src, name), dst / name)
+    for mod in ("twl", "layer"):
+        r = subprocess.run([sys.executable, "-c", f"import adaptive_top_sparse_b200.{mod}"],
+                           cwd=tmp_path, capture_output=True, text=True, timeout=300,
+                           env=dict(os.environ, PYTHONPATH=str(tmp_path)))
+        assert r.returncode != 0, mod
+        assert "ImportError" in r.stderr and "libtwl.so is missing" in r.stderr, r.stderr[-500:]
+
+
+def test_package_never_imports_the_oracle():
+    """The oracle is test infrastructure: nothing in the package imports or opens it."""
+    pkg = os.path.join(ROOT, "adaptive_top_sparse_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for name in files:
+            if name.endswith((".py", ".cu", ".h", ".cuh")):
+                text = open(os.path.join(dirpath, name)).read()
+                assert not re.search(r"\boracle\b", text), os.path.join(dirpath, name)
 
 
 def _kv(**over):
