@@ -331,7 +331,13 @@ twl_status twl_sparse_decode_noalloc(const void* q, int32_t num_q_heads, const t
  * one workspace must be stream-ordered.  Device-side errors are reported through the workspace
  * flags (twl_device_status): page-table entries outside the pool and bad sequence lengths are
  * skipped (TWL_FLAG_BAD_INDEX); a wait between work items that gives up after its bounded number
- * of polls aborts the launch (TWL_FLAG_TIMEOUT, outputs undefined). */
+ * of polls aborts the launch (TWL_FLAG_TIMEOUT, outputs undefined).
+ * Shapes: every work item keeps one head's page-score keys (4 bytes per page of the page-table
+ * stride) in its CTA's shared memory.  With more (sequence, kv-head) groups than SMs the step runs
+ * two 256-thread CTAs per SM, each with half of the SM's shared memory; there max_pages above
+ * 23296 (on a 148-SM B200: 228 KB per SM) returns TWL_ERR_UNSUPPORTED and launches nothing.
+ * Split such a batch into calls of at most SM-count groups, which take the one-CTA-per-SM build
+ * and accept max_pages up to 32768. */
 twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
                            const twl_k_aux* aux, int32_t budget_pages, int32_t budget_div,
                            int32_t max_budget, float p, float eps, float* o, float* lse,
