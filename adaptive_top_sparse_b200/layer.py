@@ -20,7 +20,31 @@ def budget_bound(max_pages: int, budget_pages: int, budget_div: int) -> int:
     return -(-max_pages // budget_div)
 
 
+def expect_tensor(name: str, t, shape, dtype, device) -> None:
+    """Raises unless `t` is a contiguous tensor of `shape` and `dtype` on `device`.  The library
+    takes raw pointers: it cannot tell a host buffer, a tensor on another GPU or a mis-shaped one
+    from a good one, and a kernel would read or write the wrong memory."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.device != device:
+        raise ValueError(f"{name}: tensor on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: tensor is not contiguous")
+
+
 class DecodeLayer:
+    """One layer's paged KV cache on a GPU and its decode step.
+
+    k, v: fp16 [num_phys_pages][num_kv_heads][16][128]; page_table: int32 [B][max_pages] (logical
+    page -> physical page, -1 unmapped); seq_lens: int32 [B].  Arrays on the host are copied to
+    `device`.  budget_pages > 0 fixes the pages each head selects, else ceil(P_b / budget_div).
+    Every call on a layer uses the layer's one workspace: issue them in order on one stream (the
+    current stream when `stream` is None)."""
+
     def __init__(self, k, v, page_table, seq_lens, num_q_heads: int, num_kv_heads: int,
                  budget_pages: int = 0, budget_div: int = 4, device="cuda"):
         dev = torch.device(device)
@@ -64,6 +88,9 @@ class DecodeLayer:
     def append(self, k_new, v_new, stream=None) -> None:
         """Append one token per sequence at position seq_lens[b] (K, V, INT4 K and page bounds
         in one launch) and advance seq_lens.  The page for the position must be mapped."""
+        for name, t in (("k_new", k_new), ("v_new", v_new)):
+            expect_tensor(name, t, (self.batch, self.num_kv_heads, 128), torch.float16,
+                          self.k.device)
         twl.twl_append_token(self.kv, self.aux, k_new, v_new, True, self.ws, stream)
 
     # ------------------------------------------------------------------ stats buffers
@@ -89,11 +116,16 @@ class DecodeLayer:
         (device tensor), one launch of the library's persistent step kernel.  Returns the
         layer's (o, lse) device tensors (o and lse are attributes a caller may point at slices
         of its own buffers)."""
+        self.expect_query(q)
         st = twl.make_stats(**stats) if stats is not None else None
         twl.twl_decode_step(q, self.num_q_heads, self.kv, self.aux, self.budget_pages,
                             self.budget_div, self.max_budget, p, eps, self.o, self.lse, st,
                             self.ws, stream)
         return self.o, self.lse
+
+    def expect_query(self, q) -> None:
+        """q must be fp16 [B][Hq][128], contiguous, on the layer's GPU."""
+        expect_tensor("q", q, (self.batch, self.num_q_heads, 128), torch.float16, self.k.device)
 
     # ------------------------------------------------------------------ other paths
     def staged(self) -> "Staged":
@@ -150,6 +182,7 @@ class DoubleP:
     def decode(self, q, p_cluster: float = 0.95, p: float = 0.85, eps: float = 1e-6,
                stream=None):
         L = self.layer
+        L.expect_query(q)
         hq, mp = L.num_q_heads, L.max_pages
         cs = 16 * mp
         twl.twl_select_clusters_top_p(q, hq, L.kv, self.centroids, p_cluster, eps, self.sel,
@@ -198,6 +231,7 @@ class Staged:
 
     def decode(self, q, p: float = 0.85, eps: float = 1e-6, stream=None):
         L = self.layer
+        L.expect_query(q)
         hq, mb = L.num_q_heads, L.max_budget
         cs = 16 * mb
         twl.twl_select_pages(q, hq, L.kv, L.aux.bounds, L.budget_pages, L.budget_div, mb,

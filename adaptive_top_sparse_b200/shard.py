@@ -28,12 +28,21 @@ def kv_head_range(num_kv_heads: int, rank: int, world: int) -> tuple[int, int]:
 def shard_layer(k, v, q, num_q_heads: int, num_kv_heads: int, rank: int, world: int):
     """The rank's slices of one layer: K and V [P][Hkv][16][128] along the kv-head axis, q
     [B][Hq][128] along the q-head axis (the q-heads of the owned groups).  Works on numpy arrays
-    and torch tensors alike.  Returns (k, v, q, num_q_heads, num_kv_heads) of the shard."""
+    and torch tensors alike; the slices are returned as contiguous copies, the layout the library
+    reads.  Returns (k, v, q, num_q_heads, num_kv_heads) of the shard."""
     if num_q_heads % num_kv_heads:
         raise ValueError("num_q_heads must be a multiple of num_kv_heads")
     g = num_q_heads // num_kv_heads
     lo, hi = kv_head_range(num_kv_heads, rank, world)
-    return (k[:, lo:hi], v[:, lo:hi], q[:, g * lo:g * hi], g * (hi - lo), hi - lo)
+
+    def dense(x):
+        if hasattr(x, "contiguous"):
+            return x.contiguous()
+        import numpy as np
+        return np.ascontiguousarray(x)
+
+    return (dense(k[:, lo:hi]), dense(v[:, lo:hi]), dense(q[:, g * lo:g * hi]), g * (hi - lo),
+            hi - lo)
 
 
 def gather_heads(o_local, lse_local, num_q_heads: int, num_kv_heads: int, world: int, group=None):

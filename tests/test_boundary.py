@@ -9,6 +9,7 @@ import shutil
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 from adaptive_top_sparse_b200 import twl
@@ -196,3 +197,37 @@ def test_workspace_sizes():
     assert wb(twl.TWL_OP_SELECT, 1, 32, 8, 2048) >= 256 + 32 * 2048 * 4
     assert wb(twl.TWL_OP_SPARSE_DECODE, 1, 32, 8, 0, 0, 0, 4096) > 256
     assert wb(twl.TWL_OP_DECODE_STEP, -1, 32, 8, 2048, 512) == 0
+
+
+def test_layer_rejects_host_and_misshaped_tensors_before_any_call():
+    """DecodeLayer checks q (and the appended rows) before handing raw pointers to the library:
+    a host tensor, another device, a wrong dtype or shape, or a strided view raises at once.
+    The layer here is a bare object whose cache lives on the meta device, so any call that got
+    through to the library would fail differently."""
+    import torch
+    from adaptive_top_sparse_b200.layer import DecodeLayer, Staged, expect_tensor
+
+    layer = DecodeLayer.__new__(DecodeLayer)
+    layer.k = torch.empty((4, 2, 16, 128), dtype=torch.float16, device="meta")
+    layer.batch, layer.num_q_heads, layer.num_kv_heads = 3, 8, 2
+    good = torch.empty((3, 8, 128), dtype=torch.float16, device="meta")
+    layer.expect_query(good)
+    bad = {
+        "host tensor": torch.zeros((3, 8, 128), dtype=torch.float16),
+        "dtype": torch.empty((3, 8, 128), dtype=torch.float32, device="meta"),
+        "shape": torch.empty((3, 8, 64), dtype=torch.float16, device="meta"),
+        "strided": torch.empty((3, 128, 8), dtype=torch.float16, device="meta").transpose(1, 2),
+    }
+    for what, q in bad.items():
+        with pytest.raises(ValueError):
+            layer.decode(q)
+        stg = Staged.__new__(Staged)
+        stg.layer = layer
+        with pytest.raises(ValueError):
+            stg.decode(q)
+    with pytest.raises(TypeError):
+        layer.decode(np.zeros((3, 8, 128), np.float16))
+    rows = torch.zeros((3, 2, 128), dtype=torch.float16)             # on the host
+    with pytest.raises(ValueError):
+        layer.append(rows, rows)
+    expect_tensor("x", rows, (3, 2, 128), torch.float16, rows.device)

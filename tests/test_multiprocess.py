@@ -155,3 +155,18 @@ def test_kv_head_ranges_cover_every_head_once():
             assert owned == list(range(hkv))
     with pytest.raises(ValueError):
         kv_head_range(2, 0, 3)
+
+
+def test_shard_slices_are_contiguous_for_numpy_and_torch():
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+    from adaptive_top_sparse_b200.shard import shard_layer
+    k = np.arange(5 * 4 * 16 * 128, dtype=np.float32).reshape(5, 4, 16, 128).astype(np.float16)
+    q = np.arange(2 * 12 * 128, dtype=np.float32).reshape(2, 12, 128).astype(np.float16)
+    for conv in (lambda x: x, torch.from_numpy):
+        ks, vs, qs, hq, hkv = shard_layer(conv(k), conv(k), conv(q), 12, 4, 1, 2)
+        assert (hq, hkv) == (6, 2)
+        for x in (ks, vs, qs):
+            assert x.flags["C_CONTIGUOUS"] if isinstance(x, np.ndarray) else x.is_contiguous()
+        assert np.array_equal(np.asarray(qs), q[:, 6:12]) and np.array_equal(np.asarray(ks), k[:, 2:4])
