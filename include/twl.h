@@ -337,7 +337,13 @@ twl_status twl_sparse_decode_noalloc(const void* q, int32_t num_q_heads, const t
  * two 256-thread CTAs per SM, each with half of the SM's shared memory; there max_pages above
  * 23296 (on a 148-SM B200: 228 KB per SM) returns TWL_ERR_UNSUPPORTED and launches nothing.
  * Split such a batch into calls of at most SM-count groups, which take the one-CTA-per-SM build
- * and accept max_pages up to 32768. */
+ * and accept max_pages up to 32768.
+ * Residency: the grid is one (or two) CTAs per SM and each CTA's first work item is fixed by its
+ * index, so the launch counts on all of its CTAs running at once.  Do not run two
+ * twl_decode_step launches concurrently (on different streams or processes sharing the GPU),
+ * nor next to a kernel that keeps SMs busy for the whole step: CTAs that cannot start hold up
+ * the items waiting on theirs, and those waits give up after their bound (2^22 polls, each at
+ * least a 64 ns sleep) with TWL_FLAG_TIMEOUT and undefined outputs rather than hang. */
 twl_status twl_decode_step(const void* q, int32_t num_q_heads, const twl_paged_kv* kv,
                            const twl_k_aux* aux, int32_t budget_pages, int32_t budget_div,
                            int32_t max_budget, float p, float eps, float* o, float* lse,
