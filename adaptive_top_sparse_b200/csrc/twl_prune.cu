@@ -7,9 +7,10 @@
 //
 // This is the direct form of the search, used for rows that the read-once kernel of
 // twl_prune_rows.cu does not take (a stride that is not a multiple of 4 weights or above 262144,
-// or a base that is not 16-byte aligned); TWL_PRUNE_BISECT=1 selects it for every row.  One block
-// per row.  The row is staged once in shared memory when it fits (else it is re-read from global
-// memory / L2 each round).  Every round is one block reduction of the mass above the midpoint, in
+// or a base that is not 16-byte aligned); a build with -DTWL_PRUNE_BISECT_ONLY takes it for every
+// row (a compile-time option; nothing selects it at run time).  One block per row.  The row is
+// staged once in shared memory when it fits (else it is re-read from global memory / L2 each
+// round).  Every round is one block reduction of the mass above the midpoint, in
 // a fixed order, so all threads take the same branch.  The kept indices are compacted in
 // ascending order with a block scan.
 #include <stdlib.h>
