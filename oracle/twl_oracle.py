@@ -268,6 +268,17 @@ def top_p_sort(w: np.ndarray, p: float):
     return k_star, m_star, kept
 
 
+def top_p_whole(w: np.ndarray, p: float):
+    """``top_p_sort`` for a normalised distribution (softmax weights summing to 1), with p = 1
+    read as the whole distribution: every entry is kept and m* = 0.  The sort form cannot decide
+    p = 1 by itself: the fp64 sum of the largest weights can round to exactly 1.0 while positive
+    weights remain, and an exact sum of the rounded weights can land on either side of 1."""
+    w = np.asarray(w)
+    if p >= 1.0:
+        return w.size, w.dtype.type(0.0), np.arange(w.size, dtype=np.int64)
+    return top_p_sort(w, p)
+
+
 def top_p_bisect(w: np.ndarray, p: float, eps: float, max_iter: int = 64):
     """Threshold bisection of [Notes] "Key designs" (efficient top-p) / [Summary] 4.2.
 
@@ -500,7 +511,7 @@ def select_clusters(q, cen, page_table, seq_lens, num_q_heads, num_kv_heads, p_c
         n = int(seq_lens[b])
         for h in range(num_q_heads):
             w = cluster_weights(q[b, h], cen, page_table, b, h // g, n)
-            _, _, kept = top_p_sort(w, p_cluster)
+            _, _, kept = top_p_whole(w, p_cluster)
             out[(b, h)] = (w, np.sort(np.asarray(kept, dtype=np.int64)))
     return out
 
@@ -522,7 +533,7 @@ def decode_step(wl, bounds=None, k_int4=None, k_sz=None, with_attention=True):
     for (b, h), (sc, pages) in sel.items():
         cand, w = estimate_head(wl.q[b, h], k_int4, k_sz, wl.page_table, b, h // g,
                                 int(wl.seq_lens[b]), pages, wl.head_dim)
-        k_star, m_star, kept = top_p_sort(w, wl.p)
+        k_star, m_star, kept = top_p_whole(w, wl.p)
         heads[(b, h)] = dict(scores=sc, sel=pages, cand=cand, w=w, k_star=k_star,
                              m_star=m_star, kept=kept, kept_tok=cand[kept])
     groups = {}

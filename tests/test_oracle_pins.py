@@ -369,6 +369,23 @@ def check_top_p_golden(top_p_fn):
     return ok
 
 
+def test_p_one_keeps_the_whole_distribution():
+    """Reading R10 by hand: w = (1/2, 1/4, 1/4 - 2^-55, 2^-55) sums to exactly 1, and every
+    entry is positive, so mass 1 needs all four.  The fp64 prefix 3/4 + (1/4 - 2^-55) = 1 - 2^-55
+    lies within half a unit (2^-54) of 1 and rounds to 1.0, so the sort form stops at three;
+    the step's reading keeps all four with m* = 0, as the bisection does."""
+    d = 2.0 ** -55
+    w = np.array([0.5, 0.25, 0.25 - d, d], dtype=F64)
+    assert math.fsum(w) == 1.0 and np.all(w > 0)
+    assert O.top_p_sort(w, 1.0)[0] == 3                  # the rounding the reading avoids
+    k, m, kept = O.top_p_whole(w, 1.0)
+    assert k == 4 and m == 0.0 and list(kept) == [0, 1, 2, 3]
+    assert list(O.top_p_bisect(w, 1.0, 1e-6)[1]) == [0, 1, 2, 3]
+    for p in (0.5, 0.75, 0.9):                           # below 1 it is the sort form
+        a, b = O.top_p_whole(w, p), O.top_p_sort(w, p)
+        assert a[0] == b[0] and a[1] == b[1] and list(a[2]) == list(b[2])
+
+
 def test_top_p_golden():
     assert check_top_p_golden(O.top_p_sort)
 
@@ -626,8 +643,8 @@ def test_dense_limit_equals_full_attention():
         v = O.gather_tokens(wl.v, wl.page_table, 0, kvh, toks)
         o, lse = O.attention(wl.q[0, h], k, v, 1 / math.sqrt(128))
         grp = r["groups"][(0, kvh)]
-        if len(grp["union"]) == 300:
-            assert np.allclose(grp["o"][h], o, atol=1e-12)
+        assert len(grp["union"]) == 300          # p = 1 keeps every candidate (R10)
+        assert np.allclose(grp["o"][h], o, atol=1e-12)
 
 
 # ------------------------------------------------------------------------------------- mutations

@@ -72,3 +72,67 @@ def test_bisection_equals_its_threshold_replay(w, frac, eps):
     p = frac * float(w.astype(F64).sum())
     m, _ = O.top_p_bisect(w, p, eps)
     assert F32(m) == _bisect_replay_from_threshold(w, p, eps)
+
+
+# ------------------------------------------------------------------ the whole step, as invariants
+
+layers = st.fixed_dictionaries({
+    "seed": st.integers(0, 10_000),
+    "hkv": st.sampled_from([1, 2]),
+    "g": st.sampled_from([1, 2, 4]),
+    "lens": st.lists(st.integers(1, 300), min_size=1, max_size=2),
+    "p": st.sampled_from([0.5, 0.85, 0.95, 1.0]),
+    "temperature": st.booleans(),
+})
+
+
+@settings(max_examples=30, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(layers)
+def test_decode_step_invariants(c):
+    """Generated small layers (ragged lengths, 1 to 4 heads per group, permuted pages, p up to 1):
+    every stage of the oracle's step satisfies what the method defines it to be, checked from the
+    definitions rather than by re-running the oracle's routines.
+      selection   ceil(P_b / 4) distinct pages of the sequence, ascending
+      candidates  exactly the valid tokens of the selected pages
+      estimate    weights >= 0 summing to 1
+      top-p       kept = {W >= m*}; its mass reaches p; the weights above m* alone do not
+                  (at p = 1 every candidate is kept)
+      union       the union of the group's kept tokens, inside the sequence
+      attention   o is a convex combination of the union's V rows (channel-wise inside their
+                  range) and lse lies in [max logit, max logit + ln |U|]"""
+    from workloads import synth
+    hkv, g = c["hkv"], c["g"]
+    wl = synth.make_decode("prop", len(c["lens"]), g * hkv, hkv, c["lens"], seed=c["seed"],
+                           permute_pages=True, temperature=c["temperature"], p=c["p"])
+    r = O.decode_step(wl)
+    scale = 1 / np.sqrt(128)
+    for b, n in enumerate(wl.seq_lens):
+        n = int(n)
+        pb = -(-n // 16)
+        for kvh in range(hkv):
+            union = set()
+            for h in range(kvh * g, (kvh + 1) * g):
+                hd = r["heads"][(b, h)]
+                sel = list(hd["sel"])
+                assert len(sel) == -(-pb // 4) and sel == sorted(set(sel))
+                assert all(0 <= j < pb for j in sel)
+                assert list(hd["cand"]) == [t for t in range(n) if t // 16 in set(sel)]
+                w = hd["w"]
+                assert np.all(w >= 0) and abs(w.sum() - 1.0) < 1e-12
+                m = hd["m_star"]
+                assert list(hd["kept"]) == list(np.nonzero(w >= m)[0])
+                if wl.p == 1.0:                       # R10: p = 1 keeps every candidate
+                    assert len(hd["kept"]) == len(w)
+                else:
+                    assert w[w >= m].sum() >= wl.p and w[w > m].sum() < wl.p
+                union |= set(hd["kept_tok"].tolist())
+            grp = r["groups"][(b, kvh)]
+            assert list(grp["union"]) == sorted(union) and max(union) < n
+            rows = [(int(wl.page_table[b, t // 16]), t % 16) for t in sorted(union)]
+            kk = np.stack([wl.k[ph, kvh, i] for ph, i in rows]).astype(F64)
+            vv = np.stack([wl.v[ph, kvh, i] for ph, i in rows]).astype(F64)
+            for h in range(kvh * g, (kvh + 1) * g):
+                o, lse = grp["o"][h], grp["lse"][h]
+                assert np.all(o >= vv.min(axis=0) - 1e-12) and np.all(o <= vv.max(axis=0) + 1e-12)
+                top = float((kk @ wl.q[b, h].astype(F64)).max()) * scale
+                assert top - 1e-12 <= lse <= top + np.log(len(rows)) + 1e-12
