@@ -145,3 +145,14 @@ def test_prune_row_checks():
     low = F32(m_star) * F32(0.5)
     with pytest.raises(AssertionError):
         K.check_prune_row(row, low, int(np.count_nonzero(row >= low)), None, 0.9, 1e-6)
+
+
+def test_prune_check_at_p_one_takes_the_whole_row():
+    """At p = 1 a pruner keeps every weight (m = 0).  fp32 weights that sum a little above 1
+    (0.5 + 0.3 + 0.2 in fp32 is 1 + 1.5e-8) reach 1.0 after three of five entries, yet keeping
+    all five is the reading's result and passes.  Below p = 1 the minimal set still binds:
+    keeping all five at p = 0.9 fails."""
+    w = np.array([0.5, 0.3, 0.2, 1e-8, 1e-8], np.float32)
+    K.check_prune_row(w, 0.0, 5, None, 1.0, 1e-6, "p=1")
+    with pytest.raises(AssertionError):
+        K.check_prune_row(w, 0.0, 5, None, 0.9, 1e-6, "too many at p=0.9")

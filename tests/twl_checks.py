@@ -5,7 +5,9 @@ Criteria (from the method's statement of correctness):
   estimated weights      |W_gpu - W_or| <= 1e-3 * W_or + 1e-9 per candidate
   pruning (on the W the device pruner consumed)
       kept = {i : W_i >= m} exactly;  sum_kept W (fp64) >= p - 1e-5;
-      |kept| <= k* + #{i : m* - eps <= W_i <= m*}   (k*, m* from the sort-based oracle)
+      |kept| <= k* + #{i : m* - eps <= W_i <= m*}   (k*, m* from the sort-based oracle; at
+      p = 1 the whole row, so a row whose fp32 weights sum a little above 1 is not held to a
+      prefix that reaches 1.0 early)
   union                  exactly the union of the heads' kept token ids
   attention              |o_gpu - o_or| <= 2e-3, |lse_gpu - lse_or| <= 2e-3 over the device's set
 The slack 1e-5 on the kept mass covers fp32 block sums of up to 131072 terms
@@ -61,7 +63,7 @@ def check_prune_row(w, m, kept_count, kept_idx, p, eps, where=""):
     total = float(w.astype(np.float64).sum())
     mass = float(w[kept].astype(np.float64).sum())
     assert mass >= min(p, total) - MASS_SLACK, f"{where}: mass {mass} < p {p}"
-    k_star, m_star, _ = O.top_p_sort(w, p)
+    k_star, m_star, _ = O.top_p_whole(w, p)        # p = 1: the whole row (reading R10)
     band = int(np.count_nonzero((w.astype(np.float64) >= float(m_star) - eps) & (w <= m_star)))
     assert kept.size <= k_star + band, f"{where}: |kept| {kept.size} > k* {k_star} + band {band}"
     return kept, mass, k_star
