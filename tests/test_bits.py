@@ -2,8 +2,9 @@
 weight-mass check (the exact weights' mass over the set kept from the estimate, against p).
 
 CPU: the oracle's bit-width restatement is pinned to the INT4 path at 4 bits, to hand-worked
-exact-grid rows at 2 and 8 bits, and to the quantisation error bound; the C entry points reject
-unsupported widths.  GPU: bit-exact codes, weights against the oracle, and the ablation on the
+exact-grid rows at 2 and 8 bits, to the quantisation error bound, and (for the estimate) to
+torch's exact softmax on K rows that lie on their own 2- or 8-bit grid; the C entry points
+reject unsupported widths.  GPU: bit-exact codes, weights against the oracle, and the ablation on the
 32K-context heads.
 """
 import ctypes as C
@@ -243,3 +244,72 @@ def test_exact_weights_closed_forms():
     x = 32 / np.sqrt(d)
     assert np.isclose(w[5], np.exp(x) / (np.exp(x) + 15), rtol=1e-12)
     assert np.allclose(np.delete(w, 5), 1 / (np.exp(x) + 15), rtol=1e-12)
+
+
+def _grid_layer(bits, seed=4):
+    """One kv-head of 150 tokens whose K rows lie on their own `bits`-wide grid (k = n*s + z,
+    codes 0 and 2^bits - 1 attained, z a nonzero multiple of s), behind a permuted page table, so
+    that quantisation at that width is exact and k_hat = k."""
+    rng = np.random.default_rng(seed)
+    levels = (1 << bits) - 1
+    n_tok, n_pages = 150, 10
+    rows = 16 * n_pages
+    s = rng.choice([1 / 64, 1 / 32] if bits == 8 else [0.25, 0.5], size=rows)
+    z = -rng.integers(1, levels + 1, size=rows) * s
+    codes = rng.integers(0, levels + 1, size=(rows, D))
+    codes[:, 0], codes[:, 1] = 0, levels
+    k = (codes * s[:, None] + z[:, None]).astype(np.float16)
+    assert np.array_equal(k.astype(np.float64), codes * s[:, None] + z[:, None])
+    perm = rng.permutation(n_pages)
+    kk = np.zeros((n_pages, 1, 16, D), np.float16)
+    for j in range(n_pages):
+        kk[perm[j], 0] = k[16 * j:16 * (j + 1)]
+    q = (rng.standard_normal(D) * 2).astype(np.float16)
+    return k, kk, perm.astype(np.int32)[None], np.array([n_tok], np.int32), q
+
+
+def check_estimate_bits(estimate_fn, bits):
+    import math
+    import torch
+    k, kk, pt, lens, q = _grid_layer(bits)
+    kq, sz = O.quantize_k_bits(kk, pt, lens, bits)
+    n = int(lens[0])
+    for sel in ([0, 3, 9], [2, 4, 5, 6, 7]):
+        cand, w = estimate_fn(q, kq, sz, pt, 0, 0, n, np.array(sel), bits)
+        want = [t for t in range(n) if t // 16 in sel]
+        if list(cand) != want:
+            return False
+        ref = torch.softmax(torch.from_numpy(k[want].astype(np.float64))
+                            @ torch.from_numpy(q.astype(np.float64)) / math.sqrt(D), 0).numpy()
+        if not np.allclose(w, ref, rtol=1e-12, atol=1e-15):
+            return False
+    return True
+
+
+@pytest.mark.parametrize("bits", [2, 8])
+def test_estimate_bits_on_its_own_grid_is_the_exact_softmax(bits):
+    """K on the 2- or 8-bit grid is quantised without loss, so the estimate must equal torch's
+    softmax of q.K/sqrt(D) over the selected pages' valid tokens; reading the codes at another
+    width, or dropping the zero point, fails."""
+    assert check_estimate_bits(O.estimate_head_bits, bits)
+
+    def other_width(q16, kq, sz, pt, b, kvh, n, sel, bits):
+        wrong = 4 if bits != 4 else 8
+        cand = O.candidates(sel, n)
+        packed = O.gather_tokens(kq, pt, b, kvh, cand)
+        s = O.gather_tokens(sz, pt, b, kvh, cand).astype(np.float64)
+        codes = O.unpack_rows_bits(packed, wrong)[:, :D]
+        if codes.shape[1] < D:
+            codes = np.pad(codes, ((0, 0), (0, D - codes.shape[1])))
+        khat = codes * s[:, 0:1] + s[:, 1:2]
+        return cand, O.softmax64(khat @ q16.astype(np.float64) / np.sqrt(D))
+
+    def no_zero(q16, kq, sz, pt, b, kvh, n, sel, bits):
+        cand = O.candidates(sel, n)
+        packed = O.gather_tokens(kq, pt, b, kvh, cand)
+        s = O.gather_tokens(sz, pt, b, kvh, cand).astype(np.float64)
+        khat = O.unpack_rows_bits(packed, bits) * s[:, 0:1]
+        return cand, O.softmax64(khat @ q16.astype(np.float64) / np.sqrt(D))
+
+    assert not check_estimate_bits(other_width, bits)
+    assert not check_estimate_bits(no_zero, bits)
