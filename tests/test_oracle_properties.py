@@ -83,6 +83,7 @@ layers = st.fixed_dictionaries({
     "lens": st.lists(st.integers(1, 300), min_size=1, max_size=2),
     "p": st.sampled_from([0.5, 0.85, 0.95, 1.0]),
     "temperature": st.booleans(),
+    "budget_pages": st.sampled_from([0, 0, 1, 5]),
 })
 
 
@@ -92,7 +93,7 @@ def test_decode_step_invariants(c):
     """Generated small layers (ragged lengths, 1 to 4 heads per group, permuted pages, p up to 1):
     every stage of the oracle's step satisfies what the method defines it to be, checked from the
     definitions rather than by re-running the oracle's routines.
-      selection   ceil(P_b / 4) distinct pages of the sequence, ascending
+      selection   ceil(P_b / 4) (or the fixed budget, at most P_b) distinct pages, ascending
       candidates  exactly the valid tokens of the selected pages
       estimate    weights >= 0 summing to 1
       top-p       kept = {W >= m*}; its mass reaches p; the weights above m* alone do not
@@ -103,7 +104,9 @@ def test_decode_step_invariants(c):
     from workloads import synth
     hkv, g = c["hkv"], c["g"]
     wl = synth.make_decode("prop", len(c["lens"]), g * hkv, hkv, c["lens"], seed=c["seed"],
-                           permute_pages=True, temperature=c["temperature"], p=c["p"])
+                           permute_pages=True, temperature=c["temperature"], p=c["p"],
+                           budget_pages=c["budget_pages"])
+    kb = lambda pb: min(c["budget_pages"], pb) if c["budget_pages"] > 0 else -(-pb // 4)
     r = O.decode_step(wl)
     scale = 1 / np.sqrt(128)
     for b, n in enumerate(wl.seq_lens):
@@ -114,7 +117,7 @@ def test_decode_step_invariants(c):
             for h in range(kvh * g, (kvh + 1) * g):
                 hd = r["heads"][(b, h)]
                 sel = list(hd["sel"])
-                assert len(sel) == -(-pb // 4) and sel == sorted(set(sel))
+                assert len(sel) == kb(pb) and sel == sorted(set(sel))
                 assert all(0 <= j < pb for j in sel)
                 assert list(hd["cand"]) == [t for t in range(n) if t // 16 in set(sel)]
                 w = hd["w"]
