@@ -1,7 +1,8 @@
-"""Property tests of the oracle's top-p (hypothesis): generated small rows, ties and zeros
+"""Property tests of the oracle (hypothesis).  Top-p: generated small rows, ties and zeros
 included, checked against brute force over every subset and against the threshold reading of the
 bisection ([Notes] "Key designs": the minimal top-p set, and the bisection on m that finds it
-without a sort).
+without a sort); fp32 softmax rows of up to 3000 weights against the same readings.  The whole
+decode step: generated small layers checked stage by stage against the definitions.
 
 Weights are multiples of 2^-20 in [0, 1], so every sum of up to 10 of them is exact in fp64 and
 the brute force needs no rounding argument.
@@ -72,6 +73,38 @@ def test_bisection_equals_its_threshold_replay(w, frac, eps):
     p = frac * float(w.astype(F64).sum())
     m, _ = O.top_p_bisect(w, p, eps)
     assert F32(m) == _bisect_replay_from_threshold(w, p, eps)
+
+
+softmax_rows = st.fixed_dictionaries({
+    "seed": st.integers(0, 10_000),
+    "n": st.integers(1, 3000),
+    "sigma": st.sampled_from([0.1, 1.0, 3.0, 8.0]),
+    "ties": st.booleans(),
+    "p": st.sampled_from([0.3, 0.8, 0.85, 0.9, 0.99, 0.999999]),
+    "eps": st.sampled_from([1e-9, 1e-6, 1e-3]),
+})
+
+
+@settings(max_examples=80, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(softmax_rows)
+def test_bisection_on_softmax_rows(c):
+    """fp32 softmax rows of up to 3000 weights (flat to peaked, with or without runs of equal
+    logits): the bisection equals its threshold replay, keeps {W >= m} with mass >= p, and keeps
+    at most the minimal set plus its epsilon band."""
+    rng = np.random.default_rng(c["seed"])
+    x = rng.normal(0.0, c["sigma"], c["n"])
+    if c["ties"]:
+        x = np.round(x * 2) / 2                           # runs of equal logits
+    w = O.softmax64(x).astype(F32)
+    p, eps = c["p"], c["eps"]
+    m, kept = O.top_p_bisect(w, p, eps)
+    assert F32(m) == _bisect_replay_from_threshold(w, p, eps)
+    w64 = w.astype(F64)
+    assert np.array_equal(kept, np.nonzero(w >= m)[0])
+    assert w64[kept].sum() >= min(p, w64.sum())
+    k_star, m_star, _ = O.top_p_sort(w, p)
+    band = np.count_nonzero((w64 >= F64(m_star) - eps) & (w64 <= F64(m_star)))
+    assert len(kept) <= k_star + band
 
 
 # ------------------------------------------------------------------ the whole step, as invariants
