@@ -246,3 +246,29 @@ def test_decode_step_after_appends_matches_oracle():
     for b in range(wl.batch):
         for kvh in range(wl.num_kv_heads):
             check_step_group(wl, b, kvh, st, o.cpu().numpy(), lse.cpu().numpy())
+
+
+def test_oracle_append_equals_recomputation_generated():
+    """Generated caches (1 to 3 sequences of 1 to 40 tokens, 1 or 3 kv-heads, 1 to 20 appends):
+    the incremental state equals page_bounds and quantize_k over the extended cache."""
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=40, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+    @given(st.lists(st.integers(1, 40), min_size=1, max_size=3), st.sampled_from([1, 3]),
+           st.integers(1, 20), st.integers(0, 1000))
+    def run(lens, hkv, appends, seed):
+        k, v, pt, n = make_cache(lens, appends, hkv=hkv, seed=seed)
+        bounds = O.page_bounds(k, pt, n)
+        q4, sz = O.quantize_k(k, pt, n)
+        rng = np.random.default_rng(seed + 1)
+        for _ in range(appends):
+            kn, vn = new_token(rng, len(lens), hkv)
+            k, v, bounds, q4, sz, n = O.append_token(k, v, bounds, q4, sz, pt, n, kn, vn)
+        assert n.tolist() == [x + appends for x in lens]
+        ref = referenced(pt, n)
+        assert np.array_equal(u16(bounds[ref]), u16(O.page_bounds(k, pt, n)[ref]))
+        rq, rs = O.quantize_k(k, pt, n)
+        assert np.array_equal(q4[ref], rq[ref]) and np.array_equal(u16(sz[ref]), u16(rs[ref]))
+
+    run()
