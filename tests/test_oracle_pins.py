@@ -259,11 +259,11 @@ def _integer_gqa_case(seed=21):
     return q, k, pt, lens, hq, hkv
 
 
-def check_select_pages(select_fn, budget_pages=0):
+def check_select_pages(select_fn, budget_pages=0, seed=21):
     """Brute force in Python integers: q-head h reads kv-head h // (Hq / Hkv); score of page j =
     sum over channels of max(q_c mn_jc, q_c mx_jc) over the page's valid tokens; keep
     ceil(P / 4) pages (or the fixed budget), highest score first, ties to the lower page."""
-    q, k, pt, lens, hq, hkv = _integer_gqa_case()
+    q, k, pt, lens, hq, hkv = _integer_gqa_case(seed)
     bounds = O.page_bounds(k, pt, lens)
     got = select_fn(q, bounds, pt, lens, hq, hkv, budget_pages, 4)
     for b, n in enumerate(lens):
@@ -290,6 +290,10 @@ def check_select_pages(select_fn, budget_pages=0):
 def test_select_pages_bruteforce_integer_gqa():
     assert check_select_pages(O.select_pages)
     assert check_select_pages(O.select_pages, budget_pages=3)
+    for seed in range(8):                   # other draws: other ties, other page permutations
+        for budget in (0, 1, 5, 100):
+            assert check_select_pages(O.select_pages, budget_pages=budget, seed=seed), \
+                (seed, budget)
 
     def kv_head_modulo(q, bounds, pt, lens, hq, hkv, budget_pages=0, budget_div=4):
         out = {}
