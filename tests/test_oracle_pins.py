@@ -74,6 +74,56 @@ def test_bounds_invariants():
     assert check_bounds(O.page_bounds, np.random.default_rng(1))
 
 
+def check_bounds_brute(bounds_fn):
+    """Ragged sequences behind permuted page tables, channels salted with +0 and -0: each bound is
+    the smallest / largest valid value found by a plain scan that orders -0 before +0."""
+    def tot(x):                                    # value, then -0 before +0
+        return (float(x), not np.signbit(x))
+    for seed in range(6):
+        rng = np.random.default_rng(100 + seed)
+        lens = rng.integers(1, 60, size=3)
+        pages = [-(-int(n) // 16) for n in lens]
+        p_phys = sum(pages) + 2
+        perm = rng.permutation(p_phys)
+        pt = np.full((3, max(pages)), -1, np.int32)
+        o = 0
+        for b, m in enumerate(pages):
+            pt[b, :m] = perm[o:o + m]
+            o += m
+        k = rng.standard_normal((p_phys, 2, 16, 8)).astype(F16)
+        zero = rng.random(k.shape) < 0.3
+        k[zero] = np.where(rng.random(k.shape) < 0.5, F16(0.0), F16(-0.0))[zero]
+        bd = bounds_fn(np.pad(k, ((0, 0), (0, 0), (0, 0), (0, 120))), pt, lens)
+        for b, n in enumerate(lens):
+            for j in range(pages[b]):
+                ph, rows = pt[b, j], min(16, int(n) - 16 * j)
+                for h in range(2):
+                    for c in range(8):
+                        col = list(k[ph, h, :rows, c])
+                        lo, hi = min(col, key=tot), max(col, key=tot)
+                        if u16_1(bd[ph, h, 0, c]) != u16_1(lo) or u16_1(bd[ph, h, 1, c]) != u16_1(hi):
+                            return False
+    return True
+
+
+def test_bounds_by_brute_force_with_signed_zeros():
+    assert check_bounds_brute(O.page_bounds)
+
+    def numpy_min_max(k, pt, lens):              # np.min / np.max: -0 and +0 compare equal
+        out = np.zeros((k.shape[0], k.shape[1], 2, k.shape[3]), F16)
+        for b, n in enumerate(lens):
+            for j in range(-(-int(n) // 16)):
+                rows = k[pt[b, j], :, :min(16, int(n) - 16 * j)]
+                out[pt[b, j], :, 0], out[pt[b, j], :, 1] = rows.min(axis=1), rows.max(axis=1)
+        return out
+
+    assert not check_bounds_brute(numpy_min_max)
+
+
+def u16_1(x):
+    return int(np.array([x], dtype=F16).view(np.uint16)[0])
+
+
 def test_bounds_single_token_page():
     rng = np.random.default_rng(2)
     k = rng.standard_normal((1, 1, 16, 128)).astype(F16)
