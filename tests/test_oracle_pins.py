@@ -5,20 +5,23 @@ Paper-Notes (NeurIPS 2025) page; [Summary] = the paperlayer summary of arXiv 250
 
 What pins what:
   bounds      invariant mn <= k <= mx with both attained; single-token page; partial page ignores
-              rows past the sequence end.
+              rows past the sequence end; a plain scan over ragged, permuted caches salted with
+              signed zeros (-0 before +0).
   INT4        hand-worked bytes (tests/golden/int4_rows.json, [Summary] B.1); round-trip error
               <= s/2 (+ fp16 rounding of s); memory identity 1/8 of the KV cache ([Notes] "Key
               designs", 4-bit K cache; [Summary] 4.3).
   scores      unit queries give the bound rows themselves; upper-bound property against every
               token of the page (fp64); equality for a page of identical tokens.
   top-k       brute-force full sort; whole page selection (GQA head map, budget rule, ties) by
-              brute force in Python integers on integer-valued q and K.
+              brute force in Python integers on integer-valued q and K (nine draws, four
+              budgets).
   order key   every non-NaN fp16 bit pattern: keys rise strictly with the value, -0 before +0.
   softmax     closed forms (uniform; logits 0 and ln 3 give 1/4 and 3/4, also at +1000) and the
               definition term by term with math.fsum.
   estimate    K on the 16-level grid makes the dequantised K exact, so the estimate must equal
               torch's softmax of q.K/sqrt(D) computed from the raw fp16 K.
-  top-p       hand examples (tests/golden/top_p_examples.json, [Notes] "Key designs");
+  top-p       hand examples (tests/golden/top_p_examples.json, [Notes] "Key designs"); p = 1
+              keeps the whole distribution even where the fp64 prefix rounds to 1 early;
               brute-force subset search for n <= 14; mass(W >= m*) >= p > mass(W > m*);
               bisection result inside the epsilon band ([Notes] "Key designs", efficient top-p).
   gather      rows that carry their own (token, head, sequence) address, behind a permuted
