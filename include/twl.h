@@ -121,7 +121,9 @@ size_t twl_workspace_bytes(int32_t op, int32_t batch, int32_t num_q_heads, int32
                            int32_t max_pages, int32_t max_budget, int32_t rows,
                            int32_t row_stride);
 
-/* Zero the workspace header (stream-ordered memset of 256 bytes). */
+/* Zero the whole workspace: a stream-ordered memset of ws_bytes, which clears the header's device
+ * flags and, for twl_decode_step, the synchronisation words and page masks that must start at
+ * zero (each step launch leaves them zero again for the next). */
 twl_status twl_workspace_init(void* ws, size_t ws_bytes, twl_stream_t stream);
 
 /* Wait for `stream`, then report the sticky device flags of `ws` in *flags (may be NULL).
