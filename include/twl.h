@@ -266,7 +266,8 @@ twl_status twl_estimate_nbit(const void* q, int32_t num_q_heads, const twl_paged
  *   m_out      float [rows] out
  *   kept_count int32 [rows] out = |{i : W_i >= m}|
  *   kept_idx   int32 [rows][row_stride] out (ascending indices) or NULL
- *   ws, ws_bytes  unused (NULL and 0 are fine; twl_workspace_bytes(TWL_OP_PRUNE, ...) is 0)
+ *   ws, ws_bytes  unused (NULL and 0 are fine; twl_workspace_bytes(TWL_OP_PRUNE, ...) gives
+ *                 the 256-byte header size, which this call does not need)
  * TWL_ERR_INVALID_ARG for NULL w / m_out / kept_count, rows < 0, row_stride < 1, p outside
  * (0, 1], eps not positive and finite, or w not 4-byte aligned; rows == 0 launches nothing. */
 twl_status twl_prune_top_p(const float* w, const int32_t* row_len, int32_t rows,

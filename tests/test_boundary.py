@@ -189,6 +189,7 @@ def test_cache_calls_reject_bad_arguments():
 def test_workspace_sizes():
     wb = twl.twl_workspace_bytes
     assert wb(twl.TWL_OP_CACHE) == 256
+    assert wb(twl.TWL_OP_PRUNE, 1, 1, 1, 1, 1, 4096, 8192) == 256     # header only, unused
     assert wb(99) == 0
     s1 = wb(twl.TWL_OP_DECODE_STEP, 1, 32, 8, 2048, 512)
     s2 = wb(twl.TWL_OP_DECODE_STEP, 2, 32, 8, 2048, 512)
@@ -231,3 +232,38 @@ def test_layer_rejects_host_and_misshaped_tensors_before_any_call():
     with pytest.raises(ValueError):
         layer.append(rows, rows)
     expect_tensor("x", rows, (3, 2, 128), torch.float16, rows.device)
+
+
+def test_header_compiles_as_c_and_a_c_program_links_and_calls(tmp_path):
+    """include/twl.h is plain C: a C99 program includes it, links libtwl.so and calls through the
+    ABI (host-side rejections only, so no GPU is needed)."""
+    src = tmp_path / "use_twl.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "twl.h"
+int main(void) {
+  twl_paged_kv kv = {0, 0, 0, 0, 2, 8, 128, 16, 64, 100};
+  twl_k_aux aux = {0, 0, 0};
+  float o[1], lse[1];
+  twl_status st = twl_decode_step(0, 32, &kv, &aux, 0, 4, 16, 0.85f, 1e-6f, o, lse, 0, 0, 0, 0);
+  if (st != TWL_ERR_INVALID_ARG) { printf("decode_step %d\n", (int)st); return 1; }
+  st = twl_prune_top_p(0, 0, 1, 8, 0.9f, 1e-6f, 0, 0, 0, 0, 0, 0);
+  if (st != TWL_ERR_INVALID_ARG) { printf("prune %d\n", (int)st); return 2; }
+  if (strcmp(twl_status_string(TWL_OK), "ok") != 0) return 3;
+  if (twl_workspace_bytes(TWL_OP_PRUNE, 1, 1, 1, 1, 1, 4, 8) != 256) return 4;
+  printf("%s\n", twl_status_string(TWL_ERR_INVALID_ARG));
+  return 0;
+}
+''')
+    lib_dir = os.path.dirname(twl.LIB_PATH)
+    exe = tmp_path / "use_twl"
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        str(src), "-o", str(exe), "-L", lib_dir, "-ltwl",
+                        "-Wl,-rpath," + lib_dir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
