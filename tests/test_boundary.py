@@ -186,6 +186,46 @@ def test_cache_calls_reject_bad_arguments():
     assert twl._lib.twl_page_bounds(C.byref(kv), A, A, 16, None) == -5
 
 
+def test_estimate_and_union_reject_bad_arguments():
+    kv = _kv()
+    est = twl._lib.twl_estimate
+
+    def e(q=A, k4=A, sz=A, sel=A, cnt=A, mb=16, w=A, tok=A, cc=A, ws=A, wsb=1 << 30, hq=32,
+          kvv=kv):
+        return est(q, hq, C.byref(kvv), k4, sz, sel, cnt, mb, w, tok, cc, ws, wsb, None)
+
+    assert e(q=0) == twl.TWL_ERR_INVALID_ARG
+    assert e(q=A + 8) == twl.TWL_ERR_INVALID_ARG            # q 16-byte aligned
+    assert e(k4=A + 4) == twl.TWL_ERR_INVALID_ARG
+    assert e(w=0) == twl.TWL_ERR_INVALID_ARG
+    assert e(mb=0) == twl.TWL_ERR_INVALID_ARG
+    assert e(mb=65) == twl.TWL_ERR_INVALID_ARG              # above max_pages
+    assert e(hq=24) == twl.TWL_ERR_UNSUPPORTED              # group of 3
+    assert e(kvv=_kv(page_size=8)) == twl.TWL_ERR_UNSUPPORTED
+    assert e(wsb=256) == twl.TWL_ERR_WORKSPACE
+    assert e(ws=0) == twl.TWL_ERR_WORKSPACE
+    uni = twl._lib.twl_group_union
+
+    def u(tok=A, ki=A, kc=A, cs=16, ut=A, uc=A, ws=None, wsb=0, hq=32):
+        return uni(hq, C.byref(kv), tok, ki, kc, cs, ut, uc, ws, wsb, None)
+
+    assert u(tok=0) == twl.TWL_ERR_INVALID_ARG
+    assert u(uc=0) == twl.TWL_ERR_INVALID_ARG
+    assert u(cs=0) == twl.TWL_ERR_INVALID_ARG
+    assert u(hq=12) == twl.TWL_ERR_INVALID_ARG               # not a multiple of the kv-heads
+    assert u(ws=A + 64, wsb=1 << 20) == twl.TWL_ERR_WORKSPACE  # misaligned workspace
+    assert u(ws=A, wsb=16) == twl.TWL_ERR_WORKSPACE          # smaller than the header
+
+
+def test_workspace_init_and_status_reject_bad_workspaces():
+    flags = C.c_uint32(7)
+    assert twl._lib.twl_workspace_init(None, 1 << 20, None) == twl.TWL_ERR_WORKSPACE
+    assert twl._lib.twl_workspace_init(A, 100, None) == twl.TWL_ERR_WORKSPACE
+    assert twl._lib.twl_workspace_init(A + 16, 1 << 20, None) == twl.TWL_ERR_WORKSPACE
+    assert twl._lib.twl_device_status(None, C.byref(flags), 0, None) == twl.TWL_ERR_WORKSPACE
+    assert twl._lib.twl_device_status(A + 16, C.byref(flags), 0, None) == twl.TWL_ERR_WORKSPACE
+
+
 def test_workspace_sizes():
     wb = twl.twl_workspace_bytes
     assert wb(twl.TWL_OP_CACHE) == 256
