@@ -31,7 +31,8 @@ Readings where the pages are silent (each also listed in the design notes):
     own candidates (valid tokens of its selected pages) in fp64.
   * Top-p: the minimal set by sort + cumulative sum ([Notes] "Key designs", formal statement),
     and the pages' threshold bisection ([Notes] "Key designs", efficient top-p;
-    [Summary] 4.2) with lo = 0, hi = max W, mid = lo + (hi - lo) / 2.
+    [Summary] 4.2) with lo = 0, hi = max W, mid = lo + (hi - lo) / 2.  p = 1 keeps every
+    candidate (m = 0) in both forms.
   * GQA: each group attends over the union of its heads' kept tokens ([Summary] B.2).
 """
 from __future__ import annotations
@@ -226,6 +227,8 @@ def page_scores(q16: np.ndarray, mn16: np.ndarray, mx16: np.ndarray) -> np.ndarr
 
 
 def budget_for(n_pages: int, budget_pages: int, budget_div: int) -> int:
+    """Pages the selector keeps: budget_pages if > 0, else ceil(P / budget_div), at most P
+    ([Notes] "Overall framework": a conservative base budget such as 1/4; [Summary] 4.3)."""
     if budget_pages > 0:
         return min(int(budget_pages), int(n_pages))
     return min(int(n_pages), -(-int(n_pages) // int(budget_div)))
@@ -270,7 +273,8 @@ def top_p_sort(w: np.ndarray, p: float):
 
 def top_p_whole(w: np.ndarray, p: float):
     """``top_p_sort`` for a normalised distribution (softmax weights summing to 1), with p = 1
-    read as the whole distribution: every entry is kept and m* = 0.  The sort form cannot decide
+    read as the whole distribution ([Notes] "Key designs": the kept mass must reach p, which at
+    p = 1 is all of it): every entry is kept and m* = 0.  The sort form cannot decide
     p = 1 by itself: the fp64 sum of the largest weights can round to exactly 1.0 while positive
     weights remain, and an exact sum of the rounded weights can land on either side of 1."""
     w = np.asarray(w)
@@ -320,7 +324,8 @@ def top_p_bisect(w: np.ndarray, p: float, eps: float, max_iter: int = 64):
 # ----------------------------------------------------------------------------------------------
 
 def attention(q16, k16, v16, scale: float):
-    """Exact softmax(q K^T * scale) V in fp64 over the given rows; lse in natural log."""
+    """Exact softmax(q K^T * scale) V in fp64 over the given rows; lse in natural log ([Notes]
+    "Overall framework": the final attention runs over the kept tokens only, renormalised)."""
     q = np.asarray(q16, dtype=F16).astype(F64)
     k = np.asarray(k16, dtype=F16).astype(F64)
     v = np.asarray(v16, dtype=F16).astype(F64)
@@ -361,13 +366,16 @@ def select_pages(q, bounds, page_table, seq_lens, num_q_heads, num_kv_heads,
 
 
 def candidates(sel_pages, n: int) -> np.ndarray:
-    """Valid logical token ids of the selected pages, ascending."""
+    """Valid logical token ids of the selected pages, ascending (the candidates the selector
+    hands to top-p: [Notes] "Overall framework"; [Summary] 4.1)."""
     toks = [np.arange(PAGE * j, PAGE * j + valid_rows(n, j)) for j in sorted(sel_pages)]
     return np.concatenate(toks).astype(np.int64) if toks else np.zeros(0, dtype=np.int64)
 
 
 def estimate_head(q16, k_int4, k_sz, page_table, b, kvh, n, sel_pages, head_dim=128):
-    """Estimated weights of one head over its candidates (fp64), with the token ids."""
+    """Estimated weights of one head over its candidates (fp64), with the token ids: softmax of
+    q . khat / sqrt(D) with khat = n*s + z from the INT4 copy ([Notes] "Key designs": top-p needs
+    weight values, estimated from the 4-bit K cache; [Summary] 4.2, B.1)."""
     cand = candidates(sel_pages, n)
     if cand.size == 0:
         return cand, np.zeros(0)
@@ -446,7 +454,8 @@ def quantize_k_bits(k, page_table, seq_lens, bits: int):
 
 
 def estimate_head_bits(q16, k_q, k_sz, page_table, b, kvh, n, sel_pages, bits, head_dim=128):
-    """``estimate_head`` from the ``bits``-wide copy of K: khat = n*s + z, fp64 logits."""
+    """``estimate_head`` from the ``bits``-wide copy of K: khat = n*s + z, fp64 logits (the
+    bit-width ablation of [Summary] 4.3)."""
     cand = candidates(sel_pages, n)
     if cand.size == 0:
         return cand, np.zeros(0)
@@ -493,7 +502,8 @@ def page_centroids(k, page_table, seq_lens, out=None):
 
 def cluster_weights(q16, cen, page_table, b, kvh, n, head_dim=128):
     """Size-weighted centroid estimate of each page's share of the attention mass:
-    A_j = n_j exp(q . c_j / sqrt(D)), normalised over the sequence's pages (fp64)."""
+    A_j = n_j exp(q . c_j / sqrt(D)), normalised over the sequence's pages (fp64) (the Double-P
+    summary page, "Key designs": clusters scored by size-weighted centroids)."""
     pb = num_pages(n)
     phys = np.asarray(page_table[b, :pb], dtype=np.int64)
     c = cen[phys, kvh].astype(F64)                                      # [pb][D]
@@ -557,7 +567,8 @@ def decode_step(wl, bounds=None, k_int4=None, k_sz=None, with_attention=True):
 
 
 def group_attention(wl, tok_lists):
-    """Attention of every q-head over its group's given token set: {(b,h): (o, lse)}."""
+    """Attention of every q-head over its group's given token set: {(b,h): (o, lse)} (GQA
+    groups attend over one token set: [Summary] B.2)."""
     g = wl.num_q_heads // wl.num_kv_heads
     scale = 1.0 / math.sqrt(wl.head_dim)
     out = {}
@@ -570,6 +581,7 @@ def group_attention(wl, tok_lists):
 
 
 def full_attention_weights(q16, k16, scale):
-    """Exact softmax weights over every token (for the top-p error bound)."""
+    """Exact softmax weights over every token (for the top-p error bound of [Notes] "Key
+    designs", oracle top-p)."""
     s = (np.asarray(k16, dtype=F16).astype(F64) @ np.asarray(q16, dtype=F16).astype(F64))
     return softmax64(s * F64(scale))
