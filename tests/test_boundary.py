@@ -307,3 +307,31 @@ int main(void) {
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+
+
+def test_readme_c_example_compiles(tmp_path):
+    """The C example in README.md compiles and links as written (it is not run: its pointers
+    would have to be device memory)."""
+    text = open(os.path.join(ROOT, "README.md")).read()
+    m = re.search(r"```c\n(.*?)```", text, flags=re.S)
+    assert m, "README has a C example"
+    cuda_inc = "/usr/local/cuda/include"
+    if not os.path.isdir(cuda_inc):
+        pytest.skip("no CUDA headers")
+    src = tmp_path / "readme_example.c"
+    src.write_text(
+        "#include <cuda_runtime.h>\n#include \"twl.h\"\n"
+        "int example(void* d_k, void* d_v, int32_t* d_page_table, int32_t* d_seq_lens,\n"
+        "            void* d_k_int4, void* d_k_scale_zero, void* d_bounds, void* d_q, float* d_o,\n"
+        "            float* d_lse, int32_t B, int32_t Hq, int32_t Hkv, int32_t max_pages,\n"
+        "            int32_t P, twl_stream_t stream) {\n" + m.group(1) + "  return (int)st;\n}\n")
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(twl.LIB_PATH)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-shared", "-fPIC",
+                        "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src),
+                        "-o", str(tmp_path / "libexample.so"), "-L", lib_dir, "-ltwl",
+                        "-L", "/usr/local/cuda/lib64", "-lcudart"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
